@@ -1,0 +1,1018 @@
+/*
+ * Plain CPU oracle for the fused recurrent-state update with quantized
+ * write-back of gated delta-rule layers (KDA: decay per key channel; GDN:
+ * decay per head).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only tests/, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  It is deliberately
+ * slow: one scalar loop per definition, one Philox call per element, no
+ * blocking or fusion beyond what the definitions below state.
+ *
+ * Precision.  The recurrence and the quantizers run in FP32, the precision
+ * the DAMP summary names for the fused update ([DAMP] Key Points >
+ * Implementation: reconstruct INT8 channels, compute the update in FP32,
+ * re-quantize, write back).  The bit allocator runs in FP64.  Build with
+ * -ffp-contract=off so that every a*b+c written below is two roundings and
+ * every fmaf() is one.
+ *
+ * Operation order (the pages fix FP32 but not the order of a sum; these
+ * orders are this implementation's reading and the CUDA library follows the
+ * same written definition):
+ *   - every sum over key rows runs i = 0, 1, ..., d-1 as an fmaf chain
+ *     starting from +0;
+ *   - every sum over value columns (variable-width fit error) runs
+ *     j = 0, 1, ..., d-1 as an fmaf chain starting from +0;
+ *   - the Hadamard transform is the unnormalised butterfly, stages
+ *     h = 1, 2, 4, ..., n/2, each pair (x, y) -> (x + y, x - y), followed by
+ *     one multiplication by the float nearest to 1/sqrt(n).
+ *
+ * Parity status:
+ *   pinned: binary16 conversion (against numpy float16), Philox4x32-10
+ *     (published known-answer vectors), Hadamard (explicit Sylvester matrix),
+ *     INT8 block quantizer and variable-width quantizer (exhaustive level
+ *     search on random blocks), stochastic rounding (mean over seeds),
+ *     allocator (worked example, budget, monotonicity, brute force),
+ *     erasure rate (worked example, closed form and brute-force Gramian),
+ *     recurrence (FP64 dense-matrix recurrence, beta=0/a=1 identity, unit-key
+ *     invariant, dead zone and error feedback), storage accounting.
+ *   parity unpinned: the order of FP32 operations inside a sum (a reading,
+ *     see above) and the rotated-domain mode, which is pinned only against
+ *     the canonical mode within the output tolerance.
+ */
+#include "brs_oracle.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------ */
+/* binary16 and bfloat16                                                     */
+/* ------------------------------------------------------------------------ */
+
+/* IEEE 754 binary16, round to nearest, ties to even, subnormals kept,
+ * overflow to infinity.  Written from the format definition: the value is
+ * rounded to the quantum of its binade (2^(E-10), with E clamped at -14 for
+ * the subnormal range) in FP64, where the division by a power of two and
+ * the rounding are exact. */
+uint16_t orc_f16_from_f32(float f) {
+  uint32_t bits;
+  memcpy(&bits, &f, 4);
+  uint16_t sign = (uint16_t)((bits >> 16) & 0x8000u);
+  if (isnan(f)) return (uint16_t)(sign | 0x7e00u);
+  if (isinf(f)) return (uint16_t)(sign | 0x7c00u);
+  double a = fabs((double)f);
+  if (a == 0.0) return sign;
+  int e;
+  frexp(a, &e);
+  int E = e - 1;                       /* floor(log2 a) */
+  if (E < -14) E = -14;
+  double quantum = ldexp(1.0, E - 10);
+  double n = nearbyint(a / quantum);   /* ties to even */
+  double r = n * quantum;
+  if (r > 65504.0) return (uint16_t)(sign | 0x7c00u);
+  if (r < ldexp(1.0, -14)) return (uint16_t)(sign | (uint16_t)n); /* subnormal */
+  frexp(r, &e);
+  int E2 = e - 1;
+  int M = (int)(r / ldexp(1.0, E2 - 10)); /* in [1024, 2047] */
+  return (uint16_t)(sign | (uint16_t)((E2 + 15) << 10) | (uint16_t)(M - 1024));
+}
+
+float orc_f32_from_f16(uint16_t h) {
+  int E = (h >> 10) & 31, M = h & 1023;
+  double v;
+  if (E == 0) v = ldexp((double)M, -24);
+  else if (E == 31) v = M ? NAN : INFINITY;
+  else v = ldexp((double)(1024 + M), E - 25);
+  return (float)((h & 0x8000u) ? -v : v);
+}
+
+float orc_f32_from_bf16(uint16_t b) {
+  uint32_t bits = (uint32_t)b << 16;
+  float f;
+  memcpy(&f, &bits, 4);
+  return f;
+}
+
+static int f16_is_inf_or_nan(uint16_t h) { return ((h >> 10) & 31) == 31; }
+
+/* ------------------------------------------------------------------------ */
+/* Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as   */
+/* easy as 1, 2, 3", SC'11): ten rounds of two 32x32->64 multiplications     */
+/* with the round keys bumped by the Weyl constants between rounds.          */
+/* ------------------------------------------------------------------------ */
+void orc_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]) {
+  uint32_t c0 = ctr[0], c1 = ctr[1], c2 = ctr[2], c3 = ctr[3];
+  uint32_t k0 = key[0], k1 = key[1];
+  for (int round = 0; round < 10; ++round) {
+    if (round > 0) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+    uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+    uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+    uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+    uint32_t n0 = hi1 ^ c1 ^ k0;
+    uint32_t n2 = hi0 ^ c3 ^ k1;
+    c0 = n0;
+    c1 = lo1;
+    c2 = n2;
+    c3 = lo0;
+  }
+  out[0] = c0;
+  out[1] = c1;
+  out[2] = c2;
+  out[3] = c3;
+}
+
+/* 24 uniform bits for element `elem` of head (b, h) at write-back step
+ * `step`: counter (elem/4, step, h, b), key (seed low, seed high), word
+ * elem % 4, top 24 bits. */
+static uint32_t sr_bits24(uint64_t seed, int64_t step, int h, int b, int elem) {
+  uint32_t ctr[4] = {(uint32_t)(elem / 4), (uint32_t)step, (uint32_t)h, (uint32_t)b};
+  uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+  uint32_t out[4];
+  orc_philox4x32_10(ctr, key, out);
+  return out[elem % 4] >> 8;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Hadamard along the value axis ([DAMP] Data & Methods > Quantization &     */
+/* calibration details: a Hadamard transform along the value dimension      */
+/* within each key channel before INT8 quantization).  Sylvester matrix in   */
+/* natural order, normalised to be orthonormal; it is its own inverse.       */
+/* ------------------------------------------------------------------------ */
+float orc_hadamard_scale(int n) { return (float)(1.0 / sqrt((double)n)); }
+
+void orc_fwht(float* x, int n) {
+  for (int h = 1; h < n; h *= 2)
+    for (int i = 0; i < n; i += 2 * h)
+      for (int j = i; j < i + h; ++j) {
+        float a = x[j], b = x[j + h];
+        x[j] = a + b;
+        x[j + h] = a - b;
+      }
+  float s = orc_hadamard_scale(n);
+  for (int j = 0; j < n; ++j) x[j] = x[j] * s;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Write-back rounding rules ([WB] Quantized GRU formulation and the         */
+/* Chinese summary's sections on error feedback and stochastic rounding):    */
+/*   nearest      q = Q(h): nearest level, half-steps to the even index,     */
+/*                clipped at the grid rails;                                  */
+/*   stochastic   one of the two adjacent levels, chosen with probability    */
+/*                set by the position between them (unbiased);               */
+/*   error feedb. q = Q(h + e_prev), e = h + e_prev - q clipped to +-Delta.  */
+/* ------------------------------------------------------------------------ */
+static float sr_round(float t, uint32_t r24) {
+  float fl = floorf(t);
+  float fr = t - fl;
+  return ((float)r24 < fr * 16777216.0f) ? fl + 1.0f : fl;
+}
+
+/* INT8 asymmetric affine block ([DAMP] Quantization & calibration details:
+ * per-block asymmetric affine quantization, b = 8; the stored scale and zero
+ * are FP16): scale = fp16((max - min) / 255), zero = fp16(min),
+ * code = clamp(round((y - zero) * (1 / scale)), 0, 255),
+ * value = fmaf(code, scale, zero). */
+int orc_int8_block(const float* y, int n, int mode, uint64_t seed, int64_t step, int h, int b,
+                   int elem0, uint16_t* e_inout, uint8_t* codes, uint16_t* scale_h,
+                   uint16_t* zero_h, float* t_out) {
+  int flags = 0;
+  if (n <= 0) return ORC_EINVAL;
+  float* tgt = (float*)malloc(sizeof(float) * (size_t)n);
+  for (int j = 0; j < n; ++j) {
+    tgt[j] = y[j];
+    if (mode == ORC_ROUND_ERRFEEDBACK) tgt[j] = y[j] + orc_f32_from_f16(e_inout[j]);
+    if (!isfinite(tgt[j])) flags |= ORC_ENONFINITE;
+  }
+  float mn = tgt[0], mx = tgt[0];
+  for (int j = 1; j < n; ++j) {
+    if (tgt[j] < mn) mn = tgt[j];
+    if (tgt[j] > mx) mx = tgt[j];
+  }
+  uint16_t sh = orc_f16_from_f32((mx - mn) / 255.0f);
+  uint16_t zh = orc_f16_from_f32(mn);
+  if (f16_is_inf_or_nan(sh) || f16_is_inf_or_nan(zh)) flags |= ORC_EOVERFLOW;
+  float s = orc_f32_from_f16(sh), z = orc_f32_from_f16(zh);
+  float rcp = (s == 0.0f) ? 0.0f : 1.0f / s;
+  for (int j = 0; j < n; ++j) {
+    float t = 0.0f, c = 0.0f;
+    if (s != 0.0f) {
+      t = (tgt[j] - z) * rcp;
+      if (mode == ORC_ROUND_STOCHASTIC)
+        c = sr_round(t, sr_bits24(seed, step, h, b, elem0 + j));
+      else
+        c = nearbyintf(t);
+      if (c < 0.0f) c = 0.0f;
+      if (c > 255.0f) c = 255.0f;
+      if (!(c == c)) c = 0.0f;
+    }
+    codes[j] = (uint8_t)(int)c;
+    if (t_out) t_out[j] = t;
+    if (mode == ORC_ROUND_ERRFEEDBACK) {
+      float xhat = fmaf(c, s, z);
+      float e = tgt[j] - xhat;
+      if (e > s) e = s;
+      else if (e < -s) e = -s;
+      e_inout[j] = orc_f16_from_f32(e);
+    }
+  }
+  *scale_h = sh;
+  *zero_h = zh;
+  free(tgt);
+  return flags;
+}
+
+/* Variable-width symmetric row ([LB] Levels and storage): levels
+ * {-n..n}*Delta, n = 2^(b-1) - 1, Delta = f*R/n with R the row's absolute
+ * maximum and f fitted over 16 values in [1/4, 1] (read as f_m = (5+m)/20)
+ * by squared error, the chosen Delta stored as an FP16 scale.  The fit
+ * error of every candidate is evaluated with nearest rounding on the target
+ * (x, or x + e_prev under error feedback); ties keep the smaller f. */
+int orc_varbit_row(const float* x, int n, int bw, int mode, uint64_t seed, int64_t step, int h,
+                   int b, int elem0, uint16_t* e_inout, int32_t* q_out, uint16_t* delta_h,
+                   int* m_star, float* t_out) {
+  int flags = 0;
+  int nl = (1 << (bw - 1)) - 1;
+  float fnl = (float)nl;
+  float* tgt = (float*)malloc(sizeof(float) * (size_t)n);
+  float R = 0.0f;
+  for (int j = 0; j < n; ++j) {
+    tgt[j] = x[j];
+    if (mode == ORC_ROUND_ERRFEEDBACK) tgt[j] = x[j] + orc_f32_from_f16(e_inout[j]);
+    if (!isfinite(tgt[j])) flags |= ORC_ENONFINITE;
+    float a = fabsf(tgt[j]);
+    if (a > R) R = a;
+  }
+  uint16_t dh = 0;
+  int best = -1;
+  if (R > 0.0f) {
+    float bestE = 0.0f;
+    for (int m = 0; m < 16; ++m) {
+      float f = (float)(5 + m) / 20.0f;
+      uint16_t ch = orc_f16_from_f32((f * R) / fnl);
+      float dm = orc_f32_from_f16(ch);
+      if (!isfinite(dm)) continue;
+      float E = 0.0f;
+      if (dm == 0.0f) {
+        for (int j = 0; j < n; ++j) E = fmaf(tgt[j], tgt[j], E);
+      } else {
+        float inv = 1.0f / dm;
+        for (int j = 0; j < n; ++j) {
+          float qf = nearbyintf(tgt[j] * inv);
+          if (qf < -fnl) qf = -fnl;
+          if (qf > fnl) qf = fnl;
+          float r = tgt[j] - dm * qf;
+          E = fmaf(r, r, E);
+        }
+      }
+      if (best < 0 || E < bestE) {
+        best = m;
+        bestE = E;
+        dh = ch;
+      }
+    }
+    if (best < 0) {
+      flags |= ORC_EOVERFLOW;
+      dh = 0x7c00u;
+      best = 15;
+    }
+  } else {
+    best = 0;
+  }
+  float D = orc_f32_from_f16(dh);
+  int ok = (D != 0.0f) && isfinite(D);
+  float inv = ok ? 1.0f / D : 0.0f;
+  for (int j = 0; j < n; ++j) {
+    float t = 0.0f, qf = 0.0f;
+    if (ok) {
+      t = tgt[j] * inv;
+      if (mode == ORC_ROUND_STOCHASTIC)
+        qf = sr_round(t, sr_bits24(seed, step, h, b, elem0 + j));
+      else
+        qf = nearbyintf(t);
+      if (qf < -fnl) qf = -fnl;
+      if (qf > fnl) qf = fnl;
+      if (!(qf == qf)) qf = 0.0f;
+    }
+    q_out[j] = (int32_t)qf;
+    if (t_out) t_out[j] = t;
+    if (mode == ORC_ROUND_ERRFEEDBACK) {
+      float xhat = D * qf;
+      if (!ok) xhat = 0.0f;
+      float e = tgt[j] - xhat;
+      float lim = ok ? D : 0.0f;
+      if (e > lim) e = lim;
+      else if (e < -lim) e = -lim;
+      e_inout[j] = orc_f16_from_f32(e);
+    }
+  }
+  *delta_h = dh;
+  if (m_star) *m_star = best;
+  free(tgt);
+  return flags;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Decay-aware allocation ([LB] Approximate erasure rate, Range              */
+/* normalization, State bit allocation; [LBX] worked example).               */
+/* ------------------------------------------------------------------------ */
+
+/* Gamma_hat = rho / [C * expm1(2 (s + r))], rho = 1, with s = -ln(A)/2 the
+ * decay rate estimated from A = EMA(a^2) and r = K/2 from
+ * K = EMA(beta (2 - beta) k^2).  The argument is floored at 1e-9. */
+double orc_gamma_hat(double A, double K, int C) {
+  double s = -0.5 * log(A);
+  double r = 0.5 * K;
+  double arg = 2.0 * (s + r);
+  if (!(arg >= 1e-9)) arg = 1e-9;
+  return 1.0 / ((double)C * expm1(arg));
+}
+
+/* b*_i = avg + log2(c_i / GM(c)) / 2 (the minimiser of sum c_i 2^(-2 b_i)
+ * at a fixed mean), GM over the rows with c_i > 0; rounded to nearest
+ * (ties to even), clipped to [b_min, b_max]; rows with c_i = 0 take b_min
+ * (all rows take round(avg) when every c_i is 0).  The sum is then brought
+ * to avg*N one bit at a time: while over budget, take a bit from the row
+ * whose cost rises least (3 c_i 4^(-b_i)); while under, give one to the
+ * row whose cost falls most (3/4 c_i 4^(-b_i)); ties to the lower row. */
+int orc_allocate_bits(int N, const double* c, double avg_bits, int b_min, int b_max,
+                      uint8_t* bits) {
+  double tgt = avg_bits * (double)N;
+  long target = (long)tgt;
+  if ((double)target != tgt || target < (long)N * b_min || target > (long)N * b_max ||
+      b_min < 1 || b_max > 16 || b_min > b_max)
+    return ORC_EINVAL;
+  int* b = (int*)malloc(sizeof(int) * (size_t)N);
+  int cnt = 0;
+  double sumlog = 0.0;
+  for (int i = 0; i < N; ++i)
+    if (c[i] > 0.0) {
+      sumlog += log(c[i]);
+      ++cnt;
+    }
+  if (cnt == 0) {
+    for (int i = 0; i < N; ++i) b[i] = (int)nearbyint(avg_bits);
+  } else {
+    double gm = exp(sumlog / (double)cnt);
+    for (int i = 0; i < N; ++i) {
+      if (c[i] > 0.0) {
+        double bs = avg_bits + 0.5 * log2(c[i] / gm);
+        double br = nearbyint(bs);
+        if (br < (double)b_min) br = (double)b_min;
+        if (br > (double)b_max) br = (double)b_max;
+        b[i] = (int)br;
+      } else {
+        b[i] = b_min;
+      }
+    }
+  }
+  for (int i = 0; i < N; ++i) {
+    if (b[i] < b_min) b[i] = b_min;
+    if (b[i] > b_max) b[i] = b_max;
+  }
+  long sum = 0;
+  for (int i = 0; i < N; ++i) sum += b[i];
+  while (sum > target) {
+    int pick = -1;
+    double pv = 0.0;
+    for (int i = 0; i < N; ++i)
+      if (b[i] > b_min) {
+        double m = (3.0 * c[i]) * ldexp(1.0, -2 * b[i]);
+        if (pick < 0 || m < pv) {
+          pick = i;
+          pv = m;
+        }
+      }
+    b[pick] -= 1;
+    sum -= 1;
+  }
+  while (sum < target) {
+    int pick = -1;
+    double pv = 0.0;
+    for (int i = 0; i < N; ++i)
+      if (b[i] < b_max) {
+        double m = (0.75 * c[i]) * ldexp(1.0, -2 * b[i]);
+        if (pick < 0 || m > pv) {
+          pick = i;
+          pv = m;
+        }
+      }
+    b[pick] += 1;
+    sum += 1;
+  }
+  for (int i = 0; i < N; ++i) bits[i] = (uint8_t)b[i];
+  free(b);
+  return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Storage layout (the byte format the CUDA library documents in its        */
+/* header; restated here independently).                                    */
+/*   FP32:   float [B][H][d][d], rows in stored (permuted) order.            */
+/*   DAMP:   per head, contiguous: FP16 rows [k_hi][d], INT8 codes           */
+/*           [d-k_hi][d], then per INT row and block an FP16 (scale, zero)   */
+/*           pair.  Error-feedback residuals: FP16 [B][H][d-k_hi][d].        */
+/*   VARBIT: [payload B x P bytes][FP16 scale B*H*d][u8 width B*H*d]         */
+/*           [u32 row offset B*(H*d+1)], each section starting on a 256-byte */
+/*           boundary; P = (d/8) * avg_bits * H * d; row i of sequence b     */
+/*           starts at byte offset[i] = (d/8) * sum of the widths before it. */
+/*           Residuals FP16 [B][H][d][d]; statistics FP64 [B][H][d][2].      */
+/* ------------------------------------------------------------------------ */
+static size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+static size_t damp_head_bytes(const orc_layout* L) {
+  size_t d = (size_t)L->d, kh = (size_t)L->k_hi;
+  return kh * d * 2 + (d - kh) * d + (d - kh) * (d / (size_t)L->block) * 4;
+}
+
+typedef struct {
+  size_t payload_per_seq, off_scale, off_width, off_offsets, total;
+} vb_sections;
+
+static vb_sections varbit_sections(const orc_layout* L) {
+  vb_sections s;
+  size_t rows = (size_t)L->H * (size_t)L->d;
+  s.payload_per_seq = (size_t)((double)(L->d / 8) * L->avg_bits * (double)rows);
+  s.off_scale = round256(s.payload_per_seq * (size_t)L->B);
+  s.off_width = s.off_scale + round256(rows * (size_t)L->B * 2);
+  s.off_offsets = s.off_width + round256(rows * (size_t)L->B);
+  s.total = s.off_offsets + round256((rows + 1) * (size_t)L->B * 4);
+  return s;
+}
+
+size_t orc_state_bytes(const orc_layout* L, size_t* aux_bytes, size_t* stats_bytes) {
+  size_t heads = (size_t)L->B * (size_t)L->H, d = (size_t)L->d;
+  size_t total = 0, aux = 0, stats = 0;
+  if (L->storage == ORC_STORE_FP32) {
+    total = heads * d * d * 4;
+  } else if (L->storage == ORC_STORE_DAMP) {
+    total = heads * damp_head_bytes(L);
+    aux = heads * (d - (size_t)L->k_hi) * d * 2;
+  } else {
+    total = varbit_sections(L).total;
+    aux = heads * d * d * 2;
+    stats = heads * d * 2 * sizeof(double);
+  }
+  if (aux_bytes) *aux_bytes = aux;
+  if (stats_bytes) *stats_bytes = stats;
+  return total;
+}
+
+/* Bits per stored value counted the way the pages count them: DAMP = FP16
+ * rows + INT8 rows + 32 bits of (scale, zero) per block ([LB] Related work;
+ * [DAMP] main operating point); VARBIT = mean width + one FP16 scale and one
+ * 3-bit width per row ([LB] Levels and storage). */
+double orc_bits_per_value(const orc_layout* L) {
+  double d = (double)L->d, kh = (double)L->k_hi;
+  if (L->storage == ORC_STORE_FP32) return 32.0;
+  if (L->storage == ORC_STORE_DAMP)
+    return (kh * d * 16.0 + (d - kh) * d * 8.0 + (d - kh) * (d / L->block) * 32.0) / (d * d);
+  return L->avg_bits + (16.0 + 3.0) / d;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Per-head state in the working domain                                      */
+/* ------------------------------------------------------------------------ */
+static int rotated(const orc_layout* L) {
+  return L->domain == ORC_DOMAIN_ROTATED && L->storage == ORC_STORE_DAMP && L->hadamard;
+}
+
+/* Dequantize one DAMP head into S (d x d, stored row order).  In the
+ * canonical domain INT8 rows are returned to the value basis with the
+ * Hadamard (its own inverse); in the rotated domain the FP16 rows are taken
+ * to the Hadamard basis instead. */
+static void damp_load(const orc_layout* L, const uint8_t* head, float* S) {
+  int d = L->d, kh = L->k_hi, nb = d / L->block;
+  const uint16_t* f16rows = (const uint16_t*)head;
+  const uint8_t* codes = head + (size_t)kh * d * 2;
+  const uint16_t* sz = (const uint16_t*)(codes + (size_t)(d - kh) * d);
+  for (int i = 0; i < d; ++i) {
+    float* row = S + (size_t)i * d;
+    if (i < kh) {
+      for (int j = 0; j < d; ++j) row[j] = orc_f32_from_f16(f16rows[(size_t)i * d + j]);
+      if (rotated(L)) orc_fwht(row, d);
+    } else {
+      int r = i - kh;
+      for (int j = 0; j < d; ++j) {
+        int bl = j / L->block;
+        float s = orc_f32_from_f16(sz[((size_t)r * nb + bl) * 2 + 0]);
+        float z = orc_f32_from_f16(sz[((size_t)r * nb + bl) * 2 + 1]);
+        row[j] = fmaf((float)codes[(size_t)r * d + j], s, z);
+      }
+      if (L->hadamard && !rotated(L)) orc_fwht(row, d);
+    }
+  }
+}
+
+static int damp_store(const orc_layout* L, const orc_writeback* wb, int64_t step, int b, int h,
+                      const float* S, uint8_t* head, uint16_t* aux_head, float* t_head) {
+  int d = L->d, kh = L->k_hi, nb = d / L->block, flags = 0;
+  uint16_t* f16rows = (uint16_t*)head;
+  uint8_t* codes = head + (size_t)kh * d * 2;
+  uint16_t* sz = (uint16_t*)(codes + (size_t)(d - kh) * d);
+  float* tmp = (float*)malloc(sizeof(float) * (size_t)d);
+  for (int i = 0; i < d; ++i) {
+    memcpy(tmp, S + (size_t)i * d, sizeof(float) * (size_t)d);
+    if (i < kh) {
+      if (rotated(L)) orc_fwht(tmp, d);
+      for (int j = 0; j < d; ++j) {
+        if (!isfinite(tmp[j])) flags |= ORC_ENONFINITE;
+        uint16_t hv = orc_f16_from_f32(tmp[j]);
+        if (f16_is_inf_or_nan(hv) && isfinite(tmp[j])) flags |= ORC_EOVERFLOW;
+        f16rows[(size_t)i * d + j] = hv;
+        if (t_head) t_head[(size_t)i * d + j] = 0.0f;
+      }
+    } else {
+      int r = i - kh;
+      if (L->hadamard && !rotated(L)) orc_fwht(tmp, d);
+      for (int bl = 0; bl < nb; ++bl) {
+        int j0 = bl * L->block;
+        uint16_t* e = aux_head ? aux_head + (size_t)r * d + j0 : NULL;
+        flags |= orc_int8_block(tmp + j0, L->block, wb->mode, wb->seed, step, h, b, i * d + j0, e,
+                                codes + (size_t)r * d + j0, &sz[((size_t)r * nb + bl) * 2 + 0],
+                                &sz[((size_t)r * nb + bl) * 2 + 1],
+                                t_head ? t_head + (size_t)i * d + j0 : NULL);
+      }
+    }
+  }
+  free(tmp);
+  return flags;
+}
+
+/* ------------------------------------------------------------------------ */
+/* One token of the gated delta rule on one head, in FP32 ([DAMP] Error      */
+/* propagation model: S = Q(A_t S + beta_t k_t v_t^T) with A_t the decayed   */
+/* delta-rule map; [LB] Accumulated readout error: outputs are read before   */
+/* the write-back quantizes the state):                                     */
+/*   S <- Diag(a) S;  u = S^T k;  w = beta (v - u);  S <- S + k w^T;         */
+/*   o = S^T q.                                                              */
+/* kk, qq, aa are gathered in stored row order; vv and the returned oo are  */
+/* in the basis of S's columns.                                             */
+/* ------------------------------------------------------------------------ */
+static void delta_rule_token(int d, float* S, const float* kk, const float* qq, const float* aa,
+                             const float* vv, float bt, float* w, float* oo) {
+  for (int i = 0; i < d; ++i)
+    for (int j = 0; j < d; ++j) S[(size_t)i * d + j] = aa[i] * S[(size_t)i * d + j];
+  for (int j = 0; j < d; ++j) {
+    float u = 0.0f;
+    for (int i = 0; i < d; ++i) u = fmaf(kk[i], S[(size_t)i * d + j], u);
+    w[j] = bt * (vv[j] - u);
+  }
+  for (int i = 0; i < d; ++i)
+    for (int j = 0; j < d; ++j) S[(size_t)i * d + j] = fmaf(kk[i], w[j], S[(size_t)i * d + j]);
+  for (int j = 0; j < d; ++j) {
+    float acc = 0.0f;
+    for (int i = 0; i < d; ++i) acc = fmaf(qq[i], S[(size_t)i * d + j], acc);
+    oo[j] = acc;
+  }
+}
+
+typedef struct {
+  const uint16_t *q, *k, *v;
+  const float *beta, *decay;
+  float* o;
+} orc_inputs;
+
+/* Gather token t's inputs for head (b, h) in stored row order. */
+static void gather_token(const orc_layout* L, const orc_inputs* in, int t, int b, int h,
+                         const int16_t* perm_h, float* kk, float* qq, float* aa, float* vv,
+                         float* bt) {
+  int d = L->d, B = L->B, H = L->H, Hk = L->Hk;
+  int kh = h * Hk / H;
+  size_t qk_base = (((size_t)t * B + b) * Hk + kh) * d;
+  size_t v_base = (((size_t)t * B + b) * H + h) * d;
+  for (int i = 0; i < d; ++i) {
+    int p = perm_h ? perm_h[i] : i;
+    kk[i] = orc_f32_from_bf16(in->k[qk_base + p]);
+    qq[i] = orc_f32_from_bf16(in->q[qk_base + p]);
+    aa[i] = L->decay_per_key ? in->decay[v_base + p] : in->decay[((size_t)t * B + b) * H + h];
+  }
+  for (int j = 0; j < d; ++j) vv[j] = orc_f32_from_bf16(in->v[v_base + j]);
+  *bt = in->beta[((size_t)t * B + b) * H + h];
+}
+
+static int run_head_unit(const orc_layout* L, const orc_writeback* wb, int64_t step0, int T,
+                         int b, int h, const uint8_t* pin, uint8_t* pout, uint16_t* aux,
+                         const int16_t* perm, const orc_inputs* in, float* t_dump) {
+  int d = L->d, flags = 0;
+  size_t unit = (size_t)b * L->H + h;
+  float* S = (float*)malloc(sizeof(float) * (size_t)d * d);
+  float *kk = malloc(sizeof(float) * d), *qq = malloc(sizeof(float) * d),
+        *aa = malloc(sizeof(float) * d), *vv = malloc(sizeof(float) * d),
+        *w = malloc(sizeof(float) * d), *oo = malloc(sizeof(float) * d);
+  const int16_t* perm_h = perm ? perm + (size_t)h * d : NULL;
+  size_t hb = (L->storage == ORC_STORE_FP32) ? (size_t)d * d * 4 : damp_head_bytes(L);
+
+  if (L->storage == ORC_STORE_FP32)
+    memcpy(S, pin + unit * hb, hb);
+  else
+    damp_load(L, pin + unit * hb, S);
+
+  for (int t = 0; t < T; ++t) {
+    int64_t step = step0 + t;
+    float bt;
+    gather_token(L, in, t, b, h, perm_h, kk, qq, aa, vv, &bt);
+    if (rotated(L)) orc_fwht(vv, d);
+    delta_rule_token(d, S, kk, qq, aa, vv, bt, w, oo);
+    if (rotated(L)) orc_fwht(oo, d);
+    memcpy(in->o + (((size_t)t * L->B + b) * L->H + h) * d, oo, sizeof(float) * (size_t)d);
+    if ((step + 1) % wb->C == 0) {
+      /* write-back: quantize, then continue from the dequantized state
+       * ([LB] Protocol: each write-back is quantized and dequantized before
+       * reuse; no unquantized residual is retained) */
+      if (L->storage == ORC_STORE_FP32) {
+        for (size_t e = 0; e < (size_t)d * d; ++e)
+          if (!isfinite(S[e])) flags |= ORC_ENONFINITE;
+        memcpy(pout + unit * hb, S, hb);
+      } else {
+        uint16_t* aux_head = aux ? aux + unit * (size_t)(d - L->k_hi) * d : NULL;
+        float* th = t_dump ? t_dump + unit * (size_t)d * d : NULL;
+        flags |= damp_store(L, wb, step, b, h, S, pout + unit * hb, aux_head, th);
+        damp_load(L, pout + unit * hb, S);
+      }
+    }
+  }
+  free(S);
+  free(kk);
+  free(qq);
+  free(aa);
+  free(vv);
+  free(w);
+  free(oo);
+  return flags;
+}
+
+/* ---- variable-width storage ([LB] State bit allocation, Allocation units,
+ * Levels and storage) ---- */
+static uint32_t get_bits(const uint8_t* p, size_t bitpos, int nb) {
+  uint32_t v = 0;
+  for (int k = 0; k < nb; ++k) {
+    size_t bp = bitpos + (size_t)k;
+    v |= (uint32_t)((p[bp >> 3] >> (bp & 7)) & 1u) << k;
+  }
+  return v;
+}
+
+static void put_bits(uint8_t* p, size_t bitpos, int nb, uint32_t v) {
+  for (int k = 0; k < nb; ++k) {
+    size_t bp = bitpos + (size_t)k;
+    uint8_t m = (uint8_t)(1u << (bp & 7));
+    if ((v >> k) & 1u)
+      p[bp >> 3] |= m;
+    else
+      p[bp >> 3] &= (uint8_t)~m;
+  }
+}
+
+static void varbit_load_seq(const orc_layout* L, const uint8_t* packed, int b, float* S) {
+  vb_sections sec = varbit_sections(L);
+  int d = L->d, rows = L->H * d;
+  const uint8_t* pay = packed + (size_t)b * sec.payload_per_seq;
+  const uint16_t* sc = (const uint16_t*)(packed + sec.off_scale) + (size_t)b * rows;
+  const uint8_t* wd = packed + sec.off_width + (size_t)b * rows;
+  const uint32_t* of = (const uint32_t*)(packed + sec.off_offsets) + (size_t)b * (rows + 1);
+  for (int r = 0; r < rows; ++r) {
+    int bw = wd[r];
+    int nl = (1 << (bw - 1)) - 1;
+    float D = orc_f32_from_f16(sc[r]);
+    for (int j = 0; j < d; ++j) {
+      uint32_t u = get_bits(pay + of[r], (size_t)j * bw, bw);
+      S[(size_t)r * d + j] = (float)((int)u - nl) * D;
+    }
+  }
+}
+
+/* Quantize every row of sequence b with widths `bits` and write payload,
+ * scales, widths and offsets. */
+static int varbit_store_seq(const orc_layout* L, const orc_writeback* wb, int64_t step, int b,
+                            const float* S, const uint8_t* bits, uint8_t* packed, uint16_t* aux,
+                            float* t_dump) {
+  vb_sections sec = varbit_sections(L);
+  int d = L->d, rows = L->H * d, flags = 0;
+  uint8_t* pay = packed + (size_t)b * sec.payload_per_seq;
+  uint16_t* sc = (uint16_t*)(packed + sec.off_scale) + (size_t)b * rows;
+  uint8_t* wd = packed + sec.off_width + (size_t)b * rows;
+  uint32_t* of = (uint32_t*)(packed + sec.off_offsets) + (size_t)b * (rows + 1);
+  int32_t* q = (int32_t*)malloc(sizeof(int32_t) * (size_t)d);
+  uint32_t off = 0;
+  for (int r = 0; r < rows; ++r) {
+    of[r] = off;
+    off += (uint32_t)(d / 8) * bits[r];
+  }
+  of[rows] = off;
+  for (int r = 0; r < rows; ++r) {
+    int h = r / d, i = r % d, bw = bits[r];
+    int nl = (1 << (bw - 1)) - 1;
+    uint16_t* e = aux ? aux + ((size_t)b * rows + r) * d : NULL;
+    float* tt = t_dump ? t_dump + ((size_t)b * rows + r) * d : NULL;
+    flags |= orc_varbit_row(S + (size_t)r * d, d, bw, wb ? wb->mode : ORC_ROUND_NEAREST,
+                            wb ? wb->seed : 0, step, h, b, i * d, e, q, &sc[r], NULL, tt);
+    wd[r] = (uint8_t)bw;
+    for (int j = 0; j < d; ++j) put_bits(pay + of[r], (size_t)j * bw, bw, (uint32_t)(q[j] + nl));
+  }
+  free(q);
+  return flags;
+}
+
+static int run_seq_unit(const orc_layout* L, const orc_writeback* wb, int64_t step0, int T, int b,
+                        const uint8_t* pin, uint8_t* pout, uint16_t* aux, double* stats,
+                        const orc_inputs* in, float* t_dump) {
+  int d = L->d, H = L->H, rows = H * d, flags = 0;
+  float* S = (float*)malloc(sizeof(float) * (size_t)rows * d);
+  float *kk = malloc(sizeof(float) * d), *qq = malloc(sizeof(float) * d),
+        *aa = malloc(sizeof(float) * d), *vv = malloc(sizeof(float) * d),
+        *w = malloc(sizeof(float) * d), *oo = malloc(sizeof(float) * d);
+  double* ca2 = (double*)calloc((size_t)rows, sizeof(double));
+  double* ck = (double*)calloc((size_t)rows, sizeof(double));
+  double* cost = (double*)malloc(sizeof(double) * (size_t)rows);
+  double* Rr = (double*)malloc(sizeof(double) * (size_t)rows);
+  uint8_t* bits = (uint8_t*)malloc((size_t)rows);
+  double* st = stats + (size_t)b * rows * 2;
+  int C = wb->C;
+  double lam = 1.0;
+  for (int c = 0; c < C; ++c) lam *= (1.0 - 2.0 / 65.0);
+
+  varbit_load_seq(L, pin, b, S);
+  for (int t = 0; t < T; ++t) {
+    int64_t step = step0 + t;
+    for (int h = 0; h < H; ++h) {
+      float bt;
+      gather_token(L, in, t, b, h, NULL, kk, qq, aa, vv, &bt);
+      delta_rule_token(d, S + (size_t)h * d * d, kk, qq, aa, vv, bt, w, oo);
+      memcpy(in->o + (((size_t)t * L->B + b) * H + h) * d, oo, sizeof(float) * (size_t)d);
+      /* per-token erasure statistics ([LB] State bit allocation: EMA of
+       * e^(2g) = a^2 and of beta (2 - beta) k^2) */
+      for (int i = 0; i < d; ++i) {
+        double a = (double)aa[i], be = (double)bt, kd = (double)kk[i];
+        ca2[h * d + i] += a * a;
+        ck[h * d + i] += (be * (2.0 - be)) * (kd * kd);
+      }
+    }
+    if ((step + 1) % C == 0) {
+      /* chunk-aware EMA with a 64-token span, initialised at the first
+       * write-back */
+      for (int r = 0; r < rows; ++r) {
+        double ma = ca2[r] / (double)C, mk = ck[r] / (double)C;
+        if (step + 1 == C) {
+          st[2 * r + 0] = ma;
+          st[2 * r + 1] = mk;
+        } else {
+          st[2 * r + 0] = lam * st[2 * r + 0] + (1.0 - lam) * ma;
+          st[2 * r + 1] = lam * st[2 * r + 1] + (1.0 - lam) * mk;
+        }
+        ca2[r] = 0.0;
+        ck[r] = 0.0;
+      }
+      /* cost c_i = Gamma_hat_i * R~_i^2 with R~ the row range normalised by
+       * the RMS of the ranges of its output group (one head) */
+      for (int r = 0; r < rows; ++r) {
+        float R = 0.0f;
+        for (int j = 0; j < d; ++j) {
+          float a = fabsf(S[(size_t)r * d + j]);
+          if (a > R) R = a;
+        }
+        Rr[r] = (double)R;
+      }
+      for (int h = 0; h < H; ++h) {
+        double ms = 0.0;
+        for (int i = 0; i < d; ++i) ms += Rr[h * d + i] * Rr[h * d + i];
+        double rms = sqrt(ms / (double)d);
+        for (int i = 0; i < d; ++i) {
+          int r = h * d + i;
+          double rt = rms > 0.0 ? Rr[r] / rms : 0.0;
+          cost[r] = orc_gamma_hat(st[2 * r + 0], st[2 * r + 1], C) * (rt * rt);
+        }
+      }
+      if (L->budget_scope == 1) {
+        flags |= orc_allocate_bits(rows, cost, L->avg_bits, L->b_min, L->b_max, bits);
+      } else {
+        for (int h = 0; h < H; ++h)
+          flags |= orc_allocate_bits(d, cost + h * d, L->avg_bits, L->b_min, L->b_max,
+                                     bits + h * d);
+      }
+      if (flags & ORC_EINVAL) break;
+      flags |= varbit_store_seq(L, wb, step, b, S, bits, pout, aux, t_dump);
+      varbit_load_seq(L, pout, b, S);
+    }
+  }
+  free(S);
+  free(kk);
+  free(qq);
+  free(aa);
+  free(vv);
+  free(w);
+  free(oo);
+  free(ca2);
+  free(ck);
+  free(cost);
+  free(Rr);
+  free(bits);
+  return flags;
+}
+
+static int layout_ok(const orc_layout* L) {
+  if (L->B <= 0 || L->H <= 0 || L->Hk <= 0 || L->H % L->Hk) return 0;
+  if (L->d != 16 && L->d != 32 && L->d != 64 && L->d != 128) return 0;
+  if (L->storage == ORC_STORE_DAMP) {
+    if (L->k_hi < 0 || L->k_hi > L->d || L->block <= 0 || L->d % L->block) return 0;
+  }
+  if (L->storage == ORC_STORE_VARBIT) {
+    if (L->hadamard || L->b_min < 2 || L->b_max > 8 || L->b_min > L->b_max) return 0;
+    double tot = L->avg_bits * (double)(L->H * L->d);
+    if (tot != floor(tot)) return 0;
+  }
+  return 1;
+}
+
+int orc_run(const orc_layout* L, const orc_writeback* wb, int64_t step0, int T, int u0, int u1,
+            const void* packed_in, void* packed_out, void* aux, double* stats,
+            const int16_t* perm, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+            const float* beta, const float* decay, float* o, float* t_dump) {
+  if (!layout_ok(L) || wb->C <= 0 || step0 % wb->C || T % wb->C) return ORC_EINVAL;
+  orc_inputs in = {q, k, v, beta, decay, o};
+  int flags = 0;
+  if (L->storage == ORC_STORE_VARBIT) {
+    for (int b = u0; b < u1; ++b)
+      flags |= run_seq_unit(L, wb, step0, T, b, (const uint8_t*)packed_in, (uint8_t*)packed_out,
+                            (uint16_t*)aux, stats, &in, t_dump);
+  } else {
+    for (int u = u0; u < u1; ++u)
+      flags |= run_head_unit(L, wb, step0, T, u / L->H, u % L->H, (const uint8_t*)packed_in,
+                             (uint8_t*)packed_out, (uint16_t*)aux, perm, &in, t_dump);
+  }
+  return flags;
+}
+
+/* ------------------------------------------------------------------------ */
+/* State conversion (deterministic rounding)                                 */
+/* ------------------------------------------------------------------------ */
+int orc_state_pack(const orc_layout* L, const float* S, const int16_t* perm,
+                   const uint8_t* widths, void* packed) {
+  if (!layout_ok(L)) return ORC_EINVAL;
+  int d = L->d, flags = 0;
+  orc_writeback wb = {ORC_ROUND_NEAREST, 0, 1};
+  orc_layout Lc = *L;
+  Lc.domain = ORC_DOMAIN_CANONICAL;
+  float* tmp = (float*)malloc(sizeof(float) * (size_t)d * d);
+  if (L->storage == ORC_STORE_VARBIT) {
+    int rows = L->H * d;
+    uint8_t* bits = (uint8_t*)malloc((size_t)rows);
+    float* seq = (float*)malloc(sizeof(float) * (size_t)rows * d);
+    for (int r = 0; r < rows; ++r) bits[r] = widths ? widths[r] : (uint8_t)nearbyint(L->avg_bits);
+    for (int b = 0; b < L->B; ++b) {
+      memcpy(seq, S + (size_t)b * rows * d, sizeof(float) * (size_t)rows * d);
+      flags |= varbit_store_seq(L, NULL, 0, b, seq, widths ? widths + (size_t)b * rows : bits,
+                                (uint8_t*)packed, NULL, NULL);
+    }
+    free(bits);
+    free(seq);
+  } else {
+    size_t hb = (L->storage == ORC_STORE_FP32) ? (size_t)d * d * 4 : damp_head_bytes(L);
+    for (int b = 0; b < L->B; ++b)
+      for (int h = 0; h < L->H; ++h) {
+        const float* src = S + ((size_t)b * L->H + h) * d * d;
+        for (int i = 0; i < d; ++i) {
+          int p = perm ? perm[(size_t)h * d + i] : i;
+          memcpy(tmp + (size_t)i * d, src + (size_t)p * d, sizeof(float) * (size_t)d);
+        }
+        uint8_t* dst = (uint8_t*)packed + ((size_t)b * L->H + h) * hb;
+        if (L->storage == ORC_STORE_FP32)
+          memcpy(dst, tmp, hb);
+        else
+          flags |= damp_store(&Lc, &wb, 0, b, h, tmp, dst, NULL, NULL);
+      }
+  }
+  free(tmp);
+  return flags;
+}
+
+int orc_state_unpack(const orc_layout* L, const void* packed, const int16_t* perm, float* S) {
+  if (!layout_ok(L)) return ORC_EINVAL;
+  int d = L->d;
+  orc_layout Lc = *L;
+  Lc.domain = ORC_DOMAIN_CANONICAL;
+  if (L->storage == ORC_STORE_VARBIT) {
+    for (int b = 0; b < L->B; ++b)
+      varbit_load_seq(L, (const uint8_t*)packed, b, S + (size_t)b * L->H * d * d);
+    return ORC_OK;
+  }
+  float* tmp = (float*)malloc(sizeof(float) * (size_t)d * d);
+  size_t hb = (L->storage == ORC_STORE_FP32) ? (size_t)d * d * 4 : damp_head_bytes(L);
+  for (int b = 0; b < L->B; ++b)
+    for (int h = 0; h < L->H; ++h) {
+      const uint8_t* src = (const uint8_t*)packed + ((size_t)b * L->H + h) * hb;
+      if (L->storage == ORC_STORE_FP32)
+        memcpy(tmp, src, hb);
+      else
+        damp_load(&Lc, src, tmp);
+      float* dst = S + ((size_t)b * L->H + h) * d * d;
+      for (int i = 0; i < d; ++i) {
+        int p = perm ? perm[(size_t)h * d + i] : i;
+        memcpy(dst + (size_t)p * d, tmp + (size_t)i * d, sizeof(float) * (size_t)d);
+      }
+    }
+  free(tmp);
+  return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Protected-row selection ([DAMP] Risk scoring and selection; Calibration): */
+/*   E_u  = mean squared error energy of row u under Hadamard-INT8           */
+/*          quantize -> dequantize, over the sampled calibration states;     */
+/*   a_eff,u = exp(mean log a_u);  P_u = 1 / max(1 - a_eff,u^2, tau);        */
+/*   C_u = E_u P_u; the top k_hi rows of each head are protected (ties to    */
+/*   the lower index) and placed first, both groups in ascending order.      */
+/* ------------------------------------------------------------------------ */
+int orc_calibrate(const orc_layout* L, int Bc, int T, int every, double tau,
+                  const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* beta,
+                  const float* decay, double* score_out, int16_t* perm_out) {
+  orc_layout Lc = *L;
+  Lc.B = Bc;
+  if (!layout_ok(&Lc) || L->storage != ORC_STORE_DAMP || every <= 0) return ORC_EINVAL;
+  int d = L->d, H = L->H, nb = d / L->block;
+  orc_inputs in = {q, k, v, beta, decay, NULL};
+  double* E = (double*)calloc((size_t)H * d, sizeof(double));
+  double* sl = (double*)calloc((size_t)H * d, sizeof(double));
+  float* S = (float*)malloc(sizeof(float) * (size_t)d * d);
+  float *kk = malloc(sizeof(float) * d), *qq = malloc(sizeof(float) * d),
+        *aa = malloc(sizeof(float) * d), *vv = malloc(sizeof(float) * d),
+        *w = malloc(sizeof(float) * d), *oo = malloc(sizeof(float) * d),
+        *row = malloc(sizeof(float) * d);
+  uint8_t* codes = (uint8_t*)malloc((size_t)L->block);
+  long nsamp = 0;
+  for (int b = 0; b < Bc; ++b)
+    for (int h = 0; h < H; ++h) {
+      memset(S, 0, sizeof(float) * (size_t)d * d);
+      for (int t = 0; t < T; ++t) {
+        float bt;
+        gather_token(&Lc, &in, t, b, h, NULL, kk, qq, aa, vv, &bt);
+        for (int i = 0; i < d; ++i) sl[h * d + i] += log((double)aa[i]);
+        delta_rule_token(d, S, kk, qq, aa, vv, bt, w, oo);
+        if ((t + 1) % every == 0) {
+          if (b == 0 && h == 0) ++nsamp;
+          for (int i = 0; i < d; ++i) {
+            memcpy(row, S + (size_t)i * d, sizeof(float) * (size_t)d);
+            if (L->hadamard) orc_fwht(row, d);
+            double err = 0.0;
+            for (int bl = 0; bl < nb; ++bl) {
+              uint16_t sh, zh;
+              int j0 = bl * L->block;
+              orc_int8_block(row + j0, L->block, ORC_ROUND_NEAREST, 0, 0, 0, 0, 0, NULL, codes,
+                             &sh, &zh, NULL);
+              float s = orc_f32_from_f16(sh), z = orc_f32_from_f16(zh);
+              for (int j = 0; j < L->block; ++j) {
+                double e = (double)row[j0 + j] - (double)fmaf((float)codes[j], s, z);
+                err += e * e;
+              }
+            }
+            E[h * d + i] += err;
+          }
+        }
+      }
+    }
+  double ns = (double)Bc * (double)nsamp, nt = (double)Bc * (double)T;
+  int* idx = (int*)malloc(sizeof(int) * (size_t)d);
+  double* sc = (double*)malloc(sizeof(double) * (size_t)d);
+  char* prot = (char*)malloc((size_t)d);
+  for (int h = 0; h < H; ++h) {
+    for (int i = 0; i < d; ++i) {
+      double aeff = exp(sl[h * d + i] / nt);
+      double den = 1.0 - aeff * aeff;
+      if (den < tau) den = tau;
+      sc[i] = (E[h * d + i] / ns) * (1.0 / den);
+      if (score_out) score_out[(size_t)h * d + i] = sc[i];
+      prot[i] = 0;
+    }
+    /* pick the k_hi largest scores, ties to the lower index */
+    for (int c = 0; c < L->k_hi; ++c) {
+      int pick = -1;
+      for (int i = 0; i < d; ++i)
+        if (!prot[i] && (pick < 0 || sc[i] > sc[pick])) pick = i;
+      prot[pick] = 1;
+    }
+    int n = 0;
+    for (int i = 0; i < d; ++i)
+      if (prot[i]) idx[n++] = i;
+    for (int i = 0; i < d; ++i)
+      if (!prot[i]) idx[n++] = i;
+    for (int i = 0; i < d; ++i) perm_out[(size_t)h * d + i] = (int16_t)idx[i];
+  }
+  free(idx);
+  free(sc);
+  free(prot);
+  free(E);
+  free(sl);
+  free(S);
+  free(kk);
+  free(qq);
+  free(aa);
+  free(vv);
+  free(w);
+  free(oo);
+  free(row);
+  free(codes);
+  return ORC_OK;
+}

@@ -1,0 +1,172 @@
+"""Pins of the oracle's write-back quantizers: exhaustive level search,
+tie-to-even, grid rails, unbiased stochastic rounding, error-feedback
+bounds, the write dead zone, the variable-width fit against an exhaustive
+FP64 scan."""
+import numpy as np
+import pytest
+
+from conftest import golden
+
+
+def f16(x):
+    return np.float32(np.float16(np.float32(x)))
+
+
+def test_int8_codes_are_nearest_level(orc):
+    rng = np.random.default_rng(1)
+    for trial in range(200):
+        n = [32, 128][trial % 2]
+        y = (rng.standard_normal(n) * 10.0 ** rng.uniform(-3, 2)).astype(np.float32)
+        r = orc.int8_block(y)
+        s = np.float64(np.uint16(r["scale"]).view(np.float16))
+        z = np.float64(np.uint16(r["zero"]).view(np.float16))
+        # the stored grid brackets the block (FP16 rounding of min and step)
+        assert abs(z - y.min()) <= 2 ** -11 * abs(y.min()) + 2 ** -25
+        assert abs(s * 255 - (y.max() - y.min())) <= 255 * 2 ** -11 * s + 2 ** -24 * 255
+        levels = np.arange(256) * s + z
+        dist = np.abs(y[:, None].astype(np.float64) - levels[None, :])
+        best = dist.min(axis=1)
+        got = dist[np.arange(n), r["codes"]]
+        # nearest level up to the FP32 rounding of the grid coordinate
+        assert np.all(got - best <= 1e-5 * s + 1e-30), trial
+
+
+def test_int8_ties_to_even_and_rails(orc):
+    # block spanning [0, 255] has step 1 and zero 0: t = y exactly
+    y = np.zeros(32, np.float32)
+    y[0], y[1] = 0.0, 255.0
+    y[2:8] = [2.5, 3.5, 4.5, 0.5, 253.5, 254.5]
+    r = orc.int8_block(y)
+    assert r["scale"] == np.float16(1.0).view(np.uint16)
+    assert list(r["codes"][2:8]) == [2, 4, 4, 0, 254, 254]
+    # rails: a zero rounded above the minimum gives t < 0 -> clipped to 0
+    y2 = np.linspace(1000.1, 1100.0, 32).astype(np.float32)
+    r2 = orc.int8_block(y2)
+    assert r2["codes"].min() == 0 and r2["codes"].max() <= 255
+
+
+def test_int8_constant_block(orc):
+    y = np.full(32, 3.25, np.float32)
+    r = orc.int8_block(y)
+    assert r["scale"] == 0 and np.all(r["codes"] == 0)
+    assert np.float16(np.uint16(r["zero"]).view(np.float16)) == np.float16(3.25)
+
+
+def test_stochastic_rounding_unbiased_and_reproducible(orc):
+    rng = np.random.default_rng(2)
+    y = (rng.standard_normal(32)).astype(np.float32)
+    a = orc.int8_block(y, mode=orc.ROUND_STOCHASTIC, seed=7, step=3, h=1, b=2)
+    b = orc.int8_block(y, mode=orc.ROUND_STOCHASTIC, seed=7, step=3, h=1, b=2)
+    np.testing.assert_array_equal(a["codes"], b["codes"])
+    s = np.float64(np.uint16(a["scale"]).view(np.float16))
+    z = np.float64(np.uint16(a["zero"]).view(np.float16))
+    N = 4000
+    acc = np.zeros(32)
+    for seed in range(N):
+        acc += orc.int8_block(y, mode=orc.ROUND_STOCHASTIC, seed=seed)["codes"]
+    mean_val = acc / N * s + z
+    t = (y.astype(np.float64) - z) / s
+    frac = t - np.floor(t)
+    sigma = s * np.sqrt(frac * (1 - frac) / N) + 1e-12
+    inside = (t >= 0) & (t <= 255)           # values past a rail are clipped, not unbiased
+    assert inside.sum() >= 28
+    assert np.all((np.abs(mean_val - y) <= 4 * sigma + 1e-5 * s)[inside])
+    # each code is one of the two adjacent levels
+    c = a["codes"].astype(np.float64)
+    assert np.all((c == np.floor(t)) | (c == np.floor(t) + 1) | (c == 0) | (c == 255))
+
+
+def test_error_feedback_residual_bounded(orc):
+    rng = np.random.default_rng(3)
+    e = np.zeros(32, np.uint16)
+    for step in range(50):
+        y = rng.standard_normal(32).astype(np.float32)
+        r = orc.int8_block(y, mode=orc.ROUND_ERRFEEDBACK, e=e)
+        s = np.float32(np.uint16(r["scale"]).view(np.float16))
+        ev = np.uint16(r["e"]).view(np.float16).astype(np.float32)
+        assert np.all(np.abs(ev) <= f16(s) + 1e-12)
+        e = r["e"]
+
+
+def _write_back_loop(orc, mode, delta, steps):
+    """Persistent drift of one interior value; min/max pinned so the step
+    stays 0.125 (the 4-bit grid spacing of the dead-zone fixture)."""
+    g = golden("dead_zone.txt")
+    D = float(g["delta_4"])
+    y = np.zeros(32, np.float32)
+    y[0], y[1] = 0.0, 255 * D            # step (max-min)/255 = 0.125 exactly
+    y[2] = 100 * D                        # on a level
+    e = np.zeros(32, np.uint16)
+    moved_at = None
+    cur = y.copy()
+    code0 = None
+    for t in range(steps):
+        target = cur.copy()
+        target[2] = cur[2] + np.float32(delta)
+        r = orc.int8_block(target, mode=mode, e=e if mode == orc.ROUND_ERRFEEDBACK else None,
+                           seed=11, step=t)
+        s = np.float32(np.uint16(r["scale"]).view(np.float16))
+        assert s == np.float32(D)
+        z = np.float32(np.uint16(r["zero"]).view(np.float16))
+        if code0 is None:
+            code0 = int(round(100))
+        if r["codes"][2] != code0 and moved_at is None:
+            moved_at = t
+        cur = (r["codes"].astype(np.float32) * s + z).astype(np.float32)
+        if mode == orc.ROUND_ERRFEEDBACK:
+            e = r["e"]
+    return moved_at
+
+
+def test_dead_zone_deterministic_never_moves(orc):
+    g = golden("dead_zone.txt")
+    half = float(g["half_step"])
+    delta = 0.8 * half                       # write margin M = 2|delta|/Delta = 0.8 < 1
+    assert 2 * delta / float(g["delta_4"]) < 1
+    assert _write_back_loop(orc, orc.ROUND_NEAREST, delta, 200) is None
+
+
+def test_dead_zone_error_feedback_moves(orc):
+    g = golden("dead_zone.txt")
+    delta = 0.1 * float(g["half_step"])      # far inside the dead zone
+    t = _write_back_loop(orc, orc.ROUND_ERRFEEDBACK, delta, 200)
+    # the residual crosses the half step after about half_step/delta steps
+    assert t is not None and t <= int(np.ceil(1 / 0.1)) + 1
+
+
+def test_dead_zone_stochastic_moves(orc):
+    g = golden("dead_zone.txt")
+    delta = 0.1 * float(g["half_step"])
+    assert _write_back_loop(orc, orc.ROUND_STOCHASTIC, delta, 400) is not None
+
+
+@pytest.mark.parametrize("bw", [2, 3, 4, 6, 8])
+def test_varbit_fit_matches_exhaustive_scan(orc, bw):
+    rng = np.random.default_rng(bw)
+    n_l = 2 ** (bw - 1) - 1
+    for trial in range(60):
+        x = (rng.standard_normal(128) * rng.uniform(0.01, 5)).astype(np.float32)
+        if trial % 3 == 0:
+            x[rng.integers(128)] *= 8                         # an outlier
+        r = orc.varbit_row(x, bw)
+        R = np.max(np.abs(x)).astype(np.float64)
+        # exhaustive FP64 scan of the 16 candidate steps, nearest level each
+        errs = []
+        for m in range(16):
+            D = np.float64(f16(np.float32(np.float32((5 + m) / 20) * np.float32(R)) / np.float32(n_l)))
+            lev = np.arange(-n_l, n_l + 1) * D
+            err = np.min((x[:, None].astype(np.float64) - lev[None, :]) ** 2, axis=1).sum()
+            errs.append(err)
+        errs = np.array(errs)
+        assert errs[r["m"]] <= errs.min() * (1 + 1e-5) + 1e-30, (trial, r["m"], errs)
+        D = np.float64(np.uint16(r["delta"]).view(np.float16))
+        lev = np.arange(-n_l, n_l + 1) * D
+        dist = np.abs(x[:, None].astype(np.float64) - lev[None, :])
+        got = dist[np.arange(128), r["q"] + n_l]
+        assert np.all(got - dist.min(axis=1) <= 1e-5 * D + 1e-30)
+        assert np.all(np.abs(r["q"]) <= n_l)
+
+
+def test_varbit_zero_row(orc):
+    r = orc.varbit_row(np.zeros(128, np.float32), 4)
+    assert r["delta"] == 0 and np.all(r["q"] == 0)

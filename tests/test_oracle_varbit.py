@@ -1,0 +1,92 @@
+"""Pins of the variable-width write-back (decay-aware allocation): layer
+budget, offsets, FP64 recomputation of the widths and of the update."""
+import math
+
+import numpy as np
+import pytest
+
+from bit_recurrent_state_b200 import synth
+from ref64 import bf16_to_f64, dense_step, f16_bits_to_f64, varbit_row_codes, varbit_sections
+
+
+@pytest.mark.parametrize("mode", [0, 1, 2])
+def test_varbit_teacher_forced_fp64(orc, mode):
+    B, H, d, T = 2, 2, 32, 6
+    w = synth.Workload("t", B=B, H=H, d=d, T=T, storage="varbit", hadamard=0, seed=20 + mode)
+    cfg = orc.Config(B=B, H=H, d=d, storage=orc.STORE_VARBIT, hadamard=0, avg_bits=4.0,
+                     b_min=2, b_max=8, budget_scope=1)
+    inp_all = synth.run_inputs(w, 0, T)
+    packed, aux, stats = orc.new_state(cfg)
+    lam = (1 - 2 / 65)
+    K64 = np.zeros((B, H * d))
+    near_ties = 0
+    for t in range(T):
+        before = packed.copy()
+        inp = {k: v[t:t + 1] for k, v in inp_all.items()}
+        o, fl, _ = orc.run(cfg, mode, 99, 1, t, inp, packed, aux=aux, stats=stats)
+        assert fl == 0
+        pay0, sc0, wd0, of0 = varbit_sections(before, B, H, d, 4.0)
+        pay, sc, wd, of = varbit_sections(packed, B, H, d, 4.0)
+        for b in range(B):
+            assert int(wd[b].astype(int).sum()) == 4 * H * d             # layer budget
+            np.testing.assert_array_equal(of[b][:-1], np.concatenate([[0], np.cumsum(wd[b].astype(int))[:-1]]) * (d // 8))
+            Rr = np.zeros(H * d)
+            S_new = np.zeros((H, d, d))
+            for h in range(H):
+                S = np.zeros((d, d))
+                for i in range(d):
+                    r = h * d + i
+                    bw = int(wd0[b, r]); nl = 2 ** (bw - 1) - 1
+                    S[i] = (varbit_row_codes(pay0[b], int(of0[b, r]), bw, d) - nl) * f16_bits_to_f64(sc0[b, r])
+                k, q, v, a, beta = (bf16_to_f64(inp["k"][0, b, h]), bf16_to_f64(inp["q"][0, b, h]),
+                                    bf16_to_f64(inp["v"][0, b, h]),
+                                    inp["decay"][0, b, h].astype(np.float64), float(inp["beta"][0, b, h]))
+                S, oo = dense_step(S, k, q, v, a, beta)
+                assert np.max(np.abs(o[0, b, h] - oo)) <= 1e-5 * (np.max(np.abs(oo)) + 1e-30)
+                S_new[h] = S
+                Rr[h * d:(h + 1) * d] = np.max(np.abs(S), axis=1)
+                kk = beta * (2 - beta) * k ** 2
+                K64[b, h * d:(h + 1) * d] = kk if t == 0 else lam * K64[b, h * d:(h + 1) * d] + (1 - lam) * kk
+            # widths from an FP64 recomputation of c = Gamma_hat * R~^2
+            a2 = np.concatenate([inp["decay"][0, b, h].astype(np.float64) ** 2 for h in range(H)])
+            s_hat = -0.5 * np.log(a2)
+            arg = np.maximum(2 * (s_hat + 0.5 * K64[b]), 1e-9)
+            gam = 1.0 / np.expm1(arg)
+            rms = np.sqrt(np.mean(Rr.reshape(H, d) ** 2, axis=1))
+            Rt = (Rr.reshape(H, d) / rms[:, None]).ravel()
+            c = gam * Rt ** 2
+            bits64, _ = orc.allocate_bits(c, 4.0, 2, 8)
+            bstar = 4.0 + 0.5 * np.log2(c / np.exp(np.mean(np.log(c))))
+            diff = bits64 != wd[b]
+            if diff.any():
+                # only where b* sits next to a half-integer
+                assert np.all(np.abs(np.abs(bstar[diff] - np.floor(bstar[diff])) - 0.5) < 1e-6)
+                near_ties += int(diff.sum())
+            # each row holds its nearest levels (deterministic) / adjacent ones (stochastic)
+            if mode == 0:
+                for r in range(H * d):
+                    bw = int(wd[b, r]); nl = 2 ** (bw - 1) - 1
+                    D = f16_bits_to_f64(sc[b, r])
+                    qv = varbit_row_codes(pay[b], int(of[b, r]), bw, d).astype(int) - nl
+                    x = S_new[r // d, r % d]
+                    if D == 0:
+                        assert np.all(qv == 0)
+                        continue
+                    lev = np.arange(-nl, nl + 1) * D
+                    dist = np.abs(x[:, None] - lev[None, :])
+                    got = dist[np.arange(d), qv + nl]
+                    assert np.all(got - dist.min(axis=1) <= 1e-4 * D)
+    assert near_ties <= 2
+
+
+def test_varbit_head_scope_budget(orc):
+    B, H, d, T = 1, 3, 32, 4
+    w = synth.Workload("t", B=B, H=H, d=d, T=T, storage="varbit", hadamard=0, seed=30)
+    cfg = orc.Config(B=B, H=H, d=d, storage=orc.STORE_VARBIT, hadamard=0, avg_bits=3.0,
+                     b_min=2, b_max=8, budget_scope=0)
+    packed, aux, stats = orc.new_state(cfg)
+    o, fl, _ = orc.run(cfg, 0, 0, 1, 0, synth.run_inputs(w, 0, T), packed, aux=aux, stats=stats)
+    assert fl == 0
+    _, _, wd, _ = varbit_sections(packed, B, H, d, 3.0)
+    for h in range(H):
+        assert int(wd[0, h * d:(h + 1) * d].astype(int).sum()) == 3 * d
