@@ -412,9 +412,10 @@ int orc_allocate_bits(int N, const double* c, double avg_bits, int b_min, int b_
 /* Storage layout (the byte format the CUDA library documents in its        */
 /* header; restated here independently).                                    */
 /*   FP32:   float [B][H][d][d], rows in stored (permuted) order.            */
-/*   DAMP:   per head, contiguous: FP16 rows [k_hi][d], INT8 codes           */
-/*           [d-k_hi][d], then per INT row and block an FP16 (scale, zero)   */
-/*           pair.  Error-feedback residuals: FP16 [B][H][d-k_hi][d].        */
+/*   DAMP:   per head, contiguous, in stored row order: INT8 codes          */
+/*           [d-k_hi][d] (rows 0..d-k_hi-1), FP16 rows [k_hi][d] (the        */
+/*           protected rows d-k_hi..d-1), then per INT8 row and block an     */
+/*           FP16 (scale, zero) pair.  Residuals: FP16 [B][H][d-k_hi][d].   */
 /*   VARBIT: [payload B x P bytes][FP16 scale B*H*d][u8 width B*H*d]         */
 /*           [u32 row offset B*(H*d+1)], each section starting on a 256-byte */
 /*           boundary; P = (d/8) * avg_bits * H * d; row i of sequence b     */
@@ -480,27 +481,27 @@ static int rotated(const orc_layout* L) {
   return L->domain == ORC_DOMAIN_ROTATED && L->storage == ORC_STORE_DAMP && L->hadamard;
 }
 
-/* Dequantize one DAMP head into S (d x d, stored row order).  In the
- * canonical domain INT8 rows are returned to the value basis with the
- * Hadamard (its own inverse); in the rotated domain the FP16 rows are taken
- * to the Hadamard basis instead. */
+/* Dequantize one DAMP head into S (d x d, stored row order: the d - k_hi
+ * INT8 rows first, then the k_hi protected FP16 rows).  In the canonical
+ * domain INT8 rows are returned to the value basis with the Hadamard (its
+ * own inverse); in the rotated domain the FP16 rows are taken to the
+ * Hadamard basis instead. */
 static void damp_load(const orc_layout* L, const uint8_t* head, float* S) {
-  int d = L->d, kh = L->k_hi, nb = d / L->block;
-  const uint16_t* f16rows = (const uint16_t*)head;
-  const uint8_t* codes = head + (size_t)kh * d * 2;
-  const uint16_t* sz = (const uint16_t*)(codes + (size_t)(d - kh) * d);
+  int d = L->d, nlo = d - L->k_hi, nb = d / L->block;
+  const uint8_t* codes = head;
+  const uint16_t* f16rows = (const uint16_t*)(head + (size_t)nlo * d);
+  const uint16_t* sz = (const uint16_t*)(head + (size_t)nlo * d + (size_t)L->k_hi * d * 2);
   for (int i = 0; i < d; ++i) {
     float* row = S + (size_t)i * d;
-    if (i < kh) {
-      for (int j = 0; j < d; ++j) row[j] = orc_f32_from_f16(f16rows[(size_t)i * d + j]);
+    if (i >= nlo) {
+      for (int j = 0; j < d; ++j) row[j] = orc_f32_from_f16(f16rows[(size_t)(i - nlo) * d + j]);
       if (rotated(L)) orc_fwht(row, d);
     } else {
-      int r = i - kh;
       for (int j = 0; j < d; ++j) {
         int bl = j / L->block;
-        float s = orc_f32_from_f16(sz[((size_t)r * nb + bl) * 2 + 0]);
-        float z = orc_f32_from_f16(sz[((size_t)r * nb + bl) * 2 + 1]);
-        row[j] = fmaf((float)codes[(size_t)r * d + j], s, z);
+        float s = orc_f32_from_f16(sz[((size_t)i * nb + bl) * 2 + 0]);
+        float z = orc_f32_from_f16(sz[((size_t)i * nb + bl) * 2 + 1]);
+        row[j] = fmaf((float)codes[(size_t)i * d + j], s, z);
       }
       if (L->hadamard && !rotated(L)) orc_fwht(row, d);
     }
@@ -509,31 +510,30 @@ static void damp_load(const orc_layout* L, const uint8_t* head, float* S) {
 
 static int damp_store(const orc_layout* L, const orc_writeback* wb, int64_t step, int b, int h,
                       const float* S, uint8_t* head, uint16_t* aux_head, float* t_head) {
-  int d = L->d, kh = L->k_hi, nb = d / L->block, flags = 0;
-  uint16_t* f16rows = (uint16_t*)head;
-  uint8_t* codes = head + (size_t)kh * d * 2;
-  uint16_t* sz = (uint16_t*)(codes + (size_t)(d - kh) * d);
+  int d = L->d, nlo = d - L->k_hi, nb = d / L->block, flags = 0;
+  uint8_t* codes = head;
+  uint16_t* f16rows = (uint16_t*)(head + (size_t)nlo * d);
+  uint16_t* sz = (uint16_t*)(head + (size_t)nlo * d + (size_t)L->k_hi * d * 2);
   float* tmp = (float*)malloc(sizeof(float) * (size_t)d);
   for (int i = 0; i < d; ++i) {
     memcpy(tmp, S + (size_t)i * d, sizeof(float) * (size_t)d);
-    if (i < kh) {
+    if (i >= nlo) {
       if (rotated(L)) orc_fwht(tmp, d);
       for (int j = 0; j < d; ++j) {
         if (!isfinite(tmp[j])) flags |= ORC_ENONFINITE;
         uint16_t hv = orc_f16_from_f32(tmp[j]);
         if (f16_is_inf_or_nan(hv) && isfinite(tmp[j])) flags |= ORC_EOVERFLOW;
-        f16rows[(size_t)i * d + j] = hv;
+        f16rows[(size_t)(i - nlo) * d + j] = hv;
         if (t_head) t_head[(size_t)i * d + j] = 0.0f;
       }
     } else {
-      int r = i - kh;
       if (L->hadamard && !rotated(L)) orc_fwht(tmp, d);
       for (int bl = 0; bl < nb; ++bl) {
         int j0 = bl * L->block;
-        uint16_t* e = aux_head ? aux_head + (size_t)r * d + j0 : NULL;
+        uint16_t* e = aux_head ? aux_head + (size_t)i * d + j0 : NULL;
         flags |= orc_int8_block(tmp + j0, L->block, wb->mode, wb->seed, step, h, b, i * d + j0, e,
-                                codes + (size_t)r * d + j0, &sz[((size_t)r * nb + bl) * 2 + 0],
-                                &sz[((size_t)r * nb + bl) * 2 + 1],
+                                codes + (size_t)i * d + j0, &sz[((size_t)i * nb + bl) * 2 + 0],
+                                &sz[((size_t)i * nb + bl) * 2 + 1],
                                 t_head ? t_head + (size_t)i * d + j0 : NULL);
       }
     }
@@ -924,7 +924,9 @@ int orc_state_unpack(const orc_layout* L, const void* packed, const int16_t* per
 /*          quantize -> dequantize, over the sampled calibration states;     */
 /*   a_eff,u = exp(mean log a_u);  P_u = 1 / max(1 - a_eff,u^2, tau);        */
 /*   C_u = E_u P_u; the top k_hi rows of each head are protected (ties to    */
-/*   the lower index) and placed first, both groups in ascending order.      */
+/*   the lower index).  The permutation lists the unprotected rows, then the */
+/*   protected ones, each group in ascending order: the protected rows sit   */
+/*   contiguously at the end of the stored order.                            */
 /* ------------------------------------------------------------------------ */
 int orc_calibrate(const orc_layout* L, int Bc, int T, int every, double tau,
                   const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* beta,
@@ -995,9 +997,9 @@ int orc_calibrate(const orc_layout* L, int Bc, int T, int every, double tau,
     }
     int n = 0;
     for (int i = 0; i < d; ++i)
-      if (prot[i]) idx[n++] = i;
-    for (int i = 0; i < d; ++i)
       if (!prot[i]) idx[n++] = i;
+    for (int i = 0; i < d; ++i)
+      if (prot[i]) idx[n++] = i;
     for (int i = 0; i < d; ++i) perm_out[(size_t)h * d + i] = (int16_t)idx[i];
   }
   free(idx);

@@ -40,23 +40,28 @@ def hadamard_n(n):
 
 
 def damp_head_sections(packed_head, d, k_hi, block):
+    """Stored head -> (FP16 rows [k_hi][d], codes [d-k_hi][d], (scale, zero)
+    [d-k_hi][d/block][2]); INT8 rows come first in stored order."""
     nb = d // block
-    f16rows = np.frombuffer(packed_head[: k_hi * d * 2].tobytes(), np.uint16).reshape(k_hi, d)
-    codes = packed_head[k_hi * d * 2: k_hi * d * 2 + (d - k_hi) * d].reshape(d - k_hi, d)
-    sz = np.frombuffer(packed_head[k_hi * d * 2 + (d - k_hi) * d:].tobytes(), np.uint16)
-    sz = sz.reshape(d - k_hi, nb, 2)
+    nlo = d - k_hi
+    codes = packed_head[: nlo * d].reshape(nlo, d)
+    f16rows = np.frombuffer(packed_head[nlo * d: nlo * d + k_hi * d * 2].tobytes(),
+                            np.uint16).reshape(k_hi, d)
+    sz = np.frombuffer(packed_head[nlo * d + k_hi * d * 2:].tobytes(), np.uint16)
+    sz = sz.reshape(nlo, nb, 2)
     return f16rows, codes, sz
 
 
 def damp_dequant64(packed_head, d, k_hi, block, had):
     """Stored head -> FP64 canonical state (stored row order)."""
     f16rows, codes, sz = damp_head_sections(packed_head, d, k_hi, block)
+    nlo = d - k_hi
     S = np.zeros((d, d))
-    S[:k_hi] = f16_bits_to_f64(f16rows)
+    S[nlo:] = f16_bits_to_f64(f16rows)
     s = np.repeat(f16_bits_to_f64(sz[:, :, 0]), block, axis=1)
     z = np.repeat(f16_bits_to_f64(sz[:, :, 1]), block, axis=1)
     r = codes.astype(np.float64) * s + z
-    S[k_hi:] = r @ hadamard_n(d) if had else r
+    S[:nlo] = r @ hadamard_n(d) if had else r
     return S
 
 

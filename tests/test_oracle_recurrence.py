@@ -126,8 +126,16 @@ def test_damp_step_matches_fp64_brute_force(orc):
                 S, oo = dense_step(S, k, q, v, a, beta)
                 assert np.max(np.abs(o[0, b, h] - oo)) <= 1e-5 * (np.max(np.abs(oo)) + 1e-30)
                 f16rows, codes, sz = damp_head_sections(packed[u * hb:(u + 1) * hb], d, k_hi, block)
-                np.testing.assert_array_equal(f16rows, S[:k_hi].astype(np.float16).view(np.uint16))
-                R = S[k_hi:] @ Hn
+                ref16 = S[d - k_hi:].astype(np.float16).view(np.uint16)
+                bad = f16rows != ref16
+                if bad.any():
+                    # only values within FP32 reach of an FP16 rounding midpoint
+                    x = np.abs(S[d - k_hi:][bad])
+                    ulp = np.spacing(x.astype(np.float16)).astype(np.float64)
+                    frac = np.abs((x / ulp) % 1 - 0.5)
+                    assert np.all(frac < 1e-3) and np.all(np.abs(f16rows[bad].astype(int) - ref16[bad]) == 1)
+                    mism += int(bad.sum())
+                R = S[:d - k_hi] @ Hn
                 for r in range(d - k_hi):
                     c64, s64, z64, t64 = int8_nearest64(R[r])
                     s_o = f16_bits_to_f64(sz[r, 0, 0])
@@ -172,7 +180,7 @@ def test_rotated_domain_matches_canonical(orc):
             # FP16 rows: a value next to an FP16 rounding midpoint may land one unit apart
             assert np.all(np.abs(fc.astype(int) - fr.astype(int)) <= 1)
             ndiff += int(np.sum(fc != fr))
-            tt = tc.reshape(w.B * w.H, w.d, w.d)[u, w.k_hi:]
+            tt = tc.reshape(w.B * w.H, w.d, w.d)[u, :w.d - w.k_hi]
             same_grid = np.all(szc == szr, axis=(1, 2))
             diff = (cc_codes != cr_codes) & same_grid[:, None]
             ncodes += cc_codes[same_grid].size
@@ -287,7 +295,7 @@ def test_pack_unpack_roundtrip(orc):
     p, _ = orc.state_pack(cfg, S, perm)
     S2, _ = orc.state_unpack(cfg, p, perm)
     for h in range(H):
-        prot = perm[h, :4]
+        prot = perm[h, d - 4:]
         np.testing.assert_array_equal(S2[:, h, prot], S[:, h, prot].astype(np.float16).astype(np.float32))
     err = np.abs(S2 - S).max()
     assert err <= (S.max() - S.min()) / 255 * 2     # half a step per coordinate, spread by H
