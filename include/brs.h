@@ -1,0 +1,196 @@
+/*
+ * brs.h -- C ABI of the B200 (sm_100a) library for the fused recurrent-state
+ * update with quantized write-back of gated delta-rule linear-attention
+ * layers (KDA: decay per key channel; GDN: decay per head).
+ *
+ * Sources, cited by page title and section:
+ *   [WB]   "When Quantization Breaks Memory: Recurrent-State Write-Back in
+ *          Low-Precision Temporal Inference" (English and Chinese summaries)
+ *   [LB]   "Low-Bit Recurrent States in Hybrid Language Models"
+ *   [LBX]  "Allocate low-bit recurrent state precision by channel decay"
+ *   [DAMP] summary of "DAMP: Decay-Aware Mixed-Precision recurrent-state
+ *          quantization" (arXiv 2608.27513)
+ *
+ * Conventions shared by every entry point
+ *   - Plain C types only.  Device pointers are CUDA global-memory addresses
+ *     on the current device; `stream` is a cudaStream_t (NULL = legacy
+ *     default stream).  bfloat16 inputs are passed as their uint16_t bit
+ *     patterns, FP16 fields are uint16_t bit patterns.
+ *   - Ownership: the caller allocates and owns every buffer (state, residual,
+ *     statistics, workspace, inputs, outputs) and the stream.  The library
+ *     allocates no device memory and keeps no state between calls except the
+ *     thread-local error string.
+ *   - Execution: every call that launches work is asynchronous on `stream`.
+ *     Argument errors are detected on the host and returned at once (no work
+ *     is launched).  Errors detected by the kernels (non-finite values, FP16
+ *     overflow) are OR-ed into a flag word at the start of `workspace` and
+ *     reported by brs_fetch_errors(), which synchronises the stream.
+ *   - Alignment: every device pointer must be 16-byte aligned (BRS_EALIGN).
+ *   - Dimensions: d_k = d_v = d with d in {32, 64, 128}.
+ *   - Inputs of one token (decode): q, k [B][H_k][d] bf16; v [B][H][d] bf16;
+ *     beta [B][H] f32; decay [B][H][d] f32 (KDA) or [B][H] f32 (GDN), holding
+ *     a = exp(-s) (not s); output o [B][H][d] f32.  q and k are expected
+ *     L2-normalised.  Value head h reads key head h * H_k / H (grouped value
+ *     heads).
+ *
+ * Stored state formats (byte layouts; all multi-byte fields little-endian)
+ *   BRS_STORE_FP32   float [B][H][d][d], rows in stored order.
+ *   BRS_STORE_DAMP   [DAMP] Key Points > Main operating point and
+ *                    Implementation; Quantization & calibration details.
+ *                    Per head (b, h), contiguous, head stride
+ *                      (d-k_hi)*d + k_hi*d*2 + (d-k_hi)*(d/block)*4 bytes:
+ *                      u8  codes[d-k_hi][d]      stored rows 0..d-k_hi-1,
+ *                                                asymmetric INT8 of the row
+ *                                                after the d-point Hadamard
+ *                                                (when `hadamard` is set);
+ *                      f16 rows [k_hi][d]        protected rows
+ *                                                d-k_hi..d-1, in the value
+ *                                                basis;
+ *                      f16 sz[d-k_hi][d/block][2] (scale, zero) per block;
+ *                                                value = fmaf(code, scale,
+ *                                                zero).
+ *                    Stored row i holds key channel perm[h][i] (the
+ *                    protected channels are the last k_hi entries).
+ *                    Error-feedback residuals: f16 [B][H][d-k_hi][d].
+ *   BRS_STORE_VARBIT [LB] State bit allocation, Allocation units, Levels and
+ *                    storage.  Sections, each starting on a 256-byte
+ *                    boundary: payload [B][P] bytes with
+ *                    P = (d/8) * avg_bits * H * d; f16 step [B][H*d];
+ *                    u8 width [B][H*d] (2..8); u32 row offset [B][H*d+1].
+ *                    Row r of sequence b holds d codes u = q + n,
+ *                    n = 2^(w-1) - 1, w bits each, little-endian bit order,
+ *                    starting at byte offset[r] = (d/8) * (sum of the
+ *                    widths of rows < r); value = (u - n) * step.
+ *                    Residuals f16 [B][H][d][d]; statistics f64
+ *                    [B][H][d][2] = (EMA of a^2, EMA of beta (2-beta) k^2).
+ *
+ * Arithmetic (identical on every path that produces stored codes)
+ *   The update runs in FP32 ([DAMP] Implementation): per token and head,
+ *   S <- Diag(a) S; u = S^T k; w = beta (v - u); S <- S + k w^T; o = S^T q,
+ *   each sum over key rows an fmaf chain over stored rows 0..d-1 from +0.
+ *   The Hadamard is the unnormalised Sylvester butterfly (stages 1, 2, 4, ...)
+ *   followed by one multiplication by the float nearest 1/sqrt(d).  With
+ *   `hadamard` set the DAMP update is computed in the Hadamard basis: the
+ *   FP16 rows and v are rotated in, o is rotated out, the INT8 rows are
+ *   used as stored.
+ *   INT8 block: scale = fp16((max - min) / 255), zero = fp16(min),
+ *   code = clamp(round((y - zero) * (1/scale)), 0, 255).  Rounding
+ *   ([WB] Quantized GRU formulation; Chinese summary, error feedback and
+ *   stochastic rounding): nearest = ties to the even code; stochastic =
+ *   floor(t) + [r24 < frac(t) * 2^24] with r24 the top 24 bits of word
+ *   (e % 4) of Philox4x32-10(counter (e/4, step, h, b), key (seed_lo,
+ *   seed_hi)), e = row * d + column; error feedback = y = x + e_prev,
+ *   e_new = fp16(clamp(y - value, -scale, +scale)).
+ */
+#ifndef BRS_H
+#define BRS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BRS_OK = 0,
+  BRS_EINVAL = 1,        /* bad argument (shape, null pointer, infeasible budget) */
+  BRS_EUNSUPPORTED = 2,  /* valid but not implemented combination              */
+  BRS_EALIGN = 3,        /* a device pointer is not 16-byte aligned             */
+  BRS_ECUDA = 4,         /* a CUDA runtime call failed                          */
+  BRS_ENONFINITE = 5,    /* a kernel met a non-finite state value               */
+  BRS_EOVERFLOW = 6,     /* an FP16 row, scale or zero overflowed               */
+  BRS_ETIMEOUT = 7       /* a bounded device-side wait gave up                  */
+} brs_status;
+
+typedef enum { BRS_STORE_FP32 = 0, BRS_STORE_DAMP = 1, BRS_STORE_VARBIT = 2 } brs_storage;
+
+typedef enum {
+  BRS_ROUND_NEAREST = 0,
+  BRS_ROUND_STOCHASTIC = 1,
+  BRS_ROUND_ERRFEEDBACK = 2
+} brs_round;
+
+/* Device flag bits OR-ed into the first 32-bit word of `workspace`. */
+#define BRS_FLAG_NONFINITE 0x1u
+#define BRS_FLAG_OVERFLOW 0x2u
+#define BRS_FLAG_TIMEOUT 0x4u
+
+typedef struct {
+  int32_t B;             /* sequences                                          */
+  int32_t H;             /* value heads                                        */
+  int32_t H_k;           /* key heads (H % H_k == 0)                           */
+  int32_t d;             /* d_k = d_v, in {32, 64, 128}                        */
+  int32_t storage;       /* brs_storage                                        */
+  int32_t k_hi;          /* DAMP: protected FP16 rows per head (multiple of 4) */
+  int32_t block;         /* DAMP: INT8 block length along the value axis      */
+  int32_t hadamard;      /* DAMP: 1 = INT8 rows stored after the Hadamard     */
+  int32_t decay_per_key; /* 1 = KDA (decay [B][H][d]), 0 = GDN ([B][H])        */
+  double avg_bits;       /* VARBIT: mean width; avg_bits*H*d integral          */
+  int32_t b_min, b_max;  /* VARBIT: width limits, 2 <= b_min <= b_max <= 8     */
+  int32_t budget_scope;  /* VARBIT: 1 = layer (all H*d rows of a sequence),
+                            0 = head                                           */
+} brs_layout;
+
+typedef struct {
+  int32_t mode;          /* brs_round                                          */
+  uint64_t seed;         /* Philox key of stochastic rounding                  */
+  int32_t C;             /* write-back interval in tokens ([LB] Accumulated
+                            readout error: once per chunk, per token, or every
+                            C tokens)                                          */
+} brs_writeback;
+
+/* Bytes of the stored state for layout L; optionally the bytes of the
+ * error-feedback residual buffer, of the allocator statistics and of the
+ * workspace a call needs.  Returns 0 for an invalid layout (see
+ * brs_last_error). */
+size_t brs_state_bytes(const brs_layout* L, size_t* aux_bytes, size_t* stats_bytes,
+                       size_t* workspace_bytes);
+
+/* FP32 state S [B][H][d][d] (rows in key-channel order) -> stored format,
+ * deterministic rounding.  perm [H][d] int16 (stored row i of head h holds
+ * channel perm[h][i]); NULL = identity.  widths (VARBIT only) u8 [B][H*d]
+ * device array of row widths, NULL = avg_bits for every row (which must
+ * then be an integer).  All pointers device, `packed` sized by
+ * brs_state_bytes.  [DAMP] Implementation (static permuted layout). */
+brs_status brs_state_pack(const brs_layout* L, const float* S, const int16_t* perm,
+                          const uint8_t* widths, void* packed, void* workspace, void* stream);
+
+/* Stored format -> FP32 state S [B][H][d][d] in key-channel order. */
+brs_status brs_state_unpack(const brs_layout* L, const void* packed, const int16_t* perm,
+                            float* S, void* workspace, void* stream);
+
+/* One decode token for every head: dequantize the stored state, apply the
+ * decay and the delta-rule write in FP32, read o from the updated FP32
+ * state, then (when (step + 1) % C == 0) requantize and write back
+ * ([DAMP] Implementation; [LB] Accumulated readout error: outputs precede
+ * quantization; [LB] Protocol: each write-back is quantized and dequantized
+ * before reuse).  Decode supports C == 1.
+ *   packed_in / packed_out: stored state before / after; they may alias
+ *     for FP32 and DAMP storage, must not alias for VARBIT.
+ *   aux: residuals (ERRFEEDBACK only, else may be NULL), updated in place.
+ *   stats: VARBIT statistics, updated in place (else may be NULL).
+ *   workspace: brs_state_bytes(...workspace) bytes; its first word
+ *     collects device flags and must be zeroed once before first use
+ *     (brs_fetch_errors clears it).
+ *   perm: [H][d] int16 device, NULL = identity.
+ * Inputs and o: see the conventions above. */
+brs_status brs_decode_step(const brs_layout* L, const brs_writeback* wb, int64_t step,
+                           const void* packed_in, void* packed_out, void* aux, void* stats,
+                           void* workspace, const int16_t* perm, const uint16_t* q,
+                           const uint16_t* k, const uint16_t* v, const float* beta,
+                           const float* decay, float* o, void* stream);
+
+/* Reads and clears the device flag word of `workspace` (synchronises
+ * `stream`).  Returns BRS_OK, or BRS_ENONFINITE / BRS_EOVERFLOW /
+ * BRS_ETIMEOUT for the first flag set; *flags_out (optional) receives the
+ * raw bits. */
+brs_status brs_fetch_errors(void* workspace, uint32_t* flags_out, void* stream);
+
+/* Message of the last error returned on this host thread ("" if none). */
+const char* brs_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BRS_H */

@@ -187,10 +187,11 @@ int orc_int8_block(const float* y, int n, int mode, uint64_t seed, int64_t step,
     if (mode == ORC_ROUND_ERRFEEDBACK) tgt[j] = y[j] + orc_f32_from_f16(e_inout[j]);
     if (!isfinite(tgt[j])) flags |= ORC_ENONFINITE;
   }
+  /* block minimum and maximum, -0 ordered below +0 */
   float mn = tgt[0], mx = tgt[0];
   for (int j = 1; j < n; ++j) {
-    if (tgt[j] < mn) mn = tgt[j];
-    if (tgt[j] > mx) mx = tgt[j];
+    if (tgt[j] < mn || (tgt[j] == mn && signbit(tgt[j]))) mn = tgt[j];
+    if (tgt[j] > mx || (tgt[j] == mx && !signbit(tgt[j]))) mx = tgt[j];
   }
   uint16_t sh = orc_f16_from_f32((mx - mn) / 255.0f);
   uint16_t zh = orc_f16_from_f32(mn);
