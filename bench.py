@@ -1,0 +1,371 @@
+"""Benchmark of the decode step (state-update tokens*heads/s and state HBM
+GB/s against the measured B200 copy bandwidth).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload kda_decode|gdn_decode|kda_tiny]
+
+A step is one decode token for every (sequence, head) of the workload: one
+launch of the fused decode kernel (dequantize, decay, delta-rule write, read
+o, requantize, write back).  Consecutive steps rotate over 8 independent
+layer states (each with its own seeded inputs), so a step never finds its
+state in L2 (8 x 38.7 MB > 126 MB).  With N GPUs (torchrun) every rank runs
+its own batch of the same size (weak scaling, no collective on the data
+path); the time is the maximum over ranks.
+
+`--impl reference` times the plain CPU oracle on this host's cores on the
+same workload and metric (bounded samples), which is the only other place
+the oracle runs besides the cpu_baseline leg.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "state-update tokens·heads/s and state HBM GB/s (% of B200 peak), decode"
+UNIT = "tokens·heads/s"
+FALLBACK_HBM_GBS = 6650.0
+NLAYERS = 8
+KERNEL_SOURCES = ["bit_recurrent_state_b200/csrc/decode.cu", "bit_recurrent_state_b200/csrc/brs_device.cuh"]
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def algorithmic_bytes(w) -> dict:
+    """Bytes one decode launch must move: the stored state read and written
+    once, the token's inputs read, o written."""
+    from bit_recurrent_state_b200 import brs
+    n, aux, _, _ = brs.state_bytes(brs.layout_of(w))
+    heads = w.B * w.H
+    inputs = (2 * w.B * w.hk * w.d * 2 + heads * w.d * 2 + heads * 4 +
+              (heads * w.d * 4 if w.decay_per_key else heads * 4) + w.H * w.d * 2)
+    out = heads * w.d * 4
+    ef = 2 * aux if w.mode == "errfeedback" else 0
+    return dict(state=2 * n, inputs=inputs, output=out, aux=ef, total=2 * n + inputs + out + ef)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def traffic_record(workload: str):
+    """DRAM bytes per launch from a committed ncu summary, only while the
+    kernel sources still hash to the profiled version."""
+    p = os.path.join(ROOT, "profiles", f"decode_{workload}_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    if rec.get("kernel_hash") != kernel_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index),
+                 "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            self.proc.wait()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _oracle_cfg(w):
+    from oracle import oracle as O
+    rot = w.storage == "damp" and w.hadamard
+    st = {"fp32": O.STORE_FP32, "damp": O.STORE_DAMP, "varbit": O.STORE_VARBIT}[w.storage]
+    return O.Config(B=w.B, H=w.H, Hk=w.hk, d=w.d, storage=st, k_hi=w.k_hi, block=w.block,
+                    hadamard=w.hadamard, decay_per_key=w.decay_per_key,
+                    domain=O.DOMAIN_ROTATED if rot else O.DOMAIN_CANONICAL)
+
+
+class OracleRunner:
+    """The oracle, as it stands, over a bounded sample of the workload: the
+    first `units` heads for `ntok` consecutive tokens per call, split over
+    the host's cores (heads are independent)."""
+
+    def __init__(self, w):
+        from bit_recurrent_state_b200 import synth
+        from oracle import oracle as O
+        self.O, self.synth, self.w = O, synth, w
+        self.cfg = _oracle_cfg(w)
+        self.packed, self.aux, self.stats = O.new_state(self.cfg)
+        self.cores = os.cpu_count() or 1
+        self.t = 0
+        self.cache = {}
+
+    def inputs(self, ntok):
+        key = (self.t, ntok)
+        if key not in self.cache:
+            self.cache = {key: self.synth.run_inputs(self.w, self.t, ntok)}
+        return self.cache[key]
+
+    def run(self, units, ntok):
+        inp = self.inputs(ntok)
+        t0 = time.perf_counter()
+        _, fl, used = self.O.run_parallel(self.cfg, 0, self.w.seed, 1, self.t, inp, self.packed,
+                                          aux=self.aux, stats=self.stats, units=(0, units),
+                                          threads=self.cores)
+        dt = time.perf_counter() - t0
+        self.t += ntok
+        return dt, used
+
+    def rate(self):
+        """unit-tokens per second, from a short calibration run."""
+        units = min(self.w.B * self.w.H, 4 * self.cores)
+        dt, _ = self.run(units, 2)
+        return units * 2 / max(dt, 1e-6)
+
+
+def cpu_oracle_sample(w, target_s: float = 12.0):
+    """cpu_baseline: the oracle on host cores, about target_s seconds of work
+    on the workload's heads (all of them when that fits, else a prefix)."""
+    R = OracleRunner(w)
+    r = R.rate()
+    total = w.B * w.H
+    want = r * target_s
+    ntok = int(max(1, min(64, want // total)))
+    units = int(max(1, min(total, want // ntok)))
+    dt, used = R.run(units, ntok)
+    return {"value": units * ntok / dt, "unit": UNIT, "cores": used, "kind": "oracle",
+            "sample": f"{units} of {total} heads x {ntok} tokens of {w.name} "
+                      f"({dt:.1f} s wall on {used} threads)"}
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    R = OracleRunner(w)
+    total = w.B * w.H
+    per_step_s = max(0.2, min(4.0, args.ref_budget / (args.warmup + args.steps)))
+    units = int(max(1, min(total, R.rate() * per_step_s)))
+    vals, used = [], 1
+    for i in range(args.warmup + args.steps):
+        dt, used = R.run(units, 1)
+        if i >= args.warmup:
+            vals.append(units / dt)
+    value = statistics.median(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total / value, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "d": w.d},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
+                             "sample": f"each step: {units} of {total} heads x 1 token of "
+                                       f"{w.name} on {used} threads"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+
+    from bit_recurrent_state_b200 import brs, synth
+    from bit_recurrent_state_b200.state import LayerState
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    # per-rank workload: same shape, own sequences (seed offset by rank)
+    wr = w.with_(seed=w.seed + 1000 * rank)
+    L = brs.layout_of(wr)
+    wb = brs.writeback_of(wr)
+    rng = np.random.default_rng(wr.seed)
+    perm = np.stack([rng.permutation(w.d) for _ in range(w.H)]).astype(np.int16)
+    layers, inputs, host_inputs = [], [], []
+    for l in range(NLAYERS):
+        st = LayerState(L, device=dev, perm=perm)
+        st.zero()
+        layers.append(st)
+        inp = synth.token_inputs(wr.with_(seed=wr.seed + 17 * l), 0)
+        host = {k: torch.from_numpy(v.view(np.int16) if v.dtype == np.uint16 else v).pin_memory()
+                for k, v in inp.items()}
+        host_inputs.append(host)
+        inputs.append({k: v.to(dev) for k, v in host.items()})
+    o = torch.zeros((w.B, w.H, w.d), dtype=torch.float32, device=dev)
+    o_host = torch.zeros_like(o, device="cpu").pin_memory()
+
+    def step(i):
+        st = layers[i % NLAYERS]
+        x = inputs[i % NLAYERS]
+        st.step(wb, i, x["q"], x["k"], x["v"], x["beta"], x["decay"], o)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    flags = layers[0].errors()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    # ---- device-resident throughput (kernel per step)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier()
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(args.warmup + i)
+        ev1.record(stream)
+        barrier()
+    ms = ev0.elapsed_time(ev1)
+    t = torch.tensor([ms], device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    ms_step = ms_max / args.steps
+
+    # ---- end to end through the public API with host buffers
+    h2d = sum(v.numel() * v.element_size() for v in host_inputs[0].values())
+    d2h = o.numel() * o.element_size()
+    barrier()
+    ev0.record(stream)
+    for i in range(args.steps):
+        l = i % NLAYERS
+        for k, v in host_inputs[l].items():
+            inputs[l][k].copy_(v, non_blocking=True)
+        step(args.warmup + args.steps + i)
+        o_host.copy_(o, non_blocking=True)
+    ev1.record(stream)
+    barrier()
+    ms_e2e = ev0.elapsed_time(ev1)
+    t = torch.tensor([ms_e2e], device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_e2e = float(t.item())
+    flags |= layers[0].errors()
+
+    units = w.B * w.H * world
+    value = units * args.steps / (ms_max * 1e-3)
+    e2e_value = units * args.steps / (ms_e2e * 1e-3)
+    ab = algorithmic_bytes(w)
+    peak, src = peaks()
+    achieved = ab["total"] / (ms_step * 1e-3) / 1e9
+    traffic = traffic_record(w.name)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "H_k": w.hk, "d": w.d,
+                   "storage": w.storage, "k_hi": w.k_hi, "block": w.block, "mode": w.mode,
+                   "per_rank_batch": w.B, "parallelism": f"dp{world}",
+                   "l2": f"{NLAYERS} rotating layer states of {ab['state'] // 2 / 1e6:.1f} MB "
+                         f"(> 126 MB L2)"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": src + " (MEASURED_PEAKS.json hbm_gbs)"
+                     if src == "measured" else "fallback 6.65 TB/s",
+                     "algorithmic_bytes_per_launch": ab["total"],
+                     "traffic": traffic,
+                     "kernel": "brs::decode_kernel", "state_gbs": ab["state"] / (ms_step * 1e-3) / 1e9},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps,
+        "device_flags": flags,
+    }
+    if rank == 0:
+        line["clocks"] = clk.summary()
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_oracle_sample(w)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="kda_decode")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-budget", type=float, default=120.0,
+                    help="seconds of oracle work for the whole --impl reference run")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    from bit_recurrent_state_b200 import synth
+    w = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        from bit_recurrent_state_b200 import brs
+        brs.lib()          # the in-tree CUDA library; fails loudly when it is missing
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,148 @@
+"""Thin Python binding of the C ABI in include/brs.h (argument marshalling
+only; every step of the update runs in the CUDA library libbrs.so).
+
+Functions keep the C names without the ``brs_`` prefix and take torch CUDA
+tensors (or raw integer device addresses) for the device pointers; the
+stream defaults to torch's current stream.  There is no CPU fallback:
+loading fails loudly when libbrs.so is missing.
+"""
+from __future__ import annotations
+
+import ctypes as ct
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libbrs.so")
+
+STORE_FP32, STORE_DAMP, STORE_VARBIT = 0, 1, 2
+ROUND_NEAREST, ROUND_STOCHASTIC, ROUND_ERRFEEDBACK = 0, 1, 2
+OK, EINVAL, EUNSUPPORTED, EALIGN, ECUDA, ENONFINITE, EOVERFLOW, ETIMEOUT = range(8)
+FLAG_NONFINITE, FLAG_OVERFLOW, FLAG_TIMEOUT = 1, 2, 4
+MODES = {"nearest": ROUND_NEAREST, "stochastic": ROUND_STOCHASTIC,
+         "errfeedback": ROUND_ERRFEEDBACK}
+STORES = {"fp32": STORE_FP32, "damp": STORE_DAMP, "varbit": STORE_VARBIT}
+
+# exported symbols declared in include/brs.h
+SYMBOLS = ["brs_state_bytes", "brs_state_pack", "brs_state_unpack", "brs_decode_step",
+           "brs_fetch_errors", "brs_last_error"]
+
+
+class BrsError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"brs status {status}: {msg}")
+        self.status = status
+
+
+class Layout(ct.Structure):
+    _fields_ = [("B", ct.c_int32), ("H", ct.c_int32), ("H_k", ct.c_int32), ("d", ct.c_int32),
+                ("storage", ct.c_int32), ("k_hi", ct.c_int32), ("block", ct.c_int32),
+                ("hadamard", ct.c_int32), ("decay_per_key", ct.c_int32),
+                ("avg_bits", ct.c_double), ("b_min", ct.c_int32), ("b_max", ct.c_int32),
+                ("budget_scope", ct.c_int32)]
+
+
+class WriteBack(ct.Structure):
+    _fields_ = [("mode", ct.c_int32), ("seed", ct.c_uint64), ("C", ct.c_int32)]
+
+
+def layout_of(w, **override) -> Layout:
+    """brs_layout of a synth.Workload (fields may be overridden)."""
+    f = dict(B=w.B, H=w.H, H_k=w.hk, d=w.d, storage=STORES[w.storage], k_hi=w.k_hi,
+             block=w.block, hadamard=w.hadamard, decay_per_key=w.decay_per_key,
+             avg_bits=w.avg_bits, b_min=w.b_min, b_max=w.b_max, budget_scope=1)
+    f.update(override)
+    return Layout(**f)
+
+
+def writeback_of(w, **override) -> WriteBack:
+    f = dict(mode=MODES[w.mode], seed=w.seed, C=w.C)
+    f.update(override)
+    return WriteBack(**f)
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"CUDA library not built: {LIB_PATH} (run __graft_entry__.build())")
+        L = ct.CDLL(LIB_PATH)
+        P, S = ct.c_void_p, ct.c_int
+        L.brs_state_bytes.restype = ct.c_size_t
+        L.brs_state_bytes.argtypes = [P, P, P, P]
+        L.brs_state_pack.restype = S
+        L.brs_state_pack.argtypes = [P, P, P, P, P, P, P]
+        L.brs_state_unpack.restype = S
+        L.brs_state_unpack.argtypes = [P, P, P, P, P, P]
+        L.brs_decode_step.restype = S
+        L.brs_decode_step.argtypes = [P, P, ct.c_int64] + [P] * 14
+        L.brs_fetch_errors.restype = S
+        L.brs_fetch_errors.argtypes = [P, P, P]
+        L.brs_last_error.restype = ct.c_char_p
+        L.brs_last_error.argtypes = []
+        _lib = L
+    return _lib
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def last_error() -> str:
+    return lib().brs_last_error().decode()
+
+
+def _check(status: int):
+    if status != OK:
+        raise BrsError(status, last_error())
+
+
+def state_bytes(layout: Layout):
+    """(state, aux, stats, workspace) byte counts."""
+    aux, st, ws = ct.c_size_t(0), ct.c_size_t(0), ct.c_size_t(0)
+    n = lib().brs_state_bytes(ct.byref(layout), ct.byref(aux), ct.byref(st), ct.byref(ws))
+    if n == 0:
+        raise BrsError(EINVAL, last_error())
+    return int(n), int(aux.value), int(st.value), int(ws.value)
+
+
+def state_pack(layout, S, perm, packed, workspace, widths=None, stream=None):
+    _check(lib().brs_state_pack(ct.byref(layout), _ptr(S), _ptr(perm), _ptr(widths),
+                                _ptr(packed), _ptr(workspace), _stream(stream)))
+
+
+def state_unpack(layout, packed, perm, S, workspace=None, stream=None):
+    _check(lib().brs_state_unpack(ct.byref(layout), _ptr(packed), _ptr(perm), _ptr(S),
+                                  _ptr(workspace), _stream(stream)))
+
+
+def decode_step(layout, wb, step, packed_in, packed_out, aux, stats, workspace, perm, q, k, v,
+                beta, decay, o, stream=None):
+    _check(lib().brs_decode_step(ct.byref(layout), ct.byref(wb), int(step), _ptr(packed_in),
+                                 _ptr(packed_out), _ptr(aux), _ptr(stats), _ptr(workspace),
+                                 _ptr(perm), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(decay),
+                                 _ptr(o), _stream(stream)))
+
+
+def fetch_errors(workspace, stream=None) -> int:
+    """Raw device flag bits (also raises BrsError if any is set)."""
+    fl = ct.c_uint32(0)
+    st = lib().brs_fetch_errors(_ptr(workspace), ct.byref(fl), _stream(stream))
+    if st != OK and st not in (ENONFINITE, EOVERFLOW, ETIMEOUT):
+        _check(st)
+    return int(fl.value)

@@ -1,0 +1,190 @@
+// Host side of the C ABI declared in include/brs.h: argument validation,
+// byte-layout arithmetic, kernel dispatch, error reporting.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "brs.h"
+#include "brs_internal.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+brs_status fail(brs_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+brs_status ok() {
+  g_err[0] = 0;
+  return BRS_OK;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+// float nearest to 1/sqrt(d)
+float hadamard_scale(int d) { return (float)(1.0 / std::sqrt((double)d)); }
+
+brs_status check_layout(const brs_layout* L) {
+  if (!L) return fail(BRS_EINVAL, "layout is NULL");
+  if (L->B <= 0 || L->H <= 0 || L->H_k <= 0) return fail(BRS_EINVAL, "B, H, H_k must be positive");
+  if (L->H % L->H_k) return fail(BRS_EINVAL, "H (%d) must be a multiple of H_k (%d)", L->H, L->H_k);
+  if (L->d != 32 && L->d != 64 && L->d != 128) return fail(BRS_EINVAL, "d must be 32, 64 or 128 (got %d)", L->d);
+  if (L->storage == BRS_STORE_DAMP) {
+    if (L->k_hi < 0 || L->k_hi > L->d || (L->k_hi % 4)) return fail(BRS_EINVAL, "k_hi must be a multiple of 4 in [0, d]");
+    if (!pow2(L->block) || L->block < 4 || L->block > L->d)
+      return fail(BRS_EINVAL, "block must be a power of two in [4, d] (got %d)", L->block);
+  } else if (L->storage == BRS_STORE_VARBIT) {
+    if (L->hadamard) return fail(BRS_EUNSUPPORTED, "variable-width storage is stored without the Hadamard");
+    if (L->b_min < 2 || L->b_max > 8 || L->b_min > L->b_max) return fail(BRS_EINVAL, "need 2 <= b_min <= b_max <= 8");
+    const double tot = L->avg_bits * (double)L->H * (double)L->d;
+    if (tot != std::floor(tot)) return fail(BRS_EINVAL, "avg_bits * H * d must be an integer");
+    if (L->avg_bits < L->b_min || L->avg_bits > L->b_max) return fail(BRS_EINVAL, "avg_bits outside [b_min, b_max]");
+  } else if (L->storage != BRS_STORE_FP32) {
+    return fail(BRS_EINVAL, "unknown storage %d", L->storage);
+  }
+  return BRS_OK;
+}
+
+size_t damp_head_bytes(const brs_layout* L) {
+  const size_t d = (size_t)L->d, kh = (size_t)L->k_hi;
+  return (d - kh) * d + kh * d * 2 + (d - kh) * (d / (size_t)L->block) * 4;
+}
+
+size_t head_bytes(const brs_layout* L) {
+  return L->storage == BRS_STORE_FP32 ? (size_t)L->d * L->d * 4 : damp_head_bytes(L);
+}
+
+brs_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(BRS_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* brs_last_error(void) { return g_err; }
+
+size_t brs_state_bytes(const brs_layout* L, size_t* aux_bytes, size_t* stats_bytes,
+                       size_t* workspace_bytes) {
+  if (check_layout(L) != BRS_OK) return 0;
+  const size_t heads = (size_t)L->B * L->H, d = (size_t)L->d;
+  size_t total = 0, aux = 0, stats = 0, ws = 256;
+  if (L->storage == BRS_STORE_FP32) {
+    total = heads * d * d * 4;
+  } else if (L->storage == BRS_STORE_DAMP) {
+    total = heads * damp_head_bytes(L);
+    aux = heads * (d - (size_t)L->k_hi) * d * 2;
+  } else {
+    const size_t rows = (size_t)L->H * d;
+    const size_t P = (size_t)((double)(d / 8) * L->avg_bits * (double)rows);
+    total = round256(P * L->B) + round256(rows * L->B * 2) + round256(rows * L->B) +
+            round256((rows + 1) * L->B * 4);
+    aux = heads * d * d * 2;
+    stats = heads * d * 2 * sizeof(double);
+  }
+  if (aux_bytes) *aux_bytes = aux;
+  if (stats_bytes) *stats_bytes = stats;
+  if (workspace_bytes) *workspace_bytes = ws;
+  ok();
+  return total;
+}
+
+brs_status brs_state_pack(const brs_layout* L, const float* S, const int16_t* perm,
+                          const uint8_t* widths, void* packed, void* workspace, void* stream) {
+  brs_status st = check_layout(L);
+  if (st != BRS_OK) return st;
+  (void)widths;
+  if (L->storage == BRS_STORE_VARBIT) return fail(BRS_EUNSUPPORTED, "variable-width pack is not built yet");
+  if (!S || !packed || !workspace) return fail(BRS_EINVAL, "S, packed and workspace are required");
+  if (!aligned16(S) || !aligned16(packed) || !aligned16(workspace) || (perm && !aligned16(perm)))
+    return fail(BRS_EALIGN, "device pointers must be 16-byte aligned");
+  brs::PackArgs a{};
+  a.B = L->B; a.H = L->H; a.d = L->d; a.storage = L->storage; a.k_hi = L->k_hi;
+  a.block = L->block; a.hadamard = L->hadamard; a.head_bytes = head_bytes(L);
+  a.hscale = hadamard_scale(L->d); a.S = S; a.perm = perm; a.packed = packed;
+  a.flags = (uint32_t*)workspace;
+  cudaError_t e = brs::launch_pack(a, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "pack launch");
+  return ok();
+}
+
+brs_status brs_state_unpack(const brs_layout* L, const void* packed, const int16_t* perm,
+                            float* S, void* workspace, void* stream) {
+  brs_status st = check_layout(L);
+  if (st != BRS_OK) return st;
+  if (L->storage == BRS_STORE_VARBIT) return fail(BRS_EUNSUPPORTED, "variable-width unpack is not built yet");
+  if (!S || !packed) return fail(BRS_EINVAL, "S and packed are required");
+  if (!aligned16(S) || !aligned16(packed) || (perm && !aligned16(perm)))
+    return fail(BRS_EALIGN, "device pointers must be 16-byte aligned");
+  brs::PackArgs a{};
+  a.B = L->B; a.H = L->H; a.d = L->d; a.storage = L->storage; a.k_hi = L->k_hi;
+  a.block = L->block; a.hadamard = L->hadamard; a.head_bytes = head_bytes(L);
+  a.hscale = hadamard_scale(L->d); a.perm = perm; a.flags = (uint32_t*)workspace;
+  cudaError_t e = brs::launch_unpack(a, S, packed, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "unpack launch");
+  return ok();
+}
+
+brs_status brs_decode_step(const brs_layout* L, const brs_writeback* wb, int64_t step,
+                           const void* packed_in, void* packed_out, void* aux, void* stats,
+                           void* workspace, const int16_t* perm, const uint16_t* q,
+                           const uint16_t* k, const uint16_t* v, const float* beta,
+                           const float* decay, float* o, void* stream) {
+  brs_status st = check_layout(L);
+  if (st != BRS_OK) return st;
+  (void)stats;
+  if (!wb) return fail(BRS_EINVAL, "writeback is NULL");
+  if (wb->C != 1) return fail(BRS_EUNSUPPORTED, "decode writes back every token (C = 1); got C = %d", wb->C);
+  if (wb->mode < 0 || wb->mode > 2) return fail(BRS_EINVAL, "unknown rounding mode %d", wb->mode);
+  if (step < 0) return fail(BRS_EINVAL, "step must be >= 0");
+  if (L->storage == BRS_STORE_VARBIT) return fail(BRS_EUNSUPPORTED, "variable-width decode is not built yet");
+  if (!packed_in || !packed_out || !workspace || !q || !k || !v || !beta || !decay || !o)
+    return fail(BRS_EINVAL, "a required pointer is NULL");
+  if (L->storage == BRS_STORE_DAMP && wb->mode == BRS_ROUND_ERRFEEDBACK && !aux)
+    return fail(BRS_EINVAL, "error feedback needs the residual buffer");
+  const void* ptrs[] = {packed_in, packed_out, aux, workspace, perm, q, k, v, beta, decay, o};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(BRS_EALIGN, "device pointers must be 16-byte aligned");
+  brs::DecodeArgs a{};
+  a.B = L->B; a.H = L->H; a.Hk = L->H_k;
+  a.k_hi = L->storage == BRS_STORE_DAMP ? L->k_hi : 0;
+  a.block = L->storage == BRS_STORE_DAMP ? L->block : L->d;
+  a.decay_per_key = L->decay_per_key; a.mode = wb->mode; a.seed = wb->seed; a.step = step;
+  a.head_bytes = head_bytes(L); a.hscale = hadamard_scale(L->d);
+  a.packed_in = packed_in; a.packed_out = packed_out; a.aux = aux; a.perm = perm;
+  a.q = q; a.k = k; a.v = v; a.beta = beta; a.decay = decay; a.o = o;
+  a.flags = (uint32_t*)workspace;
+  const bool rot = L->storage == BRS_STORE_DAMP && L->hadamard;
+  cudaError_t e = brs::launch_decode(a, L->d, L->storage, rot, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return ok();
+}
+
+brs_status brs_fetch_errors(void* workspace, uint32_t* flags_out, void* stream) {
+  if (!workspace) return fail(BRS_EINVAL, "workspace is NULL");
+  uint32_t fl = 0;
+  cudaError_t e = cudaMemcpyAsync(&fl, workspace, 4, cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(workspace, 0, 4, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device flag word");
+  if (flags_out) *flags_out = fl;
+  if (fl & BRS_FLAG_NONFINITE) return fail(BRS_ENONFINITE, "a kernel met a non-finite state value");
+  if (fl & BRS_FLAG_OVERFLOW) return fail(BRS_EOVERFLOW, "an FP16 row, scale or zero overflowed");
+  if (fl & BRS_FLAG_TIMEOUT) return fail(BRS_ETIMEOUT, "a bounded device wait gave up");
+  return ok();
+}
+
+}  // extern "C"

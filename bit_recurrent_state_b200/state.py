@@ -1,0 +1,51 @@
+"""Device buffers of one layer's recurrent state, allocated with torch, and
+a step loop over the C ABI.  Marshalling only: the arithmetic is in
+libbrs.so."""
+from __future__ import annotations
+
+import torch
+
+from . import brs
+
+
+class LayerState:
+    """Stored state + residuals + statistics + workspace of one layer."""
+
+    def __init__(self, layout: brs.Layout, device="cuda", perm=None):
+        self.layout = layout
+        self.device = torch.device(device)
+        nbytes, aux, stats, ws = brs.state_bytes(layout)
+        self.packed = torch.zeros(nbytes, dtype=torch.uint8, device=self.device)
+        self.aux = torch.zeros(max(aux, 16), dtype=torch.uint8, device=self.device)
+        self.stats = torch.zeros(max(stats, 16), dtype=torch.uint8, device=self.device)
+        self.workspace = torch.zeros(ws, dtype=torch.uint8, device=self.device)
+        self.perm = None
+        if perm is not None:
+            self.perm = torch.as_tensor(perm, dtype=torch.int16).contiguous().to(self.device)
+
+    def pack(self, S: torch.Tensor, widths=None):
+        brs.state_pack(self.layout, S.contiguous(), self.perm, self.packed, self.workspace,
+                       widths=widths)
+
+    def unpack(self) -> torch.Tensor:
+        L = self.layout
+        S = torch.empty((L.B, L.H, L.d, L.d), dtype=torch.float32, device=self.device)
+        brs.state_unpack(L, self.packed, self.perm, S, self.workspace)
+        return S
+
+    def zero(self):
+        L = self.layout
+        self.pack(torch.zeros((L.B, L.H, L.d, L.d), dtype=torch.float32, device=self.device))
+        self.aux.zero_()
+        self.stats.zero_()
+
+    def step(self, wb: brs.WriteBack, t: int, q, k, v, beta, decay, o, packed_out=None):
+        out = self.packed if packed_out is None else packed_out
+        brs.decode_step(self.layout, wb, t, self.packed, out, self.aux, self.stats,
+                        self.workspace, self.perm, q, k, v, beta, decay, o)
+        if packed_out is not None:
+            self.packed, out = out, self.packed
+        return out
+
+    def errors(self) -> int:
+        return brs.fetch_errors(self.workspace)

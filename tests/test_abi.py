@@ -1,0 +1,36 @@
+"""The C-ABI library loads on a machine without a GPU and exports every
+symbol include/brs.h declares (no compute calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "brs.h")).read()
+    return sorted(set(re.findall(r"\b(brs_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declarations_exported():
+    from bit_recurrent_state_b200 import brs
+    import __graft_entry__
+    __graft_entry__.build()
+    lib = ctypes.CDLL(brs.LIB_PATH)
+    names = _declared()
+    assert set(brs.SYMBOLS) <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_host_only_calls_without_gpu():
+    from bit_recurrent_state_b200 import brs, synth
+    w = synth.WORKLOADS["kda_decode"]
+    n, aux, st, ws = brs.state_bytes(brs.layout_of(w))
+    assert n == 18880 * 64 * 32 and aux == 112 * 128 * 2 * 2048 and ws >= 4
+    w = synth.WORKLOADS["gdn_decode"]
+    assert brs.state_bytes(brs.layout_of(w))[0] == 16896 * 256 * 32
+    with pytest.raises(brs.BrsError):
+        brs.state_bytes(brs.layout_of(w, H_k=5))

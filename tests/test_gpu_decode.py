@@ -1,0 +1,159 @@
+"""GPU parity of the decode step (FP32 and DAMP storage) against the oracle,
+through the C ABI.  Stored bytes (codes, FP16 rows, FP16 scale/zero,
+residuals) must be identical; outputs within 2e-3 x RMS (expected identical
+given the shared operation order)."""
+import numpy as np
+import pytest
+
+from bit_recurrent_state_b200 import synth
+from parity import MODE, o_tolerance, oracle_cfg, random_perm, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_both(w, T, perm=None, units=None, init_scale=0.0, seed_state=0):
+    import torch
+    from bit_recurrent_state_b200 import brs
+    from bit_recurrent_state_b200.state import LayerState
+    from oracle import oracle as O
+
+    cfg = oracle_cfg(w)
+    L = brs.layout_of(w)
+    wb = brs.writeback_of(w)
+    st = LayerState(L, perm=perm)
+    S0 = (np.random.default_rng(seed_state).standard_normal((w.B, w.H, w.d, w.d)) * init_scale).astype(np.float32)
+    st.pack(torch.from_numpy(S0).cuda())
+    packed_o, _ = O.state_pack(cfg, S0, perm)
+    _, aux_o, stats_o = O.new_state(cfg)
+    gpu_packed0 = st.packed.cpu().numpy()
+    np.testing.assert_array_equal(gpu_packed0, packed_o)      # pack parity
+    o_gpu = torch.zeros((w.B, w.H, w.d), dtype=torch.float32, device="cuda")
+    steps = []
+    for t in range(T):
+        inp = synth.token_inputs(w, t)
+        dev = to_dev(inp)
+        st.step(wb, t, dev["q"], dev["k"], dev["v"], dev["beta"], dev["decay"], o_gpu)
+        og = o_gpu.cpu().numpy()
+        oo, fl, _ = O.run_parallel(cfg, MODE[w.mode], w.seed, 1, t,
+                                   {k: v[None] for k, v in inp.items()}, packed_o, aux=aux_o,
+                                   stats=stats_o, perm=perm, units=units)
+        assert fl == 0
+        steps.append((og, oo[0], st.packed.cpu().numpy().copy(), packed_o.copy(),
+                      st.aux.cpu().numpy()[: aux_o.nbytes].copy(), aux_o.view(np.uint8).copy()))
+    assert st.errors() == 0
+    return steps
+
+
+def _compare(w, steps, units=None):
+    hb = steps[0][2].size // (w.B * w.H)
+    sel = np.arange(w.B * w.H) if units is None else np.arange(*units)
+    for t, (og, oo, pg, po, ag, ao) in enumerate(steps):
+        og_u = og.reshape(w.B * w.H, w.d)[sel]
+        oo_u = oo.reshape(w.B * w.H, w.d)[sel]
+        tol = o_tolerance(oo_u)
+        assert np.max(np.abs(og_u - oo_u)) <= tol, (t, np.max(np.abs(og_u - oo_u)), tol)
+        pg_u = pg.reshape(w.B * w.H, hb)[sel]
+        po_u = po.reshape(w.B * w.H, hb)[sel]
+        ndiff = int(np.sum(pg_u != po_u))
+        assert ndiff == 0, f"step {t}: {ndiff} stored bytes differ"
+        if w.mode == "errfeedback":
+            per = ag.size // (w.B * w.H)
+            np.testing.assert_array_equal(ag.reshape(w.B * w.H, per)[sel], ao.reshape(w.B * w.H, per)[sel])
+
+
+def test_kda_tiny_full_trajectory():
+    w = synth.WORKLOADS["kda_tiny"]
+    perm = random_perm(w)
+    steps = _run_both(w, w.T, perm=perm)
+    _compare(w, steps)
+    # outputs bit-identical too (same operation order on both sides)
+    for og, oo, *_ in steps:
+        np.testing.assert_array_equal(og.view(np.uint32), oo.view(np.uint32))
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("kda128_ragged", dict(B=3, H=5, d=128, k_hi=16, block=128)),
+    ("kda128_block32", dict(B=2, H=3, d=128, k_hi=16, block=32)),
+    ("kda64", dict(B=2, H=3, d=64, k_hi=8, block=64)),
+    ("kda32_nohad", dict(B=2, H=2, d=32, k_hi=4, block=32, hadamard=0)),
+    ("gdn128", dict(B=3, H=4, Hk=2, d=128, k_hi=0, block=128, decay_per_key=0)),
+    ("kda128_sr", dict(B=2, H=3, d=128, k_hi=16, block=128, mode="stochastic")),
+    ("kda128_ef", dict(B=2, H=3, d=128, k_hi=16, block=128, mode="errfeedback")),
+    ("kda32_ef", dict(B=1, H=2, d=32, k_hi=4, block=32, mode="errfeedback")),
+    ("fp32_64", dict(B=2, H=3, d=64, storage="fp32")),
+    ("fp32_gdn128", dict(B=2, H=4, Hk=2, d=128, storage="fp32", decay_per_key=0)),
+])
+def test_small_configs_bit_exact(name, kw):
+    w = synth.Workload(name, T=12, seed=7, **kw)
+    perm = random_perm(w, seed=3)
+    steps = _run_both(w, w.T, perm=perm, init_scale=0.05)
+    _compare(w, steps)
+
+
+def test_kda_decode_full_size_sampled():
+    """The measured KDA configuration (B=64, H=32, d=128, 16 FP16 rows +
+    112 INT8 Hadamard rows, block 128), in the benchmark's launch
+    configuration, for 48 tokens; the oracle runs 64 of the 2048 heads."""
+    w = synth.WORKLOADS["kda_decode"]
+    perm = random_perm(w, seed=5)
+    units = (1000, 1064)
+    steps = _run_both(w, 48, perm=perm, units=units)
+    _compare(w, steps, units=units)
+
+
+def test_gdn_decode_full_size_sampled():
+    w = synth.WORKLOADS["gdn_decode"]
+    units = (4000, 4064)
+    steps = _run_both(w, 24, units=units)
+    _compare(w, steps, units=units)
+
+
+def test_unpack_matches_oracle():
+    import torch
+    from bit_recurrent_state_b200 import brs
+    from bit_recurrent_state_b200.state import LayerState
+    from oracle import oracle as O
+    w = synth.Workload("u", B=2, H=3, d=128, T=1, k_hi=16, block=32)
+    perm = random_perm(w, seed=9)
+    cfg = oracle_cfg(w)
+    S0 = np.random.default_rng(4).standard_normal((w.B, w.H, w.d, w.d)).astype(np.float32)
+    st = LayerState(brs.layout_of(w), perm=perm)
+    st.pack(torch.from_numpy(S0).cuda())
+    Sg = st.unpack().cpu().numpy()
+    So, _ = O.state_unpack(cfg, st.packed.cpu().numpy(), perm)
+    np.testing.assert_array_equal(Sg.view(np.uint32), So.view(np.uint32))
+
+
+def test_nonfinite_input_raises_flag():
+    import torch
+    from bit_recurrent_state_b200 import brs
+    from bit_recurrent_state_b200.state import LayerState
+    w = synth.Workload("nf", B=1, H=2, d=128, T=1, k_hi=16, block=128)
+    st = LayerState(brs.layout_of(w))
+    st.zero()
+    dev = to_dev(synth.token_inputs(w, 0))
+    dev["beta"][0, 1] = float("nan")
+    o = torch.zeros((1, 2, 128), device="cuda")
+    st.step(brs.writeback_of(w), 0, dev["q"], dev["k"], dev["v"], dev["beta"], dev["decay"], o)
+    assert st.errors() & brs.FLAG_NONFINITE
+    assert st.errors() == 0          # cleared by the first read
+
+
+def test_argument_errors():
+    import torch
+    from bit_recurrent_state_b200 import brs
+    w = synth.Workload("e", B=1, H=2, d=128, T=1, k_hi=16, block=128)
+    L = brs.layout_of(w, d=96)
+    with pytest.raises(brs.BrsError) as e:
+        brs.state_bytes(L)
+    assert "d must be" in str(e.value)
+    L = brs.layout_of(w)
+    buf = torch.zeros(1 << 20, dtype=torch.uint8, device="cuda")
+    with pytest.raises(brs.BrsError) as e:
+        brs.decode_step(L, brs.writeback_of(w), 0, buf[1:], buf, None, None, buf, None, buf, buf,
+                        buf, buf, buf, buf)
+    assert e.value.status == brs.EALIGN
+    with pytest.raises(brs.BrsError) as e:
+        brs.decode_step(L, brs.writeback_of(w, C=4), 0, buf, buf, None, None, buf, None, buf, buf,
+                        buf, buf, buf, buf)
+    assert e.value.status == brs.EUNSUPPORTED
