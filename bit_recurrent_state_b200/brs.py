@@ -77,7 +77,7 @@ def lib():
         L.brs_state_unpack.restype = S
         L.brs_state_unpack.argtypes = [P, P, P, P, P, P]
         L.brs_decode_step.restype = S
-        L.brs_decode_step.argtypes = [P, P, ct.c_int64] + [P] * 14
+        L.brs_decode_step.argtypes = [P, P, ct.c_int64] + [P] * 13
         L.brs_fetch_errors.restype = S
         L.brs_fetch_errors.argtypes = [P, P, P]
         L.brs_last_error.restype = ct.c_char_p

@@ -34,3 +34,24 @@ def test_host_only_calls_without_gpu():
     assert brs.state_bytes(brs.layout_of(w))[0] == 16896 * 256 * 32
     with pytest.raises(brs.BrsError):
         brs.state_bytes(brs.layout_of(w, H_k=5))
+
+
+def _param_counts():
+    src = open(os.path.join(ROOT, "include", "brs.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(brs_[a-z_]+)\s*\(([^)]*)\)\s*;", src):
+        args = m.group(2).strip()
+        out[m.group(1)] = 0 if args in ("", "void") else args.count(",") + 1
+    return out
+
+
+def test_binding_argument_counts_match_header():
+    from bit_recurrent_state_b200 import brs
+    lib = brs.lib()
+    counts = _param_counts()
+    assert counts, "no prototypes parsed"
+    for name, n in counts.items():
+        fn = getattr(lib, name)
+        assert fn.argtypes is not None, name
+        assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
