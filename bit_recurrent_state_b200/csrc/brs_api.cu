@@ -152,6 +152,10 @@ brs_status brs_decode_step(const brs_layout* L, const brs_writeback* wb, int64_t
   if (L->storage == BRS_STORE_VARBIT) return fail(BRS_EUNSUPPORTED, "variable-width decode is not built yet");
   if (!packed_in || !packed_out || !workspace || !q || !k || !v || !beta || !decay || !o)
     return fail(BRS_EINVAL, "a required pointer is NULL");
+  if (L->storage == BRS_STORE_DAMP && !brs::decode_supported(L->d, L->block))
+    return fail(BRS_EUNSUPPORTED, "decode kernel built for (d, block) in {(128,128), (128,32), (64,64), (32,32)}");
+  if (L->storage == BRS_STORE_DAMP && L->k_hi > L->d / 4)
+    return fail(BRS_EUNSUPPORTED, "decode kernel supports k_hi <= d/4");
   if (L->storage == BRS_STORE_DAMP && wb->mode == BRS_ROUND_ERRFEEDBACK && !aux)
     return fail(BRS_EINVAL, "error feedback needs the residual buffer");
   const void* ptrs[] = {packed_in, packed_out, aux, workspace, perm, q, k, v, beta, decay, o};

@@ -1,6 +1,7 @@
 // Device helpers shared by the library's kernels: binary16/bfloat16
-// conversion, Philox4x32-10, the per-row Hadamard butterflies across the
-// threads of a row group, and the device flag word.
+// conversion, paired FP32 arithmetic (sm_100 f32x2), Philox4x32-10, the
+// per-row Hadamard butterflies across the threads of a row group, and the
+// device flag word.
 #pragma once
 #include <cuda_fp16.h>
 #include <cstdint>
@@ -14,9 +15,82 @@ __device__ __forceinline__ float f16_to_f32(uint16_t h) { return __half2float(__
 __device__ __forceinline__ uint16_t f32_to_f16(float x) { return __half_as_ushort(__float2half_rn(x)); }
 __device__ __forceinline__ bool f16_inf_or_nan(uint16_t h) { return ((h >> 10) & 31u) == 31u; }
 
+// two floats -> f16x2 word (lo = a, hi = b), round to nearest even
+__device__ __forceinline__ uint32_t f16x2_of(float a, float b) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+  return r;
+}
+
 __device__ __forceinline__ void raise_flag(uint32_t* flags, uint32_t bit) {
   if (flags) atomicOr(flags, bit);
 }
+
+// ---- paired FP32 (one instruction, two independent IEEE operations)
+__device__ __forceinline__ uint64_t pk(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void upk(uint64_t r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+// (a0,a1) * (b0,b1) + (c0,c1), each a single-rounding fma
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
+                                     float c0, float c1) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(pk(a0, a1)), "l"(pk(b0, b1)), "l"(pk(c0, c1)));
+  upk(r, d0, d1);
+}
+__device__ __forceinline__ void mul2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pk(a0, a1)), "l"(pk(b0, b1)));
+  upk(r, d0, d1);
+}
+__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pk(a0, a1)), "l"(pk(b0, b1)));
+  upk(r, d0, d1);
+}
+__device__ __forceinline__ void sub2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pk(a0, a1)), "l"(pk(b0, b1)));
+  upk(r, d0, d1);
+}
+
+// packed pairs kept in 64-bit registers (no repacking between operations)
+typedef unsigned long long f2_t;
+__device__ __forceinline__ f2_t f2fma(f2_t a, f2_t b, f2_t c) {
+  f2_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ f2_t f2mul(f2_t a, f2_t b) {
+  f2_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ f2_t f2add(f2_t a, f2_t b) {
+  f2_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ f2_t f2sub(f2_t a, f2_t b) {
+  f2_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float f2lo(f2_t a) { return __uint_as_float((uint32_t)a); }
+__device__ __forceinline__ float f2hi(f2_t a) { return __uint_as_float((uint32_t)(a >> 32)); }
+__device__ __forceinline__ f2_t f2make(float lo, float hi) { return pk(lo, hi); }
+__device__ __forceinline__ f2_t f2dup(float x) { return pk(x, x); }
+
+// byte k of w as an exact float: the bits 0x4B0000bb are 2^23 + bb
+__device__ __forceinline__ float byte_magic(uint32_t w, int k) {
+  return __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540u | (uint32_t)k));
+}
+constexpr float kTwo23 = 8388608.0f;          // 2^23
+constexpr float kRoundMagic = 12582912.0f;    // 1.5 * 2^23: x + magic rounds to an integer (RNE)
 
 // Philox4x32-10 (Salmon et al., SC'11): ten rounds, key bumped by the Weyl
 // constants between rounds.
@@ -51,23 +125,27 @@ __device__ __forceinline__ float sr_round(float t, uint32_t r24) {
 // Must be called by every lane of the warp (full-mask shuffles).
 template <int D>
 __device__ __forceinline__ void row_fwht4(float (&x)[4], int cb, float scale) {
-  float a0 = __fadd_rn(x[0], x[1]), a1 = __fsub_rn(x[0], x[1]);
-  float a2 = __fadd_rn(x[2], x[3]), a3 = __fsub_rn(x[2], x[3]);
-  x[0] = __fadd_rn(a0, a2);
-  x[2] = __fsub_rn(a0, a2);
-  x[1] = __fadd_rn(a1, a3);
-  x[3] = __fsub_rn(a1, a3);
+  float a0, a1, a2, a3;
+  add2(a0, a2, x[0], x[2], x[1], x[3]);
+  sub2(a1, a3, x[0], x[2], x[1], x[3]);
+  add2(x[0], x[1], a0, a1, a2, a3);
+  sub2(x[2], x[3], a0, a1, a2, a3);
 #pragma unroll
   for (int m = 1; m < D / 4; m <<= 1) {
     const bool hi = (cb & m) != 0;
+    float o[4];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const float other = __shfl_xor_sync(0xffffffffu, x[c], m);
-      x[c] = hi ? __fsub_rn(other, x[c]) : __fadd_rn(x[c], other);
+    for (int c = 0; c < 4; ++c) o[c] = __shfl_xor_sync(0xffffffffu, x[c], m);
+    if (hi) {
+      sub2(x[0], x[1], o[0], o[1], x[0], x[1]);
+      sub2(x[2], x[3], o[2], o[3], x[2], x[3]);
+    } else {
+      add2(x[0], x[1], x[0], x[1], o[0], o[1]);
+      add2(x[2], x[3], x[2], x[3], o[2], o[3]);
     }
   }
-#pragma unroll
-  for (int c = 0; c < 4; ++c) x[c] = __fmul_rn(x[c], scale);
+  mul2(x[0], x[1], x[0], x[1], scale, scale);
+  mul2(x[2], x[3], x[2], x[3], scale, scale);
 }
 
 }  // namespace brs

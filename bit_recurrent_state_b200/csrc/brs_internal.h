@@ -26,6 +26,7 @@ struct DecodeArgs {
 };
 
 cudaError_t launch_decode(const DecodeArgs& a, int d, int store, bool rot, cudaStream_t st);
+bool decode_supported(int d, int block);
 
 struct PackArgs {
   int B, H, d, storage, k_hi, block, hadamard;

@@ -1,24 +1,28 @@
 // Decode step for FP32 and DAMP storage: one token for every (sequence,
-// head).  One CTA per head; 2*D threads; thread t owns the 4 consecutive
-// columns 4*(t % (D/4)) .. +3 of the R = D/8 consecutive stored rows
-// R*(t / (D/4)) .. +R-1, so the D x D FP32 state of the head lives in
-// registers for the whole step and every state byte crosses HBM once in
-// and once out.
+// head).  One CTA per head; 2*D threads (D/16 warps); thread t owns the 4
+// consecutive columns 4*(t % (D/4)) .. +3 of the R = D/8 consecutive stored
+// rows R*(t / (D/4)) .. +R-1, so the D x D FP32 state of the head lives in
+// registers for the whole step and every state byte crosses HBM once in and
+// once out.
 //
 // Sources: DAMP summary, Key Points > Implementation (fused executor:
 // reconstruct the INT8 channels, update in FP32, re-quantize, write back;
-// static permutation with the protected channels contiguous); "Low-Bit
-// Recurrent States in Hybrid Language Models", Accumulated readout error
-// (outputs precede quantization) and Protocol (quantized and dequantized
-// before reuse).
+// static permutation with the protected channels contiguous) and Data &
+// Methods > Quantization & calibration details (per-block asymmetric INT8
+// after a Hadamard along the value axis); "Low-Bit Recurrent States in
+// Hybrid Language Models", Accumulated readout error (outputs precede
+// quantization) and Protocol (quantized and dequantized before reuse).
 //
-// Sums over key rows are fmaf chains over stored rows 0..D-1 in order: the
-// 8 row groups pass the running column sums to each other through shared
-// memory, one group at a time.
+// Operation order (shared with the oracle's written definition): sums over
+// key rows are fmaf chains over stored rows 0..D-1, the 8 row groups
+// passing the running column sums to each other through shared memory, one
+// group at a time.  Paired f32x2 instructions are two independent IEEE
+// operations, so pairing does not change any result.
 //
 // With the Hadamard enabled the update runs in the Hadamard basis: the INT8
 // rows are used as stored (already rotated), the protected FP16 rows and v
-// are rotated in, o and the FP16 rows are rotated out.
+// are rotated in, o and the FP16 rows are rotated out.  The FP16 rows are
+// transformed by all warps together through shared memory.
 #include <cuda_runtime.h>
 #include <cstdint>
 
@@ -27,313 +31,472 @@
 
 namespace brs {
 
-template <int D, int STORE, bool ROT>
-__global__ void __launch_bounds__(2 * D) decode_kernel(const DecodeArgs a) {
-  constexpr int NT = 2 * D;
-  constexpr int LPR = D / 4;   // threads per row
-  constexpr int R = D / 8;     // rows per thread
-  static_assert(NT % 32 == 0, "whole warps");
+template <int D>
+struct Geo {
+  static constexpr int NT = 2 * D;      // threads per CTA
+  static constexpr int NW = NT / 32;    // warps
+  static constexpr int LPR = D / 4;     // threads per row
+  static constexpr int R = D / 8;       // rows per thread
+  static constexpr int RPW = 32 / LPR;  // row groups per warp
+};
 
-  __shared__ float kk[D], qq[D], aa[D], vv[D], ww[D];
-  __shared__ float4 carry[LPR];
+struct __align__(16) QPrm {
+  f2_t zz, rr, ss;                      // (zero, zero), (1/scale, 1/scale), (scale, scale)
+  uint32_t bits, pad;                   // stored FP16 (scale, zero)
+};
 
-  const int t = threadIdx.x;
+template <int D>
+struct __align__(16) DecodeSmem {
+  f2_t kk2[D], qq2[D], aa2[D];          // gathered k, q, a, each duplicated into a pair
+  float vv[D], ww[D], cr[D];
+  float prot[D * D / 4];                // staging of protected rows (k_hi <= D/4)
+  QPrm prm[D][D / 32];                  // per (row, block) quantization grid
+};
+
+// Hadamard of the protected rows, done by every warp on rows staged in
+// shared memory: rows [0, nprot) of sm.prot, each of D floats.
+template <int D, bool TO_F16>
+__device__ __forceinline__ void prot_fwht(DecodeSmem<D>& sm, int nprot, float hscale, uint16_t* f16out,
+                                          uint32_t* flags) {
+  using G = Geo<D>;
+  const int t = threadIdx.x, warp = t / 32, lane = t % 32;
+  const int cb = lane % G::LPR, slot = lane / G::LPR;
+  for (int base = warp * G::RPW; base < nprot; base += G::NW * G::RPW) {  // warp-uniform bound
+    const int row = base + slot;
+    const bool live = row < nprot;
+    float x[4] = {0.f, 0.f, 0.f, 0.f};
+    if (live) {
+      const float4 v = *(const float4*)&sm.prot[row * D + 4 * cb];
+      x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+    }
+    row_fwht4<D>(x, cb, hscale);
+    if (!live) continue;
+    if constexpr (TO_F16) {
+      const uint32_t lo = f16x2_of(x[0], x[1]), hi = f16x2_of(x[2], x[3]);
+      const uint32_t e = ((lo >> 10) & 31u) == 31u || ((lo >> 26) & 31u) == 31u ||
+                         ((hi >> 10) & 31u) == 31u || ((hi >> 26) & 31u) == 31u;
+      if (e) raise_flag(flags, BRS_FLAG_OVERFLOW);
+      *(uint2*)&f16out[(size_t)row * D + 4 * cb] = make_uint2(lo, hi);
+    } else {
+      *(float4*)&sm.prot[row * D + 4 * cb] = make_float4(x[0], x[1], x[2], x[3]);
+    }
+  }
+}
+
+__device__ __forceinline__ void bar_sync_n(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+__device__ __forceinline__ void bar_arrive_n(int id, int n) { asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+
+// fmaf chain over stored rows 0..D-1 of the column pairs this thread owns;
+// the running sums pass from row group to row group through sm.cr.  With
+// one row group per warp (D = 128) the hand-off is a named barrier between
+// consecutive warps; otherwise the row groups take turns between CTA-wide
+// barriers.  Ends with a CTA-wide barrier; sm.cr then holds the sums.
+template <int D>
+__device__ __forceinline__ void row_chain(DecodeSmem<D>& sm, const f2_t* coef, const f2_t (&x)[D / 8][2],
+                                          int rb, int cb) {
+  using G = Geo<D>;
+  auto body = [&](bool first) {
+    f2_t a01 = 0ull, a23 = 0ull;
+    if (!first) {
+      a01 = *(const f2_t*)&sm.cr[4 * cb];
+      a23 = *(const f2_t*)&sm.cr[4 * cb + 2];
+    }
+#pragma unroll
+    for (int r = 0; r < G::R; ++r) {
+      const f2_t k = coef[rb * G::R + r];
+      a01 = f2fma(k, x[r][0], a01);
+      a23 = f2fma(k, x[r][1], a23);
+    }
+    *(f2_t*)&sm.cr[4 * cb] = a01;
+    *(f2_t*)&sm.cr[4 * cb + 2] = a23;
+  };
+  if constexpr (G::RPW == 1) {
+    if (rb > 0) bar_sync_n(rb, 64);
+    body(rb == 0);
+    if (rb < 7) bar_arrive_n(rb + 1, 64);
+    __syncthreads();
+  } else {
+    for (int s = 0; s < 8; ++s) {
+      if (rb == s) body(s == 0);
+      __syncthreads();
+    }
+  }
+}
+
+// Hadamard of one D-vector in shared memory, by warp 0.
+template <int D>
+__device__ __forceinline__ void vec_fwht(float* v, float hscale) {
+  const int lane = threadIdx.x % 32;
+  const int cb = lane % Geo<D>::LPR;
+  float x[4];
+  const float4 a = *(const float4*)&v[4 * cb];
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  row_fwht4<D>(x, cb, hscale);
+  __syncwarp();
+  if (lane < Geo<D>::LPR) *(float4*)&v[4 * cb] = make_float4(x[0], x[1], x[2], x[3]);
+  __syncwarp();
+}
+
+__device__ __forceinline__ uint32_t f16x2_overflow(uint32_t w) {
+  return (((w >> 10) & 31u) == 31u) | (((w >> 26) & 31u) == 31u);
+}
+
+template <int D, int STORE, bool ROT, int BLOCK, int MODE>
+__global__ void __launch_bounds__(2 * D, (D == 128) ? 2 : 4) decode_kernel(const DecodeArgs a) {
+  using G = Geo<D>;
+  constexpr int R = G::R, LPR = G::LPR;
+  constexpr int GL = BLOCK / 4;          // threads per quantization block
+  constexpr int NB = D / BLOCK;          // blocks per row
+  constexpr int V = 2 * R;               // (min, max) values per thread
+  constexpr int VPL = V / GL;            // values per lane after the reduce-scatter
+  static_assert(V >= GL, "reduce-scatter needs 2R >= BLOCK/4");
+  __shared__ DecodeSmem<D> sm;
+
+  const int t = threadIdx.x, lane = t % 32;
   const int cb = t % LPR, rb = t / LPR;
   const int row0 = rb * R, col0 = 4 * cb;
   const int head = blockIdx.x;
   const int b = head / a.H, h = head - b * a.H;
   const int kh = h * a.Hk / a.H;
-  const int nlo = D - a.k_hi;  // INT8 rows are stored rows 0..nlo-1
-
-  // ---- gather this token's inputs in stored row order
-  if (t < D) {
-    const int p = a.perm ? a.perm[h * D + t] : t;
-    const size_t qk = ((size_t)b * a.Hk + kh) * D;
-    kk[t] = bf16_to_f32(a.k[qk + p]);
-    qq[t] = bf16_to_f32(a.q[qk + p]);
-    aa[t] = a.decay_per_key ? a.decay[(size_t)head * D + p] : a.decay[head];
-    vv[t] = bf16_to_f32(a.v[(size_t)head * D + t]);
-  }
-  const float beta = a.beta[head];
-
-  // ---- load the head into registers
-  float x[R][4];
+  const int nlo = D - a.k_hi;            // INT8 rows are stored rows 0..nlo-1
   const uint8_t* hin = (const uint8_t*)a.packed_in + (size_t)head * a.head_bytes;
+  uint8_t* hout = (uint8_t*)a.packed_out + (size_t)head * a.head_bytes;
+  const uint8_t* f16in = hin + (size_t)nlo * D;
+  const uint32_t* szin = (const uint32_t*)(hin + (size_t)nlo * D + (size_t)a.k_hi * D * 2);
+
+  // ---- issue the state loads first, then gather the inputs
+  f2_t x[R][2];
+  uint32_t c4[R], sz[R];
   if constexpr (STORE == BRS_STORE_FP32) {
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-      const float4 f = *(const float4*)(hin + ((size_t)(row0 + r) * D + col0) * 4);
-      x[r][0] = f.x; x[r][1] = f.y; x[r][2] = f.z; x[r][3] = f.w;
+      const ulonglong2 f = *(const ulonglong2*)(hin + ((size_t)(row0 + r) * D + col0) * 4);
+      x[r][0] = f.x;
+      x[r][1] = f.y;
     }
   } else {
-    const int nb = D / a.block;
-    const uint8_t* f16base = hin + (size_t)nlo * D;
-    const uint32_t* szbase = (const uint32_t*)(hin + (size_t)nlo * D + (size_t)a.k_hi * D * 2);
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       const int i = row0 + r;
       if (i < nlo) {
-        const uint32_t c4 = *(const uint32_t*)(hin + (size_t)i * D + col0);
-        const uint32_t sz = szbase[i * nb + col0 / a.block];
-        const float s = f16_to_f32((uint16_t)(sz & 0xffffu));
-        const float z = f16_to_f32((uint16_t)(sz >> 16));
-#pragma unroll
-        for (int c = 0; c < 4; ++c) x[r][c] = __fmaf_rn(__uint2float_rn((c4 >> (8 * c)) & 0xffu), s, z);
+        c4[r] = __ldg((const uint32_t*)(hin + (size_t)i * D + col0));
+        sz[r] = __ldg(szin + i * NB + col0 / BLOCK);
       } else {
-        const uint2 hv = *(const uint2*)(f16base + ((size_t)(i - nlo) * D + col0) * 2);
-        x[r][0] = f16_to_f32((uint16_t)(hv.x & 0xffffu));
-        x[r][1] = f16_to_f32((uint16_t)(hv.x >> 16));
-        x[r][2] = f16_to_f32((uint16_t)(hv.y & 0xffffu));
-        x[r][3] = f16_to_f32((uint16_t)(hv.y >> 16));
+        const uint2 hv = __ldg((const uint2*)(f16in + ((size_t)(i - nlo) * D + col0) * 2));
+        c4[r] = hv.x;
+        sz[r] = hv.y;
       }
     }
   }
-  __syncthreads();  // kk/qq/aa/vv visible
+  if (t < D) {
+    const int p = a.perm ? a.perm[h * D + t] : t;
+    const size_t qk = ((size_t)b * a.Hk + kh) * D;
+    sm.kk2[t] = f2dup(bf16_to_f32(a.k[qk + p]));
+    sm.qq2[t] = f2dup(bf16_to_f32(a.q[qk + p]));
+    sm.aa2[t] = f2dup(a.decay_per_key ? a.decay[(size_t)head * D + p] : a.decay[head]);
+    sm.vv[t] = bf16_to_f32(a.v[(size_t)head * D + t]);
+  }
+  const float beta = a.beta[head];
 
-  if constexpr (ROT) {
-    // protected rows to the Hadamard basis (row groups are warp-aligned
-    // runs of lanes; loop bounds are kept warp-uniform for the shuffles)
+  // ---- dequantize
+  if constexpr (STORE != BRS_STORE_FP32) {
+    const f2_t two23 = f2dup(kTwo23);
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-      const bool mine = (row0 + r) >= nlo;
-      if (__any_sync(0xffffffffu, mine)) {
-        float y[4] = {x[r][0], x[r][1], x[r][2], x[r][3]};
-        row_fwht4<D>(y, cb, a.hscale);
-        if (mine) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c) x[r][c] = y[c];
+      const int i = row0 + r;
+      if (i < nlo) {
+        const f2_t ss = f2dup(f16_to_f32((uint16_t)(sz[r] & 0xffffu)));
+        const f2_t zz = f2dup(f16_to_f32((uint16_t)(sz[r] >> 16)));
+        const f2_t c01 = f2sub(f2make(byte_magic(c4[r], 0), byte_magic(c4[r], 1)), two23);
+        const f2_t c23 = f2sub(f2make(byte_magic(c4[r], 2), byte_magic(c4[r], 3)), two23);
+        x[r][0] = f2fma(c01, ss, zz);
+        x[r][1] = f2fma(c23, ss, zz);
+      } else {
+        x[r][0] = f2make(f16_to_f32((uint16_t)(c4[r] & 0xffffu)), f16_to_f32((uint16_t)(c4[r] >> 16)));
+        x[r][1] = f2make(f16_to_f32((uint16_t)(sz[r] & 0xffffu)), f16_to_f32((uint16_t)(sz[r] >> 16)));
+        if constexpr (ROT) {
+          *(f2_t*)&sm.prot[(i - nlo) * D + col0] = x[r][0];
+          *(f2_t*)&sm.prot[(i - nlo) * D + col0 + 2] = x[r][1];
         }
       }
     }
-    // v to the Hadamard basis: warp 0, butterflies on shared memory
-    if (t < 32) {
-      for (int hs = 1; hs < D; hs <<= 1) {
-        for (int p = t; p < D / 2; p += 32) {
-          const int i = (p / hs) * 2 * hs + (p % hs);
-          const float u0 = vv[i], u1 = vv[i + hs];
-          vv[i] = __fadd_rn(u0, u1);
-          vv[i + hs] = __fsub_rn(u0, u1);
-        }
-        __syncwarp();
+  }
+  __syncthreads();  // inputs and staged protected rows visible
+
+  if constexpr (ROT) {
+    prot_fwht<D, false>(sm, a.k_hi, a.hscale, nullptr, nullptr);
+    if (t < 32) vec_fwht<D>(sm.vv, a.hscale);
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int i = row0 + r;
+      if (i >= nlo) {
+        x[r][0] = *(const f2_t*)&sm.prot[(i - nlo) * D + col0];
+        x[r][1] = *(const f2_t*)&sm.prot[(i - nlo) * D + col0 + 2];
       }
-      for (int j = t; j < D; j += 32) vv[j] = __fmul_rn(vv[j], a.hscale);
     }
   }
 
   // ---- decay: S <- Diag(a) S
 #pragma unroll
   for (int r = 0; r < R; ++r) {
-    const float ar = aa[row0 + r];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) x[r][c] = __fmul_rn(ar, x[r][c]);
+    const f2_t ar = sm.aa2[row0 + r];
+    x[r][0] = f2mul(ar, x[r][0]);
+    x[r][1] = f2mul(ar, x[r][1]);
   }
 
-  // ---- u = S^T k, fmaf chain over stored rows 0..D-1
-  for (int s = 0; s < 8; ++s) {
-    if (rb == s) {
-      float4 acc = s ? carry[cb] : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const float kv = kk[row0 + r];
-        acc.x = __fmaf_rn(kv, x[r][0], acc.x);
-        acc.y = __fmaf_rn(kv, x[r][1], acc.y);
-        acc.z = __fmaf_rn(kv, x[r][2], acc.z);
-        acc.w = __fmaf_rn(kv, x[r][3], acc.w);
-      }
-      carry[cb] = acc;
-    }
-    __syncthreads();
-  }
-  // w = beta (v - u)
+  // ---- u = S^T k;  w = beta (v - u)
+  row_chain<D>(sm, sm.kk2, x, rb, cb);
   if (t < D) {
-    const float u = ((const float*)carry)[t];
+    const float u = sm.cr[t];
     if (!isfinite(u)) raise_flag(a.flags, BRS_FLAG_NONFINITE);
-    ww[t] = __fmul_rn(beta, __fsub_rn(vv[t], u));
+    sm.ww[t] = __fmul_rn(beta, __fsub_rn(sm.vv[t], u));
   }
   __syncthreads();
 
   // ---- S <- S + k w^T
   {
-    const float4 w4 = ((const float4*)ww)[cb];
+    const f2_t w01 = *(const f2_t*)&sm.ww[col0], w23 = *(const f2_t*)&sm.ww[col0 + 2];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-      const float kv = kk[row0 + r];
-      x[r][0] = __fmaf_rn(kv, w4.x, x[r][0]);
-      x[r][1] = __fmaf_rn(kv, w4.y, x[r][1]);
-      x[r][2] = __fmaf_rn(kv, w4.z, x[r][2]);
-      x[r][3] = __fmaf_rn(kv, w4.w, x[r][3]);
+      const f2_t kv = sm.kk2[row0 + r];
+      x[r][0] = f2fma(kv, w01, x[r][0]);
+      x[r][1] = f2fma(kv, w23, x[r][1]);
     }
   }
 
   // ---- o = S^T q from the updated FP32 state (before quantization)
-  for (int s = 0; s < 8; ++s) {
-    if (rb == s) {
-      float4 acc = s ? carry[cb] : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const float qv = qq[row0 + r];
-        acc.x = __fmaf_rn(qv, x[r][0], acc.x);
-        acc.y = __fmaf_rn(qv, x[r][1], acc.y);
-        acc.z = __fmaf_rn(qv, x[r][2], acc.z);
-        acc.w = __fmaf_rn(qv, x[r][3], acc.w);
-      }
-      carry[cb] = acc;
-    }
-    __syncthreads();
-  }
+  row_chain<D>(sm, sm.qq2, x, rb, cb);
   if constexpr (ROT) {
-    if (t < 32) {
-      float* oo = (float*)carry;
-      for (int hs = 1; hs < D; hs <<= 1) {
-        for (int p = t; p < D / 2; p += 32) {
-          const int i = (p / hs) * 2 * hs + (p % hs);
-          const float u0 = oo[i], u1 = oo[i + hs];
-          oo[i] = __fadd_rn(u0, u1);
-          oo[i + hs] = __fsub_rn(u0, u1);
-        }
-        __syncwarp();
-      }
-      for (int j = t; j < D; j += 32) oo[j] = __fmul_rn(oo[j], a.hscale);
-    }
+    if (t < 32) vec_fwht<D>(sm.cr, a.hscale);
     __syncthreads();
   }
   if (t < D) {
-    const float ov = ((const float*)carry)[t];
+    const float ov = sm.cr[t];
     if (!isfinite(ov)) raise_flag(a.flags, BRS_FLAG_NONFINITE);
     a.o[(size_t)head * D + t] = ov;
   }
 
   // ---- write-back
-  uint8_t* hout = (uint8_t*)a.packed_out + (size_t)head * a.head_bytes;
   if constexpr (STORE == BRS_STORE_FP32) {
 #pragma unroll
     for (int r = 0; r < R; ++r)
-      *(float4*)(hout + ((size_t)(row0 + r) * D + col0) * 4) =
-          make_float4(x[r][0], x[r][1], x[r][2], x[r][3]);
+      *(ulonglong2*)(hout + ((size_t)(row0 + r) * D + col0) * 4) = make_ulonglong2(x[r][0], x[r][1]);
+    return;
   } else {
-    const int nb = D / a.block;
-    uint8_t* f16base = hout + (size_t)nlo * D;
-    uint32_t* szbase = (uint32_t*)(hout + (size_t)nlo * D + (size_t)a.k_hi * D * 2);
-    const int gl = a.block / 4;                          // threads per block
-    const uint32_t lane = t & 31;
-    // lanes of this thread's block group and of its row group (aligned runs)
-    const uint32_t gmask = (gl >= 32) ? 0xffffffffu : (((1u << gl) - 1u) << (lane & ~(uint32_t)(gl - 1)));
-    const uint32_t rmask = (LPR >= 32) ? 0xffffffffu : (((1u << LPR) - 1u) << (lane & ~(uint32_t)(LPR - 1)));
+    // protected rows: back to the value basis (all warps), FP16, stored
+    uint16_t* f16out = (uint16_t*)(hout + (size_t)nlo * D);
+    if constexpr (ROT) {
+      __syncthreads();  // every reader of sm.prot is done
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int i = row0 + r;
+        if (i >= nlo) {
+          *(f2_t*)&sm.prot[(i - nlo) * D + col0] = x[r][0];
+          *(f2_t*)&sm.prot[(i - nlo) * D + col0 + 2] = x[r][1];
+        }
+      }
+      __syncthreads();
+      prot_fwht<D, true>(sm, a.k_hi, a.hscale, f16out, a.flags);
+    } else {
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int i = row0 + r;
+        if (i >= nlo) {
+          const uint32_t lo = f16x2_of(f2lo(x[r][0]), f2hi(x[r][0]));
+          const uint32_t hi = f16x2_of(f2lo(x[r][1]), f2hi(x[r][1]));
+          if (f16x2_overflow(lo) | f16x2_overflow(hi)) raise_flag(a.flags, BRS_FLAG_OVERFLOW);
+          *(uint2*)&f16out[(size_t)(i - nlo) * D + col0] = make_uint2(lo, hi);
+        }
+      }
+    }
+
+    // INT8 rows: error-feedback target, block extremes
+    uint16_t* auxb = (MODE == BRS_ROUND_ERRFEEDBACK) ? (uint16_t*)a.aux + (size_t)head * nlo * D : nullptr;
+    if constexpr (MODE == BRS_ROUND_ERRFEEDBACK) {
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int i = row0 + r;
+        if (i < nlo) {
+          const uint2 ev = *(const uint2*)&auxb[(size_t)i * D + col0];
+          x[r][0] = f2add(x[r][0], f2make(f16_to_f32((uint16_t)(ev.x & 0xffffu)), f16_to_f32((uint16_t)(ev.x >> 16))));
+          x[r][1] = f2add(x[r][1], f2make(f16_to_f32((uint16_t)(ev.y & 0xffffu)), f16_to_f32((uint16_t)(ev.y >> 16))));
+        }
+      }
+    }
+    float v[V];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const float y0 = f2lo(x[r][0]), y1 = f2hi(x[r][0]), y2 = f2lo(x[r][1]), y3 = f2hi(x[r][1]);
+      v[2 * r] = fminf(fminf(y0, y1), fminf(y2, y3));
+      v[2 * r + 1] = fmaxf(fmaxf(y0, y1), fmaxf(y2, y3));
+    }
+    // reduce-scatter over the GL lanes of the block group: afterwards lane
+    // g (of its group) holds entries [g*VPL, (g+1)*VPL) reduced over the
+    // group (even entries minima, odd entries maxima)
+#pragma unroll
+    for (int m = GL / 2, len = V; m >= 1; m >>= 1, len >>= 1) {
+      const bool up = (lane & m) != 0;
+#pragma unroll
+      for (int i = 0; i < len / 2; ++i) {
+        const float lo = v[i], hi = v[i + len / 2];
+        const float other = __shfl_xor_sync(0xffffffffu, up ? lo : hi, m);
+        const float mine = up ? hi : lo;
+        if (len / 2 >= 2)
+          v[i] = (i & 1) ? fmaxf(mine, other) : fminf(mine, other);
+        else
+          v[i] = (lane & 1) ? fmaxf(mine, other) : fminf(mine, other);
+      }
+    }
+    constexpr int RPL = (VPL >= 2) ? VPL / 2 : 1;
+    float mnv[RPL], mxv[RPL];
+    if constexpr (VPL >= 2) {
+#pragma unroll
+      for (int q = 0; q < RPL; ++q) { mnv[q] = v[2 * q]; mxv[q] = v[2 * q + 1]; }
+    } else {
+      const float other = __shfl_xor_sync(0xffffffffu, v[0], 1);
+      mnv[0] = (lane & 1) ? other : v[0];
+      mxv[0] = (lane & 1) ? v[0] : other;
+    }
+    const int g = (lane % LPR) % GL;            // lane within its block group
+    const int blk = (lane % LPR) / GL;          // block index within the row
+    const int lr0 = (VPL >= 2) ? g * RPL : g / 2;
+    // a zero extreme takes the sign rule (-0 below +0): rare, warp-wide
+    bool zc = false;
+#pragma unroll
+    for (int q = 0; q < RPL; ++q) zc |= (mnv[q] == 0.0f) || (mxv[q] == 0.0f);
+    if (__any_sync(0xffffffffu, zc)) {
+      uint32_t nz = 0, pz = 0;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const float y[4] = {f2lo(x[r][0]), f2hi(x[r][0]), f2lo(x[r][1]), f2hi(x[r][1])};
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (y[c] == 0.0f) {
+            if (signbit(y[c])) nz |= 1u << r; else pz |= 1u << r;
+          }
+      }
+#pragma unroll
+      for (int m = 1; m < GL; m <<= 1) {
+        nz |= __shfl_xor_sync(0xffffffffu, nz, m);
+        pz |= __shfl_xor_sync(0xffffffffu, pz, m);
+      }
+#pragma unroll
+      for (int q = 0; q < RPL; ++q) {
+        const int lr = lr0 + q;
+        if (mnv[q] == 0.0f) mnv[q] = ((nz >> lr) & 1u) ? -0.0f : 0.0f;
+        if (mxv[q] == 0.0f) mxv[q] = ((pz >> lr) & 1u) ? 0.0f : -0.0f;
+      }
+    }
+    // grid of each (row, block): one division per row, spread over lanes
+#pragma unroll
+    for (int q = 0; q < RPL; ++q) {
+      const int i = rb * R + lr0 + q;            // stored row
+      if (((VPL >= 2) || ((lane & 1) == 0)) && i < nlo) {
+        if (!isfinite(mnv[q]) || !isfinite(mxv[q])) raise_flag(a.flags, BRS_FLAG_NONFINITE);
+        const uint16_t sh = f32_to_f16(__fdiv_rn(__fsub_rn(mxv[q], mnv[q]), 255.0f));
+        const uint16_t zh = f32_to_f16(mnv[q]);
+        if (f16_inf_or_nan(sh) || f16_inf_or_nan(zh)) raise_flag(a.flags, BRS_FLAG_OVERFLOW);
+        const float s = f16_to_f32(sh), z = f16_to_f32(zh);
+        const float rcp = (s == 0.0f) ? 0.0f : __frcp_rn(s);
+        const uint32_t bits = (uint32_t)sh | ((uint32_t)zh << 16);
+        QPrm pr;
+        pr.zz = f2dup(z); pr.rr = f2dup(rcp); pr.ss = f2dup(s); pr.bits = bits; pr.pad = 0;
+        sm.prm[i][blk] = pr;
+        ((uint32_t*)(hout + (size_t)nlo * D + (size_t)a.k_hi * D * 2))[i * NB + blk] = bits;
+      }
+    }
+    __syncwarp();
+
+    // quantize and store: code = clamp(round((y - zero) * (1/scale)), 0, 255);
+    // when scale is 0 the factor 1/scale is 0 and every code is 0
+    const f2_t magic = f2dup(kRoundMagic);
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       const int i = row0 + r;
-      if constexpr (ROT) {
-        const bool mine = i >= nlo;
-        if (__any_sync(0xffffffffu, mine)) {
-          float y[4] = {x[r][0], x[r][1], x[r][2], x[r][3]};
-          row_fwht4<D>(y, cb, a.hscale);
-          if (mine) {
+      if (i >= nlo) continue;
+      const QPrm& pr = sm.prm[i][col0 / BLOCK];
+      const f2_t t01 = f2mul(f2sub(x[r][0], pr.zz), pr.rr);
+      const f2_t t23 = f2mul(f2sub(x[r][1], pr.zz), pr.rr);
+      float c[4] = {f2lo(t01), f2hi(t01), f2lo(t23), f2hi(t23)};
+      if constexpr (MODE == BRS_ROUND_STOCHASTIC) {
+        const uint4 rnd = philox4x32_10(
+            make_uint4((uint32_t)(i * (D / 4) + cb), (uint32_t)a.step, (uint32_t)h, (uint32_t)b),
+            make_uint2((uint32_t)a.seed, (uint32_t)(a.seed >> 32)));
+        c[0] = sr_round(c[0], rnd.x >> 8);
+        c[1] = sr_round(c[1], rnd.y >> 8);
+        c[2] = sr_round(c[2], rnd.z >> 8);
+        c[3] = sr_round(c[3], rnd.w >> 8);
+      }
 #pragma unroll
-            for (int c = 0; c < 4; ++c) x[r][c] = y[c];
-          }
-        }
-      }
-      if (i >= nlo) {
-        // protected row: FP16, nearest
-        uint16_t hv[4];
-        bool ovf = false;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          hv[c] = f32_to_f16(x[r][c]);
-          ovf |= f16_inf_or_nan(hv[c]) && isfinite(x[r][c]);
-        }
-        if (ovf) raise_flag(a.flags, BRS_FLAG_OVERFLOW);
-        *(uint2*)(f16base + ((size_t)(i - nlo) * D + col0) * 2) =
-            make_uint2((uint32_t)hv[0] | ((uint32_t)hv[1] << 16), (uint32_t)hv[2] | ((uint32_t)hv[3] << 16));
-        continue;
-      }
-      // INT8 row, asymmetric block quantizer
-      float y[4] = {x[r][0], x[r][1], x[r][2], x[r][3]};
-      uint16_t* auxrow = nullptr;
-      if (a.mode == BRS_ROUND_ERRFEEDBACK) {
-        auxrow = (uint16_t*)a.aux + ((size_t)head * nlo + i) * D + col0;
-        const uint2 ev = *(const uint2*)auxrow;
-        y[0] = __fadd_rn(y[0], f16_to_f32((uint16_t)(ev.x & 0xffffu)));
-        y[1] = __fadd_rn(y[1], f16_to_f32((uint16_t)(ev.x >> 16)));
-        y[2] = __fadd_rn(y[2], f16_to_f32((uint16_t)(ev.y & 0xffffu)));
-        y[3] = __fadd_rn(y[3], f16_to_f32((uint16_t)(ev.y >> 16)));
-      }
-      float mn = fminf(fminf(y[0], y[1]), fminf(y[2], y[3]));
-      float mx = fmaxf(fmaxf(y[0], y[1]), fmaxf(y[2], y[3]));
-      for (int m = 1; m < gl; m <<= 1) {
-        mn = fminf(mn, __shfl_xor_sync(rmask, mn, m));
-        mx = fmaxf(mx, __shfl_xor_sync(rmask, mx, m));
-      }
-      if (mn == 0.0f || mx == 0.0f) {
-        // a zero extreme: -0 ranks below +0 (uniform within the block group)
-        bool negz = false, posz = false;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          negz |= (y[c] == 0.0f) && signbit(y[c]);
-          posz |= (y[c] == 0.0f) && !signbit(y[c]);
-        }
-        const unsigned nz = __reduce_or_sync(gmask, negz ? 1u : 0u);
-        const unsigned pz = __reduce_or_sync(gmask, posz ? 1u : 0u);
-        if (mn == 0.0f) mn = nz ? -0.0f : 0.0f;
-        if (mx == 0.0f) mx = pz ? 0.0f : -0.0f;
-      }
-      const uint16_t sh = f32_to_f16(__fdiv_rn(__fsub_rn(mx, mn), 255.0f));
-      const uint16_t zh = f32_to_f16(mn);
-      if (f16_inf_or_nan(sh) || f16_inf_or_nan(zh)) raise_flag(a.flags, BRS_FLAG_OVERFLOW);
-      const float s = f16_to_f32(sh), z = f16_to_f32(zh);
-      const float rcp = (s == 0.0f) ? 0.0f : __frcp_rn(s);
-      uint4 rnd = make_uint4(0, 0, 0, 0);
-      if (a.mode == BRS_ROUND_STOCHASTIC)
-        rnd = philox4x32_10(make_uint4((uint32_t)(i * (D / 4) + cb), (uint32_t)a.step, (uint32_t)h, (uint32_t)b),
-                            make_uint2((uint32_t)a.seed, (uint32_t)(a.seed >> 32)));
-      const uint32_t rw[4] = {rnd.x >> 8, rnd.y >> 8, rnd.z >> 8, rnd.w >> 8};
-      uint32_t packed4 = 0;
-      uint16_t e16[4];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float code = 0.0f;
-        if (s != 0.0f) {
-          const float tt = __fmul_rn(__fsub_rn(y[c], z), rcp);
-          code = (a.mode == BRS_ROUND_STOCHASTIC) ? sr_round(tt, rw[c]) : rintf(tt);
-          code = fminf(fmaxf(code, 0.0f), 255.0f);
-        }
-        packed4 |= ((uint32_t)(int)code) << (8 * c);
-        if (a.mode == BRS_ROUND_ERRFEEDBACK) {
-          const float xhat = __fmaf_rn(code, s, z);
-          float e = __fsub_rn(y[c], xhat);
-          if (e > s) e = s;
-          else if (e < -s) e = -s;
-          e16[c] = f32_to_f16(e);
-        }
-      }
+      for (int k = 0; k < 4; ++k) c[k] = fminf(fmaxf(c[k], 0.0f), 255.0f);
+      // nearest integer (ties to even): the low byte of (c + 1.5*2^23)
+      const f2_t m01 = f2add(f2make(c[0], c[1]), magic);
+      const f2_t m23 = f2add(f2make(c[2], c[3]), magic);
+      const uint32_t packed4 = __byte_perm(__byte_perm((uint32_t)m01, (uint32_t)(m01 >> 32), 0x0040u),
+                                           __byte_perm((uint32_t)m23, (uint32_t)(m23 >> 32), 0x0040u), 0x5410u);
       *(uint32_t*)(hout + (size_t)i * D + col0) = packed4;
-      if ((col0 % a.block) == 0) szbase[i * nb + col0 / a.block] = (uint32_t)sh | ((uint32_t)zh << 16);
-      if (a.mode == BRS_ROUND_ERRFEEDBACK)
-        *(uint2*)auxrow = make_uint2((uint32_t)e16[0] | ((uint32_t)e16[1] << 16),
-                                     (uint32_t)e16[2] | ((uint32_t)e16[3] << 16));
+      if constexpr (MODE == BRS_ROUND_ERRFEEDBACK) {
+        const f2_t q01 = f2fma(f2sub(m01, magic), pr.ss, pr.zz);   // stored value
+        const f2_t q23 = f2fma(f2sub(m23, magic), pr.ss, pr.zz);
+        const f2_t e01 = f2sub(x[r][0], q01), e23 = f2sub(x[r][1], q23);
+        const float s = f2lo(pr.ss);
+        float e[4] = {f2lo(e01), f2hi(e01), f2lo(e23), f2hi(e23)};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          if (e[k] > s) e[k] = s;
+          else if (e[k] < -s) e[k] = -s;
+        }
+        *(uint2*)&auxb[(size_t)i * D + col0] = make_uint2(f16x2_of(e[0], e[1]), f16x2_of(e[2], e[3]));
+      }
     }
   }
 }
 
-template <int D>
-static cudaError_t launch_d(const DecodeArgs& a, int store, bool rot, cudaStream_t st) {
+template <int D, int BLOCK, int MODE>
+static cudaError_t launch_dbm(const DecodeArgs& a, int store, bool rot, cudaStream_t st) {
   const dim3 grid(a.B * a.H), block(2 * D);
   if (store == BRS_STORE_FP32)
-    decode_kernel<D, BRS_STORE_FP32, false><<<grid, block, 0, st>>>(a);
+    decode_kernel<D, BRS_STORE_FP32, false, D, BRS_ROUND_NEAREST><<<grid, block, 0, st>>>(a);
   else if (rot)
-    decode_kernel<D, BRS_STORE_DAMP, true><<<grid, block, 0, st>>>(a);
+    decode_kernel<D, BRS_STORE_DAMP, true, BLOCK, MODE><<<grid, block, 0, st>>>(a);
   else
-    decode_kernel<D, BRS_STORE_DAMP, false><<<grid, block, 0, st>>>(a);
+    decode_kernel<D, BRS_STORE_DAMP, false, BLOCK, MODE><<<grid, block, 0, st>>>(a);
   return cudaGetLastError();
 }
 
-cudaError_t launch_decode(const DecodeArgs& a, int d, int store, bool rot, cudaStream_t st) {
-  switch (d) {
-    case 32: return launch_d<32>(a, store, rot, st);
-    case 64: return launch_d<64>(a, store, rot, st);
-    case 128: return launch_d<128>(a, store, rot, st);
-    default: return cudaErrorInvalidValue;
+template <int D, int BLOCK>
+static cudaError_t launch_db(const DecodeArgs& a, int store, bool rot, cudaStream_t st) {
+  switch (a.mode) {
+    case BRS_ROUND_NEAREST: return launch_dbm<D, BLOCK, BRS_ROUND_NEAREST>(a, store, rot, st);
+    case BRS_ROUND_STOCHASTIC: return launch_dbm<D, BLOCK, BRS_ROUND_STOCHASTIC>(a, store, rot, st);
+    case BRS_ROUND_ERRFEEDBACK: return launch_dbm<D, BLOCK, BRS_ROUND_ERRFEEDBACK>(a, store, rot, st);
   }
+  return cudaErrorInvalidValue;
+}
+
+bool decode_supported(int d, int block) {
+  return (d == 128 && (block == 128 || block == 32)) || (d == 64 && block == 64) ||
+         (d == 32 && block == 32);
+}
+
+cudaError_t launch_decode(const DecodeArgs& a, int d, int store, bool rot, cudaStream_t st) {
+  if (store == BRS_STORE_FP32) {
+    DecodeArgs f = a;
+    f.mode = BRS_ROUND_NEAREST;
+    f.k_hi = 0;
+    switch (d) {
+      case 32: return launch_dbm<32, 32, BRS_ROUND_NEAREST>(f, store, false, st);
+      case 64: return launch_dbm<64, 64, BRS_ROUND_NEAREST>(f, store, false, st);
+      case 128: return launch_dbm<128, 128, BRS_ROUND_NEAREST>(f, store, false, st);
+    }
+    return cudaErrorInvalidValue;
+  }
+  if (d == 128 && a.block == 128) return launch_db<128, 128>(a, store, rot, st);
+  if (d == 128 && a.block == 32) return launch_db<128, 32>(a, store, rot, st);
+  if (d == 64 && a.block == 64) return launch_db<64, 64>(a, store, rot, st);
+  if (d == 32 && a.block == 32) return launch_db<32, 32>(a, store, rot, st);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace brs

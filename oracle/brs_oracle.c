@@ -36,8 +36,9 @@
  *     recurrence (FP64 dense-matrix recurrence, beta=0/a=1 identity, unit-key
  *     invariant, dead zone and error feedback), storage accounting.
  *   parity unpinned: the order of FP32 operations inside a sum (a reading,
- *     see above) and the rotated-domain mode, which is pinned only against
- *     the canonical mode within the output tolerance.
+ *     see above) and the rotated-domain and mixed-basis modes, which are
+ *     pinned only against the canonical mode (teacher-forced: outputs to
+ *     FP32 rounding, codes apart only next to a rounding boundary).
  */
 #include "brs_oracle.h"
 
@@ -482,6 +483,14 @@ static int rotated(const orc_layout* L) {
   return L->domain == ORC_DOMAIN_ROTATED && L->storage == ORC_STORE_DAMP && L->hadamard;
 }
 
+/* Mixed basis: each tier of a DAMP head is updated in the basis it is
+ * stored in (INT8 rows in the Hadamard basis when the Hadamard is on, FP16
+ * rows in the value basis); only the k- and q-weighted row sums and w move
+ * between the bases. */
+static int mixed(const orc_layout* L) {
+  return L->domain == ORC_DOMAIN_MIXED && L->storage == ORC_STORE_DAMP;
+}
+
 /* Dequantize one DAMP head into S (d x d, stored row order: the d - k_hi
  * INT8 rows first, then the k_hi protected FP16 rows).  In the canonical
  * domain INT8 rows are returned to the value basis with the Hadamard (its
@@ -504,7 +513,7 @@ static void damp_load(const orc_layout* L, const uint8_t* head, float* S) {
         float z = orc_f32_from_f16(sz[((size_t)i * nb + bl) * 2 + 1]);
         row[j] = fmaf((float)codes[(size_t)i * d + j], s, z);
       }
-      if (L->hadamard && !rotated(L)) orc_fwht(row, d);
+      if (L->hadamard && !rotated(L) && !mixed(L)) orc_fwht(row, d);
     }
   }
 }
@@ -528,7 +537,7 @@ static int damp_store(const orc_layout* L, const orc_writeback* wb, int64_t step
         if (t_head) t_head[(size_t)i * d + j] = 0.0f;
       }
     } else {
-      if (L->hadamard && !rotated(L)) orc_fwht(tmp, d);
+      if (L->hadamard && !rotated(L) && !mixed(L)) orc_fwht(tmp, d);
       for (int bl = 0; bl < nb; ++bl) {
         int j0 = bl * L->block;
         uint16_t* e = aux_head ? aux_head + (size_t)i * d + j0 : NULL;
@@ -569,6 +578,50 @@ static void delta_rule_token(int d, float* S, const float* kk, const float* qq, 
     for (int i = 0; i < d; ++i) acc = fmaf(qq[i], S[(size_t)i * d + j], acc);
     oo[j] = acc;
   }
+}
+
+/* The same token in the mixed basis: rows 0..nlo-1 (INT8 tier) are in the
+ * basis T (the Hadamard, or the identity without it), rows nlo..d-1 (FP16
+ * tier) in the value basis.
+ *   u  = U2 + T(U1),  U1 = sum over rows < nlo of k_i S_i,  U2 = the rest;
+ *   w  = beta (v - u);  S_i += k_i T(w) for rows < nlo, S_i += k_i w else;
+ *   o  = O2 + T(O1) with O1, O2 the q-weighted sums of the updated rows.
+ * Each partial sum is an fmaf chain over its rows in stored order from +0. */
+static void delta_rule_token_mixed(int d, int nlo, int had, float* S, const float* kk,
+                                   const float* qq, const float* aa, const float* vv, float bt,
+                                   float* w, float* oo) {
+  float* p1 = (float*)malloc(sizeof(float) * (size_t)d);
+  float* wt = (float*)malloc(sizeof(float) * (size_t)d);
+  for (int i = 0; i < d; ++i)
+    for (int j = 0; j < d; ++j) S[(size_t)i * d + j] = aa[i] * S[(size_t)i * d + j];
+  for (int j = 0; j < d; ++j) {
+    float u1 = 0.0f, u2 = 0.0f;
+    for (int i = 0; i < nlo; ++i) u1 = fmaf(kk[i], S[(size_t)i * d + j], u1);
+    for (int i = nlo; i < d; ++i) u2 = fmaf(kk[i], S[(size_t)i * d + j], u2);
+    p1[j] = u1;
+    oo[j] = u2;
+  }
+  if (had) orc_fwht(p1, d);
+  for (int j = 0; j < d; ++j) {
+    float u = oo[j] + p1[j];
+    w[j] = bt * (vv[j] - u);
+    wt[j] = w[j];
+  }
+  if (had) orc_fwht(wt, d);
+  for (int i = 0; i < d; ++i)
+    for (int j = 0; j < d; ++j)
+      S[(size_t)i * d + j] = fmaf(kk[i], (i < nlo) ? wt[j] : w[j], S[(size_t)i * d + j]);
+  for (int j = 0; j < d; ++j) {
+    float o1 = 0.0f, o2 = 0.0f;
+    for (int i = 0; i < nlo; ++i) o1 = fmaf(qq[i], S[(size_t)i * d + j], o1);
+    for (int i = nlo; i < d; ++i) o2 = fmaf(qq[i], S[(size_t)i * d + j], o2);
+    p1[j] = o1;
+    oo[j] = o2;
+  }
+  if (had) orc_fwht(p1, d);
+  for (int j = 0; j < d; ++j) oo[j] = oo[j] + p1[j];
+  free(p1);
+  free(wt);
 }
 
 typedef struct {
@@ -616,9 +669,13 @@ static int run_head_unit(const orc_layout* L, const orc_writeback* wb, int64_t s
     int64_t step = step0 + t;
     float bt;
     gather_token(L, in, t, b, h, perm_h, kk, qq, aa, vv, &bt);
-    if (rotated(L)) orc_fwht(vv, d);
-    delta_rule_token(d, S, kk, qq, aa, vv, bt, w, oo);
-    if (rotated(L)) orc_fwht(oo, d);
+    if (mixed(L)) {
+      delta_rule_token_mixed(d, d - L->k_hi, L->hadamard, S, kk, qq, aa, vv, bt, w, oo);
+    } else {
+      if (rotated(L)) orc_fwht(vv, d);
+      delta_rule_token(d, S, kk, qq, aa, vv, bt, w, oo);
+      if (rotated(L)) orc_fwht(oo, d);
+    }
     memcpy(in->o + (((size_t)t * L->B + b) * L->H + h) * d, oo, sizeof(float) * (size_t)d);
     if ((step + 1) % wb->C == 0) {
       /* write-back: quantize, then continue from the dequantized state

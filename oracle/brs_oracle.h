@@ -28,7 +28,7 @@ extern "C" {
 
 enum { ORC_STORE_FP32 = 0, ORC_STORE_DAMP = 1, ORC_STORE_VARBIT = 2 };
 enum { ORC_ROUND_NEAREST = 0, ORC_ROUND_STOCHASTIC = 1, ORC_ROUND_ERRFEEDBACK = 2 };
-enum { ORC_DOMAIN_CANONICAL = 0, ORC_DOMAIN_ROTATED = 1 };
+enum { ORC_DOMAIN_CANONICAL = 0, ORC_DOMAIN_ROTATED = 1, ORC_DOMAIN_MIXED = 2 };
 
 /* status flags (OR-ed) */
 enum { ORC_OK = 0, ORC_EINVAL = 1, ORC_ENONFINITE = 2, ORC_EOVERFLOW = 4 };

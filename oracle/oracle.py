@@ -27,7 +27,7 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 
 STORE_FP32, STORE_DAMP, STORE_VARBIT = 0, 1, 2
 ROUND_NEAREST, ROUND_STOCHASTIC, ROUND_ERRFEEDBACK = 0, 1, 2
-DOMAIN_CANONICAL, DOMAIN_ROTATED = 0, 1
+DOMAIN_CANONICAL, DOMAIN_ROTATED, DOMAIN_MIXED = 0, 1, 2
 OK, EINVAL, ENONFINITE, EOVERFLOW = 0, 1, 2, 4
 
 
