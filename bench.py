@@ -135,11 +135,10 @@ class ClockSampler:
 
 def _oracle_cfg(w):
     from oracle import oracle as O
-    rot = w.storage == "damp" and w.hadamard
     st = {"fp32": O.STORE_FP32, "damp": O.STORE_DAMP, "varbit": O.STORE_VARBIT}[w.storage]
     return O.Config(B=w.B, H=w.H, Hk=w.hk, d=w.d, storage=st, k_hi=w.k_hi, block=w.block,
                     hadamard=w.hadamard, decay_per_key=w.decay_per_key,
-                    domain=O.DOMAIN_ROTATED if rot else O.DOMAIN_CANONICAL)
+                    domain=O.DOMAIN_MIXED if w.storage == "damp" else O.DOMAIN_CANONICAL)
 
 
 class OracleRunner:

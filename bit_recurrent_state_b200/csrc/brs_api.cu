@@ -152,10 +152,10 @@ brs_status brs_decode_step(const brs_layout* L, const brs_writeback* wb, int64_t
   if (L->storage == BRS_STORE_VARBIT) return fail(BRS_EUNSUPPORTED, "variable-width decode is not built yet");
   if (!packed_in || !packed_out || !workspace || !q || !k || !v || !beta || !decay || !o)
     return fail(BRS_EINVAL, "a required pointer is NULL");
-  if (L->storage == BRS_STORE_DAMP && !brs::decode_supported(L->d, L->block))
-    return fail(BRS_EUNSUPPORTED, "decode kernel built for (d, block) in {(128,128), (128,32), (64,64), (32,32)}");
-  if (L->storage == BRS_STORE_DAMP && L->k_hi > L->d / 4)
-    return fail(BRS_EUNSUPPORTED, "decode kernel supports k_hi <= d/4");
+  if (L->storage == BRS_STORE_DAMP && !brs::decode_supported(L->d, L->block, L->k_hi))
+    return fail(BRS_EUNSUPPORTED,
+                "decode kernel built for (d, block) in {(128,128), (128,32), (64,64), (32,32)} and "
+                "k_hi a multiple of d/8 up to d/4 (got d=%d block=%d k_hi=%d)", L->d, L->block, L->k_hi);
   if (L->storage == BRS_STORE_DAMP && wb->mode == BRS_ROUND_ERRFEEDBACK && !aux)
     return fail(BRS_EINVAL, "error feedback needs the residual buffer");
   const void* ptrs[] = {packed_in, packed_out, aux, workspace, perm, q, k, v, beta, decay, o};
@@ -170,8 +170,8 @@ brs_status brs_decode_step(const brs_layout* L, const brs_writeback* wb, int64_t
   a.packed_in = packed_in; a.packed_out = packed_out; a.aux = aux; a.perm = perm;
   a.q = q; a.k = k; a.v = v; a.beta = beta; a.decay = decay; a.o = o;
   a.flags = (uint32_t*)workspace;
-  const bool rot = L->storage == BRS_STORE_DAMP && L->hadamard;
-  cudaError_t e = brs::launch_decode(a, L->d, L->storage, rot, (cudaStream_t)stream);
+  const bool had = L->storage == BRS_STORE_DAMP && L->hadamard;
+  cudaError_t e = brs::launch_decode(a, L->d, L->storage, had, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return ok();
 }

@@ -25,8 +25,8 @@ struct DecodeArgs {
   uint32_t* flags;
 };
 
-cudaError_t launch_decode(const DecodeArgs& a, int d, int store, bool rot, cudaStream_t st);
-bool decode_supported(int d, int block);
+cudaError_t launch_decode(const DecodeArgs& a, int d, int store, bool had, cudaStream_t st);
+bool decode_supported(int d, int block, int k_hi);
 
 struct PackArgs {
   int B, H, d, storage, k_hi, block, hadamard;

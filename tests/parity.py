@@ -11,13 +11,12 @@ STORE = {"fp32": O.STORE_FP32, "damp": O.STORE_DAMP, "varbit": O.STORE_VARBIT}
 
 
 def oracle_cfg(w: synth.Workload) -> O.Config:
-    """The oracle mode the CUDA path follows: the DAMP update with the
-    Hadamard runs in the rotated domain."""
-    rot = w.storage == "damp" and w.hadamard
+    """The oracle mode the CUDA path follows: DAMP heads are updated in the
+    mixed basis (each tier in the basis it is stored in)."""
     return O.Config(B=w.B, H=w.H, Hk=w.hk, d=w.d, storage=STORE[w.storage], k_hi=w.k_hi,
                     block=w.block, hadamard=w.hadamard, decay_per_key=w.decay_per_key,
                     avg_bits=w.avg_bits, b_min=w.b_min, b_max=w.b_max,
-                    domain=O.DOMAIN_ROTATED if rot else O.DOMAIN_CANONICAL)
+                    domain=O.DOMAIN_MIXED if w.storage == "damp" else O.DOMAIN_CANONICAL)
 
 
 def random_perm(w: synth.Workload, seed=0):
