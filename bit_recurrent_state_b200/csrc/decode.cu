@@ -1,9 +1,12 @@
 // Decode step for FP32 and DAMP storage: one token for every (sequence,
-// head).  One CTA per head; 2*D threads (D/16 warps); thread t owns the 4
-// consecutive columns 4*(t % (D/4)) .. +3 of the R = D/8 consecutive stored
-// rows R*(t / (D/4)) .. +R-1 (its "row group"), so the D x D FP32 state of
-// the head lives in registers for the whole step and every state byte
-// crosses HBM once in and once out.
+// head).  One warp per head: lane l owns the CPL = D/32 consecutive columns
+// CPL*l .. CPL*l+CPL-1 of every row and streams the head's rows in stored
+// order twice: pass 1 dequantizes, decays and accumulates u = S^T k; pass 2
+// reads the rows again (from L2), repeats the identical dequantize and
+// decay, applies the delta-rule write, accumulates o = S^T q and requantizes
+// in batches of NRB rows.  Every sum over rows is therefore a lane-local
+// fmaf chain in stored order, no thread block barrier is involved, and many
+// heads run concurrently on every SM.
 //
 // Sources: DAMP summary, Key Points > Implementation (fused executor:
 // reconstruct the INT8 channels, update in FP32, re-quantize, write back;
@@ -19,9 +22,9 @@
 //   u = U2 + T(U1), w = beta (v - u), S_i += k_i T(w) (INT8 rows),
 //   S_i += k_i w (FP16 rows), o = O2 + T(O1),
 // with U1/O1 and U2/O2 fmaf chains over the INT8 and the FP16 rows in
-// stored order and T the Hadamard (or the identity).  Only three vectors of
-// D values are transformed per head.  Paired f32x2 instructions are two
-// independent IEEE operations, so pairing changes no result.
+// stored order and T the Hadamard (or the identity).  Paired f32x2
+// instructions are two independent IEEE operations: pairing changes no
+// result.
 #include <cuda_runtime.h>
 #include <cstdint>
 
@@ -30,413 +33,584 @@
 
 namespace brs {
 
+constexpr int kWarpsPerCta = 2;   // small CTAs: an even spread of heads over the SMs
+
 template <int D>
-struct Geo {
-  static constexpr int NT = 2 * D;      // threads per CTA
-  static constexpr int NW = NT / 32;    // warps
-  static constexpr int LPR = D / 4;     // threads per row
-  static constexpr int R = D / 8;       // rows per thread (8 row groups)
-  static constexpr int RPW = 32 / LPR;  // row groups per warp
+struct WGeo {
+  static constexpr int CPL = D / 32;             // columns per lane
+  static constexpr int NRB = (D >= 64) ? 8 : 4;  // rows per requantization batch
+};
+
+// per stored row, duplicated into pairs for the paired FP32 instructions:
+// ka = (k, k, a, a), sz = (scale, scale, zero, zero) of an INT8 row with one
+// block per row, qq = (q, q)
+struct __align__(16) RowScal {
+  float4 ka, sz;
 };
 
 struct __align__(16) QPrm {
-  f2_t zz, rr;                          // (zero, zero), (1/scale, 1/scale)
-  f2_t ss;                              // (scale, scale)
-  uint32_t ok, pad;                     // grid keeps every rounded code in [0, 255]
+  float z, rcp, s;
+  uint32_t pad;
 };
 
 template <int D>
-struct __align__(16) DecodeSmem {
-  f2_t kk2[D], qq2[D], aa2[D];          // gathered k, q, a, each duplicated into a pair
-  float vv[D], ww[D], wt[D];            // v, w (value basis), T(w)
-  float c1[D], c2[D];                   // running / final sums of the two tiers
-  QPrm prm[D][D / 32];                  // per (row, block) quantization grid
+struct __align__(16) WarpSmem {
+  RowScal rs[D];                                 // per stored row: k, a, grid
+  float2 qq[D];                                  // per stored row: q
+  float vec[D];                                  // vector scratch (sums, w)
+  QPrm prm[8][D / 32];                           // grids of one batch (row, block)
 };
 
-__device__ __forceinline__ void bar_sync_n(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
-__device__ __forceinline__ void bar_arrive_n(int id, int n) { asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory"); }
-
-// The row chains: row groups [0, ng1) accumulate into sm.c1, row groups
-// [ng1, 8) into sm.c2, each an fmaf chain over its rows in stored order
-// from +0.  With one row group per warp (D = 128) consecutive warps hand
-// off through named barriers (the two tiers run concurrently); otherwise
-// the row groups take turns between CTA-wide barriers.  Ends with a
-// CTA-wide barrier.
-template <int D>
-__device__ __forceinline__ void row_chains(DecodeSmem<D>& sm, const f2_t* coef, const f2_t (&x)[D / 8][2],
-                                           int rb, int cb, int ng1) {
-  using G = Geo<D>;
-  auto body = [&](bool first, float* acc) {
-    f2_t a01 = 0ull, a23 = 0ull;
-    if (!first) {
-      a01 = *(const f2_t*)&acc[4 * cb];
-      a23 = *(const f2_t*)&acc[4 * cb + 2];
-    }
-#pragma unroll
-    for (int r = 0; r < G::R; ++r) {
-      const f2_t k = coef[rb * G::R + r];
-      a01 = f2fma(k, x[r][0], a01);
-      a23 = f2fma(k, x[r][1], a23);
-    }
-    *(f2_t*)&acc[4 * cb] = a01;
-    *(f2_t*)&acc[4 * cb + 2] = a23;
-  };
-  if constexpr (G::RPW == 1) {
-    const bool tier1 = rb < ng1;
-    const int first = tier1 ? 0 : ng1, last = tier1 ? ng1 - 1 : 7;
-    if (rb > first) bar_sync_n(rb, 64);
-    body(rb == first, tier1 ? sm.c1 : sm.c2);
-    if (rb < last) bar_arrive_n(rb + 1, 64);
-    __syncthreads();
+// ---- per-lane vector helpers over CPL values (pairs use f32x2); scalar
+// factors arrive as the two halves of a duplicated pair
+template <int C>
+__device__ __forceinline__ void v_fma_s(float (&acc)[C], float k0, float k1, const float (&x)[C]) {
+  if constexpr (C == 1) {
+    acc[0] = __fmaf_rn(k0, x[0], acc[0]);
   } else {
-    for (int s = 0; s < 8; ++s) {
-      if (rb == s) body(s == 0 || s == ng1, (s < ng1) ? sm.c1 : sm.c2);
-      __syncthreads();
+#pragma unroll
+    for (int c = 0; c < C; c += 2) fma2(acc[c], acc[c + 1], k0, k1, x[c], x[c + 1], acc[c], acc[c + 1]);
+  }
+}
+template <int C>
+__device__ __forceinline__ void v_fma_vec(float (&x)[C], float k0, float k1, const float (&w)[C]) {
+  if constexpr (C == 1) {
+    x[0] = __fmaf_rn(k0, w[0], x[0]);
+  } else {
+#pragma unroll
+    for (int c = 0; c < C; c += 2) fma2(x[c], x[c + 1], k0, k1, w[c], w[c + 1], x[c], x[c + 1]);
+  }
+}
+template <int C>
+__device__ __forceinline__ void v_scale(float (&x)[C], float a0, float a1) {
+  if constexpr (C == 1) {
+    x[0] = __fmul_rn(a0, x[0]);
+  } else {
+#pragma unroll
+    for (int c = 0; c < C; c += 2) mul2(x[c], x[c + 1], a0, a1, x[c], x[c + 1]);
+  }
+}
+
+// dequantize CPL INT8 codes (the low CPL bytes of w, in column order):
+// value = fmaf(code, scale, zero)
+template <int C>
+__device__ __forceinline__ void dequant_int8(float (&x)[C], uint32_t w, float s0, float s1, float z0,
+                                             float z1) {
+  if constexpr (C == 1) {
+    const float c0 = __fsub_rn(byte_magic(w, 0), kTwo23);
+    x[0] = __fmaf_rn(c0, s0, z0);
+  } else {
+#pragma unroll
+    for (int c = 0; c < C; c += 2) {
+      float c0 = byte_magic(w, c), c1 = byte_magic(w, c + 1);
+      sub2(c0, c1, c0, c1, kTwo23, kTwo23);
+      fma2(x[c], x[c + 1], c0, c1, s0, s1, z0, z1);
     }
   }
 }
 
-// T of one D-vector in shared memory, in place, by the calling warp.
+// Sylvester Hadamard of a D-vector held CPL values per lane (lane l holds
+// elements CPL*l ..), butterflies h = 1, 2, 4, ... then one scaling; every
+// output is the same single add or subtract as in the sequential
+// transform.
 template <int D>
-__device__ __forceinline__ void vec_fwht(float* v, float hscale) {
-  const int lane = threadIdx.x % 32;
-  const int cb = lane % Geo<D>::LPR;
-  float x[4];
-  const float4 a = *(const float4*)&v[4 * cb];
-  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-  row_fwht4<D>(x, cb, hscale);
-  __syncwarp();
-  if (lane < Geo<D>::LPR) *(float4*)&v[4 * cb] = make_float4(x[0], x[1], x[2], x[3]);
-  __syncwarp();
+__device__ __forceinline__ void warp_fwht(float (&x)[D / 32], int lane, float scale) {
+  constexpr int C = D / 32;
+#pragma unroll
+  for (int hs = 1; hs < C; hs <<= 1)
+#pragma unroll
+    for (int i = 0; i < C; ++i)
+      if ((i & hs) == 0) {
+        const float u0 = x[i], u1 = x[i + hs];
+        x[i] = __fadd_rn(u0, u1);
+        x[i + hs] = __fsub_rn(u0, u1);
+      }
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) {
+    const bool hi = (lane & m) != 0;
+#pragma unroll
+    for (int i = 0; i < C; ++i) {
+      const float o = __shfl_xor_sync(0xffffffffu, x[i], m);
+      x[i] = hi ? __fsub_rn(o, x[i]) : __fadd_rn(x[i], o);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < C; ++i) x[i] = __fmul_rn(x[i], scale);
 }
 
 __device__ __forceinline__ uint32_t f16x2_overflow(uint32_t w) {
   return (((w >> 10) & 31u) == 31u) | (((w >> 26) & 31u) == 31u);
 }
 
-template <int D, int STORE, bool HAD, int BLOCK, int MODE>
-__global__ void __launch_bounds__(2 * D, (D == 128) ? 2 : 4) decode_kernel(const DecodeArgs a) {
-  using G = Geo<D>;
-  constexpr int R = G::R, LPR = G::LPR;
-  constexpr int GL = BLOCK / 4;          // threads per quantization block
-  constexpr int NB = D / BLOCK;          // blocks per row
-  constexpr int V = 2 * R;               // (min, max) values per thread
-  constexpr int VPL = V / GL;            // values per lane after the reduce-scatter
-  constexpr int RPL = (VPL >= 2) ? VPL / 2 : 1;
-  static_assert(V >= GL, "reduce-scatter needs 2R >= BLOCK/4");
-  __shared__ DecodeSmem<D> sm;
+// packed code byte of a float holding (code + 1.5*2^23)
+__device__ __forceinline__ uint32_t magic_byte(float m) { return __float_as_uint(m) & 0xffu; }
 
-  const int t = threadIdx.x, lane = t % 32;
-  const int cb = t % LPR, rb = t / LPR;
-  const int row0 = rb * R, col0 = 4 * cb;
-  const int head = blockIdx.x;
+template <int D, int STORE, bool HAD, int BLOCK, int MODE>
+__global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const DecodeArgs a) {
+  using G = WGeo<D>;
+  constexpr int C = G::CPL, NRB = G::NRB;
+  constexpr int NB = D / BLOCK;                  // blocks per row
+  constexpr int GL = BLOCK / C;                  // lanes per block
+  constexpr int V = 2 * NRB;                     // (min, max) entries per lane and batch
+  constexpr int HALV = (V < GL) ? V : GL;        // halving stages keep min(V, GL) entries apart
+  static_assert(GL <= 32 && (GL & (GL - 1)) == 0, "block spans a power-of-two run of lanes");
+  __shared__ WarpSmem<D> smem_all[kWarpsPerCta];
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int head = blockIdx.x * kWarpsPerCta + warp;
+  if (head >= a.B * a.H) return;                 // whole warp leaves together
+  WarpSmem<D>& sm = smem_all[warp];
   const int b = head / a.H, h = head - b * a.H;
   const int kh = h * a.Hk / a.H;
-  const int nlo = (STORE == BRS_STORE_FP32) ? D : D - a.k_hi;  // INT8 rows: 0..nlo-1
-  const int ng1 = nlo / R;               // row groups of the INT8 tier
-  const bool tier1 = rb < ng1;           // whole row group in one tier (k_hi % R == 0)
+  const int nlo = (STORE == BRS_STORE_FP32) ? D : D - a.k_hi;   // INT8 rows 0..nlo-1
+  const int col0 = C * lane;
   const uint8_t* hin = (const uint8_t*)a.packed_in + (size_t)head * a.head_bytes;
   uint8_t* hout = (uint8_t*)a.packed_out + (size_t)head * a.head_bytes;
+  const uint32_t* szin = (const uint32_t*)(hin + (size_t)nlo * D + (size_t)a.k_hi * D * 2);
+  uint32_t* szout = (uint32_t*)(hout + (size_t)nlo * D + (size_t)a.k_hi * D * 2);
+  const uint8_t* f16in = hin + (size_t)nlo * D;
+  uint16_t* f16out = (uint16_t*)(hout + (size_t)nlo * D);
+  uint16_t* auxb = (MODE == BRS_ROUND_ERRFEEDBACK) ? (uint16_t*)a.aux + (size_t)head * nlo * D : nullptr;
 
-  // ---- issue the state loads first, then gather the inputs
-  f2_t x[R][2];
-  uint32_t c4[R], sz[R];
-  if constexpr (STORE == BRS_STORE_FP32) {
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const ulonglong2 f = __ldg((const ulonglong2*)(hin + ((size_t)(row0 + r) * D + col0) * 4));
-      x[r][0] = f.x;
-      x[r][1] = f.y;
-    }
-  } else if (tier1) {
-    const uint32_t* szin = (const uint32_t*)(hin + (size_t)nlo * D + (size_t)a.k_hi * D * 2);
-#pragma unroll
-    for (int r = 0; r < R; ++r) c4[r] = __ldg((const uint32_t*)(hin + (size_t)(row0 + r) * D + col0));
-    if constexpr (NB == 1) {
-#pragma unroll
-      for (int r = 0; r < R; r += 4) {
-        const uint4 q4 = __ldg((const uint4*)(szin + row0 + r));
-        sz[r] = q4.x; sz[r + 1] = q4.y; sz[r + 2] = q4.z; sz[r + 3] = q4.w;
-      }
-    } else {
-#pragma unroll
-      for (int r = 0; r < R; ++r) sz[r] = __ldg(szin + (row0 + r) * NB + col0 / BLOCK);
-    }
-  } else {
-    const uint8_t* f16in = hin + (size_t)nlo * D;
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const uint2 hv = __ldg((const uint2*)(f16in + ((size_t)(row0 + r - nlo) * D + col0) * 2));
-      c4[r] = hv.x;
-      sz[r] = hv.y;
-    }
-  }
-  if (t < D) {
-    const int p = a.perm ? a.perm[h * D + t] : t;
+  // ---- inputs: k, a, q gathered through the permutation and the stored
+  // grid of every INT8 row, as ready pairs; v of my columns
+  for (int i = lane; i < D; i += 32) {
+    const int p = a.perm ? a.perm[h * D + i] : i;
     const size_t qk = ((size_t)b * a.Hk + kh) * D;
-    sm.kk2[t] = f2dup(bf16_to_f32(a.k[qk + p]));
-    sm.qq2[t] = f2dup(bf16_to_f32(a.q[qk + p]));
-    sm.aa2[t] = f2dup(a.decay_per_key ? a.decay[(size_t)head * D + p] : a.decay[head]);
-    sm.vv[t] = bf16_to_f32(a.v[(size_t)head * D + t]);
-    sm.c2[t] = 0.0f;                     // an empty FP16 tier sums to +0
+    const float kv = bf16_to_f32(a.k[qk + p]);
+    const float av = a.decay_per_key ? a.decay[(size_t)head * D + p] : a.decay[head];
+    const float qv = bf16_to_f32(a.q[qk + p]);
+    float sv = 0.f, zv = 0.f;
+    if (STORE != BRS_STORE_FP32 && NB == 1 && i < nlo) {
+      const uint32_t w = __ldg(szin + i);
+      sv = f16_to_f32((uint16_t)(w & 0xffffu));
+      zv = f16_to_f32((uint16_t)(w >> 16));
+    }
+    RowScal r;
+    r.ka = make_float4(kv, kv, av, av);
+    r.sz = make_float4(sv, sv, zv, zv);
+    sm.rs[i] = r;
+    sm.qq[i] = make_float2(qv, qv);
   }
+  float vv[C];
+#pragma unroll
+  for (int c = 0; c < C; ++c) vv[c] = bf16_to_f32(a.v[(size_t)head * D + col0 + c]);
   const float beta = a.beta[head];
+  __syncwarp();
 
-  // ---- dequantize
-  if constexpr (STORE != BRS_STORE_FP32) {
-    if (tier1) {
-      const f2_t two23 = f2dup(kTwo23);
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const f2_t ss = f2dup(f16_to_f32((uint16_t)(sz[r] & 0xffffu)));
-        const f2_t zz = f2dup(f16_to_f32((uint16_t)(sz[r] >> 16)));
-        const f2_t c01 = f2sub(f2make(byte_magic(c4[r], 0), byte_magic(c4[r], 1)), two23);
-        const f2_t c23 = f2sub(f2make(byte_magic(c4[r], 2), byte_magic(c4[r], 3)), two23);
-        x[r][0] = f2fma(c01, ss, zz);
-        x[r][1] = f2fma(c23, ss, zz);
+  // one stored row -> FP32 values of my columns (before decay)
+  auto load_row = [&](int i, float (&x)[C]) {
+    if constexpr (STORE == BRS_STORE_FP32) {
+      const float* src = (const float*)hin + (size_t)i * D + col0;
+      if constexpr (C == 4) {
+        const float4 f = __ldg((const float4*)src);
+        x[0] = f.x; x[1] = f.y; x[2] = f.z; x[3] = f.w;
+      } else if constexpr (C == 2) {
+        const float2 f = __ldg((const float2*)src);
+        x[0] = f.x; x[1] = f.y;
+      } else {
+        x[0] = __ldg(src);
       }
     } else {
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        x[r][0] = f2make(f16_to_f32((uint16_t)(c4[r] & 0xffffu)), f16_to_f32((uint16_t)(c4[r] >> 16)));
-        x[r][1] = f2make(f16_to_f32((uint16_t)(sz[r] & 0xffffu)), f16_to_f32((uint16_t)(sz[r] >> 16)));
+      if (i < nlo) {
+        uint32_t w;
+        if constexpr (C == 4) w = __ldg((const uint32_t*)(hin + (size_t)i * D + col0));
+        else if constexpr (C == 2) w = __ldg((const uint16_t*)(hin + (size_t)i * D + col0));
+        else w = __ldg(hin + (size_t)i * D + col0);
+        if constexpr (NB == 1) {
+          const float4 g = sm.rs[i].sz;
+          dequant_int8<C>(x, w, g.x, g.y, g.z, g.w);
+        } else {
+          const uint32_t szw = __ldg(szin + i * NB + col0 / BLOCK);
+          const float sv = f16_to_f32((uint16_t)(szw & 0xffffu)), zv = f16_to_f32((uint16_t)(szw >> 16));
+          dequant_int8<C>(x, w, sv, sv, zv, zv);
+        }
+      } else {
+        const uint16_t* src = (const uint16_t*)f16in + (size_t)(i - nlo) * D + col0;
+        if constexpr (C == 4) {
+          const uint2 hv = __ldg((const uint2*)src);
+          x[0] = f16_to_f32((uint16_t)(hv.x & 0xffffu)); x[1] = f16_to_f32((uint16_t)(hv.x >> 16));
+          x[2] = f16_to_f32((uint16_t)(hv.y & 0xffffu)); x[3] = f16_to_f32((uint16_t)(hv.y >> 16));
+        } else if constexpr (C == 2) {
+          const uint32_t hv = __ldg((const uint32_t*)src);
+          x[0] = f16_to_f32((uint16_t)(hv & 0xffffu)); x[1] = f16_to_f32((uint16_t)(hv >> 16));
+        } else {
+          x[0] = f16_to_f32(__ldg(src));
+        }
       }
     }
-  }
-  __syncthreads();  // inputs visible
+  };
 
-  // ---- decay: S <- Diag(a) S
+  // ---- pass 1: u = U2 + T(U1) over the decayed rows.  INT8 rows stream in
+  // chunks of CH rows with the next chunk's codes and grids already in
+  // flight (double buffering keeps 2*CH row loads per warp outstanding).
+  float u1[C], u2[C];
 #pragma unroll
-  for (int r = 0; r < R; ++r) {
-    const f2_t ar = sm.aa2[row0 + r];
-    x[r][0] = f2mul(ar, x[r][0]);
-    x[r][1] = f2mul(ar, x[r][1]);
-  }
-
-  // ---- u = U2 + T(U1);  w = beta (v - u);  T(w)
-  row_chains<D>(sm, sm.kk2, x, rb, cb, ng1);
-  if (t < 32) {
-    if constexpr (STORE != BRS_STORE_FP32 && HAD) vec_fwht<D>(sm.c1, a.hscale);
-    for (int j = t; j < D; j += 32) {
-      const float u = (STORE == BRS_STORE_FP32) ? sm.c1[j] : __fadd_rn(sm.c2[j], sm.c1[j]);
-      if (!isfinite(u)) raise_flag(a.flags, BRS_FLAG_NONFINITE);
-      const float w = __fmul_rn(beta, __fsub_rn(sm.vv[j], u));
-      sm.ww[j] = w;
-      sm.wt[j] = w;
-    }
-    __syncwarp();
-    if constexpr (STORE != BRS_STORE_FP32 && HAD) vec_fwht<D>(sm.wt, a.hscale);
-  }
-  __syncthreads();
-
-  // ---- S_i <- S_i + k_i T(w) (INT8 tier), S_i + k_i w (FP16 tier)
-  {
-    const float* wsrc = tier1 ? sm.wt : sm.ww;
-    const f2_t w01 = *(const f2_t*)&wsrc[col0], w23 = *(const f2_t*)&wsrc[col0 + 2];
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const f2_t kv = sm.kk2[row0 + r];
-      x[r][0] = f2fma(kv, w01, x[r][0]);
-      x[r][1] = f2fma(kv, w23, x[r][1]);
-    }
-  }
-
-  // ---- o = O2 + T(O1) from the updated FP32 state (before quantization)
-  if (t < D) sm.c2[t] = 0.0f;
-  __syncthreads();
-  row_chains<D>(sm, sm.qq2, x, rb, cb, ng1);
-  if (t < 32) {
-    if constexpr (STORE != BRS_STORE_FP32 && HAD) vec_fwht<D>(sm.c1, a.hscale);
-    for (int j = t; j < D; j += 32) {
-      const float ov = (STORE == BRS_STORE_FP32) ? sm.c1[j] : __fadd_rn(sm.c2[j], sm.c1[j]);
-      if (!isfinite(ov)) raise_flag(a.flags, BRS_FLAG_NONFINITE);
-      a.o[(size_t)head * D + j] = ov;
-    }
-  }
-
-  // ---- write-back
+  for (int c = 0; c < C; ++c) { u1[c] = 0.f; u2[c] = 0.f; }
   if constexpr (STORE == BRS_STORE_FP32) {
-#pragma unroll
-    for (int r = 0; r < R; ++r)
-      *(ulonglong2*)(hout + ((size_t)(row0 + r) * D + col0) * 4) = make_ulonglong2(x[r][0], x[r][1]);
-    return;
+#pragma unroll 8
+    for (int i = 0; i < D; ++i) {
+      float x[C];
+      load_row(i, x);
+      const float4 ka = sm.rs[i].ka;
+      v_scale<C>(x, ka.z, ka.w);
+      v_fma_s<C>(u1, ka.x, ka.y, x);
+    }
   } else {
-    if (!tier1) {
-      // protected rows: FP16, nearest
-      uint16_t* f16out = (uint16_t*)(hout + (size_t)nlo * D);
-      uint32_t ovf = 0;
+    // chunks of CH = NRB rows (nlo is a multiple of NRB), two in flight
+    constexpr int CH = NRB;
+    uint32_t cw[2][CH], sw[2][(NB > 1) ? CH : 1];
+    const uint8_t* crow = hin + col0;
+    const uint32_t* srow = szin + col0 / BLOCK;
+    auto fetch = [&](int buf) {
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const uint32_t lo = f16x2_of(f2lo(x[r][0]), f2hi(x[r][0]));
-        const uint32_t hi = f16x2_of(f2lo(x[r][1]), f2hi(x[r][1]));
-        ovf |= f16x2_overflow(lo) | f16x2_overflow(hi);
-        *(uint2*)&f16out[(size_t)(row0 + r - nlo) * D + col0] = make_uint2(lo, hi);
+      for (int r = 0; r < CH; ++r) {
+        if constexpr (C == 4) cw[buf][r] = __ldg((const uint32_t*)(crow + r * D));
+        else if constexpr (C == 2) cw[buf][r] = __ldg((const uint16_t*)(crow + r * D));
+        else cw[buf][r] = __ldg(crow + r * D);
+        if constexpr (NB > 1) sw[buf][r] = __ldg(srow + r * NB);
       }
-      if (ovf) raise_flag(a.flags, BRS_FLAG_OVERFLOW);
-      return;
-    }
-    // INT8 rows: error-feedback target, block extremes
-    uint16_t* auxb = (MODE == BRS_ROUND_ERRFEEDBACK) ? (uint16_t*)a.aux + (size_t)head * nlo * D : nullptr;
-    if constexpr (MODE == BRS_ROUND_ERRFEEDBACK) {
+      crow += CH * D;
+      srow += CH * NB;
+    };
+    auto consume = [&](int buf, int i0) {
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const uint2 ev = *(const uint2*)&auxb[(size_t)(row0 + r) * D + col0];
-        x[r][0] = f2add(x[r][0], f2make(f16_to_f32((uint16_t)(ev.x & 0xffffu)), f16_to_f32((uint16_t)(ev.x >> 16))));
-        x[r][1] = f2add(x[r][1], f2make(f16_to_f32((uint16_t)(ev.y & 0xffffu)), f16_to_f32((uint16_t)(ev.y >> 16))));
+      for (int r = 0; r < CH; ++r) {
+        float x[C];
+        const RowScal rsc = sm.rs[i0 + r];
+        if constexpr (NB == 1) {
+          dequant_int8<C>(x, cw[buf][r], rsc.sz.x, rsc.sz.y, rsc.sz.z, rsc.sz.w);
+        } else {
+          const float sv = f16_to_f32((uint16_t)(sw[buf][r] & 0xffffu));
+          const float zv = f16_to_f32((uint16_t)(sw[buf][r] >> 16));
+          dequant_int8<C>(x, cw[buf][r], sv, sv, zv, zv);
+        }
+        v_scale<C>(x, rsc.ka.z, rsc.ka.w);
+        v_fma_s<C>(u1, rsc.ka.x, rsc.ka.y, x);
+      }
+    };
+    const int nch = nlo / CH;
+    if (nch > 0) fetch(0);
+    for (int ch = 0; ch < nch; ch += 2) {
+      if (ch + 1 < nch) fetch(1);
+      consume(0, ch * CH);
+      if (ch + 2 < nch) fetch(0);
+      if (ch + 1 < nch) consume(1, (ch + 1) * CH);
+    }
+#pragma unroll 8
+    for (int i = nlo; i < D; ++i) {
+      float x[C];
+      load_row(i, x);
+      const float4 ka = sm.rs[i].ka;
+      v_scale<C>(x, ka.z, ka.w);
+      v_fma_s<C>(u2, ka.x, ka.y, x);
+    }
+  }
+  float w[C], wt[C];
+  {
+    if constexpr (STORE != BRS_STORE_FP32 && HAD) warp_fwht<D>(u1, lane, a.hscale);
+    bool bad = false;
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+      const float u = (STORE == BRS_STORE_FP32) ? u1[c] : __fadd_rn(u2[c], u1[c]);
+      bad |= !isfinite(u);
+      w[c] = __fmul_rn(beta, __fsub_rn(vv[c], u));
+      wt[c] = w[c];
+    }
+    if (bad) raise_flag(a.flags, BRS_FLAG_NONFINITE);
+    if constexpr (STORE != BRS_STORE_FP32 && HAD) warp_fwht<D>(wt, lane, a.hscale);
+  }
+
+  // ---- pass 2: write, o, requantize (batches of NRB rows)
+  float o1[C], o2[C];
+#pragma unroll
+  for (int c = 0; c < C; ++c) { o1[c] = 0.f; o2[c] = 0.f; }
+  // the next batch's rows are fetched while this batch is requantized
+  uint32_t pw[NRB], ps[(NB > 1) ? NRB : 1];
+  const uint8_t* prow = hin + col0;
+  const uint32_t* psrow = szin + col0 / BLOCK;
+  auto prefetch = [&]() {
+#pragma unroll
+    for (int r = 0; r < NRB; ++r) {
+      if constexpr (C == 4) pw[r] = __ldg((const uint32_t*)(prow + r * D));
+      else if constexpr (C == 2) pw[r] = __ldg((const uint16_t*)(prow + r * D));
+      else pw[r] = __ldg(prow + r * D);
+      if constexpr (NB > 1) ps[r] = __ldg(psrow + r * NB);
+    }
+    prow += NRB * D;
+    psrow += NRB * NB;
+  };
+  if (STORE != BRS_STORE_FP32 && nlo > 0) prefetch();
+  for (int i0 = 0; i0 < D; i0 += NRB) {
+    const bool int8_batch = (STORE != BRS_STORE_FP32) && (i0 < nlo);   // batches are tier-uniform
+    float x[NRB][C];
+#pragma unroll
+    for (int r = 0; r < NRB; ++r) {
+      const int i = i0 + r;
+      const RowScal rsc = sm.rs[i];
+      const float2 qv = sm.qq[i];
+      if (int8_batch) {
+        if constexpr (NB == 1) {
+          dequant_int8<C>(x[r], pw[r], rsc.sz.x, rsc.sz.y, rsc.sz.z, rsc.sz.w);
+        } else {
+          const float sv = f16_to_f32((uint16_t)(ps[r] & 0xffffu)), zv = f16_to_f32((uint16_t)(ps[r] >> 16));
+          dequant_int8<C>(x[r], pw[r], sv, sv, zv, zv);
+        }
+      } else {
+        load_row(i, x[r]);
+      }
+      v_scale<C>(x[r], rsc.ka.z, rsc.ka.w);
+      if (STORE == BRS_STORE_FP32 || i0 < nlo) {
+        v_fma_vec<C>(x[r], rsc.ka.x, rsc.ka.y, wt);
+        v_fma_s<C>(o1, qv.x, qv.y, x[r]);
+      } else {
+        v_fma_vec<C>(x[r], rsc.ka.x, rsc.ka.y, w);
+        v_fma_s<C>(o2, qv.x, qv.y, x[r]);
       }
     }
-    // lanes of this row group (every lane of a row group takes this path)
-    const uint32_t rmask = (LPR >= 32) ? 0xffffffffu : (((1u << LPR) - 1u) << (lane & ~(uint32_t)(LPR - 1)));
-    float v[V];
+    if (STORE != BRS_STORE_FP32 && i0 + NRB < nlo) prefetch();
+    if constexpr (STORE == BRS_STORE_FP32) {
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const float y0 = f2lo(x[r][0]), y1 = f2hi(x[r][0]), y2 = f2lo(x[r][1]), y3 = f2hi(x[r][1]);
-      v[2 * r] = fminf(fminf(y0, y1), fminf(y2, y3));
-      v[2 * r + 1] = fmaxf(fmaxf(y0, y1), fmaxf(y2, y3));
-    }
-    // reduce-scatter over the GL lanes of the block group: afterwards lane
-    // g (of its group) holds entries [g*VPL, (g+1)*VPL) reduced over the
-    // group (even entries minima, odd entries maxima)
-#pragma unroll
-    for (int m = GL / 2, len = V; m >= 1; m >>= 1, len >>= 1) {
-      const bool up = (lane & m) != 0;
-#pragma unroll
-      for (int i = 0; i < len / 2; ++i) {
-        const float lo = v[i], hi = v[i + len / 2];
-        const float other = __shfl_xor_sync(rmask, up ? lo : hi, m);
-        const float mine = up ? hi : lo;
-        if (len / 2 >= 2)
-          v[i] = (i & 1) ? fmaxf(mine, other) : fminf(mine, other);
-        else
-          v[i] = (lane & 1) ? fmaxf(mine, other) : fminf(mine, other);
+      for (int r = 0; r < NRB; ++r) {
+        float* dst = (float*)hout + (size_t)(i0 + r) * D + col0;
+        if constexpr (C == 4) *(float4*)dst = make_float4(x[r][0], x[r][1], x[r][2], x[r][3]);
+        else if constexpr (C == 2) *(float2*)dst = make_float2(x[r][0], x[r][1]);
+        else *dst = x[r][0];
       }
-    }
-    float mnv[RPL], mxv[RPL];
-    if constexpr (VPL >= 2) {
-#pragma unroll
-      for (int q = 0; q < RPL; ++q) { mnv[q] = v[2 * q]; mxv[q] = v[2 * q + 1]; }
+      continue;
     } else {
-      const float other = __shfl_xor_sync(rmask, v[0], 1);
-      mnv[0] = (lane & 1) ? other : v[0];
-      mxv[0] = (lane & 1) ? v[0] : other;
-    }
-    const int g = (lane % LPR) % GL;            // lane within its block group
-    const int blk = (lane % LPR) / GL;          // block index within the row
-    const int lr0 = (VPL >= 2) ? g * RPL : g / 2;
-    // a zero extreme takes the sign rule (-0 below +0): rare, warp-wide
-    bool zc = false;
+      if (!int8_batch) {
+        // protected rows: FP16, nearest
+        uint32_t ovf = 0;
 #pragma unroll
-    for (int q = 0; q < RPL; ++q) zc |= (mnv[q] == 0.0f) || (mxv[q] == 0.0f);
-    if (__any_sync(rmask, zc)) {
-      uint32_t nz = 0, pz = 0;
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const float y[4] = {f2lo(x[r][0]), f2hi(x[r][0]), f2lo(x[r][1]), f2hi(x[r][1])};
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          if (y[c] == 0.0f) {
-            if (signbit(y[c])) nz |= 1u << r; else pz |= 1u << r;
+        for (int r = 0; r < NRB; ++r) {
+          uint16_t* dst = f16out + (size_t)(i0 + r - nlo) * D + col0;
+          if constexpr (C == 4) {
+            const uint32_t lo = f16x2_of(x[r][0], x[r][1]), hi = f16x2_of(x[r][2], x[r][3]);
+            ovf |= f16x2_overflow(lo) | f16x2_overflow(hi);
+            *(uint2*)dst = make_uint2(lo, hi);
+          } else if constexpr (C == 2) {
+            const uint32_t lo = f16x2_of(x[r][0], x[r][1]);
+            ovf |= f16x2_overflow(lo);
+            *(uint32_t*)dst = lo;
+          } else {
+            const uint16_t hv = f32_to_f16(x[r][0]);
+            ovf |= f16_inf_or_nan(hv);
+            *dst = hv;
           }
+        }
+        if (ovf) raise_flag(a.flags, BRS_FLAG_OVERFLOW);
+        continue;
       }
+      // ---- INT8 batch: error-feedback target
+      if constexpr (MODE == BRS_ROUND_ERRFEEDBACK) {
 #pragma unroll
-      for (int m = 1; m < GL; m <<= 1) {
-        nz |= __shfl_xor_sync(rmask, nz, m);
-        pz |= __shfl_xor_sync(rmask, pz, m);
+        for (int r = 0; r < NRB; ++r) {
+          const uint16_t* e = auxb + (size_t)(i0 + r) * D + col0;
+          uint16_t ev[C];
+          if constexpr (C == 4) {
+            const uint2 q = *(const uint2*)e;
+            ev[0] = (uint16_t)(q.x & 0xffffu); ev[1] = (uint16_t)(q.x >> 16);
+            ev[2] = (uint16_t)(q.y & 0xffffu); ev[3] = (uint16_t)(q.y >> 16);
+          } else if constexpr (C == 2) {
+            const uint32_t q = *(const uint32_t*)e;
+            ev[0] = (uint16_t)(q & 0xffffu); ev[1] = (uint16_t)(q >> 16);
+          } else {
+            ev[0] = *e;
+          }
+#pragma unroll
+          for (int c = 0; c < C; ++c) x[r][c] = __fadd_rn(x[r][c], f16_to_f32(ev[c]));
+        }
       }
+      // ---- block extremes: local, then a reduce-scatter over the GL lanes
+      // of the block; entry 2r / 2r+1 is the min / max of batch row r
+      float v[V];
 #pragma unroll
-      for (int q = 0; q < RPL; ++q) {
-        const int lr = lr0 + q;
-        if (mnv[q] == 0.0f) mnv[q] = ((nz >> lr) & 1u) ? -0.0f : 0.0f;
-        if (mxv[q] == 0.0f) mxv[q] = ((pz >> lr) & 1u) ? 0.0f : -0.0f;
+      for (int r = 0; r < NRB; ++r) {
+        float mn = x[r][0], mx = x[r][0];
+#pragma unroll
+        for (int c = 1; c < C; ++c) { mn = fminf(mn, x[r][c]); mx = fmaxf(mx, x[r][c]); }
+        v[2 * r] = mn;
+        v[2 * r + 1] = mx;
       }
-    }
-    // grid of each (row, block): one division per row, spread over lanes.
-    // ok: the smallest and largest grid coordinates of the block (the same
-    // FP32 operations as the elements', which are monotone in y) round into
-    // [0, 255], so no code of the block needs the clip at the rails.
-    bool ok_all = true;
-    uint32_t* szout = (uint32_t*)(hout + (size_t)nlo * D + (size_t)a.k_hi * D * 2);
+      // halving stages (offsets GL/2 .. GL/HALV), then all-reduce stages
+      // (offsets below GL/HALV); afterwards lane g of the block group holds
+      // entries [j0, j0 + VPL) with j0 = (g / (GL/HALV)) * VPL
+      constexpr int VPL = V / HALV;
+      static_assert(VPL <= 2, "one row per lane after the reduce-scatter");
 #pragma unroll
-    for (int q = 0; q < RPL; ++q) {
-      const int i = row0 + lr0 + q;               // stored row
-      if ((VPL >= 2) || ((lane & 1) == 0)) {
-        if (!isfinite(mnv[q]) || !isfinite(mxv[q])) raise_flag(a.flags, BRS_FLAG_NONFINITE);
-        const uint16_t sh = f32_to_f16(__fdiv_rn(__fsub_rn(mxv[q], mnv[q]), 255.0f));
-        const uint16_t zh = f32_to_f16(mnv[q]);
+      for (int m = GL / 2, len = V; m >= 1; m >>= 1) {
+        if (len > VPL) {
+          const bool up = (lane & m) != 0;
+#pragma unroll
+          for (int e = 0; e < len / 2; ++e) {
+            const float lo = v[e], hi = v[e + len / 2];
+            const float other = __shfl_xor_sync(0xffffffffu, up ? lo : hi, m);
+            const float mine = up ? hi : lo;
+            // entry parity: e's own while the kept length stays even,
+            // else the lane bit that chose the half
+            const bool is_max = (len / 2 >= 2) ? (e & 1) : up;
+            v[e] = is_max ? fmaxf(mine, other) : fminf(mine, other);
+          }
+          len >>= 1;
+        } else {
+#pragma unroll
+          for (int e = 0; e < VPL; ++e) {
+            const float other = __shfl_xor_sync(0xffffffffu, v[e], m);
+            const bool is_max = (VPL >= 2) ? (e & 1) : ((lane & (GL / HALV)) != 0);
+            v[e] = is_max ? fmaxf(v[e], other) : fminf(v[e], other);
+          }
+        }
+      }
+      const int g = lane % GL, blk = col0 / BLOCK;
+      const int j0 = (g / (GL / HALV)) * VPL;          // first entry held by this lane
+      float mnv, mxv;
+      int prow;
+      bool param_lane;
+      if constexpr (VPL >= 2) {
+        mnv = v[0]; mxv = v[1];
+        prow = j0 / 2;
+        param_lane = (g % (GL / HALV)) == 0;
+      } else {
+        const int pbit = GL / HALV;                    // lane bit of the entry parity
+        const float other = __shfl_xor_sync(0xffffffffu, v[0], pbit);
+        const bool odd = (lane & pbit) != 0;
+        mnv = odd ? other : v[0];
+        mxv = odd ? v[0] : other;
+        prow = j0 / 2;
+        param_lane = (g % (2 * pbit)) == 0;
+      }
+      // a zero extreme takes the sign rule (-0 below +0): rare, warp-wide
+      const bool zc = param_lane && ((mnv == 0.0f) || (mxv == 0.0f));
+      if (__any_sync(0xffffffffu, zc)) {
+        uint32_t nz = 0, pz = 0;
+#pragma unroll
+        for (int r = 0; r < NRB; ++r)
+#pragma unroll
+          for (int c = 0; c < C; ++c)
+            if (x[r][c] == 0.0f) {
+              if (signbit(x[r][c])) nz |= 1u << r; else pz |= 1u << r;
+            }
+#pragma unroll
+        for (int m = 1; m < GL; m <<= 1) {
+          nz |= __shfl_xor_sync(0xffffffffu, nz, m);
+          pz |= __shfl_xor_sync(0xffffffffu, pz, m);
+        }
+        if (mnv == 0.0f) mnv = ((nz >> prow) & 1u) ? -0.0f : 0.0f;
+        if (mxv == 0.0f) mxv = ((pz >> prow) & 1u) ? 0.0f : -0.0f;
+      }
+      // the grid of each (row, block), one division per lane; ok = the
+      // block's extreme grid coordinates (the same monotone FP32 operations
+      // as its elements') round into [0, 255]: no clip needed
+      bool ok = true;
+      if (param_lane) {
+        const int i = i0 + prow;
+        if (!isfinite(mnv) || !isfinite(mxv)) raise_flag(a.flags, BRS_FLAG_NONFINITE);
+        const uint16_t sh = f32_to_f16(__fdiv_rn(__fsub_rn(mxv, mnv), 255.0f));
+        const uint16_t zh = f32_to_f16(mnv);
         if (f16_inf_or_nan(sh) || f16_inf_or_nan(zh)) raise_flag(a.flags, BRS_FLAG_OVERFLOW);
         const float s = f16_to_f32(sh), z = f16_to_f32(zh);
         const float rcp = (s == 0.0f) ? 0.0f : __frcp_rn(s);
-        const float tlo = __fmul_rn(__fsub_rn(mnv[q], z), rcp), thi = __fmul_rn(__fsub_rn(mxv[q], z), rcp);
-        const bool ok = (tlo >= -0.5f) && (thi < 255.5f);
-        ok_all &= ok;
-        QPrm pr;
-        pr.zz = f2dup(z); pr.rr = f2dup(rcp); pr.ss = f2dup(s); pr.ok = ok; pr.pad = 0;
-        sm.prm[i][blk] = pr;
+        const float tlo = __fmul_rn(__fsub_rn(mnv, z), rcp), thi = __fmul_rn(__fsub_rn(mxv, z), rcp);
+        ok = (tlo >= -0.5f) && (thi < 255.5f);
+        QPrm p;
+        p.z = z; p.rcp = rcp; p.s = s; p.pad = 0;
+        sm.prm[prow][blk] = p;
         szout[i * NB + blk] = (uint32_t)sh | ((uint32_t)zh << 16);
       }
-    }
-    const bool fast = (MODE != BRS_ROUND_STOCHASTIC) && __all_sync(rmask, ok_all);
-    __syncwarp();
-
-    // quantize and store: code = clamp(round((y - zero) * (1/scale)), 0, 255);
-    // when scale is 0 the factor 1/scale is 0 and every code is 0
-    const f2_t magic = f2dup(kRoundMagic);
+      const bool fast = (MODE != BRS_ROUND_STOCHASTIC) && __all_sync(0xffffffffu, ok);
+      __syncwarp();
+      // ---- codes: clamp(round((y - zero) * (1/scale)), 0, 255); a zero
+      // scale has 1/scale = 0, so every code of the block is 0
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const int i = row0 + r;
-      const QPrm& pr = sm.prm[i][col0 / BLOCK];
-      const f2_t t01 = f2mul(f2sub(x[r][0], pr.zz), pr.rr);
-      const f2_t t23 = f2mul(f2sub(x[r][1], pr.zz), pr.rr);
-      f2_t m01, m23;
-      if (fast) {
-        // nearest integer (ties to even): the low byte of (t + 1.5*2^23)
-        m01 = f2add(t01, magic);
-        m23 = f2add(t23, magic);
-      } else {
-        float c[4] = {f2lo(t01), f2hi(t01), f2lo(t23), f2hi(t23)};
-        if constexpr (MODE == BRS_ROUND_STOCHASTIC) {
-          const uint4 rnd = philox4x32_10(
-              make_uint4((uint32_t)(i * (D / 4) + cb), (uint32_t)a.step, (uint32_t)h, (uint32_t)b),
-              make_uint2((uint32_t)a.seed, (uint32_t)(a.seed >> 32)));
-          c[0] = sr_round(c[0], rnd.x >> 8);
-          c[1] = sr_round(c[1], rnd.y >> 8);
-          c[2] = sr_round(c[2], rnd.z >> 8);
-          c[3] = sr_round(c[3], rnd.w >> 8);
+      for (int r = 0; r < NRB; ++r) {
+        const int i = i0 + r;
+        const QPrm p = sm.prm[r][blk];
+        float tq[C];
+#pragma unroll
+        for (int c = 0; c < C; c += (C >= 2 ? 2 : 1)) {
+          if constexpr (C >= 2) {
+            float d0, d1;
+            sub2(d0, d1, x[r][c], x[r][c + 1], p.z, p.z);
+            mul2(tq[c], tq[c + 1], d0, d1, p.rcp, p.rcp);
+          } else {
+            tq[c] = __fmul_rn(__fsub_rn(x[r][c], p.z), p.rcp);
+          }
         }
+        if (!fast) {
+          if constexpr (MODE == BRS_ROUND_STOCHASTIC) {
+            const int e0 = i * D + col0;
+            const uint4 rnd = philox4x32_10(make_uint4((uint32_t)(e0 / 4), (uint32_t)a.step, (uint32_t)h, (uint32_t)b),
+                                            make_uint2((uint32_t)a.seed, (uint32_t)(a.seed >> 32)));
+            const uint32_t words[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
 #pragma unroll
-        for (int k = 0; k < 4; ++k) c[k] = fminf(fmaxf(c[k], 0.0f), 255.0f);
-        m01 = f2add(f2make(c[0], c[1]), magic);
-        m23 = f2add(f2make(c[2], c[3]), magic);
-      }
-      const uint32_t packed4 = __byte_perm(__byte_perm((uint32_t)m01, (uint32_t)(m01 >> 32), 0x0040u),
-                                           __byte_perm((uint32_t)m23, (uint32_t)(m23 >> 32), 0x0040u), 0x5410u);
-      *(uint32_t*)(hout + (size_t)i * D + col0) = packed4;
-      if constexpr (MODE == BRS_ROUND_ERRFEEDBACK) {
-        const f2_t q01 = f2fma(f2sub(m01, magic), pr.ss, pr.zz);   // stored value
-        const f2_t q23 = f2fma(f2sub(m23, magic), pr.ss, pr.zz);
-        const f2_t e01 = f2sub(x[r][0], q01), e23 = f2sub(x[r][1], q23);
-        const float s = f2lo(pr.ss);
-        float e[4] = {f2lo(e01), f2hi(e01), f2lo(e23), f2hi(e23)};
+            for (int c = 0; c < C; ++c) tq[c] = sr_round(tq[c], words[(e0 + c) & 3] >> 8);
+          }
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          if (e[k] > s) e[k] = s;
-          else if (e[k] < -s) e[k] = -s;
+          for (int c = 0; c < C; ++c) tq[c] = fminf(fmaxf(tq[c], 0.0f), 255.0f);
         }
-        *(uint2*)&auxb[(size_t)i * D + col0] = make_uint2(f16x2_of(e[0], e[1]), f16x2_of(e[2], e[3]));
+        // nearest integer (ties to even): the low byte of t + 1.5*2^23
+        float mq[C];
+#pragma unroll
+        for (int c = 0; c < C; c += (C >= 2 ? 2 : 1)) {
+          if constexpr (C >= 2) add2(mq[c], mq[c + 1], tq[c], tq[c + 1], kRoundMagic, kRoundMagic);
+          else mq[c] = __fadd_rn(tq[c], kRoundMagic);
+        }
+        uint8_t* dst = hout + (size_t)i * D + col0;
+        if constexpr (C == 4) {
+          *(uint32_t*)dst = __byte_perm(__byte_perm(__float_as_uint(mq[0]), __float_as_uint(mq[1]), 0x0040u),
+                                        __byte_perm(__float_as_uint(mq[2]), __float_as_uint(mq[3]), 0x0040u), 0x5410u);
+        } else if constexpr (C == 2) {
+          *(uint16_t*)dst = (uint16_t)__byte_perm(__float_as_uint(mq[0]), __float_as_uint(mq[1]), 0x0040u);
+        } else {
+          *dst = (uint8_t)magic_byte(mq[0]);
+        }
+        if constexpr (MODE == BRS_ROUND_ERRFEEDBACK) {
+          uint16_t ev[C];
+#pragma unroll
+          for (int c = 0; c < C; ++c) {
+            const float code = __fsub_rn(mq[c], kRoundMagic);          // exact
+            float e = __fsub_rn(x[r][c], __fmaf_rn(code, p.s, p.z));
+            if (e > p.s) e = p.s;
+            else if (e < -p.s) e = -p.s;
+            ev[c] = f32_to_f16(e);
+          }
+          uint16_t* ed = auxb + (size_t)i * D + col0;
+          if constexpr (C == 4) *(uint2*)ed = make_uint2((uint32_t)ev[0] | ((uint32_t)ev[1] << 16), (uint32_t)ev[2] | ((uint32_t)ev[3] << 16));
+          else if constexpr (C == 2) *(uint32_t*)ed = (uint32_t)ev[0] | ((uint32_t)ev[1] << 16);
+          else *ed = ev[0];
+        }
       }
+      __syncwarp();                                    // sm.prm reused by the next batch
     }
   }
+
+  // ---- o = O2 + T(O1)
+  if constexpr (STORE != BRS_STORE_FP32 && HAD) warp_fwht<D>(o1, lane, a.hscale);
+  float ov[C];
+  bool bad = false;
+#pragma unroll
+  for (int c = 0; c < C; ++c) {
+    ov[c] = (STORE == BRS_STORE_FP32) ? o1[c] : __fadd_rn(o2[c], o1[c]);
+    bad |= !isfinite(ov[c]);
+  }
+  if (bad) raise_flag(a.flags, BRS_FLAG_NONFINITE);
+  float* od = a.o + (size_t)head * D + col0;
+  if constexpr (C == 4) *(float4*)od = make_float4(ov[0], ov[1], ov[2], ov[3]);
+  else if constexpr (C == 2) *(float2*)od = make_float2(ov[0], ov[1]);
+  else *od = ov[0];
 }
 
 template <int D, int BLOCK, int MODE>
 static cudaError_t launch_dbm(const DecodeArgs& a, int store, bool had, cudaStream_t st) {
-  const dim3 grid(a.B * a.H), block(2 * D);
+  const int heads = a.B * a.H;
+  const dim3 grid((heads + kWarpsPerCta - 1) / kWarpsPerCta), block(32 * kWarpsPerCta);
   if (store == BRS_STORE_FP32)
-    decode_kernel<D, BRS_STORE_FP32, false, D, BRS_ROUND_NEAREST><<<grid, block, 0, st>>>(a);
+    decode_warp_kernel<D, BRS_STORE_FP32, false, D, BRS_ROUND_NEAREST><<<grid, block, 0, st>>>(a);
   else if (had)
-    decode_kernel<D, BRS_STORE_DAMP, true, BLOCK, MODE><<<grid, block, 0, st>>>(a);
+    decode_warp_kernel<D, BRS_STORE_DAMP, true, BLOCK, MODE><<<grid, block, 0, st>>>(a);
   else
-    decode_kernel<D, BRS_STORE_DAMP, false, BLOCK, MODE><<<grid, block, 0, st>>>(a);
+    decode_warp_kernel<D, BRS_STORE_DAMP, false, BLOCK, MODE><<<grid, block, 0, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -453,7 +627,8 @@ static cudaError_t launch_db(const DecodeArgs& a, int store, bool had, cudaStrea
 bool decode_supported(int d, int block, int k_hi) {
   const bool shape = (d == 128 && (block == 128 || block == 32)) || (d == 64 && block == 64) ||
                      (d == 32 && block == 32);
-  return shape && k_hi % (d / 8) == 0 && k_hi <= d / 4;
+  const int nrb = (d >= 64) ? 8 : 4;
+  return shape && k_hi % nrb == 0;
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, int d, int store, bool had, cudaStream_t st) {
