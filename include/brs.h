@@ -66,13 +66,16 @@
  *
  * Arithmetic (identical on every path that produces stored codes)
  *   The update runs in FP32 ([DAMP] Implementation): per token and head,
- *   S <- Diag(a) S; u = S^T k; w = beta (v - u); S <- S + k w^T; o = S^T q,
- *   each sum over key rows an fmaf chain over stored rows 0..d-1 from +0.
- *   The Hadamard is the unnormalised Sylvester butterfly (stages 1, 2, 4, ...)
- *   followed by one multiplication by the float nearest 1/sqrt(d).  With
- *   `hadamard` set the DAMP update is computed in the Hadamard basis: the
- *   FP16 rows and v are rotated in, o is rotated out, the INT8 rows are
- *   used as stored.
+ *   S <- Diag(a) S; u = S^T k; w = beta (v - u); S <- S + k w^T; o = S^T q.
+ *   FP32 storage: each sum over key rows is an fmaf chain over stored rows
+ *   0..d-1 from +0.  DAMP storage: each tier is updated in the basis it is
+ *   stored in (INT8 rows in the basis T = the Hadamard when `hadamard` is
+ *   set, else the identity; FP16 rows in the value basis):
+ *     u = U2 + T(U1), w = beta (v - u), INT8 rows S_i += k_i T(w),
+ *     FP16 rows S_i += k_i w, o = O2 + T(O1),
+ *   where U1/O1 (U2/O2) are fmaf chains over the INT8 (FP16) rows in stored
+ *   order from +0.  T is the unnormalised Sylvester butterfly (stages 1, 2,
+ *   4, ...) followed by one multiplication by the float nearest 1/sqrt(d).
  *   INT8 block: scale = fp16((max - min) / 255), zero = fp16(min),
  *   code = clamp(round((y - zero) * (1/scale)), 0, 255).  Rounding
  *   ([WB] Quantized GRU formulation; Chinese summary, error feedback and
