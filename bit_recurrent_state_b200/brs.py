@@ -24,7 +24,7 @@ STORES = {"fp32": STORE_FP32, "damp": STORE_DAMP, "varbit": STORE_VARBIT}
 
 # exported symbols declared in include/brs.h
 SYMBOLS = ["brs_state_bytes", "brs_state_pack", "brs_state_unpack", "brs_decode_step",
-           "brs_fetch_errors", "brs_last_error"]
+           "brs_decode_step_noalloc", "brs_fetch_errors", "brs_last_error"]
 
 
 class BrsError(RuntimeError):
@@ -78,6 +78,8 @@ def lib():
         L.brs_state_unpack.argtypes = [P, P, P, P, P, P]
         L.brs_decode_step.restype = S
         L.brs_decode_step.argtypes = [P, P, ct.c_int64] + [P] * 13
+        L.brs_decode_step_noalloc.restype = S
+        L.brs_decode_step_noalloc.argtypes = [P, P, ct.c_int64] + [P] * 12
         L.brs_fetch_errors.restype = S
         L.brs_fetch_errors.argtypes = [P, P, P]
         L.brs_last_error.restype = ct.c_char_p
@@ -137,6 +139,16 @@ def decode_step(layout, wb, step, packed_in, packed_out, aux, stats, workspace, 
                                  _ptr(packed_out), _ptr(aux), _ptr(stats), _ptr(workspace),
                                  _ptr(perm), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(decay),
                                  _ptr(o), _stream(stream)))
+
+
+def decode_step_noalloc(layout, wb, step, packed_in, packed_out, aux, stats, perm, q, k, v, beta,
+                        decay, o, stream=None):
+    """brs_decode_step without a workspace: the library's static scratch is
+    used instead (for callers that cannot allocate device memory)."""
+    _check(lib().brs_decode_step_noalloc(ct.byref(layout), ct.byref(wb), int(step), _ptr(packed_in),
+                                         _ptr(packed_out), _ptr(aux), _ptr(stats), _ptr(perm), _ptr(q),
+                                         _ptr(k), _ptr(v), _ptr(beta), _ptr(decay), _ptr(o),
+                                         _stream(stream)))
 
 
 def fetch_errors(workspace, stream=None) -> int:

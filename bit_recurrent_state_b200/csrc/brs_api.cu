@@ -72,6 +72,11 @@ brs_status cuda_fail(cudaError_t e, const char* what) {
 
 }  // namespace
 
+namespace brs {
+// lets other translation units of the library report through brs_last_error
+void set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+}  // namespace brs
+
 extern "C" {
 
 const char* brs_last_error(void) { return g_err; }

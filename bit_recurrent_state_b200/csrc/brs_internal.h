@@ -41,4 +41,6 @@ struct PackArgs {
 cudaError_t launch_pack(const PackArgs& a, cudaStream_t st);
 cudaError_t launch_unpack(const PackArgs& a, float* S_out, const void* packed, cudaStream_t st);
 
+void set_last_error(const char* msg);
+
 }  // namespace brs

@@ -184,6 +184,24 @@ brs_status brs_decode_step(const brs_layout* L, const brs_writeback* wb, int64_t
                            const uint16_t* k, const uint16_t* v, const float* beta,
                            const float* decay, float* o, void* stream);
 
+/* Allocation-free variant of brs_decode_step (the pages have no
+ * counterpart; it exists for callers that cannot allocate device memory,
+ * such as a host framework whose allocator owns the whole device or a
+ * serving loop with a fixed memory budget).  Same arguments and semantics
+ * as brs_decode_step without `workspace`: the scratch is a static device
+ * array of 4096 bytes inside the library, reserved on every device that
+ * loads it until the process exits.  Layouts whose workspace
+ * (brs_state_bytes) exceeds 4096 bytes are rejected with BRS_EINVAL.  The
+ * first call on a device looks the array's address up (cudaGetSymbolAddress)
+ * and should precede any stream capture.  All calls share the array, so
+ * calls that overlap on the GPU race; each call clears the flag word before
+ * its kernel, and device-raised flags are not reported by this entry. */
+brs_status brs_decode_step_noalloc(const brs_layout* L, const brs_writeback* wb, int64_t step,
+                                   const void* packed_in, void* packed_out, void* aux, void* stats,
+                                   const int16_t* perm, const uint16_t* q, const uint16_t* k,
+                                   const uint16_t* v, const float* beta, const float* decay,
+                                   float* o, void* stream);
+
 /* Reads and clears the device flag word of `workspace` (synchronises
  * `stream`).  Returns BRS_OK, or BRS_ENONFINITE / BRS_EOVERFLOW /
  * BRS_ETIMEOUT for the first flag set; *flags_out (optional) receives the
