@@ -24,7 +24,7 @@ STORES = {"fp32": STORE_FP32, "damp": STORE_DAMP, "varbit": STORE_VARBIT}
 
 # exported symbols declared in include/brs.h
 SYMBOLS = ["brs_state_bytes", "brs_state_pack", "brs_state_unpack", "brs_decode_step",
-           "brs_decode_step_noalloc", "brs_fetch_errors", "brs_last_error"]
+           "brs_decode_step_noalloc", "brs_allocate_bits", "brs_fetch_errors", "brs_last_error"]
 
 
 class BrsError(RuntimeError):
@@ -80,6 +80,9 @@ def lib():
         L.brs_decode_step.argtypes = [P, P, ct.c_int64] + [P] * 13
         L.brs_decode_step_noalloc.restype = S
         L.brs_decode_step_noalloc.argtypes = [P, P, ct.c_int64] + [P] * 12
+        L.brs_allocate_bits.restype = S
+        L.brs_allocate_bits.argtypes = [ct.c_int, ct.c_int, P, ct.c_double, ct.c_int, ct.c_int,
+                                        ct.c_uint32, P, P, P]
         L.brs_fetch_errors.restype = S
         L.brs_fetch_errors.argtypes = [P, P, P]
         L.brs_last_error.restype = ct.c_char_p
@@ -149,6 +152,14 @@ def decode_step_noalloc(layout, wb, step, packed_in, packed_out, aux, stats, per
                                          _ptr(packed_out), _ptr(aux), _ptr(stats), _ptr(perm), _ptr(q),
                                          _ptr(k), _ptr(v), _ptr(beta), _ptr(decay), _ptr(o),
                                          _stream(stream)))
+
+
+def allocate_bits(cost, rows_per_group, avg_bits, b_min, b_max, bits_out, offsets_out=None,
+                  offset_unit=1, stream=None):
+    """brs_allocate_bits on device f64 costs (torch tensor)."""
+    _check(lib().brs_allocate_bits(int(cost.numel()), int(rows_per_group), _ptr(cost), float(avg_bits),
+                                   int(b_min), int(b_max), int(offset_unit), _ptr(bits_out),
+                                   _ptr(offsets_out), _stream(stream)))
 
 
 def fetch_errors(workspace, stream=None) -> int:

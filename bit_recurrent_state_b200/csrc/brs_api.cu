@@ -92,12 +92,10 @@ size_t brs_state_bytes(const brs_layout* L, size_t* aux_bytes, size_t* stats_byt
     total = heads * damp_head_bytes(L);
     aux = heads * (d - (size_t)L->k_hi) * d * 2;
   } else {
-    const size_t rows = (size_t)L->H * d;
-    const size_t P = (size_t)((double)(d / 8) * L->avg_bits * (double)rows);
-    total = round256(P * L->B) + round256(rows * L->B * 2) + round256(rows * L->B) +
-            round256((rows + 1) * L->B * 4);
+    total = brs::varbit_sections(L->B, L->H, L->d, L->avg_bits).total;
     aux = heads * d * d * 2;
     stats = heads * d * 2 * sizeof(double);
+    ws = 256 + heads * d * sizeof(double);   // flag word, then one FP64 cost per row
   }
   if (aux_bytes) *aux_bytes = aux;
   if (stats_bytes) *stats_bytes = stats;
@@ -110,9 +108,22 @@ brs_status brs_state_pack(const brs_layout* L, const float* S, const int16_t* pe
                           const uint8_t* widths, void* packed, void* workspace, void* stream) {
   brs_status st = check_layout(L);
   if (st != BRS_OK) return st;
-  (void)widths;
-  if (L->storage == BRS_STORE_VARBIT) return fail(BRS_EUNSUPPORTED, "variable-width pack is not built yet");
   if (!S || !packed || !workspace) return fail(BRS_EINVAL, "S, packed and workspace are required");
+  if (L->storage == BRS_STORE_VARBIT) {
+    if (perm) return fail(BRS_EINVAL, "variable-width storage keeps rows in key-channel order (perm must be NULL)");
+    if (!widths && L->avg_bits != std::floor(L->avg_bits))
+      return fail(BRS_EINVAL, "uniform widths need an integer avg_bits");
+    if (!aligned16(S) || !aligned16(packed) || !aligned16(workspace))
+      return fail(BRS_EALIGN, "device pointers must be 16-byte aligned");
+    brs::VbPackArgs v{};
+    v.B = L->B; v.H = L->H; v.d = L->d; v.avg_bits = L->avg_bits;
+    v.sec = brs::varbit_sections(L->B, L->H, L->d, L->avg_bits);
+    v.S = S; v.widths = widths; v.packed = packed; v.flags = (uint32_t*)workspace;
+    cudaError_t e = brs::launch_varbit_pack(v, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "variable-width pack launch");
+    return ok();
+  }
+  (void)widths;
   if (!aligned16(S) || !aligned16(packed) || !aligned16(workspace) || (perm && !aligned16(perm)))
     return fail(BRS_EALIGN, "device pointers must be 16-byte aligned");
   brs::PackArgs a{};
@@ -129,8 +140,18 @@ brs_status brs_state_unpack(const brs_layout* L, const void* packed, const int16
                             float* S, void* workspace, void* stream) {
   brs_status st = check_layout(L);
   if (st != BRS_OK) return st;
-  if (L->storage == BRS_STORE_VARBIT) return fail(BRS_EUNSUPPORTED, "variable-width unpack is not built yet");
   if (!S || !packed) return fail(BRS_EINVAL, "S and packed are required");
+  if (L->storage == BRS_STORE_VARBIT) {
+    if (perm) return fail(BRS_EINVAL, "variable-width storage keeps rows in key-channel order (perm must be NULL)");
+    if (!aligned16(S) || !aligned16(packed)) return fail(BRS_EALIGN, "device pointers must be 16-byte aligned");
+    brs::VbPackArgs v{};
+    v.B = L->B; v.H = L->H; v.d = L->d; v.avg_bits = L->avg_bits;
+    v.sec = brs::varbit_sections(L->B, L->H, L->d, L->avg_bits);
+    v.flags = (uint32_t*)workspace;
+    cudaError_t e = brs::launch_varbit_unpack(v, packed, S, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "variable-width unpack launch");
+    return ok();
+  }
   if (!aligned16(S) || !aligned16(packed) || (perm && !aligned16(perm)))
     return fail(BRS_EALIGN, "device pointers must be 16-byte aligned");
   brs::PackArgs a{};
@@ -154,9 +175,32 @@ brs_status brs_decode_step(const brs_layout* L, const brs_writeback* wb, int64_t
   if (wb->C != 1) return fail(BRS_EUNSUPPORTED, "decode writes back every token (C = 1); got C = %d", wb->C);
   if (wb->mode < 0 || wb->mode > 2) return fail(BRS_EINVAL, "unknown rounding mode %d", wb->mode);
   if (step < 0) return fail(BRS_EINVAL, "step must be >= 0");
-  if (L->storage == BRS_STORE_VARBIT) return fail(BRS_EUNSUPPORTED, "variable-width decode is not built yet");
   if (!packed_in || !packed_out || !workspace || !q || !k || !v || !beta || !decay || !o)
     return fail(BRS_EINVAL, "a required pointer is NULL");
+  if (L->storage == BRS_STORE_VARBIT) {
+    if (L->d != 128) return fail(BRS_EUNSUPPORTED, "variable-width decode is built for d = 128");
+    if (packed_in == packed_out) return fail(BRS_EINVAL, "variable-width decode needs packed_out != packed_in");
+    if (perm) return fail(BRS_EINVAL, "variable-width storage keeps rows in key-channel order (perm must be NULL)");
+    if (!stats) return fail(BRS_EINVAL, "variable-width decode needs the statistics buffer");
+    if (wb->mode == BRS_ROUND_ERRFEEDBACK && !aux) return fail(BRS_EINVAL, "error feedback needs the residual buffer");
+    const void* ptrs[] = {packed_in, packed_out, aux, stats, workspace, q, k, v, beta, decay, o};
+    for (const void* p : ptrs)
+      if (p && !aligned16(p)) return fail(BRS_EALIGN, "device pointers must be 16-byte aligned");
+    brs::VbArgs a{};
+    a.B = L->B; a.H = L->H; a.Hk = L->H_k; a.decay_per_key = L->decay_per_key; a.mode = wb->mode;
+    a.first = step == 0; a.C = wb->C; a.b_min = L->b_min; a.b_max = L->b_max;
+    a.budget_scope = L->budget_scope; a.seed = wb->seed; a.step = step;
+    double lam = 1.0;
+    for (int c = 0; c < wb->C; ++c) lam *= (1.0 - 2.0 / 65.0);   // EMA weight of a C-token chunk, span 64
+    a.lambda = lam; a.avg_bits = L->avg_bits;
+    a.sec = brs::varbit_sections(L->B, L->H, L->d, L->avg_bits);
+    a.packed_in = packed_in; a.packed_out = packed_out; a.aux = aux; a.stats = (double*)stats;
+    a.cost = (double*)((uint8_t*)workspace + 256);
+    a.q = q; a.k = k; a.v = v; a.beta = beta; a.decay = decay; a.o = o; a.flags = (uint32_t*)workspace;
+    cudaError_t e = brs::launch_varbit_decode(a, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "variable-width decode launch");
+    return ok();
+  }
   if (L->storage == BRS_STORE_DAMP && !brs::decode_supported(L->d, L->block, L->k_hi))
     return fail(BRS_EUNSUPPORTED,
                 "decode kernel built for (d, block) in {(128,128), (128,32), (64,64), (32,32)} and "
@@ -178,6 +222,28 @@ brs_status brs_decode_step(const brs_layout* L, const brs_writeback* wb, int64_t
   const bool had = L->storage == BRS_STORE_DAMP && L->hadamard;
   cudaError_t e = brs::launch_decode(a, L->d, L->storage, had, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return ok();
+}
+
+brs_status brs_allocate_bits(int n_rows, int rows_per_group, const double* cost, double avg_bits,
+                             int b_min, int b_max, uint32_t offset_unit, uint8_t* bits_out,
+                             uint32_t* offsets_out, void* stream) {
+  if (n_rows <= 0 || rows_per_group <= 0 || n_rows % rows_per_group)
+    return fail(BRS_EINVAL, "n_rows must be a positive multiple of rows_per_group");
+  if (rows_per_group > brs::allocate_max_rows())
+    return fail(BRS_EUNSUPPORTED, "groups of up to %d rows", brs::allocate_max_rows());
+  if (b_min < 1 || b_max > 16 || b_min > b_max) return fail(BRS_EINVAL, "need 1 <= b_min <= b_max <= 16");
+  const double tgt = avg_bits * (double)rows_per_group;
+  if (tgt != std::floor(tgt) || tgt < (double)b_min * rows_per_group || tgt > (double)b_max * rows_per_group)
+    return fail(BRS_EINVAL, "avg_bits * rows_per_group must be an integer inside [b_min, b_max] * rows");
+  if (!cost || !bits_out) return fail(BRS_EINVAL, "cost and bits_out are required");
+  if (!aligned16(cost) || (offsets_out && !aligned16(offsets_out)))
+    return fail(BRS_EALIGN, "device pointers must be 16-byte aligned");
+  brs::AllocArgs a{};
+  a.groups = n_rows / rows_per_group; a.rows_per_group = rows_per_group; a.b_min = b_min; a.b_max = b_max;
+  a.avg_bits = avg_bits; a.offset_unit = offset_unit; a.cost = cost; a.bits = bits_out; a.offsets = offsets_out;
+  cudaError_t e = brs::launch_allocate(a, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "allocate launch");
   return ok();
 }
 

@@ -149,3 +149,28 @@ __device__ __forceinline__ void row_fwht4(float (&x)[4], int cb, float scale) {
 }
 
 }  // namespace brs
+
+namespace brs {
+
+// Variable-width row quantizer ("Low-Bit Recurrent States in Hybrid Language
+// Models", Levels and storage): levels {-n..n} * step, n = 2^(w-1) - 1,
+// step = fp16(f * R / n) with R the row's absolute maximum and f fitted over
+// the 16 values f_m = (5+m)/20 by squared error (nearest rounding on the
+// target, an fmaf chain over the row's values in order, ties to the smaller
+// f).  Candidate m's step and reciprocal; reciprocal 0 when the step is 0.
+__device__ __forceinline__ void varbit_candidate(int m, float R, int n, float& step, float& inv,
+                                                 uint16_t& bits, bool& valid) {
+  const float f = __fdiv_rn((float)(5 + m), 20.0f);
+  bits = f32_to_f16(__fdiv_rn(__fmul_rn(f, R), (float)n));
+  step = f16_to_f32(bits);
+  valid = isfinite(step);
+  inv = (step == 0.0f || !valid) ? 0.0f : __frcp_rn(step);
+}
+
+// nearest level index of y on a grid with reciprocal step inv, clipped
+__device__ __forceinline__ float varbit_nearest(float y, float inv, float fn) {
+  const float q = rintf(__fmul_rn(y, inv));
+  return fminf(fmaxf(q, -fn), fn);
+}
+
+}  // namespace brs

@@ -41,6 +41,55 @@ struct PackArgs {
 cudaError_t launch_pack(const PackArgs& a, cudaStream_t st);
 cudaError_t launch_unpack(const PackArgs& a, float* S_out, const void* packed, cudaStream_t st);
 
+// Sections of a variable-width stored state (see the header's layout).
+struct VbSections {
+  size_t payload_per_seq, off_scale, off_width, off_offsets, total;
+};
+VbSections varbit_sections(int B, int H, int d, double avg_bits);
+
+struct VbPackArgs {
+  int B, H, d;
+  double avg_bits;
+  VbSections sec;
+  const float* S;                // [B][H][d][d]
+  const uint8_t* widths;         // [B][H*d] or null (avg_bits everywhere)
+  void* packed;
+  uint32_t* flags;
+};
+cudaError_t launch_varbit_pack(const VbPackArgs& a, cudaStream_t st);
+cudaError_t launch_varbit_unpack(const VbPackArgs& a, const void* packed, float* S, cudaStream_t st);
+
+struct VbArgs {
+  int B, H, Hk, decay_per_key, mode, first, C, b_min, b_max, budget_scope;
+  uint64_t seed;
+  int64_t step;
+  double lambda, avg_bits;
+  VbSections sec;
+  const void* packed_in;
+  void* packed_out;
+  void* aux;
+  double* stats;
+  double* cost;                  // workspace: one FP64 cost per row
+  const uint16_t *q, *k, *v;
+  const float *beta, *decay;
+  float* o;
+  uint32_t* flags;
+};
+cudaError_t launch_varbit_decode(const VbArgs& a, cudaStream_t st);
+cudaError_t launch_varbit_offsets(const VbArgs& a, cudaStream_t st);
+
+struct AllocArgs {
+  int groups, rows_per_group, b_min, b_max;
+  double avg_bits;
+  uint32_t offset_unit;
+  const double* cost;
+  uint8_t* bits;
+  uint32_t* offsets;
+};
+
+cudaError_t launch_allocate(const AllocArgs& a, cudaStream_t st);
+int allocate_max_rows();
+
 void set_last_error(const char* msg);
 
 }  // namespace brs

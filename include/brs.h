@@ -184,6 +184,25 @@ brs_status brs_decode_step(const brs_layout* L, const brs_writeback* wb, int64_t
                            const uint16_t* k, const uint16_t* v, const float* beta,
                            const float* decay, float* o, void* stream);
 
+/* Decay-aware width allocation ([LB] State bit allocation; [LBX] Worked
+ * example).  For each of n_rows / rows_per_group groups of rows (a layer's
+ * H*d rows, or one head's d rows), in FP64: b*_i = avg + log2(c_i/GM)/2
+ * with GM the geometric mean over the rows with c_i > 0; rounded to
+ * nearest (ties to even) and clipped to [b_min, b_max] (b_min when
+ * c_i = 0; round(avg) for every row when all c_i are 0); then bits are
+ * moved one at a time, while over budget from the row whose cost
+ * 3 c_i 4^(-b_i) is smallest, while under budget to the row whose gain
+ * 3/4 c_i 4^(-b_i) is largest, ties to the lower row, until the group sums
+ * to avg * rows_per_group.
+ *   cost: device f64 [n_rows]; bits_out: device u8 [n_rows];
+ *   offsets_out (optional): device u32 [groups][rows_per_group + 1], the
+ *   exclusive prefix sums of the widths times offset_unit.
+ * rows_per_group <= 8192; avg * rows_per_group must be an integer in
+ * [b_min, b_max] * rows_per_group (BRS_EINVAL). */
+brs_status brs_allocate_bits(int n_rows, int rows_per_group, const double* cost, double avg_bits,
+                             int b_min, int b_max, uint32_t offset_unit, uint8_t* bits_out,
+                             uint32_t* offsets_out, void* stream);
+
 /* Allocation-free variant of brs_decode_step (the pages have no
  * counterpart; it exists for callers that cannot allocate device memory,
  * such as a host framework whose allocator owns the whole device or a

@@ -920,6 +920,16 @@ int orc_state_pack(const orc_layout* L, const float* S, const int16_t* perm,
     uint8_t* bits = (uint8_t*)malloc((size_t)rows);
     float* seq = (float*)malloc(sizeof(float) * (size_t)rows * d);
     for (int r = 0; r < rows; ++r) bits[r] = widths ? widths[r] : (uint8_t)nearbyint(L->avg_bits);
+    /* every sequence must fill exactly its payload: widths summing to avg_bits * H * d */
+    for (int b = 0; b < L->B; ++b) {
+      long sum = 0;
+      for (int r = 0; r < rows; ++r) sum += widths ? widths[(size_t)b * rows + r] : bits[r];
+      if ((double)sum != L->avg_bits * (double)rows) {
+        free(bits);
+        free(tmp);
+        return ORC_EINVAL;
+      }
+    }
     for (int b = 0; b < L->B; ++b) {
       memcpy(seq, S + (size_t)b * rows * d, sizeof(float) * (size_t)rows * d);
       flags |= varbit_store_seq(L, NULL, 0, b, seq, widths ? widths + (size_t)b * rows : bits,

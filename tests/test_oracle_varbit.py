@@ -90,3 +90,14 @@ def test_varbit_head_scope_budget(orc):
     _, _, wd, _ = varbit_sections(packed, B, H, d, 3.0)
     for h in range(H):
         assert int(wd[0, h * d:(h + 1) * d].astype(int).sum()) == 3 * d
+
+
+def test_varbit_pack_rejects_widths_off_budget(orc):
+    cfg = orc.Config(B=1, H=1, d=32, storage=orc.STORE_VARBIT, hadamard=0, avg_bits=4.0)
+    S = np.zeros((1, 1, 32, 32), np.float32)
+    w = np.full(32, 4, np.uint8)
+    _, fl = orc.state_pack(cfg, S, None, w)
+    assert fl == 0
+    w[0] = 8
+    _, fl = orc.state_pack(cfg, S, None, w)
+    assert fl == orc.EINVAL
