@@ -51,13 +51,16 @@ def algorithmic_bytes(w) -> dict:
     """Bytes one decode launch must move: the stored state read and written
     once, the token's inputs read, o written."""
     from bit_recurrent_state_b200 import brs
-    n, aux, _, _ = brs.state_bytes(brs.layout_of(w))
+    n, aux, stats, _ = brs.state_bytes(brs.layout_of(w))
     heads = w.B * w.H
     inputs = (2 * w.B * w.hk * w.d * 2 + heads * w.d * 2 + heads * 4 +
-              (heads * w.d * 4 if w.decay_per_key else heads * 4) + w.H * w.d * 2)
+              (heads * w.d * 4 if w.decay_per_key else heads * 4) +
+              (w.H * w.d * 2 if w.storage != "varbit" else 0))
     out = heads * w.d * 4
     ef = 2 * aux if w.mode == "errfeedback" else 0
-    return dict(state=2 * n, inputs=inputs, output=out, aux=ef, total=2 * n + inputs + out + ef)
+    st = 2 * stats
+    return dict(state=2 * n, inputs=inputs, output=out, aux=ef, stats=st,
+                total=2 * n + inputs + out + ef + st)
 
 
 def peaks():
@@ -137,14 +140,16 @@ def _oracle_cfg(w):
     from oracle import oracle as O
     st = {"fp32": O.STORE_FP32, "damp": O.STORE_DAMP, "varbit": O.STORE_VARBIT}[w.storage]
     return O.Config(B=w.B, H=w.H, Hk=w.hk, d=w.d, storage=st, k_hi=w.k_hi, block=w.block,
-                    hadamard=w.hadamard, decay_per_key=w.decay_per_key,
+                    hadamard=w.hadamard, decay_per_key=w.decay_per_key, avg_bits=w.avg_bits,
+                    b_min=w.b_min, b_max=w.b_max,
                     domain=O.DOMAIN_MIXED if w.storage == "damp" else O.DOMAIN_CANONICAL)
 
 
 class OracleRunner:
     """The oracle, as it stands, over a bounded sample of the workload: the
-    first `units` heads for `ntok` consecutive tokens per call, split over
-    the host's cores (heads are independent)."""
+    first `units` units (heads, or whole sequences for variable-width
+    storage, whose width budget spans a sequence) for `ntok` consecutive
+    tokens per call, split over the host's cores (units are independent)."""
 
     def __init__(self, w):
         from bit_recurrent_state_b200 import synth
@@ -155,6 +160,11 @@ class OracleRunner:
         self.cores = os.cpu_count() or 1
         self.t = 0
         self.cache = {}
+        self.varbit = w.storage == "varbit"
+        self.units_total = w.B if self.varbit else w.B * w.H
+        self.heads_per_unit = w.H if self.varbit else 1
+        self.mode = {"nearest": O.ROUND_NEAREST, "stochastic": O.ROUND_STOCHASTIC,
+                     "errfeedback": O.ROUND_ERRFEEDBACK}[w.mode]
 
     def inputs(self, ntok):
         key = (self.t, ntok)
@@ -163,34 +173,35 @@ class OracleRunner:
         return self.cache[key]
 
     def run(self, units, ntok):
+        """Returns (seconds, threads used, token*heads processed)."""
         inp = self.inputs(ntok)
         t0 = time.perf_counter()
-        _, fl, used = self.O.run_parallel(self.cfg, 0, self.w.seed, 1, self.t, inp, self.packed,
-                                          aux=self.aux, stats=self.stats, units=(0, units),
-                                          threads=self.cores)
+        _, fl, used = self.O.run_parallel(self.cfg, self.mode, self.w.seed, 1, self.t, inp,
+                                          self.packed, aux=self.aux, stats=self.stats,
+                                          units=(0, units), threads=self.cores)
         dt = time.perf_counter() - t0
         self.t += ntok
-        return dt, used
+        return dt, used, units * self.heads_per_unit * ntok
 
     def rate(self):
-        """unit-tokens per second, from a short calibration run."""
-        units = min(self.w.B * self.w.H, 4 * self.cores)
-        dt, _ = self.run(units, 2)
-        return units * 2 / max(dt, 1e-6)
+        """token*heads per second, from a short calibration run."""
+        units = max(1, min(self.units_total, 4 * self.cores // self.heads_per_unit))
+        dt, _, th = self.run(units, 1)
+        return th / max(dt, 1e-6)
 
 
 def cpu_oracle_sample(w, target_s: float = 12.0):
     """cpu_baseline: the oracle on host cores, about target_s seconds of work
-    on the workload's heads (all of them when that fits, else a prefix)."""
+    on the workload's units (all of them when that fits, else a prefix)."""
     R = OracleRunner(w)
     r = R.rate()
-    total = w.B * w.H
-    want = r * target_s
-    ntok = int(max(1, min(64, want // total)))
-    units = int(max(1, min(total, want // ntok)))
-    dt, used = R.run(units, ntok)
-    return {"value": units * ntok / dt, "unit": UNIT, "cores": used, "kind": "oracle",
-            "sample": f"{units} of {total} heads x {ntok} tokens of {w.name} "
+    want = r * target_s / R.heads_per_unit            # unit-tokens in the budget
+    ntok = int(max(1, min(64, want // R.units_total)))
+    units = int(max(1, min(R.units_total, want // ntok)))
+    dt, used, th = R.run(units, ntok)
+    what = "sequences" if R.varbit else "heads"
+    return {"value": th / dt, "unit": UNIT, "cores": used, "kind": "oracle",
+            "sample": f"{units} of {R.units_total} {what} x {ntok} tokens of {w.name} "
                       f"({dt:.1f} s wall on {used} threads)"}
 
 
@@ -201,21 +212,23 @@ def run_reference(args, w):
     R = OracleRunner(w)
     total = w.B * w.H
     per_step_s = max(0.2, min(4.0, args.ref_budget / (args.warmup + args.steps)))
-    units = int(max(1, min(total, R.rate() * per_step_s)))
+    units = int(max(1, min(R.units_total, R.rate() * per_step_s / R.heads_per_unit)))
     vals, used = [], 1
     for i in range(args.warmup + args.steps):
-        dt, used = R.run(units, 1)
+        dt, used, th = R.run(units, 1)
         if i >= args.warmup:
-            vals.append(units / dt)
+            vals.append(th / dt)
     value = statistics.median(vals)
+    what = "sequences" if R.varbit else "heads"
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total / value, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "H": w.H, "d": w.d},
+            "config": {"workload": w.name if w.mode == "nearest" else f"{w.name}_{w.mode}",
+                       "B": w.B, "H": w.H, "d": w.d},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
-                             "sample": f"each step: {units} of {total} heads x 1 token of "
-                                       f"{w.name} on {used} threads"},
+                             "sample": f"each step: {units} of {R.units_total} {what} x 1 token "
+                                       f"of {w.name} on {used} threads"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -243,11 +256,15 @@ def run_ours(args, w):
     wb = brs.writeback_of(wr)
     rng = np.random.default_rng(wr.seed)
     perm = np.stack([rng.permutation(w.d) for _ in range(w.H)]).astype(np.int16)
-    layers, inputs, host_inputs = [], [], []
+    varbit = w.storage == "varbit"
+    if varbit:
+        perm = None                    # variable-width rows stay in key-channel order
+    layers, spares, inputs, host_inputs = [], [], [], []
     for l in range(NLAYERS):
         st = LayerState(L, device=dev, perm=perm)
         st.zero()
         layers.append(st)
+        spares.append(torch.empty_like(st.packed) if varbit else None)
         inp = synth.token_inputs(wr.with_(seed=wr.seed + 17 * l), 0)
         host = {k: torch.from_numpy(v.view(np.int16) if v.dtype == np.uint16 else v).pin_memory()
                 for k, v in inp.items()}
@@ -257,9 +274,15 @@ def run_ours(args, w):
     o_host = torch.zeros_like(o, device="cpu").pin_memory()
 
     def step(i):
-        st = layers[i % NLAYERS]
-        x = inputs[i % NLAYERS]
-        st.step(wb, i, x["q"], x["k"], x["v"], x["beta"], x["decay"], o)
+        l = i % NLAYERS
+        st = layers[l]
+        x = inputs[l]
+        if varbit:
+            # variable-width states change their row offsets: write to the other buffer
+            spares[l] = st.step(wb, i, x["q"], x["k"], x["v"], x["beta"], x["decay"], o,
+                                packed_out=spares[l])
+        else:
+            st.step(wb, i, x["q"], x["k"], x["v"], x["beta"], x["decay"], o)
 
     for i in range(args.warmup):
         step(i)
@@ -318,7 +341,8 @@ def run_ours(args, w):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "H_k": w.hk, "d": w.d,
+        "config": {"workload": w.name if w.mode == "nearest" else f"{w.name}_{w.mode}",
+                   "B": w.B, "H": w.H, "H_k": w.hk, "d": w.d,
                    "storage": w.storage, "k_hi": w.k_hi, "block": w.block, "mode": w.mode,
                    "per_rank_batch": w.B, "parallelism": f"dp{world}",
                    "l2": f"{NLAYERS} rotating layer states of {ab['state'] // 2 / 1e6:.1f} MB "
@@ -330,7 +354,7 @@ def run_ours(args, w):
                      "traffic": traffic,
                      "kernel": "brs::decode_kernel", "state_gbs": ab["state"] / (ms_step * 1e-3) / 1e9},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * (3 if varbit else 1),
         "device_flags": flags,
     }
     if rank == 0:
@@ -350,6 +374,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="kda_decode")
+    ap.add_argument("--mode", default=None, help="write-back rounding: nearest | stochastic | errfeedback")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-budget", type=float, default=120.0,
                     help="seconds of oracle work for the whole --impl reference run")
@@ -358,6 +383,8 @@ def main():
         args.warmup = 3
     from bit_recurrent_state_b200 import synth
     w = synth.WORKLOADS[args.workload]
+    if args.mode:
+        w = w.with_(mode=args.mode)
     if args.impl == "reference":
         run_reference(args, w)
     else:

@@ -66,6 +66,8 @@ WORKLOADS = {
     "kda_decode": Workload("kda_decode", B=64, H=32, d=128, T=1024, k_hi=16, block=128, seed=1),
     "gdn_decode": Workload("gdn_decode", B=256, H=32, Hk=16, d=128, T=512, k_hi=0, block=128,
                            decay_per_key=0, seed=2),
+    "gdn_decode_fp32": Workload("gdn_decode_fp32", B=256, H=32, Hk=16, d=128, T=512, storage="fp32",
+                                hadamard=0, decay_per_key=0, seed=2),
     "varbit_decode": Workload("varbit_decode", B=128, H=32, d=128, T=1024, storage="varbit",
                               hadamard=0, avg_bits=4.0, b_min=2, b_max=8, seed=3),
     "kda_prefill": Workload("kda_prefill", B=8, H=32, d=128, T=8192, k_hi=16, block=128, C=64,
