@@ -24,7 +24,8 @@ STORES = {"fp32": STORE_FP32, "damp": STORE_DAMP, "varbit": STORE_VARBIT}
 
 # exported symbols declared in include/brs.h
 SYMBOLS = ["brs_state_bytes", "brs_state_pack", "brs_state_unpack", "brs_decode_step",
-           "brs_decode_step_noalloc", "brs_allocate_bits", "brs_fetch_errors", "brs_last_error"]
+           "brs_decode_step_noalloc", "brs_chunk_prefill", "brs_allocate_bits", "brs_fetch_errors",
+           "brs_last_error"]
 
 
 class BrsError(RuntimeError):
@@ -80,6 +81,8 @@ def lib():
         L.brs_decode_step.argtypes = [P, P, ct.c_int64] + [P] * 13
         L.brs_decode_step_noalloc.restype = S
         L.brs_decode_step_noalloc.argtypes = [P, P, ct.c_int64] + [P] * 12
+        L.brs_chunk_prefill.restype = S
+        L.brs_chunk_prefill.argtypes = [P, P, ct.c_int64, ct.c_int] + [P] * 12
         L.brs_allocate_bits.restype = S
         L.brs_allocate_bits.argtypes = [ct.c_int, ct.c_int, P, ct.c_double, ct.c_int, ct.c_int,
                                         ct.c_uint32, P, P, P]
@@ -152,6 +155,14 @@ def decode_step_noalloc(layout, wb, step, packed_in, packed_out, aux, stats, per
                                          _ptr(packed_out), _ptr(aux), _ptr(stats), _ptr(perm), _ptr(q),
                                          _ptr(k), _ptr(v), _ptr(beta), _ptr(decay), _ptr(o),
                                          _stream(stream)))
+
+
+def chunk_prefill(layout, wb, step0, T, packed, aux, workspace, perm, q, k, v, beta, decay, o,
+                  state_dump=None, stream=None):
+    """brs_chunk_prefill: T tokens per sequence, write-back every wb.C tokens."""
+    _check(lib().brs_chunk_prefill(ct.byref(layout), ct.byref(wb), int(step0), int(T), _ptr(packed),
+                                   _ptr(aux), _ptr(workspace), _ptr(perm), _ptr(q), _ptr(k), _ptr(v),
+                                   _ptr(beta), _ptr(decay), _ptr(o), _ptr(state_dump), _stream(stream)))
 
 
 def allocate_bits(cost, rows_per_group, avg_bits, b_min, b_max, bits_out, offsets_out=None,

@@ -225,6 +225,37 @@ brs_status brs_decode_step(const brs_layout* L, const brs_writeback* wb, int64_t
   return ok();
 }
 
+brs_status brs_chunk_prefill(const brs_layout* L, const brs_writeback* wb, int64_t step0, int T,
+                             void* packed, void* aux, void* workspace, const int16_t* perm,
+                             const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                             const float* beta, const float* decay, float* o, float* state_dump,
+                             void* stream) {
+  brs_status st = check_layout(L);
+  if (st != BRS_OK) return st;
+  if (!wb) return fail(BRS_EINVAL, "writeback is NULL");
+  if (L->storage != BRS_STORE_DAMP) return fail(BRS_EUNSUPPORTED, "chunked prefill is built for DAMP storage");
+  if (!brs::prefill_supported(L->d, L->block, L->k_hi, wb->C))
+    return fail(BRS_EUNSUPPORTED, "chunked prefill is built for d = 128, C = 64, block 128 or 32");
+  if (wb->mode < 0 || wb->mode > 2) return fail(BRS_EINVAL, "unknown rounding mode %d", wb->mode);
+  if (T <= 0 || T % wb->C || step0 < 0 || step0 % wb->C)
+    return fail(BRS_EINVAL, "T and step0 must be multiples of C (T = %d, C = %d)", T, wb->C);
+  if (!packed || !workspace || !q || !k || !v || !beta || !decay || !o)
+    return fail(BRS_EINVAL, "a required pointer is NULL");
+  if (wb->mode == BRS_ROUND_ERRFEEDBACK && !aux) return fail(BRS_EINVAL, "error feedback needs the residual buffer");
+  const void* ptrs[] = {packed, aux, workspace, perm, q, k, v, beta, decay, o, state_dump};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(BRS_EALIGN, "device pointers must be 16-byte aligned");
+  brs::PrefillArgs a{};
+  a.B = L->B; a.H = L->H; a.Hk = L->H_k; a.T = T; a.k_hi = L->k_hi; a.block = L->block;
+  a.decay_per_key = L->decay_per_key; a.mode = wb->mode; a.seed = wb->seed; a.step0 = step0;
+  a.head_bytes = head_bytes(L); a.hscale = hadamard_scale(L->d);
+  a.packed = packed; a.aux = aux; a.perm = perm; a.q = q; a.k = k; a.v = v; a.beta = beta;
+  a.decay = decay; a.o = o; a.sdump = state_dump; a.flags = (uint32_t*)workspace;
+  cudaError_t e = brs::launch_prefill(a, L->hadamard != 0, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+  return ok();
+}
+
 brs_status brs_allocate_bits(int n_rows, int rows_per_group, const double* cost, double avg_bits,
                              int b_min, int b_max, uint32_t offset_unit, uint8_t* bits_out,
                              uint32_t* offsets_out, void* stream) {

@@ -78,6 +78,24 @@ struct VbArgs {
 cudaError_t launch_varbit_decode(const VbArgs& a, cudaStream_t st);
 cudaError_t launch_varbit_offsets(const VbArgs& a, cudaStream_t st);
 
+struct PrefillArgs {
+  int B, H, Hk, T, k_hi, block, decay_per_key, mode;
+  uint64_t seed;
+  int64_t step0;
+  size_t head_bytes;
+  float hscale;
+  void* packed;                  // updated in place
+  void* aux;
+  const int16_t* perm;
+  const uint16_t *q, *k, *v;     // [B][T][Hk|H][d]
+  const float *beta, *decay;     // [B][T][H], [B][T][H][d] or [B][T][H]
+  float* o;                      // [B][T][H][d]
+  float* sdump;                  // optional [B][H][d][d]
+  uint32_t* flags;
+};
+cudaError_t launch_prefill(const PrefillArgs& a, bool had, cudaStream_t st);
+bool prefill_supported(int d, int block, int k_hi, int C);
+
 struct AllocArgs {
   int groups, rows_per_group, b_min, b_max;
   double avg_bits;

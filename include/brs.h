@@ -184,6 +184,32 @@ brs_status brs_decode_step(const brs_layout* L, const brs_writeback* wb, int64_t
                            const uint16_t* k, const uint16_t* v, const float* beta,
                            const float* decay, float* o, void* stream);
 
+/* Chunked prefill with deferred write-back ([LB] Accumulated readout error:
+ * write-back once per prefill chunk; [LB] Protocol).  Tokens
+ * [step0, step0 + T) of every (sequence, head) with write-back after every
+ * chunk of C tokens: the chunk's C delta-rule steps are evaluated together
+ * (WY form: A = strictly-lower(diag(beta) K~ K^T), (I + A) W =
+ * diag(beta) (V - K~ S0), O = Q~ S0 + lower(Q~ K^T) W,
+ * S_C = diag(Gamma_C) (S0 + K^T W), with Gamma the cumulative decay, K~ =
+ * K Gamma, K^ = K / Gamma, Q~ = Q Gamma) in FP32, then the state is
+ * requantized (value basis -> Hadamard -> INT8 blocks; FP16 rows) with the
+ * write-back rounding of `wb` at the chunk's last token.  DAMP storage,
+ * d = 128, C = 64, block 128 or 32.
+ *   packed: stored state, updated in place.  aux: residuals (error
+ *     feedback).  workspace: flag word (as brs_decode_step).
+ *   q, k [B][T][H_k][d] bf16; v [B][T][H][d] bf16; beta [B][T][H] f32;
+ *     decay [B][T][H][d] (KDA) or [B][T][H] (GDN) f32; o [B][T][H][d] f32.
+ *   state_dump (optional): [B][H][d][d] f32, the state just before the last
+ *     write-back of the call (stored row order, value basis).
+ * Results agree with the token-by-token recurrence within FP32 rounding of
+ * the reordered sums; the stored codes are the documented quantizer applied
+ * to state_dump. */
+brs_status brs_chunk_prefill(const brs_layout* L, const brs_writeback* wb, int64_t step0, int T,
+                             void* packed, void* aux, void* workspace, const int16_t* perm,
+                             const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                             const float* beta, const float* decay, float* o, float* state_dump,
+                             void* stream);
+
 /* Decay-aware width allocation ([LB] State bit allocation; [LBX] Worked
  * example).  For each of n_rows / rows_per_group groups of rows (a layer's
  * H*d rows, or one head's d rows), in FP64: b*_i = avg + log2(c_i/GM)/2

@@ -650,7 +650,8 @@ static void gather_token(const orc_layout* L, const orc_inputs* in, int t, int b
 
 static int run_head_unit(const orc_layout* L, const orc_writeback* wb, int64_t step0, int T,
                          int b, int h, const uint8_t* pin, uint8_t* pout, uint16_t* aux,
-                         const int16_t* perm, const orc_inputs* in, float* t_dump) {
+                         const int16_t* perm, const orc_inputs* in, float* t_dump,
+                         float* s_dump) {
   int d = L->d, flags = 0;
   size_t unit = (size_t)b * L->H + h;
   float* S = (float*)malloc(sizeof(float) * (size_t)d * d);
@@ -678,6 +679,7 @@ static int run_head_unit(const orc_layout* L, const orc_writeback* wb, int64_t s
     }
     memcpy(in->o + (((size_t)t * L->B + b) * L->H + h) * d, oo, sizeof(float) * (size_t)d);
     if ((step + 1) % wb->C == 0) {
+      if (s_dump) memcpy(s_dump + unit * (size_t)d * d, S, sizeof(float) * (size_t)d * d);
       /* write-back: quantize, then continue from the dequantized state
        * ([LB] Protocol: each write-back is quantized and dequantized before
        * reuse; no unquantized residual is retained) */
@@ -888,7 +890,7 @@ static int layout_ok(const orc_layout* L) {
 int orc_run(const orc_layout* L, const orc_writeback* wb, int64_t step0, int T, int u0, int u1,
             const void* packed_in, void* packed_out, void* aux, double* stats,
             const int16_t* perm, const uint16_t* q, const uint16_t* k, const uint16_t* v,
-            const float* beta, const float* decay, float* o, float* t_dump) {
+            const float* beta, const float* decay, float* o, float* t_dump, float* s_dump) {
   if (!layout_ok(L) || wb->C <= 0 || step0 % wb->C || T % wb->C) return ORC_EINVAL;
   orc_inputs in = {q, k, v, beta, decay, o};
   int flags = 0;
@@ -899,7 +901,7 @@ int orc_run(const orc_layout* L, const orc_writeback* wb, int64_t step0, int T, 
   } else {
     for (int u = u0; u < u1; ++u)
       flags |= run_head_unit(L, wb, step0, T, u / L->H, u % L->H, (const uint8_t*)packed_in,
-                             (uint8_t*)packed_out, (uint16_t*)aux, perm, &in, t_dump);
+                             (uint8_t*)packed_out, (uint16_t*)aux, perm, &in, t_dump, s_dump);
   }
   return flags;
 }

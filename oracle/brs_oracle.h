@@ -101,13 +101,16 @@ int orc_state_unpack(const orc_layout* L, const void* packed, const int16_t* per
  * a = exp(-s).  o [T][B][H][d].  packed_in may equal packed_out.  aux: FP16
  * error-feedback residuals, stats: FP64 EMA statistics (VARBIT).
  * t_dump (optional): pre-rounding grid coordinate of every stored code of
- * the LAST write-back, laid out like the codes.  Write-back happens after
+ * the LAST write-back, laid out like the codes.  s_dump (optional,
+ * FP32/DAMP storage): the FP32 state just before the LAST write-back,
+ * [B][H][d][d] in stored row order, in the working basis of the mode.
+ * Write-back happens after
  * every token whose global index t satisfies (t + 1) % C == 0; step0 and T
  * must be multiples of C.  Returns ORC_* flags. */
 int orc_run(const orc_layout* L, const orc_writeback* wb, int64_t step0, int T, int u0, int u1,
             const void* packed_in, void* packed_out, void* aux, double* stats,
             const int16_t* perm, const uint16_t* q, const uint16_t* k, const uint16_t* v,
-            const float* beta, const float* decay, float* o, float* t_dump);
+            const float* beta, const float* decay, float* o, float* t_dump, float* s_dump);
 
 /* Protected-row selection by the DAMP risk score on a calibration run.
  * Inputs as orc_run for Bc sequences and T tokens (FP32 recurrence from a

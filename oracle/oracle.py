@@ -98,7 +98,7 @@ def lib():
             L.orc_state_unpack.argtypes = [P, P, P, P]
             L.orc_run.restype = ct.c_int
             L.orc_run.argtypes = [P, P, ct.c_int64, ct.c_int, ct.c_int, ct.c_int, P, P, P, P, P,
-                                  P, P, P, P, P, P, P]
+                                  P, P, P, P, P, P, P, P]
             L.orc_calibrate.restype = ct.c_int
             L.orc_calibrate.argtypes = [P, ct.c_int, ct.c_int, ct.c_int, ct.c_double, P, P, P, P,
                                         P, P, P]
@@ -250,7 +250,7 @@ def new_state(cfg: Config):
 
 
 def run(cfg: Config, wb_mode: int, seed: int, C: int, step0: int, inputs: dict, packed, aux=None,
-        stats=None, perm=None, units=None, dump_t=False):
+        stats=None, perm=None, units=None, dump_t=False, dump_s=False):
     """Run T tokens (T = inputs['q'].shape[0]) over the given units.
 
     ``packed``/``aux``/``stats`` are updated in place.  Returns (o, flags,
@@ -268,11 +268,14 @@ def run(cfg: Config, wb_mode: int, seed: int, C: int, step0: int, inputs: dict, 
     nunits = cfg.B if cfg.storage == STORE_VARBIT else cfg.B * cfg.H
     u0, u1 = (0, nunits) if units is None else units
     t = np.zeros(cfg.B * cfg.H * cfg.d * cfg.d, np.float32) if dump_t else None
+    sd = np.zeros((cfg.B, cfg.H, cfg.d, cfg.d), np.float32) if dump_s else None
     assert packed.flags["C_CONTIGUOUS"]
     perm = _c(perm, np.int16)
     fl = lib().orc_run(ct.byref(L), ct.byref(wb), step0, T, u0, u1, _p(packed), _p(packed),
                        _p(aux), _p(stats), _p(perm), _p(q), _p(k), _p(v), _p(beta), _p(decay),
-                       _p(o), _p(t))
+                       _p(o), _p(t), _p(sd))
+    if dump_s:
+        return o, fl, t, sd
     return o, fl, t
 
 
@@ -299,7 +302,8 @@ def run_parallel(cfg: Config, wb_mode: int, seed: int, C: int, step0: int, input
     def work(i):
         return lib().orc_run(ct.byref(L), ct.byref(wb), step0, T, int(bounds[i]),
                              int(bounds[i + 1]), _p(packed), _p(packed), _p(aux), _p(stats),
-                             _p(perm), _p(q), _p(k), _p(v), _p(beta), _p(decay), _p(o), None)
+                             _p(perm), _p(q), _p(k), _p(v), _p(beta), _p(decay), _p(o), None,
+                             None)
 
     with ThreadPoolExecutor(nthr) as ex:
         flags = list(ex.map(work, range(nthr)))

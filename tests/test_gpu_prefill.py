@@ -1,0 +1,98 @@
+"""GPU parity of the chunked prefill (WY form, write-back once per 64-token
+chunk) against the oracle's token-by-token recurrence, teacher-forced per
+chunk: both start every chunk from the same stored state.  Outputs and the
+pre-write-back state within 2e-3 x RMS; the stored codes equal the oracle
+quantizer applied to the GPU's own pre-write-back state (replay)."""
+import numpy as np
+import pytest
+
+from bit_recurrent_state_b200 import synth
+from oracle import oracle as O
+from parity import MODE, random_perm
+
+pytestmark = pytest.mark.gpu
+
+
+def _tok_major(inp):
+    """[B][T][...] -> [T][B][...] for the oracle."""
+    return {k: np.ascontiguousarray(np.swapaxes(v, 0, 1)) for k, v in inp.items()}
+
+
+def _seq_major(w, t0, T):
+    """Inputs of tokens [t0, t0+T) laid out [B][T][...] for the prefill call."""
+    r = synth.run_inputs(w, t0, T)
+    return {k: np.ascontiguousarray(np.swapaxes(v, 0, 1)) for k, v in r.items()}
+
+
+def _dev(a):
+    import torch
+    a = np.ascontiguousarray(a)
+    return torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).cuda()
+
+
+def _run_chunks(w, nchunks, units=None, mode="nearest"):
+    import torch
+    from bit_recurrent_state_b200 import brs
+    from bit_recurrent_state_b200.state import LayerState
+    perm = random_perm(w, seed=11)
+    cfg = O.Config(B=w.B, H=w.H, Hk=w.hk, d=w.d, storage=O.STORE_DAMP, k_hi=w.k_hi, block=w.block,
+                   hadamard=w.hadamard, decay_per_key=w.decay_per_key, domain=O.DOMAIN_CANONICAL)
+    L, wb = brs.layout_of(w), brs.writeback_of(w, C=64, mode=brs.MODES[mode])
+    rng = np.random.default_rng(5)
+    S0 = (rng.standard_normal((w.B, w.H, w.d, w.d)) * 0.05).astype(np.float32)
+    packed_o, _ = O.state_pack(cfg, S0, perm)
+    _, aux_o, _ = O.new_state(cfg)
+    st = LayerState(L, perm=perm)
+    hb = packed_o.size // (w.B * w.H)
+    sel = np.arange(w.B * w.H) if units is None else np.arange(*units)
+    for c in range(nchunks):
+        t0 = 64 * c
+        inp = _seq_major(w, t0, 64)
+        st.packed.copy_(torch.from_numpy(packed_o))
+        st.aux.copy_(torch.from_numpy(np.pad(aux_o.view(np.uint8), (0, st.aux.numel() - aux_o.nbytes))))
+        o = torch.zeros((w.B, 64, w.H, w.d), device="cuda")
+        dump = torch.zeros((w.B, w.H, w.d, w.d), device="cuda")
+        d = {k: _dev(v) for k, v in inp.items()}
+        brs.chunk_prefill(L, wb, t0, 64, st.packed, st.aux, st.workspace, st.perm, d["q"], d["k"], d["v"],
+                          d["beta"], d["decay"], o, dump)
+        assert st.errors() == 0
+        og = o.cpu().numpy()
+        sg = dump.cpu().numpy()
+        pg = st.packed.cpu().numpy()
+        oo, fl, _, so = O.run(cfg, MODE[mode], w.seed, 64, t0, _tok_major(inp), packed_o, aux=aux_o,
+                              perm=perm, units=units, dump_s=True)
+        assert fl == 0
+        # outputs and pre-write-back state, over the compared heads
+        og_u = np.swapaxes(og, 1, 2).reshape(w.B * w.H, 64, w.d)[sel]
+        oo_u = np.swapaxes(oo, 0, 1).swapaxes(1, 2).reshape(w.B * w.H, 64, w.d)[sel]
+        rms_o = np.sqrt(np.mean(oo_u.astype(np.float64) ** 2))
+        assert np.max(np.abs(og_u - oo_u)) <= 2e-3 * rms_o, (c, np.max(np.abs(og_u - oo_u)) / rms_o)
+        sg_u = sg.reshape(w.B * w.H, w.d, w.d)[sel]
+        so_u = so.reshape(w.B * w.H, w.d, w.d)[sel]
+        rms_s = np.sqrt(np.mean(so_u.astype(np.float64) ** 2))
+        assert np.max(np.abs(sg_u - so_u)) <= 2e-3 * rms_s, (c, np.max(np.abs(sg_u - so_u)) / rms_s)
+        if mode == "nearest":
+            # replay: the documented quantizer on the GPU's own state gives its codes
+            rp, fl = O.state_pack(cfg, sg, None)
+            assert fl == 0
+            np.testing.assert_array_equal(pg.reshape(w.B * w.H, hb)[sel], rp.reshape(w.B * w.H, hb)[sel])
+
+
+@pytest.mark.parametrize("kw,mode", [
+    (dict(B=2, H=3, d=128, k_hi=16, block=128), "nearest"),
+    (dict(B=1, H=2, d=128, k_hi=16, block=32), "nearest"),
+    (dict(B=2, H=4, Hk=2, d=128, k_hi=0, block=128, decay_per_key=0), "nearest"),
+    (dict(B=1, H=2, d=128, k_hi=16, block=128), "errfeedback"),
+    (dict(B=1, H=2, d=128, k_hi=16, block=128), "stochastic"),
+])
+def test_prefill_teacher_forced(kw, mode):
+    w = synth.Workload("pf", T=192, C=64, seed=60, **kw)
+    _run_chunks(w, 3, mode=mode)
+
+
+def test_prefill_full_size_sampled():
+    """The measured prefill configuration (B=8, H=32, d=128, 16 FP16 + 112
+    INT8-Hadamard rows, block 128), in the benchmark's launch configuration,
+    for the first two chunks; the oracle runs 6 of the 256 heads."""
+    w = synth.WORKLOADS["kda_prefill"]
+    _run_chunks(w, 2, units=(97, 103))
