@@ -2,7 +2,8 @@
 GB/s against the measured B200 copy bandwidth).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload kda_decode|gdn_decode|kda_tiny]
+                    [--workload kda_decode|gdn_decode|gdn_decode_fp32|varbit_decode|
+                                kda_prefill|kda_tiny]
 
 A step is one decode token for every (sequence, head) of the workload: one
 launch of the fused decode kernel (dequantize, decay, delta-rule write, read
@@ -11,6 +12,9 @@ layer states (each with its own seeded inputs), so a step never finds its
 state in L2 (8 x 38.7 MB > 126 MB).  With N GPUs (torchrun) every rank runs
 its own batch of the same size (weak scaling, no collective on the data
 path); the time is the maximum over ranks.
+
+With `--workload kda_prefill` a step is instead one chunked-prefill launch
+over the whole batch (B x T tokens x H heads, write-back every 64 tokens).
 
 `--impl reference` times the plain CPU oracle on this host's cores on the
 same workload and metric (bounded samples), which is the only other place
@@ -145,6 +149,18 @@ def _oracle_cfg(w):
                     domain=O.DOMAIN_MIXED if w.storage == "damp" else O.DOMAIN_CANONICAL)
 
 
+def workload_config(w, world: int) -> dict:
+    """The `config` object of both arms: the workload by name and sizes."""
+    cfg = {"workload": w.name if w.mode == "nearest" else f"{w.name}_{w.mode}",
+           "B": w.B, "H": w.H, "H_k": w.hk, "d": w.d, "storage": w.storage, "k_hi": w.k_hi,
+           "block": w.block, "mode": w.mode, "per_rank_batch": w.B, "parallelism": f"dp{world}"}
+    if w.C > 1:
+        cfg.update(T=w.T, C=w.C)
+    if w.storage == "varbit":
+        cfg.update(avg_bits=w.avg_bits, b_min=w.b_min, b_max=w.b_max)
+    return cfg
+
+
 class OracleRunner:
     """The oracle, as it stands, over a bounded sample of the workload: the
     first `units` units (heads, or whole sequences for variable-width
@@ -176,7 +192,7 @@ class OracleRunner:
         """Returns (seconds, threads used, token*heads processed)."""
         inp = self.inputs(ntok)
         t0 = time.perf_counter()
-        _, fl, used = self.O.run_parallel(self.cfg, self.mode, self.w.seed, 1, self.t, inp,
+        _, fl, used = self.O.run_parallel(self.cfg, self.mode, self.w.seed, self.w.C, self.t, inp,
                                           self.packed, aux=self.aux, stats=self.stats,
                                           units=(0, units), threads=self.cores)
         dt = time.perf_counter() - t0
@@ -196,7 +212,7 @@ def cpu_oracle_sample(w, target_s: float = 12.0):
     R = OracleRunner(w)
     r = R.rate()
     want = r * target_s / R.heads_per_unit            # unit-tokens in the budget
-    ntok = int(max(1, min(64, want // R.units_total)))
+    ntok = w.C if w.C > 1 else int(max(1, min(64, want // R.units_total)))
     units = int(max(1, min(R.units_total, want // ntok)))
     dt, used, th = R.run(units, ntok)
     what = "sequences" if R.varbit else "heads"
@@ -210,27 +226,133 @@ def run_reference(args, w):
     if rank != 0:
         return
     R = OracleRunner(w)
-    total = w.B * w.H
+    total = w.B * w.H * (w.T if w.C > 1 else 1)      # token*heads of one step of our arm
     per_step_s = max(0.2, min(4.0, args.ref_budget / (args.warmup + args.steps)))
-    units = int(max(1, min(R.units_total, R.rate() * per_step_s / R.heads_per_unit)))
+    units = int(max(1, min(R.units_total, R.rate() * per_step_s / (R.heads_per_unit * w.C))))
     vals, used = [], 1
     for i in range(args.warmup + args.steps):
-        dt, used, th = R.run(units, 1)
+        dt, used, th = R.run(units, w.C)
         if i >= args.warmup:
             vals.append(th / dt)
     value = statistics.median(vals)
     what = "sequences" if R.varbit else "heads"
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+    metric = METRIC.replace("decode", "chunked prefill") if w.C > 1 else METRIC
+    line = {"impl": "reference", "metric": metric, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total / value, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": w.name if w.mode == "nearest" else f"{w.name}_{w.mode}",
-                       "B": w.B, "H": w.H, "d": w.d},
+            "config": workload_config(w, args.gpus),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
-                             "sample": f"each step: {units} of {R.units_total} {what} x 1 token "
-                                       f"of {w.name} on {used} threads"},
+                             "sample": f"each step: {units} of {R.units_total} {what} x {w.C} "
+                                       f"token(s) of {w.name} on {used} threads"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def run_prefill(args, w):
+    """A step = the chunked prefill of the whole batch (B sequences x T
+    tokens x H heads, write-back every 64 tokens); value = tokens*heads/s."""
+    import torch
+    import torch.distributed as dist
+
+    from bit_recurrent_state_b200 import brs, synth
+    from bit_recurrent_state_b200.state import LayerState
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    wr = w.with_(seed=w.seed + 1000 * rank)
+    L, wb = brs.layout_of(wr), brs.writeback_of(wr)
+    rng = np.random.default_rng(wr.seed)
+    perm = np.stack([rng.permutation(w.d) for _ in range(w.H)]).astype(np.int16)
+    st = LayerState(L, device=dev, perm=perm)
+    st.zero()
+    inp = synth.run_inputs(wr, 0, w.T)
+    host = {k: torch.from_numpy(np.ascontiguousarray(np.swapaxes(v, 0, 1)).view(np.int16)
+                                if v.dtype == np.uint16 else np.ascontiguousarray(np.swapaxes(v, 0, 1)))
+            for k, v in inp.items()}
+    x = {k: v.to(dev) for k, v in host.items()}
+    o = torch.empty((w.B, w.T, w.H, w.d), dtype=torch.float32, device=dev)
+
+    def step(i):
+        brs.chunk_prefill(L, wb, i * w.T, w.T, st.packed, st.aux, st.workspace, st.perm, x["q"], x["k"],
+                          x["v"], x["beta"], x["decay"], o)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier()
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        ev1.record(stream)
+        barrier()
+    ms = ev0.elapsed_time(ev1)
+    t = torch.tensor([ms], device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_step = float(t.item()) / args.steps
+    flags = st.errors()
+    # end to end: inputs copied from pinned host memory and o read back every step
+    pinned = {k: v.pin_memory() for k, v in host.items()}
+    o_host = torch.empty_like(o, device="cpu").pin_memory()
+    barrier()
+    ev0.record(stream)
+    for i in range(args.steps):
+        for k, v in pinned.items():
+            x[k].copy_(v, non_blocking=True)
+        step(i)
+        o_host.copy_(o, non_blocking=True)
+    ev1.record(stream)
+    barrier()
+    t = torch.tensor([ev0.elapsed_time(ev1)], device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_e2e = float(t.item()) / args.steps
+    units = w.B * w.H * w.T * world
+    n, aux, _, _ = brs.state_bytes(L)
+    chunks = w.T // 64
+    inputs_b = sum(v.numel() * v.element_size() for v in host.values())
+    out_b = o.numel() * o.element_size()
+    total = 2 * n * chunks + inputs_b + out_b
+    peak, src = peaks()
+    achieved = total / (ms_step * 1e-3) / 1e9
+    line = {
+        "metric": METRIC.replace("decode", "chunked prefill"), "value": units / (ms_step * 1e-3),
+        "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": dict(workload_config(w, world),
+                       l2=f"inputs {inputs_b / 1e9:.1f} GB per step (> 126 MB L2)"),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": src, "algorithmic_bytes_per_launch": total,
+                     "traffic": None, "kernel": "brs::prefill_kernel"},
+        "e2e": {"value": units / (ms_e2e * 1e-3), "unit": UNIT, "h2d_bytes_per_step": inputs_b,
+                "d2h_bytes_per_step": out_b},
+        "gpu_launches": args.steps, "device_flags": flags,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_oracle_sample(w)
+    if rank == 0:
+        line["clocks"] = clk.summary()
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
 
 
 def run_ours(args, w):
@@ -341,12 +463,9 @@ def run_ours(args, w):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": w.name if w.mode == "nearest" else f"{w.name}_{w.mode}",
-                   "B": w.B, "H": w.H, "H_k": w.hk, "d": w.d,
-                   "storage": w.storage, "k_hi": w.k_hi, "block": w.block, "mode": w.mode,
-                   "per_rank_batch": w.B, "parallelism": f"dp{world}",
-                   "l2": f"{NLAYERS} rotating layer states of {ab['state'] // 2 / 1e6:.1f} MB "
-                         f"(> 126 MB L2)"},
+        "config": dict(workload_config(w, world),
+                       l2=f"{NLAYERS} rotating layer states of {ab['state'] // 2 / 1e6:.1f} MB "
+                          f"(> 126 MB L2)"),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": src + " (MEASURED_PEAKS.json hbm_gbs)"
                      if src == "measured" else "fallback 6.65 TB/s",
@@ -390,7 +509,10 @@ def main():
     else:
         from bit_recurrent_state_b200 import brs
         brs.lib()          # the in-tree CUDA library; fails loudly when it is missing
-        run_ours(args, w)
+        if w.name == "kda_prefill":
+            run_prefill(args, w)
+        else:
+            run_ours(args, w)
 
 
 if __name__ == "__main__":
