@@ -212,7 +212,10 @@ def cpu_oracle_sample(w, target_s: float = 12.0):
     R = OracleRunner(w)
     r = R.rate()
     want = r * target_s / R.heads_per_unit            # unit-tokens in the budget
-    ntok = w.C if w.C > 1 else int(max(1, min(64, want // R.units_total)))
+    if w.C > 1:                      # whole write-back chunks, up to the sequence length
+        ntok = w.C * int(max(1, min(w.T // w.C, want // (R.units_total * w.C))))
+    else:
+        ntok = int(max(1, min(64, want // R.units_total)))
     units = int(max(1, min(R.units_total, want // ntok)))
     dt, used, th = R.run(units, ntok)
     what = "sequences" if R.varbit else "heads"

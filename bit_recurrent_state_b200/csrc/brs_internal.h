@@ -27,6 +27,9 @@ struct DecodeArgs {
 
 cudaError_t launch_decode(const DecodeArgs& a, int d, int store, bool had, cudaStream_t st);
 bool decode_supported(int d, int block, int k_hi);
+// d = 128 DAMP decode with bulk-copy staging of the stored rows
+bool decode_tma_supported(int d, int store, int block, int k_hi);
+cudaError_t launch_decode_tma(const DecodeArgs& a, bool had, cudaStream_t st);
 
 struct PackArgs {
   int B, H, d, storage, k_hi, block, hadamard;

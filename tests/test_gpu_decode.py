@@ -74,6 +74,10 @@ def test_kda_tiny_full_trajectory():
 @pytest.mark.parametrize("name,kw", [
     ("kda128_ragged", dict(B=3, H=5, d=128, k_hi=16, block=128)),
     ("kda128_block32", dict(B=2, H=3, d=128, k_hi=16, block=32)),
+    ("kda128_khi8", dict(B=2, H=3, d=128, k_hi=8, block=128)),
+    ("kda128_khi24_nohad_b32", dict(B=2, H=2, d=128, k_hi=24, block=32, hadamard=0)),
+    ("kda128_all_fp16", dict(B=1, H=2, d=128, k_hi=128, block=128)),
+    ("kda128_b32_sr", dict(B=2, H=2, d=128, k_hi=16, block=32, mode="stochastic")),
     ("kda64", dict(B=2, H=3, d=64, k_hi=8, block=64)),
     ("kda32_nohad", dict(B=2, H=2, d=32, k_hi=4, block=32, hadamard=0)),
     ("gdn128", dict(B=3, H=4, Hk=2, d=128, k_hi=0, block=128, decay_per_key=0)),
