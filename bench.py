@@ -40,7 +40,8 @@ METRIC = "state-update tokens·heads/s and state HBM GB/s (% of B200 peak), deco
 UNIT = "tokens·heads/s"
 FALLBACK_HBM_GBS = 6650.0
 NLAYERS = 8
-KERNEL_SOURCES = ["bit_recurrent_state_b200/csrc/decode.cu", "bit_recurrent_state_b200/csrc/brs_device.cuh"]
+KERNEL_SOURCES = ["bit_recurrent_state_b200/csrc/decode.cu", "bit_recurrent_state_b200/csrc/decode_tma.cu",
+                  "bit_recurrent_state_b200/csrc/brs_device.cuh"]
 
 
 def kernel_hash() -> str:
@@ -65,6 +66,15 @@ def algorithmic_bytes(w) -> dict:
     st = 2 * stats
     return dict(state=2 * n, inputs=inputs, output=out, aux=ef, stats=st,
                 total=2 * n + inputs + out + ef + st)
+
+
+def kernel_name(w) -> str:
+    """The kernel a decode step of workload w launches (the dominant one)."""
+    if w.storage == "varbit":
+        return "brs::varbit_kernel (update pass + fit pass) and brs::allocate_kernel"
+    if w.storage == "damp" and w.d == 128:
+        return "brs::decode_tma_kernel"
+    return "brs::decode_warp_kernel"
 
 
 def peaks():
@@ -108,6 +118,15 @@ class ClockSampler:
                 stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+            return self
+        # nvidia-smi takes a moment to start: the timed region begins once
+        # the first sample is written (at most 10 s)
+        t0 = time.time()
+        while time.time() - t0 < 10.0 and self.proc.poll() is None:
+            self.f.flush()
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.05)
         return self
 
     def __exit__(self, *exc):
@@ -230,7 +249,7 @@ def run_reference(args, w):
         return
     R = OracleRunner(w)
     total = w.B * w.H * (w.T if w.C > 1 else 1)      # token*heads of one step of our arm
-    per_step_s = max(0.2, min(4.0, args.ref_budget / (args.warmup + args.steps)))
+    per_step_s = max(0.005, min(4.0, args.ref_budget / (args.warmup + args.steps)))
     units = int(max(1, min(R.units_total, R.rate() * per_step_s / (R.heads_per_unit * w.C))))
     vals, used = [], 1
     for i in range(args.warmup + args.steps):
@@ -474,7 +493,7 @@ def run_ours(args, w):
                      if src == "measured" else "fallback 6.65 TB/s",
                      "algorithmic_bytes_per_launch": ab["total"],
                      "traffic": traffic,
-                     "kernel": "brs::decode_kernel", "state_gbs": ab["state"] / (ms_step * 1e-3) / 1e9},
+                     "kernel": kernel_name(w), "state_gbs": ab["state"] / (ms_step * 1e-3) / 1e9},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps * (3 if varbit else 1),
         "device_flags": flags,
@@ -492,7 +511,8 @@ def run_ours(args, w):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: 20000 decode steps, 5 prefill steps)")
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="kda_decode")
@@ -507,6 +527,10 @@ def main():
     w = synth.WORKLOADS[args.workload]
     if args.mode:
         w = w.with_(mode=args.mode)
+    if args.steps is None:
+        # long enough a timed region for the clock sampler (>= ~0.5 s on
+        # the GPU); the oracle arm times a few bounded samples
+        args.steps = 10 if args.impl == "reference" else (5 if w.C > 1 else 20000)
     if args.impl == "reference":
         run_reference(args, w)
     else:

@@ -33,7 +33,7 @@ namespace brs {
 namespace {
 
 constexpr int kD = 128, kC = 4, kNrb = 8;
-constexpr int kTmaWarps = 2;                       // heads per CTA
+constexpr int kTmaWarps = 1;                       // heads per CTA (one: finest spread over the SMs)
 constexpr int kSlot = 2048;                        // bytes per ring stage
 constexpr int kStages = 3;
 constexpr int kRows8 = kSlot / kD;                 // INT8 rows per slot
@@ -191,7 +191,7 @@ __device__ __forceinline__ void fwht128(float (&x)[4], int lane, float scale) {
 }
 
 template <bool HAD, int BLOCK, int MODE>
-__global__ void __launch_bounds__(32 * kTmaWarps, 7) decode_tma_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(32 * kTmaWarps, 16) decode_tma_kernel(const DecodeArgs a) {
   constexpr int NB = kD / BLOCK;                   // blocks per row: 1 (whole row) or 4
   static_assert(NB == 1 || NB == 4, "blocks of 128 or 32 columns");
   __shared__ TmaSmem smem_all[kTmaWarps];
