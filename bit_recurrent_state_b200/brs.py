@@ -25,7 +25,7 @@ STORES = {"fp32": STORE_FP32, "damp": STORE_DAMP, "varbit": STORE_VARBIT}
 # exported symbols declared in include/brs.h
 SYMBOLS = ["brs_state_bytes", "brs_state_pack", "brs_state_unpack", "brs_decode_step",
            "brs_decode_step_noalloc", "brs_chunk_prefill", "brs_allocate_bits", "brs_fetch_errors",
-           "brs_last_error"]
+           "brs_last_error", "brs_calibrate_workspace_bytes", "brs_calibrate"]
 
 
 class BrsError(RuntimeError):
@@ -86,6 +86,10 @@ def lib():
         L.brs_allocate_bits.restype = S
         L.brs_allocate_bits.argtypes = [ct.c_int, ct.c_int, P, ct.c_double, ct.c_int, ct.c_int,
                                         ct.c_uint32, P, P, P]
+        L.brs_calibrate_workspace_bytes.restype = ct.c_size_t
+        L.brs_calibrate_workspace_bytes.argtypes = [P, ct.c_int, ct.c_int, ct.c_int]
+        L.brs_calibrate.restype = S
+        L.brs_calibrate.argtypes = [P, ct.c_int, ct.c_int, ct.c_int, ct.c_double] + [P] * 9
         L.brs_fetch_errors.restype = S
         L.brs_fetch_errors.argtypes = [P, P, P]
         L.brs_last_error.restype = ct.c_char_p
@@ -171,6 +175,19 @@ def allocate_bits(cost, rows_per_group, avg_bits, b_min, b_max, bits_out, offset
     _check(lib().brs_allocate_bits(int(cost.numel()), int(rows_per_group), _ptr(cost), float(avg_bits),
                                    int(b_min), int(b_max), int(offset_unit), _ptr(bits_out),
                                    _ptr(offsets_out), _stream(stream)))
+
+
+def calibrate_workspace_bytes(layout, Bc: int, T: int, every: int) -> int:
+    """brs_calibrate_workspace_bytes."""
+    return int(lib().brs_calibrate_workspace_bytes(ct.byref(layout), int(Bc), int(T), int(every)))
+
+
+def calibrate(layout, Bc, T, every, tau, q, k, v, beta, decay, workspace, perm_out, score_out=None,
+              stream=None):
+    """brs_calibrate: protected-row selection on a calibration batch (token-major inputs)."""
+    _check(lib().brs_calibrate(ct.byref(layout), int(Bc), int(T), int(every), float(tau), _ptr(q), _ptr(k),
+                               _ptr(v), _ptr(beta), _ptr(decay), _ptr(workspace), _ptr(score_out),
+                               _ptr(perm_out), _stream(stream)))
 
 
 def fetch_errors(workspace, stream=None) -> int:

@@ -278,6 +278,81 @@ brs_status brs_allocate_bits(int n_rows, int rows_per_group, const double* cost,
   return ok();
 }
 
+namespace {
+// calibration workspace: [flag word, 256 B][states Bc*H*d*d f32][o Bc*H*d f32]
+// [err nsamp*Bc*H*d f64][score H*d f64]
+struct CalibLayout {
+  size_t states, o, err, score, total;
+};
+CalibLayout calib_layout(const brs_layout* L, int Bc, int T, int every) {
+  CalibLayout c{};
+  const size_t heads = (size_t)Bc * L->H, d = (size_t)L->d;
+  const size_t nsamp = (size_t)(T / every);
+  c.states = 256;
+  c.o = c.states + round256(heads * d * d * 4);
+  c.err = c.o + round256(heads * d * 4);
+  c.score = c.err + round256(nsamp * heads * d * 8);
+  c.total = c.score + round256((size_t)L->H * d * 8);
+  return c;
+}
+}  // namespace
+
+size_t brs_calibrate_workspace_bytes(const brs_layout* L, int Bc, int T, int every) {
+  if (!L || Bc <= 0 || T <= 0 || every <= 0 || L->d <= 0 || L->H <= 0) return 0;
+  return calib_layout(L, Bc, T, every).total;
+}
+
+brs_status brs_calibrate(const brs_layout* L, int Bc, int T, int every, double tau,
+                         const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* beta,
+                         const float* decay, void* workspace, double* score_out, int16_t* perm_out,
+                         void* stream) {
+  if (!L) return fail(BRS_EINVAL, "layout is NULL");
+  brs_layout Lc = *L;
+  Lc.B = Bc > 0 ? Bc : 1;
+  brs_status st = check_layout(&Lc);
+  if (st != BRS_OK) return st;
+  if (L->storage != BRS_STORE_DAMP) return fail(BRS_EINVAL, "calibration scores the rows of a DAMP layout");
+  if (Bc <= 0 || T <= 0 || every <= 0 || every > T) return fail(BRS_EINVAL, "need Bc > 0 and 0 < every <= T");
+  if (!(tau > 0.0)) return fail(BRS_EINVAL, "tau must be positive");
+  if (!q || !k || !v || !beta || !decay || !workspace || !perm_out)
+    return fail(BRS_EINVAL, "q, k, v, beta, decay, workspace and perm_out are required");
+  const void* ptrs[] = {q, k, v, beta, decay, workspace, score_out, perm_out};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(BRS_EALIGN, "device pointers must be 16-byte aligned");
+  const CalibLayout cl = calib_layout(L, Bc, T, every);
+  cudaStream_t s = (cudaStream_t)stream;
+  uint8_t* ws = (uint8_t*)workspace;
+  float* states = (float*)(ws + cl.states);
+  double* score = score_out ? score_out : (double*)(ws + cl.score);
+  cudaError_t e = cudaMemsetAsync(ws, 0, cl.o, s);                 // flag word and zero states
+  if (e != cudaSuccess) return cuda_fail(e, "calibration state clear");
+  brs::DecodeArgs a{};
+  a.B = Bc; a.H = L->H; a.Hk = L->H_k; a.k_hi = 0; a.block = L->d;
+  a.decay_per_key = L->decay_per_key; a.mode = BRS_ROUND_NEAREST; a.seed = 0;
+  a.head_bytes = (size_t)L->d * L->d * 4; a.hscale = hadamard_scale(L->d);
+  a.packed_in = states; a.packed_out = states; a.aux = nullptr; a.perm = nullptr;
+  a.o = (float*)(ws + cl.o); a.flags = (uint32_t*)ws;
+  brs::CalibArgs c{};
+  c.B = Bc; c.H = L->H; c.d = L->d; c.block = L->block; c.hadamard = L->hadamard; c.k_hi = L->k_hi;
+  c.T = T; c.nsamp = T / every; c.decay_per_key = L->decay_per_key; c.hscale = hadamard_scale(L->d);
+  c.tau = tau; c.S = states; c.err = (double*)(ws + cl.err); c.decay = decay; c.score = score;
+  c.perm = perm_out; c.flags = (uint32_t*)ws;
+  const size_t qk = (size_t)Bc * L->H_k * L->d, vv = (size_t)Bc * L->H * L->d, bh = (size_t)Bc * L->H;
+  const size_t dk = L->decay_per_key ? vv : bh;
+  for (int t = 0; t < T && e == cudaSuccess; ++t) {
+    a.step = t;
+    a.q = q + t * qk; a.k = k + t * qk; a.v = v + t * vv; a.beta = beta + t * bh; a.decay = decay + t * dk;
+    e = brs::launch_decode(a, L->d, BRS_STORE_FP32, false, s);
+    if (e == cudaSuccess && (t + 1) % every == 0) {
+      c.sample = (t + 1) / every - 1;
+      e = brs::launch_calib_sample(c, s);
+    }
+  }
+  if (e == cudaSuccess) e = brs::launch_calib_finish(c, s);
+  if (e != cudaSuccess) return cuda_fail(e, "calibration launch");
+  return ok();
+}
+
 brs_status brs_fetch_errors(void* workspace, uint32_t* flags_out, void* stream) {
   if (!workspace) return fail(BRS_EINVAL, "workspace is NULL");
   uint32_t fl = 0;

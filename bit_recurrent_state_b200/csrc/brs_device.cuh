@@ -148,6 +148,20 @@ __device__ __forceinline__ void row_fwht4(float (&x)[4], int cb, float scale) {
   mul2(x[2], x[3], x[2], x[3], scale, scale);
 }
 
+// Sylvester Hadamard, unnormalised butterflies h = 1, 2, 4, ... then one
+// scaling, on a row held by one thread.
+template <int D>
+__device__ inline void seq_fwht(float* x, float scale) {
+  for (int hs = 1; hs < D; hs <<= 1)
+    for (int i = 0; i < D; i += 2 * hs)
+      for (int j = i; j < i + hs; ++j) {
+        const float u0 = x[j], u1 = x[j + hs];
+        x[j] = __fadd_rn(u0, u1);
+        x[j + hs] = __fsub_rn(u0, u1);
+      }
+  for (int j = 0; j < D; ++j) x[j] = __fmul_rn(x[j], scale);
+}
+
 }  // namespace brs
 
 namespace brs {

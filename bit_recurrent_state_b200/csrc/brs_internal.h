@@ -27,6 +27,20 @@ struct DecodeArgs {
 
 cudaError_t launch_decode(const DecodeArgs& a, int d, int store, bool had, cudaStream_t st);
 bool decode_supported(int d, int block, int k_hi);
+
+struct CalibArgs {
+  int B, H, d, block, hadamard, k_hi, T, nsamp, sample, decay_per_key;
+  float hscale;
+  double tau;
+  const float* S;                // [B][H][d][d] FP32 calibration states
+  double* err;                   // [nsamp][B][H][d] per-sample error energies
+  const float* decay;            // [T][B][H][d] or [T][B][H]
+  double* score;                 // [H][d]
+  int16_t* perm;                 // [H][d]
+  uint32_t* flags;
+};
+cudaError_t launch_calib_sample(const CalibArgs& a, cudaStream_t st);
+cudaError_t launch_calib_finish(const CalibArgs& a, cudaStream_t st);
 // d = 128 DAMP decode with bulk-copy staging of the stored rows
 bool decode_tma_supported(int d, int store, int block, int k_hi);
 cudaError_t launch_decode_tma(const DecodeArgs& a, bool had, cudaStream_t st);

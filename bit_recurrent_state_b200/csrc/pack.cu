@@ -15,20 +15,6 @@
 
 namespace brs {
 
-// Sylvester Hadamard, unnormalised butterflies h = 1, 2, 4, ... then one
-// scaling, on a row held by one thread.
-template <int D>
-__device__ void seq_fwht(float* x, float scale) {
-  for (int hs = 1; hs < D; hs <<= 1)
-    for (int i = 0; i < D; i += 2 * hs)
-      for (int j = i; j < i + hs; ++j) {
-        const float u0 = x[j], u1 = x[j + hs];
-        x[j] = __fadd_rn(u0, u1);
-        x[j + hs] = __fsub_rn(u0, u1);
-      }
-  for (int j = 0; j < D; ++j) x[j] = __fmul_rn(x[j], scale);
-}
-
 template <int D>
 __global__ void pack_kernel(const PackArgs a) {
   const int head = blockIdx.x, h = head % a.H, i = threadIdx.x;

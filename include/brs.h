@@ -229,6 +229,37 @@ brs_status brs_allocate_bits(int n_rows, int rows_per_group, const double* cost,
                              int b_min, int b_max, uint32_t offset_unit, uint8_t* bits_out,
                              uint32_t* offsets_out, void* stream);
 
+/* Protected-row selection on a calibration run ([DAMP] Risk scoring and
+ * selection; Calibration): the FP32 recurrence (the FP32-storage decode
+ * step) runs from a zero state over T tokens of a calibration batch of Bc
+ * sequences; every `every` tokens each key row u of each head is scored by
+ * the squared error energy of its Hadamard-INT8 quantize -> dequantize
+ * (nearest rounding, L's block and Hadamard setting); then
+ *   E_u = the mean energy over sequences and samples,
+ *   a_eff,u = exp(mean over sequences and tokens of log a_u),
+ *   C_u = E_u / max(1 - a_eff,u^2, tau),
+ * and the k_hi largest C_u of a head (ties to the lower row) are protected.
+ *   L: a DAMP layout (B is ignored; d in {32, 64, 128}, k_hi <= d).
+ *   q, k: device bf16 [T][Bc][H_k][d]; v: bf16 [T][Bc][H][d];
+ *   beta: f32 [T][Bc][H]; decay: f32 [T][Bc][H][d] (KDA) or [T][Bc][H]
+ *   (GDN), key-channel order, no permutation.
+ *   workspace: device, brs_calibrate_workspace_bytes(L, Bc, T, every) bytes,
+ *   16-byte aligned; its first 256 bytes are the device flag word
+ *   (brs_fetch_errors).
+ *   score_out (optional): device f64 [H][d], C_u in key-channel order (kept
+ *   in the workspace when NULL).
+ *   perm_out: device int16 [H][d], the stored order to pass to the other
+ *   calls: the unprotected rows ascending, then the protected rows
+ *   ascending.
+ * Sums are taken in FP64 in a fixed order (per row over its values; per
+ * (head, row) over sequences, then samples or tokens in order).  Setup
+ * work; the call issues T + T/every + 2 kernels on the stream. */
+size_t brs_calibrate_workspace_bytes(const brs_layout* L, int Bc, int T, int every);
+brs_status brs_calibrate(const brs_layout* L, int Bc, int T, int every, double tau,
+                         const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* beta,
+                         const float* decay, void* workspace, double* score_out, int16_t* perm_out,
+                         void* stream);
+
 /* Allocation-free variant of brs_decode_step (the pages have no
  * counterpart; it exists for callers that cannot allocate device memory,
  * such as a host framework whose allocator owns the whole device or a
