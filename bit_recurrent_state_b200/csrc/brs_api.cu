@@ -251,7 +251,13 @@ brs_status brs_chunk_prefill(const brs_layout* L, const brs_writeback* wb, int64
   a.head_bytes = head_bytes(L); a.hscale = hadamard_scale(L->d);
   a.packed = packed; a.aux = aux; a.perm = perm; a.q = q; a.k = k; a.v = v; a.beta = beta;
   a.decay = decay; a.o = o; a.sdump = state_dump; a.flags = (uint32_t*)workspace;
-  cudaError_t e = brs::launch_prefill(a, L->hadamard != 0, (cudaStream_t)stream);
+  // the FP32 state between chunks: a stream-ordered scratch for this call
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMallocAsync((void**)&a.s0, brs::prefill_tc_scratch_bytes(L->B, L->H), s);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill scratch");
+  e = brs::launch_prefill_tc(a, L->hadamard != 0, s);
+  cudaError_t e2 = cudaFreeAsync(a.s0, s);
+  if (e == cudaSuccess) e = e2;
   if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
   return ok();
 }

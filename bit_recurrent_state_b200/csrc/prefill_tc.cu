@@ -1,0 +1,566 @@
+// Chunked prefill on the tcgen05 tensor cores (DAMP storage, d = 128,
+// C = 64): the chunk's WY-form contractions run as TF32 UMMA with FP32
+// accumulation in tensor memory, each product split 3 ways
+// (hi*hi + hi*lo + lo*hi, hi = the operand truncated to TF32, lo = the
+// remainder) so the contractions keep FP32-level accuracy; the forward
+// substitution, the masks, the requantization and the write-back run on
+// the CUDA cores.  Same math and the same write-back protocol as the
+// CUDA-core prefill ("Low-Bit Recurrent States in Hybrid Language Models",
+// Accumulated readout error: write-back once per prefill chunk; Protocol:
+// quantized and dequantized before reuse):
+//   Gamma_t = prod_{r <= t} a_r, K~ = K * Gamma, K^ = K / Gamma, Q~ = Q * Gamma;
+//   A = strictly-lower(diag(beta) K~ K^T);  (I + A) W = diag(beta)(V - K~ S_0);
+//   O = Q~ S_0 + lower-incl(Q~ K^T) W;  S_C = diag(Gamma_63)(S_0 + K^T W).
+//
+// One CTA of 256 threads per (sequence, head) walks the chunks in order.
+// Tensor-memory accumulators (lanes x columns, FP32):
+//   D2 [128 j][128 t]: (K~ S_0)^T for t < 64, O^T = (Q~ S_0 + P W)^T for t >= 64
+//   D1 [128 t][64 s] : K~ K^T (t < 64) and Q~ K^T (t >= 64)
+//   D4 [128 i][128 j]: K^T W
+// All operands are K-major, no swizzle: 8-row x 16-byte core matrices,
+// consecutive along K at 128 B, row groups of 8 at Kt/4 * 128 B.
+// Products in tensor-memory orientation:
+//   D1 = [K~;Q~] . K^^T     (A: X[t][i], B: X[s][i]; K = i in 4 slices of 32)
+//   D2 = S_0^T . [K~;Q~]^T   (A: X[j][i], B: X[t][i])
+//   D2[:, 64:] += W^T . P^T  (A: X[j][s], B: X[t][s]; P = lower-incl(Q~ K^T))
+//   D4 = K^T . W             (A: X[i][s], B: X[j][s])
+// The FP32 state S_0 between chunks lives in a global scratch (dequantized
+// stored state, stored row order, value basis).
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "brs_device.cuh"
+#include "brs_internal.h"
+
+namespace brs {
+namespace {
+
+constexpr int kD = 128, kC = 64, kThreads = 256;
+constexpr int kSl = 32;                                   // K slice of the i-contractions
+constexpr unsigned long long kTcWaitNs = 200000000ull;    // bound on one MMA wait (200 ms)
+
+// ---- shared-memory map (bytes from the 1 KB-aligned dynamic base)
+// phase 1: two slice buffers, each: KQ hi/lo [128][32], KH hi/lo [64][32], S0T hi/lo [128][32]
+constexpr int kKQ = 128 * kSl * 4, kKH = 64 * kSl * 4, kS0T = 128 * kSl * 4;
+constexpr int kBuf = 2 * (kKQ + kKH + kS0T);              // 80 KB
+// phase 2: W hi/lo [128 j][64 s], KT hi/lo [128 i][64 s], P hi/lo [64 t][64 s], A fp32 [64][68]
+constexpr int kWt = 128 * 64 * 4, kKT = 128 * 64 * 4, kPt = 64 * 64 * 4;
+constexpr int kOffW = 0, kOffKT = 2 * kWt, kOffP = kOffKT + 2 * kKT, kOffA = kOffP + 2 * kPt;
+constexpr int kAStride = 68;
+constexpr int kRegion = kOffA + 64 * kAStride * 4;        // 177 KB (covers the two slice buffers)
+// requantization: S [128][132] fp32 at the start of the region
+constexpr int kSStride = 132;
+constexpr int kOffGam = kRegion;                          // Gamma [64][128] fp32
+constexpr int kOffBeta = kOffGam + kC * kD * 4;           // beta [64]
+constexpr int kOffMisc = kOffBeta + kC * 4;               // mbarriers, tensor-memory base, flags
+constexpr int kSmem = kOffMisc + 64;
+static_assert(2 * kBuf <= kRegion, "slice buffers fit the phase region");
+static_assert(kD * kSStride * 4 <= kRegion, "requantization rows fit the phase region");
+static_assert(kSmem <= 227 * 1024, "shared memory of one CTA");
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+// ---- K-major no-swizzle operand tile X[R][Kt]: byte offset of (r, k)
+__device__ __forceinline__ uint32_t kmaj(int r, int k, int Kt) {
+  return (uint32_t)(((r >> 3) * (Kt >> 2) + (k >> 2)) * 128 + (r & 7) * 16 + (k & 3) * 4);
+}
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t sbo) {
+  // start >> 4, leading offset 128 B (next 4 elements along K), stride offset
+  // sbo (next 8 rows), descriptor version 1, no swizzle
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)(128u >> 4) << 16) | ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) |
+         (1ull << 46);
+}
+// kind::tf32 instruction descriptor: D f32, A/B tf32, both K-major
+constexpr uint32_t idesc_tf32(int M, int N) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+__device__ __forceinline__ void umma_tf32(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+// 3-way split product: D (+)= Ah Bh + Ah Bl + Al Bh
+__device__ __forceinline__ void umma3(uint32_t d, uint32_t ah, uint32_t al, uint32_t bh, uint32_t bl, uint32_t sboa,
+                                      uint32_t sbob, uint32_t idesc, uint32_t acc) {
+  umma_tf32(d, sdesc(ah, sboa), sdesc(bh, sbob), idesc, acc);
+  umma_tf32(d, sdesc(ah, sboa), sdesc(bl, sbob), idesc, 1u);
+  umma_tf32(d, sdesc(al, sboa), sdesc(bh, sbob), idesc, 1u);
+}
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void proxy_fence() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// bounded wait for one phase of an MMA-completion barrier
+__device__ __noinline__ bool mbar_wait_tc(uint32_t bar, uint32_t parity) {
+  if (mbar_try(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  while (!mbar_try(bar, parity))
+    if (global_ns() - t0 > kTcWaitNs) return false;
+  return true;
+}
+
+// 16 consecutive FP32 columns of this thread's tensor-memory lane
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int c = 0; c < 16; ++c) v[c] = __uint_as_float(r[c]);
+}
+
+// the operand split: hi = x truncated to TF32, lo = x - hi (exact)
+__device__ __forceinline__ float tf32_hi(float x) { return __uint_as_float(__float_as_uint(x) & 0xFFFFE000u); }
+// store 4 consecutive-K values of row r at (hi tile, lo tile)
+__device__ __forceinline__ void st_split4(uint8_t* hi, uint8_t* lo, uint32_t off, float x0, float x1, float x2,
+                                          float x3) {
+  const float h0 = tf32_hi(x0), h1 = tf32_hi(x1), h2 = tf32_hi(x2), h3 = tf32_hi(x3);
+  *(float4*)(hi + off) = make_float4(h0, h1, h2, h3);
+  *(float4*)(lo + off) = make_float4(__fsub_rn(x0, h0), __fsub_rn(x1, h1), __fsub_rn(x2, h2), __fsub_rn(x3, h3));
+}
+
+// stored head -> FP32 rows (stored order, value basis) in the global scratch
+template <bool HAD, int BLOCK>
+__device__ void tc_load_state(const uint8_t* head, float* S, int nlo, int k_hi, float hscale) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, col0 = 4 * lane;
+  constexpr int NB = kD / BLOCK;
+  const uint8_t* f16in = head + (size_t)nlo * kD;
+  const uint32_t* szin = (const uint32_t*)(head + (size_t)nlo * kD + (size_t)k_hi * kD * 2);
+  for (int r = warp; r < kD; r += kThreads / 32) {
+    float x[4];
+    if (r < nlo) {
+      const uint32_t c4 = *(const uint32_t*)(head + (size_t)r * kD + col0);
+      const uint32_t sz = szin[r * NB + col0 / BLOCK];
+      const float s = f16_to_f32((uint16_t)(sz & 0xffffu)), z = f16_to_f32((uint16_t)(sz >> 16));
+#pragma unroll
+      for (int c = 0; c < 4; ++c) x[c] = __fmaf_rn(__fsub_rn(byte_magic(c4, c), kTwo23), s, z);
+      if (HAD) row_fwht4<kD>(x, lane, hscale);
+    } else {
+      const uint2 hv = *(const uint2*)(f16in + ((size_t)(r - nlo) * kD + col0) * 2);
+      x[0] = f16_to_f32((uint16_t)(hv.x & 0xffffu)); x[1] = f16_to_f32((uint16_t)(hv.x >> 16));
+      x[2] = f16_to_f32((uint16_t)(hv.y & 0xffffu)); x[3] = f16_to_f32((uint16_t)(hv.y >> 16));
+    }
+    *(float4*)&S[(size_t)r * kD + col0] = make_float4(x[0], x[1], x[2], x[3]);
+  }
+}
+
+// S_C rows (shared, stride kSStride) -> stored head; the dequantized rows
+// (the state the next chunk starts from) go to the global scratch
+template <bool HAD, int BLOCK, int MODE>
+__device__ void tc_store_state(const float* Ss, float* S, uint8_t* head, uint16_t* aux, int nlo, int k_hi,
+                               float hscale, const PrefillArgs& a, int64_t step, int h, int b, float* sdump,
+                               uint32_t& err) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, col0 = 4 * lane;
+  constexpr int NB = kD / BLOCK, GL = BLOCK / 4;
+  uint16_t* f16out = (uint16_t*)(head + (size_t)nlo * kD);
+  uint32_t* szout = (uint32_t*)(head + (size_t)nlo * kD + (size_t)k_hi * kD * 2);
+  for (int r = warp; r < kD; r += kThreads / 32) {
+    const float4 v4 = *(const float4*)&Ss[r * kSStride + col0];
+    if (sdump) *(float4*)&sdump[(size_t)r * kD + col0] = v4;
+    float x[4] = {v4.x, v4.y, v4.z, v4.w};
+    if (r >= nlo) {
+      const uint32_t lo = f16x2_of(x[0], x[1]), hi = f16x2_of(x[2], x[3]);
+      if ((((lo >> 10) & 31u) == 31u) || (((lo >> 26) & 31u) == 31u) || (((hi >> 10) & 31u) == 31u) ||
+          (((hi >> 26) & 31u) == 31u))
+        err |= BRS_FLAG_OVERFLOW;
+      *(uint2*)&f16out[(size_t)(r - nlo) * kD + col0] = make_uint2(lo, hi);
+      *(float4*)&S[(size_t)r * kD + col0] =
+          make_float4(f16_to_f32((uint16_t)(lo & 0xffffu)), f16_to_f32((uint16_t)(lo >> 16)),
+                      f16_to_f32((uint16_t)(hi & 0xffffu)), f16_to_f32((uint16_t)(hi >> 16)));
+      continue;
+    }
+    if (HAD) row_fwht4<kD>(x, lane, hscale);
+    if (MODE == BRS_ROUND_ERRFEEDBACK) {
+      const uint2 ev = *(const uint2*)&aux[(size_t)r * kD + col0];
+      x[0] = __fadd_rn(x[0], f16_to_f32((uint16_t)(ev.x & 0xffffu)));
+      x[1] = __fadd_rn(x[1], f16_to_f32((uint16_t)(ev.x >> 16)));
+      x[2] = __fadd_rn(x[2], f16_to_f32((uint16_t)(ev.y & 0xffffu)));
+      x[3] = __fadd_rn(x[3], f16_to_f32((uint16_t)(ev.y >> 16)));
+    }
+    float mn = fminf(fminf(x[0], x[1]), fminf(x[2], x[3]));
+    float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+#pragma unroll
+    for (int m = 1; m < GL; m <<= 1) {
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, m));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
+    }
+    if (mn == 0.0f || mx == 0.0f) {             // -0 ranks below +0 (uniform per block group)
+      bool nz = false, pz = false;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        nz |= (x[c] == 0.0f) && signbit(x[c]);
+        pz |= (x[c] == 0.0f) && !signbit(x[c]);
+      }
+      const uint32_t gmask = (GL >= 32) ? 0xffffffffu : (((1u << GL) - 1u) << (lane & ~(uint32_t)(GL - 1)));
+      const unsigned anz = __reduce_or_sync(gmask, nz ? 1u : 0u), apz = __reduce_or_sync(gmask, pz ? 1u : 0u);
+      if (mn == 0.0f) mn = anz ? -0.0f : 0.0f;
+      if (mx == 0.0f) mx = apz ? 0.0f : -0.0f;
+    }
+    if (!isfinite(mn) || !isfinite(mx)) err |= BRS_FLAG_NONFINITE;
+    const uint16_t sh = f32_to_f16(__fdiv_rn(__fsub_rn(mx, mn), 255.0f));
+    const uint16_t zh = f32_to_f16(mn);
+    if (f16_inf_or_nan(sh) || f16_inf_or_nan(zh)) err |= BRS_FLAG_OVERFLOW;
+    const float s = f16_to_f32(sh), z = f16_to_f32(zh);
+    const float rcp = (s == 0.0f) ? 0.0f : __frcp_rn(s);
+    uint4 rnd = make_uint4(0, 0, 0, 0);
+    if (MODE == BRS_ROUND_STOCHASTIC)
+      rnd = philox4x32_10(make_uint4((uint32_t)(r * (kD / 4) + lane), (uint32_t)step, (uint32_t)h, (uint32_t)b),
+                          make_uint2((uint32_t)a.seed, (uint32_t)(a.seed >> 32)));
+    const uint32_t rw[4] = {rnd.x >> 8, rnd.y >> 8, rnd.z >> 8, rnd.w >> 8};
+    uint32_t packed4 = 0;
+    float xh[4];
+    uint16_t e16[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float code = 0.0f;
+      if (s != 0.0f) {
+        const float tt = __fmul_rn(__fsub_rn(x[c], z), rcp);
+        code = (MODE == BRS_ROUND_STOCHASTIC) ? sr_round(tt, rw[c]) : rintf(tt);
+        code = fminf(fmaxf(code, 0.0f), 255.0f);
+      }
+      packed4 |= ((uint32_t)(int)code) << (8 * c);
+      xh[c] = __fmaf_rn(code, s, z);
+      if (MODE == BRS_ROUND_ERRFEEDBACK) {
+        float e = __fsub_rn(x[c], xh[c]);
+        if (e > s) e = s;
+        else if (e < -s) e = -s;
+        e16[c] = f32_to_f16(e);
+      }
+    }
+    *(uint32_t*)(head + (size_t)r * kD + col0) = packed4;
+    if ((col0 % BLOCK) == 0) szout[r * NB + col0 / BLOCK] = (uint32_t)sh | ((uint32_t)zh << 16);
+    if (MODE == BRS_ROUND_ERRFEEDBACK)
+      *(uint2*)&aux[(size_t)r * kD + col0] =
+          make_uint2((uint32_t)e16[0] | ((uint32_t)e16[1] << 16), (uint32_t)e16[2] | ((uint32_t)e16[3] << 16));
+    if (HAD) row_fwht4<kD>(xh, lane, hscale);          // continue from the stored values
+    *(float4*)&S[(size_t)r * kD + col0] = make_float4(xh[0], xh[1], xh[2], xh[3]);
+  }
+}
+
+template <bool HAD, int BLOCK, int MODE>
+__global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int sub = warp & 3;                        // tensor-memory lanes 32 sub .. 32 sub + 31
+  const int half = warp >> 2;                      // which half of a readout's columns
+  const int head = blockIdx.x;
+  const int b = head / a.H, h = head - b * a.H, kh = h * a.Hk / a.H;
+  const int nlo = kD - a.k_hi;
+  uint8_t* hst = (uint8_t*)a.packed + (size_t)head * a.head_bytes;
+  uint16_t* aux = (MODE == BRS_ROUND_ERRFEEDBACK) ? (uint16_t*)a.aux + (size_t)head * nlo * kD : nullptr;
+  float* S0g = a.s0 + (size_t)head * kD * kD;      // FP32 state between chunks
+  float* gam = (float*)(smem + kOffGam);           // Gamma [64 t][128 i]
+  float* betas = (float*)(smem + kOffBeta);
+  unsigned long long* bars = (unsigned long long*)(smem + kOffMisc);   // slice buffers 0, 1; phase 2
+  uint32_t* tslot = (uint32_t*)(smem + kOffMisc + 32);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = smem_u32(&bars[0]);
+  uint32_t err = 0;
+
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tslot)),
+                 "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  if (tid == 0) {
+#pragma unroll
+    for (int i = 0; i < 3; ++i) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar0 + 8u * i));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  tc_load_state<HAD, BLOCK>(hst, S0g, nlo, a.k_hi, a.hscale);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = *tslot;
+  const uint32_t tD2 = tm, tD1 = tm + 128, tD4 = tm + 256;
+  const uint32_t lrow = (uint32_t)(32 * sub) << 16;          // this warp's lane base in tensor memory
+  const int myrow = 32 * sub + lane;                          // the tensor-memory lane this thread reads
+  uint32_t ph0 = 0, ph1 = 0, ph2 = 0;
+  bool alive = true;
+  // every thread waits; the CTA agrees on the outcome
+  auto wait_all = [&](int which, uint32_t& ph) -> bool {
+    const bool ok = mbar_wait_tc(bar0 + 8u * which, ph);
+    ph ^= 1u;
+    return !__syncthreads_or(ok ? 0 : 1);
+  };
+
+  const int nchunks = a.T / kC;
+  for (int ch = 0; ch < nchunks && alive; ++ch) {
+    const int t0 = ch * kC;
+    const size_t tokb = (size_t)b * a.T + t0;                 // first token of the chunk
+    // ---- Gamma (cumulative decay per stored row) and beta
+    if (tid < kD) {
+      const int p = a.perm ? a.perm[h * kD + tid] : tid;
+      float g = 1.0f;
+      for (int r = 0; r < kC; ++r) {
+        const size_t tok = tokb + r;
+        const float av = a.decay_per_key ? a.decay[(tok * a.H + h) * kD + p] : a.decay[tok * a.H + h];
+        g = __fmul_rn(g, av);
+        gam[r * kD + tid] = g;
+      }
+    } else if (tid < kD + kC) {
+      betas[tid - kD] = a.beta[(tokb + (tid - kD)) * a.H + h];
+    }
+    __syncthreads();
+
+    // ---- phase 1: D1 = [K~;Q~] K^^T, D2 = S_0^T [K~;Q~]^T over 4 slices of
+    // 32 stored rows i, the slices double-buffered against the MMAs
+    for (int sl = 0; sl < kD / kSl && alive; ++sl) {
+      const int buf = sl & 1;
+      if (sl >= 2) {
+        alive = buf ? wait_all(1, ph1) : wait_all(0, ph0);
+        if (!alive) break;
+      }
+      uint8_t* B0 = smem + buf * kBuf;
+      uint8_t *KQh = B0, *KQl = B0 + kKQ, *KHh = B0 + 2 * kKQ, *KHl = KHh + kKH, *STh = KHl + kKH, *STl = STh + kS0T;
+      const int i0 = sl * kSl;
+      for (int task = tid; task < 2560; task += kThreads) {
+        if (task < 1024) {                           // [K~;Q~] rows t, 4 columns 4g..4g+3 of the slice
+          const int t = task & 127, g = task >> 7;
+          const int tt = t & 63;
+          const uint16_t* src = (t < 64) ? a.k : a.q;
+          float x[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int i = i0 + 4 * g + c;
+            const int p = a.perm ? a.perm[h * kD + i] : i;
+            x[c] = __fmul_rn(bf16_to_f32(src[((tokb + tt) * a.Hk + kh) * kD + p]), gam[tt * kD + i]);
+          }
+          st_split4(KQh, KQl, kmaj(t, 4 * g, kSl), x[0], x[1], x[2], x[3]);
+        } else if (task < 1536) {                    // K^ rows s
+          const int u = task - 1024, s = u & 63, g = u >> 6;
+          float x[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int i = i0 + 4 * g + c;
+            const int p = a.perm ? a.perm[h * kD + i] : i;
+            x[c] = __fdiv_rn(bf16_to_f32(a.k[((tokb + s) * a.Hk + kh) * kD + p]), gam[s * kD + i]);
+          }
+          st_split4(KHh, KHl, kmaj(s, 4 * g, kSl), x[0], x[1], x[2], x[3]);
+        } else {                                     // S_0^T rows j
+          const int u = task - 1536, j = u & 127, g = u >> 7;
+          const int i = i0 + 4 * g;
+          st_split4(STh, STl, kmaj(j, 4 * g, kSl), S0g[(size_t)i * kD + j], S0g[(size_t)(i + 1) * kD + j],
+                    S0g[(size_t)(i + 2) * kD + j], S0g[(size_t)(i + 3) * kD + j]);
+        }
+      }
+      proxy_fence();
+      tc_fence_before();
+      __syncthreads();
+      if (tid == 0) {
+        tc_fence_after();
+        const uint32_t base = sbase + buf * kBuf;
+        const uint32_t aKQh = base, aKQl = base + kKQ, aKHh = base + 2 * kKQ, aKHl = aKHh + kKH;
+        const uint32_t aSTh = aKHl + kKH, aSTl = aSTh + kS0T;
+        constexpr uint32_t sbo = (kSl / 4) * 128;
+#pragma unroll
+        for (int k = 0; k < kSl / 8; ++k) {
+          const uint32_t o = 256u * k, acc = (sl > 0 || k > 0) ? 1u : 0u;
+          umma3(tD1, aKQh + o, aKQl + o, aKHh + o, aKHl + o, sbo, sbo, idesc_tf32(128, 64), acc);
+          umma3(tD2, aSTh + o, aSTl + o, aKQh + o, aKQl + o, sbo, sbo, idesc_tf32(128, 128), acc);
+        }
+        umma_commit(bar0 + 8u * buf);
+      }
+    }
+    if (!alive) break;
+    alive = wait_all(0, ph0) && wait_all(1, ph1);
+    if (!alive) break;
+    tc_fence_after();
+
+    // ---- readouts of D1: A = strictly-lower(diag(beta) K~ K^T) (fp32, shared),
+    // P = lower-incl(Q~ K^T) as the split operand X[t][s]
+    float* Am = (float*)(smem + kOffA);
+    {
+      float v[16];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int c0 = 32 * half + 16 * q;
+        tmem_ld16(tD1 + lrow + c0, v);
+        if (myrow < 64) {
+          const int t = myrow;
+          const float bt = betas[t];
+#pragma unroll
+          for (int c = 0; c < 16; c += 4)
+            *(float4*)&Am[t * kAStride + c0 + c] =
+                make_float4((c0 + c + 0 < t) ? __fmul_rn(bt, v[c + 0]) : 0.0f, (c0 + c + 1 < t) ? __fmul_rn(bt, v[c + 1]) : 0.0f,
+                            (c0 + c + 2 < t) ? __fmul_rn(bt, v[c + 2]) : 0.0f, (c0 + c + 3 < t) ? __fmul_rn(bt, v[c + 3]) : 0.0f);
+        } else {
+          const int t = myrow - 64;
+#pragma unroll
+          for (int c = 0; c < 16; c += 4)
+            st_split4(smem + kOffP, smem + kOffP + kPt, kmaj(t, c0 + c, 64), (c0 + c + 0 <= t) ? v[c + 0] : 0.0f,
+                      (c0 + c + 1 <= t) ? v[c + 1] : 0.0f, (c0 + c + 2 <= t) ? v[c + 2] : 0.0f,
+                      (c0 + c + 3 <= t) ? v[c + 3] : 0.0f);
+        }
+      }
+    }
+    __syncthreads();
+
+    if (half == 0) {
+      // ---- W by forward substitution, one value column j per thread:
+      // (I + A) W = diag(beta)(V - K~ S_0), the right side from D2[j][0..63]
+      const int j = myrow;
+      float w[kC];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float v[16];
+        tmem_ld16(tD2 + lrow + 16 * q, v);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int t = 16 * q + c;
+          const float vv = bf16_to_f32(a.v[((tokb + t) * a.H + h) * kD + j]);
+          w[t] = __fmul_rn(betas[t], __fsub_rn(vv, v[c]));
+        }
+      }
+#pragma unroll
+      for (int t = 1; t < kC; ++t) {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int s = 0; s < t; s += 4) {
+          const float4 a4 = *(const float4*)&Am[t * kAStride + s];
+          acc[0] = __fmaf_rn(a4.x, w[s], acc[0]);
+          if (s + 1 < t) acc[1] = __fmaf_rn(a4.y, w[s + 1], acc[1]);
+          if (s + 2 < t) acc[2] = __fmaf_rn(a4.z, w[s + 2], acc[2]);
+          if (s + 3 < t) acc[3] = __fmaf_rn(a4.w, w[s + 3], acc[3]);
+        }
+        w[t] = __fsub_rn(w[t], __fadd_rn(__fadd_rn(acc[0], acc[1]), __fadd_rn(acc[2], acc[3])));
+      }
+#pragma unroll
+      for (int s = 0; s < kC; s += 4)
+        st_split4(smem + kOffW, smem + kOffW + kWt, kmaj(j, s, 64), w[s], w[s + 1], w[s + 2], w[s + 3]);
+    } else {
+      // ---- K^ transposed: X[i][s] = K[s][p_i] / Gamma[s][i]
+      const int tl = tid - 128;
+      for (int task = tl; task < kD * (kC / 4); task += 128) {
+        const int i = task & 127, sg = task >> 7;
+        const int p = a.perm ? a.perm[h * kD + i] : i;
+        float x[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int s = 4 * sg + c;
+          x[c] = __fdiv_rn(bf16_to_f32(a.k[((tokb + s) * a.Hk + kh) * kD + p]), gam[s * kD + i]);
+        }
+        st_split4(smem + kOffKT, smem + kOffKT + kKT, kmaj(i, 4 * sg, 64), x[0], x[1], x[2], x[3]);
+      }
+    }
+    proxy_fence();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      // ---- phase 2: D2[:, 64:] += W^T P^T (O^T), D4 = K^T W
+      tc_fence_after();
+      const uint32_t aWh = sbase + kOffW, aWl = aWh + kWt, aKTh = sbase + kOffKT, aKTl = aKTh + kKT;
+      const uint32_t aPh = sbase + kOffP, aPl = aPh + kPt;
+      constexpr uint32_t sbo = (64 / 4) * 128;
+#pragma unroll
+      for (int k = 0; k < kC / 8; ++k) {
+        const uint32_t o = 256u * k;
+        umma3(tD2 + 64, aWh + o, aWl + o, aPh + o, aPl + o, sbo, sbo, idesc_tf32(128, 64), 1u);
+        umma3(tD4, aKTh + o, aKTl + o, aWh + o, aWl + o, sbo, sbo, idesc_tf32(128, 128), k > 0 ? 1u : 0u);
+      }
+      umma_commit(bar0 + 16u);
+    }
+    alive = wait_all(2, ph2);
+    if (!alive) break;
+    tc_fence_after();
+
+    // ---- O = (D2[:, 64:])^T to global; S_C = Gamma_63 (S_0 + D4) to the
+    // requantization rows
+    {
+      const int j = myrow;
+      float v[16];
+      bool bad = false;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int c0 = 32 * half + 16 * q;
+        tmem_ld16(tD2 + lrow + 64 + c0, v);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          bad |= !isfinite(v[c]);
+          a.o[((tokb + c0 + c) * a.H + h) * kD + j] = v[c];
+        }
+      }
+      if (bad) err |= BRS_FLAG_NONFINITE;
+      float* Ss = (float*)smem;
+      const int i = myrow;
+      const float g63 = gam[63 * kD + i];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int c0 = 64 * half + 16 * q;
+        tmem_ld16(tD4 + lrow + c0, v);
+#pragma unroll
+        for (int c = 0; c < 16; c += 4) {
+          const float4 s4 = *(const float4*)&S0g[(size_t)i * kD + c0 + c];
+          *(float4*)&Ss[i * kSStride + c0 + c] =
+              make_float4(__fmul_rn(g63, __fadd_rn(s4.x, v[c])), __fmul_rn(g63, __fadd_rn(s4.y, v[c + 1])),
+                          __fmul_rn(g63, __fadd_rn(s4.z, v[c + 2])), __fmul_rn(g63, __fadd_rn(s4.w, v[c + 3])));
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    // ---- write-back of the chunk
+    const bool last = ch == nchunks - 1;
+    tc_store_state<HAD, BLOCK, MODE>((const float*)smem, S0g, hst, aux, nlo, a.k_hi, a.hscale, a,
+                                     a.step0 + t0 + kC - 1, h, b,
+                                     (last && a.sdump) ? a.sdump + (size_t)head * kD * kD : nullptr, err);
+    __syncthreads();
+  }
+  if (!alive) err |= BRS_FLAG_TIMEOUT;
+  if (err) raise_flag(a.flags, err);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tm), "r"(512));
+}
+
+template <bool HAD, int BLOCK, int MODE>
+cudaError_t tc_launch(const PrefillArgs& a, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<HAD, BLOCK, MODE>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  if (e != cudaSuccess) return e;
+  prefill_tc_kernel<HAD, BLOCK, MODE><<<a.B * a.H, kThreads, kSmem, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <bool HAD, int BLOCK>
+cudaError_t tc_launch_hb(const PrefillArgs& a, cudaStream_t st) {
+  switch (a.mode) {
+    case BRS_ROUND_NEAREST: return tc_launch<HAD, BLOCK, BRS_ROUND_NEAREST>(a, st);
+    case BRS_ROUND_STOCHASTIC: return tc_launch<HAD, BLOCK, BRS_ROUND_STOCHASTIC>(a, st);
+    case BRS_ROUND_ERRFEEDBACK: return tc_launch<HAD, BLOCK, BRS_ROUND_ERRFEEDBACK>(a, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+size_t prefill_tc_scratch_bytes(int B, int H) { return (size_t)B * H * kD * kD * sizeof(float); }
+
+cudaError_t launch_prefill_tc(const PrefillArgs& a, bool had, cudaStream_t st) {
+  if (a.block == 128) return had ? tc_launch_hb<true, 128>(a, st) : tc_launch_hb<false, 128>(a, st);
+  if (a.block == 32) return had ? tc_launch_hb<true, 32>(a, st) : tc_launch_hb<false, 32>(a, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace brs
