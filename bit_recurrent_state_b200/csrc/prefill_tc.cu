@@ -8,7 +8,7 @@
 // CUDA-core prefill ("Low-Bit Recurrent States in Hybrid Language Models",
 // Accumulated readout error: write-back once per prefill chunk; Protocol:
 // quantized and dequantized before reuse):
-//   Gamma_t = prod_{r <= t} a_r, K~ = K * Gamma, K^ = K / Gamma, Q~ = Q * Gamma;
+//   Gamma_t = prod_{r <= t} a_r, K~ = K * Gamma, K^ = K * (1 / Gamma), Q~ = Q * Gamma;
 //   A = strictly-lower(diag(beta) K~ K^T);  (I + A) W = diag(beta)(V - K~ S_0);
 //   O = Q~ S_0 + lower-incl(Q~ K^T) W;  S_C = diag(Gamma_63)(S_0 + K^T W).
 //
@@ -35,27 +35,38 @@
 namespace brs {
 namespace {
 
-constexpr int kD = 128, kC = 64, kThreads = 256;
+constexpr int kD = 128, kC = 64, kThreads = 512;
+constexpr int kParts = kThreads / 128;                   // warps per tensor-memory sub-partition
 constexpr int kSl = 32;                                   // K slice of the i-contractions
 constexpr unsigned long long kTcWaitNs = 200000000ull;    // bound on one MMA wait (200 ms)
 
 // ---- shared-memory map (bytes from the 1 KB-aligned dynamic base)
-// phase 1: two slice buffers, each: KQ hi/lo [128][32], KH hi/lo [64][32], S0T hi/lo [128][32]
+// chunk inputs, FP32 rows of stride kRS floats (stored-row order columns):
+//   Kt = K~ [64 t][128 i], Kh = K^, Qt = Q~
+constexpr int kRS = 132;
+constexpr int kRowB = kRS * 4;
+// phase 1: one slice buffer: KQ hi/lo [128][32], KH hi/lo [64][32], S0T hi/lo [128][32]
 constexpr int kKQ = 128 * kSl * 4, kKH = 64 * kSl * 4, kS0T = 128 * kSl * 4;
-constexpr int kBuf = 2 * (kKQ + kKH + kS0T);              // 80 KB
-// phase 2: W hi/lo [128 j][64 s], KT hi/lo [128 i][64 s], P hi/lo [64 t][64 s], A fp32 [64][68]
+constexpr int kOffSlice = 0;
+constexpr int kSliceB = 2 * (kKQ + kKH + kS0T);           // 80 KB
+constexpr int kOffKt = kOffSlice + kSliceB, kOffKh = kOffKt + kC * kRowB, kOffQt = kOffKh + kC * kRowB;
+// phase 2: KT hi/lo [128 i][64 s] over the slice buffer, P hi/lo [64 t][64 s] and A fp32 [64][68]
+// over Kt, W hi/lo [128 j][64 s] over Qt; Kh stays readable while KT is built
 constexpr int kWt = 128 * 64 * 4, kKT = 128 * 64 * 4, kPt = 64 * 64 * 4;
-constexpr int kOffW = 0, kOffKT = 2 * kWt, kOffP = kOffKT + 2 * kKT, kOffA = kOffP + 2 * kPt;
 constexpr int kAStride = 68;
-constexpr int kRegion = kOffA + 64 * kAStride * 4;        // 177 KB (covers the two slice buffers)
+constexpr int kOffKT = 0, kOffP = kOffKT + 2 * kKT, kOffA = kOffP + 2 * kPt, kOffW = kOffQt;
+constexpr int kRegion = kOffW + 2 * kWt;                   // 210 KB
 // requantization: S [128][132] fp32 at the start of the region
 constexpr int kSStride = 132;
-constexpr int kOffGam = kRegion;                          // Gamma [64][128] fp32
-constexpr int kOffBeta = kOffGam + kC * kD * 4;           // beta [64]
-constexpr int kOffMisc = kOffBeta + kC * 4;               // mbarriers, tensor-memory base, flags
-constexpr int kSmem = kOffMisc + 64;
-static_assert(2 * kBuf <= kRegion, "slice buffers fit the phase region");
-static_assert(kD * kSStride * 4 <= kRegion, "requantization rows fit the phase region");
+constexpr int kOffG63 = kRegion;                           // Gamma_63 [128]
+constexpr int kOffBeta = kOffG63 + kD * 4;                 // beta [64]
+constexpr int kOffMisc = kOffBeta + kC * 4;                // mbarriers, tensor-memory base
+constexpr int kOffPerm = kOffMisc + 64;                    // stored row -> key channel [128] int16
+constexpr int kSmem = kOffPerm + kD * 2;
+static_assert(kOffA + 64 * kAStride * 4 <= kOffKh, "P and A leave Kh intact");
+static_assert(kOffKT + 2 * kKT <= kOffKt, "KT over the slice buffer only");
+static_assert(kOffQt + kC * kRowB <= kRegion, "Qt inside the region");
+static_assert(kD * kSStride * 4 <= kOffW, "requantization rows fit below W");
 static_assert(kSmem <= 227 * 1024, "shared memory of one CTA");
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -263,17 +274,21 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int sub = warp & 3;                        // tensor-memory lanes 32 sub .. 32 sub + 31
-  const int half = warp >> 2;                      // which half of a readout's columns
+  const int part = warp >> 2;                      // which part of a readout's columns
   const int head = blockIdx.x;
   const int b = head / a.H, h = head - b * a.H, kh = h * a.Hk / a.H;
   const int nlo = kD - a.k_hi;
   uint8_t* hst = (uint8_t*)a.packed + (size_t)head * a.head_bytes;
   uint16_t* aux = (MODE == BRS_ROUND_ERRFEEDBACK) ? (uint16_t*)a.aux + (size_t)head * nlo * kD : nullptr;
   float* S0g = a.s0 + (size_t)head * kD * kD;      // FP32 state between chunks
-  float* gam = (float*)(smem + kOffGam);           // Gamma [64 t][128 i]
+  float* Kt = (float*)(smem + kOffKt);
+  float* Kh = (float*)(smem + kOffKh);
+  float* Qt = (float*)(smem + kOffQt);
+  float* g63 = (float*)(smem + kOffG63);
   float* betas = (float*)(smem + kOffBeta);
-  unsigned long long* bars = (unsigned long long*)(smem + kOffMisc);   // slice buffers 0, 1; phase 2
+  unsigned long long* bars = (unsigned long long*)(smem + kOffMisc);   // phase 1, phase 2
   uint32_t* tslot = (uint32_t*)(smem + kOffMisc + 32);
+  int16_t* permS = (int16_t*)(smem + kOffPerm);
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = smem_u32(&bars[0]);
   uint32_t err = 0;
@@ -284,10 +299,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   if (tid == 0) {
-#pragma unroll
-    for (int i = 0; i < 3; ++i) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar0 + 8u * i));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar0));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar0 + 8u));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  if (tid < kD) permS[tid] = a.perm ? a.perm[h * kD + tid] : (int16_t)tid;
   tc_load_state<HAD, BLOCK>(hst, S0g, nlo, a.k_hi, a.hscale);
   tc_fence_before();
   __syncthreads();
@@ -296,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
   const uint32_t tD2 = tm, tD1 = tm + 128, tD4 = tm + 256;
   const uint32_t lrow = (uint32_t)(32 * sub) << 16;          // this warp's lane base in tensor memory
   const int myrow = 32 * sub + lane;                          // the tensor-memory lane this thread reads
-  uint32_t ph0 = 0, ph1 = 0, ph2 = 0;
+  uint32_t ph0 = 0, ph1 = 0;
   bool alive = true;
   // every thread waits; the CTA agrees on the outcome
   auto wait_all = [&](int which, uint32_t& ph) -> bool {
@@ -309,55 +325,60 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
   for (int ch = 0; ch < nchunks && alive; ++ch) {
     const int t0 = ch * kC;
     const size_t tokb = (size_t)b * a.T + t0;                 // first token of the chunk
-    // ---- Gamma (cumulative decay per stored row) and beta
-    if (tid < kD) {
-      const int p = a.perm ? a.perm[h * kD + tid] : tid;
-      float g = 1.0f;
-      for (int r = 0; r < kC; ++r) {
-        const size_t tok = tokb + r;
-        const float av = a.decay_per_key ? a.decay[(tok * a.H + h) * kD + p] : a.decay[tok * a.H + h];
-        g = __fmul_rn(g, av);
-        gam[r * kD + tid] = g;
+    // ---- chunk inputs: thread (row i, quarter qq) takes tokens 16 qq .. 16 qq + 15
+    // of stored row i: cumulative decay (local products, then the earlier
+    // quarters' totals), K~ = K Gamma, K^ = K (1 / Gamma), Q~ = Q Gamma
+    {
+      const int i = tid & 127, qq = tid >> 7, p = permS[i];
+      float av[16], kv[16], qv[16];
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {                 // all loads in flight at once
+        const size_t tok = tokb + 16 * qq + r;
+        av[r] = a.decay_per_key ? a.decay[(tok * a.H + h) * kD + p] : a.decay[tok * a.H + h];
+        kv[r] = bf16_to_f32(a.k[(tok * a.Hk + kh) * kD + p]);
+        qv[r] = bf16_to_f32(a.q[(tok * a.Hk + kh) * kD + p]);
       }
-    } else if (tid < kD + kC) {
-      betas[tid - kD] = a.beta[(tokb + (tid - kD)) * a.H + h];
+      if (tid < kC) betas[tid] = a.beta[(tokb + tid) * a.H + h];
+#pragma unroll
+      for (int r = 1; r < 16; ++r) av[r] = __fmul_rn(av[r - 1], av[r]);
+      float* tot = (float*)(smem + kOffSlice);       // [4][128] quarter totals
+      tot[qq * kD + i] = av[15];
+      __syncthreads();
+      float carry = 1.0f;
+      for (int u = 0; u < qq; ++u) carry = __fmul_rn(carry, tot[u * kD + i]);
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        const float g = qq ? __fmul_rn(carry, av[r]) : av[r];
+        const int t = 16 * qq + r;
+        Kt[t * kRS + i] = __fmul_rn(kv[r], g);
+        Kh[t * kRS + i] = __fmul_rn(kv[r], __frcp_rn(g));
+        Qt[t * kRS + i] = __fmul_rn(qv[r], g);
+        if (t == kC - 1) g63[i] = g;
+      }
+      __syncthreads();
     }
-    __syncthreads();
 
     // ---- phase 1: D1 = [K~;Q~] K^^T, D2 = S_0^T [K~;Q~]^T over 4 slices of
-    // 32 stored rows i, the slices double-buffered against the MMAs
-    for (int sl = 0; sl < kD / kSl && alive; ++sl) {
-      const int buf = sl & 1;
-      if (sl >= 2) {
-        alive = buf ? wait_all(1, ph1) : wait_all(0, ph0);
+    // 32 stored rows i (one slice buffer)
+    for (int sl = 0; sl < kD / kSl; ++sl) {
+      if (sl > 0) {
+        alive = wait_all(0, ph0);                    // the previous slice's MMAs read the buffer
         if (!alive) break;
       }
-      uint8_t* B0 = smem + buf * kBuf;
+      uint8_t* B0 = smem + kOffSlice;
       uint8_t *KQh = B0, *KQl = B0 + kKQ, *KHh = B0 + 2 * kKQ, *KHl = KHh + kKH, *STh = KHl + kKH, *STl = STh + kS0T;
       const int i0 = sl * kSl;
-      for (int task = tid; task < 2560; task += kThreads) {
-        if (task < 1024) {                           // [K~;Q~] rows t, 4 columns 4g..4g+3 of the slice
+#pragma unroll
+      for (int q = 0; q < 2560 / kThreads; ++q) {
+        const int task = tid + q * kThreads;
+        if (q < 1024 / kThreads) {                   // [K~;Q~] rows t, columns 4g .. 4g+3 of the slice
           const int t = task & 127, g = task >> 7;
-          const int tt = t & 63;
-          const uint16_t* src = (t < 64) ? a.k : a.q;
-          float x[4];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int i = i0 + 4 * g + c;
-            const int p = a.perm ? a.perm[h * kD + i] : i;
-            x[c] = __fmul_rn(bf16_to_f32(src[((tokb + tt) * a.Hk + kh) * kD + p]), gam[tt * kD + i]);
-          }
-          st_split4(KQh, KQl, kmaj(t, 4 * g, kSl), x[0], x[1], x[2], x[3]);
-        } else if (task < 1536) {                    // K^ rows s
+          const float4 x = *(const float4*)((t < 64) ? &Kt[t * kRS + i0 + 4 * g] : &Qt[(t - 64) * kRS + i0 + 4 * g]);
+          st_split4(KQh, KQl, kmaj(t, 4 * g, kSl), x.x, x.y, x.z, x.w);
+        } else if (q < 1536 / kThreads) {            // K^ rows s
           const int u = task - 1024, s = u & 63, g = u >> 6;
-          float x[4];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int i = i0 + 4 * g + c;
-            const int p = a.perm ? a.perm[h * kD + i] : i;
-            x[c] = __fdiv_rn(bf16_to_f32(a.k[((tokb + s) * a.Hk + kh) * kD + p]), gam[s * kD + i]);
-          }
-          st_split4(KHh, KHl, kmaj(s, 4 * g, kSl), x[0], x[1], x[2], x[3]);
+          const float4 x = *(const float4*)&Kh[s * kRS + i0 + 4 * g];
+          st_split4(KHh, KHl, kmaj(s, 4 * g, kSl), x.x, x.y, x.z, x.w);
         } else {                                     // S_0^T rows j
           const int u = task - 1536, j = u & 127, g = u >> 7;
           const int i = i0 + 4 * g;
@@ -370,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
       __syncthreads();
       if (tid == 0) {
         tc_fence_after();
-        const uint32_t base = sbase + buf * kBuf;
+        const uint32_t base = sbase + kOffSlice;
         const uint32_t aKQh = base, aKQl = base + kKQ, aKHh = base + 2 * kKQ, aKHl = aKHh + kKH;
         const uint32_t aSTh = aKHl + kKH, aSTl = aSTh + kS0T;
         constexpr uint32_t sbo = (kSl / 4) * 128;
@@ -380,22 +401,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
           umma3(tD1, aKQh + o, aKQl + o, aKHh + o, aKHl + o, sbo, sbo, idesc_tf32(128, 64), acc);
           umma3(tD2, aSTh + o, aSTl + o, aKQh + o, aKQl + o, sbo, sbo, idesc_tf32(128, 128), acc);
         }
-        umma_commit(bar0 + 8u * buf);
+        umma_commit(bar0);
       }
     }
     if (!alive) break;
-    alive = wait_all(0, ph0) && wait_all(1, ph1);
+    alive = wait_all(0, ph0);
     if (!alive) break;
     tc_fence_after();
 
-    // ---- readouts of D1: A = strictly-lower(diag(beta) K~ K^T) (fp32, shared),
-    // P = lower-incl(Q~ K^T) as the split operand X[t][s]
-    float* Am = (float*)(smem + kOffA);
-    {
-      float v[16];
+    if (part == 0) {
+      // ---- D1: A = strictly-lower(diag(beta) K~ K^T) (fp32), P = lower-incl(Q~ K^T)
+      // as the split operand X[t][s]
+      float* Am = (float*)(smem + kOffA);
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const int c0 = 32 * half + 16 * q;
+      for (int q = 0; q < 4; ++q) {
+        float v[16];
+        const int c0 = 16 * q;
         tmem_ld16(tD1 + lrow + c0, v);
         if (myrow < 64) {
           const int t = myrow;
@@ -414,14 +435,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
                       (c0 + c + 3 <= t) ? v[c + 3] : 0.0f);
         }
       }
-    }
-    __syncthreads();
-
-    if (half == 0) {
+      asm volatile("bar.sync 1, 128;" ::: "memory");   // A complete for the 128 column threads
       // ---- W by forward substitution, one value column j per thread:
       // (I + A) W = diag(beta)(V - K~ S_0), the right side from D2[j][0..63]
       const int j = myrow;
       float w[kC];
+#pragma unroll
+      for (int t = 0; t < kC; ++t) w[t] = bf16_to_f32(a.v[((tokb + t) * a.H + h) * kD + j]);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         float v[16];
@@ -429,8 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           const int t = 16 * q + c;
-          const float vv = bf16_to_f32(a.v[((tokb + t) * a.H + h) * kD + j]);
-          w[t] = __fmul_rn(betas[t], __fsub_rn(vv, v[c]));
+          w[t] = __fmul_rn(betas[t], __fsub_rn(w[t], v[c]));
         }
       }
 #pragma unroll
@@ -450,18 +469,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
       for (int s = 0; s < kC; s += 4)
         st_split4(smem + kOffW, smem + kOffW + kWt, kmaj(j, s, 64), w[s], w[s + 1], w[s + 2], w[s + 3]);
     } else {
-      // ---- K^ transposed: X[i][s] = K[s][p_i] / Gamma[s][i]
-      const int tl = tid - 128;
-      for (int task = tl; task < kD * (kC / 4); task += 128) {
+      // ---- K^ transposed: X[i][s] = K^[s][i]
+      for (int task = tid - 128; task < kD * (kC / 4); task += kThreads - 128) {
         const int i = task & 127, sg = task >> 7;
-        const int p = a.perm ? a.perm[h * kD + i] : i;
-        float x[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int s = 4 * sg + c;
-          x[c] = __fdiv_rn(bf16_to_f32(a.k[((tokb + s) * a.Hk + kh) * kD + p]), gam[s * kD + i]);
-        }
-        st_split4(smem + kOffKT, smem + kOffKT + kKT, kmaj(i, 4 * sg, 64), x[0], x[1], x[2], x[3]);
+        st_split4(smem + kOffKT, smem + kOffKT + kKT, kmaj(i, 4 * sg, 64), Kh[(4 * sg) * kRS + i],
+                  Kh[(4 * sg + 1) * kRS + i], Kh[(4 * sg + 2) * kRS + i], Kh[(4 * sg + 3) * kRS + i]);
       }
     }
     proxy_fence();
@@ -479,9 +491,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
         umma3(tD2 + 64, aWh + o, aWl + o, aPh + o, aPl + o, sbo, sbo, idesc_tf32(128, 64), 1u);
         umma3(tD4, aKTh + o, aKTl + o, aWh + o, aWl + o, sbo, sbo, idesc_tf32(128, 128), k > 0 ? 1u : 0u);
       }
-      umma_commit(bar0 + 16u);
+      umma_commit(bar0 + 8u);
     }
-    alive = wait_all(2, ph2);
+    alive = wait_all(1, ph1);
     if (!alive) break;
     tc_fence_after();
 
@@ -492,8 +504,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
       float v[16];
       bool bad = false;
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const int c0 = 32 * half + 16 * q;
+      for (int q = 0; q < 64 / kParts / 16; ++q) {
+        const int c0 = (64 / kParts) * part + 16 * q;
         tmem_ld16(tD2 + lrow + 64 + c0, v);
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
@@ -504,17 +516,21 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
       if (bad) err |= BRS_FLAG_NONFINITE;
       float* Ss = (float*)smem;
       const int i = myrow;
-      const float g63 = gam[63 * kD + i];
+      const float gi = g63[i];
+      constexpr int kCols = kD / kParts;             // this thread's columns of its row
+      float4 s0v[kCols / 4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int c0 = 64 * half + 16 * q;
+      for (int c = 0; c < kCols / 4; ++c) s0v[c] = *(const float4*)&S0g[(size_t)i * kD + kCols * part + 4 * c];
+#pragma unroll
+      for (int q = 0; q < kCols / 16; ++q) {
+        const int c0 = kCols * part + 16 * q;
         tmem_ld16(tD4 + lrow + c0, v);
 #pragma unroll
         for (int c = 0; c < 16; c += 4) {
-          const float4 s4 = *(const float4*)&S0g[(size_t)i * kD + c0 + c];
+          const float4 s4 = s0v[4 * q + c / 4];
           *(float4*)&Ss[i * kSStride + c0 + c] =
-              make_float4(__fmul_rn(g63, __fadd_rn(s4.x, v[c])), __fmul_rn(g63, __fadd_rn(s4.y, v[c + 1])),
-                          __fmul_rn(g63, __fadd_rn(s4.z, v[c + 2])), __fmul_rn(g63, __fadd_rn(s4.w, v[c + 3])));
+              make_float4(__fmul_rn(gi, __fadd_rn(s4.x, v[c])), __fmul_rn(gi, __fadd_rn(s4.y, v[c + 1])),
+                          __fmul_rn(gi, __fadd_rn(s4.z, v[c + 2])), __fmul_rn(gi, __fadd_rn(s4.w, v[c + 3])));
         }
       }
     }
