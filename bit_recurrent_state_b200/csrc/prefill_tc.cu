@@ -141,6 +141,20 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int c = 0; c < 16; ++c) v[c] = __uint_as_float(r[c]);
 }
 
+// fl(x / 255) for any float x, as fl32(fl64(x * fl64(1/255))): the quotient
+// of a float by 255 stays at least 2^-33 (relative) from every float
+// rounding midpoint while the double product is within 2^-52 of it
+__device__ __forceinline__ float div255(float x) { return (float)((double)x * (1.0 / 255.0)); }
+// fl(1 / s) for s a positive binary16 value: one Newton-Raphson correction
+// of the hardware approximation (exact residual; 1/s for an 11-bit s stays
+// at least 2^-36 from every midpoint, the corrected value within 2^-40)
+__device__ __forceinline__ float rcp_of_f16(float s) {
+  float r0;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r0) : "f"(s));
+  const float e = __fmaf_rn(-s, r0, 1.0f);
+  return __fmaf_rn(r0, e, r0);
+}
+
 // the operand split: hi = x truncated to TF32, lo = x - hi (exact)
 __device__ __forceinline__ float tf32_hi(float x) { return __uint_as_float(__float_as_uint(x) & 0xFFFFE000u); }
 // store 4 consecutive-K values of row r at (hi tile, lo tile)
@@ -211,10 +225,15 @@ __device__ void tc_store_state(const float* Ss, float* S, uint8_t* head, uint16_
     }
     float mn = fminf(fminf(x[0], x[1]), fminf(x[2], x[3]));
     float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+    if constexpr (GL == 32) {
+      asm volatile("redux.sync.min.f32 %0, %0, 0xffffffff;" : "+f"(mn));
+      asm volatile("redux.sync.max.f32 %0, %0, 0xffffffff;" : "+f"(mx));
+    } else {
 #pragma unroll
-    for (int m = 1; m < GL; m <<= 1) {
-      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, m));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
+      for (int m = 1; m < GL; m <<= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, m));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
+      }
     }
     if (mn == 0.0f || mx == 0.0f) {             // -0 ranks below +0 (uniform per block group)
       bool nz = false, pz = false;
@@ -229,11 +248,11 @@ __device__ void tc_store_state(const float* Ss, float* S, uint8_t* head, uint16_
       if (mx == 0.0f) mx = apz ? 0.0f : -0.0f;
     }
     if (!isfinite(mn) || !isfinite(mx)) err |= BRS_FLAG_NONFINITE;
-    const uint16_t sh = f32_to_f16(__fdiv_rn(__fsub_rn(mx, mn), 255.0f));
-    const uint16_t zh = f32_to_f16(mn);
+    const uint32_t gz = f16x2_of(div255(__fsub_rn(mx, mn)), mn);    // lo scale, hi zero
+    const uint16_t sh = (uint16_t)(gz & 0xffffu), zh = (uint16_t)(gz >> 16);
     if (f16_inf_or_nan(sh) || f16_inf_or_nan(zh)) err |= BRS_FLAG_OVERFLOW;
     const float s = f16_to_f32(sh), z = f16_to_f32(zh);
-    const float rcp = (s == 0.0f) ? 0.0f : __frcp_rn(s);
+    const float rcp = (s == 0.0f) ? 0.0f : rcp_of_f16(s);
     uint4 rnd = make_uint4(0, 0, 0, 0);
     if (MODE == BRS_ROUND_STOCHASTIC)
       rnd = philox4x32_10(make_uint4((uint32_t)(r * (kD / 4) + lane), (uint32_t)step, (uint32_t)h, (uint32_t)b),
@@ -244,13 +263,14 @@ __device__ void tc_store_state(const float* Ss, float* S, uint8_t* head, uint16_
     uint16_t e16[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      float code = 0.0f;
-      if (s != 0.0f) {
-        const float tt = __fmul_rn(__fsub_rn(x[c], z), rcp);
-        code = (MODE == BRS_ROUND_STOCHASTIC) ? sr_round(tt, rw[c]) : rintf(tt);
-        code = fminf(fmaxf(code, 0.0f), 255.0f);
-      }
-      packed4 |= ((uint32_t)(int)code) << (8 * c);
+      // a zero scale has 1/scale = 0: every code is 0
+      float tt = __fmul_rn(__fsub_rn(x[c], z), rcp);
+      if (MODE == BRS_ROUND_STOCHASTIC) tt = sr_round(tt, rw[c]);
+      // clip, then the nearest integer (ties to even) as the low byte of
+      // t + 1.5*2^23 (exact for the integers SR produces)
+      const float m = __fadd_rn(fminf(fmaxf(tt, 0.0f), 255.0f), kRoundMagic);
+      const float code = __fsub_rn(m, kRoundMagic);
+      packed4 |= (__float_as_uint(m) & 0xffu) << (8 * c);
       xh[c] = __fmaf_rn(code, s, z);
       if (MODE == BRS_ROUND_ERRFEEDBACK) {
         float e = __fsub_rn(x[c], xh[c]);
@@ -361,13 +381,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
     // ---- phase 1: D1 = [K~;Q~] K^^T, D2 = S_0^T [K~;Q~]^T over 4 slices of
     // 32 stored rows i (one slice buffer)
     for (int sl = 0; sl < kD / kSl; ++sl) {
+      const int i0 = sl * kSl;
+      // this thread's two S_0^T tasks (rows j, 4 stored rows i each), loaded
+      // from the global scratch while the previous slice's MMAs run
+      float pre[2][4];
+#pragma unroll
+      for (int q2 = 0; q2 < 2; ++q2) {
+        const int u = tid + q2 * kThreads, j = u & 127, i = i0 + 4 * (u >> 7);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) pre[q2][c] = S0g[(size_t)(i + c) * kD + j];
+      }
       if (sl > 0) {
         alive = wait_all(0, ph0);                    // the previous slice's MMAs read the buffer
         if (!alive) break;
       }
       uint8_t* B0 = smem + kOffSlice;
       uint8_t *KQh = B0, *KQl = B0 + kKQ, *KHh = B0 + 2 * kKQ, *KHl = KHh + kKH, *STh = KHl + kKH, *STl = STh + kS0T;
-      const int i0 = sl * kSl;
 #pragma unroll
       for (int q = 0; q < 2560 / kThreads; ++q) {
         const int task = tid + q * kThreads;
@@ -381,9 +410,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
           st_split4(KHh, KHl, kmaj(s, 4 * g, kSl), x.x, x.y, x.z, x.w);
         } else {                                     // S_0^T rows j
           const int u = task - 1536, j = u & 127, g = u >> 7;
-          const int i = i0 + 4 * g;
-          st_split4(STh, STl, kmaj(j, 4 * g, kSl), S0g[(size_t)i * kD + j], S0g[(size_t)(i + 1) * kD + j],
-                    S0g[(size_t)(i + 2) * kD + j], S0g[(size_t)(i + 3) * kD + j]);
+          const int q2 = (q * kThreads - 1536) / kThreads;
+          st_split4(STh, STl, kmaj(j, 4 * g, kSl), pre[q2][0], pre[q2][1], pre[q2][2], pre[q2][3]);
         }
       }
       proxy_fence();
@@ -405,6 +433,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
       }
     }
     if (!alive) break;
+    if (part == 0) {                                 // the chunk's V rows into L1 while the MMAs run
+      const uint16_t* vrow = a.v + ((tokb + (myrow & 63)) * a.H + h) * kD + 64 * (myrow >> 6);
+      asm volatile("prefetch.global.L1 [%0];" ::"l"(vrow));
+    }
     alive = wait_all(0, ph0);
     if (!alive) break;
     tc_fence_after();
@@ -452,18 +484,31 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
           w[t] = __fmul_rn(betas[t], __fsub_rn(w[t], v[c]));
         }
       }
+      // blocks of 16 rows: the terms from earlier blocks are 16 independent
+      // sums, then the block's own triangle is solved row by row
 #pragma unroll
-      for (int t = 1; t < kC; ++t) {
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int B = 0; B < kC / 16; ++B) {
+        float acc[16];
 #pragma unroll
-        for (int s = 0; s < t; s += 4) {
-          const float4 a4 = *(const float4*)&Am[t * kAStride + s];
-          acc[0] = __fmaf_rn(a4.x, w[s], acc[0]);
-          if (s + 1 < t) acc[1] = __fmaf_rn(a4.y, w[s + 1], acc[1]);
-          if (s + 2 < t) acc[2] = __fmaf_rn(a4.z, w[s + 2], acc[2]);
-          if (s + 3 < t) acc[3] = __fmaf_rn(a4.w, w[s + 3], acc[3]);
+        for (int r = 0; r < 16; ++r) acc[r] = 0.0f;
+#pragma unroll
+        for (int s = 0; s < 16 * B; s += 4)
+#pragma unroll
+          for (int r = 0; r < 16; ++r) {
+            const float4 a4 = *(const float4*)&Am[(16 * B + r) * kAStride + s];
+            acc[r] = __fmaf_rn(a4.x, w[s], acc[r]);
+            acc[r] = __fmaf_rn(a4.y, w[s + 1], acc[r]);
+            acc[r] = __fmaf_rn(a4.z, w[s + 2], acc[r]);
+            acc[r] = __fmaf_rn(a4.w, w[s + 3], acc[r]);
+          }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+          const int t = 16 * B + r;
+          float x = acc[r];
+#pragma unroll
+          for (int s = 16 * B; s < t; ++s) x = __fmaf_rn(Am[t * kAStride + s], w[s], x);
+          w[t] = __fsub_rn(w[t], x);
         }
-        w[t] = __fsub_rn(w[t], __fadd_rn(__fadd_rn(acc[0], acc[1]), __fadd_rn(acc[2], acc[3])));
       }
 #pragma unroll
       for (int s = 0; s < kC; s += 4)
@@ -493,6 +538,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
       }
       umma_commit(bar0 + 8u);
     }
+    constexpr int kCols = kD / kParts;               // this thread's columns of its S row
+    float4 s0v[kCols / 4];                           // S_0 row part, loaded while the MMAs run
+#pragma unroll
+    for (int c = 0; c < kCols / 4; ++c) s0v[c] = *(const float4*)&S0g[(size_t)myrow * kD + kCols * part + 4 * c];
     alive = wait_all(1, ph1);
     if (!alive) break;
     tc_fence_after();
@@ -517,10 +566,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
       float* Ss = (float*)smem;
       const int i = myrow;
       const float gi = g63[i];
-      constexpr int kCols = kD / kParts;             // this thread's columns of its row
-      float4 s0v[kCols / 4];
-#pragma unroll
-      for (int c = 0; c < kCols / 4; ++c) s0v[c] = *(const float4*)&S0g[(size_t)i * kD + kCols * part + 4 * c];
 #pragma unroll
       for (int q = 0; q < kCols / 16; ++q) {
         const int c0 = kCols * part + 16 * q;
