@@ -111,7 +111,6 @@ struct PrefillArgs {
   uint32_t* flags;
   float* s0;                     // scratch [B][H][d][d]: the FP32 state between chunks
 };
-cudaError_t launch_prefill(const PrefillArgs& a, bool had, cudaStream_t st);
 size_t prefill_tc_scratch_bytes(int B, int H);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, bool had, cudaStream_t st);
 bool prefill_supported(int d, int block, int k_hi, int C);

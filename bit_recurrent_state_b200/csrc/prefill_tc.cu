@@ -4,10 +4,10 @@
 // (hi*hi + hi*lo + lo*hi, hi = the operand truncated to TF32, lo = the
 // remainder) so the contractions keep FP32-level accuracy; the forward
 // substitution, the masks, the requantization and the write-back run on
-// the CUDA cores.  Same math and the same write-back protocol as the
-// CUDA-core prefill ("Low-Bit Recurrent States in Hybrid Language Models",
-// Accumulated readout error: write-back once per prefill chunk; Protocol:
-// quantized and dequantized before reuse):
+// the CUDA cores.  The state is written back once per chunk ("Low-Bit
+// Recurrent States in Hybrid Language Models", Accumulated readout error:
+// write-back once per prefill chunk; Protocol: quantized and dequantized
+// before reuse).  The chunk in WY form:
 //   Gamma_t = prod_{r <= t} a_r, K~ = K * Gamma, K^ = K * (1 / Gamma), Q~ = Q * Gamma;
 //   A = strictly-lower(diag(beta) K~ K^T);  (I + A) W = diag(beta)(V - K~ S_0);
 //   O = Q~ S_0 + lower-incl(Q~ K^T) W;  S_C = diag(Gamma_63)(S_0 + K^T W).
@@ -615,6 +615,10 @@ cudaError_t tc_launch_hb(const PrefillArgs& a, cudaStream_t st) {
 }
 
 }  // namespace
+
+bool prefill_supported(int d, int block, int k_hi, int C) {
+  return d == kD && C == kC && (block == 128 || block == 32) && k_hi % 4 == 0 && k_hi <= kD;
+}
 
 size_t prefill_tc_scratch_bytes(int B, int H) { return (size_t)B * H * kD * kD * sizeof(float); }
 
