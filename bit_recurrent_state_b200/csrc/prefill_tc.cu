@@ -91,12 +91,14 @@ __device__ __forceinline__ void umma_tf32(uint32_t d, uint64_t a, uint64_t b, ui
       "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
       "l"(a), "l"(b), "r"(idesc), "r"(acc));
 }
-// 3-way split product: D (+)= Ah Bh + Ah Bl + Al Bh
-__device__ __forceinline__ void umma3(uint32_t d, uint32_t ah, uint32_t al, uint32_t bh, uint32_t bl, uint32_t sboa,
-                                      uint32_t sbob, uint32_t idesc, uint32_t acc) {
-  umma_tf32(d, sdesc(ah, sboa), sdesc(bh, sbob), idesc, acc);
-  umma_tf32(d, sdesc(ah, sboa), sdesc(bl, sbob), idesc, 1u);
-  umma_tf32(d, sdesc(al, sboa), sdesc(bh, sbob), idesc, 1u);
+// 3-way split product D (+)= Ah Bh + Ah Bl + Al Bh from prebuilt hi/lo operand
+// descriptors; off16 = byte offset / 16 added to the start-address field (no
+// carry: shared addresses are below 256 KB)
+__device__ __forceinline__ void umma3d(uint32_t d, uint64_t ah, uint64_t al, uint64_t bh, uint64_t bl, uint32_t off16,
+                                       uint32_t idesc, uint32_t acc) {
+  umma_tf32(d, ah + off16, bh + off16, idesc, acc);
+  umma_tf32(d, ah + off16, bl + off16, idesc, 1u);
+  umma_tf32(d, al + off16, bh + off16, idesc, 1u);
 }
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
@@ -423,11 +425,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
         const uint32_t aKQh = base, aKQl = base + kKQ, aKHh = base + 2 * kKQ, aKHl = aKHh + kKH;
         const uint32_t aSTh = aKHl + kKH, aSTl = aSTh + kS0T;
         constexpr uint32_t sbo = (kSl / 4) * 128;
+        const uint64_t dKQh = sdesc(aKQh, sbo), dKQl = sdesc(aKQl, sbo), dKHh = sdesc(aKHh, sbo),
+                       dKHl = sdesc(aKHl, sbo), dSTh = sdesc(aSTh, sbo), dSTl = sdesc(aSTl, sbo);
 #pragma unroll
         for (int k = 0; k < kSl / 8; ++k) {
-          const uint32_t o = 256u * k, acc = (sl > 0 || k > 0) ? 1u : 0u;
-          umma3(tD1, aKQh + o, aKQl + o, aKHh + o, aKHl + o, sbo, sbo, idesc_tf32(128, 64), acc);
-          umma3(tD2, aSTh + o, aSTl + o, aKQh + o, aKQl + o, sbo, sbo, idesc_tf32(128, 128), acc);
+          const uint32_t o16 = 16u * k, acc = (sl > 0 || k > 0) ? 1u : 0u;
+          umma3d(tD1, dKQh, dKQl, dKHh, dKHl, o16, idesc_tf32(128, 64), acc);
+          umma3d(tD2, dSTh, dSTl, dKQh, dKQl, o16, idesc_tf32(128, 128), acc);
         }
         umma_commit(bar0);
       }
@@ -530,11 +534,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
       const uint32_t aWh = sbase + kOffW, aWl = aWh + kWt, aKTh = sbase + kOffKT, aKTl = aKTh + kKT;
       const uint32_t aPh = sbase + kOffP, aPl = aPh + kPt;
       constexpr uint32_t sbo = (64 / 4) * 128;
+      const uint64_t dWh = sdesc(aWh, sbo), dWl = sdesc(aWl, sbo), dKTh = sdesc(aKTh, sbo), dKTl = sdesc(aKTl, sbo),
+                     dPh = sdesc(aPh, sbo), dPl = sdesc(aPl, sbo);
 #pragma unroll
       for (int k = 0; k < kC / 8; ++k) {
-        const uint32_t o = 256u * k;
-        umma3(tD2 + 64, aWh + o, aWl + o, aPh + o, aPl + o, sbo, sbo, idesc_tf32(128, 64), 1u);
-        umma3(tD4, aKTh + o, aKTl + o, aWh + o, aWl + o, sbo, sbo, idesc_tf32(128, 128), k > 0 ? 1u : 0u);
+        const uint32_t o16 = 16u * k;
+        umma3d(tD2 + 64, dWh, dWl, dPh, dPl, o16, idesc_tf32(128, 64), 1u);
+        umma3d(tD4, dKTh, dKTl, dWh, dWl, o16, idesc_tf32(128, 128), k > 0 ? 1u : 0u);
       }
       umma_commit(bar0 + 8u);
     }
