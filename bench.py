@@ -68,6 +68,22 @@ def algorithmic_bytes(w) -> dict:
                 total=2 * n + inputs + out + ef + st)
 
 
+def rank_workload(w, rank: int):
+    """A rank's own batch: the same shape, its own sequences (seed offset by
+    rank).  Units are independent, so ranks exchange nothing on the data path."""
+    return w.with_(seed=w.seed + 1000 * rank)
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The job's time for a per-rank time: its maximum over the ranks."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def kernel_name(w) -> str:
     """The kernel a decode step of workload w launches (the dominant one)."""
     if w.storage == "varbit":
@@ -319,7 +335,7 @@ def run_prefill(args, w):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
-    wr = w.with_(seed=w.seed + 1000 * rank)
+    wr = rank_workload(w, rank)
     L, wb = brs.layout_of(wr), brs.writeback_of(wr)
     rng = np.random.default_rng(wr.seed)
     perm = np.stack([rng.permutation(w.d) for _ in range(w.H)]).astype(np.int16)
@@ -353,11 +369,7 @@ def run_prefill(args, w):
             step(i)
         ev1.record(stream)
         barrier()
-    ms = ev0.elapsed_time(ev1)
-    t = torch.tensor([ms], device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_step = float(t.item()) / args.steps
+    ms_step = max_over_ranks(ev0.elapsed_time(ev1), world, dev) / args.steps
     flags = st.errors()
     # end to end: inputs copied from pinned host memory and o read back every step
     pinned = {k: v.pin_memory() for k, v in host.items()}
@@ -371,10 +383,7 @@ def run_prefill(args, w):
         o_host.copy_(o, non_blocking=True)
     ev1.record(stream)
     barrier()
-    t = torch.tensor([ev0.elapsed_time(ev1)], device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_e2e = float(t.item()) / args.steps
+    ms_e2e = max_over_ranks(ev0.elapsed_time(ev1), world, dev) / args.steps
     units = w.B * w.H * w.T * world
     n, aux, _, _ = brs.state_bytes(L)
     chunks = w.T // 64
@@ -433,7 +442,7 @@ def run_ours(args, w):
     stream = torch.cuda.current_stream()
 
     # per-rank workload: same shape, own sequences (seed offset by rank)
-    wr = w.with_(seed=w.seed + 1000 * rank)
+    wr = rank_workload(w, rank)
     L = brs.layout_of(wr)
     wb = brs.writeback_of(wr)
     rng = np.random.default_rng(wr.seed)
@@ -485,11 +494,7 @@ def run_ours(args, w):
             step(args.warmup + i)
         ev1.record(stream)
         barrier()
-    ms = ev0.elapsed_time(ev1)
-    t = torch.tensor([ms], device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     ms_step = ms_max / args.steps
 
     # ---- end to end through the public API with host buffers
@@ -505,11 +510,7 @@ def run_ours(args, w):
         o_host.copy_(o, non_blocking=True)
     ev1.record(stream)
     barrier()
-    ms_e2e = ev0.elapsed_time(ev1)
-    t = torch.tensor([ms_e2e], device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_e2e = float(t.item())
+    ms_e2e = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     flags |= layers[0].errors()
 
     units = w.B * w.H * world
