@@ -15,6 +15,7 @@ struct DecodeArgs {
   int64_t step;
   size_t head_bytes;
   float hscale;                  // float nearest 1/sqrt(d)
+  float one = 1.0f;              // 1 read at run time: a multiplier the compiler cannot fold
   const void* packed_in;
   void* packed_out;
   void* aux;
@@ -81,6 +82,7 @@ struct VbArgs {
   uint64_t seed;
   int64_t step;
   double lambda, avg_bits;
+  float one = 1.0f;              // 1 read at run time: a multiplier the compiler cannot fold
   VbSections sec;
   const void* packed_in;
   void* packed_out;

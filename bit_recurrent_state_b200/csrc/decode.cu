@@ -549,11 +549,14 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
 #pragma unroll
           for (int c = 0; c < C; ++c) tq[c] = fminf(fmaxf(tq[c], 0.0f), 255.0f);
         }
-        // nearest integer (ties to even): the low byte of t + 1.5*2^23
+        // nearest integer (ties to even): the low byte of t + 1.5*2^23; the
+        // paired add is written t * one + magic with one = 1 read at run
+        // time (the same single rounding), so it cannot be merged with the
+        // multiply before it
         float mq[C];
 #pragma unroll
         for (int c = 0; c < C; c += (C >= 2 ? 2 : 1)) {
-          if constexpr (C >= 2) add2(mq[c], mq[c + 1], tq[c], tq[c + 1], kRoundMagic, kRoundMagic);
+          if constexpr (C >= 2) fma2(mq[c], mq[c + 1], tq[c], tq[c + 1], a.one, a.one, kRoundMagic, kRoundMagic);
           else mq[c] = __fadd_rn(tq[c], kRoundMagic);
         }
         uint8_t* dst = hout + (size_t)i * D + col0;

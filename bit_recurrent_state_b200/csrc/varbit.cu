@@ -226,8 +226,10 @@ __global__ void __launch_bounds__(32 * kVbWarps) varbit_kernel(const VbArgs a) {
         float t0, t1, t2, t3;
         mul2(t0, t1, y, y, iv[0], iv[1]);
         mul2(t2, t3, y, y, iv[2], iv[3]);
-        add2(t0, t1, t0, t1, kRoundMagic, kRoundMagic);   // nearest integer (ties to even)
-        add2(t2, t3, t2, t3, kRoundMagic, kRoundMagic);
+        // nearest integer (ties to even); t * one + magic with one = 1 read at
+        // run time, the add's single rounding, never merged with the multiply
+        fma2(t0, t1, t0, t1, a.one, a.one, kRoundMagic, kRoundMagic);
+        fma2(t2, t3, t2, t3, a.one, a.one, kRoundMagic, kRoundMagic);
         sub2(t0, t1, t0, t1, kRoundMagic, kRoundMagic);
         sub2(t2, t3, t2, t3, kRoundMagic, kRoundMagic);
         t0 = fminf(fmaxf(t0, -fn), fn);
