@@ -464,16 +464,17 @@ def run_ours(args, w):
     o = torch.zeros((w.B, w.H, w.d), dtype=torch.float32, device=dev)
     o_host = torch.zeros_like(o, device="cpu").pin_memory()
 
-    def step(i):
+    def step(i, out=None):
         l = i % NLAYERS
         st = layers[l]
         x = inputs[l]
+        out = o if out is None else out
         if varbit:
             # variable-width states change their row offsets: write to the other buffer
-            spares[l] = st.step(wb, i, x["q"], x["k"], x["v"], x["beta"], x["decay"], o,
+            spares[l] = st.step(wb, i, x["q"], x["k"], x["v"], x["beta"], x["decay"], out,
                                 packed_out=spares[l])
         else:
-            st.step(wb, i, x["q"], x["k"], x["v"], x["beta"], x["decay"], o)
+            st.step(wb, i, x["q"], x["k"], x["v"], x["beta"], x["decay"], out)
 
     for i in range(args.warmup):
         step(i)
@@ -497,17 +498,52 @@ def run_ours(args, w):
     ms_max = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     ms_step = ms_max / args.steps
 
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers: every token's
+    # inputs are copied from pinned host memory and its o read back inside the
+    # timed region.  Copies run on their own streams (host to device on one,
+    # device to host on another) so that token i+1's inputs and token i-1's
+    # output move while token i's kernel runs; events order each buffer's reuse
+    # (an input set is rewritten only after the kernel that read it, an o
+    # buffer only after its read-back).
     h2d = sum(v.numel() * v.element_size() for v in host_inputs[0].values())
     d2h = o.numel() * o.element_size()
+    h2d_s, d2h_s = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    outs = [o, torch.zeros_like(o)]
+    outs_h = [o_host, torch.zeros_like(o_host).pin_memory()]
+    R = 2 * NLAYERS                                  # event ring (slots reused after R tokens)
+    in_ready = [torch.cuda.Event() for _ in range(R)]
+    k_done = [torch.cuda.Event() for _ in range(R)]
+    out_done = [torch.cuda.Event() for _ in range(R)]
+    n = args.steps
+    base = args.warmup + args.steps
+
+    def issue_h2d(i):
+        l = (base + i) % NLAYERS                     # the input set token base + i reads
+        if i >= NLAYERS:
+            h2d_s.wait_event(k_done[(i - NLAYERS) % R])
+        with torch.cuda.stream(h2d_s):
+            for k, v in host_inputs[l].items():
+                inputs[l][k].copy_(v, non_blocking=True)
+        in_ready[i % R].record(h2d_s)
+
     barrier()
     ev0.record(stream)
-    for i in range(args.steps):
-        l = i % NLAYERS
-        for k, v in host_inputs[l].items():
-            inputs[l][k].copy_(v, non_blocking=True)
-        step(args.warmup + args.steps + i)
-        o_host.copy_(o, non_blocking=True)
+    h2d_s.wait_event(ev0)
+    d2h_s.wait_event(ev0)
+    issue_h2d(0)
+    for i in range(n):
+        if i + 1 < n:
+            issue_h2d(i + 1)
+        stream.wait_event(in_ready[i % R])
+        if i >= 2:
+            stream.wait_event(out_done[(i - 2) % R])
+        step(base + i, outs[i % 2])
+        k_done[i % R].record(stream)
+        d2h_s.wait_event(k_done[i % R])
+        with torch.cuda.stream(d2h_s):
+            outs_h[i % 2].copy_(outs[i % 2], non_blocking=True)
+        out_done[i % R].record(d2h_s)
+    stream.wait_event(out_done[(n - 1) % R])
     ev1.record(stream)
     barrier()
     ms_e2e = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
