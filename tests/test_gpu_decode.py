@@ -161,3 +161,13 @@ def test_argument_errors():
         brs.decode_step(L, brs.writeback_of(w, C=4), 0, buf, buf, None, None, buf, None, buf, buf,
                         buf, buf, buf, buf)
     assert e.value.status == brs.EUNSUPPORTED
+
+
+def test_gdn_decode_fp32_full_size_sampled():
+    """The GDN configuration's unquantized reference run (FP32 state,
+    B=256, 16 key / 32 value heads) in the benchmark's launch
+    configuration; the oracle runs 64 of the 8192 heads."""
+    w = synth.WORKLOADS["gdn_decode_fp32"]
+    units = (4000, 4064)
+    steps = _run_both(w, 16, units=units)
+    _compare(w, steps, units=units)

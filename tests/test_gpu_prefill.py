@@ -96,3 +96,44 @@ def test_prefill_full_size_sampled():
     for the first two chunks; the oracle runs 6 of the 256 heads."""
     w = synth.WORKLOADS["kda_prefill"]
     _run_chunks(w, 2, units=(97, 103))
+
+
+@pytest.mark.parametrize("kw,mode", [
+    (dict(B=2, H=3, d=128, k_hi=16, block=128), "nearest"),
+    (dict(B=1, H=4, Hk=2, d=128, k_hi=0, block=128, decay_per_key=0), "nearest"),
+    (dict(B=1, H=2, d=128, k_hi=16, block=32), "errfeedback"),
+])
+def test_prefill_multi_chunk_one_launch(kw, mode):
+    """Four chunks in ONE launch (the chunk-to-chunk hand-over inside the
+    kernel) equal, bit for bit, four one-chunk launches (each of which the
+    teacher-forced tests compare with the oracle): the same outputs, the same
+    stored state and residuals, the same state before the last write-back."""
+    import torch
+    from bit_recurrent_state_b200 import brs
+    from bit_recurrent_state_b200.state import LayerState
+    w = synth.Workload("pf1", T=256, C=64, seed=61, **kw)
+    perm = random_perm(w, seed=12)
+    cfg = O.Config(B=w.B, H=w.H, Hk=w.hk, d=w.d, storage=O.STORE_DAMP, k_hi=w.k_hi, block=w.block,
+                   hadamard=w.hadamard, decay_per_key=w.decay_per_key, domain=O.DOMAIN_CANONICAL)
+    L, wb = brs.layout_of(w), brs.writeback_of(w, C=64, mode=brs.MODES[mode])
+    S0 = (np.random.default_rng(6).standard_normal((w.B, w.H, w.d, w.d)) * 0.05).astype(np.float32)
+    packed0, _ = O.state_pack(cfg, S0, perm)
+    inp = _seq_major(w, 0, w.T)
+    d = {k: _dev(v) for k, v in inp.items()}
+    runs = []
+    for chunked in (False, True):
+        st = LayerState(L, perm=perm)
+        st.packed.copy_(torch.from_numpy(packed0))
+        o = torch.zeros((w.B, w.T, w.H, w.d), device="cuda")
+        dump = torch.zeros((w.B, w.H, w.d, w.d), device="cuda")
+        spans = [(c * 64, 64) for c in range(w.T // 64)] if chunked else [(0, w.T)]
+        for t0, T in spans:
+            dc = {k: v[:, t0:t0 + T].contiguous() for k, v in d.items()}
+            oc = torch.zeros((w.B, T, w.H, w.d), device="cuda")
+            brs.chunk_prefill(L, wb, t0, T, st.packed, st.aux, st.workspace, st.perm, dc["q"], dc["k"], dc["v"],
+                              dc["beta"], dc["decay"], oc, dump)
+            o[:, t0:t0 + T] = oc
+        assert st.errors() == 0
+        runs.append((o.cpu().numpy(), st.packed.cpu().numpy(), st.aux.cpu().numpy(), dump.cpu().numpy()))
+    for a, b in zip(runs[0], runs[1]):
+        np.testing.assert_array_equal(a.view(np.uint8), b.view(np.uint8))
