@@ -201,9 +201,15 @@ brs_status brs_decode_step(const brs_layout* L, const brs_writeback* wb, int64_t
  *     decay [B][T][H][d] (KDA) or [B][T][H] (GDN) f32; o [B][T][H][d] f32.
  *   state_dump (optional): [B][H][d][d] f32, the state just before the last
  *     write-back of the call (stored row order, value basis).
- * Results agree with the token-by-token recurrence within FP32 rounding of
- * the reordered sums; the stored codes are the documented quantizer applied
- * to state_dump. */
+ * The contractions run on the tensor cores in TF32 with each operand split
+ * into a TF32 part and its remainder (three products), which keeps FP32-level
+ * accuracy.  Results agree with the token-by-token recurrence within the
+ * rounding of the reordered sums; the stored codes are the documented
+ * quantizer applied to state_dump.  A call over several chunks equals
+ * consecutive one-chunk calls bit for bit.  The call takes a stream-ordered
+ * scratch of B*H*d*d floats for its duration (cudaMallocAsync / cudaFreeAsync
+ * on `stream`).  Per-channel decays whose 64-token product underflows FP32
+ * are outside the form (the outputs become non-finite: BRS_ENONFINITE). */
 brs_status brs_chunk_prefill(const brs_layout* L, const brs_writeback* wb, int64_t step0, int T,
                              void* packed, void* aux, void* workspace, const int16_t* perm,
                              const uint16_t* q, const uint16_t* k, const uint16_t* v,
