@@ -12,18 +12,24 @@
 //   A = strictly-lower(diag(beta) K~ K^T);  (I + A) W = diag(beta)(V - K~ S_0);
 //   O = Q~ S_0 + lower-incl(Q~ K^T) W;  S_C = diag(Gamma_63)(S_0 + K^T W).
 //
-// One CTA of 256 threads per (sequence, head) walks the chunks in order.
-// Tensor-memory accumulators (lanes x columns, FP32):
-//   D2 [128 j][128 t]: (K~ S_0)^T for t < 64, O^T = (Q~ S_0 + P W)^T for t >= 64
-//   D1 [128 t][64 s] : K~ K^T (t < 64) and Q~ K^T (t >= 64)
-//   D4 [128 i][128 j]: K^T W
+// One CTA of 512 threads per (sequence, head) walks the chunks in order.
+// A tcgen05.mma instruction takes about the same time for any N up to 256
+// (and M = 64 or 128), so the products are packed into few wide
+// instructions: operands that share A are stacked along N, and the hi and lo
+// halves of a B operand sit next to each other so one instruction forms
+// hi*hi and hi*lo.  Tensor-memory accumulators (lanes x columns, FP32):
+//   phase 1, columns 0..191 (lanes t: K~ rows 0..63, Q~ rows 64..127):
+//     [K~;Q~] . [S_0 | K^^T]  ->  K~ S_0, Q~ S_0 (cols 0..127), K~ K^^T, Q~ K^^T (128..191)
+//   phase 2, columns 0..255 (lanes 64..127 = t):  P W, hi*hi + lo*hi (0..127), hi*lo (128..255)
+//   phase 2, columns 256..511 (lanes i):          K^^T W, the same split
 // All operands are K-major, no swizzle: 8-row x 16-byte core matrices,
 // consecutive along K at 128 B, row groups of 8 at Kt/4 * 128 B.
-// Products in tensor-memory orientation:
-//   D1 = [K~;Q~] . K^^T     (A: X[t][i], B: X[s][i]; K = i in 4 slices of 32)
-//   D2 = S_0^T . [K~;Q~]^T   (A: X[j][i], B: X[t][i])
-//   D2[:, 64:] += W^T . P^T  (A: X[j][s], B: X[t][s]; P = lower-incl(Q~ K^T))
-//   D4 = K^T . W             (A: X[i][s], B: X[j][s])
+// Products in tensor-memory orientation (A rows = lanes, B rows = columns):
+//   phase 1:  A = X[t][i] ([K~;Q~]),  B = X[n][i] = [S_0^T (n = j) ; K^ (n = s)]    (K = i, 4 slices of 32)
+//   phase 2:  A = X[t][s] (rows 64.. = P = lower-incl(Q~ K^^T); rows below unused),  B = X[j][s] = [W_hi ; W_lo]
+//             A = X[i][s] (K^^T),                                                     B = [W_hi ; W_lo]
+// The right side of the substitution, diag(beta)(V - K~ S_0), is read out by
+// rows t and handed to the column threads j through shared memory.
 // The FP32 state S_0 between chunks lives in a global scratch (dequantized
 // stored state, stored row order, value basis).
 #include <cuda_runtime.h>
@@ -45,13 +51,16 @@ constexpr unsigned long long kTcWaitNs = 200000000ull;    // bound on one MMA wa
 //   Kt = K~ [64 t][128 i], Kh = K^, Qt = Q~
 constexpr int kRS = 132;
 constexpr int kRowB = kRS * 4;
-// phase 1: one slice buffer: KQ hi/lo [128][32], KH hi/lo [64][32], S0T hi/lo [128][32]
+// phase 1: one slice buffer: KQ hi, KQ lo [128][32], then the B operands
+// [S0T [128 j][32] ; KH [64 s][32]] hi and lo (192 rows each)
 constexpr int kKQ = 128 * kSl * 4, kKH = 64 * kSl * 4, kS0T = 128 * kSl * 4;
+constexpr int kBN = kS0T + kKH;                           // one [S0T ; KH] operand
 constexpr int kOffSlice = 0;
-constexpr int kSliceB = 2 * (kKQ + kKH + kS0T);           // 80 KB
+constexpr int kSliceB = 2 * (kKQ + kBN);                  // 80 KB
 constexpr int kOffKt = kOffSlice + kSliceB, kOffKh = kOffKt + kC * kRowB, kOffQt = kOffKh + kC * kRowB;
 // phase 2: KT hi/lo [128 i][64 s] over the slice buffer, P hi/lo [64 t][64 s] and A fp32 [64][68]
-// over Kt, W hi/lo [128 j][64 s] over Qt; Kh stays readable while KT is built
+// over Kt, W hi/lo [128 j][64 s] over Qt (W hi first holds the substitution's right side,
+// [64 t][128 j] FP32 with 16-byte groups swizzled by t); Kh stays readable while KT is built
 constexpr int kWt = 128 * 64 * 4, kKT = 128 * 64 * 4, kPt = 64 * 64 * 4;
 constexpr int kAStride = 68;
 constexpr int kOffKT = 0, kOffP = kOffKT + 2 * kKT, kOffA = kOffP + 2 * kPt, kOffW = kOffQt;
@@ -68,6 +77,8 @@ static_assert(kOffKT + 2 * kKT <= kOffKt, "KT over the slice buffer only");
 static_assert(kOffQt + kC * kRowB <= kRegion, "Qt inside the region");
 static_assert(kD * kSStride * 4 <= kOffW, "requantization rows fit below W");
 static_assert(kSmem <= 227 * 1024, "shared memory of one CTA");
+static_assert(kOffP >= 8 * 2048 && kOffP + kPt >= 8 * 2048, "the unused rows of the P operand stay in shared memory");
+static_assert(kC * kD * 4 <= kWt, "the right side fits the W hi tile");
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -107,10 +118,13 @@ __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence:
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void proxy_fence() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
+// one phase of an mbarrier; a thread parked in try_wait is suspended for at
+// most ~128 ns per attempt (parked without a bound it can stay suspended for
+// microseconds after the phase completes)
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 128; selp.u32 %0, 1, 0, p; }"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
       : "memory");
@@ -122,7 +136,7 @@ __device__ __forceinline__ unsigned long long global_ns() {
   return t;
 }
 // bounded wait for one phase of an MMA-completion barrier
-__device__ __noinline__ bool mbar_wait_tc(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_tc(uint32_t bar, uint32_t parity) {
   if (mbar_try(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   while (!mbar_try(bar, parity))
@@ -192,20 +206,30 @@ __device__ void tc_load_state(const uint8_t* head, float* S, int nlo, int k_hi, 
   }
 }
 
-// S_C rows (shared, stride kSStride) -> stored head; the dequantized rows
-// (the state the next chunk starts from) go to the global scratch
+// Write-back of the chunk, a warp per stored row (rows warp, warp + 16, ...),
+// lane l owning columns 4l .. 4l+3: S_C = Gamma_63 (S_0 + K^^T W) from the
+// product rows Ds (shared, stride kSStride) and S_0 (the global scratch,
+// whole rows per load), then the stored row; the dequantized row (the state
+// the next chunk starts from) replaces S_0 in the scratch.
 template <bool HAD, int BLOCK, int MODE>
-__device__ void tc_store_state(const float* Ss, float* S, uint8_t* head, uint16_t* aux, int nlo, int k_hi,
-                               float hscale, const PrefillArgs& a, int64_t step, int h, int b, float* sdump,
+__device__ void tc_store_state(const float* Ds, const float* g63, float* S, uint8_t* head, uint16_t* aux, int nlo,
+                               int k_hi, float hscale, const PrefillArgs& a, int64_t step, int h, int b, float* sdump,
                                uint32_t& err) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, col0 = 4 * lane;
-  constexpr int NB = kD / BLOCK, GL = BLOCK / 4;
+  constexpr int NB = kD / BLOCK, GL = BLOCK / 4, kRowsW = kD / (kThreads / 32);
   uint16_t* f16out = (uint16_t*)(head + (size_t)nlo * kD);
   uint32_t* szout = (uint32_t*)(head + (size_t)nlo * kD + (size_t)k_hi * kD * 2);
-  for (int r = warp; r < kD; r += kThreads / 32) {
-    const float4 v4 = *(const float4*)&Ss[r * kSStride + col0];
-    if (sdump) *(float4*)&sdump[(size_t)r * kD + col0] = v4;
-    float x[4] = {v4.x, v4.y, v4.z, v4.w};
+  float4 s0r[kRowsW];                              // this warp's S_0 rows, all loads in flight at once
+#pragma unroll
+  for (int k = 0; k < kRowsW; ++k) s0r[k] = *(const float4*)&S[(size_t)(warp + 16 * k) * kD + col0];
+#pragma unroll
+  for (int k = 0; k < kRowsW; ++k) {
+    const int r = warp + 16 * k;
+    const float4 d4 = *(const float4*)&Ds[r * kSStride + col0];
+    const float gi = g63[r];
+    float x[4] = {__fmul_rn(gi, __fadd_rn(s0r[k].x, d4.x)), __fmul_rn(gi, __fadd_rn(s0r[k].y, d4.y)),
+                  __fmul_rn(gi, __fadd_rn(s0r[k].z, d4.z)), __fmul_rn(gi, __fadd_rn(s0r[k].w, d4.w))};
+    if (sdump) *(float4*)&sdump[(size_t)r * kD + col0] = make_float4(x[0], x[1], x[2], x[3]);
     if (r >= nlo) {
       const uint32_t lo = f16x2_of(x[0], x[1]), hi = f16x2_of(x[2], x[3]);
       if ((((lo >> 10) & 31u) == 31u) || (((lo >> 26) & 31u) == 31u) || (((hi >> 10) & 31u) == 31u) ||
@@ -331,14 +355,15 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = *tslot;
-  const uint32_t tD2 = tm, tD1 = tm + 128, tD4 = tm + 256;
+  const uint32_t tO = tm, tD4 = tm + 256;         // phase 1 uses columns 0..191, phase 2 all 512
   const uint32_t lrow = (uint32_t)(32 * sub) << 16;          // this warp's lane base in tensor memory
   const int myrow = 32 * sub + lane;                          // the tensor-memory lane this thread reads
   uint32_t ph0 = 0, ph1 = 0;
   bool alive = true;
-  // every thread waits; the CTA agrees on the outcome
+  // thread 0 waits on the mbarrier, the others at the CTA barrier; the CTA
+  // agrees on the outcome
   auto wait_all = [&](int which, uint32_t& ph) -> bool {
-    const bool ok = mbar_wait_tc(bar0 + 8u * which, ph);
+    const bool ok = (tid == 0) ? mbar_wait_tc(bar0 + 8u * which, ph) : true;
     ph ^= 1u;
     return !__syncthreads_or(ok ? 0 : 1);
   };
@@ -398,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
         if (!alive) break;
       }
       uint8_t* B0 = smem + kOffSlice;
-      uint8_t *KQh = B0, *KQl = B0 + kKQ, *KHh = B0 + 2 * kKQ, *KHl = KHh + kKH, *STh = KHl + kKH, *STl = STh + kS0T;
+      uint8_t *KQh = B0, *KQl = B0 + kKQ, *STh = B0 + 2 * kKQ, *KHh = STh + kS0T, *STl = STh + kBN, *KHl = STl + kS0T;
 #pragma unroll
       for (int q = 0; q < 2560 / kThreads; ++q) {
         const int task = tid + q * kThreads;
@@ -422,72 +447,87 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
       if (tid == 0) {
         tc_fence_after();
         const uint32_t base = sbase + kOffSlice;
-        const uint32_t aKQh = base, aKQl = base + kKQ, aKHh = base + 2 * kKQ, aKHl = aKHh + kKH;
-        const uint32_t aSTh = aKHl + kKH, aSTl = aSTh + kS0T;
         constexpr uint32_t sbo = (kSl / 4) * 128;
-        const uint64_t dKQh = sdesc(aKQh, sbo), dKQl = sdesc(aKQl, sbo), dKHh = sdesc(aKHh, sbo),
-                       dKHl = sdesc(aKHl, sbo), dSTh = sdesc(aSTh, sbo), dSTl = sdesc(aSTl, sbo);
+        // [K~;Q~] . [S_0^T ; K^]: N = 192, three instructions per k-step
+        const uint64_t dKQh = sdesc(base, sbo), dKQl = sdesc(base + kKQ, sbo);
+        const uint64_t dBh = sdesc(base + 2 * kKQ, sbo), dBl = sdesc(base + 2 * kKQ + kBN, sbo);
 #pragma unroll
         for (int k = 0; k < kSl / 8; ++k) {
           const uint32_t o16 = 16u * k, acc = (sl > 0 || k > 0) ? 1u : 0u;
-          umma3d(tD1, dKQh, dKQl, dKHh, dKHl, o16, idesc_tf32(128, 64), acc);
-          umma3d(tD2, dSTh, dSTl, dKQh, dKQl, o16, idesc_tf32(128, 128), acc);
+          umma3d(tO, dKQh, dKQl, dBh, dBl, o16, idesc_tf32(128, 3 * kC), acc);
         }
         umma_commit(bar0);
       }
     }
     if (!alive) break;
-    if (part == 0) {                                 // the chunk's V rows into L1 while the MMAs run
-      const uint16_t* vrow = a.v + ((tokb + (myrow & 63)) * a.H + h) * kD + 64 * (myrow >> 6);
+    if (sub < 2) {                                   // this thread's part of a V row into L1 while the MMAs run
+      const uint16_t* vrow = a.v + ((tokb + myrow) * a.H + h) * kD + 32 * part;
       asm volatile("prefetch.global.L1 [%0];" ::"l"(vrow));
     }
     alive = wait_all(0, ph0);
     if (!alive) break;
     tc_fence_after();
 
-    if (part == 0) {
-      // ---- D1: A = strictly-lower(diag(beta) K~ K^T) (fp32), P = lower-incl(Q~ K^T)
-      // as the split operand X[t][s]
-      float* Am = (float*)(smem + kOffA);
+    // ---- phase-1 readout, every warp: tensor-memory lanes t of its
+    // sub-partition, value columns 32 part .. 32 part + 31, key columns
+    // 16 part .. 16 part + 15 (Q~ S_0 stays in tensor memory for O)
+    float* Am = (float*)(smem + kOffA);
+    float* Rs = (float*)(smem + kOffW);              // right side [64 t][128 j], 16-byte groups ^ (t & 7)
+    {
+      float v[16];
+      const int c0 = 16 * part;
+      if (sub < 2) {
+        // right side diag(beta)(V - K~ S_0), by rows
+        const int t = myrow;
+        const float bt = betas[t];
+        const uint4* vp = (const uint4*)(a.v + ((tokb + t) * a.H + h) * kD + 32 * part);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float v[16];
-        const int c0 = 16 * q;
-        tmem_ld16(tD1 + lrow + c0, v);
-        if (myrow < 64) {
-          const int t = myrow;
-          const float bt = betas[t];
+        for (int q = 0; q < 2; ++q) {
+          tmem_ld16(tO + lrow + 32 * part + 16 * q, v);
+          const uint4 r0 = vp[2 * q], r1 = vp[2 * q + 1];
+          const uint32_t vw[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+          float x[16];
 #pragma unroll
-          for (int c = 0; c < 16; c += 4)
-            *(float4*)&Am[t * kAStride + c0 + c] =
-                make_float4((c0 + c + 0 < t) ? __fmul_rn(bt, v[c + 0]) : 0.0f, (c0 + c + 1 < t) ? __fmul_rn(bt, v[c + 1]) : 0.0f,
-                            (c0 + c + 2 < t) ? __fmul_rn(bt, v[c + 2]) : 0.0f, (c0 + c + 3 < t) ? __fmul_rn(bt, v[c + 3]) : 0.0f);
-        } else {
-          const int t = myrow - 64;
+          for (int c = 0; c < 16; ++c) {
+            const float vv = bf16_to_f32((uint16_t)((c & 1) ? (vw[c >> 1] >> 16) : (vw[c >> 1] & 0xffffu)));
+            x[c] = __fmul_rn(bt, __fsub_rn(vv, v[c]));
+          }
 #pragma unroll
-          for (int c = 0; c < 16; c += 4)
-            st_split4(smem + kOffP, smem + kOffP + kPt, kmaj(t, c0 + c, 64), (c0 + c + 0 <= t) ? v[c + 0] : 0.0f,
-                      (c0 + c + 1 <= t) ? v[c + 1] : 0.0f, (c0 + c + 2 <= t) ? v[c + 2] : 0.0f,
-                      (c0 + c + 3 <= t) ? v[c + 3] : 0.0f);
+          for (int c = 0; c < 16; c += 4) {
+            const int g = (32 * part + 16 * q + c) >> 2;
+            *(float4*)&Rs[t * kD + ((g ^ (t & 7)) << 2)] = make_float4(x[c], x[c + 1], x[c + 2], x[c + 3]);
+          }
         }
+        // A = strictly-lower(diag(beta) K~ K^T), FP32
+        tmem_ld16(tO + lrow + kD + c0, v);
+#pragma unroll
+        for (int c = 0; c < 16; c += 4)
+          *(float4*)&Am[t * kAStride + c0 + c] =
+              make_float4((c0 + c + 0 < t) ? __fmul_rn(bt, v[c + 0]) : 0.0f, (c0 + c + 1 < t) ? __fmul_rn(bt, v[c + 1]) : 0.0f,
+                          (c0 + c + 2 < t) ? __fmul_rn(bt, v[c + 2]) : 0.0f, (c0 + c + 3 < t) ? __fmul_rn(bt, v[c + 3]) : 0.0f);
+      } else {
+        // P = lower-incl(Q~ K^T) as the split operand X[t][s]
+        const int t = myrow - 64;
+        tmem_ld16(tO + lrow + kD + c0, v);
+#pragma unroll
+        for (int c = 0; c < 16; c += 4)
+          st_split4(smem + kOffP, smem + kOffP + kPt, kmaj(t, c0 + c, 64), (c0 + c + 0 <= t) ? v[c + 0] : 0.0f,
+                    (c0 + c + 1 <= t) ? v[c + 1] : 0.0f, (c0 + c + 2 <= t) ? v[c + 2] : 0.0f,
+                    (c0 + c + 3 <= t) ? v[c + 3] : 0.0f);
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");   // A complete for the 128 column threads
+    }
+    tc_fence_before();
+    __syncthreads();                                 // right side, A and P complete; key columns read
+
+    const bool solver = (sub < 2) && (part < 2);     // warps 0, 1, 4, 5: one value column each
+    if (solver) {
       // ---- W by forward substitution, one value column j per thread:
-      // (I + A) W = diag(beta)(V - K~ S_0), the right side from D2[j][0..63]
-      const int j = myrow;
+      // (I + A) W = diag(beta)(V - K~ S_0)
+      const int j = 32 * (2 * part + sub) + lane;
       float w[kC];
 #pragma unroll
-      for (int t = 0; t < kC; ++t) w[t] = bf16_to_f32(a.v[((tokb + t) * a.H + h) * kD + j]);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float v[16];
-        tmem_ld16(tD2 + lrow + 16 * q, v);
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int t = 16 * q + c;
-          w[t] = __fmul_rn(betas[t], __fsub_rn(w[t], v[c]));
-        }
-      }
+      for (int t = 0; t < kC; ++t) w[t] = Rs[t * kD + ((((j >> 2) ^ (t & 7))) << 2) + (j & 3)];
+      asm volatile("bar.sync 1, 128;" ::: "memory");   // every column read before W replaces the right side
       // blocks of 16 rows: the terms from earlier blocks are 16 independent
       // sums, then the block's own triangle is solved row by row
 #pragma unroll
@@ -518,8 +558,19 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
       for (int s = 0; s < kC; s += 4)
         st_split4(smem + kOffW, smem + kOffW + kWt, kmaj(j, s, 64), w[s], w[s + 1], w[s + 2], w[s + 3]);
     } else {
-      // ---- K^ transposed: X[i][s] = K^[s][i]
-      for (int task = tid - 128; task < kD * (kC / 4); task += kThreads - 128) {
+      if (sub >= 2) {
+        // zero the hi*lo columns of O (lanes 64..127, columns 128..255): phase 2
+        // accumulates onto Q~ S_0 in columns 0..127 and onto zero here
+        uint32_t zr = 0;
+        asm volatile(
+            "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,"
+            "%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(tO + lrow + kD + 32 * part), "r"(zr)
+            : "memory");
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      }
+      // ---- K^ transposed: X[i][s] = K^[s][i], by the other 12 warps
+      const int wr = (warp < 8) ? 2 * (warp >> 2) + (warp & 3) - 2 : warp - 4;
+      for (int task = 32 * wr + lane; task < kD * (kC / 4); task += kThreads - 128) {
         const int i = task & 127, sg = task >> 7;
         st_split4(smem + kOffKT, smem + kOffKT + kKT, kmaj(i, 4 * sg, 64), Kh[(4 * sg) * kRS + i],
                   Kh[(4 * sg + 1) * kRS + i], Kh[(4 * sg + 2) * kRS + i], Kh[(4 * sg + 3) * kRS + i]);
@@ -529,67 +580,72 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
     tc_fence_before();
     __syncthreads();
     if (tid == 0) {
-      // ---- phase 2: D2[:, 64:] += W^T P^T (O^T), D4 = K^T W
+      // ---- phase 2: B = [W_hi ; W_lo] (N = 256) gives hi*hi and hi*lo in one
+      // instruction, B = W_hi adds lo*hi to the first half.
+      //   O: A = X[t'][s] whose rows 64..127 are P (rows 0..63: the 16 KB
+      //      below P, unused lanes), accumulated onto Q~ S_0;
+      //   K^^T W: A = X[i][s], fresh.
       tc_fence_after();
-      const uint32_t aWh = sbase + kOffW, aWl = aWh + kWt, aKTh = sbase + kOffKT, aKTl = aKTh + kKT;
-      const uint32_t aPh = sbase + kOffP, aPl = aPh + kPt;
       constexpr uint32_t sbo = (64 / 4) * 128;
-      const uint64_t dWh = sdesc(aWh, sbo), dWl = sdesc(aWl, sbo), dKTh = sdesc(aKTh, sbo), dKTl = sdesc(aKTl, sbo),
+      const uint32_t aKTh = sbase + kOffKT, aKTl = aKTh + kKT;
+      const uint32_t aPh = sbase + kOffP - 8 * sbo, aPl = sbase + kOffP + kPt - 8 * sbo;
+      const uint64_t dW = sdesc(sbase + kOffW, sbo), dKTh = sdesc(aKTh, sbo), dKTl = sdesc(aKTl, sbo),
                      dPh = sdesc(aPh, sbo), dPl = sdesc(aPl, sbo);
 #pragma unroll
       for (int k = 0; k < kC / 8; ++k) {
         const uint32_t o16 = 16u * k;
-        umma3d(tD2 + 64, dWh, dWl, dPh, dPl, o16, idesc_tf32(128, 64), 1u);
-        umma3d(tD4, dKTh, dKTl, dWh, dWl, o16, idesc_tf32(128, 128), k > 0 ? 1u : 0u);
+        umma_tf32(tO, dPh + o16, dW + o16, idesc_tf32(128, 2 * kD), 1u);
+        umma_tf32(tO, dPl + o16, dW + o16, idesc_tf32(128, kD), 1u);
+        umma_tf32(tD4, dKTh + o16, dW + o16, idesc_tf32(128, 2 * kD), k > 0 ? 1u : 0u);
+        umma_tf32(tD4, dKTl + o16, dW + o16, idesc_tf32(128, kD), 1u);
       }
       umma_commit(bar0 + 8u);
     }
-    constexpr int kCols = kD / kParts;               // this thread's columns of its S row
-    float4 s0v[kCols / 4];                           // S_0 row part, loaded while the MMAs run
-#pragma unroll
-    for (int c = 0; c < kCols / 4; ++c) s0v[c] = *(const float4*)&S0g[(size_t)myrow * kD + kCols * part + 4 * c];
+    constexpr int kCols = kD / kParts;               // this thread's columns of a product row
     alive = wait_all(1, ph1);
     if (!alive) break;
     tc_fence_after();
 
-    // ---- O = (D2[:, 64:])^T to global; S_C = Gamma_63 (S_0 + D4) to the
-    // requantization rows
+    // ---- O = (Q~ S_0 + P W) rows to global (lanes 64..127); K^^T W rows to
+    // shared memory for the write-back
     {
-      const int j = myrow;
-      float v[16];
-      bool bad = false;
+      float v[16], u[16];
+      if (sub >= 2) {
+        const int t = myrow - 64;
+        float* orow = a.o + ((tokb + t) * a.H + h) * kD + 32 * part;
+        bool bad = false;
 #pragma unroll
-      for (int q = 0; q < 64 / kParts / 16; ++q) {
-        const int c0 = (64 / kParts) * part + 16 * q;
-        tmem_ld16(tD2 + lrow + 64 + c0, v);
+        for (int q = 0; q < 2; ++q) {
+          tmem_ld16(tO + lrow + 32 * part + 16 * q, v);
+          tmem_ld16(tO + lrow + kD + 32 * part + 16 * q, u);
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          bad |= !isfinite(v[c]);
-          a.o[((tokb + c0 + c) * a.H + h) * kD + j] = v[c];
+          for (int c = 0; c < 16; c += 4) {
+            const float4 x = make_float4(__fadd_rn(v[c], u[c]), __fadd_rn(v[c + 1], u[c + 1]),
+                                         __fadd_rn(v[c + 2], u[c + 2]), __fadd_rn(v[c + 3], u[c + 3]));
+            bad |= !isfinite(x.x) || !isfinite(x.y) || !isfinite(x.z) || !isfinite(x.w);
+            *(float4*)&orow[16 * q + c] = x;
+          }
         }
+        if (bad) err |= BRS_FLAG_NONFINITE;
       }
-      if (bad) err |= BRS_FLAG_NONFINITE;
-      float* Ss = (float*)smem;
+      float* Ds = (float*)smem;                     // K^^T W rows for the write-back
       const int i = myrow;
-      const float gi = g63[i];
 #pragma unroll
       for (int q = 0; q < kCols / 16; ++q) {
         const int c0 = kCols * part + 16 * q;
         tmem_ld16(tD4 + lrow + c0, v);
+        tmem_ld16(tD4 + lrow + kD + c0, u);
 #pragma unroll
-        for (int c = 0; c < 16; c += 4) {
-          const float4 s4 = s0v[4 * q + c / 4];
-          *(float4*)&Ss[i * kSStride + c0 + c] =
-              make_float4(__fmul_rn(gi, __fadd_rn(s4.x, v[c])), __fmul_rn(gi, __fadd_rn(s4.y, v[c + 1])),
-                          __fmul_rn(gi, __fadd_rn(s4.z, v[c + 2])), __fmul_rn(gi, __fadd_rn(s4.w, v[c + 3])));
-        }
+        for (int c = 0; c < 16; c += 4)
+          *(float4*)&Ds[i * kSStride + c0 + c] = make_float4(__fadd_rn(v[c], u[c]), __fadd_rn(v[c + 1], u[c + 1]),
+                                                             __fadd_rn(v[c + 2], u[c + 2]), __fadd_rn(v[c + 3], u[c + 3]));
       }
     }
     tc_fence_before();
     __syncthreads();
     // ---- write-back of the chunk
     const bool last = ch == nchunks - 1;
-    tc_store_state<HAD, BLOCK, MODE>((const float*)smem, S0g, hst, aux, nlo, a.k_hi, a.hscale, a,
+    tc_store_state<HAD, BLOCK, MODE>((const float*)smem, g63, S0g, hst, aux, nlo, a.k_hi, a.hscale, a,
                                      a.step0 + t0 + kC - 1, h, b,
                                      (last && a.sdump) ? a.sdump + (size_t)head * kD * kD : nullptr, err);
     __syncthreads();
