@@ -227,8 +227,10 @@ __device__ void tc_store_state(const float* Ds, const float* g63, float* S, uint
     const int r = warp + 16 * k;
     const float4 d4 = *(const float4*)&Ds[r * kSStride + col0];
     const float gi = g63[r];
-    float x[4] = {__fmul_rn(gi, __fadd_rn(s0r[k].x, d4.x)), __fmul_rn(gi, __fadd_rn(s0r[k].y, d4.y)),
-                  __fmul_rn(gi, __fadd_rn(s0r[k].z, d4.z)), __fmul_rn(gi, __fadd_rn(s0r[k].w, d4.w))};
+    // Gamma_63 * (S_0 + K^^T W); the product as an fma with -0 (the same
+    // rounded product) so that it is never merged with the transform's adds
+    float x[4] = {__fmaf_rn(gi, __fadd_rn(s0r[k].x, d4.x), -0.0f), __fmaf_rn(gi, __fadd_rn(s0r[k].y, d4.y), -0.0f),
+                  __fmaf_rn(gi, __fadd_rn(s0r[k].z, d4.z), -0.0f), __fmaf_rn(gi, __fadd_rn(s0r[k].w, d4.w), -0.0f)};
     if (sdump) *(float4*)&sdump[(size_t)r * kD + col0] = make_float4(x[0], x[1], x[2], x[3]);
     if (r >= nlo) {
       const uint32_t lo = f16x2_of(x[0], x[1]), hi = f16x2_of(x[2], x[3]);
