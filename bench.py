@@ -648,7 +648,7 @@ def main():
     if args.steps is None:
         # long enough a timed region for the clock sampler (>= ~0.5 s on
         # the GPU); the oracle arm times a few bounded samples
-        args.steps = 10 if args.impl == "reference" else (5 if w.C > 1 else 20000)
+        args.steps = 10 if args.impl == "reference" else (40 if w.C > 1 else 20000)
     if args.impl == "reference":
         run_reference(args, w)
     else:

@@ -44,7 +44,7 @@ template <int D>
 struct __align__(16) VbSmem {
   VbRow row[D];
   float R[D];                    // row ranges (phase 0)
-  float y[kVbBatch][D + 1];      // one batch of targets (phase 1), padded
+  float y[kVbBatch][D + 4];      // one batch of target magnitudes (phase 1), rows 16-byte aligned
   uint32_t pk[kVbBatch][32];     // bit-packed output rows of the batch
   float pstep[kVbBatch], pinv[kVbBatch];
 };
@@ -200,11 +200,13 @@ __global__ void __launch_bounds__(32 * kVbWarps) varbit_kernel(const VbArgs a) {
       continue;
     } else {
       const float R = v[0];
-      // ---- targets of the batch to shared memory (rows padded by one)
+      // ---- magnitudes of the batch's targets to shared memory (rows padded
+      // by one): the fit error of -y equals that of y (rounding to nearest
+      // even and the clip at +-n are odd functions, each residual only
+      // changes sign), so the fit runs on |y| with a one-sided clip
 #pragma unroll
       for (int r = 0; r < kVbBatch; ++r)
-#pragma unroll
-        for (int c = 0; c < C; ++c) sm.y[r][col0 + c] = x[r][c];
+        *(float4*)&sm.y[r][col0] = make_float4(fabsf(x[r][0]), fabsf(x[r][1]), fabsf(x[r][2]), fabsf(x[r][3]));
       __syncwarp();
       // ---- fitted step: row jr, candidates m = q, q+4, q+8, q+12
       const int q4 = lane & 3;
@@ -220,9 +222,12 @@ __global__ void __launch_bounds__(32 * kVbWarps) varbit_kernel(const VbArgs a) {
         E[k] = 0.f;
       }
       const float* yrow = sm.y[jr];
-#pragma unroll 4
-      for (int j = 0; j < D; ++j) {
-        const float y = yrow[j];
+#pragma unroll 2
+      for (int j4 = 0; j4 < D; j4 += 4) {
+        const float4 y4 = *(const float4*)&yrow[j4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+        const float y = jj == 0 ? y4.x : jj == 1 ? y4.y : jj == 2 ? y4.z : y4.w;
         float t0, t1, t2, t3;
         mul2(t0, t1, y, y, iv[0], iv[1]);
         mul2(t2, t3, y, y, iv[2], iv[3]);
@@ -232,16 +237,17 @@ __global__ void __launch_bounds__(32 * kVbWarps) varbit_kernel(const VbArgs a) {
         fma2(t2, t3, t2, t3, a.one, a.one, kRoundMagic, kRoundMagic);
         sub2(t0, t1, t0, t1, kRoundMagic, kRoundMagic);
         sub2(t2, t3, t2, t3, kRoundMagic, kRoundMagic);
-        t0 = fminf(fmaxf(t0, -fn), fn);
-        t1 = fminf(fmaxf(t1, -fn), fn);
-        t2 = fminf(fmaxf(t2, -fn), fn);
-        t3 = fminf(fmaxf(t3, -fn), fn);
+        t0 = fminf(t0, fn);
+        t1 = fminf(t1, fn);
+        t2 = fminf(t2, fn);
+        t3 = fminf(t3, fn);
         mul2(t0, t1, st[0], st[1], t0, t1);                 // step * level
         mul2(t2, t3, st[2], st[3], t2, t3);
         sub2(t0, t1, y, y, t0, t1);                         // residual
         sub2(t2, t3, y, y, t2, t3);
         fma2(E[0], E[1], t0, t1, t0, t1, E[0], E[1]);
         fma2(E[2], E[3], t2, t3, t2, t3, E[2], E[3]);
+        }
       }
       // best of the lane (ascending m), then of the row's four lanes
       int bm = 99;
