@@ -3,7 +3,7 @@ GB/s against the measured B200 copy bandwidth).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload kda_decode|gdn_decode|gdn_decode_fp32|varbit_decode|
-                                kda_prefill|kda_tiny]
+                                kda_decode_c8|kda_prefill|kda_tiny]
 
 A step is one decode token for every (sequence, head) of the workload: one
 launch of the fused decode kernel (dequantize, decay, delta-rule write, read
@@ -15,6 +15,9 @@ path); the time is the maximum over ranks.
 
 With `--workload kda_prefill` a step is instead one chunked-prefill launch
 over the whole batch (B x T tokens x H heads, write-back every 64 tokens).
+`--workload kda_decode_c8` decodes with write-back every 8 tokens (the FP32
+state carried in HBM between write-backs; state bytes averaged over the
+interval).
 
 `--impl reference` times the plain CPU oracle on this host's cores on the
 same workload and metric (bounded samples), which is the only other place
@@ -65,8 +68,17 @@ def algorithmic_bytes(w) -> dict:
     out = heads * w.d * 4
     ef = 2 * aux if w.mode == "errfeedback" else 0
     st = 2 * stats
-    return dict(state=2 * n, inputs=inputs, output=out, aux=ef, stats=st,
-                total=2 * n + inputs + out + ef + st)
+    state = 2 * n
+    if w.C > 1 and w.storage == "damp":
+        # deferred write-back, averaged over an interval of C tokens: the
+        # stored state is read at its first token and written at its last,
+        # the FP32 interval state written at the other C - 1 and read at the
+        # other C - 1 (residuals touched at the write-back only)
+        f32 = heads * w.d * w.d * 4
+        state = (2 * n + 2 * (w.C - 1) * f32) / w.C
+        ef = ef / w.C
+    return dict(state=state, inputs=inputs, output=out, aux=ef, stats=st,
+                total=state + inputs + out + ef + st)
 
 
 def rank_workload(w, rank: int):
@@ -89,7 +101,7 @@ def kernel_name(w) -> str:
     """The kernel a decode step of workload w launches (the dominant one)."""
     if w.storage == "varbit":
         return "brs::varbit_kernel (update pass + fit pass) and brs::allocate_kernel"
-    if w.storage == "damp" and w.d == 128:
+    if w.storage == "damp" and w.d == 128 and w.C == 1:
         return "brs::decode_tma_kernel"
     return "brs::decode_warp_kernel"
 
@@ -511,7 +523,9 @@ def run_ours(args, w):
             spares[l] = st.step(wb, i, x["q"], x["k"], x["v"], x["beta"], x["decay"], out,
                                 packed_out=spares[l])
         else:
-            st.step(wb, i, x["q"], x["k"], x["v"], x["beta"], x["decay"], out)
+            # with deferred write-back a layer's calls must cover consecutive
+            # steps: its own token counter
+            st.step(wb, i // NLAYERS if w.C > 1 else i, x["q"], x["k"], x["v"], x["beta"], x["decay"], out)
 
     for i in range(args.warmup):
         step(i)

@@ -25,7 +25,8 @@ STORES = {"fp32": STORE_FP32, "damp": STORE_DAMP, "varbit": STORE_VARBIT}
 # exported symbols declared in include/brs.h
 SYMBOLS = ["brs_state_bytes", "brs_state_pack", "brs_state_unpack", "brs_decode_step",
            "brs_decode_step_noalloc", "brs_chunk_prefill", "brs_allocate_bits", "brs_fetch_errors",
-           "brs_last_error", "brs_calibrate_workspace_bytes", "brs_calibrate"]
+           "brs_last_error", "brs_calibrate_workspace_bytes", "brs_calibrate", "brs_decode_state32_bytes",
+           "brs_decode_step_deferred"]
 
 
 class BrsError(RuntimeError):
@@ -79,6 +80,10 @@ def lib():
         L.brs_state_unpack.argtypes = [P, P, P, P, P, P]
         L.brs_decode_step.restype = S
         L.brs_decode_step.argtypes = [P, P, ct.c_int64] + [P] * 13
+        L.brs_decode_state32_bytes.restype = ct.c_size_t
+        L.brs_decode_state32_bytes.argtypes = [P]
+        L.brs_decode_step_deferred.restype = S
+        L.brs_decode_step_deferred.argtypes = [P, P, ct.c_int64] + [P] * 12
         L.brs_decode_step_noalloc.restype = S
         L.brs_decode_step_noalloc.argtypes = [P, P, ct.c_int64] + [P] * 12
         L.brs_chunk_prefill.restype = S
@@ -149,6 +154,22 @@ def decode_step(layout, wb, step, packed_in, packed_out, aux, stats, workspace, 
                                  _ptr(packed_out), _ptr(aux), _ptr(stats), _ptr(workspace),
                                  _ptr(perm), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(decay),
                                  _ptr(o), _stream(stream)))
+
+
+def decode_state32_bytes(layout) -> int:
+    """brs_decode_state32_bytes: the FP32 interval state of deferred write-back."""
+    n = int(lib().brs_decode_state32_bytes(ct.byref(layout)))
+    if n == 0:
+        _check(EUNSUPPORTED)
+    return n
+
+
+def decode_step_deferred(layout, wb, step, packed, aux, workspace, state32, perm, q, k, v, beta, decay, o,
+                         stream=None):
+    """brs_decode_step_deferred: one decode token with write-back every wb.C tokens."""
+    _check(lib().brs_decode_step_deferred(ct.byref(layout), ct.byref(wb), int(step), _ptr(packed), _ptr(aux),
+                                          _ptr(workspace), _ptr(state32), _ptr(perm), _ptr(q), _ptr(k), _ptr(v),
+                                          _ptr(beta), _ptr(decay), _ptr(o), _stream(stream)))
 
 
 def decode_step_noalloc(layout, wb, step, packed_in, packed_out, aux, stats, perm, q, k, v, beta,

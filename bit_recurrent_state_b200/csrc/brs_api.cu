@@ -225,6 +225,53 @@ brs_status brs_decode_step(const brs_layout* L, const brs_writeback* wb, int64_t
   return ok();
 }
 
+size_t brs_decode_state32_bytes(const brs_layout* L) {
+  if (check_layout(L) != BRS_OK) return 0;
+  if (L->storage != BRS_STORE_DAMP) {
+    fail(BRS_EUNSUPPORTED, "the interval state is defined for DAMP storage");
+    return 0;
+  }
+  ok();
+  return (size_t)L->B * L->H * L->d * L->d * sizeof(float);
+}
+
+brs_status brs_decode_step_deferred(const brs_layout* L, const brs_writeback* wb, int64_t step, void* packed,
+                                    void* aux, void* workspace, void* state32, const int16_t* perm,
+                                    const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* beta,
+                                    const float* decay, float* o, void* stream) {
+  brs_status st = check_layout(L);
+  if (st != BRS_OK) return st;
+  if (!wb) return fail(BRS_EINVAL, "writeback is NULL");
+  if (L->storage != BRS_STORE_DAMP) return fail(BRS_EUNSUPPORTED, "deferred decode write-back is built for DAMP storage");
+  if (wb->C < 1) return fail(BRS_EINVAL, "write-back interval C must be >= 1 (got %d)", wb->C);
+  if (wb->mode < 0 || wb->mode > 2) return fail(BRS_EINVAL, "unknown rounding mode %d", wb->mode);
+  if (step < 0) return fail(BRS_EINVAL, "step must be >= 0");
+  if (!brs::decode_supported(L->d, L->block, L->k_hi))
+    return fail(BRS_EUNSUPPORTED,
+                "decode kernel built for (d, block) in {(128,128), (128,32), (64,64), (32,32)} and "
+                "k_hi a multiple of d/8 up to d/4 (got d=%d block=%d k_hi=%d)", L->d, L->block, L->k_hi);
+  const bool src32 = step % wb->C != 0, dst32 = (step + 1) % wb->C != 0;
+  if (!packed || !workspace || !q || !k || !v || !beta || !decay || !o)
+    return fail(BRS_EINVAL, "a required pointer is NULL");
+  if ((src32 || dst32) && !state32) return fail(BRS_EINVAL, "C > 1 needs the interval state");
+  if (wb->mode == BRS_ROUND_ERRFEEDBACK && !aux) return fail(BRS_EINVAL, "error feedback needs the residual buffer");
+  const void* ptrs[] = {packed, aux, workspace, state32, perm, q, k, v, beta, decay, o};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(BRS_EALIGN, "device pointers must be 16-byte aligned");
+  brs::DecodeArgs a{};
+  a.B = L->B; a.H = L->H; a.Hk = L->H_k; a.k_hi = L->k_hi; a.block = L->block;
+  a.decay_per_key = L->decay_per_key; a.mode = wb->mode; a.seed = wb->seed; a.step = step;
+  a.head_bytes = head_bytes(L); a.hscale = hadamard_scale(L->d);
+  a.packed_in = packed; a.packed_out = packed; a.aux = aux; a.perm = perm;
+  a.q = q; a.k = k; a.v = v; a.beta = beta; a.decay = decay; a.o = o;
+  a.flags = (uint32_t*)workspace;
+  a.s32 = (float*)state32; a.src32 = src32; a.dst32 = dst32;
+  cudaError_t e = (src32 || dst32) ? brs::launch_decode_deferred(a, L->d, L->hadamard != 0, (cudaStream_t)stream)
+                                   : brs::launch_decode(a, L->d, L->storage, L->hadamard != 0, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return ok();
+}
+
 brs_status brs_chunk_prefill(const brs_layout* L, const brs_writeback* wb, int64_t step0, int T,
                              void* packed, void* aux, void* workspace, const int16_t* perm,
                              const uint16_t* q, const uint16_t* k, const uint16_t* v,

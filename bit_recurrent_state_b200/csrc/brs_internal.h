@@ -24,9 +24,18 @@ struct DecodeArgs {
   const float *beta, *decay;
   float* o;
   uint32_t* flags;
+  // deferred write-back (DAMP): the FP32 state between write-backs,
+  // [B*H][d][d] in stored row order and the tiers' own bases; src32 reads the
+  // rows from it instead of the stored state, dst32 writes the updated rows
+  // to it instead of the write-back
+  float* s32 = nullptr;
+  int src32 = 0, dst32 = 0;
 };
 
 cudaError_t launch_decode(const DecodeArgs& a, int d, int store, bool had, cudaStream_t st);
+// the general (warp-per-head) kernel for every shape it supports, with the
+// interval-state flags honoured (DAMP storage)
+cudaError_t launch_decode_deferred(const DecodeArgs& a, int d, bool had, cudaStream_t st);
 bool decode_supported(int d, int block, int k_hi);
 
 struct CalibArgs {

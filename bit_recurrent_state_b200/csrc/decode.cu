@@ -198,10 +198,14 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
   const float beta = a.beta[head];
   __syncwarp();
 
+  float* s32h = (STORE != BRS_STORE_FP32 && a.s32) ? a.s32 + (size_t)head * D * D : nullptr;
+  const bool src32 = (STORE != BRS_STORE_FP32) && a.src32;   // rows from the interval state
+  const bool dst32 = (STORE != BRS_STORE_FP32) && a.dst32;   // updated rows to the interval state
   // one stored row -> FP32 values of my columns (before decay)
   auto load_row = [&](int i, float (&x)[C]) {
-    if constexpr (STORE == BRS_STORE_FP32) {
-      const float* src = (const float*)hin + (size_t)i * D + col0;
+    if (STORE == BRS_STORE_FP32 || src32) {
+      const float* src = (STORE == BRS_STORE_FP32) ? (const float*)hin + (size_t)i * D + col0
+                                                  : s32h + (size_t)i * D + col0;
       if constexpr (C == 4) {
         const float4 f = __ldg((const float4*)src);
         x[0] = f.x; x[1] = f.y; x[2] = f.z; x[3] = f.w;
@@ -255,6 +259,17 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
       const float4 ka = sm.rs[i].ka;
       v_scale<C>(x, ka.z, ka.w);
       v_fma_s<C>(u1, ka.x, ka.y, x);
+    }
+  } else if (src32) {
+    // FP32 rows from the interval state: the same chains, INT8 tier then FP16 tier
+#pragma unroll 8
+    for (int i = 0; i < D; ++i) {
+      float x[C];
+      load_row(i, x);
+      const float4 ka = sm.rs[i].ka;
+      v_scale<C>(x, ka.z, ka.w);
+      if (i < nlo) v_fma_s<C>(u1, ka.x, ka.y, x);
+      else v_fma_s<C>(u2, ka.x, ka.y, x);
     }
   } else {
     // chunks of CH = NRB rows (nlo is a multiple of NRB), two in flight
@@ -340,7 +355,7 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
     prow += NRB * D;
     psrow += NRB * NB;
   };
-  if (STORE != BRS_STORE_FP32 && nlo > 0) prefetch();
+  if (STORE != BRS_STORE_FP32 && !src32 && nlo > 0) prefetch();
   for (int i0 = 0; i0 < D; i0 += NRB) {
     const bool int8_batch = (STORE != BRS_STORE_FP32) && (i0 < nlo);   // batches are tier-uniform
     float x[NRB][C];
@@ -349,7 +364,7 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
       const int i = i0 + r;
       const RowScal rsc = sm.rs[i];
       const float2 qv = sm.qq[i];
-      if (int8_batch) {
+      if (int8_batch && !src32) {
         if constexpr (NB == 1) {
           dequant_int8<C>(x[r], pw[r], rsc.sz.x, rsc.sz.y, rsc.sz.z, rsc.sz.w);
         } else {
@@ -368,17 +383,20 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
         v_fma_s<C>(o2, qv.x, qv.y, x[r]);
       }
     }
-    if (STORE != BRS_STORE_FP32 && i0 + NRB < nlo) prefetch();
-    if constexpr (STORE == BRS_STORE_FP32) {
+    if (STORE != BRS_STORE_FP32 && !src32 && i0 + NRB < nlo) prefetch();
+    if (STORE == BRS_STORE_FP32 || dst32) {
+      // FP32 rows: the stored state (FP32 storage) or the interval state
 #pragma unroll
       for (int r = 0; r < NRB; ++r) {
-        float* dst = (float*)hout + (size_t)(i0 + r) * D + col0;
+        float* dst = (STORE == BRS_STORE_FP32) ? (float*)hout + (size_t)(i0 + r) * D + col0
+                                              : s32h + (size_t)(i0 + r) * D + col0;
         if constexpr (C == 4) *(float4*)dst = make_float4(x[r][0], x[r][1], x[r][2], x[r][3]);
         else if constexpr (C == 2) *(float2*)dst = make_float2(x[r][0], x[r][1]);
         else *dst = x[r][0];
       }
       continue;
-    } else {
+    }
+    if constexpr (STORE != BRS_STORE_FP32) {
       if (!int8_batch) {
         // protected rows: FP16, nearest
         uint32_t ovf = 0;
@@ -624,6 +642,14 @@ static cudaError_t launch_db(const DecodeArgs& a, int store, bool had, cudaStrea
     case BRS_ROUND_STOCHASTIC: return launch_dbm<D, BLOCK, BRS_ROUND_STOCHASTIC>(a, store, had, st);
     case BRS_ROUND_ERRFEEDBACK: return launch_dbm<D, BLOCK, BRS_ROUND_ERRFEEDBACK>(a, store, had, st);
   }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_decode_deferred(const DecodeArgs& a, int d, bool had, cudaStream_t st) {
+  if (d == 128 && a.block == 128) return launch_db<128, 128>(a, BRS_STORE_DAMP, had, st);
+  if (d == 128 && a.block == 32) return launch_db<128, 32>(a, BRS_STORE_DAMP, had, st);
+  if (d == 64 && a.block == 64) return launch_db<64, 64>(a, BRS_STORE_DAMP, had, st);
+  if (d == 32 && a.block == 32) return launch_db<32, 32>(a, BRS_STORE_DAMP, had, st);
   return cudaErrorInvalidValue;
 }
 

@@ -19,6 +19,7 @@ class LayerState:
         self.aux = torch.zeros(max(aux, 16), dtype=torch.uint8, device=self.device)
         self.stats = torch.zeros(max(stats, 16), dtype=torch.uint8, device=self.device)
         self.workspace = torch.zeros(ws, dtype=torch.uint8, device=self.device)
+        self.state32 = None            # FP32 state between write-backs (deferred write-back)
         self.perm = None
         if perm is not None:
             self.perm = torch.as_tensor(perm, dtype=torch.int16).contiguous().to(self.device)
@@ -40,6 +41,14 @@ class LayerState:
         self.stats.zero_()
 
     def step(self, wb: brs.WriteBack, t: int, q, k, v, beta, decay, o, packed_out=None):
+        if wb.C > 1:
+            # deferred write-back: the FP32 state between write-backs
+            if self.state32 is None:
+                self.state32 = torch.zeros(brs.decode_state32_bytes(self.layout) // 4, dtype=torch.float32,
+                                           device=self.device)
+            brs.decode_step_deferred(self.layout, wb, t, self.packed, self.aux, self.workspace, self.state32,
+                                     self.perm, q, k, v, beta, decay, o)
+            return self.packed
         out = self.packed if packed_out is None else packed_out
         brs.decode_step(self.layout, wb, t, self.packed, out, self.aux, self.stats,
                         self.workspace, self.perm, q, k, v, beta, decay, o)

@@ -72,6 +72,8 @@ WORKLOADS = {
                               hadamard=0, avg_bits=4.0, b_min=2, b_max=8, seed=3),
     "kda_prefill": Workload("kda_prefill", B=8, H=32, d=128, T=8192, k_hi=16, block=128, C=64,
                             seed=4),
+    # decode with deferred write-back every 8 tokens (a NEXT configuration)
+    "kda_decode_c8": Workload("kda_decode_c8", B=64, H=32, d=128, T=1024, k_hi=16, block=128, C=8, seed=1),
 }
 
 

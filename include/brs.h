@@ -184,6 +184,30 @@ brs_status brs_decode_step(const brs_layout* L, const brs_writeback* wb, int64_t
                            const uint16_t* k, const uint16_t* v, const float* beta,
                            const float* decay, float* o, void* stream);
 
+/* Decode with deferred write-back ([LB] Accumulated readout error: the state
+ * is written back every C tokens; between write-backs it is carried in FP32).
+ * DAMP storage.  One token for every head, as brs_decode_step, with write-back
+ * rounding `wb` applied when (step + 1) % C == 0; the other tokens leave the
+ * stored state untouched and carry the updated FP32 state in `state32`:
+ *   state32: device, brs_decode_state32_bytes(L) bytes, [B][H][d][d] FP32 in
+ *     stored row order, each tier in the basis its arithmetic uses (INT8-tier
+ *     rows after the Hadamard, FP16-tier rows in the value basis).  Read when
+ *     step % C != 0 (else the stored state is read), written when
+ *     (step + 1) % C != 0.  May be NULL when C == 1.
+ *   packed: stored state, updated in place at write-backs.  aux: residuals
+ *     (error feedback), used and updated at write-backs only.
+ *   workspace: flag word (as brs_decode_step).
+ * Calls must cover consecutive steps, starting at a multiple of C, for the
+ * result to equal the recurrence with write-back every C tokens (the state
+ * between write-backs is exactly the FP32 state of the token-by-token
+ * arithmetic).  C == 1 is brs_decode_step.  Returns BRS_EUNSUPPORTED for
+ * other storage formats or shapes outside brs_decode_step's. */
+size_t brs_decode_state32_bytes(const brs_layout* L);
+brs_status brs_decode_step_deferred(const brs_layout* L, const brs_writeback* wb, int64_t step, void* packed,
+                                    void* aux, void* workspace, void* state32, const int16_t* perm,
+                                    const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* beta,
+                                    const float* decay, float* o, void* stream);
+
 /* Chunked prefill with deferred write-back ([LB] Accumulated readout error:
  * write-back once per prefill chunk; [LB] Protocol).  Tokens
  * [step0, step0 + T) of every (sequence, head) with write-back after every

@@ -11,7 +11,7 @@ from conftest import ROOT
 
 def _declared():
     src = open(os.path.join(ROOT, "include", "brs.h")).read()
-    return sorted(set(re.findall(r"\b(brs_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(brs_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_header_declarations_exported():
