@@ -21,6 +21,7 @@
 // row, so each sum over rows is a lane-local fmaf chain in row order.
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <type_traits>
 
 #include "brs_device.cuh"
 #include "brs_internal.h"
@@ -40,40 +41,52 @@ struct __align__(16) VbRow {
   float pad[2];
 };
 
-template <int D>
+template <int D, bool WIDE>
 struct __align__(16) VbSmem {
   VbRow row[D];
   float R[D];                    // row ranges (phase 0)
   float y[kVbBatch][D + 4];      // one batch of target magnitudes (phase 1), rows 16-byte aligned
-  uint32_t pk[kVbBatch][32];     // bit-packed output rows of the batch
+  uint32_t pk[kVbBatch][WIDE ? 64 : 32];   // bit-packed output rows of the batch (widths up to 16 / 8)
   float pstep[kVbBatch], pinv[kVbBatch];
 };
 
-// decode the CPL codes of lane `lane` in one input row
-template <int C>
+// decode the CPL codes of lane `lane` in one input row (widths up to 8: C *
+// width <= 32 bits over one or two words; WIDE, up to 16: <= 64 bits over up
+// to three words)
+template <int C, bool WIDE>
 __device__ __forceinline__ void vb_dequant(float (&x)[C], const uint8_t* rowbase, const VbRow& r, int lane) {
   const uint32_t* rp = (const uint32_t*)rowbase;
   const int sb = C * lane * r.bw;
   const int sh = sb & 31;
-  uint32_t chunk = __ldg(rp + (sb >> 5)) >> sh;
-  if (sh + C * r.bw > 32) chunk |= __ldg(rp + (sb >> 5) + 1) << (32 - sh);
+  uint64_t chunk;
+  if constexpr (WIDE) {
+    const int w0 = sb >> 5, need = sh + C * r.bw;
+    uint64_t lo = __ldg(rp + w0);
+    if (need > 32) lo |= (uint64_t)__ldg(rp + w0 + 1) << 32;
+    chunk = lo >> sh;
+    if (need > 64) chunk |= (uint64_t)__ldg(rp + w0 + 2) << (64 - sh);
+  } else {
+    uint32_t c32 = __ldg(rp + (sb >> 5)) >> sh;
+    if (sh + C * r.bw > 32) c32 |= __ldg(rp + (sb >> 5) + 1) << (32 - sh);
+    chunk = c32;
+  }
   const uint32_t mask = (1u << r.bw) - 1u;
 #pragma unroll
   for (int c = 0; c < C; ++c) {
-    const int qv = (int)((chunk >> (c * r.bw)) & mask) - r.n;
+    const int qv = (int)((uint32_t)(chunk >> (c * r.bw)) & mask) - r.n;
     x[c] = __fmul_rn(__fsub_rn(__int_as_float(0x4B400000 + qv), kRoundMagic), r.step);  // (u - n) * step
   }
 }
 
-template <int D, int PHASE, int MODE>
+template <int D, int PHASE, int MODE, bool WIDE>
 __global__ void __launch_bounds__(32 * kVbWarps) varbit_kernel(const VbArgs a) {
   constexpr int C = D / 32;
   static_assert(D == 128, "variable-width decode is built for d = 128");
-  __shared__ VbSmem<D> smem_all[kVbWarps];
+  __shared__ VbSmem<D, WIDE> smem_all[kVbWarps];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int head = blockIdx.x * kVbWarps + warp;
   if (head >= a.B * a.H) return;
-  VbSmem<D>& sm = smem_all[warp];
+  VbSmem<D, WIDE>& sm = smem_all[warp];
   const int b = head / a.H, h = head - b * a.H;
   const int rows = a.H * D;
   const int col0 = C * lane;
@@ -114,7 +127,7 @@ __global__ void __launch_bounds__(32 * kVbWarps) varbit_kernel(const VbArgs a) {
   for (int i = 0; i < D; ++i) {
     const VbRow r = sm.row[i];
     float x[C];
-    vb_dequant<C>(x, pay_in + r.off, r, lane);
+    vb_dequant<C, WIDE>(x, pay_in + r.off, r, lane);
 #pragma unroll
     for (int c = 0; c < C; c += 2) {
       mul2(x[c], x[c + 1], r.ka.z, r.ka.w, x[c], x[c + 1]);
@@ -147,7 +160,7 @@ __global__ void __launch_bounds__(32 * kVbWarps) varbit_kernel(const VbArgs a) {
 #pragma unroll
     for (int r = 0; r < kVbBatch; ++r) {
       const VbRow rr = sm.row[i0 + r];
-      vb_dequant<C>(x[r], pay_in + rr.off, rr, lane);
+      vb_dequant<C, WIDE>(x[r], pay_in + rr.off, rr, lane);
 #pragma unroll
       for (int c = 0; c < C; c += 2) {
         mul2(x[r][c], x[r][c + 1], rr.ka.z, rr.ka.w, x[r][c], x[r][c + 1]);
@@ -273,7 +286,7 @@ __global__ void __launch_bounds__(32 * kVbWarps) varbit_kernel(const VbArgs a) {
         sm.pinv[jr] = good ? __frcp_rn(step) : 0.0f;
         sc_out[i0 + jr] = bbits;
       }
-      for (int k = lane; k < kVbBatch * 32; k += 32) (&sm.pk[0][0])[k] = 0u;
+      for (int k = lane; k < kVbBatch * (WIDE ? 64 : 32); k += 32) (&sm.pk[0][0])[k] = 0u;
       __syncwarp();
       // ---- codes of my columns, bit-packed into the batch rows
 #pragma unroll
@@ -289,18 +302,26 @@ __global__ void __launch_bounds__(32 * kVbWarps) varbit_kernel(const VbArgs a) {
           rnd = philox4x32_10(make_uint4((uint32_t)((i * D + col0) / 4), (uint32_t)a.step, (uint32_t)h, (uint32_t)b),
                               make_uint2((uint32_t)a.seed, (uint32_t)(a.seed >> 32)));
         const uint32_t words[4] = {rnd.x >> 8, rnd.y >> 8, rnd.z >> 8, rnd.w >> 8};
-        uint32_t chunk = 0;
+        using chunk_t = std::conditional_t<WIDE, uint64_t, uint32_t>;
+        chunk_t chunk = 0;
 #pragma unroll
         for (int c = 0; c < C; ++c) {
           const float t = __fmul_rn(x[r][c], inv);
           float qf = (MODE == BRS_ROUND_STOCHASTIC) ? sr_round(t, words[c]) : rintf(t);
           qf = fminf(fmaxf(qf, -rfn), rfn);
           qv[c] = qf;
-          chunk |= (uint32_t)((int)qf + rn) << (c * rbw);
+          chunk |= (chunk_t)(uint32_t)((int)qf + rn) << (c * rbw);
         }
-        const int sbit = C * lane * rbw;
-        atomicOr(&sm.pk[r][sbit >> 5], chunk << (sbit & 31));
-        if ((sbit & 31) + C * rbw > 32) atomicOr(&sm.pk[r][(sbit >> 5) + 1], chunk >> (32 - (sbit & 31)));
+        const int sbit = C * lane * rbw, sh = sbit & 31, w0 = sbit >> 5;
+        if constexpr (WIDE) {
+          atomicOr(&sm.pk[r][w0], (uint32_t)(chunk << sh));
+          if (sh + C * rbw > 32) atomicOr(&sm.pk[r][w0 + 1], (uint32_t)(chunk >> (32 - sh)));
+          if (sh + C * rbw > 64) atomicOr(&sm.pk[r][w0 + 2], (uint32_t)(chunk >> (64 - sh)));
+        } else {
+          const uint32_t c32 = (uint32_t)chunk;
+          atomicOr(&sm.pk[r][w0], c32 << sh);
+          if (sh + C * rbw > 32) atomicOr(&sm.pk[r][w0 + 1], c32 >> (32 - sh));
+        }
         if constexpr (MODE == BRS_ROUND_ERRFEEDBACK) {
           uint16_t e16[C];
 #pragma unroll
@@ -319,7 +340,11 @@ __global__ void __launch_bounds__(32 * kVbWarps) varbit_kernel(const VbArgs a) {
       for (int r = 0; r < kVbBatch; ++r) {
         const int i = i0 + r;
         const int nw = D * wd_out[i] / 32;               // 32-bit words of the row
-        if (lane < nw) ((uint32_t*)(pay_out + of_out[i]))[lane] = sm.pk[r][lane];
+        if constexpr (WIDE) {
+          for (int k = lane; k < nw; k += 32) ((uint32_t*)(pay_out + of_out[i]))[k] = sm.pk[r][k];
+        } else {
+          if (lane < nw) ((uint32_t*)(pay_out + of_out[i]))[lane] = sm.pk[r][lane];
+        }
       }
       __syncwarp();
     }
@@ -370,16 +395,22 @@ __global__ void __launch_bounds__(32 * kVbWarps) varbit_kernel(const VbArgs a) {
 
 cudaError_t launch_varbit_offsets(const VbArgs& a, cudaStream_t st);
 
-template <int PHASE>
-static cudaError_t launch_phase(const VbArgs& a, cudaStream_t st) {
+template <int PHASE, bool WIDE>
+static cudaError_t launch_phase_w(const VbArgs& a, cudaStream_t st) {
   const dim3 grid((a.B * a.H + kVbWarps - 1) / kVbWarps), block(32 * kVbWarps);
   switch (a.mode) {
-    case BRS_ROUND_NEAREST: varbit_kernel<128, PHASE, BRS_ROUND_NEAREST><<<grid, block, 0, st>>>(a); break;
-    case BRS_ROUND_STOCHASTIC: varbit_kernel<128, PHASE, BRS_ROUND_STOCHASTIC><<<grid, block, 0, st>>>(a); break;
-    case BRS_ROUND_ERRFEEDBACK: varbit_kernel<128, PHASE, BRS_ROUND_ERRFEEDBACK><<<grid, block, 0, st>>>(a); break;
+    case BRS_ROUND_NEAREST: varbit_kernel<128, PHASE, BRS_ROUND_NEAREST, WIDE><<<grid, block, 0, st>>>(a); break;
+    case BRS_ROUND_STOCHASTIC: varbit_kernel<128, PHASE, BRS_ROUND_STOCHASTIC, WIDE><<<grid, block, 0, st>>>(a); break;
+    case BRS_ROUND_ERRFEEDBACK: varbit_kernel<128, PHASE, BRS_ROUND_ERRFEEDBACK, WIDE><<<grid, block, 0, st>>>(a); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
+}
+
+// widths above 8 (b_max up to 16) take the wide packing
+template <int PHASE>
+static cudaError_t launch_phase(const VbArgs& a, cudaStream_t st) {
+  return a.b_max > 8 ? launch_phase_w<PHASE, true>(a, st) : launch_phase_w<PHASE, false>(a, st);
 }
 
 cudaError_t launch_varbit_decode(const VbArgs& a, cudaStream_t st) {

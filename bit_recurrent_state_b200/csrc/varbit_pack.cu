@@ -78,7 +78,7 @@ __global__ void varbit_pack_kernel(const VbPackArgs a) {
   }
   ((uint16_t*)(packed + a.sec.off_scale))[(size_t)b * rows + r] = best_bits;
   const float inv = (best_step != 0.0f && isfinite(best_step)) ? __frcp_rn(best_step) : 0.0f;
-  uint32_t words[32];
+  uint32_t words[64];                                          // d * 16 bits at most
   for (int k = 0; k < 4 * bw; ++k) words[k] = 0u;
   for (int j = 0; j < D; ++j) {
     const uint32_t u = (uint32_t)((int)varbit_nearest(x[j], inv, fn) + n);

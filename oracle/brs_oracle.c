@@ -880,7 +880,8 @@ static int layout_ok(const orc_layout* L) {
     if (L->k_hi < 0 || L->k_hi > L->d || L->block <= 0 || L->d % L->block) return 0;
   }
   if (L->storage == ORC_STORE_VARBIT) {
-    if (L->hadamard || L->b_min < 2 || L->b_max > 8 || L->b_min > L->b_max) return 0;
+    /* b_max = 8, or 16 at C = 1 ([LB] State bit allocation) */
+    if (L->hadamard || L->b_min < 2 || L->b_max > 16 || L->b_min > L->b_max) return 0;
     double tot = L->avg_bits * (double)(L->H * L->d);
     if (tot != floor(tot)) return 0;
   }

@@ -57,12 +57,16 @@ def _compare_step(w, cfg, pg, po, og, oo, tag, seqs=None):
     return flips
 
 
-@pytest.mark.parametrize("mode,scope", [("nearest", 1), ("stochastic", 1), ("errfeedback", 1), ("nearest", 0)])
-def test_varbit_teacher_forced(mode, scope):
+@pytest.mark.parametrize("mode,scope,b_max", [("nearest", 1, 8), ("stochastic", 1, 8), ("errfeedback", 1, 8),
+                                             ("nearest", 0, 8), ("nearest", 1, 16), ("errfeedback", 1, 16),
+                                             ("stochastic", 0, 16)])
+def test_varbit_teacher_forced(mode, scope, b_max):
+    """b_max = 16 as at C = 1: widths up to 16 bits, a lane's four codes
+    spanning up to three words of the row payload."""
     import torch
     from bit_recurrent_state_b200 import brs
     from oracle import oracle as O
-    w = _vb_workload(mode=mode)
+    w = _vb_workload(mode=mode, b_max=b_max, avg_bits=4.0 if b_max == 8 else 6.0)
     cfg = oracle_cfg(w)
     cfg.budget_scope = scope
     packed_o, aux_o, stats_o = O.new_state(cfg)
@@ -88,21 +92,22 @@ def test_varbit_teacher_forced(mode, scope):
     assert flips <= 2
 
 
-def test_varbit_pack_unpack_match_oracle():
+@pytest.mark.parametrize("b_max", [8, 16])
+def test_varbit_pack_unpack_match_oracle(b_max):
     import torch
     from bit_recurrent_state_b200 import brs
     from bit_recurrent_state_b200.state import LayerState
     from oracle import oracle as O
-    w = _vb_workload()
+    w = _vb_workload(b_max=b_max)
     cfg = oracle_cfg(w)
     rng = np.random.default_rng(3)
     S = (rng.standard_normal((w.B, w.H, w.d, w.d)) * rng.uniform(0.01, 2, (w.B, w.H, w.d, 1))).astype(np.float32)
-    # widths 2..8 that fill the budget exactly: move bits between random rows
+    # widths 2..b_max that fill the budget exactly: move bits between random rows
     widths = np.full((w.B, w.H * w.d), 4, np.int64)
     for b in range(w.B):
         for _ in range(3000):
             i, j = rng.integers(w.H * w.d, size=2)
-            if widths[b, i] < 8 and widths[b, j] > 2 and i != j:
+            if widths[b, i] < b_max and widths[b, j] > 2 and i != j:
                 widths[b, i] += 1
                 widths[b, j] -= 1
     widths = widths.astype(np.uint8)

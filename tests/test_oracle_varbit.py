@@ -9,12 +9,14 @@ from bit_recurrent_state_b200 import synth
 from ref64 import bf16_to_f64, dense_step, f16_bits_to_f64, varbit_row_codes, varbit_sections
 
 
-@pytest.mark.parametrize("mode", [0, 1, 2])
-def test_varbit_teacher_forced_fp64(orc, mode):
+@pytest.mark.parametrize("mode,b_max", [(0, 8), (1, 8), (2, 8), (0, 16), (2, 16)])
+def test_varbit_teacher_forced_fp64(orc, mode, b_max):
+    """b_max = 8, and 16 as at C = 1 (widths up to 16 bits, codes that span
+    words of the row payload)."""
     B, H, d, T = 2, 2, 32, 6
     w = synth.Workload("t", B=B, H=H, d=d, T=T, storage="varbit", hadamard=0, seed=20 + mode)
     cfg = orc.Config(B=B, H=H, d=d, storage=orc.STORE_VARBIT, hadamard=0, avg_bits=4.0,
-                     b_min=2, b_max=8, budget_scope=1)
+                     b_min=2, b_max=b_max, budget_scope=1)
     inp_all = synth.run_inputs(w, 0, T)
     packed, aux, stats = orc.new_state(cfg)
     lam = (1 - 2 / 65)
@@ -55,7 +57,7 @@ def test_varbit_teacher_forced_fp64(orc, mode):
             rms = np.sqrt(np.mean(Rr.reshape(H, d) ** 2, axis=1))
             Rt = (Rr.reshape(H, d) / rms[:, None]).ravel()
             c = gam * Rt ** 2
-            bits64, _ = orc.allocate_bits(c, 4.0, 2, 8)
+            bits64, _ = orc.allocate_bits(c, 4.0, 2, b_max)
             bstar = 4.0 + 0.5 * np.log2(c / np.exp(np.mean(np.log(c))))
             diff = bits64 != wd[b]
             if diff.any():
@@ -72,10 +74,12 @@ def test_varbit_teacher_forced_fp64(orc, mode):
                     if D == 0:
                         assert np.all(qv == 0)
                         continue
-                    lev = np.arange(-nl, nl + 1) * D
-                    dist = np.abs(x[:, None] - lev[None, :])
-                    got = dist[np.arange(d), qv + nl]
-                    assert np.all(got - dist.min(axis=1) <= 1e-4 * D)
+                    # the nearest level lies among the neighbours of round(x / D)
+                    qn = np.clip(np.rint(x / D), -nl, nl).astype(int)
+                    cand = np.clip(qn[:, None] + np.array([-1, 0, 1])[None, :], -nl, nl)
+                    best = np.min(np.abs(x[:, None] - cand * D), axis=1)
+                    got = np.abs(x - qv * D)
+                    assert np.all(got - best <= 1e-4 * D)
     assert near_ties <= 2
 
 
