@@ -47,7 +47,7 @@ brs_status check_layout(const brs_layout* L) {
       return fail(BRS_EINVAL, "block must be a power of two in [4, d] (got %d)", L->block);
   } else if (L->storage == BRS_STORE_VARBIT) {
     if (L->hadamard) return fail(BRS_EUNSUPPORTED, "variable-width storage is stored without the Hadamard");
-    if (L->b_min < 2 || L->b_max > 16 || L->b_min > L->b_max) return fail(BRS_EINVAL, "need 2 <= b_min <= b_max <= 16");
+    if (L->b_min < 1 || L->b_max > 16 || L->b_min > L->b_max) return fail(BRS_EINVAL, "need 1 <= b_min <= b_max <= 16");
     const double tot = L->avg_bits * (double)L->H * (double)L->d;
     if (tot != std::floor(tot)) return fail(BRS_EINVAL, "avg_bits * H * d must be an integer");
     if (L->avg_bits < L->b_min || L->avg_bits > L->b_max) return fail(BRS_EINVAL, "avg_bits outside [b_min, b_max]");

@@ -37,8 +37,9 @@ struct __align__(16) VbRow {
   float step;                    // stored step of the input row
   int bw;                        // input width
   uint32_t off;                  // input byte offset within the sequence payload
-  int n;                         // 2^(bw-1) - 1
-  float pad[2];
+  int n;                         // 2^(bw-1) - 1 (1 for one-bit rows)
+  int one;                       // one-bit row: level = 2 u - 1
+  float pad;
 };
 
 template <int D, bool WIDE>
@@ -53,7 +54,7 @@ struct __align__(16) VbSmem {
 // decode the CPL codes of lane `lane` in one input row (widths up to 8: C *
 // width <= 32 bits over one or two words; WIDE, up to 16: <= 64 bits over up
 // to three words)
-template <int C, bool WIDE>
+template <int C, bool WIDE, bool ONE>
 __device__ __forceinline__ void vb_dequant(float (&x)[C], const uint8_t* rowbase, const VbRow& r, int lane) {
   const uint32_t* rp = (const uint32_t*)rowbase;
   const int sb = C * lane * r.bw;
@@ -73,12 +74,13 @@ __device__ __forceinline__ void vb_dequant(float (&x)[C], const uint8_t* rowbase
   const uint32_t mask = (1u << r.bw) - 1u;
 #pragma unroll
   for (int c = 0; c < C; ++c) {
-    const int qv = (int)((uint32_t)(chunk >> (c * r.bw)) & mask) - r.n;
+    const uint32_t u = (uint32_t)(chunk >> (c * r.bw)) & mask;
+    const int qv = ONE ? (int)(u << r.one) - r.n : (int)u - r.n;   // one bit: 2u - 1
     x[c] = __fmul_rn(__fsub_rn(__int_as_float(0x4B400000 + qv), kRoundMagic), r.step);  // (u - n) * step
   }
 }
 
-template <int D, int PHASE, int MODE, bool WIDE>
+template <int D, int PHASE, int MODE, bool WIDE, bool ONE>
 __global__ void __launch_bounds__(32 * kVbWarps) varbit_kernel(const VbArgs a) {
   constexpr int C = D / 32;
   static_assert(D == 128, "variable-width decode is built for d = 128");
@@ -109,8 +111,9 @@ __global__ void __launch_bounds__(32 * kVbWarps) varbit_kernel(const VbArgs a) {
     r.step = f16_to_f32(sc_in[i]);
     r.bw = wd_in[i];
     r.off = of_in[i];
-    r.n = (1 << (r.bw - 1)) - 1;
-    r.pad[0] = r.pad[1] = 0.f;
+    r.one = r.bw == 1;
+    r.n = r.one ? 1 : (1 << (r.bw - 1)) - 1;
+    r.pad = 0.f;
     sm.row[i] = r;
   }
   float vv[C];
@@ -127,7 +130,7 @@ __global__ void __launch_bounds__(32 * kVbWarps) varbit_kernel(const VbArgs a) {
   for (int i = 0; i < D; ++i) {
     const VbRow r = sm.row[i];
     float x[C];
-    vb_dequant<C, WIDE>(x, pay_in + r.off, r, lane);
+    vb_dequant<C, WIDE, ONE>(x, pay_in + r.off, r, lane);
 #pragma unroll
     for (int c = 0; c < C; c += 2) {
       mul2(x[c], x[c + 1], r.ka.z, r.ka.w, x[c], x[c + 1]);
@@ -160,7 +163,7 @@ __global__ void __launch_bounds__(32 * kVbWarps) varbit_kernel(const VbArgs a) {
 #pragma unroll
     for (int r = 0; r < kVbBatch; ++r) {
       const VbRow rr = sm.row[i0 + r];
-      vb_dequant<C, WIDE>(x[r], pay_in + rr.off, rr, lane);
+      vb_dequant<C, WIDE, ONE>(x[r], pay_in + rr.off, rr, lane);
 #pragma unroll
       for (int c = 0; c < C; c += 2) {
         mul2(x[r][c], x[r][c + 1], rr.ka.z, rr.ka.w, x[r][c], x[r][c + 1]);
@@ -224,7 +227,8 @@ __global__ void __launch_bounds__(32 * kVbWarps) varbit_kernel(const VbArgs a) {
       // ---- fitted step: row jr, candidates m = q, q+4, q+8, q+12
       const int q4 = lane & 3;
       const int bw = wd_out[i0 + jr];
-      const int n = (1 << (bw - 1)) - 1;
+      const bool one = ONE && bw == 1;             // one-bit row: no fitted step
+      const int n = one ? 1 : (1 << (bw - 1)) - 1;
       const float fn = (float)n;
       float st[4], iv[4], E[4];
       uint16_t sb[4];
@@ -236,7 +240,7 @@ __global__ void __launch_bounds__(32 * kVbWarps) varbit_kernel(const VbArgs a) {
       }
       const float* yrow = sm.y[jr];
 #pragma unroll 2
-      for (int j4 = 0; j4 < D; j4 += 4) {
+      for (int j4 = 0; j4 < (one ? 0 : D); j4 += 4) {
         const float4 y4 = *(const float4*)&yrow[j4];
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
@@ -278,6 +282,17 @@ __global__ void __launch_bounds__(32 * kVbWarps) varbit_kernel(const VbArgs a) {
         if (take) { bm = om; bE = oE; bbits = ob; }
       }
       if (R == 0.0f) { bm = 0; bbits = 0; }
+      if (one) {
+        // one-bit row ([LB] Levels and storage): the sign times the row's mean
+        // absolute value, the magnitudes summed in element order by the row's
+        // first lane, times 1/d, stored as the FP16 scale
+        if (q4 == 0) {
+          float sum = 0.0f;
+          for (int j = 0; j < D; ++j) sum = __fadd_rn(sum, yrow[j]);
+          bbits = f32_to_f16(__fmul_rn(sum, 1.0f / (float)D));
+        }
+        bm = 0;
+      }
       if (bm == 99) { bbits = 0x7c00u; if (q4 == 0) raise_flag(a.flags, BRS_FLAG_OVERFLOW); }
       if (q4 == 0) {
         const float step = f16_to_f32(bbits);
@@ -293,7 +308,8 @@ __global__ void __launch_bounds__(32 * kVbWarps) varbit_kernel(const VbArgs a) {
       for (int r = 0; r < kVbBatch; ++r) {
         const int i = i0 + r;
         const int rbw = wd_out[i];
-        const int rn = (1 << (rbw - 1)) - 1;
+        const bool rone = ONE && rbw == 1;
+        const int rn = rone ? 0 : (1 << (rbw - 1)) - 1;
         const float rfn = (float)rn;
         const float step = sm.pstep[r], inv = sm.pinv[r];
         float qv[C];
@@ -307,10 +323,25 @@ __global__ void __launch_bounds__(32 * kVbWarps) varbit_kernel(const VbArgs a) {
 #pragma unroll
         for (int c = 0; c < C; ++c) {
           const float t = __fmul_rn(x[r][c], inv);
-          float qf = (MODE == BRS_ROUND_STOCHASTIC) ? sr_round(t, words[c]) : rintf(t);
-          qf = fminf(fmaxf(qf, -rfn), rfn);
+          float qf;
+          uint32_t u;
+          if (rone) {
+            // one bit: +mu for a target >= 0 (nearest), or with probability
+            // (t + 1) / 2 (stochastic); the level is +-1
+            if (MODE == BRS_ROUND_STOCHASTIC) {
+              const float cc = fminf(fmaxf(sr_round(__fmul_rn(__fadd_rn(t, 1.0f), 0.5f), words[c]), 0.0f), 1.0f);
+              u = cc > 0.0f ? 1u : 0u;
+            } else {
+              u = x[r][c] >= 0.0f ? 1u : 0u;
+            }
+            qf = u ? 1.0f : -1.0f;
+          } else {
+            qf = (MODE == BRS_ROUND_STOCHASTIC) ? sr_round(t, words[c]) : rintf(t);
+            qf = fminf(fmaxf(qf, -rfn), rfn);
+            u = (uint32_t)((int)qf + rn);
+          }
           qv[c] = qf;
-          chunk |= (chunk_t)(uint32_t)((int)qf + rn) << (c * rbw);
+          chunk |= (chunk_t)u << (c * rbw);
         }
         const int sbit = C * lane * rbw, sh = sbit & 31, w0 = sbit >> 5;
         if constexpr (WIDE) {
@@ -324,11 +355,12 @@ __global__ void __launch_bounds__(32 * kVbWarps) varbit_kernel(const VbArgs a) {
         }
         if constexpr (MODE == BRS_ROUND_ERRFEEDBACK) {
           uint16_t e16[C];
+          const float lim = rone ? __fmul_rn(2.0f, step) : step;   // one bit: the distance between the levels
 #pragma unroll
           for (int c = 0; c < C; ++c) {
             float e = __fsub_rn(x[r][c], __fmul_rn(step, qv[c]));
-            if (e > step) e = step;
-            else if (e < -step) e = -step;
+            if (e > lim) e = lim;
+            else if (e < -lim) e = -lim;
             e16[c] = f32_to_f16(e);
           }
           *(uint2*)&auxh[(size_t)i * D + col0] =
@@ -395,22 +427,25 @@ __global__ void __launch_bounds__(32 * kVbWarps) varbit_kernel(const VbArgs a) {
 
 cudaError_t launch_varbit_offsets(const VbArgs& a, cudaStream_t st);
 
-template <int PHASE, bool WIDE>
+template <int PHASE, bool WIDE, bool ONE>
 static cudaError_t launch_phase_w(const VbArgs& a, cudaStream_t st) {
   const dim3 grid((a.B * a.H + kVbWarps - 1) / kVbWarps), block(32 * kVbWarps);
   switch (a.mode) {
-    case BRS_ROUND_NEAREST: varbit_kernel<128, PHASE, BRS_ROUND_NEAREST, WIDE><<<grid, block, 0, st>>>(a); break;
-    case BRS_ROUND_STOCHASTIC: varbit_kernel<128, PHASE, BRS_ROUND_STOCHASTIC, WIDE><<<grid, block, 0, st>>>(a); break;
-    case BRS_ROUND_ERRFEEDBACK: varbit_kernel<128, PHASE, BRS_ROUND_ERRFEEDBACK, WIDE><<<grid, block, 0, st>>>(a); break;
+    case BRS_ROUND_NEAREST: varbit_kernel<128, PHASE, BRS_ROUND_NEAREST, WIDE, ONE><<<grid, block, 0, st>>>(a); break;
+    case BRS_ROUND_STOCHASTIC: varbit_kernel<128, PHASE, BRS_ROUND_STOCHASTIC, WIDE, ONE><<<grid, block, 0, st>>>(a); break;
+    case BRS_ROUND_ERRFEEDBACK: varbit_kernel<128, PHASE, BRS_ROUND_ERRFEEDBACK, WIDE, ONE><<<grid, block, 0, st>>>(a); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
 }
 
-// widths above 8 (b_max up to 16) take the wide packing
+// widths above 8 (b_max up to 16) take the wide packing, b_min = 1 the
+// one-bit rows
 template <int PHASE>
 static cudaError_t launch_phase(const VbArgs& a, cudaStream_t st) {
-  return a.b_max > 8 ? launch_phase_w<PHASE, true>(a, st) : launch_phase_w<PHASE, false>(a, st);
+  if (a.b_min == 1)
+    return a.b_max > 8 ? launch_phase_w<PHASE, true, true>(a, st) : launch_phase_w<PHASE, false, true>(a, st);
+  return a.b_max > 8 ? launch_phase_w<PHASE, true, false>(a, st) : launch_phase_w<PHASE, false, false>(a, st);
 }
 
 cudaError_t launch_varbit_decode(const VbArgs& a, cudaStream_t st) {

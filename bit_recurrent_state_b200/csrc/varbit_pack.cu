@@ -58,7 +58,15 @@ __global__ void varbit_pack_kernel(const VbPackArgs a) {
   for (int j = 0; j < D; ++j) R = fmaxf(R, fabsf(x[j]));
   uint16_t best_bits = 0;
   float best_step = 0.0f;
-  if (R > 0.0f) {
+  if (bw == 1) {
+    // one bit: the sign times the row's mean absolute value (FP16), the
+    // magnitudes summed in element order
+    float sum = 0.0f;
+    for (int j = 0; j < D; ++j) sum = __fadd_rn(sum, fabsf(x[j]));
+    best_bits = f32_to_f16(__fmul_rn(sum, 1.0f / (float)D));
+    best_step = f16_to_f32(best_bits);
+    if (!isfinite(best_step)) raise_flag(a.flags, BRS_FLAG_OVERFLOW);
+  } else if (R > 0.0f) {
     float bestE = 0.0f;
     int best = -1;
     for (int m = 0; m < 16; ++m) {
@@ -81,7 +89,7 @@ __global__ void varbit_pack_kernel(const VbPackArgs a) {
   uint32_t words[64];                                          // d * 16 bits at most
   for (int k = 0; k < 4 * bw; ++k) words[k] = 0u;
   for (int j = 0; j < D; ++j) {
-    const uint32_t u = (uint32_t)((int)varbit_nearest(x[j], inv, fn) + n);
+    const uint32_t u = (bw == 1) ? (x[j] >= 0.0f ? 1u : 0u) : (uint32_t)((int)varbit_nearest(x[j], inv, fn) + n);
     const int bit = j * bw;
     words[bit >> 5] |= u << (bit & 31);
     if ((bit & 31) + bw > 32) words[(bit >> 5) + 1] |= u >> (32 - (bit & 31));
@@ -112,7 +120,8 @@ __global__ void varbit_unpack_kernel(const VbPackArgs a, const void* packed_v, f
     uint32_t u = src[bit >> 5] >> (bit & 31);
     if ((bit & 31) + bw > 32) u |= src[(bit >> 5) + 1] << (32 - (bit & 31));
     u &= (1u << bw) - 1u;
-    S[(size_t)row * D + j] = __fmul_rn((float)((int)u - n), step);
+    const int lv = (bw == 1) ? 2 * (int)u - 1 : (int)u - n;     // one bit: 2u - 1
+    S[(size_t)row * D + j] = __fmul_rn((float)lv, step);
   }
 }
 

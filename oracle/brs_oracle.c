@@ -248,6 +248,50 @@ int orc_varbit_row(const float* x, int n, int bw, int mode, uint64_t seed, int64
     float a = fabsf(tgt[j]);
     if (a > R) R = a;
   }
+  if (bw == 1) {
+    /* One bit ([LB] Levels and storage): the sign times the row's mean
+     * absolute value, that mean stored as the FP16 scale.  Mean: the
+     * absolute values summed in element order in FP32, times 1/n (n a power
+     * of two, so exact).  Code 1 holds +mu, code 0 holds -mu.  Nearest: 1
+     * for a target >= 0 (a zero target is a tie between the two levels and
+     * takes +mu).  Stochastic: +mu with probability (t/mu + 1)/2, clipped to
+     * [0, 1].  Error feedback: residual clipped to +-2 mu, the distance
+     * between the two levels. */
+    float sum = 0.0f;
+    for (int j = 0; j < n; ++j) sum = sum + fabsf(tgt[j]);
+    uint16_t mh = orc_f16_from_f32(sum * (1.0f / (float)n));
+    float mu = orc_f32_from_f16(mh);
+    int okm = isfinite(mu);
+    if (!okm) flags |= ORC_EOVERFLOW;
+    float inv1 = (okm && mu != 0.0f) ? 1.0f / mu : 0.0f;
+    for (int j = 0; j < n; ++j) {
+      float t = tgt[j] * inv1;
+      int u;
+      if (mode == ORC_ROUND_STOCHASTIC) {
+        float c = sr_round((t + 1.0f) * 0.5f, sr_bits24(seed, step, h, b, elem0 + j));
+        if (c < 0.0f) c = 0.0f;
+        if (c > 1.0f) c = 1.0f;
+        if (!(c == c)) c = 0.0f;
+        u = (int)c;
+      } else {
+        u = tgt[j] >= 0.0f ? 1 : 0;
+      }
+      q_out[j] = u;
+      if (t_out) t_out[j] = t;
+      if (mode == ORC_ROUND_ERRFEEDBACK) {
+        float xhat = okm ? (u ? mu : -mu) : 0.0f;
+        float e = tgt[j] - xhat;
+        float lim = okm ? 2.0f * mu : 0.0f;
+        if (e > lim) e = lim;
+        else if (e < -lim) e = -lim;
+        e_inout[j] = orc_f16_from_f32(e);
+      }
+    }
+    *delta_h = mh;
+    if (m_star) *m_star = 0;
+    free(tgt);
+    return flags;
+  }
   uint16_t dh = 0;
   int best = -1;
   if (R > 0.0f) {
@@ -740,7 +784,9 @@ static void varbit_load_seq(const orc_layout* L, const uint8_t* packed, int b, f
     float D = orc_f32_from_f16(sc[r]);
     for (int j = 0; j < d; ++j) {
       uint32_t u = get_bits(pay + of[r], (size_t)j * bw, bw);
-      S[(size_t)r * d + j] = (float)((int)u - nl) * D;
+      /* one bit: code 1 = +scale, 0 = -scale */
+      int lv = (bw == 1) ? 2 * (int)u - 1 : (int)u - nl;
+      S[(size_t)r * d + j] = (float)lv * D;
     }
   }
 }
@@ -880,8 +926,9 @@ static int layout_ok(const orc_layout* L) {
     if (L->k_hi < 0 || L->k_hi > L->d || L->block <= 0 || L->d % L->block) return 0;
   }
   if (L->storage == ORC_STORE_VARBIT) {
-    /* b_max = 8, or 16 at C = 1 ([LB] State bit allocation) */
-    if (L->hadamard || L->b_min < 2 || L->b_max > 16 || L->b_min > L->b_max) return 0;
+    /* b_min = 1 for row units, b_max = 8, or 16 at C = 1 ([LB] State bit
+     * allocation, Allocation units) */
+    if (L->hadamard || L->b_min < 1 || L->b_max > 16 || L->b_min > L->b_max) return 0;
     double tot = L->avg_bits * (double)(L->H * L->d);
     if (tot != floor(tot)) return 0;
   }

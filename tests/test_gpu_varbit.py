@@ -57,16 +57,19 @@ def _compare_step(w, cfg, pg, po, og, oo, tag, seqs=None):
     return flips
 
 
-@pytest.mark.parametrize("mode,scope,b_max", [("nearest", 1, 8), ("stochastic", 1, 8), ("errfeedback", 1, 8),
-                                             ("nearest", 0, 8), ("nearest", 1, 16), ("errfeedback", 1, 16),
-                                             ("stochastic", 0, 16)])
-def test_varbit_teacher_forced(mode, scope, b_max):
+@pytest.mark.parametrize("mode,scope,b_min,b_max,avg", [
+    ("nearest", 1, 2, 8, 4.0), ("stochastic", 1, 2, 8, 4.0), ("errfeedback", 1, 2, 8, 4.0),
+    ("nearest", 0, 2, 8, 4.0), ("nearest", 1, 2, 16, 6.0), ("errfeedback", 1, 2, 16, 6.0),
+    ("stochastic", 0, 2, 16, 6.0), ("nearest", 1, 1, 8, 2.0), ("stochastic", 1, 1, 8, 2.0),
+    ("errfeedback", 1, 1, 8, 2.0), ("nearest", 0, 1, 16, 3.0)])
+def test_varbit_teacher_forced(mode, scope, b_min, b_max, avg):
     """b_max = 16 as at C = 1: widths up to 16 bits, a lane's four codes
-    spanning up to three words of the row payload."""
+    spanning up to three words of the row payload; b_min = 1: one-bit rows
+    (the sign times the row's mean absolute value)."""
     import torch
     from bit_recurrent_state_b200 import brs
     from oracle import oracle as O
-    w = _vb_workload(mode=mode, b_max=b_max, avg_bits=4.0 if b_max == 8 else 6.0)
+    w = _vb_workload(mode=mode, b_min=b_min, b_max=b_max, avg_bits=avg)
     cfg = oracle_cfg(w)
     cfg.budget_scope = scope
     packed_o, aux_o, stats_o = O.new_state(cfg)
@@ -92,13 +95,13 @@ def test_varbit_teacher_forced(mode, scope, b_max):
     assert flips <= 2
 
 
-@pytest.mark.parametrize("b_max", [8, 16])
-def test_varbit_pack_unpack_match_oracle(b_max):
+@pytest.mark.parametrize("b_min,b_max", [(2, 8), (2, 16), (1, 8)])
+def test_varbit_pack_unpack_match_oracle(b_min, b_max):
     import torch
     from bit_recurrent_state_b200 import brs
     from bit_recurrent_state_b200.state import LayerState
     from oracle import oracle as O
-    w = _vb_workload(b_max=b_max)
+    w = _vb_workload(b_min=b_min, b_max=b_max)
     cfg = oracle_cfg(w)
     rng = np.random.default_rng(3)
     S = (rng.standard_normal((w.B, w.H, w.d, w.d)) * rng.uniform(0.01, 2, (w.B, w.H, w.d, 1))).astype(np.float32)
@@ -107,7 +110,7 @@ def test_varbit_pack_unpack_match_oracle(b_max):
     for b in range(w.B):
         for _ in range(3000):
             i, j = rng.integers(w.H * w.d, size=2)
-            if widths[b, i] < b_max and widths[b, j] > 2 and i != j:
+            if widths[b, i] < b_max and widths[b, j] > b_min and i != j:
                 widths[b, i] += 1
                 widths[b, j] -= 1
     widths = widths.astype(np.uint8)

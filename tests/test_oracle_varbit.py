@@ -9,14 +9,23 @@ from bit_recurrent_state_b200 import synth
 from ref64 import bf16_to_f64, dense_step, f16_bits_to_f64, varbit_row_codes, varbit_sections
 
 
-@pytest.mark.parametrize("mode,b_max", [(0, 8), (1, 8), (2, 8), (0, 16), (2, 16)])
-def test_varbit_teacher_forced_fp64(orc, mode, b_max):
+def _levels(codes, bw):
+    """Stored codes -> integer levels: offset binary, or +-1 for one-bit rows."""
+    codes = codes.astype(int)
+    return 2 * codes - 1 if bw == 1 else codes - (2 ** (bw - 1) - 1)
+
+
+@pytest.mark.parametrize("mode,b_min,b_max,avg", [(0, 2, 8, 4.0), (1, 2, 8, 4.0), (2, 2, 8, 4.0),
+                                                  (0, 2, 16, 4.0), (2, 2, 16, 4.0),
+                                                  (0, 1, 8, 2.0), (1, 1, 8, 2.0), (2, 1, 8, 2.0)])
+def test_varbit_teacher_forced_fp64(orc, mode, b_min, b_max, avg):
     """b_max = 8, and 16 as at C = 1 (widths up to 16 bits, codes that span
-    words of the row payload)."""
+    words of the row payload); b_min = 1 with one-bit rows (the sign times
+    the row's mean absolute value)."""
     B, H, d, T = 2, 2, 32, 6
     w = synth.Workload("t", B=B, H=H, d=d, T=T, storage="varbit", hadamard=0, seed=20 + mode)
-    cfg = orc.Config(B=B, H=H, d=d, storage=orc.STORE_VARBIT, hadamard=0, avg_bits=4.0,
-                     b_min=2, b_max=b_max, budget_scope=1)
+    cfg = orc.Config(B=B, H=H, d=d, storage=orc.STORE_VARBIT, hadamard=0, avg_bits=avg,
+                     b_min=b_min, b_max=b_max, budget_scope=1)
     inp_all = synth.run_inputs(w, 0, T)
     packed, aux, stats = orc.new_state(cfg)
     lam = (1 - 2 / 65)
@@ -27,10 +36,10 @@ def test_varbit_teacher_forced_fp64(orc, mode, b_max):
         inp = {k: v[t:t + 1] for k, v in inp_all.items()}
         o, fl, _ = orc.run(cfg, mode, 99, 1, t, inp, packed, aux=aux, stats=stats)
         assert fl == 0
-        pay0, sc0, wd0, of0 = varbit_sections(before, B, H, d, 4.0)
-        pay, sc, wd, of = varbit_sections(packed, B, H, d, 4.0)
+        pay0, sc0, wd0, of0 = varbit_sections(before, B, H, d, avg)
+        pay, sc, wd, of = varbit_sections(packed, B, H, d, avg)
         for b in range(B):
-            assert int(wd[b].astype(int).sum()) == 4 * H * d             # layer budget
+            assert int(wd[b].astype(int).sum()) == int(avg * H * d)       # layer budget
             np.testing.assert_array_equal(of[b][:-1], np.concatenate([[0], np.cumsum(wd[b].astype(int))[:-1]]) * (d // 8))
             Rr = np.zeros(H * d)
             S_new = np.zeros((H, d, d))
@@ -38,8 +47,8 @@ def test_varbit_teacher_forced_fp64(orc, mode, b_max):
                 S = np.zeros((d, d))
                 for i in range(d):
                     r = h * d + i
-                    bw = int(wd0[b, r]); nl = 2 ** (bw - 1) - 1
-                    S[i] = (varbit_row_codes(pay0[b], int(of0[b, r]), bw, d) - nl) * f16_bits_to_f64(sc0[b, r])
+                    bw = int(wd0[b, r])
+                    S[i] = _levels(varbit_row_codes(pay0[b], int(of0[b, r]), bw, d), bw) * f16_bits_to_f64(sc0[b, r])
                 k, q, v, a, beta = (bf16_to_f64(inp["k"][0, b, h]), bf16_to_f64(inp["q"][0, b, h]),
                                     bf16_to_f64(inp["v"][0, b, h]),
                                     inp["decay"][0, b, h].astype(np.float64), float(inp["beta"][0, b, h]))
@@ -57,17 +66,33 @@ def test_varbit_teacher_forced_fp64(orc, mode, b_max):
             rms = np.sqrt(np.mean(Rr.reshape(H, d) ** 2, axis=1))
             Rt = (Rr.reshape(H, d) / rms[:, None]).ravel()
             c = gam * Rt ** 2
-            bits64, _ = orc.allocate_bits(c, 4.0, 2, b_max)
-            bstar = 4.0 + 0.5 * np.log2(c / np.exp(np.mean(np.log(c))))
+            bits64, _ = orc.allocate_bits(c, avg, b_min, b_max)
+            bstar = avg + 0.5 * np.log2(c / np.exp(np.mean(np.log(c))))
             diff = bits64 != wd[b]
             if diff.any():
                 # only where b* sits next to a half-integer
                 assert np.all(np.abs(np.abs(bstar[diff] - np.floor(bstar[diff])) - 0.5) < 1e-6)
                 near_ties += int(diff.sum())
             # each row holds its nearest levels (deterministic) / adjacent ones (stochastic)
+            for r in range(H * d):
+                bw = int(wd[b, r])
+                if bw != 1:
+                    continue
+                # one-bit rows: scale = the mean absolute value (FP16), code = sign
+                x = S_new[r // d, r % d]
+                mu = f16_bits_to_f64(sc[b, r])
+                if mode != 2:                     # (error feedback quantizes x + residual)
+                    m64 = float(np.mean(np.abs(x)))
+                    assert abs(mu - m64) <= 2.0 ** -10 * m64 + 1e-12, (mu, m64)
+                if mode == 0:
+                    lv = _levels(varbit_row_codes(pay[b], int(of[b, r]), bw, d), 1)
+                    clear = np.abs(x) > 1e-6 * np.max(np.abs(x))
+                    np.testing.assert_array_equal(lv[clear], np.where(x[clear] >= 0, 1, -1))
             if mode == 0:
                 for r in range(H * d):
                     bw = int(wd[b, r]); nl = 2 ** (bw - 1) - 1
+                    if bw == 1:
+                        continue
                     D = f16_bits_to_f64(sc[b, r])
                     qv = varbit_row_codes(pay[b], int(of[b, r]), bw, d).astype(int) - nl
                     x = S_new[r // d, r % d]
