@@ -44,13 +44,24 @@ METRIC = "state-update tokens·heads/s and state HBM GB/s (% of B200 peak), deco
 UNIT = "tokens·heads/s"
 FALLBACK_HBM_GBS = 6650.0
 NLAYERS = 8
-KERNEL_SOURCES = ["bit_recurrent_state_b200/csrc/decode.cu", "bit_recurrent_state_b200/csrc/decode_tma.cu",
-                  "bit_recurrent_state_b200/csrc/brs_device.cuh"]
+# the sources of each decode kernel (a DRAM record stays valid while they hash the same)
+KERNEL_SOURCES = {
+    "tma": ["bit_recurrent_state_b200/csrc/decode_tma.cu", "bit_recurrent_state_b200/csrc/brs_device.cuh"],
+    "warp": ["bit_recurrent_state_b200/csrc/decode.cu", "bit_recurrent_state_b200/csrc/brs_device.cuh"],
+    "varbit": ["bit_recurrent_state_b200/csrc/varbit.cu", "bit_recurrent_state_b200/csrc/allocate.cu",
+               "bit_recurrent_state_b200/csrc/brs_device.cuh"],
+}
 
 
-def kernel_hash() -> str:
+def kernel_family(w) -> str:
+    if w.storage == "varbit":
+        return "varbit"
+    return "tma" if (w.storage == "damp" and w.d == 128 and w.C == 1) else "warp"
+
+
+def kernel_hash(family: str = "tma") -> str:
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
+    for p in KERNEL_SOURCES[family]:
         with open(os.path.join(ROOT, p), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -142,15 +153,15 @@ def prefill_traffic():
     return rec.get("dram_bytes_per_launch")
 
 
-def traffic_record(workload: str):
+def traffic_record(w):
     """DRAM bytes per launch from a committed ncu summary, only while the
-    kernel sources still hash to the profiled version."""
-    p = os.path.join(ROOT, "profiles", f"decode_{workload}_traffic.json")
+    sources of the workload's kernel still hash to the profiled version."""
+    p = os.path.join(ROOT, "profiles", f"decode_{w.name}_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         rec = json.load(f)
-    if rec.get("kernel_hash") != kernel_hash():
+    if rec.get("kernel_hash") != kernel_hash(kernel_family(w)):
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -606,7 +617,7 @@ def run_ours(args, w):
     ab = algorithmic_bytes(w)
     peak, src = peaks()
     achieved = ab["total"] / (ms_step * 1e-3) / 1e9
-    traffic = traffic_record(w.name)
+    traffic = traffic_record(w)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
