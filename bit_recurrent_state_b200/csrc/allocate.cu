@@ -92,6 +92,8 @@ __device__ __forceinline__ unsigned long long cand_key(double c, int level, bool
   return ~(unsigned long long)__double_as_longlong((0.75 * c) * ldexp(1.0, -2 * level));
 }
 
+// RPT rows per thread at most (8 for groups up to 4096 rows: fewer registers)
+template <int RPT>
 __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const AllocArgs a) {
   __shared__ AllocShared sh;
   const int t = threadIdx.x;
@@ -100,10 +102,10 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const AllocArgs
   const double* c = a.cost + (size_t)g * N;
   const int rpt = (N + kAllocThreads - 1) / kAllocThreads;   // rows per thread, contiguous
   const int r0 = t * rpt;
-  double cv[kMaxRowsPerThread];
-  int bv[kMaxRowsPerThread];
+  double cv[RPT];
+  int bv[RPT];
 #pragma unroll
-  for (int q = 0; q < kMaxRowsPerThread; ++q) {
+  for (int q = 0; q < RPT; ++q) {
     cv[q] = 0.0;
     bv[q] = 0;
     if (q < rpt && r0 + q < N) cv[q] = c[r0 + q];
@@ -112,7 +114,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const AllocArgs
   double ls = 0.0;
   int cnt = 0;
 #pragma unroll
-  for (int q = 0; q < kMaxRowsPerThread; ++q)
+  for (int q = 0; q < RPT; ++q)
     if (q < rpt && r0 + q < N && cv[q] > 0.0) {
       ls += log(cv[q]);
       ++cnt;
@@ -123,7 +125,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const AllocArgs
   // ---- rounded, clipped widths
   long long mysum = 0;
 #pragma unroll
-  for (int q = 0; q < kMaxRowsPerThread; ++q) {
+  for (int q = 0; q < RPT; ++q) {
     if (q < rpt && r0 + q < N) {
       int b;
       if (ncnt == 0) {
@@ -154,26 +156,55 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const AllocArgs
       __syncthreads();
       const unsigned long long pre = sh.prefix;
       const unsigned long long hmask = (shift == 56) ? 0ull : (~0ull << (shift + 8));
+      // a thread's candidates come in runs with the same digit (a row's
+      // levels differ by a factor of 4): count a run, add it once
+      unsigned run_digit = 0xffffffffu, run_n = 0;
 #pragma unroll
-      for (int q = 0; q < kMaxRowsPerThread; ++q) {
+      for (int q = 0; q < RPT; ++q) {
         if (q < rpt && r0 + q < N) {
           const int lo = dec ? a.b_min + 1 : bv[q], hi = dec ? bv[q] : a.b_max - 1;
           for (int L = lo; L <= hi; ++L) {
             const unsigned long long k = cand_key(cv[q], L, dec);
-            if ((k & hmask) == (pre & hmask)) atomicAdd(&sh.hist[(k >> shift) & 0xffu], 1u);
+            if ((k & hmask) == (pre & hmask)) {
+              const unsigned dg = (unsigned)((k >> shift) & 0xffu);
+              if (dg != run_digit) {
+                if (run_n) atomicAdd(&sh.hist[run_digit], run_n);
+                run_digit = dg;
+                run_n = 0;
+              }
+              ++run_n;
+            }
           }
         }
       }
+      if (run_n) atomicAdd(&sh.hist[run_digit], run_n);
       __syncthreads();
-      if (t == 0) {
-        int r = sh.rank;
-        unsigned digit = 0;
-        for (; digit < 256; ++digit) {
-          if (r <= (int)sh.hist[digit]) break;
-          r -= (int)sh.hist[digit];
+      if (t < 32) {
+        // the digit holding the rank-th candidate: lane l scans digits
+        // 8l .. 8l+7 after an exclusive prefix of the lanes' totals
+        const int lane = t;
+        unsigned cnt[8], tot = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) { cnt[e] = sh.hist[8 * lane + e]; tot += cnt[e]; }
+        unsigned incl = tot;
+#pragma unroll
+        for (int m = 1; m < 32; m <<= 1) {
+          const unsigned y = __shfl_up_sync(0xffffffffu, incl, m);
+          if (lane >= m) incl += y;
         }
-        sh.prefix = pre | ((unsigned long long)digit << shift);
-        sh.rank = r;
+        const int r = sh.rank;
+        const unsigned before = incl - tot;
+        if ((int)before < r && r <= (int)incl) {
+          int rr = r - (int)before;
+          unsigned digit = 8 * lane;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            if (rr <= (int)cnt[e]) { digit = 8 * lane + e; break; }
+            rr -= (int)cnt[e];
+          }
+          sh.prefix = pre | ((unsigned long long)digit << shift);
+          sh.rank = rr;
+        }
       }
       __syncthreads();
     }
@@ -181,9 +212,9 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const AllocArgs
     // every candidate below tau is taken; among those equal to tau, the
     // first (need - #below) in row order
     long long below = 0, myeq = 0;
-    int eq[kMaxRowsPerThread];
+    int eq[RPT];
 #pragma unroll
-    for (int q = 0; q < kMaxRowsPerThread; ++q) {
+    for (int q = 0; q < RPT; ++q) {
       eq[q] = 0;
       if (q < rpt && r0 + q < N) {
         const int lo = dec ? a.b_min + 1 : bv[q], hi = dec ? bv[q] : a.b_max - 1;
@@ -200,7 +231,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const AllocArgs
     long long eqbefore = block_exclusive_scan(myeq, sh, &eqtot);
     long long rem = need - nbelow;                // taken among the ties
 #pragma unroll
-    for (int q = 0; q < kMaxRowsPerThread; ++q) {
+    for (int q = 0; q < RPT; ++q) {
       if (q < rpt && r0 + q < N) {
         const int lo = dec ? a.b_min + 1 : bv[q], hi = dec ? bv[q] : a.b_max - 1;
         long long take = 0;
@@ -217,7 +248,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const AllocArgs
   // ---- widths and prefix offsets
   long long mybits = 0;
 #pragma unroll
-  for (int q = 0; q < kMaxRowsPerThread; ++q)
+  for (int q = 0; q < RPT; ++q)
     if (q < rpt && r0 + q < N) {
       a.bits[(size_t)g * N + r0 + q] = (uint8_t)bv[q];
       mybits += bv[q];
@@ -227,7 +258,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const AllocArgs
   if (a.offsets) {
     uint32_t* of = a.offsets + (size_t)g * (N + 1);
 #pragma unroll
-    for (int q = 0; q < kMaxRowsPerThread; ++q)
+    for (int q = 0; q < RPT; ++q)
       if (q < rpt && r0 + q < N) {
         of[r0 + q] = (uint32_t)(off * a.offset_unit);
         off += bv[q];
@@ -237,7 +268,10 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const AllocArgs
 }
 
 cudaError_t launch_allocate(const AllocArgs& a, cudaStream_t st) {
-  allocate_kernel<<<a.groups, kAllocThreads, 0, st>>>(a);
+  if (a.rows_per_group <= kAllocThreads * 8)
+    allocate_kernel<8><<<a.groups, kAllocThreads, 0, st>>>(a);
+  else
+    allocate_kernel<kMaxRowsPerThread><<<a.groups, kAllocThreads, 0, st>>>(a);
   return cudaGetLastError();
 }
 
