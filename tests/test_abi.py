@@ -40,7 +40,7 @@ def _param_counts():
     src = open(os.path.join(ROOT, "include", "brs.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     out = {}
-    for m in re.finditer(r"\b(brs_[a-z_]+)\s*\(([^)]*)\)\s*;", src):
+    for m in re.finditer(r"\b(brs_[a-z0-9_]+)\s*\(([^)]*)\)\s*;", src):
         args = m.group(2).strip()
         out[m.group(1)] = 0 if args in ("", "void") else args.count(",") + 1
     return out
@@ -55,3 +55,35 @@ def test_binding_argument_counts_match_header():
         fn = getattr(lib, name)
         assert fn.argtypes is not None, name
         assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
+
+
+def test_deferred_decode_host_checks():
+    """Deferred write-back: the interval state's size, and the argument
+    errors that return before any device work."""
+    from bit_recurrent_state_b200 import brs, synth
+    w = synth.WORKLOADS["kda_decode"]
+    L = brs.layout_of(w)
+    assert brs.decode_state32_bytes(L) == 64 * 32 * 128 * 128 * 4
+    with pytest.raises(brs.BrsError) as e:
+        brs.decode_state32_bytes(brs.layout_of(synth.WORKLOADS["varbit_decode"]))
+    assert e.value.status == brs.EUNSUPPORTED
+    p = 1 << 20                      # an aligned address that is never dereferenced on these paths
+    args = dict(packed=p, aux=None, workspace=p, perm=None, q=p, k=p, v=p, beta=p, decay=p, o=p)
+
+    def call(wb, step, state32):
+        brs.decode_step_deferred(L, wb, step, args["packed"], args["aux"], args["workspace"], state32, args["perm"],
+                                 args["q"], args["k"], args["v"], args["beta"], args["decay"], args["o"], stream=0)
+
+    with pytest.raises(brs.BrsError) as e:              # C > 1 needs the interval state
+        call(brs.writeback_of(w, C=4), 1, None)
+    assert e.value.status == brs.EINVAL
+    with pytest.raises(brs.BrsError) as e:              # C >= 1
+        call(brs.writeback_of(w, C=0), 0, p)
+    assert e.value.status == brs.EINVAL
+    with pytest.raises(brs.BrsError) as e:              # 16-byte alignment
+        call(brs.writeback_of(w, C=4), 1, p + 4)
+    assert e.value.status == brs.EALIGN
+    with pytest.raises(brs.BrsError) as e:              # DAMP storage only
+        brs.decode_step_deferred(brs.layout_of(synth.WORKLOADS["gdn_decode_fp32"]), brs.writeback_of(w, C=4), 1,
+                                 p, None, p, p, None, p, p, p, p, p, p, stream=0)
+    assert e.value.status == brs.EUNSUPPORTED
