@@ -240,6 +240,12 @@ def _oracle_cfg(w):
                     domain=O.DOMAIN_MIXED if w.storage == "damp" else O.DOMAIN_CANONICAL)
 
 
+def is_prefill(w) -> bool:
+    """Workloads whose step is one chunked-prefill launch (decode workloads
+    may still write back every C > 1 tokens)."""
+    return w.name == "kda_prefill"
+
+
 def workload_config(w, world: int) -> dict:
     """The `config` object of both arms: the workload by name and sizes."""
     cfg = {"workload": w.name if w.mode == "nearest" else f"{w.name}_{w.mode}",
@@ -323,7 +329,8 @@ def run_reference(args, w):
     if rank != 0:
         return
     R = OracleRunner(w)
-    total = w.B * w.H * (w.T if w.C > 1 else 1)      # token*heads of one step of our arm
+    prefill = is_prefill(w)
+    total = w.B * w.H * (w.T if prefill else 1)      # token*heads of one step of our arm
     per_step_s = max(0.005, min(4.0, args.ref_budget / (args.warmup + args.steps)))
     units = int(max(1, min(R.units_total, R.rate() * per_step_s / (R.heads_per_unit * w.C))))
     vals, used = [], 1
@@ -333,7 +340,7 @@ def run_reference(args, w):
             vals.append(th / dt)
     value = statistics.median(vals)
     what = "sequences" if R.varbit else "heads"
-    metric = METRIC.replace("decode", "chunked prefill") if w.C > 1 else METRIC
+    metric = METRIC.replace("decode", "chunked prefill") if prefill else METRIC
     line = {"impl": "reference", "metric": metric, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total / value, "higher_is_better": True,
@@ -673,13 +680,13 @@ def main():
     if args.steps is None:
         # long enough a timed region for the clock sampler (>= ~0.5 s on
         # the GPU); the oracle arm times a few bounded samples
-        args.steps = 10 if args.impl == "reference" else (40 if w.C > 1 else 20000)
+        args.steps = 10 if args.impl == "reference" else (40 if is_prefill(w) else 20000)
     if args.impl == "reference":
         run_reference(args, w)
     else:
         from bit_recurrent_state_b200 import brs
         brs.lib()          # the in-tree CUDA library; fails loudly when it is missing
-        if w.name == "kda_prefill":
+        if is_prefill(w):
             run_prefill(args, w)
         else:
             run_ours(args, w)
