@@ -48,6 +48,7 @@ brs_status check_layout(const brs_layout* L) {
   } else if (L->storage == BRS_STORE_VARBIT) {
     if (L->hadamard) return fail(BRS_EUNSUPPORTED, "variable-width storage is stored without the Hadamard");
     if (L->b_min < 1 || L->b_max > 16 || L->b_min > L->b_max) return fail(BRS_EINVAL, "need 1 <= b_min <= b_max <= 16");
+    if (L->persistence < 0 || L->persistence > 2) return fail(BRS_EINVAL, "persistence must be 0, 1 or 2");
     const double tot = L->avg_bits * (double)L->H * (double)L->d;
     if (tot != std::floor(tot)) return fail(BRS_EINVAL, "avg_bits * H * d must be an integer");
     if (L->avg_bits < L->b_min || L->avg_bits > L->b_max) return fail(BRS_EINVAL, "avg_bits outside [b_min, b_max]");
@@ -189,7 +190,7 @@ brs_status brs_decode_step(const brs_layout* L, const brs_writeback* wb, int64_t
     brs::VbArgs a{};
     a.B = L->B; a.H = L->H; a.Hk = L->H_k; a.decay_per_key = L->decay_per_key; a.mode = wb->mode;
     a.first = step == 0; a.C = wb->C; a.b_min = L->b_min; a.b_max = L->b_max;
-    a.budget_scope = L->budget_scope; a.seed = wb->seed; a.step = step;
+    a.budget_scope = L->budget_scope; a.persistence = L->persistence; a.seed = wb->seed; a.step = step;
     double lam = 1.0;
     for (int c = 0; c < wb->C; ++c) lam *= (1.0 - 2.0 / 65.0);   // EMA weight of a C-token chunk, span 64
     a.lambda = lam; a.avg_bits = L->avg_bits;

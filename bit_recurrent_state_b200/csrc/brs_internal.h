@@ -87,7 +87,7 @@ cudaError_t launch_varbit_pack(const VbPackArgs& a, cudaStream_t st);
 cudaError_t launch_varbit_unpack(const VbPackArgs& a, const void* packed, float* S, cudaStream_t st);
 
 struct VbArgs {
-  int B, H, Hk, decay_per_key, mode, first, C, b_min, b_max, budget_scope;
+  int B, H, Hk, decay_per_key, mode, first, C, b_min, b_max, budget_scope, persistence;
   uint64_t seed;
   int64_t step;
   double lambda, avg_bits;

@@ -415,10 +415,17 @@ __global__ void __launch_bounds__(32 * kVbWarps) varbit_kernel(const VbArgs a) {
       st[0] = A;
       st[1] = K;
       const double s_hat = -0.5 * log(A);
-      const double rr = 0.5 * K;
-      double arg = 2.0 * (s_hat + rr);
-      if (!(arg >= 1e-9)) arg = 1e-9;
-      const double gam = 1.0 / ((double)a.C * expm1(arg));
+      double gam;
+      if (a.persistence == 0) {                    // erasure rate Gamma_hat
+        const double rr = 0.5 * K;
+        double arg = 2.0 * (s_hat + rr);
+        if (!(arg >= 1e-9)) arg = 1e-9;
+        gam = 1.0 / ((double)a.C * expm1(arg));
+      } else {                                     // w^(1) = 1/(1 - e^-2s), h^(C) = 1/(1 - e^-2Cs)
+        double arg = 2.0 * s_hat * (double)(a.persistence == 2 ? a.C : 1);
+        if (!(arg >= 1e-9)) arg = 1e-9;
+        gam = 1.0 / -expm1(-arg);
+      }
       const double rt = rms > 0.0 ? (double)sm.R[i] / rms : 0.0;
       a.cost[(size_t)b * rows + h * D + i] = gam * (rt * rt);
     }

@@ -130,9 +130,13 @@ typedef struct {
   int32_t hadamard;      /* DAMP: 1 = INT8 rows stored after the Hadamard     */
   int32_t decay_per_key; /* 1 = KDA (decay [B][H][d]), 0 = GDN ([B][H])        */
   double avg_bits;       /* VARBIT: mean width; avg_bits*H*d integral          */
-  int32_t b_min, b_max;  /* VARBIT: width limits, 2 <= b_min <= b_max <= 8     */
+  int32_t b_min, b_max;  /* VARBIT: width limits, 1 <= b_min <= b_max <= 16    */
   int32_t budget_scope;  /* VARBIT: 1 = layer (all H*d rows of a sequence),
                             0 = head                                           */
+  int32_t persistence;   /* VARBIT: row weight of the allocation cost ([LB]
+                            Choice of persistence factor): 0 = the erasure
+                            rate Gamma_hat, 1 = DAMP's uncapped w^(1) =
+                            1/(1 - e^-2s), 2 = h^(C) = 1/(1 - e^-2Cs)           */
 } brs_layout;
 
 typedef struct {

@@ -377,6 +377,19 @@ double orc_gamma_hat(double A, double K, int C) {
   return 1.0 / ((double)C * expm1(arg));
 }
 
+/* The row weight of the allocation cost c = weight * R~^2 ([LB] Choice of
+ * persistence factor): 0 the erasure rate Gamma_hat above; 1 DAMP's
+ * uncapped persistence w^(1) = 1 / (1 - e^(-2 s)); 2 the write-back-time
+ * factor h^(C) = 1 / (1 - e^(-2 C s)); s = -ln(A)/2, the exponent's
+ * argument floored at 1e-9 as for Gamma_hat. */
+double orc_persistence(int kind, double A, double K, int C) {
+  if (kind == 0) return orc_gamma_hat(A, K, C);
+  double s = -0.5 * log(A);
+  double arg = 2.0 * s * (double)(kind == 2 ? C : 1);
+  if (!(arg >= 1e-9)) arg = 1e-9;
+  return 1.0 / -expm1(-arg);
+}
+
 /* b*_i = avg + log2(c_i / GM(c)) / 2 (the minimiser of sum c_i 2^(-2 b_i)
  * at a fixed mean), GM over the rows with c_i > 0; rounded to nearest
  * (ties to even), clipped to [b_min, b_max]; rows with c_i = 0 take b_min
@@ -889,7 +902,7 @@ static int run_seq_unit(const orc_layout* L, const orc_writeback* wb, int64_t st
         for (int i = 0; i < d; ++i) {
           int r = h * d + i;
           double rt = rms > 0.0 ? Rr[r] / rms : 0.0;
-          cost[r] = orc_gamma_hat(st[2 * r + 0], st[2 * r + 1], C) * (rt * rt);
+          cost[r] = orc_persistence(L->persistence, st[2 * r + 0], st[2 * r + 1], C) * (rt * rt);
         }
       }
       if (L->budget_scope == 1) {

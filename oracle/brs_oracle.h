@@ -44,7 +44,11 @@ typedef struct {
   int b_min, b_max;     /* VARBIT width limits                                */
   int budget_scope;     /* VARBIT: 1 layer (all H*d rows of a sequence), 0 head */
   int domain;           /* ORC_DOMAIN_*: where the FP32 update is computed    */
+  int persistence;      /* VARBIT cost weight: 0 erasure rate Gamma_hat, 1 w^(1), 2 h^(C) */
 } orc_layout;
+
+/* persistence weight of a row from A = EMA(a^2), K = EMA(beta (2-beta) k^2) */
+double orc_persistence(int kind, double A, double K, int C);
 
 typedef struct {
   int mode;             /* ORC_ROUND_*                                        */

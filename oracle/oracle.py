@@ -51,7 +51,7 @@ class Layout(ct.Structure):
         ("storage", ct.c_int), ("k_hi", ct.c_int), ("block", ct.c_int),
         ("hadamard", ct.c_int), ("decay_per_key", ct.c_int),
         ("avg_bits", ct.c_double), ("b_min", ct.c_int), ("b_max", ct.c_int),
-        ("budget_scope", ct.c_int), ("domain", ct.c_int),
+        ("budget_scope", ct.c_int), ("domain", ct.c_int), ("persistence", ct.c_int),
     ]
 
 
@@ -81,6 +81,8 @@ def lib():
             L.orc_int8_block.restype = ct.c_int
             L.orc_int8_block.argtypes = [P, ct.c_int, ct.c_int, ct.c_uint64, ct.c_int64, ct.c_int,
                                          ct.c_int, ct.c_int, P, P, P, P, P]
+            L.orc_persistence.restype = ct.c_double
+            L.orc_persistence.argtypes = [ct.c_int, ct.c_double, ct.c_double, ct.c_int]
             L.orc_varbit_row.restype = ct.c_int
             L.orc_varbit_row.argtypes = [P, ct.c_int, ct.c_int, ct.c_int, ct.c_uint64, ct.c_int64,
                                          ct.c_int, ct.c_int, ct.c_int, P, P, P, P, P]
@@ -131,11 +133,12 @@ class Config:
     b_max: int = 8
     budget_scope: int = 1
     domain: int = DOMAIN_CANONICAL
+    persistence: int = 0
 
     def layout(self) -> Layout:
         return Layout(self.B, self.H, self.Hk or self.H, self.d, self.storage, self.k_hi,
                       self.block, self.hadamard, self.decay_per_key, self.avg_bits, self.b_min,
-                      self.b_max, self.budget_scope, self.domain)
+                      self.b_max, self.budget_scope, self.domain, self.persistence)
 
 
 # ---------------------------------------------------------------- scalars
@@ -326,3 +329,8 @@ def calibrate(cfg: Config, inputs: dict, every: int = 8, tau: float = 1e-3):
                              _p(_c(inputs["decay"], np.float32)), _p(score), _p(perm))
     assert fl == OK, fl
     return perm, score
+
+
+def persistence(kind: int, A: float, K: float, C: int) -> float:
+    """The allocation cost's row weight (orc_persistence)."""
+    return float(lib().orc_persistence(int(kind), float(A), float(K), int(C)))

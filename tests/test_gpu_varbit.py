@@ -57,19 +57,20 @@ def _compare_step(w, cfg, pg, po, og, oo, tag, seqs=None):
     return flips
 
 
-@pytest.mark.parametrize("mode,scope,b_min,b_max,avg", [
-    ("nearest", 1, 2, 8, 4.0), ("stochastic", 1, 2, 8, 4.0), ("errfeedback", 1, 2, 8, 4.0),
-    ("nearest", 0, 2, 8, 4.0), ("nearest", 1, 2, 16, 6.0), ("errfeedback", 1, 2, 16, 6.0),
-    ("stochastic", 0, 2, 16, 6.0), ("nearest", 1, 1, 8, 2.0), ("stochastic", 1, 1, 8, 2.0),
-    ("errfeedback", 1, 1, 8, 2.0), ("nearest", 0, 1, 16, 3.0)])
-def test_varbit_teacher_forced(mode, scope, b_min, b_max, avg):
+@pytest.mark.parametrize("mode,scope,b_min,b_max,avg,pers", [
+    ("nearest", 1, 2, 8, 4.0, 0), ("stochastic", 1, 2, 8, 4.0, 0), ("errfeedback", 1, 2, 8, 4.0, 0),
+    ("nearest", 0, 2, 8, 4.0, 0), ("nearest", 1, 2, 16, 6.0, 0), ("errfeedback", 1, 2, 16, 6.0, 0),
+    ("stochastic", 0, 2, 16, 6.0, 0), ("nearest", 1, 1, 8, 2.0, 0), ("stochastic", 1, 1, 8, 2.0, 0),
+    ("errfeedback", 1, 1, 8, 2.0, 0), ("nearest", 0, 1, 16, 3.0, 0), ("nearest", 1, 2, 8, 4.0, 1),
+    ("stochastic", 0, 2, 8, 4.0, 2)])
+def test_varbit_teacher_forced(mode, scope, b_min, b_max, avg, pers):
     """b_max = 16 as at C = 1: widths up to 16 bits, a lane's four codes
     spanning up to three words of the row payload; b_min = 1: one-bit rows
     (the sign times the row's mean absolute value)."""
     import torch
     from bit_recurrent_state_b200 import brs
     from oracle import oracle as O
-    w = _vb_workload(mode=mode, b_min=b_min, b_max=b_max, avg_bits=avg)
+    w = _vb_workload(mode=mode, b_min=b_min, b_max=b_max, avg_bits=avg, persistence=pers)
     cfg = oracle_cfg(w)
     cfg.budget_scope = scope
     packed_o, aux_o, stats_o = O.new_state(cfg)

@@ -15,17 +15,18 @@ def _levels(codes, bw):
     return 2 * codes - 1 if bw == 1 else codes - (2 ** (bw - 1) - 1)
 
 
-@pytest.mark.parametrize("mode,b_min,b_max,avg", [(0, 2, 8, 4.0), (1, 2, 8, 4.0), (2, 2, 8, 4.0),
-                                                  (0, 2, 16, 4.0), (2, 2, 16, 4.0),
-                                                  (0, 1, 8, 2.0), (1, 1, 8, 2.0), (2, 1, 8, 2.0)])
-def test_varbit_teacher_forced_fp64(orc, mode, b_min, b_max, avg):
+@pytest.mark.parametrize("mode,b_min,b_max,avg,pers", [(0, 2, 8, 4.0, 0), (1, 2, 8, 4.0, 0), (2, 2, 8, 4.0, 0),
+                                                       (0, 2, 16, 4.0, 0), (2, 2, 16, 4.0, 0),
+                                                       (0, 1, 8, 2.0, 0), (1, 1, 8, 2.0, 0), (2, 1, 8, 2.0, 0),
+                                                       (0, 2, 8, 4.0, 1), (0, 2, 8, 4.0, 2)])
+def test_varbit_teacher_forced_fp64(orc, mode, b_min, b_max, avg, pers):
     """b_max = 8, and 16 as at C = 1 (widths up to 16 bits, codes that span
     words of the row payload); b_min = 1 with one-bit rows (the sign times
     the row's mean absolute value)."""
     B, H, d, T = 2, 2, 32, 6
     w = synth.Workload("t", B=B, H=H, d=d, T=T, storage="varbit", hadamard=0, seed=20 + mode)
     cfg = orc.Config(B=B, H=H, d=d, storage=orc.STORE_VARBIT, hadamard=0, avg_bits=avg,
-                     b_min=b_min, b_max=b_max, budget_scope=1)
+                     b_min=b_min, b_max=b_max, budget_scope=1, persistence=pers)
     inp_all = synth.run_inputs(w, 0, T)
     packed, aux, stats = orc.new_state(cfg)
     lam = (1 - 2 / 65)
@@ -61,8 +62,11 @@ def test_varbit_teacher_forced_fp64(orc, mode, b_min, b_max, avg):
             # widths from an FP64 recomputation of c = Gamma_hat * R~^2
             a2 = np.concatenate([inp["decay"][0, b, h].astype(np.float64) ** 2 for h in range(H)])
             s_hat = -0.5 * np.log(a2)
-            arg = np.maximum(2 * (s_hat + 0.5 * K64[b]), 1e-9)
-            gam = 1.0 / np.expm1(arg)
+            if pers == 0:
+                arg = np.maximum(2 * (s_hat + 0.5 * K64[b]), 1e-9)
+                gam = 1.0 / np.expm1(arg)
+            else:                                       # w^(1), and h^(C) at C = 1
+                gam = 1.0 / (1.0 - a2)
             rms = np.sqrt(np.mean(Rr.reshape(H, d) ** 2, axis=1))
             Rt = (Rr.reshape(H, d) / rms[:, None]).ravel()
             c = gam * Rt ** 2
@@ -130,3 +134,15 @@ def test_varbit_pack_rejects_widths_off_budget(orc):
     w[0] = 8
     _, fl = orc.state_pack(cfg, S, None, w)
     assert fl == orc.EINVAL
+
+
+def test_persistence_weights_closed_forms(orc):
+    """w^(1) = 1/(1 - A) and h^(C) = 1/(1 - A^C) for A = EMA(a^2) = e^(-2s),
+    computed by the oracle through logarithms; the erasure rate with r = 0 is
+    1/(C expm1(2s)) = 1/(C (1/A - 1))."""
+    for A in (0.5, 0.81, 0.999):
+        assert orc.persistence(1, A, 0.3, 7) == pytest.approx(1.0 / (1.0 - A), rel=1e-12)
+        assert orc.persistence(2, A, 0.3, 4) == pytest.approx(1.0 / (1.0 - A ** 4), rel=1e-12)
+        assert orc.persistence(2, A, 0.3, 1) == pytest.approx(orc.persistence(1, A, 0.0, 1), rel=1e-15)
+        assert orc.persistence(0, A, 0.0, 4) == pytest.approx(1.0 / (4 * (1.0 / A - 1.0)), rel=1e-12)
+    assert orc.persistence(1, 1.0, 0.0, 1) == pytest.approx(1e9, rel=1e-6)      # no decay: floored argument
