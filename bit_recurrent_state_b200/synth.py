@@ -50,7 +50,7 @@ class Workload:
     b_max: int = 8
     C: int = 1
     persistence: int = 0              # variable-width cost weight (0 Gamma_hat, 1 w^(1), 2 h^(C))
-    mode: str = "nearest"          # "nearest" | "stochastic" | "errfeedback"
+    mode: str = "nearest"          # "nearest" | "stochastic" | "errfeedback" | "direction"
     seed: int = 0
 
     @property

@@ -227,6 +227,40 @@ int orc_int8_block(const float* y, int n, int mode, uint64_t seed, int64_t step,
   return flags;
 }
 
+/* Direction memory on the INT8 block ([WB] Post-training write-back
+ * interventions and diagnostics: signed sub-threshold votes, a trigger that
+ * moves the stored state by one level and resets the counter, transitions
+ * clipped at the grid rails; Trajectory analysis: the voting region
+ * Delta/8 < |delta| < Delta/2; the Chinese summary's core method: a k-bit sign
+ * counter with threshold T_k = 2^(k-1)).  Counter of k = 2 bits: m in
+ * {-1, 0, 1}, T = 2.  The grid and the codes are those of nearest write-back
+ * of y; then per element the proposed change delta = y - xprev (xprev: the
+ * stored value the step started from, in the stored basis) votes sign(delta)
+ * when Delta/8 < |delta| < Delta/2 (Delta: the block's new step); a counter
+ * that reaches +-2 moves the code one level that way (clipped to [0, 255])
+ * and returns to 0. */
+int orc_int8_block_dm(const float* y, const float* xprev, int n, int8_t* m_inout, uint8_t* codes,
+                      uint16_t* scale_h, uint16_t* zero_h, float* t_out) {
+  int flags = orc_int8_block(y, n, ORC_ROUND_NEAREST, 0, 0, 0, 0, 0, NULL, codes, scale_h, zero_h, t_out);
+  float s = orc_f32_from_f16(*scale_h);
+  float lo = s * 0.125f, hi = s * 0.5f;
+  for (int j = 0; j < n; ++j) {
+    float dl = y[j] - xprev[j];
+    float ad = fabsf(dl);
+    int m = m_inout[j];
+    if (ad > lo && ad < hi) m += (dl > 0.0f) ? 1 : -1;
+    if (m >= 2 || m <= -2) {
+      int c = (int)codes[j] + (m > 0 ? 1 : -1);
+      if (c < 0) c = 0;
+      if (c > 255) c = 255;
+      codes[j] = (uint8_t)c;
+      m = 0;
+    }
+    m_inout[j] = (int8_t)m;
+  }
+  return flags;
+}
+
 /* Variable-width symmetric row ([LB] Levels and storage): levels
  * {-n..n}*Delta, n = 2^(b-1) - 1, Delta = f*R/n with R the row's absolute
  * maximum and f fitted over 16 values in [1/4, 1] (read as f_m = (5+m)/20)
@@ -575,12 +609,30 @@ static void damp_load(const orc_layout* L, const uint8_t* head, float* S) {
   }
 }
 
+/* 2-bit two's-complement direction counters, four to a byte in column
+ * order (element e of a head at bits 2(e mod 4) of byte e/4) */
+static int dm_get(const uint8_t* dm, size_t e) {
+  int f = (dm[e >> 2] >> (2 * (e & 3))) & 3;
+  return (f & 2) ? f - 4 : f;
+}
+static void dm_put(uint8_t* dm, size_t e, int m) {
+  int sh = 2 * (int)(e & 3);
+  dm[e >> 2] = (uint8_t)((dm[e >> 2] & ~(3 << sh)) | ((m & 3) << sh));
+}
+
+/* prev: the stored head this write-back replaces (read block by block just
+ * before it is overwritten, so it may be the same memory as head); used by
+ * direction memory only, whose counters sit in aux_head as bytes. */
 static int damp_store(const orc_layout* L, const orc_writeback* wb, int64_t step, int b, int h,
-                      const float* S, uint8_t* head, uint16_t* aux_head, float* t_head) {
+                      const float* S, const uint8_t* prev, uint8_t* head, uint16_t* aux_head,
+                      float* t_head) {
   int d = L->d, nlo = d - L->k_hi, nb = d / L->block, flags = 0;
   uint8_t* codes = head;
   uint16_t* f16rows = (uint16_t*)(head + (size_t)nlo * d);
   uint16_t* sz = (uint16_t*)(head + (size_t)nlo * d + (size_t)L->k_hi * d * 2);
+  const uint16_t* psz = (const uint16_t*)(prev + (size_t)nlo * d + (size_t)L->k_hi * d * 2);
+  float* xp = (float*)malloc(sizeof(float) * (size_t)L->block);
+  int8_t* mm = (int8_t*)malloc((size_t)L->block);
   float* tmp = (float*)malloc(sizeof(float) * (size_t)d);
   for (int i = 0; i < d; ++i) {
     memcpy(tmp, S + (size_t)i * d, sizeof(float) * (size_t)d);
@@ -597,6 +649,20 @@ static int damp_store(const orc_layout* L, const orc_writeback* wb, int64_t step
       if (L->hadamard && !rotated(L) && !mixed(L)) orc_fwht(tmp, d);
       for (int bl = 0; bl < nb; ++bl) {
         int j0 = bl * L->block;
+        if (wb->mode == ORC_ROUND_DIRECTION) {
+          uint8_t* dmh = (uint8_t*)aux_head;
+          float ps = orc_f32_from_f16(psz[((size_t)i * nb + bl) * 2 + 0]);
+          float pz = orc_f32_from_f16(psz[((size_t)i * nb + bl) * 2 + 1]);
+          for (int j = 0; j < L->block; ++j) {
+            xp[j] = fmaf((float)prev[(size_t)i * d + j0 + j], ps, pz);
+            mm[j] = (int8_t)dm_get(dmh, (size_t)i * d + j0 + j);
+          }
+          flags |= orc_int8_block_dm(tmp + j0, xp, L->block, mm, codes + (size_t)i * d + j0,
+                                     &sz[((size_t)i * nb + bl) * 2 + 0], &sz[((size_t)i * nb + bl) * 2 + 1],
+                                     t_head ? t_head + (size_t)i * d + j0 : NULL);
+          for (int j = 0; j < L->block; ++j) dm_put(dmh, (size_t)i * d + j0 + j, mm[j]);
+          continue;
+        }
         uint16_t* e = aux_head ? aux_head + (size_t)i * d + j0 : NULL;
         flags |= orc_int8_block(tmp + j0, L->block, wb->mode, wb->seed, step, h, b, i * d + j0, e,
                                 codes + (size_t)i * d + j0, &sz[((size_t)i * nb + bl) * 2 + 0],
@@ -606,6 +672,8 @@ static int damp_store(const orc_layout* L, const orc_writeback* wb, int64_t step
     }
   }
   free(tmp);
+  free(xp);
+  free(mm);
   return flags;
 }
 
@@ -745,9 +813,13 @@ static int run_head_unit(const orc_layout* L, const orc_writeback* wb, int64_t s
           if (!isfinite(S[e])) flags |= ORC_ENONFINITE;
         memcpy(pout + unit * hb, S, hb);
       } else {
-        uint16_t* aux_head = aux ? aux + unit * (size_t)(d - L->k_hi) * d : NULL;
+        size_t nel = (size_t)(d - L->k_hi) * d;
+        uint16_t* aux_head = NULL;
+        if (aux) aux_head = (wb->mode == ORC_ROUND_DIRECTION) ? (uint16_t*)((uint8_t*)aux + unit * (nel / 4))
+                                                             : aux + unit * nel;
         float* th = t_dump ? t_dump + unit * (size_t)d * d : NULL;
-        flags |= damp_store(L, wb, step, b, h, S, pout + unit * hb, aux_head, th);
+        const uint8_t* prev = (t == 0) ? pin + unit * hb : pout + unit * hb;
+        flags |= damp_store(L, wb, step, b, h, S, prev, pout + unit * hb, aux_head, th);
         damp_load(L, pout + unit * hb, S);
       }
     }
@@ -953,6 +1025,11 @@ int orc_run(const orc_layout* L, const orc_writeback* wb, int64_t step0, int T, 
             const int16_t* perm, const uint16_t* q, const uint16_t* k, const uint16_t* v,
             const float* beta, const float* decay, float* o, float* t_dump, float* s_dump) {
   if (!layout_ok(L) || wb->C <= 0 || step0 % wb->C || T % wb->C) return ORC_EINVAL;
+  if (wb->mode < ORC_ROUND_NEAREST || wb->mode > ORC_ROUND_DIRECTION) return ORC_EINVAL;
+  /* direction memory: DAMP at a write-back every token (the votes compare
+   * each token's proposal with the value stored after the previous token) */
+  if (wb->mode == ORC_ROUND_DIRECTION && (L->storage != ORC_STORE_DAMP || wb->C != 1 || !aux))
+    return ORC_EINVAL;
   orc_inputs in = {q, k, v, beta, decay, o};
   int flags = 0;
   if (L->storage == ORC_STORE_VARBIT) {
@@ -1013,7 +1090,7 @@ int orc_state_pack(const orc_layout* L, const float* S, const int16_t* perm,
         if (L->storage == ORC_STORE_FP32)
           memcpy(dst, tmp, hb);
         else
-          flags |= damp_store(&Lc, &wb, 0, b, h, tmp, dst, NULL, NULL);
+          flags |= damp_store(&Lc, &wb, 0, b, h, tmp, dst, dst, NULL, NULL);
       }
   }
   free(tmp);

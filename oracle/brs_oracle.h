@@ -27,7 +27,7 @@ extern "C" {
 #endif
 
 enum { ORC_STORE_FP32 = 0, ORC_STORE_DAMP = 1, ORC_STORE_VARBIT = 2 };
-enum { ORC_ROUND_NEAREST = 0, ORC_ROUND_STOCHASTIC = 1, ORC_ROUND_ERRFEEDBACK = 2 };
+enum { ORC_ROUND_NEAREST = 0, ORC_ROUND_STOCHASTIC = 1, ORC_ROUND_ERRFEEDBACK = 2, ORC_ROUND_DIRECTION = 3 };
 enum { ORC_DOMAIN_CANONICAL = 0, ORC_DOMAIN_ROTATED = 1, ORC_DOMAIN_MIXED = 2 };
 
 /* status flags (OR-ed) */
@@ -73,6 +73,13 @@ float    orc_hadamard_scale(int n);
 int orc_int8_block(const float* y, int n, int mode, uint64_t seed, int64_t step, int h, int b,
                    int elem0, uint16_t* e_inout, uint8_t* codes, uint16_t* scale_h,
                    uint16_t* zero_h, float* t_out);
+
+/* The INT8 block under direction memory: nearest codes of y on the block's
+ * grid, then 2-bit sign counters m_inout (values -1, 0, 1) take a vote from
+ * each proposed change y - xprev inside (scale/8, scale/2); a counter that
+ * reaches +-2 moves its code one level (clipped to [0, 255]) and is reset. */
+int orc_int8_block_dm(const float* y, const float* xprev, int n, int8_t* m_inout, uint8_t* codes,
+                      uint16_t* scale_h, uint16_t* zero_h, float* t_out);
 
 /* One variable-width row (decay-aware allocation tier), width bw in [2, 8]. */
 int orc_varbit_row(const float* x, int n, int bw, int mode, uint64_t seed, int64_t step, int h,

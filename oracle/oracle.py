@@ -26,7 +26,7 @@ _SRC = os.path.join(_HERE, "brs_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
 STORE_FP32, STORE_DAMP, STORE_VARBIT = 0, 1, 2
-ROUND_NEAREST, ROUND_STOCHASTIC, ROUND_ERRFEEDBACK = 0, 1, 2
+ROUND_NEAREST, ROUND_STOCHASTIC, ROUND_ERRFEEDBACK, ROUND_DIRECTION = 0, 1, 2, 3
 DOMAIN_CANONICAL, DOMAIN_ROTATED, DOMAIN_MIXED = 0, 1, 2
 OK, EINVAL, ENONFINITE, EOVERFLOW = 0, 1, 2, 4
 
@@ -81,6 +81,8 @@ def lib():
             L.orc_int8_block.restype = ct.c_int
             L.orc_int8_block.argtypes = [P, ct.c_int, ct.c_int, ct.c_uint64, ct.c_int64, ct.c_int,
                                          ct.c_int, ct.c_int, P, P, P, P, P]
+            L.orc_int8_block_dm.restype = ct.c_int
+            L.orc_int8_block_dm.argtypes = [P, P, ct.c_int, P, P, P, P, P]
             L.orc_persistence.restype = ct.c_double
             L.orc_persistence.argtypes = [ct.c_int, ct.c_double, ct.c_double, ct.c_int]
             L.orc_varbit_row.restype = ct.c_int
@@ -183,6 +185,21 @@ def int8_block(y, mode=ROUND_NEAREST, seed=0, step=0, h=0, b=0, elem0=0, e=None)
     fl = lib().orc_int8_block(_p(y), n, mode, seed, step, h, b, elem0, _p(e), _p(codes), _p(sh),
                               _p(zh), _p(t))
     return dict(codes=codes, scale=sh[0], zero=zh[0], t=t, e=e, flags=fl)
+
+
+def int8_block_dm(y, xprev, m):
+    """One INT8 block under direction memory; m (int8 counters in -1..1) is
+    returned updated."""
+    y = _c(y, np.float32)
+    xp = _c(xprev, np.float32)
+    n = y.size
+    codes = np.zeros(n, np.uint8)
+    sh = np.zeros(1, np.uint16)
+    zh = np.zeros(1, np.uint16)
+    t = np.zeros(n, np.float32)
+    m = np.array(m, dtype=np.int8)
+    fl = lib().orc_int8_block_dm(_p(y), _p(xp), n, _p(m), _p(codes), _p(sh), _p(zh), _p(t))
+    return dict(codes=codes, scale=sh[0], zero=zh[0], t=t, m=m, flags=fl)
 
 
 def varbit_row(x, bw, mode=ROUND_NEAREST, seed=0, step=0, h=0, b=0, elem0=0, e=None):

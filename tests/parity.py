@@ -6,7 +6,7 @@ from bit_recurrent_state_b200 import synth
 from oracle import oracle as O
 
 MODE = {"nearest": O.ROUND_NEAREST, "stochastic": O.ROUND_STOCHASTIC,
-        "errfeedback": O.ROUND_ERRFEEDBACK}
+        "errfeedback": O.ROUND_ERRFEEDBACK, "direction": O.ROUND_DIRECTION}
 STORE = {"fp32": O.STORE_FP32, "damp": O.STORE_DAMP, "varbit": O.STORE_VARBIT}
 
 

@@ -170,3 +170,113 @@ def test_varbit_fit_matches_exhaustive_scan(orc, bw):
 def test_varbit_zero_row(orc):
     r = orc.varbit_row(np.zeros(128, np.float32), 4)
     assert r["delta"] == 0 and np.all(r["q"] == 0)
+
+
+# ---- direction memory ([WB] Post-training write-back interventions:
+# signed sub-threshold votes, a trigger of one level, a reset counter,
+# rails; Trajectory analysis: the voting region Delta/8 < |delta| < Delta/2;
+# the Chinese summary's core method: threshold T_k = 2^(k-1), here k = 2)
+
+def _dm_loop(orc, deltas, start_level=100):
+    """One interior value drifting by deltas[t] per step on a fixed grid of
+    spacing 0.125 (min and max pinned); returns its code after each step."""
+    D = float(golden("dead_zone.txt")["delta_4"])
+    cur = np.zeros(32, np.float32)
+    cur[1] = 255 * D
+    cur[2] = start_level * D
+    m = np.zeros(32, np.int8)
+    out = []
+    for dl in deltas:
+        tgt = cur.copy()
+        tgt[2] = cur[2] + np.float32(dl)
+        r = orc.int8_block_dm(tgt, cur, m)
+        s = np.float32(np.uint16(r["scale"]).view(np.float16))
+        assert s == np.float32(D)
+        z = np.float32(np.uint16(r["zero"]).view(np.float16))
+        m = r["m"]
+        assert set(np.unique(m)) <= {-1, 0, 1}
+        cur = (r["codes"].astype(np.float32) * s + z).astype(np.float32)
+        out.append(int(r["codes"][2]))
+    return out
+
+
+@pytest.mark.parametrize("frac", [0.2, 0.3, 0.45])
+def test_direction_memory_moves_one_level_per_two_votes(orc, frac):
+    """A constant drift inside the voting region (inside the dead zone, so
+    nearest write-back never moves) moves the stored value by one level at
+    every second step: T_2 = 2 votes, then the counter restarts from 0."""
+    D = float(golden("dead_zone.txt")["delta_4"])
+    codes = _dm_loop(orc, [frac * D] * 12)
+    assert codes == [100 + (t + 1) // 2 for t in range(12)]
+    down = _dm_loop(orc, [-frac * D] * 12)
+    assert down == [100 - (t + 1) // 2 for t in range(12)]
+
+
+def test_direction_memory_ignores_changes_outside_the_region(orc):
+    D = float(golden("dead_zone.txt")["delta_4"])
+    # below Delta/8: no vote, no move
+    assert _dm_loop(orc, [0.1 * D] * 20) == [100] * 20
+    # alternating directions cancel in the signed counter
+    assert _dm_loop(orc, [0.3 * D, -0.3 * D] * 10) == [100] * 20
+    # above Delta/2 the nearest level moves by itself and nothing votes
+    assert _dm_loop(orc, [0.75 * D] * 6) == [101, 102, 103, 104, 105, 106]
+
+
+def test_direction_memory_trigger_is_clipped_at_the_rail(orc):
+    D = float(golden("dead_zone.txt")["delta_4"])
+    y = np.zeros(32, np.float32)
+    y[1] = 255 * D                                   # on the top rail
+    xp = y.copy()
+    xp[1] = y[1] - np.float32(0.3 * D)               # a vote up
+    m = np.zeros(32, np.int8)
+    m[1] = 1                                         # ... that completes the count
+    r = orc.int8_block_dm(y, xp, m)
+    assert r["codes"][1] == 255 and r["m"][1] == 0   # clipped, counter reset
+    assert np.all(r["codes"][2:] == 0) and np.all(r["m"][2:] == 0)
+
+
+def test_direction_memory_recurrence_keeps_a_still_state(orc):
+    """beta = 0, a = 1 through the whole decode recurrence (no Hadamard): the
+    proposals equal the stored values, nothing votes, and the stored state
+    and counters stay as they are.  Reading the stored value the step started
+    from anywhere else would give nonzero proposals of up to half a step."""
+    from bit_recurrent_state_b200 import synth
+    from parity import oracle_cfg, random_perm
+    w = synth.Workload("dm_still", B=2, H=2, d=32, k_hi=4, block=32, hadamard=0, T=6, seed=3, mode="direction")
+    cfg = oracle_cfg(w)
+    S0 = (np.random.default_rng(5).standard_normal((w.B, w.H, w.d, w.d))).astype(np.float32)
+    perm = random_perm(w, seed=2)
+    packed, fl = orc.state_pack(cfg, S0, perm)
+    assert fl == 0
+    _, aux, stats = orc.new_state(cfg)
+    before = packed.copy()
+    inp = synth.run_inputs(w, 0, w.T)
+    inp["beta"][:] = 0.0
+    inp["decay"][:] = 1.0
+    o, fl, _ = orc.run(cfg, orc.ROUND_DIRECTION, w.seed, 1, 0, inp, packed, aux=aux, stats=stats, perm=perm)
+    assert fl == 0
+    np.testing.assert_array_equal(packed, before)
+    assert not np.any(aux)
+
+
+def test_direction_memory_recurrence_counters_are_two_bit_fields(orc):
+    """A decode run under direction memory: every stored counter field is
+    one of -1, 0, 1 (the value -2 is never stored), some counters are
+    nonzero, and the run only departs from nearest write-back after votes."""
+    from bit_recurrent_state_b200 import synth
+    from parity import oracle_cfg
+    w = synth.Workload("dm_run", B=1, H=2, d=32, k_hi=4, block=32, T=12, seed=4, mode="direction")
+    cfg = oracle_cfg(w)
+    inp = synth.run_inputs(w, 0, w.T)
+    pd, aux, stats = orc.new_state(cfg)
+    o_d, fl, _ = orc.run(cfg, orc.ROUND_DIRECTION, w.seed, 1, 0, inp, pd, aux=aux, stats=stats)
+    assert fl == 0
+    fields = np.unpackbits(aux.view(np.uint8)[: w.B * w.H * (w.d - w.k_hi) * w.d // 4][:, None],
+                           axis=1, bitorder="little").reshape(-1, 4, 2)
+    vals = fields[..., 0] + 2 * fields[..., 1]
+    assert not np.any(vals == 2)
+    assert np.any(vals != 0)
+    pn, auxn, statsn = orc.new_state(cfg)
+    o_n, fl, _ = orc.run(cfg, orc.ROUND_NEAREST, w.seed, 1, 0, inp, pn, aux=auxn, stats=statsn)
+    # the first token starts from the zero state on both sides: identical
+    np.testing.assert_array_equal(o_d[0], o_n[0])
