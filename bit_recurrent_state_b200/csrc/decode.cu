@@ -171,6 +171,8 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
   const uint8_t* f16in = hin + (size_t)nlo * D;
   uint16_t* f16out = (uint16_t*)(hout + (size_t)nlo * D);
   uint16_t* auxb = (MODE == BRS_ROUND_ERRFEEDBACK) ? (uint16_t*)a.aux + (size_t)head * nlo * D : nullptr;
+  // direction memory: 2-bit counters, four to a byte in column order
+  uint8_t* dmb = (MODE == BRS_ROUND_DIRECTION) ? (uint8_t*)a.aux + (size_t)head * nlo * (D / 4) : nullptr;
 
   // ---- inputs: k, a, q gathered through the permutation and the stored
   // grid of every INT8 row, as ready pairs; v of my columns
@@ -359,6 +361,7 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
   for (int i0 = 0; i0 < D; i0 += NRB) {
     const bool int8_batch = (STORE != BRS_STORE_FP32) && (i0 < nlo);   // batches are tier-uniform
     float x[NRB][C];
+    float xp[(MODE == BRS_ROUND_DIRECTION) ? NRB : 1][C];   // stored values the step started from
 #pragma unroll
     for (int r = 0; r < NRB; ++r) {
       const int i = i0 + r;
@@ -370,6 +373,10 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
         } else {
           const float sv = f16_to_f32((uint16_t)(ps[r] & 0xffffu)), zv = f16_to_f32((uint16_t)(ps[r] >> 16));
           dequant_int8<C>(x[r], pw[r], sv, sv, zv, zv);
+        }
+        if constexpr (MODE == BRS_ROUND_DIRECTION) {
+#pragma unroll
+          for (int c = 0; c < C; ++c) xp[r][c] = x[r][c];
         }
       } else {
         load_row(i, x[r]);
@@ -577,6 +584,35 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
           if constexpr (C >= 2) fma2(mq[c], mq[c + 1], tq[c], tq[c + 1], a.one, a.one, kRoundMagic, kRoundMagic);
           else mq[c] = __fadd_rn(tq[c], kRoundMagic);
         }
+        if constexpr (MODE == BRS_ROUND_DIRECTION) {
+          // votes of the proposed changes y - xp inside (scale/8, scale/2);
+          // a counter at +-2 moves the nearest code one level (clipped to
+          // [0, 255]) and is reset.  The lanes of one counter byte merge
+          // their fields before one of them stores it.
+          uint8_t* dmp = dmb + (size_t)i * (D / 4) + col0 / 4;
+          const uint32_t old = *dmp;
+          const int sh0 = 2 * (col0 & 3);
+          const float lo = __fmul_rn(p.s, 0.125f), hi = __fmul_rn(p.s, 0.5f);
+          uint32_t nb = 0;
+#pragma unroll
+          for (int c = 0; c < C; ++c) {
+            const int f = (int)((old >> (sh0 + 2 * c)) & 3u);
+            int m = (f & 2) ? f - 4 : f;
+            const float dl = __fsub_rn(x[r][c], xp[r][c]);
+            const float ad = fabsf(dl);
+            if (ad > lo && ad < hi) m += (dl > 0.0f) ? 1 : -1;
+            if (m >= 2 || m <= -2) {
+              const uint32_t mb = __float_as_uint(mq[c]);
+              const int code = min(max((int)(mb & 0xffu) + (m > 0 ? 1 : -1), 0), 255);
+              mq[c] = __uint_as_float((mb & ~0xffu) | (uint32_t)code);
+              m = 0;
+            }
+            nb |= ((uint32_t)m & 3u) << (sh0 + 2 * c);
+          }
+          if constexpr (C <= 2) nb |= __shfl_xor_sync(0xffffffffu, nb, 1);
+          if constexpr (C == 1) nb |= __shfl_xor_sync(0xffffffffu, nb, 2);
+          if ((col0 & 3) == 0) *dmp = (uint8_t)nb;
+        }
         uint8_t* dst = hout + (size_t)i * D + col0;
         if constexpr (C == 4) {
           *(uint32_t*)dst = __byte_perm(__byte_perm(__float_as_uint(mq[0]), __float_as_uint(mq[1]), 0x0040u),
@@ -641,6 +677,7 @@ static cudaError_t launch_db(const DecodeArgs& a, int store, bool had, cudaStrea
     case BRS_ROUND_NEAREST: return launch_dbm<D, BLOCK, BRS_ROUND_NEAREST>(a, store, had, st);
     case BRS_ROUND_STOCHASTIC: return launch_dbm<D, BLOCK, BRS_ROUND_STOCHASTIC>(a, store, had, st);
     case BRS_ROUND_ERRFEEDBACK: return launch_dbm<D, BLOCK, BRS_ROUND_ERRFEEDBACK>(a, store, had, st);
+    case BRS_ROUND_DIRECTION: return launch_dbm<D, BLOCK, BRS_ROUND_DIRECTION>(a, store, had, st);
   }
   return cudaErrorInvalidValue;
 }
@@ -672,7 +709,8 @@ cudaError_t launch_decode(const DecodeArgs& a, int d, int store, bool had, cudaS
     }
     return cudaErrorInvalidValue;
   }
-  if (decode_tma_supported(d, store, a.block, a.k_hi)) return launch_decode_tma(a, had, st);
+  if (a.mode != BRS_ROUND_DIRECTION && decode_tma_supported(d, store, a.block, a.k_hi))
+    return launch_decode_tma(a, had, st);
   if (d == 128 && a.block == 128) return launch_db<128, 128>(a, store, had, st);
   if (d == 128 && a.block == 32) return launch_db<128, 32>(a, store, had, st);
   if (d == 64 && a.block == 64) return launch_db<64, 64>(a, store, had, st);

@@ -111,7 +111,17 @@ typedef enum { BRS_STORE_FP32 = 0, BRS_STORE_DAMP = 1, BRS_STORE_VARBIT = 2 } br
 typedef enum {
   BRS_ROUND_NEAREST = 0,
   BRS_ROUND_STOCHASTIC = 1,
-  BRS_ROUND_ERRFEEDBACK = 2
+  BRS_ROUND_ERRFEEDBACK = 2,
+  /* Direction memory ([WB] Post-training write-back interventions; the
+     voting region of its Trajectory analysis): nearest write-back plus a
+     2-bit sign counter per INT8 element.  A proposed change y - x_prev (x_prev:
+     the stored value the token started from) with scale/8 < |y - x_prev| <
+     scale/2 votes its sign; a counter reaching +-2 moves the code one level
+     that way (clipped to [0, 255]) and is reset.  DAMP decode with C = 1
+     only.  The counters live in the first B*H*(d-k_hi)*d/4 bytes of the
+     residual buffer (four to a byte, column order, two's complement), which
+     starts zeroed. */
+  BRS_ROUND_DIRECTION = 3
 } brs_round;
 
 /* Device flag bits OR-ed into the first 32-bit word of `workspace`. */
@@ -175,7 +185,8 @@ brs_status brs_state_unpack(const brs_layout* L, const void* packed, const int16
  * before reuse).  Decode supports C == 1.
  *   packed_in / packed_out: stored state before / after; they may alias
  *     for FP32 and DAMP storage, must not alias for VARBIT.
- *   aux: residuals (ERRFEEDBACK only, else may be NULL), updated in place.
+ *   aux: residuals (ERRFEEDBACK) or direction counters (DIRECTION, DAMP
+ *     only), updated in place; else may be NULL.
  *   stats: VARBIT statistics, updated in place (else may be NULL).
  *   workspace: brs_state_bytes(...workspace) bytes; its first word
  *     collects device flags and must be zeroed once before first use
@@ -199,7 +210,8 @@ brs_status brs_decode_step(const brs_layout* L, const brs_writeback* wb, int64_t
  *     step % C != 0 (else the stored state is read), written when
  *     (step + 1) % C != 0.  May be NULL when C == 1.
  *   packed: stored state, updated in place at write-backs.  aux: residuals
- *     (error feedback), used and updated at write-backs only.
+ *     (error feedback), used and updated at write-backs only; direction
+ *     memory needs C == 1.
  *   workspace: flag word (as brs_decode_step).
  * Calls must cover consecutive steps, starting at a multiple of C, for the
  * result to equal the recurrence with write-back every C tokens (the state
@@ -224,7 +236,8 @@ brs_status brs_decode_step_deferred(const brs_layout* L, const brs_writeback* wb
  * write-back rounding of `wb` at the chunk's last token.  DAMP storage,
  * d = 128, C = 64, block 128 or 32.
  *   packed: stored state, updated in place.  aux: residuals (error
- *     feedback).  workspace: flag word (as brs_decode_step).
+ *     feedback; direction memory is not built for the prefill).
+ *     workspace: flag word (as brs_decode_step).
  *   q, k [B][T][H_k][d] bf16; v [B][T][H][d] bf16; beta [B][T][H] f32;
  *     decay [B][T][H][d] (KDA) or [B][T][H] (GDN) f32; o [B][T][H][d] f32.
  *   state_dump (optional): [B][H][d][d] f32, the state just before the last

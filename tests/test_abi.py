@@ -87,3 +87,29 @@ def test_deferred_decode_host_checks():
         brs.decode_step_deferred(brs.layout_of(synth.WORKLOADS["gdn_decode_fp32"]), brs.writeback_of(w, C=4), 1,
                                  p, None, p, p, None, p, p, p, p, p, p, stream=0)
     assert e.value.status == brs.EUNSUPPORTED
+
+
+def test_direction_memory_host_checks():
+    """Direction memory: the argument errors that return before any device
+    work (C = 1 only, DAMP only, the counter buffer required, no prefill)."""
+    import dataclasses
+    from bit_recurrent_state_b200 import brs, synth
+    w = dataclasses.replace(synth.WORKLOADS["kda_decode"], mode="direction")
+    L = brs.layout_of(w)
+    p = 1 << 20                      # an aligned address that is never dereferenced on these paths
+    with pytest.raises(brs.BrsError) as e:              # write-back every token only
+        brs.decode_step_deferred(L, brs.writeback_of(w, C=4), 1, p, p, p, p, None, p, p, p, p, p, p, stream=0)
+    assert e.value.status == brs.EUNSUPPORTED
+    with pytest.raises(brs.BrsError) as e:              # the counters are required
+        brs.decode_step(L, brs.writeback_of(w), 0, p, p, None, None, p, None, p, p, p, p, p, p, stream=0)
+    assert e.value.status == brs.EINVAL
+    wv = dataclasses.replace(synth.WORKLOADS["varbit_decode"], mode="direction")
+    with pytest.raises(brs.BrsError) as e:              # DAMP storage only
+        brs.decode_step(brs.layout_of(wv), brs.writeback_of(wv), 0, p, p + 16, p, p, p, None, p, p, p, p, p, p,
+                        stream=0)
+    assert e.value.status == brs.EUNSUPPORTED
+    wp = dataclasses.replace(synth.WORKLOADS["kda_prefill"], mode="direction")
+    with pytest.raises(brs.BrsError) as e:              # not built for the prefill
+        brs.chunk_prefill(brs.layout_of(wp), brs.writeback_of(wp), 0, 64, p, p, p, None, p, p, p, p, p, p,
+                          stream=0)
+    assert e.value.status == brs.EUNSUPPORTED

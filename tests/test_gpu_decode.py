@@ -59,6 +59,9 @@ def _compare(w, steps, units=None):
         if w.mode == "errfeedback":
             per = ag.size // (w.B * w.H)
             np.testing.assert_array_equal(ag.reshape(w.B * w.H, per)[sel], ao.reshape(w.B * w.H, per)[sel])
+        if w.mode == "direction":
+            # 2-bit counters of every head, then the unused rest of the buffer
+            np.testing.assert_array_equal(ag, ao, err_msg=f"direction counters after step {t}")
 
 
 def test_kda_tiny_full_trajectory():
@@ -84,6 +87,11 @@ def test_kda_tiny_full_trajectory():
     ("kda128_sr", dict(B=2, H=3, d=128, k_hi=16, block=128, mode="stochastic")),
     ("kda128_ef", dict(B=2, H=3, d=128, k_hi=16, block=128, mode="errfeedback")),
     ("kda32_ef", dict(B=1, H=2, d=32, k_hi=4, block=32, mode="errfeedback")),
+    ("kda128_dm", dict(B=2, H=3, d=128, k_hi=16, block=128, mode="direction")),
+    ("kda128_b32_dm", dict(B=2, H=2, d=128, k_hi=16, block=32, mode="direction")),
+    ("kda64_dm", dict(B=2, H=3, d=64, k_hi=8, block=64, mode="direction")),
+    ("kda32_nohad_dm", dict(B=2, H=2, d=32, k_hi=4, block=32, hadamard=0, mode="direction")),
+    ("gdn128_dm", dict(B=3, H=4, Hk=2, d=128, k_hi=0, block=128, decay_per_key=0, mode="direction")),
     ("fp32_64", dict(B=2, H=3, d=64, storage="fp32")),
     ("fp32_gdn128", dict(B=2, H=4, Hk=2, d=128, storage="fp32", decay_per_key=0)),
 ])
