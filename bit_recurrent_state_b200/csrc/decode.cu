@@ -263,15 +263,41 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
       v_fma_s<C>(u1, ka.x, ka.y, x);
     }
   } else if (src32) {
-    // FP32 rows from the interval state: the same chains, INT8 tier then FP16 tier
-#pragma unroll 8
-    for (int i = 0; i < D; ++i) {
-      float x[C];
-      load_row(i, x);
-      const float4 ka = sm.rs[i].ka;
-      v_scale<C>(x, ka.z, ka.w);
-      if (i < nlo) v_fma_s<C>(u1, ka.x, ka.y, x);
-      else v_fma_s<C>(u2, ka.x, ka.y, x);
+    // FP32 rows from the interval state: the same chains, INT8 tier then
+    // FP16 tier, in batches of NRB rows with the next batch's loads in flight
+    float xb[2][NRB][C];
+    const float* rb = s32h + col0;
+    auto fetch32 = [&](int buf, int i0) {
+#pragma unroll
+      for (int r = 0; r < NRB; ++r) {
+        const float* src = rb + (size_t)(i0 + r) * D;
+        if constexpr (C == 4) {
+          const float4 f = __ldg((const float4*)src);
+          xb[buf][r][0] = f.x; xb[buf][r][1] = f.y; xb[buf][r][2] = f.z; xb[buf][r][3] = f.w;
+        } else if constexpr (C == 2) {
+          const float2 f = __ldg((const float2*)src);
+          xb[buf][r][0] = f.x; xb[buf][r][1] = f.y;
+        } else {
+          xb[buf][r][0] = __ldg(src);
+        }
+      }
+    };
+    auto consume32 = [&](int buf, int i0) {
+#pragma unroll
+      for (int r = 0; r < NRB; ++r) {
+        const float4 ka = sm.rs[i0 + r].ka;
+        v_scale<C>(xb[buf][r], ka.z, ka.w);
+        if (i0 + r < nlo) v_fma_s<C>(u1, ka.x, ka.y, xb[buf][r]);
+        else v_fma_s<C>(u2, ka.x, ka.y, xb[buf][r]);
+      }
+    };
+    static_assert(D % (2 * NRB) == 0, "pairs of batches");
+    fetch32(0, 0);
+    for (int i0 = 0; i0 < D; i0 += 2 * NRB) {
+      fetch32(1, i0 + NRB);
+      consume32(0, i0);
+      if (i0 + 2 * NRB < D) fetch32(0, i0 + 2 * NRB);
+      consume32(1, i0 + NRB);
     }
   } else {
     // chunks of CH = NRB rows (nlo is a multiple of NRB), two in flight
@@ -362,14 +388,14 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
     const bool int8_batch = (STORE != BRS_STORE_FP32) && (i0 < nlo);   // batches are tier-uniform
     float x[NRB][C];
     float xp[(MODE == BRS_ROUND_DIRECTION) ? NRB : 1][C];   // stored values the step started from
+    // the batch's rows: dequantized from the prefetched codes, or loaded
+    // (all NRB loads issued before the first use)
+    if (int8_batch && !src32) {
 #pragma unroll
-    for (int r = 0; r < NRB; ++r) {
-      const int i = i0 + r;
-      const RowScal rsc = sm.rs[i];
-      const float2 qv = sm.qq[i];
-      if (int8_batch && !src32) {
+      for (int r = 0; r < NRB; ++r) {
         if constexpr (NB == 1) {
-          dequant_int8<C>(x[r], pw[r], rsc.sz.x, rsc.sz.y, rsc.sz.z, rsc.sz.w);
+          const float4 g = sm.rs[i0 + r].sz;
+          dequant_int8<C>(x[r], pw[r], g.x, g.y, g.z, g.w);
         } else {
           const float sv = f16_to_f32((uint16_t)(ps[r] & 0xffffu)), zv = f16_to_f32((uint16_t)(ps[r] >> 16));
           dequant_int8<C>(x[r], pw[r], sv, sv, zv, zv);
@@ -378,9 +404,16 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
 #pragma unroll
           for (int c = 0; c < C; ++c) xp[r][c] = x[r][c];
         }
-      } else {
-        load_row(i, x[r]);
       }
+    } else {
+#pragma unroll
+      for (int r = 0; r < NRB; ++r) load_row(i0 + r, x[r]);
+    }
+#pragma unroll
+    for (int r = 0; r < NRB; ++r) {
+      const int i = i0 + r;
+      const RowScal rsc = sm.rs[i];
+      const float2 qv = sm.qq[i];
       v_scale<C>(x[r], rsc.ka.z, rsc.ka.w);
       if (STORE == BRS_STORE_FP32 || i0 < nlo) {
         v_fma_vec<C>(x[r], rsc.ka.x, rsc.ka.y, wt);
