@@ -59,7 +59,7 @@ def _compare(w, steps, units=None):
         if w.mode == "errfeedback":
             per = ag.size // (w.B * w.H)
             np.testing.assert_array_equal(ag.reshape(w.B * w.H, per)[sel], ao.reshape(w.B * w.H, per)[sel])
-        if w.mode == "direction":
+        if w.mode == "direction" and units is None:
             # 2-bit counters of every head, then the unused rest of the buffer
             np.testing.assert_array_equal(ag, ao, err_msg=f"direction counters after step {t}")
 
@@ -111,6 +111,22 @@ def test_kda_decode_full_size_sampled():
     units = (1000, 1064)
     steps = _run_both(w, 48, perm=perm, units=units)
     _compare(w, steps, units=units)
+
+
+def test_kda_decode_direction_memory_full_size_sampled():
+    """Direction-memory write-back at the KDA decode size (B=64, H=32,
+    d=128; the general kernel) for 16 tokens from a nonzero state; the
+    oracle runs 64 of the 2048 heads, whose codes, grids and 2-bit counters
+    must match."""
+    import dataclasses
+    w = dataclasses.replace(synth.WORKLOADS["kda_decode"], mode="direction")
+    perm = random_perm(w, seed=6)
+    units = (500, 564)
+    steps = _run_both(w, 16, perm=perm, units=units, init_scale=0.05)
+    _compare(w, steps, units=units)
+    nel = (w.d - w.k_hi) * w.d // 4
+    for *_, ag, ao in steps:
+        np.testing.assert_array_equal(ag[units[0] * nel: units[1] * nel], ao[units[0] * nel: units[1] * nel])
 
 
 def test_gdn_decode_full_size_sampled():
