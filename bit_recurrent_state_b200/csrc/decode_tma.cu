@@ -35,7 +35,7 @@ namespace {
 constexpr int kD = 128, kC = 4, kNrb = 8;
 constexpr int kTmaWarps = 1;                       // heads per CTA (one: finest spread over the SMs)
 constexpr int kSlot = 2048;                        // bytes per ring stage
-constexpr int kStages = 3;
+constexpr int kStages = 3;                         // ring stages while every head is resident at once
 constexpr int kRows8 = kSlot / kD;                 // INT8 rows per slot
 constexpr int kRows16 = kSlot / (2 * kD);          // FP16 rows per slot
 constexpr unsigned long long kWaitNs = 200000000ull;   // bound on one slot wait (200 ms)
@@ -44,12 +44,13 @@ struct __align__(16) Scal {
   float4 ka, sz;                                   // (k, k, a, a), (s, s, z, z)
 };
 
+template <int NST>
 struct __align__(128) TmaSmem {
-  uint8_t ring[kStages][kSlot];
+  uint8_t ring[NST][kSlot];
   Scal rs[kD];
   float2 qq[kD];
   float4 prm[kNrb][4];                             // (zero, 1/scale, scale, -) per (batch row, block)
-  unsigned long long bar[kStages];
+  unsigned long long bar[NST];
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -190,16 +191,16 @@ __device__ __forceinline__ void fwht128(float (&x)[4], int lane, float scale) {
   for (int i = 0; i < 4; ++i) x[i] = __fmul_rn(x[i], scale);
 }
 
-template <bool HAD, int BLOCK, int MODE>
+template <bool HAD, int BLOCK, int MODE, int NST>
 __global__ void __launch_bounds__(32 * kTmaWarps, 16) decode_tma_kernel(const DecodeArgs a) {
   constexpr int NB = kD / BLOCK;                   // blocks per row: 1 (whole row) or 4
   static_assert(NB == 1 || NB == 4, "blocks of 128 or 32 columns");
-  __shared__ TmaSmem smem_all[kTmaWarps];
+  __shared__ TmaSmem<NST> smem_all[kTmaWarps];
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int head = blockIdx.x * kTmaWarps + warp;
   if (head >= a.B * a.H) return;                   // whole warp leaves together
-  TmaSmem& sm = smem_all[warp];
+  TmaSmem<NST>& sm = smem_all[warp];
   const int b = head / a.H, h = head - b * a.H;
   const int kh = h * a.Hk / a.H;
   const int nlo = kD - a.k_hi;                     // INT8 rows 0 .. nlo-1, FP16 rows after
@@ -233,19 +234,19 @@ __global__ void __launch_bounds__(32 * kTmaWarps, 16) decode_tma_kernel(const De
       }
       if (lane == 0) bulk_load(bar0 + 8u * pst, ring0 + (uint32_t)(pst * kSlot), src, bytes);
       ++pj;
-      pst = (pst + 1 == kStages) ? 0 : pst + 1;
+      pst = (pst + 1 == NST) ? 0 : pst + 1;
       ps = (ps + 1 == nslot) ? 0 : ps + 1;
     }
   };
   if (lane == 0) {
 #pragma unroll
-    for (int st = 0; st < kStages; ++st)
+    for (int st = 0; st < NST; ++st)
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar0 + 8u * st));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncwarp();
 #pragma unroll
-  for (int st = 0; st < kStages; ++st) issue_next();
+  for (int st = 0; st < NST; ++st) issue_next();
 
   // ---- inputs (while the first slots are in flight): k, a, q through the
   // permutation and the grid of every INT8 row, as ready pairs; v, beta
@@ -293,14 +294,14 @@ __global__ void __launch_bounds__(32 * kTmaWarps, 16) decode_tma_kernel(const De
   auto release = [&]() {                           // every lane is done with the stage
     __syncwarp();
     ++cj;
-    cst = (cst + 1 == kStages) ? 0 : cst + 1;
+    cst = (cst + 1 == NST) ? 0 : cst + 1;
     cph ^= (cst == 0) ? 1u : 0u;
     issue_next();
   };
   // after a timeout: the loads still in flight are waited for (bounded)
   // before the warp leaves, then the flag is raised
   auto abandon = [&]() {
-    for (int jj = cj; jj < pj; ++jj) mbar_wait(bar0 + 8u * (jj % kStages), (uint32_t)((jj / kStages) & 1));
+    for (int jj = cj; jj < pj; ++jj) mbar_wait(bar0 + 8u * (jj % NST), (uint32_t)((jj / NST) & 1));
     raise_flag(a.flags, BRS_FLAG_TIMEOUT);
   };
   uint32_t err = 0;                                // flag bits, raised once at the end
@@ -565,8 +566,22 @@ template <int BLOCK, int MODE>
 cudaError_t launch_bm(const DecodeArgs& a, bool had, cudaStream_t st) {
   const int heads = a.B * a.H;
   const dim3 grid((heads + kTmaWarps - 1) / kTmaWarps), block(32 * kTmaWarps);
-  if (had) decode_tma_kernel<true, BLOCK, MODE><<<grid, block, 0, st>>>(a);
-  else decode_tma_kernel<false, BLOCK, MODE><<<grid, block, 0, st>>>(a);
+  // more heads than one wave of 16 per SM: two ring stages, whose smaller
+  // shared-memory footprint lets more warps share an SM
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      sms = 148;
+  }
+  const bool many = heads > 16 * sms;
+  if (had) {
+    if (many) decode_tma_kernel<true, BLOCK, MODE, 2><<<grid, block, 0, st>>>(a);
+    else decode_tma_kernel<true, BLOCK, MODE, kStages><<<grid, block, 0, st>>>(a);
+  } else {
+    if (many) decode_tma_kernel<false, BLOCK, MODE, 2><<<grid, block, 0, st>>>(a);
+    else decode_tma_kernel<false, BLOCK, MODE, kStages><<<grid, block, 0, st>>>(a);
+  }
   return cudaGetLastError();
 }
 
