@@ -25,6 +25,15 @@
 // stored order and T the Hadamard (or the identity).  Paired f32x2
 // instructions are two independent IEEE operations: pairing changes no
 // result.
+//
+// Write-back modes: nearest, stochastic (Philox4x32-10), error feedback
+// (FP16 residual), and direction memory ("When Quantization Breaks Memory",
+// Post-training write-back interventions and diagnostics; Trajectory
+// analysis): nearest codes plus a 2-bit sign counter per INT8 element that
+// takes a vote from every proposed change inside (scale/8, scale/2) and
+// moves the code one level at +-2.  The kernel also carries the FP32 state
+// between write-backs when the write-back interval is C > 1 (interval-state
+// flags).
 #include <cuda_runtime.h>
 #include <cstdint>
 
