@@ -158,8 +158,9 @@ typedef struct {
 } brs_writeback;
 
 /* Bytes of the stored state for layout L; optionally the bytes of the
- * error-feedback residual buffer, of the allocator statistics and of the
- * workspace a call needs.  Returns 0 for an invalid layout (see
+ * auxiliary buffer (error-feedback residuals; direction-memory counters use
+ * its first quarter), of the allocator statistics and of the workspace a
+ * call needs.  Returns 0 for an invalid layout (see
  * brs_last_error). */
 size_t brs_state_bytes(const brs_layout* L, size_t* aux_bytes, size_t* stats_bytes,
                        size_t* workspace_bytes);
