@@ -56,7 +56,7 @@ KERNEL_SOURCES = {
 def kernel_family(w) -> str:
     if w.storage == "varbit":
         return "varbit"
-    return "tma" if (w.storage == "damp" and w.d == 128 and w.C == 1) else "warp"
+    return "tma" if (w.storage == "damp" and w.d == 128 and w.C == 1 and w.mode != "direction") else "warp"
 
 
 def kernel_hash(family: str = "tma") -> str:
@@ -78,6 +78,9 @@ def algorithmic_bytes(w) -> dict:
               (w.H * w.d * 2 if w.storage != "varbit" else 0))
     out = heads * w.d * 4
     ef = 2 * aux if w.mode == "errfeedback" else 0
+    if w.mode == "direction":
+        # 2-bit counters of the INT8 rows, read and written
+        ef = 2 * (heads * (w.d - w.k_hi) * w.d // 4)
     st = 2 * stats
     state = 2 * n
     if w.C > 1 and w.storage == "damp":
@@ -112,7 +115,7 @@ def kernel_name(w) -> str:
     """The kernel a decode step of workload w launches (the dominant one)."""
     if w.storage == "varbit":
         return "brs::varbit_kernel (update pass + fit pass) and brs::allocate_kernel"
-    if w.storage == "damp" and w.d == 128 and w.C == 1:
+    if kernel_family(w) == "tma":
         return "brs::decode_tma_kernel"
     return "brs::decode_warp_kernel"
 
@@ -277,7 +280,7 @@ class OracleRunner:
         self.units_total = w.B if self.varbit else w.B * w.H
         self.heads_per_unit = w.H if self.varbit else 1
         self.mode = {"nearest": O.ROUND_NEAREST, "stochastic": O.ROUND_STOCHASTIC,
-                     "errfeedback": O.ROUND_ERRFEEDBACK}[w.mode]
+                     "errfeedback": O.ROUND_ERRFEEDBACK, "direction": O.ROUND_DIRECTION}[w.mode]
 
     def inputs(self, ntok):
         key = (self.t, ntok)
@@ -660,7 +663,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="kda_decode")
-    ap.add_argument("--mode", default=None, help="write-back rounding: nearest | stochastic | errfeedback")
+    ap.add_argument("--mode", default=None,
+                    help="write-back rounding: nearest | stochastic | errfeedback | direction")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (small profiling cases)")
     ap.add_argument("--tokens", type=int, default=None, help="override the prefill length (small profiling cases)")

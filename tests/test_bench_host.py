@@ -1,0 +1,37 @@
+"""Host-side pieces of the benchmark that need no GPU: which kernel a
+workload's decode step runs (and so which DRAM record may describe it), the
+algorithmic bytes per launch, and the reference arm (the oracle) under a
+non-default write-back mode."""
+import json
+import os
+import subprocess
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+
+def test_kernel_family_and_bytes():
+    import bench
+    from bit_recurrent_state_b200 import synth
+    w = synth.WORKLOADS["kda_decode"]
+    assert bench.kernel_family(w) == "tma"
+    assert bench.kernel_family(w.with_(mode="direction")) == "warp"      # direction memory: general kernel
+    assert bench.kernel_family(synth.WORKLOADS["kda_decode_c8"]) == "warp"
+    assert bench.kernel_family(synth.WORKLOADS["varbit_decode"]) == "varbit"
+    base = bench.algorithmic_bytes(w)
+    assert base["state"] == 2 * 64 * 32 * 18880                           # stored state read + written
+    dm = bench.algorithmic_bytes(w.with_(mode="direction"))
+    assert dm["aux"] == 2 * 64 * 32 * (112 * 128 // 4)                    # 2-bit counters read + written
+    assert dm["total"] - base["total"] == dm["aux"]
+    # a DRAM record keyed to the TMA kernel does not describe the general kernel
+    assert bench.traffic_record(w.with_(mode="direction")) is None
+
+
+def test_reference_arm_direction_mode():
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+                        "kda_tiny", "--mode", "direction", "--steps", "3", "--warmup", "3", "--ref-budget", "2"],
+                       env=dict(os.environ, CUDA_VISIBLE_DEVICES=""), capture_output=True, text=True, timeout=300)
+    assert p.returncode == 0, p.stderr
+    line = json.loads(p.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0
