@@ -25,6 +25,9 @@ class LayerState:
             self.perm = torch.as_tensor(perm, dtype=torch.int16).contiguous().to(self.device)
 
     def pack(self, S: torch.Tensor, widths=None):
+        """Store S (deterministic rounding).  The auxiliary buffer (error-
+        feedback residuals or direction counters) is left as it is: zero()
+        or aux.zero_() starts those from 0."""
         brs.state_pack(self.layout, S.contiguous(), self.perm, self.packed, self.workspace,
                        widths=widths)
 
