@@ -113,3 +113,53 @@ def test_direction_memory_host_checks():
         brs.chunk_prefill(brs.layout_of(wp), brs.writeback_of(wp), 0, 64, p, p, p, None, p, p, p, p, p, p,
                           stream=0)
     assert e.value.status == brs.EUNSUPPORTED
+
+
+def test_argument_errors_before_device_work():
+    """Argument errors of the decode and prefill entries come back as a
+    status before any device work: unknown rounding modes, the decode's
+    write-back interval, required pointers, 16-byte alignment, the missing
+    residual buffer of error feedback, unsupported DAMP shapes, and the
+    variable-width storage's own rules."""
+    import dataclasses
+    from bit_recurrent_state_b200 import brs, synth
+    p = 1 << 20                      # an aligned address that is never dereferenced on these paths
+    w = synth.WORKLOADS["kda_decode"]
+    L = brs.layout_of(w)
+
+    def dec(wb, *, L=L, pin=p, pout=p, aux=p, stats=None, ws=p, perm=None, q=p):
+        brs.decode_step(L, wb, 0, pin, pout, aux, stats, ws, perm, q, p, p, p, p, p, stream=0)
+
+    def status(fn):
+        with pytest.raises(brs.BrsError) as e:
+            fn()
+        return e.value.status
+
+    for mode in (-1, 4):
+        wb = brs.writeback_of(w, mode=mode)
+        assert status(lambda: dec(wb)) == brs.EINVAL
+        assert status(lambda: brs.decode_step_deferred(L, wb, 0, p, p, p, None, None, p, p, p, p, p, p,
+                                                        stream=0)) == brs.EINVAL
+    assert status(lambda: dec(brs.writeback_of(w, C=2))) == brs.EUNSUPPORTED          # decode writes back every token
+    assert status(lambda: dec(brs.writeback_of(w), q=None)) == brs.EINVAL               # required pointer
+    assert status(lambda: dec(brs.writeback_of(w), q=p + 8)) == brs.EALIGN              # 16-byte alignment
+    assert status(lambda: dec(brs.writeback_of(w, mode=brs.ROUND_ERRFEEDBACK), aux=None)) == brs.EINVAL
+    odd = brs.layout_of(dataclasses.replace(w, block=64))                                # (128, 64) not built
+    assert status(lambda: dec(brs.writeback_of(w), L=odd)) == brs.EUNSUPPORTED
+    # variable-width storage: packed_out distinct, no permutation, statistics required
+    wv = synth.WORKLOADS["varbit_decode"]
+    Lv = brs.layout_of(wv)
+    assert status(lambda: dec(brs.writeback_of(wv), L=Lv, stats=p)) == brs.EINVAL      # packed_in == packed_out
+    assert status(lambda: dec(brs.writeback_of(wv), L=Lv, pout=p + 16, stats=p, perm=p)) == brs.EINVAL
+    assert status(lambda: dec(brs.writeback_of(wv), L=Lv, pout=p + 16, stats=None)) == brs.EINVAL
+    # prefill: T and step0 multiples of C, known modes
+    wp = synth.WORKLOADS["kda_prefill"]
+    Lp = brs.layout_of(wp)
+
+    def pre(wb, T=64, step0=0):
+        brs.chunk_prefill(Lp, wb, step0, T, p, p, p, None, p, p, p, p, p, p, stream=0)
+
+    assert status(lambda: pre(brs.writeback_of(wp), T=100)) == brs.EINVAL
+    assert status(lambda: pre(brs.writeback_of(wp), step0=32)) == brs.EINVAL
+    assert status(lambda: pre(brs.writeback_of(wp, mode=7))) == brs.EINVAL
+    assert status(lambda: pre(brs.writeback_of(wp, C=32))) == brs.EUNSUPPORTED
