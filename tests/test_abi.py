@@ -163,3 +163,29 @@ def test_argument_errors_before_device_work():
     assert status(lambda: pre(brs.writeback_of(wp), step0=32)) == brs.EINVAL
     assert status(lambda: pre(brs.writeback_of(wp, mode=7))) == brs.EINVAL
     assert status(lambda: pre(brs.writeback_of(wp, C=32))) == brs.EUNSUPPORTED
+
+
+def test_allocator_argument_errors():
+    """brs_allocate_bits rejects, before any device work: rows not a
+    multiple of the group, widths outside 1..16 or crossed, a budget that is
+    not an integer number of bits or lies outside [b_min, b_max] per row,
+    missing or misaligned device pointers."""
+    from bit_recurrent_state_b200 import brs
+    lib = brs.lib()
+    p = 1 << 20
+
+    def call(n, g, avg, bmin, bmax, cost=p, bits=p, offs=None):
+        return lib.brs_allocate_bits(n, g, cost, avg, bmin, bmax, 1, bits, offs, None)
+
+    assert call(100, 64, 4.0, 2, 8) == brs.EINVAL            # 100 rows, groups of 64
+    assert call(0, 64, 4.0, 2, 8) == brs.EINVAL
+    assert call(128, 64, 4.0, 0, 8) == brs.EINVAL            # b_min >= 1
+    assert call(128, 64, 4.0, 2, 17) == brs.EINVAL           # b_max <= 16
+    assert call(128, 64, 4.0, 8, 2) == brs.EINVAL            # crossed limits
+    assert call(128, 64, 4.01, 2, 8) == brs.EINVAL           # 64 * 4.01 bits is not an integer
+    assert call(128, 64, 9.0, 2, 8) == brs.EINVAL            # above b_max per row
+    assert call(128, 64, 1.5, 2, 8) == brs.EINVAL            # below b_min per row
+    assert call(128, 64, 4.0, 2, 8, cost=None) == brs.EINVAL
+    assert call(128, 64, 4.0, 2, 8, bits=None) == brs.EINVAL
+    assert call(128, 64, 4.0, 2, 8, cost=p + 8) == brs.EALIGN
+    assert call(128, 64, 4.0, 2, 8, offs=p + 4) == brs.EALIGN
