@@ -189,3 +189,57 @@ def test_allocator_argument_errors():
     assert call(128, 64, 4.0, 2, 8, bits=None) == brs.EINVAL
     assert call(128, 64, 4.0, 2, 8, cost=p + 8) == brs.EALIGN
     assert call(128, 64, 4.0, 2, 8, offs=p + 4) == brs.EALIGN
+
+
+def test_layout_and_conversion_argument_errors():
+    """Layout validation (shared by every entry) and the state conversion
+    and calibration entries' own argument errors."""
+    import dataclasses
+    from bit_recurrent_state_b200 import brs, synth
+    p = 1 << 20
+    w = synth.WORKLOADS["kda_decode"]
+
+    def size_status(**kw):
+        with pytest.raises(brs.BrsError) as e:
+            brs.state_bytes(brs.layout_of(dataclasses.replace(w, **kw)))
+        return e.value.status
+
+    assert size_status(d=96) == brs.EINVAL                 # d in {32, 64, 128}
+    assert size_status(k_hi=6) == brs.EINVAL               # multiple of 4
+    assert size_status(block=48) == brs.EINVAL             # power of two
+    assert size_status(block=256) == brs.EINVAL            # at most d
+    assert size_status(B=0) == brs.EINVAL
+    wv = synth.WORKLOADS["varbit_decode"]
+
+    def vsize_status(**kw):
+        with pytest.raises(brs.BrsError) as e:
+            brs.state_bytes(brs.layout_of(dataclasses.replace(wv, **kw)))
+        return e.value.status
+
+    with pytest.raises(brs.BrsError) as e:                 # stored without the Hadamard (status from pack)
+        brs.state_pack(brs.layout_of(dataclasses.replace(wv, hadamard=1)), p, None, p, p, stream=0)
+    assert e.value.status == brs.EUNSUPPORTED and "Hadamard" in str(e.value)
+    assert vsize_status(b_min=0) == brs.EINVAL
+    assert vsize_status(avg_bits=9.0) == brs.EINVAL        # above b_max
+    assert vsize_status(persistence=3) == brs.EINVAL
+    L = brs.layout_of(w)
+    Lv = brs.layout_of(wv)
+    with pytest.raises(brs.BrsError) as e:                 # S required
+        brs.state_pack(L, None, None, p, p, stream=0)
+    assert e.value.status == brs.EINVAL
+    with pytest.raises(brs.BrsError) as e:                 # variable-width rows stay in key-channel order
+        brs.state_pack(Lv, p, p, p, p, stream=0)
+    assert e.value.status == brs.EINVAL
+    with pytest.raises(brs.BrsError) as e:
+        brs.state_unpack(Lv, p, p, p, stream=0)
+    assert e.value.status == brs.EINVAL
+    with pytest.raises(brs.BrsError) as e:                 # 16-byte alignment
+        brs.state_unpack(Lv, p + 4, None, p, stream=0)
+    assert e.value.status == brs.EALIGN
+    # calibration: DAMP layouts only, 0 < every <= T, tau > 0
+    assert brs.calibrate_workspace_bytes(L, 4, 64, 8) > 0
+    for args, st in [((Lv, 4, 64, 8, 1e-3), brs.EINVAL), ((L, 4, 64, 128, 1e-3), brs.EINVAL),
+                     ((L, 4, 64, 8, 0.0), brs.EINVAL), ((L, 0, 64, 8, 1e-3), brs.EINVAL)]:
+        with pytest.raises(brs.BrsError) as e:
+            brs.calibrate(*args, p, p, p, p, p, p, p, stream=0)
+        assert e.value.status == st, args
