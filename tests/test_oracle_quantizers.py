@@ -200,22 +200,35 @@ def _dm_loop(orc, deltas, start_level=100):
     return out
 
 
+def test_direction_memory_fixture_is_consistent():
+    g = golden("direction_memory.txt")
+    k = int(g["counter_bits"])
+    assert int(g["threshold"]) == 2 ** (k - 1)          # T_k = 2^(k-1)
+    assert int(g["active_states"]) == 2 ** k - 1        # counter values -(T-1) .. T-1
+    assert float(g["vote_lo_frac"]) == 1 / 8 and float(g["vote_hi_frac"]) == 1 / 2
+
+
 @pytest.mark.parametrize("frac", [0.2, 0.3, 0.45])
 def test_direction_memory_moves_one_level_per_two_votes(orc, frac):
     """A constant drift inside the voting region (inside the dead zone, so
     nearest write-back never moves) moves the stored value by one level at
-    every second step: T_2 = 2 votes, then the counter restarts from 0."""
+    every T-th step (T = 2 votes), then the counter restarts from 0."""
+    g = golden("direction_memory.txt")
+    lo, hi, T = float(g["vote_lo_frac"]), float(g["vote_hi_frac"]), int(g["threshold"])
+    assert lo < frac < hi
     D = float(golden("dead_zone.txt")["delta_4"])
     codes = _dm_loop(orc, [frac * D] * 12)
-    assert codes == [100 + (t + 1) // 2 for t in range(12)]
+    assert codes == [100 + (t + 1) // T for t in range(12)]
     down = _dm_loop(orc, [-frac * D] * 12)
-    assert down == [100 - (t + 1) // 2 for t in range(12)]
+    assert down == [100 - (t + 1) // T for t in range(12)]
 
 
 def test_direction_memory_ignores_changes_outside_the_region(orc):
     D = float(golden("dead_zone.txt")["delta_4"])
-    # below Delta/8: no vote, no move
+    g = golden("direction_memory.txt")
+    # below Delta/8 (and at it: the region is open): no vote, no move
     assert _dm_loop(orc, [0.1 * D] * 20) == [100] * 20
+    assert _dm_loop(orc, [float(g["vote_lo_frac"]) * D] * 20) == [100] * 20
     # alternating directions cancel in the signed counter
     assert _dm_loop(orc, [0.3 * D, -0.3 * D] * 10) == [100] * 20
     # above Delta/2 the nearest level moves by itself and nothing votes
