@@ -26,7 +26,7 @@ STORES = {"fp32": STORE_FP32, "damp": STORE_DAMP, "varbit": STORE_VARBIT}
 SYMBOLS = ["brs_state_bytes", "brs_state_pack", "brs_state_unpack", "brs_decode_step",
            "brs_decode_step_noalloc", "brs_chunk_prefill", "brs_allocate_bits", "brs_fetch_errors",
            "brs_last_error", "brs_calibrate_workspace_bytes", "brs_calibrate", "brs_decode_state32_bytes",
-           "brs_decode_step_deferred"]
+           "brs_decode_step_deferred", "brs_prefill_workspace_bytes", "brs_fetch_errors_noalloc"]
 
 
 class BrsError(RuntimeError):
@@ -87,6 +87,8 @@ def lib():
         L.brs_decode_step_deferred.argtypes = [P, P, ct.c_int64] + [P] * 12
         L.brs_decode_step_noalloc.restype = S
         L.brs_decode_step_noalloc.argtypes = [P, P, ct.c_int64] + [P] * 12
+        L.brs_prefill_workspace_bytes.restype = ct.c_size_t
+        L.brs_prefill_workspace_bytes.argtypes = [P]
         L.brs_chunk_prefill.restype = S
         L.brs_chunk_prefill.argtypes = [P, P, ct.c_int64, ct.c_int] + [P] * 12
         L.brs_allocate_bits.restype = S
@@ -98,6 +100,8 @@ def lib():
         L.brs_calibrate.argtypes = [P, ct.c_int, ct.c_int, ct.c_int, ct.c_double] + [P] * 9
         L.brs_fetch_errors.restype = S
         L.brs_fetch_errors.argtypes = [P, P, P]
+        L.brs_fetch_errors_noalloc.restype = S
+        L.brs_fetch_errors_noalloc.argtypes = [P, P]
         L.brs_last_error.restype = ct.c_char_p
         L.brs_last_error.argtypes = []
         _lib = L
@@ -183,6 +187,14 @@ def decode_step_noalloc(layout, wb, step, packed_in, packed_out, aux, stats, per
                                          _stream(stream)))
 
 
+def prefill_workspace_bytes(layout) -> int:
+    """brs_prefill_workspace_bytes: flag word + the FP32 state between chunks."""
+    n = int(lib().brs_prefill_workspace_bytes(ct.byref(layout)))
+    if n == 0:
+        raise BrsError(EUNSUPPORTED, last_error())
+    return n
+
+
 def chunk_prefill(layout, wb, step0, T, packed, aux, workspace, perm, q, k, v, beta, decay, o,
                   state_dump=None, stream=None):
     """brs_chunk_prefill: T tokens per sequence, write-back every wb.C tokens."""
@@ -216,6 +228,16 @@ def fetch_errors(workspace, stream=None) -> int:
     """Raw device flag bits (also raises BrsError if any is set)."""
     fl = ct.c_uint32(0)
     st = lib().brs_fetch_errors(_ptr(workspace), ct.byref(fl), _stream(stream))
+    if st != OK and st not in (ENONFINITE, EOVERFLOW, ETIMEOUT):
+        _check(st)
+    return int(fl.value)
+
+
+def fetch_errors_noalloc(stream=None) -> int:
+    """Raw device flag bits collected by brs_decode_step_noalloc calls on the
+    current device since the last read (also cleared)."""
+    fl = ct.c_uint32(0)
+    st = lib().brs_fetch_errors_noalloc(ct.byref(fl), _stream(stream))
     if st != OK and st not in (ENONFINITE, EOVERFLOW, ETIMEOUT):
         _check(st)
     return int(fl.value)

@@ -306,15 +306,21 @@ brs_status brs_chunk_prefill(const brs_layout* L, const brs_writeback* wb, int64
   a.head_bytes = head_bytes(L); a.hscale = hadamard_scale(L->d);
   a.packed = packed; a.aux = aux; a.perm = perm; a.q = q; a.k = k; a.v = v; a.beta = beta;
   a.decay = decay; a.o = o; a.sdump = state_dump; a.flags = (uint32_t*)workspace;
-  // the FP32 state between chunks: a stream-ordered scratch for this call
-  cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = cudaMallocAsync((void**)&a.s0, brs::prefill_tc_scratch_bytes(L->B, L->H), s);
-  if (e != cudaSuccess) return cuda_fail(e, "prefill scratch");
-  e = brs::launch_prefill_tc(a, L->hadamard != 0, s);
-  cudaError_t e2 = cudaFreeAsync(a.s0, s);
-  if (e == cudaSuccess) e = e2;
+  // the FP32 state between chunks: the caller's workspace after the flag word
+  a.s0 = (float*)((uint8_t*)workspace + 256);
+  cudaError_t e = brs::launch_prefill_tc(a, L->hadamard != 0, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
   return ok();
+}
+
+size_t brs_prefill_workspace_bytes(const brs_layout* L) {
+  if (check_layout(L) != BRS_OK) return 0;
+  if (L->storage != BRS_STORE_DAMP || L->d != 128) {
+    fail(BRS_EUNSUPPORTED, "chunked prefill is built for DAMP storage at d = 128");
+    return 0;
+  }
+  ok();
+  return 256 + brs::prefill_tc_scratch_bytes(L->B, L->H);
 }
 
 brs_status brs_allocate_bits(int n_rows, int rows_per_group, const double* cost, double avg_bits,

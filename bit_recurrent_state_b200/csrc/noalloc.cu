@@ -1,4 +1,4 @@
-// Allocation-free variant of brs_decode_step.
+// Allocation-free variant of brs_decode_step, and the read-out of its flags.
 //
 // Who needs it: callers that must not allocate device memory themselves,
 // for example a host framework whose own allocator owns every byte of the
@@ -12,10 +12,14 @@
 // process exits.  Host code cannot use the array's name as a device address,
 // so the first call on each device looks the address up with
 // cudaGetSymbolAddress (that device current) and caches it; that first call
-// should therefore be made before any stream capture.  All calls share the
-// one array: calls that overlap on the GPU race on it, and each call clears
-// the part it uses (the device flag word) before its kernel runs.  Flags the
-// kernel raises stay in the array and are not reported by this entry.
+// should therefore be made before any stream capture, and the device must
+// not be reset (cudaDeviceReset) while the library stays loaded, since a
+// reset invalidates the cached address.  All calls share the one array:
+// calls that overlap on the GPU race on it.  Its first word collects the
+// device flags of every call (it starts at zero when the library is loaded);
+// brs_fetch_errors_noalloc reads and clears it.  The rest of the scratch (the
+// per-row costs of variable-width decode) is written by each call before it
+// is read, so nothing else needs clearing.
 #include <cuda_runtime.h>
 
 #include <cstdio>
@@ -51,6 +55,13 @@ cudaError_t scratch_address(void** out) {
   return cudaSuccess;
 }
 
+brs_status address_failed(const char* who, cudaError_t e) {
+  char msg[256];
+  snprintf(msg, sizeof(msg), "%s: cudaGetSymbolAddress: %s", who, cudaGetErrorString(e));
+  brs::set_last_error(msg);
+  return BRS_ECUDA;
+}
+
 }  // namespace
 
 extern "C" brs_status brs_decode_step_noalloc(const brs_layout* L, const brs_writeback* wb,
@@ -62,8 +73,8 @@ extern "C" brs_status brs_decode_step_noalloc(const brs_layout* L, const brs_wri
                                               void* stream) {
   size_t ws = 0;
   if (brs_state_bytes(L, nullptr, nullptr, &ws) == 0) return BRS_EINVAL;  // message already set
-  char msg[256];
   if (ws > kScratchBytes) {
+    char msg[256];
     snprintf(msg, sizeof(msg),
              "brs_decode_step_noalloc: the layout needs %zu bytes of scratch, the static array holds %zu",
              ws, kScratchBytes);
@@ -72,17 +83,14 @@ extern "C" brs_status brs_decode_step_noalloc(const brs_layout* L, const brs_wri
   }
   void* scratch = nullptr;
   cudaError_t e = scratch_address(&scratch);
-  if (e != cudaSuccess) {
-    snprintf(msg, sizeof(msg), "brs_decode_step_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
-    brs::set_last_error(msg);
-    return BRS_ECUDA;
-  }
-  e = cudaMemsetAsync(scratch, 0, ws, (cudaStream_t)stream);
-  if (e != cudaSuccess) {
-    snprintf(msg, sizeof(msg), "brs_decode_step_noalloc: clearing the scratch: %s", cudaGetErrorString(e));
-    brs::set_last_error(msg);
-    return BRS_ECUDA;
-  }
+  if (e != cudaSuccess) return address_failed("brs_decode_step_noalloc", e);
   return brs_decode_step(L, wb, step, packed_in, packed_out, aux, stats, scratch, perm, q, k, v,
                          beta, decay, o, stream);
+}
+
+extern "C" brs_status brs_fetch_errors_noalloc(uint32_t* flags_out, void* stream) {
+  void* scratch = nullptr;
+  cudaError_t e = scratch_address(&scratch);
+  if (e != cudaSuccess) return address_failed("brs_fetch_errors_noalloc", e);
+  return brs_fetch_errors(scratch, flags_out, stream);
 }

@@ -20,6 +20,7 @@ class LayerState:
         self.stats = torch.zeros(max(stats, 16), dtype=torch.uint8, device=self.device)
         self.workspace = torch.zeros(ws, dtype=torch.uint8, device=self.device)
         self.state32 = None            # FP32 state between write-backs (deferred write-back)
+        self.prefill_ws = None         # chunked prefill: flag word + FP32 state between chunks
         self.perm = None
         if perm is not None:
             self.perm = torch.as_tensor(perm, dtype=torch.int16).contiguous().to(self.device)
@@ -59,5 +60,16 @@ class LayerState:
             self.packed, out = out, self.packed
         return out
 
+    def prefill(self, wb: brs.WriteBack, step0: int, T: int, q, k, v, beta, decay, o, state_dump=None):
+        """brs_chunk_prefill over T tokens (sequence-major inputs)."""
+        if self.prefill_ws is None:
+            self.prefill_ws = torch.zeros(brs.prefill_workspace_bytes(self.layout), dtype=torch.uint8,
+                                          device=self.device)
+        brs.chunk_prefill(self.layout, wb, step0, T, self.packed, self.aux, self.prefill_ws, self.perm,
+                          q, k, v, beta, decay, o, state_dump=state_dump)
+
     def errors(self) -> int:
-        return brs.fetch_errors(self.workspace)
+        fl = brs.fetch_errors(self.workspace)
+        if self.prefill_ws is not None:
+            fl |= brs.fetch_errors(self.prefill_ws)
+        return fl

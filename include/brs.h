@@ -238,7 +238,10 @@ brs_status brs_decode_step_deferred(const brs_layout* L, const brs_writeback* wb
  * d = 128, C = 64, block 128 or 32.
  *   packed: stored state, updated in place.  aux: residuals (error
  *     feedback; direction memory is not built for the prefill).
- *     workspace: flag word (as brs_decode_step).
+ *   workspace: brs_prefill_workspace_bytes(L) bytes, 16-byte aligned: the
+ *     flag word in its first 256 bytes (as brs_decode_step), then the FP32
+ *     state carried between the chunks of the call, B*H*d*d floats, which
+ *     the call overwrites (its contents between calls do not matter).
  *   q, k [B][T][H_k][d] bf16; v [B][T][H][d] bf16; beta [B][T][H] f32;
  *     decay [B][T][H][d] (KDA) or [B][T][H] (GDN) f32; o [B][T][H][d] f32.
  *   state_dump (optional): [B][H][d][d] f32, the state just before the last
@@ -248,10 +251,12 @@ brs_status brs_decode_step_deferred(const brs_layout* L, const brs_writeback* wb
  * accuracy.  Results agree with the token-by-token recurrence within the
  * rounding of the reordered sums; the stored codes are the documented
  * quantizer applied to state_dump.  A call over several chunks equals
- * consecutive one-chunk calls bit for bit.  The call takes a stream-ordered
- * scratch of B*H*d*d floats for its duration (cudaMallocAsync / cudaFreeAsync
- * on `stream`).  Per-channel decays whose 64-token product underflows FP32
- * are outside the form (the outputs become non-finite: BRS_ENONFINITE). */
+ * consecutive one-chunk calls bit for bit.  The call allocates nothing.
+ * Per-channel decays whose 64-token product underflows FP32 are outside the
+ * form (the outputs become non-finite: BRS_ENONFINITE).
+ * brs_prefill_workspace_bytes: the workspace size for layout L (0 for an
+ * invalid layout or one the prefill does not support; see brs_last_error). */
+size_t brs_prefill_workspace_bytes(const brs_layout* L);
 brs_status brs_chunk_prefill(const brs_layout* L, const brs_writeback* wb, int64_t step0, int T,
                              void* packed, void* aux, void* workspace, const int16_t* perm,
                              const uint16_t* q, const uint16_t* k, const uint16_t* v,
@@ -317,14 +322,23 @@ brs_status brs_calibrate(const brs_layout* L, int Bc, int T, int every, double t
  * loads it until the process exits.  Layouts whose workspace
  * (brs_state_bytes) exceeds 4096 bytes are rejected with BRS_EINVAL.  The
  * first call on a device looks the array's address up (cudaGetSymbolAddress)
- * and should precede any stream capture.  All calls share the array, so
- * calls that overlap on the GPU race; each call clears the flag word before
- * its kernel, and device-raised flags are not reported by this entry. */
+ * and should precede any stream capture; the device must not be reset
+ * (cudaDeviceReset) while the library stays loaded, since that invalidates
+ * the address.  All calls share the array, so calls that overlap on the GPU
+ * race.  The array's first word collects the device flags of every call on
+ * that device (zero when the library is loaded) until
+ * brs_fetch_errors_noalloc reads and clears it; the rest of the layout's
+ * scratch is written by each call before it is read. */
 brs_status brs_decode_step_noalloc(const brs_layout* L, const brs_writeback* wb, int64_t step,
                                    const void* packed_in, void* packed_out, void* aux, void* stats,
                                    const int16_t* perm, const uint16_t* q, const uint16_t* k,
                                    const uint16_t* v, const float* beta, const float* decay,
                                    float* o, void* stream);
+
+/* brs_fetch_errors for the static scratch of brs_decode_step_noalloc on the
+ * current device: reads and clears the flags its calls raised (synchronises
+ * `stream`). */
+brs_status brs_fetch_errors_noalloc(uint32_t* flags_out, void* stream);
 
 /* Reads and clears the device flag word of `workspace` (synchronises
  * `stream`).  Returns BRS_OK, or BRS_ENONFINITE / BRS_EOVERFLOW /

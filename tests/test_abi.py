@@ -36,6 +36,18 @@ def test_host_only_calls_without_gpu():
         brs.state_bytes(brs.layout_of(w, H_k=5))
 
 
+def test_prefill_workspace_size():
+    """The prefill's workspace: the 256-byte flag word, then the FP32 state
+    carried between chunks (B*H*d*d floats); layouts the prefill does not
+    support have none."""
+    from bit_recurrent_state_b200 import brs, synth
+    w = synth.WORKLOADS["kda_prefill"]
+    assert brs.prefill_workspace_bytes(brs.layout_of(w)) == 256 + 8 * 32 * 128 * 128 * 4
+    with pytest.raises(brs.BrsError) as e:
+        brs.prefill_workspace_bytes(brs.layout_of(synth.WORKLOADS["kda_tiny"]))
+    assert e.value.status == brs.EUNSUPPORTED
+
+
 def _param_counts():
     src = open(os.path.join(ROOT, "include", "brs.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)

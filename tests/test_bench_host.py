@@ -35,3 +35,9 @@ def test_reference_arm_direction_mode():
     assert p.returncode == 0, p.stderr
     line = json.loads(p.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["value"] > 0
+    # both arms print the same config object (the GPU arm prints workload_config too)
+    import bench
+    from bit_recurrent_state_b200 import synth
+    w = synth.WORKLOADS["kda_tiny"].with_(mode="direction")
+    assert line["config"] == bench.workload_config(w, 1)
+    assert "l2" in line["config"]

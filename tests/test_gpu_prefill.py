@@ -53,8 +53,7 @@ def _run_chunks(w, nchunks, units=None, mode="nearest"):
         o = torch.zeros((w.B, 64, w.H, w.d), device="cuda")
         dump = torch.zeros((w.B, w.H, w.d, w.d), device="cuda")
         d = {k: _dev(v) for k, v in inp.items()}
-        brs.chunk_prefill(L, wb, t0, 64, st.packed, st.aux, st.workspace, st.perm, d["q"], d["k"], d["v"],
-                          d["beta"], d["decay"], o, dump)
+        st.prefill(wb, t0, 64, d["q"], d["k"], d["v"], d["beta"], d["decay"], o, state_dump=dump)
         assert st.errors() == 0
         og = o.cpu().numpy()
         sg = dump.cpu().numpy()
@@ -130,8 +129,7 @@ def test_prefill_multi_chunk_one_launch(kw, mode):
         for t0, T in spans:
             dc = {k: v[:, t0:t0 + T].contiguous() for k, v in d.items()}
             oc = torch.zeros((w.B, T, w.H, w.d), device="cuda")
-            brs.chunk_prefill(L, wb, t0, T, st.packed, st.aux, st.workspace, st.perm, dc["q"], dc["k"], dc["v"],
-                              dc["beta"], dc["decay"], oc, dump)
+            st.prefill(wb, t0, T, dc["q"], dc["k"], dc["v"], dc["beta"], dc["decay"], oc, state_dump=dump)
             o[:, t0:t0 + T] = oc
         assert st.errors() == 0
         runs.append((o.cpu().numpy(), st.packed.cpu().numpy(), st.aux.cpu().numpy(), dump.cpu().numpy()))
