@@ -152,17 +152,25 @@ def test_damp_step_matches_fp64_brute_force(orc):
     assert mism <= 2
 
 
-@pytest.mark.parametrize("name,dom", [("kda_tiny", 1), ("kda_tiny", 2), ("gdn", 2), ("nohad", 2)])
+@pytest.mark.parametrize("name,dom", [("kda_tiny", 1), ("kda_tiny", 2), ("gdn", 2), ("nohad", 2),
+                                      ("kda128", 2), ("kda128", 1), ("kda128_b32", 2), ("gdn128", 2)])
 def test_reordered_modes_match_canonical(orc, name, dom):
     """The rotated mode (the whole update in the Hadamard basis) and the
     mixed-basis mode (each tier in its stored basis) compute the same update
     as the canonical mode in a different FP32 order.  Teacher-forced from the
     canonical trajectory, one step at a time: outputs agree to FP32 rounding
     and stored codes differ only next to a rounding boundary of the canonical
-    grid coordinate."""
+    grid coordinate.  The d = 128 cases are the measured layouts: 16 FP16 +
+    112 INT8 Hadamard rows in blocks of 128 and of 32 (KDA decode and
+    prefill), and all 128 rows INT8 with grouped key heads and one decay per
+    head (GDN decode)."""
     w = {"kda_tiny": synth.WORKLOADS["kda_tiny"],
          "gdn": synth.Workload("g", B=2, H=4, Hk=2, d=32, T=32, k_hi=0, block=32, decay_per_key=0, seed=12),
-         "nohad": synth.Workload("n", B=1, H=2, d=32, T=32, k_hi=8, block=16, hadamard=0, seed=13)}[name]
+         "nohad": synth.Workload("n", B=1, H=2, d=32, T=32, k_hi=8, block=16, hadamard=0, seed=13),
+         "kda128": synth.Workload("k", B=2, H=3, d=128, T=16, k_hi=16, block=128, seed=14),
+         "kda128_b32": synth.Workload("kb", B=2, H=3, d=128, T=16, k_hi=16, block=32, seed=15),
+         "gdn128": synth.Workload("gg", B=2, H=4, Hk=2, d=128, T=16, k_hi=0, block=128, decay_per_key=0,
+                                  seed=16)}[name]
     rng = np.random.default_rng(9)
     perm = _rand_perm(rng, w.H, w.d)
     inp_all = synth.run_inputs(w, 0, w.T)
