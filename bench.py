@@ -46,7 +46,7 @@ FALLBACK_HBM_GBS = 6650.0
 NLAYERS = 8
 # the sources of each decode kernel (a DRAM record stays valid while they hash the same)
 KERNEL_SOURCES = {
-    "tma": ["bit_recurrent_state_b200/csrc/decode_tma.cu", "bit_recurrent_state_b200/csrc/brs_device.cuh"],
+    "cta": ["bit_recurrent_state_b200/csrc/decode_cta.cu", "bit_recurrent_state_b200/csrc/brs_device.cuh"],
     "warp": ["bit_recurrent_state_b200/csrc/decode.cu", "bit_recurrent_state_b200/csrc/brs_device.cuh"],
     "varbit": ["bit_recurrent_state_b200/csrc/varbit.cu", "bit_recurrent_state_b200/csrc/allocate.cu",
                "bit_recurrent_state_b200/csrc/brs_device.cuh"],
@@ -56,10 +56,12 @@ KERNEL_SOURCES = {
 def kernel_family(w) -> str:
     if w.storage == "varbit":
         return "varbit"
-    return "tma" if (w.storage == "damp" and w.d == 128 and w.C == 1 and w.mode != "direction") else "warp"
+    cta = (w.storage == "damp" and w.d == 128 and w.C == 1 and w.k_hi % 16 == 0 and
+           w.mode in ("nearest", "stochastic", "errfeedback"))
+    return "cta" if cta else "warp"
 
 
-def kernel_hash(family: str = "tma") -> str:
+def kernel_hash(family: str = "cta") -> str:
     h = hashlib.sha256()
     for p in KERNEL_SOURCES[family]:
         with open(os.path.join(ROOT, p), "rb") as f:
@@ -115,8 +117,8 @@ def kernel_name(w) -> str:
     """The kernel a decode step of workload w launches (the dominant one)."""
     if w.storage == "varbit":
         return "brs::varbit_kernel (update pass + fit pass) and brs::allocate_kernel"
-    if kernel_family(w) == "tma":
-        return "brs::decode_tma_kernel"
+    if kernel_family(w) == "cta":
+        return "brs::decode_cta_kernel"
     return "brs::decode_warp_kernel"
 
 

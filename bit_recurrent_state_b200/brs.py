@@ -26,7 +26,8 @@ STORES = {"fp32": STORE_FP32, "damp": STORE_DAMP, "varbit": STORE_VARBIT}
 SYMBOLS = ["brs_state_bytes", "brs_state_pack", "brs_state_unpack", "brs_decode_step",
            "brs_decode_step_noalloc", "brs_chunk_prefill", "brs_allocate_bits", "brs_fetch_errors",
            "brs_last_error", "brs_calibrate_workspace_bytes", "brs_calibrate", "brs_decode_state32_bytes",
-           "brs_decode_step_deferred", "brs_prefill_workspace_bytes", "brs_fetch_errors_noalloc"]
+           "brs_decode_step_deferred", "brs_prefill_workspace_bytes", "brs_fetch_errors_noalloc",
+           "brs_test_starve_copies"]
 
 
 class BrsError(RuntimeError):
@@ -102,6 +103,8 @@ def lib():
         L.brs_fetch_errors.argtypes = [P, P, P]
         L.brs_fetch_errors_noalloc.restype = S
         L.brs_fetch_errors_noalloc.argtypes = [P, P]
+        L.brs_test_starve_copies.restype = None
+        L.brs_test_starve_copies.argtypes = [ct.c_int]
         L.brs_last_error.restype = ct.c_char_p
         L.brs_last_error.argtypes = []
         _lib = L
@@ -241,3 +244,9 @@ def fetch_errors_noalloc(stream=None) -> int:
     if st != OK and st not in (ENONFINITE, EOVERFLOW, ETIMEOUT):
         _check(st)
     return int(fl.value)
+
+
+def test_starve_copies(on: bool):
+    """brs_test_starve_copies: make the decode kernel's bounded copy waits run
+    out (test hook)."""
+    lib().brs_test_starve_copies(1 if on else 0)

@@ -13,6 +13,7 @@
 namespace {
 
 thread_local char g_err[512] = "";
+thread_local uint32_t g_starve_tx = 0;   // test hook: brs_test_starve_copies
 
 brs_status fail(brs_status st, const char* fmt, ...) {
   va_list ap;
@@ -76,11 +77,14 @@ brs_status cuda_fail(cudaError_t e, const char* what) {
 namespace brs {
 // lets other translation units of the library report through brs_last_error
 void set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+uint32_t starve_tx_bytes() { return g_starve_tx; }
 }  // namespace brs
 
 extern "C" {
 
 const char* brs_last_error(void) { return g_err; }
+
+void brs_test_starve_copies(int on) { g_starve_tx = on ? 16u : 0u; }
 
 size_t brs_state_bytes(const brs_layout* L, size_t* aux_bytes, size_t* stats_bytes,
                        size_t* workspace_bytes) {
@@ -223,6 +227,7 @@ brs_status brs_decode_step(const brs_layout* L, const brs_writeback* wb, int64_t
   a.packed_in = packed_in; a.packed_out = packed_out; a.aux = aux; a.perm = perm;
   a.q = q; a.k = k; a.v = v; a.beta = beta; a.decay = decay; a.o = o;
   a.flags = (uint32_t*)workspace;
+  a.tx_extra = brs::starve_tx_bytes();
   const bool had = L->storage == BRS_STORE_DAMP && L->hadamard;
   cudaError_t e = brs::launch_decode(a, L->d, L->storage, had, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");

@@ -85,6 +85,70 @@ __device__ __forceinline__ float f2hi(f2_t a) { return __uint_as_float((uint32_t
 __device__ __forceinline__ f2_t f2make(float lo, float hi) { return pk(lo, hi); }
 __device__ __forceinline__ f2_t f2dup(float x) { return pk(x, x); }
 
+// The library's order of every sum over key rows (per tier): groups of 8
+// consecutive rows, each an fmaf chain in row order from +0, whose sums are
+// added in a pairwise tree -- adjacent pairs first, an unpaired last element
+// passing up unchanged, until one value remains.  GroupTree takes the group
+// sums in row order (up to 16 groups): level k holds the pending left
+// operand of a block of 2^k groups, and a block is added to its right
+// neighbour as soon as that one is complete, which gives the tree's
+// additions.  The result then adds the pending blocks from the smallest
+// (rightmost) to the largest: with n groups, the blocks of n's set bits.
+template <int C>
+struct GroupTree {
+  float lv[5][C];
+  int n;
+
+  __device__ __forceinline__ GroupTree() : n(0) {}
+
+  __device__ __forceinline__ static void vadd(float (&d)[C], const float (&a)[C], const float (&b)[C]) {
+#pragma unroll
+    for (int c = 0; c < C; ++c) d[c] = __fadd_rn(a[c], b[c]);
+  }
+  __device__ __forceinline__ static void vcopy(float (&d)[C], const float (&a)[C]) {
+#pragma unroll
+    for (int c = 0; c < C; ++c) d[c] = a[c];
+  }
+  // the next group's sum (consumed)
+  __device__ __forceinline__ void push(float (&e)[C]) {
+    if ((n & 1) == 0) {
+      vcopy(lv[0], e);
+    } else {
+      vadd(e, lv[0], e);
+      if ((n & 2) == 0) {
+        vcopy(lv[1], e);
+      } else {
+        vadd(e, lv[1], e);
+        if ((n & 4) == 0) {
+          vcopy(lv[2], e);
+        } else {
+          vadd(e, lv[2], e);
+          if ((n & 8) == 0) {
+            vcopy(lv[3], e);
+          } else {
+            vadd(e, lv[3], e);
+            vcopy(lv[4], e);
+          }
+        }
+      }
+    }
+    ++n;
+  }
+  // the tree's root (+0 when no group was pushed)
+  __device__ __forceinline__ void result(float (&out)[C]) const {
+    bool have = false;
+#pragma unroll
+    for (int c = 0; c < C; ++c) out[c] = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 5; ++k)
+      if ((n >> k) & 1) {
+        if (have) vadd(out, lv[k], out);
+        else vcopy(out, lv[k]);
+        have = true;
+      }
+  }
+};
+
 // byte k of w as an exact float: the bits 0x4B0000bb are 2^23 + bb
 __device__ __forceinline__ float byte_magic(uint32_t w, int k) {
   return __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540u | (uint32_t)k));

@@ -30,7 +30,13 @@ struct DecodeArgs {
   // to it instead of the write-back
   float* s32 = nullptr;
   int src32 = 0, dst32 = 0;
+  // test hook (brs_test_starve_copies): bytes a head's copy barrier expects
+  // beyond what its copies deliver (0 in normal use)
+  uint32_t tx_extra = 0;
 };
+
+// the host thread's test-hook setting (brs_test_starve_copies)
+uint32_t starve_tx_bytes();
 
 cudaError_t launch_decode(const DecodeArgs& a, int d, int store, bool had, cudaStream_t st);
 // the general (warp-per-head) kernel for every shape it supports, with the
@@ -51,9 +57,10 @@ struct CalibArgs {
 };
 cudaError_t launch_calib_sample(const CalibArgs& a, cudaStream_t st);
 cudaError_t launch_calib_finish(const CalibArgs& a, cudaStream_t st);
-// d = 128 DAMP decode with bulk-copy staging of the stored rows
-bool decode_tma_supported(int d, int store, int block, int k_hi);
-cudaError_t launch_decode_tma(const DecodeArgs& a, bool had, cudaStream_t st);
+// d = 128 DAMP decode, one CTA per head with the state in registers
+// (persistent CTAs, bulk-copy staging of each head's stored bytes)
+bool decode_cta_supported(int d, int store, int block, int k_hi, int mode);
+cudaError_t launch_decode_cta(const DecodeArgs& a, bool had, cudaStream_t st);
 
 struct PackArgs {
   int B, H, d, storage, k_hi, block, hadamard;

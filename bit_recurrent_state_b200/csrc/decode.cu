@@ -4,9 +4,9 @@
 // order twice: pass 1 dequantizes, decays and accumulates u = S^T k; pass 2
 // reads the rows again (from L2), repeats the identical dequantize and
 // decay, applies the delta-rule write, accumulates o = S^T q and requantizes
-// in batches of NRB rows.  Every sum over rows is therefore a lane-local
-// fmaf chain in stored order, no thread block barrier is involved, and many
-// heads run concurrently on every SM.
+// in batches of NRB rows.  Every sum over rows is therefore lane-local (8-row
+// chains and their pairwise tree), no thread block barrier is involved, and
+// many heads run concurrently on every SM.
 //
 // Sources: DAMP summary, Key Points > Implementation (fused executor:
 // reconstruct the INT8 channels, update in FP32, re-quantize, write back;
@@ -21,10 +21,11 @@
 // the INT8 rows in the Hadamard basis, the FP16 rows in the value basis.
 //   u = U2 + T(U1), w = beta (v - u), S_i += k_i T(w) (INT8 rows),
 //   S_i += k_i w (FP16 rows), o = O2 + T(O1),
-// with U1/O1 and U2/O2 fmaf chains over the INT8 and the FP16 rows in
-// stored order and T the Hadamard (or the identity).  Paired f32x2
-// instructions are two independent IEEE operations: pairing changes no
-// result.
+// with U1/O1 and U2/O2 the sums over the INT8 and the FP16 rows and T the
+// Hadamard (or the identity).  Every sum over rows is taken in the library's
+// order: 8-row fmaf chains in stored order, added in a pairwise tree
+// (GroupTree).  Paired f32x2 instructions are two independent IEEE
+// operations: pairing changes no result.
 //
 // Write-back modes: nearest, stochastic (Philox4x32-10), error feedback
 // (FP16 residual), and direction memory ("When Quantization Breaks Memory",
@@ -259,9 +260,27 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
   // ---- pass 1: u = U2 + T(U1) over the decayed rows.  INT8 rows stream in
   // chunks of CH rows with the next chunk's codes and grids already in
   // flight (double buffering keeps 2*CH row loads per warp outstanding).
-  float u1[C], u2[C];
+  // sums over rows in the library's order: rows arrive in stored order; a
+  // group closes after 8 rows of its tier (or at the tier's end) and goes to
+  // the tier's tree; the INT8 tier's tree gives U1, the FP16 tier's U2
+  float u1[C], u2[C], acc[C];
+  GroupTree<C> tree;
 #pragma unroll
-  for (int c = 0; c < C; ++c) { u1[c] = 0.f; u2[c] = 0.f; }
+  for (int c = 0; c < C; ++c) { u1[c] = 0.f; u2[c] = 0.f; acc[c] = 0.f; }
+  auto feed = [&](int i, float k0, float k1, const float (&x)[C], float (&t1)[C]) {
+    v_fma_s<C>(acc, k0, k1, x);
+    const bool lo_tier = i < nlo;
+    const int rel = lo_tier ? i : i - nlo;
+    if ((rel & 7) == 7 || i + 1 == (lo_tier ? nlo : D)) {
+      tree.push(acc);
+#pragma unroll
+      for (int c = 0; c < C; ++c) acc[c] = 0.f;
+    }
+    if (i + 1 == nlo) {
+      tree.result(t1);
+      tree.n = 0;
+    }
+  };
   if constexpr (STORE == BRS_STORE_FP32) {
 #pragma unroll 8
     for (int i = 0; i < D; ++i) {
@@ -269,7 +288,7 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
       load_row(i, x);
       const float4 ka = sm.rs[i].ka;
       v_scale<C>(x, ka.z, ka.w);
-      v_fma_s<C>(u1, ka.x, ka.y, x);
+      feed(i, ka.x, ka.y, x, u1);
     }
   } else if (src32) {
     // FP32 rows from the interval state: the same chains, INT8 tier then
@@ -296,8 +315,7 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
       for (int r = 0; r < NRB; ++r) {
         const float4 ka = sm.rs[i0 + r].ka;
         v_scale<C>(xb[buf][r], ka.z, ka.w);
-        if (i0 + r < nlo) v_fma_s<C>(u1, ka.x, ka.y, xb[buf][r]);
-        else v_fma_s<C>(u2, ka.x, ka.y, xb[buf][r]);
+        feed(i0 + r, ka.x, ka.y, xb[buf][r], u1);
       }
     };
     static_assert(D % (2 * NRB) == 0, "pairs of batches");
@@ -338,7 +356,7 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
           dequant_int8<C>(x, cw[buf][r], sv, sv, zv, zv);
         }
         v_scale<C>(x, rsc.ka.z, rsc.ka.w);
-        v_fma_s<C>(u1, rsc.ka.x, rsc.ka.y, x);
+        feed(i0 + r, rsc.ka.x, rsc.ka.y, x, u1);
       }
     };
     const int nch = nlo / CH;
@@ -355,9 +373,10 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
       load_row(i, x);
       const float4 ka = sm.rs[i].ka;
       v_scale<C>(x, ka.z, ka.w);
-      v_fma_s<C>(u2, ka.x, ka.y, x);
+      feed(i, ka.x, ka.y, x, u1);
     }
   }
+  if (STORE != BRS_STORE_FP32) tree.result(u2);     // the FP16 tier (+0 when it is empty)
   float w[C], wt[C];
   {
     if constexpr (STORE != BRS_STORE_FP32 && HAD) warp_fwht<D>(u1, lane, a.hscale);
@@ -376,7 +395,8 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
   // ---- pass 2: write, o, requantize (batches of NRB rows)
   float o1[C], o2[C];
 #pragma unroll
-  for (int c = 0; c < C; ++c) { o1[c] = 0.f; o2[c] = 0.f; }
+  for (int c = 0; c < C; ++c) { o1[c] = 0.f; o2[c] = 0.f; acc[c] = 0.f; }
+  tree.n = 0;
   // the next batch's rows are fetched while this batch is requantized
   uint32_t pw[NRB], ps[(NB > 1) ? NRB : 1];
   const uint8_t* prow = hin + col0;
@@ -424,13 +444,9 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
       const RowScal rsc = sm.rs[i];
       const float2 qv = sm.qq[i];
       v_scale<C>(x[r], rsc.ka.z, rsc.ka.w);
-      if (STORE == BRS_STORE_FP32 || i0 < nlo) {
-        v_fma_vec<C>(x[r], rsc.ka.x, rsc.ka.y, wt);
-        v_fma_s<C>(o1, qv.x, qv.y, x[r]);
-      } else {
-        v_fma_vec<C>(x[r], rsc.ka.x, rsc.ka.y, w);
-        v_fma_s<C>(o2, qv.x, qv.y, x[r]);
-      }
+      if (STORE == BRS_STORE_FP32 || i0 < nlo) v_fma_vec<C>(x[r], rsc.ka.x, rsc.ka.y, wt);
+      else v_fma_vec<C>(x[r], rsc.ka.x, rsc.ka.y, w);
+      feed(i, qv.x, qv.y, x[r], o1);
     }
     if (STORE != BRS_STORE_FP32 && !src32 && i0 + NRB < nlo) prefetch();
     if (STORE == BRS_STORE_FP32 || dst32) {
@@ -685,6 +701,7 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
   }
 
   // ---- o = O2 + T(O1)
+  if (STORE != BRS_STORE_FP32) tree.result(o2);
   if constexpr (STORE != BRS_STORE_FP32 && HAD) warp_fwht<D>(o1, lane, a.hscale);
   float ov[C];
   bool bad = false;
@@ -751,8 +768,7 @@ cudaError_t launch_decode(const DecodeArgs& a, int d, int store, bool had, cudaS
     }
     return cudaErrorInvalidValue;
   }
-  if (a.mode != BRS_ROUND_DIRECTION && decode_tma_supported(d, store, a.block, a.k_hi))
-    return launch_decode_tma(a, had, st);
+  if (decode_cta_supported(d, store, a.block, a.k_hi, a.mode)) return launch_decode_cta(a, had, st);
   if (d == 128 && a.block == 128) return launch_db<128, 128>(a, store, had, st);
   if (d == 128 && a.block == 32) return launch_db<128, 32>(a, store, had, st);
   if (d == 64 && a.block == 64) return launch_db<64, 64>(a, store, had, st);

@@ -18,7 +18,8 @@
 //      the codes (nearest / Philox stochastic / error feedback) and the
 //      bit-packed row at its new offset.
 // Layout of the update: lane l owns columns 4l..4l+3 (d = 128) of every
-// row, so each sum over rows is a lane-local fmaf chain in row order.
+// row, so each sum over rows is lane-local: 8-row fmaf chains in row order
+// added in a pairwise tree (the library's order, GroupTree).
 #include <cuda_runtime.h>
 #include <cstdint>
 #include <type_traits>
@@ -122,21 +123,27 @@ __global__ void __launch_bounds__(32 * kVbWarps) varbit_kernel(const VbArgs a) {
   const float beta = a.beta[head];
   __syncwarp();
 
-  // ---- pass 1: u = S^T k over the decayed rows
+  // ---- pass 1: u = S^T k over the decayed rows (8-row chains, pairwise tree)
   float u[C];
+  GroupTree<C> tree;
+  for (int g = 0; g < D / 8; ++g) {
+    float acc[C];
 #pragma unroll
-  for (int c = 0; c < C; ++c) u[c] = 0.f;
+    for (int c = 0; c < C; ++c) acc[c] = 0.f;
 #pragma unroll 4
-  for (int i = 0; i < D; ++i) {
-    const VbRow r = sm.row[i];
-    float x[C];
-    vb_dequant<C, WIDE, ONE>(x, pay_in + r.off, r, lane);
+    for (int i = 8 * g; i < 8 * g + 8; ++i) {
+      const VbRow r = sm.row[i];
+      float x[C];
+      vb_dequant<C, WIDE, ONE>(x, pay_in + r.off, r, lane);
 #pragma unroll
-    for (int c = 0; c < C; c += 2) {
-      mul2(x[c], x[c + 1], r.ka.z, r.ka.w, x[c], x[c + 1]);
-      fma2(u[c], u[c + 1], r.ka.x, r.ka.y, x[c], x[c + 1], u[c], u[c + 1]);
+      for (int c = 0; c < C; c += 2) {
+        mul2(x[c], x[c + 1], r.ka.z, r.ka.w, x[c], x[c + 1]);
+        fma2(acc[c], acc[c + 1], r.ka.x, r.ka.y, x[c], x[c + 1], acc[c], acc[c + 1]);
+      }
     }
+    tree.push(acc);
   }
+  tree.result(u);
   float w[C];
   {
     bool bad = false;
@@ -148,10 +155,10 @@ __global__ void __launch_bounds__(32 * kVbWarps) varbit_kernel(const VbArgs a) {
     if (bad) raise_flag(a.flags, BRS_FLAG_NONFINITE);
   }
 
-  // ---- pass 2 in batches
+  // ---- pass 2 in batches (a batch is one 8-row group of o's sum)
+  static_assert(kVbBatch == 8, "a requantization batch is one group of the row sums");
   float o[C];
-#pragma unroll
-  for (int c = 0; c < C; ++c) o[c] = 0.f;
+  tree.n = 0;
   const uint8_t* pay_out = pout + (size_t)b * a.sec.payload_per_seq;
   const uint8_t* wd_out = pout + a.sec.off_width + (size_t)b * rows + h * D;
   const uint32_t* of_out = (const uint32_t*)(pout + a.sec.off_offsets) + (size_t)b * (rows + 1) + h * D;
@@ -159,7 +166,9 @@ __global__ void __launch_bounds__(32 * kVbWarps) varbit_kernel(const VbArgs a) {
   uint16_t* auxh = (MODE == BRS_ROUND_ERRFEEDBACK) ? (uint16_t*)a.aux + (size_t)head * D * D : nullptr;
 
   for (int i0 = 0; i0 < D; i0 += kVbBatch) {
-    float x[kVbBatch][C];
+    float x[kVbBatch][C], og[C];
+#pragma unroll
+    for (int c = 0; c < C; ++c) og[c] = 0.f;
 #pragma unroll
     for (int r = 0; r < kVbBatch; ++r) {
       const VbRow rr = sm.row[i0 + r];
@@ -171,9 +180,10 @@ __global__ void __launch_bounds__(32 * kVbWarps) varbit_kernel(const VbArgs a) {
       }
       if constexpr (PHASE == 0) {
 #pragma unroll
-        for (int c = 0; c < C; c += 2) fma2(o[c], o[c + 1], rr.qq.x, rr.qq.y, x[r][c], x[r][c + 1], o[c], o[c + 1]);
+        for (int c = 0; c < C; c += 2) fma2(og[c], og[c + 1], rr.qq.x, rr.qq.y, x[r][c], x[r][c + 1], og[c], og[c + 1]);
       }
     }
+    if constexpr (PHASE == 0) tree.push(og);
     if constexpr (MODE == BRS_ROUND_ERRFEEDBACK && PHASE == 1) {
 #pragma unroll
       for (int r = 0; r < kVbBatch; ++r) {
@@ -384,6 +394,7 @@ __global__ void __launch_bounds__(32 * kVbWarps) varbit_kernel(const VbArgs a) {
 
   if constexpr (PHASE == 0) {
     // ---- o
+    tree.result(o);
     bool bad = false;
 #pragma unroll
     for (int c = 0; c < C; ++c) bad |= !isfinite(o[c]);

@@ -24,11 +24,11 @@ import numpy as np
 
 
 def bf16_bits(x: np.ndarray) -> np.ndarray:
-    """float -> bfloat16 bit patterns, round to nearest, ties to even."""
+    """float -> bfloat16 bit patterns, round to nearest, ties to even (finite
+    inputs: the sum below stays under 2^32 for every finite float)."""
     f = np.ascontiguousarray(x, dtype=np.float32)
-    u = f.view(np.uint32).astype(np.uint64)
-    lsb = (u >> 16) & 1
-    r = ((u + 0x7FFF + lsb) >> 16).astype(np.uint16)
+    u = f.view(np.uint32)
+    r = ((u + (np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1)))) >> np.uint32(16)).astype(np.uint16)
     return r
 
 

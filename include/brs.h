@@ -346,6 +346,17 @@ brs_status brs_fetch_errors_noalloc(uint32_t* flags_out, void* stream);
  * raw bits. */
 brs_status brs_fetch_errors(void* workspace, uint32_t* flags_out, void* stream);
 
+/* Test hook for the bounded device waits (the pages have no counterpart).
+ * While `on` is nonzero, brs_decode_step calls made from this host thread
+ * make the copy barrier of every head of the CTA-per-head decode kernel
+ * (DAMP storage, d = 128) expect 16 bytes more than the head's copies
+ * deliver: the copies complete, the barrier never does, every bounded wait
+ * runs out (200 ms), and the kernel raises BRS_FLAG_TIMEOUT and returns
+ * without writing the stored state or the outputs.  Nothing faults and the
+ * context stays usable; brs_fetch_errors then reports BRS_ETIMEOUT.  Off by
+ * default; not for use outside tests. */
+void brs_test_starve_copies(int on);
+
 /* Message of the last error returned on this host thread ("" if none). */
 const char* brs_last_error(void);
 

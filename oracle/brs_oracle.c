@@ -18,8 +18,10 @@
  * Operation order (the pages fix FP32 but not the order of a sum; these
  * orders are this implementation's reading and the CUDA library follows the
  * same written definition):
- *   - every sum over key rows runs i = 0, 1, ..., d-1 as an fmaf chain
- *     starting from +0;
+ *   - every sum over key rows (over one tier's rows in the mixed basis)
+ *     is taken in groups of 8 consecutive rows, each an fmaf chain in row
+ *     order from +0, whose sums are then added in a pairwise tree (adjacent
+ *     pairs first, an unpaired last element passing up): row_sum below;
  *   - every sum over value columns (variable-width fit error) runs
  *     j = 0, 1, ..., d-1 as an fmaf chain starting from +0;
  *   - the Hadamard transform is the unnormalised butterfly, stages
@@ -677,6 +679,28 @@ static int damp_store(const orc_layout* L, const orc_writeback* wb, int64_t step
   return flags;
 }
 
+/* One write-back of given FP32 states (the quantizer of the recurrence on
+ * its own, so that a state computed elsewhere can be replayed through it):
+ * units [u0, u1) of S [B][H][d][d] (stored row order, in the working basis of
+ * the layout's domain) are quantized with the rounding of wb at token
+ * `step` into packed (DAMP storage), with residuals or direction counters in
+ * aux as orc_run keeps them.  For direction memory packed holds, on entry,
+ * the stored state the write-back replaces.  Returns ORC_* flags. */
+int orc_damp_writeback(const orc_layout* L, const orc_writeback* wb, int64_t step, int u0, int u1,
+                       const float* S, void* packed, void* aux) {
+  if (L->storage != ORC_STORE_DAMP || u0 < 0 || u1 > L->B * L->H || u0 > u1) return ORC_EINVAL;
+  int d = L->d, flags = 0;
+  size_t hb = damp_head_bytes(L), nel = (size_t)(d - L->k_hi) * d;
+  for (int u = u0; u < u1; ++u) {
+    uint8_t* head = (uint8_t*)packed + (size_t)u * hb;
+    uint16_t* aux_head = NULL;
+    if (aux) aux_head = (wb->mode == ORC_ROUND_DIRECTION) ? (uint16_t*)((uint8_t*)aux + (size_t)u * (nel / 4))
+                                                         : (uint16_t*)aux + (size_t)u * nel;
+    flags |= damp_store(L, wb, step, u / L->H, u % L->H, S + (size_t)u * d * d, head, head, aux_head, NULL);
+  }
+  return flags;
+}
+
 /* ------------------------------------------------------------------------ */
 /* One token of the gated delta rule on one head, in FP32 ([DAMP] Error      */
 /* propagation model: S = Q(A_t S + beta_t k_t v_t^T) with A_t the decayed   */
@@ -687,22 +711,42 @@ static int damp_store(const orc_layout* L, const orc_writeback* wb, int64_t step
 /* kk, qq, aa are gathered in stored row order; vv and the returned oo are  */
 /* in the basis of S's columns.                                             */
 /* ------------------------------------------------------------------------ */
+/* Sum over the key rows i0 .. i1-1 of c_i S_ij (column j), in the order of
+ * the arithmetic contract: each group of 8 consecutive rows (the last one
+ * may be shorter) is an fmaf chain in row order from +0; the group sums are
+ * then added in a pairwise tree, adjacent pairs first (g0 + g1, g2 + g3,
+ * ...), an unpaired last element passing up unchanged, level after level
+ * until one value remains.  No rows: +0. */
+static float row_sum(const float* c, const float* S, int d, int j, int i0, int i1) {
+  float part[64];
+  int n = 0;
+  for (int g = i0; g < i1; g += 8) {
+    float acc = 0.0f;
+    int ge = g + 8 < i1 ? g + 8 : i1;
+    for (int i = g; i < ge; ++i) acc = fmaf(c[i], S[(size_t)i * d + j], acc);
+    part[n++] = acc;
+  }
+  if (n == 0) return 0.0f;
+  while (n > 1) {
+    int m = 0;
+    for (int p = 0; p + 1 < n; p += 2) part[m++] = part[p] + part[p + 1];
+    if (n & 1) part[m++] = part[n - 1];
+    n = m;
+  }
+  return part[0];
+}
+
 static void delta_rule_token(int d, float* S, const float* kk, const float* qq, const float* aa,
                              const float* vv, float bt, float* w, float* oo) {
   for (int i = 0; i < d; ++i)
     for (int j = 0; j < d; ++j) S[(size_t)i * d + j] = aa[i] * S[(size_t)i * d + j];
   for (int j = 0; j < d; ++j) {
-    float u = 0.0f;
-    for (int i = 0; i < d; ++i) u = fmaf(kk[i], S[(size_t)i * d + j], u);
+    float u = row_sum(kk, S, d, j, 0, d);
     w[j] = bt * (vv[j] - u);
   }
   for (int i = 0; i < d; ++i)
     for (int j = 0; j < d; ++j) S[(size_t)i * d + j] = fmaf(kk[i], w[j], S[(size_t)i * d + j]);
-  for (int j = 0; j < d; ++j) {
-    float acc = 0.0f;
-    for (int i = 0; i < d; ++i) acc = fmaf(qq[i], S[(size_t)i * d + j], acc);
-    oo[j] = acc;
-  }
+  for (int j = 0; j < d; ++j) oo[j] = row_sum(qq, S, d, j, 0, d);
 }
 
 /* The same token in the mixed basis: rows 0..nlo-1 (INT8 tier) are in the
@@ -711,7 +755,8 @@ static void delta_rule_token(int d, float* S, const float* kk, const float* qq, 
  *   u  = U2 + T(U1),  U1 = sum over rows < nlo of k_i S_i,  U2 = the rest;
  *   w  = beta (v - u);  S_i += k_i T(w) for rows < nlo, S_i += k_i w else;
  *   o  = O2 + T(O1) with O1, O2 the q-weighted sums of the updated rows.
- * Each partial sum is an fmaf chain over its rows in stored order from +0. */
+ * Each partial sum is a row_sum over its tier's rows (8-row chains in stored
+ * order, then the pairwise tree). */
 static void delta_rule_token_mixed(int d, int nlo, int had, float* S, const float* kk,
                                    const float* qq, const float* aa, const float* vv, float bt,
                                    float* w, float* oo) {
@@ -720,11 +765,8 @@ static void delta_rule_token_mixed(int d, int nlo, int had, float* S, const floa
   for (int i = 0; i < d; ++i)
     for (int j = 0; j < d; ++j) S[(size_t)i * d + j] = aa[i] * S[(size_t)i * d + j];
   for (int j = 0; j < d; ++j) {
-    float u1 = 0.0f, u2 = 0.0f;
-    for (int i = 0; i < nlo; ++i) u1 = fmaf(kk[i], S[(size_t)i * d + j], u1);
-    for (int i = nlo; i < d; ++i) u2 = fmaf(kk[i], S[(size_t)i * d + j], u2);
-    p1[j] = u1;
-    oo[j] = u2;
+    p1[j] = row_sum(kk, S, d, j, 0, nlo);
+    oo[j] = row_sum(kk, S, d, j, nlo, d);
   }
   if (had) orc_fwht(p1, d);
   for (int j = 0; j < d; ++j) {
@@ -737,11 +779,8 @@ static void delta_rule_token_mixed(int d, int nlo, int had, float* S, const floa
     for (int j = 0; j < d; ++j)
       S[(size_t)i * d + j] = fmaf(kk[i], (i < nlo) ? wt[j] : w[j], S[(size_t)i * d + j]);
   for (int j = 0; j < d; ++j) {
-    float o1 = 0.0f, o2 = 0.0f;
-    for (int i = 0; i < nlo; ++i) o1 = fmaf(qq[i], S[(size_t)i * d + j], o1);
-    for (int i = nlo; i < d; ++i) o2 = fmaf(qq[i], S[(size_t)i * d + j], o2);
-    p1[j] = o1;
-    oo[j] = o2;
+    p1[j] = row_sum(qq, S, d, j, 0, nlo);
+    oo[j] = row_sum(qq, S, d, j, nlo, d);
   }
   if (had) orc_fwht(p1, d);
   for (int j = 0; j < d; ++j) oo[j] = oo[j] + p1[j];

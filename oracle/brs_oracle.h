@@ -123,6 +123,12 @@ int orc_run(const orc_layout* L, const orc_writeback* wb, int64_t step0, int T, 
             const int16_t* perm, const uint16_t* q, const uint16_t* k, const uint16_t* v,
             const float* beta, const float* decay, float* o, float* t_dump, float* s_dump);
 
+/* One write-back (quantizer only) of the FP32 states of units [u0, u1)
+ * (S [B][H][d][d], stored row order, the domain's working basis) at token
+ * `step` into DAMP storage `packed`, residuals / counters in aux. */
+int orc_damp_writeback(const orc_layout* L, const orc_writeback* wb, int64_t step, int u0, int u1,
+                       const float* S, void* packed, void* aux);
+
 /* Protected-row selection by the DAMP risk score on a calibration run.
  * Inputs as orc_run for Bc sequences and T tokens (FP32 recurrence from a
  * zero state, identity order); the state is sampled every `every` tokens.

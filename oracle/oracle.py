@@ -103,6 +103,8 @@ def lib():
             L.orc_run.restype = ct.c_int
             L.orc_run.argtypes = [P, P, ct.c_int64, ct.c_int, ct.c_int, ct.c_int, P, P, P, P, P,
                                   P, P, P, P, P, P, P, P]
+            L.orc_damp_writeback.restype = ct.c_int
+            L.orc_damp_writeback.argtypes = [P, P, ct.c_int64, ct.c_int, ct.c_int, P, P, P]
             L.orc_calibrate.restype = ct.c_int
             L.orc_calibrate.argtypes = [P, ct.c_int, ct.c_int, ct.c_int, ct.c_double, P, P, P, P,
                                         P, P, P]
@@ -299,11 +301,25 @@ def run(cfg: Config, wb_mode: int, seed: int, C: int, step0: int, inputs: dict, 
     return o, fl, t
 
 
+def damp_writeback(cfg: Config, wb_mode: int, seed: int, step: int, S, packed, aux=None, units=None):
+    """One write-back (the quantizer alone) of the FP32 states S [B][H][d][d]
+    (stored row order, the domain's working basis) of the given units into
+    ``packed`` (updated in place, as are the residuals / counters ``aux``).
+    Returns the flags."""
+    L = cfg.layout()
+    wb = WriteBack(wb_mode, seed, 1)
+    S = _c(S, np.float32)
+    u0, u1 = (0, cfg.B * cfg.H) if units is None else units
+    assert packed.flags["C_CONTIGUOUS"] and (aux is None or aux.flags["C_CONTIGUOUS"])
+    return lib().orc_damp_writeback(ct.byref(L), ct.byref(wb), step, u0, u1, _p(S), _p(packed), _p(aux))
+
+
 def run_parallel(cfg: Config, wb_mode: int, seed: int, C: int, step0: int, inputs: dict, packed,
-                 aux=None, stats=None, perm=None, units=None, threads=None):
+                 aux=None, stats=None, perm=None, units=None, threads=None, dump_s=False):
     """``run`` with the units split over threads (units are independent).
 
-    Returns (o, flags, threads_used)."""
+    Returns (o, flags, threads_used), and the state dump of ``run`` last when
+    ``dump_s`` is set."""
     nunits = cfg.B if cfg.storage == STORE_VARBIT else cfg.B * cfg.H
     u0, u1 = (0, nunits) if units is None else units
     nthr = max(1, min(threads or os.cpu_count() or 1, u1 - u0))
@@ -318,18 +334,21 @@ def run_parallel(cfg: Config, wb_mode: int, seed: int, C: int, step0: int, input
     o = np.zeros((T, cfg.B, cfg.H, cfg.d), np.float32)
     perm = _c(perm, np.int16)
     bounds = np.linspace(u0, u1, nthr + 1).astype(int)
+    sd = np.zeros((cfg.B, cfg.H, cfg.d, cfg.d), np.float32) if dump_s else None
 
     def work(i):
         return lib().orc_run(ct.byref(L), ct.byref(wb), step0, T, int(bounds[i]),
                              int(bounds[i + 1]), _p(packed), _p(packed), _p(aux), _p(stats),
                              _p(perm), _p(q), _p(k), _p(v), _p(beta), _p(decay), _p(o), None,
-                             None)
+                             _p(sd))
 
     with ThreadPoolExecutor(nthr) as ex:
         flags = list(ex.map(work, range(nthr)))
     fl = 0
     for f in flags:
         fl |= f
+    if dump_s:
+        return o, fl, nthr, sd
     return o, fl, nthr
 
 

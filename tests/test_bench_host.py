@@ -15,7 +15,7 @@ def test_kernel_family_and_bytes():
     import bench
     from bit_recurrent_state_b200 import synth
     w = synth.WORKLOADS["kda_decode"]
-    assert bench.kernel_family(w) == "tma"
+    assert bench.kernel_family(w) == "cta"
     assert bench.kernel_family(w.with_(mode="direction")) == "warp"      # direction memory: general kernel
     assert bench.kernel_family(synth.WORKLOADS["kda_decode_c8"]) == "warp"
     assert bench.kernel_family(synth.WORKLOADS["varbit_decode"]) == "varbit"
@@ -24,7 +24,7 @@ def test_kernel_family_and_bytes():
     dm = bench.algorithmic_bytes(w.with_(mode="direction"))
     assert dm["aux"] == 2 * 64 * 32 * (112 * 128 // 4)                    # 2-bit counters read + written
     assert dm["total"] - base["total"] == dm["aux"]
-    # a DRAM record keyed to the TMA kernel does not describe the general kernel
+    # a DRAM record keyed to the CTA kernel does not describe the general kernel
     assert bench.traffic_record(w.with_(mode="direction")) is None
 
 

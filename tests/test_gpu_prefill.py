@@ -50,6 +50,7 @@ def _run_chunks(w, nchunks, units=None, mode="nearest"):
         inp = _seq_major(w, t0, 64)
         st.packed.copy_(torch.from_numpy(packed_o))
         st.aux.copy_(torch.from_numpy(np.pad(aux_o.view(np.uint8), (0, st.aux.numel() - aux_o.nbytes))))
+        before_p, before_a = packed_o.copy(), aux_o.copy()
         o = torch.zeros((w.B, 64, w.H, w.d), device="cuda")
         dump = torch.zeros((w.B, w.H, w.d, w.d), device="cuda")
         d = {k: _dev(v) for k, v in inp.items()}
@@ -70,11 +71,14 @@ def _run_chunks(w, nchunks, units=None, mode="nearest"):
         so_u = so.reshape(w.B * w.H, w.d, w.d)[sel]
         rms_s = np.sqrt(np.mean(so_u.astype(np.float64) ** 2))
         assert np.max(np.abs(sg_u - so_u)) <= 2e-3 * rms_s, (c, np.max(np.abs(sg_u - so_u)) / rms_s)
-        if mode == "nearest":
-            # replay: the documented quantizer on the GPU's own state gives its codes
-            rp, fl = O.state_pack(cfg, sg, None)
-            assert fl == 0
-            np.testing.assert_array_equal(pg.reshape(w.B * w.H, hb)[sel], rp.reshape(w.B * w.H, hb)[sel])
+        # replay: the oracle's write-back (mode, seed, step, residuals) of the
+        # GPU's own pre-write-back state gives the GPU's codes and residuals
+        fl = O.damp_writeback(cfg, MODE[mode], w.seed, t0 + 63, sg, before_p, before_a)
+        assert fl == 0
+        np.testing.assert_array_equal(pg.reshape(w.B * w.H, hb)[sel], before_p.reshape(w.B * w.H, hb)[sel])
+        if mode == "errfeedback":
+            ag = st.aux.cpu().numpy()[: aux_o.nbytes].view(np.uint16)
+            np.testing.assert_array_equal(ag, before_a)
 
 
 @pytest.mark.parametrize("kw,mode", [
@@ -87,14 +91,6 @@ def _run_chunks(w, nchunks, units=None, mode="nearest"):
 def test_prefill_teacher_forced(kw, mode):
     w = synth.Workload("pf", T=192, C=64, seed=60, **kw)
     _run_chunks(w, 3, mode=mode)
-
-
-def test_prefill_full_size_sampled():
-    """The measured prefill configuration (B=8, H=32, d=128, 16 FP16 + 112
-    INT8-Hadamard rows, block 128), in the benchmark's launch configuration,
-    for the first two chunks; the oracle runs 6 of the 256 heads."""
-    w = synth.WORKLOADS["kda_prefill"]
-    _run_chunks(w, 2, units=(97, 103))
 
 
 @pytest.mark.parametrize("kw,mode", [

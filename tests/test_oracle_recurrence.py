@@ -311,3 +311,28 @@ def test_pack_unpack_roundtrip(orc):
         np.testing.assert_array_equal(S2[:, h, prot], S[:, h, prot].astype(np.float16).astype(np.float32))
     err = np.abs(S2 - S).max()
     assert err <= (S.max() - S.min()) / 255 * 2     # half a step per coordinate, spread by H
+
+
+@pytest.mark.parametrize("mode,dom", [(0, 0), (1, 0), (2, 0), (3, 2), (2, 2)])
+def test_writeback_replay_equals_the_run(orc, mode, dom):
+    """The write-back entry (the quantizer alone, used to replay a state
+    computed elsewhere) applied to the FP32 state the recurrence held just
+    before its write-back reproduces the recurrence's stored bytes and
+    residuals / counters, in every rounding mode."""
+    w = synth.Workload("rp", B=2, H=3, d=32, T=4, k_hi=4, block=32, seed=21)
+    cfg = _cfg(orc, w, domain=dom)
+    rng = np.random.default_rng(22)
+    perm = _rand_perm(rng, w.H, w.d)
+    S0 = (rng.standard_normal((w.B, w.H, w.d, w.d)) * 0.1).astype(np.float32)
+    packed, _ = orc.state_pack(cfg, S0, perm)
+    _, aux, _ = orc.new_state(cfg)
+    inp = synth.run_inputs(w, 0, w.T)
+    for t in range(w.T):
+        before_p, before_a = packed.copy(), aux.copy()
+        _, fl, _, sd = orc.run(cfg, mode, 5, 1, t, {k: v[t:t + 1] for k, v in inp.items()}, packed,
+                               aux=aux, perm=perm, dump_s=True)
+        assert fl == 0
+        fl = orc.damp_writeback(cfg, mode, 5, t, sd, before_p, before_a)
+        assert fl == 0
+        np.testing.assert_array_equal(before_p, packed)
+        np.testing.assert_array_equal(before_a, aux)
