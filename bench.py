@@ -342,6 +342,37 @@ def cpu_oracle_sample(w, target_s: float = 12.0):
                       f"({dt:.1f} s wall on {used} threads)"}
 
 
+def time_steps(args, step, first: int, stream, barrier):
+    """Device time of args.steps consecutive steps (first, first+1, ...),
+    bracketed by a barrier and a synchronize on both sides, CUDA events on
+    the launching stream.  The steps are captured once into a CUDA graph and
+    replayed (no host launch overhead between the timed kernels) unless
+    --eager is given."""
+    import torch
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if args.eager:
+        barrier()
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(first + i)
+        ev1.record(stream)
+        barrier()
+        return ev0.elapsed_time(ev1)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):              # captured on torch's side stream (the library launches on
+        for i in range(args.steps):        # the current stream, which is the capture stream here)
+            step(first + i)
+    barrier()
+    ev0.record(stream)
+    with torch.cuda.stream(stream):
+        g.replay()
+    ev1.record(stream)
+    barrier()
+    t = ev0.elapsed_time(ev1)
+    del g
+    return t
+
+
 def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -418,13 +449,8 @@ def run_prefill(args, w):
 
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
-        barrier()
-        ev0.record(stream)
-        for i in range(args.steps):
-            step(i)
-        ev1.record(stream)
-        barrier()
-    ms_step = max_over_ranks(ev0.elapsed_time(ev1), world, dev) / args.steps
+        ms_run = time_steps(args, step, 0, stream, barrier)
+    ms_step = max_over_ranks(ms_run, world, dev) / args.steps
     flags = st.errors()
     # end to end: every step's inputs copied from pinned host memory and its o
     # read back inside the timed region, on copy streams that overlap the
@@ -496,6 +522,7 @@ def run_prefill(args, w):
         "e2e": {"value": units / (ms_e2e * 1e-3), "unit": UNIT, "h2d_bytes_per_step": inputs_b,
                 "d2h_bytes_per_step": out_b},
         "gpu_launches": args.steps, "device_flags": flags,
+        "launch": "eager" if args.eager else "cuda_graph (the timed steps captured once, replayed)",
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_sample(w)
@@ -574,13 +601,8 @@ def run_ours(args, w):
     # ---- device-resident throughput (kernel per step)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
-        barrier()
-        ev0.record(stream)
-        for i in range(args.steps):
-            step(args.warmup + i)
-        ev1.record(stream)
-        barrier()
-    ms_max = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+        ms_run = time_steps(args, step, args.warmup, stream, barrier)
+    ms_max = max_over_ranks(ms_run, world, dev)
     ms_step = ms_max / args.steps
 
     # ---- end to end through the public API with host buffers: every token's
@@ -655,6 +677,7 @@ def run_ours(args, w):
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps * (3 if varbit else 1),
         "device_flags": flags,
+        "launch": "eager" if args.eager else "cuda_graph (the timed steps captured once, replayed)",
     }
     if rank == 0:
         line["clocks"] = clk.summary()
@@ -677,6 +700,8 @@ def main():
     ap.add_argument("--mode", default=None,
                     help="write-back rounding: nearest | stochastic | errfeedback | direction")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="launch the timed steps one by one instead of replaying them as a CUDA graph")
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (small profiling cases)")
     ap.add_argument("--tokens", type=int, default=None, help="override the prefill length (small profiling cases)")
     ap.add_argument("--ref-budget", type=float, default=120.0,
