@@ -83,6 +83,9 @@ def algorithmic_bytes(w) -> dict:
     if w.mode == "direction":
         # 2-bit counters of the INT8 rows, read and written
         ef = 2 * (heads * (w.d - w.k_hi) * w.d // 4)
+    if w.mode.startswith("residual"):
+        # k-bit residual integers of the INT8 rows (kept in 4 bits), read and written
+        ef = 2 * (heads * (w.d - w.k_hi) * w.d // 2)
     st = 2 * stats
     state = 2 * n
     if w.C > 1 and w.storage == "damp":
@@ -295,7 +298,9 @@ class OracleRunner:
         self.units_total = w.B if self.varbit else w.B * w.H
         self.heads_per_unit = w.H if self.varbit else 1
         self.mode = {"nearest": O.ROUND_NEAREST, "stochastic": O.ROUND_STOCHASTIC,
-                     "errfeedback": O.ROUND_ERRFEEDBACK, "direction": O.ROUND_DIRECTION}[w.mode]
+                     "errfeedback": O.ROUND_ERRFEEDBACK, "direction": O.ROUND_DIRECTION,
+                     "residual2": O.ROUND_RESIDUAL2, "residual3": O.ROUND_RESIDUAL3,
+                     "residual4": O.ROUND_RESIDUAL4}[w.mode]
 
     def inputs(self, ntok):
         key = (self.t, ntok)

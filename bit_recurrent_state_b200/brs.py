@@ -16,10 +16,12 @@ LIB_PATH = os.path.join(_PKG, "libbrs.so")
 
 STORE_FP32, STORE_DAMP, STORE_VARBIT = 0, 1, 2
 ROUND_NEAREST, ROUND_STOCHASTIC, ROUND_ERRFEEDBACK, ROUND_DIRECTION = 0, 1, 2, 3
+ROUND_RESIDUAL2, ROUND_RESIDUAL3, ROUND_RESIDUAL4 = 4, 5, 6
 OK, EINVAL, EUNSUPPORTED, EALIGN, ECUDA, ENONFINITE, EOVERFLOW, ETIMEOUT = range(8)
 FLAG_NONFINITE, FLAG_OVERFLOW, FLAG_TIMEOUT = 1, 2, 4
 MODES = {"nearest": ROUND_NEAREST, "stochastic": ROUND_STOCHASTIC,
-         "errfeedback": ROUND_ERRFEEDBACK, "direction": ROUND_DIRECTION}
+         "errfeedback": ROUND_ERRFEEDBACK, "direction": ROUND_DIRECTION,
+         "residual2": ROUND_RESIDUAL2, "residual3": ROUND_RESIDUAL3, "residual4": ROUND_RESIDUAL4}
 STORES = {"fp32": STORE_FP32, "damp": STORE_DAMP, "varbit": STORE_VARBIT}
 
 # exported symbols declared in include/brs.h

@@ -178,10 +178,11 @@ brs_status brs_decode_step(const brs_layout* L, const brs_writeback* wb, int64_t
   (void)stats;
   if (!wb) return fail(BRS_EINVAL, "writeback is NULL");
   if (wb->C != 1) return fail(BRS_EUNSUPPORTED, "decode writes back every token (C = 1); got C = %d", wb->C);
-  if (wb->mode < 0 || wb->mode > 3) return fail(BRS_EINVAL, "unknown rounding mode %d", wb->mode);
-  if (wb->mode == BRS_ROUND_DIRECTION && L->storage != BRS_STORE_DAMP)
-    return fail(BRS_EUNSUPPORTED, "direction memory is built for DAMP storage");
-  if (wb->mode == BRS_ROUND_DIRECTION && !aux) return fail(BRS_EINVAL, "direction memory needs the counter buffer");
+  if (wb->mode < 0 || wb->mode > 6) return fail(BRS_EINVAL, "unknown rounding mode %d", wb->mode);
+  if (wb->mode >= BRS_ROUND_DIRECTION && L->storage != BRS_STORE_DAMP)
+    return fail(BRS_EUNSUPPORTED, "direction and residual memory are built for DAMP storage");
+  if (wb->mode >= BRS_ROUND_DIRECTION && !aux)
+    return fail(BRS_EINVAL, "direction and residual memory need the auxiliary buffer");
   if (step < 0) return fail(BRS_EINVAL, "step must be >= 0");
   if (!packed_in || !packed_out || !workspace || !q || !k || !v || !beta || !decay || !o)
     return fail(BRS_EINVAL, "a required pointer is NULL");
@@ -253,10 +254,11 @@ brs_status brs_decode_step_deferred(const brs_layout* L, const brs_writeback* wb
   if (!wb) return fail(BRS_EINVAL, "writeback is NULL");
   if (L->storage != BRS_STORE_DAMP) return fail(BRS_EUNSUPPORTED, "deferred decode write-back is built for DAMP storage");
   if (wb->C < 1) return fail(BRS_EINVAL, "write-back interval C must be >= 1 (got %d)", wb->C);
-  if (wb->mode < 0 || wb->mode > 3) return fail(BRS_EINVAL, "unknown rounding mode %d", wb->mode);
-  if (wb->mode == BRS_ROUND_DIRECTION && wb->C != 1)
-    return fail(BRS_EUNSUPPORTED, "direction memory is built for write-back every token (C = 1)");
-  if (wb->mode == BRS_ROUND_DIRECTION && !aux) return fail(BRS_EINVAL, "direction memory needs the counter buffer");
+  if (wb->mode < 0 || wb->mode > 6) return fail(BRS_EINVAL, "unknown rounding mode %d", wb->mode);
+  if (wb->mode >= BRS_ROUND_DIRECTION && wb->C != 1)
+    return fail(BRS_EUNSUPPORTED, "direction and residual memory are built for write-back every token (C = 1)");
+  if (wb->mode >= BRS_ROUND_DIRECTION && !aux)
+    return fail(BRS_EINVAL, "direction and residual memory need the auxiliary buffer");
   if (step < 0) return fail(BRS_EINVAL, "step must be >= 0");
   if (!brs::decode_supported(L->d, L->block, L->k_hi))
     return fail(BRS_EUNSUPPORTED,
@@ -295,8 +297,9 @@ brs_status brs_chunk_prefill(const brs_layout* L, const brs_writeback* wb, int64
   if (L->storage != BRS_STORE_DAMP) return fail(BRS_EUNSUPPORTED, "chunked prefill is built for DAMP storage");
   if (!brs::prefill_supported(L->d, L->block, L->k_hi, wb->C))
     return fail(BRS_EUNSUPPORTED, "chunked prefill is built for d = 128, C = 64, block 128 or 32");
-  if (wb->mode < 0 || wb->mode > 3) return fail(BRS_EINVAL, "unknown rounding mode %d", wb->mode);
-  if (wb->mode == BRS_ROUND_DIRECTION) return fail(BRS_EUNSUPPORTED, "direction memory is not built for the prefill");
+  if (wb->mode < 0 || wb->mode > 6) return fail(BRS_EINVAL, "unknown rounding mode %d", wb->mode);
+  if (wb->mode >= BRS_ROUND_DIRECTION)
+    return fail(BRS_EUNSUPPORTED, "direction and residual memory are not built for the prefill");
   if (T <= 0 || T % wb->C || step0 < 0 || step0 % wb->C)
     return fail(BRS_EINVAL, "T and step0 must be multiples of C (T = %d, C = %d)", T, wb->C);
   if (!packed || !workspace || !q || !k || !v || !beta || !decay || !o)

@@ -32,7 +32,9 @@
 // Post-training write-back interventions and diagnostics; Trajectory
 // analysis): nearest codes plus a 2-bit sign counter per INT8 element that
 // takes a vote from every proposed change inside (scale/8, scale/2) and
-// moves the code one level at +-2.  The kernel also carries the FP32 state
+// moves the code one level at +-2; and k-bit residual memory (error feedback
+// whose residual is kept as a k-bit integer of step/2^k, nibbles in the
+// auxiliary buffer).  The kernel also carries the FP32 state
 // between write-backs when the write-back interval is C > 1 (interval-state
 // flags).
 #include <cuda_runtime.h>
@@ -44,6 +46,8 @@
 namespace brs {
 
 constexpr int kWarpsPerCta = 2;   // small CTAs: an even spread of heads over the SMs
+// kernel instantiation of k-bit residual memory (ABI modes BRS_ROUND_RESIDUAL2..4; k at run time)
+constexpr int kModeResidual = 16;
 
 template <int D>
 struct WGeo {
@@ -183,6 +187,11 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
   uint16_t* auxb = (MODE == BRS_ROUND_ERRFEEDBACK) ? (uint16_t*)a.aux + (size_t)head * nlo * D : nullptr;
   // direction memory: 2-bit counters, four to a byte in column order
   uint8_t* dmb = (MODE == BRS_ROUND_DIRECTION) ? (uint8_t*)a.aux + (size_t)head * nlo * (D / 4) : nullptr;
+  // residual memory: k-bit integers, two to a byte in column order
+  uint8_t* rmb = (MODE == kModeResidual) ? (uint8_t*)a.aux + (size_t)head * nlo * (D / 2) : nullptr;
+  const int rm_k = (MODE == kModeResidual) ? a.mode - BRS_ROUND_RESIDUAL2 + 2 : 2;   // residual bits
+  const float rm_unit = (float)(1 << rm_k), rm_inv = __fdiv_rn(1.0f, rm_unit);   // 2^k, 2^-k (exact)
+  const int rm_max = (1 << (rm_k - 1)) - 1;
 
   // ---- inputs: k, a, q gathered through the permutation and the stored
   // grid of every INT8 row, as ready pairs; v of my columns
@@ -417,6 +426,7 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
     const bool int8_batch = (STORE != BRS_STORE_FP32) && (i0 < nlo);   // batches are tier-uniform
     float x[NRB][C];
     float xp[(MODE == BRS_ROUND_DIRECTION) ? NRB : 1][C];   // stored values the step started from
+    float sp[(MODE == kModeResidual) ? NRB : 1];                // stored steps the step started from
     // the batch's rows: dequantized from the prefetched codes, or loaded
     // (all NRB loads issued before the first use)
     if (int8_batch && !src32) {
@@ -425,9 +435,11 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
         if constexpr (NB == 1) {
           const float4 g = sm.rs[i0 + r].sz;
           dequant_int8<C>(x[r], pw[r], g.x, g.y, g.z, g.w);
+          if constexpr (MODE == kModeResidual) sp[r] = g.x;
         } else {
           const float sv = f16_to_f32((uint16_t)(ps[r] & 0xffffu)), zv = f16_to_f32((uint16_t)(ps[r] >> 16));
           dequant_int8<C>(x[r], pw[r], sv, sv, zv, zv);
+          if constexpr (MODE == kModeResidual) sp[r] = sv;
         }
         if constexpr (MODE == BRS_ROUND_DIRECTION) {
 #pragma unroll
@@ -503,6 +515,24 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
           }
 #pragma unroll
           for (int c = 0; c < C; ++c) x[r][c] = __fadd_rn(x[r][c], f16_to_f32(ev[c]));
+        }
+      }
+      // ---- INT8 batch: residual-memory target y + m (sprev / 2^k)
+      uint32_t rmw[(MODE == kModeResidual) ? NRB : 1];     // my elements' integers, 4 bits each
+      if constexpr (MODE == kModeResidual) {
+#pragma unroll
+        for (int r = 0; r < NRB; ++r) {
+          const uint8_t* src = rmb + ((size_t)(i0 + r) * D + col0) / 2;
+          if constexpr (C == 4) rmw[r] = *(const uint16_t*)src;
+          else if constexpr (C == 2) rmw[r] = *src;
+          else rmw[r] = (*src >> (4 * (col0 & 1))) & 15u;
+          const float su = __fmul_rn(sp[r], rm_inv);       // exact
+#pragma unroll
+          for (int c = 0; c < C; ++c) {
+            const int f = (int)((rmw[r] >> (4 * c)) & 15u);
+            const int m = (f & 8) ? f - 16 : f;
+            x[r][c] = __fadd_rn(x[r][c], __fmul_rn((float)m, su));
+          }
         }
       }
       // ---- block extremes: local, then a reduce-scatter over the GL lanes
@@ -680,6 +710,29 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
         } else {
           *dst = (uint8_t)magic_byte(mq[0]);
         }
+        if constexpr (MODE == kModeResidual) {
+          // the new integers: rne((y - value) * (1/scale) * 2^k), clipped to
+          // +-(2^(k-1) - 1); the lanes of one byte merge their nibbles
+          uint32_t nb = 0;
+#pragma unroll
+          for (int c = 0; c < C; ++c) {
+            const float code = __fsub_rn(mq[c], kRoundMagic);          // exact
+            const float res = __fsub_rn(x[r][c], __fmaf_rn(code, p.s, p.z));
+            const float q = rintf(__fmul_rn(__fmul_rn(res, p.rcp), rm_unit));
+            int m = (q != q) ? 0 : (int)fminf(fmaxf(q, (float)-rm_max), (float)rm_max);
+            nb |= ((uint32_t)m & 15u) << (4 * c);
+          }
+          uint8_t* dst = rmb + ((size_t)i * D + col0) / 2;
+          if constexpr (C == 4) {
+            *(uint16_t*)dst = (uint16_t)nb;
+          } else if constexpr (C == 2) {
+            *dst = (uint8_t)nb;
+          } else {
+            nb <<= 4 * (col0 & 1);
+            nb |= __shfl_xor_sync(0xffffffffu, nb, 1);
+            if ((col0 & 1) == 0) *dst = (uint8_t)nb;
+          }
+        }
         if constexpr (MODE == BRS_ROUND_ERRFEEDBACK) {
           uint16_t ev[C];
 #pragma unroll
@@ -737,6 +790,9 @@ static cudaError_t launch_db(const DecodeArgs& a, int store, bool had, cudaStrea
     case BRS_ROUND_STOCHASTIC: return launch_dbm<D, BLOCK, BRS_ROUND_STOCHASTIC>(a, store, had, st);
     case BRS_ROUND_ERRFEEDBACK: return launch_dbm<D, BLOCK, BRS_ROUND_ERRFEEDBACK>(a, store, had, st);
     case BRS_ROUND_DIRECTION: return launch_dbm<D, BLOCK, BRS_ROUND_DIRECTION>(a, store, had, st);
+    case BRS_ROUND_RESIDUAL2:
+    case BRS_ROUND_RESIDUAL3:
+    case BRS_ROUND_RESIDUAL4: return launch_dbm<D, BLOCK, kModeResidual>(a, store, had, st);
   }
   return cudaErrorInvalidValue;
 }

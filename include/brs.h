@@ -121,7 +121,21 @@ typedef enum {
      only.  The counters live in the first B*H*(d-k_hi)*d/4 bytes of the
      residual buffer (four to a byte, column order, two's complement), which
      starts zeroed. */
-  BRS_ROUND_DIRECTION = 3
+  BRS_ROUND_DIRECTION = 3,
+  /* k-bit residual memory, k = 2, 3, 4 ([WB] Post-training write-back
+     interventions: error feedback's residual with evaluated widths
+     k = 2, 3, 4; Matched recurrent-memory training campaign: a 4-bit visible
+     state plus two auxiliary bits): error feedback whose residual is kept as
+     a k-bit signed integer m of step/2^k, |m| <= 2^(k-1) - 1.  The target is
+     y + m (sprev / 2^k), sprev the block's stored step the token started
+     from; codes and grid are those of nearest write-back of the target; the
+     new m = clamp(rne((target - value) * (1/scale) * 2^k)).  DAMP decode with
+     C = 1 only.  The integers live in the first B*H*(d-k_hi)*d/2 bytes of
+     the residual buffer (two to a byte, column order, element e in bits
+     4 (e % 2), two's complement), which starts zeroed. */
+  BRS_ROUND_RESIDUAL2 = 4,
+  BRS_ROUND_RESIDUAL3 = 5,
+  BRS_ROUND_RESIDUAL4 = 6
 } brs_round;
 
 /* Device flag bits OR-ed into the first 32-bit word of `workspace`. */

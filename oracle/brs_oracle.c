@@ -263,6 +263,38 @@ int orc_int8_block_dm(const float* y, const float* xprev, int n, int8_t* m_inout
   return flags;
 }
 
+/* k-bit residual memory ([WB] Post-training write-back interventions and
+ * diagnostics: error feedback's auxiliary residual carries the quantization
+ * error forward, with evaluated widths k = 2, 3, 4; Matched recurrent-memory
+ * training campaign: a 4-bit visible state plus two auxiliary bits; the
+ * Chinese summary's core method lists k-bit quantized residual memory beside
+ * error feedback).  Reading: error feedback whose residual is kept in k bits,
+ * as the signed integer m of step/2^k nearest to it, symmetric range
+ * |m| <= 2^(k-1) - 1.  The target is y + m_prev * (sprev / 2^k), sprev being
+ * the block's step when m_prev was stored; the grid and codes are those of
+ * nearest rounding of the target; then m = clamp(rne(r * (1/scale) * 2^k))
+ * with r = target - value. */
+int orc_int8_block_rm(const float* y, int n, int kbits, float sprev, int8_t* m_inout, uint8_t* codes,
+                      uint16_t* scale_h, uint16_t* zero_h, float* t_out) {
+  if (kbits < 2 || kbits > 4 || n <= 0) return ORC_EINVAL;
+  const float unit = ldexpf(1.0f, kbits);                 /* 2^k */
+  const float sunit = sprev / unit;                       /* exact: a power-of-two scaling of an FP16 value */
+  const int mmax = (1 << (kbits - 1)) - 1;
+  float* tgt = (float*)malloc(sizeof(float) * (size_t)n);
+  for (int j = 0; j < n; ++j) tgt[j] = y[j] + (float)m_inout[j] * sunit;
+  int flags = orc_int8_block(tgt, n, ORC_ROUND_NEAREST, 0, 0, 0, 0, 0, NULL, codes, scale_h, zero_h, t_out);
+  float s = orc_f32_from_f16(*scale_h), z = orc_f32_from_f16(*zero_h);
+  float rcp = (s == 0.0f) ? 0.0f : 1.0f / s;
+  for (int j = 0; j < n; ++j) {
+    float r = tgt[j] - fmaf((float)codes[j], s, z);
+    float q = nearbyintf((r * rcp) * unit);
+    int m = (q != q) ? 0 : (q > (float)mmax ? mmax : (q < (float)-mmax ? -mmax : (int)q));
+    m_inout[j] = (int8_t)m;
+  }
+  free(tgt);
+  return flags;
+}
+
 /* Variable-width symmetric row ([LB] Levels and storage): levels
  * {-n..n}*Delta, n = 2^(b-1) - 1, Delta = f*R/n with R the row's absolute
  * maximum and f fitted over 16 values in [1/4, 1] (read as f_m = (5+m)/20)
@@ -622,6 +654,17 @@ static void dm_put(uint8_t* dm, size_t e, int m) {
   dm[e >> 2] = (uint8_t)((dm[e >> 2] & ~(3 << sh)) | ((m & 3) << sh));
 }
 
+/* k-bit residual-memory integers, two to a byte in column order (element e
+ * of a head in bits 4(e mod 2) .. +3 of byte e/2, two's complement) */
+static int rm_get(const uint8_t* rm, size_t e) {
+  int f = (rm[e >> 1] >> (4 * (e & 1))) & 15;
+  return (f & 8) ? f - 16 : f;
+}
+static void rm_put(uint8_t* rm, size_t e, int m) {
+  int sh = 4 * (int)(e & 1);
+  rm[e >> 1] = (uint8_t)((rm[e >> 1] & ~(15 << sh)) | ((m & 15) << sh));
+}
+
 /* prev: the stored head this write-back replaces (read block by block just
  * before it is overwritten, so it may be the same memory as head); used by
  * direction memory only, whose counters sit in aux_head as bytes. */
@@ -651,6 +694,16 @@ static int damp_store(const orc_layout* L, const orc_writeback* wb, int64_t step
       if (L->hadamard && !rotated(L) && !mixed(L)) orc_fwht(tmp, d);
       for (int bl = 0; bl < nb; ++bl) {
         int j0 = bl * L->block;
+        if (wb->mode >= ORC_ROUND_RESIDUAL2 && wb->mode <= ORC_ROUND_RESIDUAL4) {
+          uint8_t* rmh = (uint8_t*)aux_head;
+          float ps = orc_f32_from_f16(psz[((size_t)i * nb + bl) * 2 + 0]);
+          for (int j = 0; j < L->block; ++j) mm[j] = (int8_t)rm_get(rmh, (size_t)i * d + j0 + j);
+          flags |= orc_int8_block_rm(tmp + j0, L->block, wb->mode - 2, ps, mm, codes + (size_t)i * d + j0,
+                                     &sz[((size_t)i * nb + bl) * 2 + 0], &sz[((size_t)i * nb + bl) * 2 + 1],
+                                     t_head ? t_head + (size_t)i * d + j0 : NULL);
+          for (int j = 0; j < L->block; ++j) rm_put(rmh, (size_t)i * d + j0 + j, mm[j]);
+          continue;
+        }
         if (wb->mode == ORC_ROUND_DIRECTION) {
           uint8_t* dmh = (uint8_t*)aux_head;
           float ps = orc_f32_from_f16(psz[((size_t)i * nb + bl) * 2 + 0]);
@@ -694,8 +747,11 @@ int orc_damp_writeback(const orc_layout* L, const orc_writeback* wb, int64_t ste
   for (int u = u0; u < u1; ++u) {
     uint8_t* head = (uint8_t*)packed + (size_t)u * hb;
     uint16_t* aux_head = NULL;
-    if (aux) aux_head = (wb->mode == ORC_ROUND_DIRECTION) ? (uint16_t*)((uint8_t*)aux + (size_t)u * (nel / 4))
-                                                         : (uint16_t*)aux + (size_t)u * nel;
+    if (aux) {
+      if (wb->mode == ORC_ROUND_DIRECTION) aux_head = (uint16_t*)((uint8_t*)aux + (size_t)u * (nel / 4));
+      else if (wb->mode >= ORC_ROUND_RESIDUAL2) aux_head = (uint16_t*)((uint8_t*)aux + (size_t)u * (nel / 2));
+      else aux_head = (uint16_t*)aux + (size_t)u * nel;
+    }
     flags |= damp_store(L, wb, step, u / L->H, u % L->H, S + (size_t)u * d * d, head, head, aux_head, NULL);
   }
   return flags;
@@ -854,8 +910,11 @@ static int run_head_unit(const orc_layout* L, const orc_writeback* wb, int64_t s
       } else {
         size_t nel = (size_t)(d - L->k_hi) * d;
         uint16_t* aux_head = NULL;
-        if (aux) aux_head = (wb->mode == ORC_ROUND_DIRECTION) ? (uint16_t*)((uint8_t*)aux + unit * (nel / 4))
-                                                             : aux + unit * nel;
+        if (aux) {
+          if (wb->mode == ORC_ROUND_DIRECTION) aux_head = (uint16_t*)((uint8_t*)aux + unit * (nel / 4));
+          else if (wb->mode >= ORC_ROUND_RESIDUAL2) aux_head = (uint16_t*)((uint8_t*)aux + unit * (nel / 2));
+          else aux_head = aux + unit * nel;
+        }
         float* th = t_dump ? t_dump + unit * (size_t)d * d : NULL;
         const uint8_t* prev = (t == 0) ? pin + unit * hb : pout + unit * hb;
         flags |= damp_store(L, wb, step, b, h, S, prev, pout + unit * hb, aux_head, th);
@@ -1064,7 +1123,9 @@ int orc_run(const orc_layout* L, const orc_writeback* wb, int64_t step0, int T, 
             const int16_t* perm, const uint16_t* q, const uint16_t* k, const uint16_t* v,
             const float* beta, const float* decay, float* o, float* t_dump, float* s_dump) {
   if (!layout_ok(L) || wb->C <= 0 || step0 % wb->C || T % wb->C) return ORC_EINVAL;
-  if (wb->mode < ORC_ROUND_NEAREST || wb->mode > ORC_ROUND_DIRECTION) return ORC_EINVAL;
+  if (wb->mode < ORC_ROUND_NEAREST || wb->mode > ORC_ROUND_RESIDUAL4) return ORC_EINVAL;
+  /* residual memory: DAMP storage, integers kept in the auxiliary buffer */
+  if (wb->mode >= ORC_ROUND_RESIDUAL2 && (L->storage != ORC_STORE_DAMP || !aux)) return ORC_EINVAL;
   /* direction memory: DAMP at a write-back every token (the votes compare
    * each token's proposal with the value stored after the previous token) */
   if (wb->mode == ORC_ROUND_DIRECTION && (L->storage != ORC_STORE_DAMP || wb->C != 1 || !aux))

@@ -27,7 +27,8 @@ extern "C" {
 #endif
 
 enum { ORC_STORE_FP32 = 0, ORC_STORE_DAMP = 1, ORC_STORE_VARBIT = 2 };
-enum { ORC_ROUND_NEAREST = 0, ORC_ROUND_STOCHASTIC = 1, ORC_ROUND_ERRFEEDBACK = 2, ORC_ROUND_DIRECTION = 3 };
+enum { ORC_ROUND_NEAREST = 0, ORC_ROUND_STOCHASTIC = 1, ORC_ROUND_ERRFEEDBACK = 2, ORC_ROUND_DIRECTION = 3,
+       ORC_ROUND_RESIDUAL2 = 4, ORC_ROUND_RESIDUAL3 = 5, ORC_ROUND_RESIDUAL4 = 6 };
 enum { ORC_DOMAIN_CANONICAL = 0, ORC_DOMAIN_ROTATED = 1, ORC_DOMAIN_MIXED = 2 };
 
 /* status flags (OR-ed) */
@@ -79,6 +80,15 @@ int orc_int8_block(const float* y, int n, int mode, uint64_t seed, int64_t step,
  * each proposed change y - xprev inside (scale/8, scale/2); a counter that
  * reaches +-2 moves its code one level (clipped to [0, 255]) and is reset. */
 int orc_int8_block_dm(const float* y, const float* xprev, int n, int8_t* m_inout, uint8_t* codes,
+                      uint16_t* scale_h, uint16_t* zero_h, float* t_out);
+
+/* The INT8 block under k-bit residual memory (k = 2, 3, 4): error feedback
+ * whose residual is kept as a k-bit signed integer m (|m| <= 2^(k-1) - 1) in
+ * units of step/2^k.  e_prev = m * (sprev / 2^k) with sprev the block's step
+ * when m was stored (0 when sprev is 0); the target y + e_prev is quantized
+ * with nearest rounding; the new m = clamp(rne((y + e_prev - value) *
+ * (1/scale) * 2^k)) with the new block's scale (0 when the scale is 0). */
+int orc_int8_block_rm(const float* y, int n, int kbits, float sprev, int8_t* m_inout, uint8_t* codes,
                       uint16_t* scale_h, uint16_t* zero_h, float* t_out);
 
 /* One variable-width row (decay-aware allocation tier), width bw in [2, 8]. */

@@ -27,6 +27,7 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 
 STORE_FP32, STORE_DAMP, STORE_VARBIT = 0, 1, 2
 ROUND_NEAREST, ROUND_STOCHASTIC, ROUND_ERRFEEDBACK, ROUND_DIRECTION = 0, 1, 2, 3
+ROUND_RESIDUAL2, ROUND_RESIDUAL3, ROUND_RESIDUAL4 = 4, 5, 6
 DOMAIN_CANONICAL, DOMAIN_ROTATED, DOMAIN_MIXED = 0, 1, 2
 OK, EINVAL, ENONFINITE, EOVERFLOW = 0, 1, 2, 4
 
@@ -83,6 +84,8 @@ def lib():
                                          ct.c_int, ct.c_int, P, P, P, P, P]
             L.orc_int8_block_dm.restype = ct.c_int
             L.orc_int8_block_dm.argtypes = [P, P, ct.c_int, P, P, P, P, P]
+            L.orc_int8_block_rm.restype = ct.c_int
+            L.orc_int8_block_rm.argtypes = [P, ct.c_int, ct.c_int, ct.c_float, P, P, P, P, P]
             L.orc_persistence.restype = ct.c_double
             L.orc_persistence.argtypes = [ct.c_int, ct.c_double, ct.c_double, ct.c_int]
             L.orc_varbit_row.restype = ct.c_int
@@ -202,6 +205,19 @@ def int8_block_dm(y, xprev, m):
     m = np.array(m, dtype=np.int8)
     fl = lib().orc_int8_block_dm(_p(y), _p(xp), n, _p(m), _p(codes), _p(sh), _p(zh), _p(t))
     return dict(codes=codes, scale=sh[0], zero=zh[0], t=t, m=m, flags=fl)
+
+
+def int8_block_rm(y, kbits, sprev, m):
+    """One INT8 block under k-bit residual memory: (codes, scale_h, zero_h,
+    m_new, flags) for targets y, previous integers m (int8) and the step
+    sprev they were stored with."""
+    y = _c(y, np.float32)
+    m = np.array(m, dtype=np.int8)
+    codes = np.zeros(len(y), np.uint8)
+    sh, zh = ct.c_uint16(0), ct.c_uint16(0)
+    fl = lib().orc_int8_block_rm(_p(y), len(y), int(kbits), float(sprev), _p(m), _p(codes), ct.byref(sh),
+                                 ct.byref(zh), None)
+    return codes, sh.value, zh.value, m, fl
 
 
 def varbit_row(x, bw, mode=ROUND_NEAREST, seed=0, step=0, h=0, b=0, elem0=0, e=None):

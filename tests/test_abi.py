@@ -147,7 +147,7 @@ def test_argument_errors_before_device_work():
             fn()
         return e.value.status
 
-    for mode in (-1, 4):
+    for mode in (-1, 7):
         wb = brs.writeback_of(w, mode=mode)
         assert status(lambda: dec(wb)) == brs.EINVAL
         assert status(lambda: brs.decode_step_deferred(L, wb, 0, p, p, p, None, None, p, p, p, p, p, p,

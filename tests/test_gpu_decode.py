@@ -59,9 +59,10 @@ def _compare(w, steps, units=None):
         if w.mode == "errfeedback":
             per = ag.size // (w.B * w.H)
             np.testing.assert_array_equal(ag.reshape(w.B * w.H, per)[sel], ao.reshape(w.B * w.H, per)[sel])
-        if w.mode == "direction" and units is None:
-            # 2-bit counters of every head, then the unused rest of the buffer
-            np.testing.assert_array_equal(ag, ao, err_msg=f"direction counters after step {t}")
+        if (w.mode == "direction" or w.mode.startswith("residual")) and units is None:
+            # 2-bit counters / k-bit residual integers of every head, then the
+            # unused rest of the buffer
+            np.testing.assert_array_equal(ag, ao, err_msg=f"{w.mode} auxiliary state after step {t}")
 
 
 def test_kda_tiny_full_trajectory():
@@ -92,6 +93,12 @@ def test_kda_tiny_full_trajectory():
     ("kda64_dm", dict(B=2, H=3, d=64, k_hi=8, block=64, mode="direction")),
     ("kda32_nohad_dm", dict(B=2, H=2, d=32, k_hi=4, block=32, hadamard=0, mode="direction")),
     ("gdn128_dm", dict(B=3, H=4, Hk=2, d=128, k_hi=0, block=128, decay_per_key=0, mode="direction")),
+    ("kda128_rm2", dict(B=2, H=3, d=128, k_hi=16, block=128, mode="residual2")),
+    ("kda128_b32_rm3", dict(B=2, H=2, d=128, k_hi=16, block=32, mode="residual3")),
+    ("kda128_rm4", dict(B=2, H=3, d=128, k_hi=16, block=128, mode="residual4")),
+    ("kda64_rm4", dict(B=2, H=3, d=64, k_hi=8, block=64, mode="residual4")),
+    ("kda32_nohad_rm3", dict(B=2, H=2, d=32, k_hi=4, block=32, hadamard=0, mode="residual3")),
+    ("gdn128_rm2", dict(B=3, H=4, Hk=2, d=128, k_hi=0, block=128, decay_per_key=0, mode="residual2")),
     ("fp32_64", dict(B=2, H=3, d=64, storage="fp32")),
     ("fp32_gdn128", dict(B=2, H=4, Hk=2, d=128, storage="fp32", decay_per_key=0)),
 ])
@@ -102,18 +109,20 @@ def test_small_configs_bit_exact(name, kw):
     _compare(w, steps)
 
 
-def test_kda_decode_direction_memory_full_size_sampled():
-    """Direction-memory write-back at the KDA decode size (B=64, H=32,
-    d=128; the general kernel) for 16 tokens from a nonzero state; the
-    oracle runs 64 of the 2048 heads, whose codes, grids and 2-bit counters
-    must match."""
+@pytest.mark.parametrize("mode", ["direction", "residual2", "residual4"])
+def test_kda_decode_aux_memory_full_size_sampled(mode):
+    """Direction-memory and residual-memory write-back at the KDA decode
+    size (B=64, H=32, d=128; the general kernel) for 16 tokens from a
+    nonzero state; the oracle runs 64 of the 2048 heads, whose codes, grids
+    and auxiliary states (2-bit counters, k-bit residual integers) must
+    match."""
     import dataclasses
-    w = dataclasses.replace(synth.WORKLOADS["kda_decode"], mode="direction")
+    w = dataclasses.replace(synth.WORKLOADS["kda_decode"], mode=mode)
     perm = random_perm(w, seed=6)
     units = (500, 564)
     steps = _run_both(w, 16, perm=perm, units=units, init_scale=0.05)
     _compare(w, steps, units=units)
-    nel = (w.d - w.k_hi) * w.d // 4
+    nel = (w.d - w.k_hi) * w.d // (4 if mode == "direction" else 2)
     for *_, ag, ao in steps:
         np.testing.assert_array_equal(ag[units[0] * nel: units[1] * nel], ao[units[0] * nel: units[1] * nel])
 

@@ -336,3 +336,82 @@ def test_writeback_replay_equals_the_run(orc, mode, dom):
         assert fl == 0
         np.testing.assert_array_equal(before_p, packed)
         np.testing.assert_array_equal(before_a, aux)
+
+
+def test_residual_memory_through_the_recurrence(orc):
+    """k-bit residual memory on the dead-zone fixture of the test above
+    (fixed grid, step 1/128, one element drifting by about 0.064 step per
+    token).  The kept residual is at most (2^(k-1) - 1) step / 2^k: Delta/4
+    for k = 2 and 3 Delta/8 for k = 3, so the target never reaches the half
+    step and the code never moves, as under deterministic write-back; for
+    k = 4 it reaches 7 Delta/16, which with the drift passes the half step:
+    the code moves after 8 tokens (residual 1/16, 2/16, ..., 7/16 of a step),
+    in the same token as error feedback (whose residual is kept in FP16)."""
+    d, H, J = 32, 1, 17
+    w = synth.Workload("t", B=1, H=H, d=d, T=1, seed=6)
+    codes = np.random.default_rng(10).integers(1, 255, d)
+    codes[0], codes[1] = 0, 255
+    row = ((codes - 128) / 128.0).astype(np.float32)
+    v = row.copy()
+    v[J] += 0.5
+    moved = {}
+    for mode in (orc.ROUND_RESIDUAL2, orc.ROUND_RESIDUAL3, orc.ROUND_RESIDUAL4, orc.ROUND_ERRFEEDBACK):
+        cfg = orc.Config(B=1, H=H, d=d, storage=orc.STORE_DAMP, k_hi=0, block=32, hadamard=0)
+        S0 = np.zeros((1, H, d, d), np.float32)
+        S0[0, 0, 0] = row
+        packed, _ = orc.state_pack(cfg, S0)
+        _, aux, _ = orc.new_state(cfg)
+        key = np.zeros(d, np.float32)
+        key[0] = 1.0
+        first = None
+        for t in range(100):
+            inp = synth.run_inputs(w, t, 1)
+            inp["k"][0, 0, 0] = synth.bf16_bits(key)
+            inp["v"][0, 0, 0] = synth.bf16_bits(v)
+            inp["beta"][:] = 1e-3
+            inp["decay"][:] = 1.0
+            _, fl, _ = orc.run(cfg, mode, 0, 1, t, inp, packed, aux=aux)
+            assert fl == 0
+            if first is None and np.any(packed[:d] != codes):
+                first = t
+                assert packed[J] == codes[J] + 1
+        moved[mode] = first
+    assert moved[orc.ROUND_RESIDUAL2] is None and moved[orc.ROUND_RESIDUAL3] is None
+    assert moved[orc.ROUND_RESIDUAL4] == 7
+    assert moved[orc.ROUND_ERRFEEDBACK] == moved[orc.ROUND_RESIDUAL4]
+
+
+@pytest.mark.parametrize("kbits", [2, 3, 4])
+def test_residual_memory_block_against_fp64(orc, kbits):
+    """The residual-memory block against an FP64 restatement: the target
+    y + m_prev sprev / 2^k, its nearest INT8 codes on the block's FP16 grid
+    (exhaustive search over the 256 levels), and the new integer = the
+    residual in units of step / 2^k rounded to nearest (ties to even) and
+    clipped to +-(2^(k-1) - 1).  Values next to a rounding point of either
+    rounding (FP32 against FP64) are skipped and counted."""
+    from ref64 import int8_nearest64
+    rng = np.random.default_rng(40 + kbits)
+    mmax = 2 ** (kbits - 1) - 1
+    skipped = total = 0
+    for trial in range(300):
+        n = 32
+        y = (rng.standard_normal(n) * rng.uniform(0.01, 3.0)).astype(np.float32)
+        sprev = float(np.float16(rng.uniform(0.0, 0.05)))
+        mp = rng.integers(-mmax, mmax + 1, n).astype(np.int8)
+        codes, sh, zh, m, fl = orc.int8_block_rm(y, kbits, sprev, mp)
+        assert fl == 0
+        tgt = y.astype(np.float64) + mp.astype(np.float64) * sprev / 2 ** kbits
+        c64, s64, z64, t64 = int8_nearest64(tgt.astype(np.float32).astype(np.float64))
+        for j in range(n):
+            total += 1
+            frac_t = abs(t64[j] - np.floor(t64[j]) - 0.5)
+            if s64 == 0 or frac_t < 1e-3 or codes[j] != c64[j]:
+                skipped += 1
+                continue
+            q = (tgt[j] - (c64[j] * s64 + z64)) / s64 * 2 ** kbits
+            if abs(abs(q - np.floor(q)) - 0.5) < 1e-3:
+                skipped += 1
+                continue
+            want = int(np.clip(np.rint(q), -mmax, mmax))
+            assert m[j] == want, (trial, j, m[j], want, q)
+    assert skipped <= 0.02 * total
