@@ -174,14 +174,15 @@ static float sr_round(float t, uint32_t r24) {
   return ((float)r24 < fr * 16777216.0f) ? fl + 1.0f : fl;
 }
 
-/* INT8 asymmetric affine block ([DAMP] Quantization & calibration details:
- * per-block asymmetric affine quantization, b = 8; the stored scale and zero
- * are FP16): scale = fp16((max - min) / 255), zero = fp16(min),
- * code = clamp(round((y - zero) * (1 / scale)), 0, 255),
+/* Asymmetric affine block ([DAMP] Quantization & calibration details:
+ * per-block asymmetric affine quantization with b = 8 or 4; the stored
+ * scale and zero are FP16), L = 2^b - 1 levels above zero:
+ * scale = fp16((max - min) / L), zero = fp16(min),
+ * code = clamp(round((y - zero) * (1 / scale)), 0, L),
  * value = fmaf(code, scale, zero). */
-int orc_int8_block(const float* y, int n, int mode, uint64_t seed, int64_t step, int h, int b,
-                   int elem0, uint16_t* e_inout, uint8_t* codes, uint16_t* scale_h,
-                   uint16_t* zero_h, float* t_out) {
+int orc_lowbit_block(const float* y, int n, int levels, int mode, uint64_t seed, int64_t step, int h,
+                     int b, int elem0, uint16_t* e_inout, uint8_t* codes, uint16_t* scale_h,
+                     uint16_t* zero_h, float* t_out) {
   int flags = 0;
   if (n <= 0) return ORC_EINVAL;
   float* tgt = (float*)malloc(sizeof(float) * (size_t)n);
@@ -196,7 +197,7 @@ int orc_int8_block(const float* y, int n, int mode, uint64_t seed, int64_t step,
     if (tgt[j] < mn || (tgt[j] == mn && signbit(tgt[j]))) mn = tgt[j];
     if (tgt[j] > mx || (tgt[j] == mx && !signbit(tgt[j]))) mx = tgt[j];
   }
-  uint16_t sh = orc_f16_from_f32((mx - mn) / 255.0f);
+  uint16_t sh = orc_f16_from_f32((mx - mn) / (float)levels);
   uint16_t zh = orc_f16_from_f32(mn);
   if (f16_is_inf_or_nan(sh) || f16_is_inf_or_nan(zh)) flags |= ORC_EOVERFLOW;
   float s = orc_f32_from_f16(sh), z = orc_f32_from_f16(zh);
@@ -210,7 +211,7 @@ int orc_int8_block(const float* y, int n, int mode, uint64_t seed, int64_t step,
       else
         c = nearbyintf(t);
       if (c < 0.0f) c = 0.0f;
-      if (c > 255.0f) c = 255.0f;
+      if (c > (float)levels) c = (float)levels;
       if (!(c == c)) c = 0.0f;
     }
     codes[j] = (uint8_t)(int)c;
@@ -229,6 +230,13 @@ int orc_int8_block(const float* y, int n, int mode, uint64_t seed, int64_t step,
   return flags;
 }
 
+/* The INT8 block (b = 8, L = 255). */
+int orc_int8_block(const float* y, int n, int mode, uint64_t seed, int64_t step, int h, int b,
+                   int elem0, uint16_t* e_inout, uint8_t* codes, uint16_t* scale_h,
+                   uint16_t* zero_h, float* t_out) {
+  return orc_lowbit_block(y, n, 255, mode, seed, step, h, b, elem0, e_inout, codes, scale_h, zero_h, t_out);
+}
+
 /* Direction memory on the INT8 block ([WB] Post-training write-back
  * interventions and diagnostics: signed sub-threshold votes, a trigger that
  * moves the stored state by one level and resets the counter, transitions
@@ -241,9 +249,10 @@ int orc_int8_block(const float* y, int n, int mode, uint64_t seed, int64_t step,
  * when Delta/8 < |delta| < Delta/2 (Delta: the block's new step); a counter
  * that reaches +-2 moves the code one level that way (clipped to [0, 255])
  * and returns to 0. */
-int orc_int8_block_dm(const float* y, const float* xprev, int n, int8_t* m_inout, uint8_t* codes,
-                      uint16_t* scale_h, uint16_t* zero_h, float* t_out) {
-  int flags = orc_int8_block(y, n, ORC_ROUND_NEAREST, 0, 0, 0, 0, 0, NULL, codes, scale_h, zero_h, t_out);
+static int lowbit_block_dm(const float* y, const float* xprev, int n, int levels, int8_t* m_inout,
+                           uint8_t* codes, uint16_t* scale_h, uint16_t* zero_h, float* t_out) {
+  int flags = orc_lowbit_block(y, n, levels, ORC_ROUND_NEAREST, 0, 0, 0, 0, 0, NULL, codes, scale_h, zero_h,
+                               t_out);
   float s = orc_f32_from_f16(*scale_h);
   float lo = s * 0.125f, hi = s * 0.5f;
   for (int j = 0; j < n; ++j) {
@@ -254,13 +263,18 @@ int orc_int8_block_dm(const float* y, const float* xprev, int n, int8_t* m_inout
     if (m >= 2 || m <= -2) {
       int c = (int)codes[j] + (m > 0 ? 1 : -1);
       if (c < 0) c = 0;
-      if (c > 255) c = 255;
+      if (c > levels) c = levels;
       codes[j] = (uint8_t)c;
       m = 0;
     }
     m_inout[j] = (int8_t)m;
   }
   return flags;
+}
+
+int orc_int8_block_dm(const float* y, const float* xprev, int n, int8_t* m_inout, uint8_t* codes,
+                      uint16_t* scale_h, uint16_t* zero_h, float* t_out) {
+  return lowbit_block_dm(y, xprev, n, 255, m_inout, codes, scale_h, zero_h, t_out);
 }
 
 /* k-bit residual memory ([WB] Post-training write-back interventions and
@@ -274,15 +288,16 @@ int orc_int8_block_dm(const float* y, const float* xprev, int n, int8_t* m_inout
  * the block's step when m_prev was stored; the grid and codes are those of
  * nearest rounding of the target; then m = clamp(rne(r * (1/scale) * 2^k))
  * with r = target - value. */
-int orc_int8_block_rm(const float* y, int n, int kbits, float sprev, int8_t* m_inout, uint8_t* codes,
-                      uint16_t* scale_h, uint16_t* zero_h, float* t_out) {
+static int lowbit_block_rm(const float* y, int n, int levels, int kbits, float sprev, int8_t* m_inout,
+                           uint8_t* codes, uint16_t* scale_h, uint16_t* zero_h, float* t_out) {
   if (kbits < 2 || kbits > 4 || n <= 0) return ORC_EINVAL;
   const float unit = ldexpf(1.0f, kbits);                 /* 2^k */
   const float sunit = sprev / unit;                       /* exact: a power-of-two scaling of an FP16 value */
   const int mmax = (1 << (kbits - 1)) - 1;
-  float* tgt = (float*)malloc(sizeof(float) * (size_t)n);
+  float* tgt = (float*)calloc((size_t)n, sizeof(float));
   for (int j = 0; j < n; ++j) tgt[j] = y[j] + (float)m_inout[j] * sunit;
-  int flags = orc_int8_block(tgt, n, ORC_ROUND_NEAREST, 0, 0, 0, 0, 0, NULL, codes, scale_h, zero_h, t_out);
+  int flags = orc_lowbit_block(tgt, n, levels, ORC_ROUND_NEAREST, 0, 0, 0, 0, 0, NULL, codes, scale_h, zero_h,
+                               t_out);
   float s = orc_f32_from_f16(*scale_h), z = orc_f32_from_f16(*zero_h);
   float rcp = (s == 0.0f) ? 0.0f : 1.0f / s;
   for (int j = 0; j < n; ++j) {
@@ -293,6 +308,11 @@ int orc_int8_block_rm(const float* y, int n, int kbits, float sprev, int8_t* m_i
   }
   free(tgt);
   return flags;
+}
+
+int orc_int8_block_rm(const float* y, int n, int kbits, float sprev, int8_t* m_inout, uint8_t* codes,
+                      uint16_t* scale_h, uint16_t* zero_h, float* t_out) {
+  return lowbit_block_rm(y, n, 255, kbits, sprev, m_inout, codes, scale_h, zero_h, t_out);
 }
 
 /* Variable-width symmetric row ([LB] Levels and storage): levels
@@ -551,9 +571,31 @@ int orc_allocate_bits(int N, const double* c, double avg_bits, int b_min, int b_
 /* ------------------------------------------------------------------------ */
 static size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
+/* width of the DAMP low tier and its top code */
+static int low_bits(const orc_layout* L) { return L->low_bits == 4 ? 4 : 8; }
+static int low_levels(const orc_layout* L) { return (1 << low_bits(L)) - 1; }
+/* code e of a low-tier code array (bytes, or two codes to a byte with code e
+ * in bits 4 (e % 2) for the 4-bit tier) */
+static int code_get(const uint8_t* c, size_t e, int bits) {
+  return bits == 8 ? c[e] : (c[e >> 1] >> (4 * (e & 1))) & 15;
+}
+static void code_put(uint8_t* c, size_t e, int bits, int v) {
+  if (bits == 8) {
+    c[e] = (uint8_t)v;
+  } else {
+    int sh = 4 * (int)(e & 1);
+    c[e >> 1] = (uint8_t)((c[e >> 1] & ~(15 << sh)) | ((v & 15) << sh));
+  }
+}
+
+/* head layout: low-tier codes [d - k_hi][d * b / 8], FP16 rows [k_hi][d],
+ * (scale, zero) FP16 pairs [d - k_hi][d / block] */
+static size_t damp_code_bytes(const orc_layout* L) {
+  return (size_t)(L->d - L->k_hi) * (size_t)L->d * (size_t)low_bits(L) / 8;
+}
 static size_t damp_head_bytes(const orc_layout* L) {
   size_t d = (size_t)L->d, kh = (size_t)L->k_hi;
-  return kh * d * 2 + (d - kh) * d + (d - kh) * (d / (size_t)L->block) * 4;
+  return kh * d * 2 + damp_code_bytes(L) + (d - kh) * (d / (size_t)L->block) * 4;
 }
 
 typedef struct {
@@ -597,7 +639,7 @@ double orc_bits_per_value(const orc_layout* L) {
   double d = (double)L->d, kh = (double)L->k_hi;
   if (L->storage == ORC_STORE_FP32) return 32.0;
   if (L->storage == ORC_STORE_DAMP)
-    return (kh * d * 16.0 + (d - kh) * d * 8.0 + (d - kh) * (d / L->block) * 32.0) / (d * d);
+    return (kh * d * 16.0 + (d - kh) * d * (double)low_bits(L) + (d - kh) * (d / L->block) * 32.0) / (d * d);
   return L->avg_bits + (16.0 + 3.0) / d;
 }
 
@@ -622,10 +664,10 @@ static int mixed(const orc_layout* L) {
  * own inverse); in the rotated domain the FP16 rows are taken to the
  * Hadamard basis instead. */
 static void damp_load(const orc_layout* L, const uint8_t* head, float* S) {
-  int d = L->d, nlo = d - L->k_hi, nb = d / L->block;
+  int d = L->d, nlo = d - L->k_hi, nb = d / L->block, bits = low_bits(L);
   const uint8_t* codes = head;
-  const uint16_t* f16rows = (const uint16_t*)(head + (size_t)nlo * d);
-  const uint16_t* sz = (const uint16_t*)(head + (size_t)nlo * d + (size_t)L->k_hi * d * 2);
+  const uint16_t* f16rows = (const uint16_t*)(head + damp_code_bytes(L));
+  const uint16_t* sz = (const uint16_t*)(head + damp_code_bytes(L) + (size_t)L->k_hi * d * 2);
   for (int i = 0; i < d; ++i) {
     float* row = S + (size_t)i * d;
     if (i >= nlo) {
@@ -636,7 +678,7 @@ static void damp_load(const orc_layout* L, const uint8_t* head, float* S) {
         int bl = j / L->block;
         float s = orc_f32_from_f16(sz[((size_t)i * nb + bl) * 2 + 0]);
         float z = orc_f32_from_f16(sz[((size_t)i * nb + bl) * 2 + 1]);
-        row[j] = fmaf((float)codes[(size_t)i * d + j], s, z);
+        row[j] = fmaf((float)code_get(codes, (size_t)i * d + j, bits), s, z);
       }
       if (L->hadamard && !rotated(L) && !mixed(L)) orc_fwht(row, d);
     }
@@ -672,12 +714,14 @@ static int damp_store(const orc_layout* L, const orc_writeback* wb, int64_t step
                       const float* S, const uint8_t* prev, uint8_t* head, uint16_t* aux_head,
                       float* t_head) {
   int d = L->d, nlo = d - L->k_hi, nb = d / L->block, flags = 0;
+  int bits = low_bits(L), levels = low_levels(L);
   uint8_t* codes = head;
-  uint16_t* f16rows = (uint16_t*)(head + (size_t)nlo * d);
-  uint16_t* sz = (uint16_t*)(head + (size_t)nlo * d + (size_t)L->k_hi * d * 2);
-  const uint16_t* psz = (const uint16_t*)(prev + (size_t)nlo * d + (size_t)L->k_hi * d * 2);
+  uint16_t* f16rows = (uint16_t*)(head + damp_code_bytes(L));
+  uint16_t* sz = (uint16_t*)(head + damp_code_bytes(L) + (size_t)L->k_hi * d * 2);
+  const uint16_t* psz = (const uint16_t*)(prev + damp_code_bytes(L) + (size_t)L->k_hi * d * 2);
   float* xp = (float*)malloc(sizeof(float) * (size_t)L->block);
   int8_t* mm = (int8_t*)malloc((size_t)L->block);
+  uint8_t* cb = (uint8_t*)malloc((size_t)L->block);           /* one block's codes, one per byte */
   float* tmp = (float*)malloc(sizeof(float) * (size_t)d);
   for (int i = 0; i < d; ++i) {
     memcpy(tmp, S + (size_t)i * d, sizeof(float) * (size_t)d);
@@ -694,41 +738,38 @@ static int damp_store(const orc_layout* L, const orc_writeback* wb, int64_t step
       if (L->hadamard && !rotated(L) && !mixed(L)) orc_fwht(tmp, d);
       for (int bl = 0; bl < nb; ++bl) {
         int j0 = bl * L->block;
+        uint16_t* sh = &sz[((size_t)i * nb + bl) * 2 + 0];
+        uint16_t* zh = &sz[((size_t)i * nb + bl) * 2 + 1];
+        float* tb = t_head ? t_head + (size_t)i * d + j0 : NULL;
         if (wb->mode >= ORC_ROUND_RESIDUAL2 && wb->mode <= ORC_ROUND_RESIDUAL4) {
           uint8_t* rmh = (uint8_t*)aux_head;
           float ps = orc_f32_from_f16(psz[((size_t)i * nb + bl) * 2 + 0]);
           for (int j = 0; j < L->block; ++j) mm[j] = (int8_t)rm_get(rmh, (size_t)i * d + j0 + j);
-          flags |= orc_int8_block_rm(tmp + j0, L->block, wb->mode - 2, ps, mm, codes + (size_t)i * d + j0,
-                                     &sz[((size_t)i * nb + bl) * 2 + 0], &sz[((size_t)i * nb + bl) * 2 + 1],
-                                     t_head ? t_head + (size_t)i * d + j0 : NULL);
+          flags |= lowbit_block_rm(tmp + j0, L->block, levels, wb->mode - 2, ps, mm, cb, sh, zh, tb);
           for (int j = 0; j < L->block; ++j) rm_put(rmh, (size_t)i * d + j0 + j, mm[j]);
-          continue;
-        }
-        if (wb->mode == ORC_ROUND_DIRECTION) {
+        } else if (wb->mode == ORC_ROUND_DIRECTION) {
           uint8_t* dmh = (uint8_t*)aux_head;
           float ps = orc_f32_from_f16(psz[((size_t)i * nb + bl) * 2 + 0]);
           float pz = orc_f32_from_f16(psz[((size_t)i * nb + bl) * 2 + 1]);
           for (int j = 0; j < L->block; ++j) {
-            xp[j] = fmaf((float)prev[(size_t)i * d + j0 + j], ps, pz);
+            xp[j] = fmaf((float)code_get(prev, (size_t)i * d + j0 + j, bits), ps, pz);
             mm[j] = (int8_t)dm_get(dmh, (size_t)i * d + j0 + j);
           }
-          flags |= orc_int8_block_dm(tmp + j0, xp, L->block, mm, codes + (size_t)i * d + j0,
-                                     &sz[((size_t)i * nb + bl) * 2 + 0], &sz[((size_t)i * nb + bl) * 2 + 1],
-                                     t_head ? t_head + (size_t)i * d + j0 : NULL);
+          flags |= lowbit_block_dm(tmp + j0, xp, L->block, levels, mm, cb, sh, zh, tb);
           for (int j = 0; j < L->block; ++j) dm_put(dmh, (size_t)i * d + j0 + j, mm[j]);
-          continue;
+        } else {
+          uint16_t* e = aux_head ? aux_head + (size_t)i * d + j0 : NULL;
+          flags |= orc_lowbit_block(tmp + j0, L->block, levels, wb->mode, wb->seed, step, h, b, i * d + j0, e,
+                                    cb, sh, zh, tb);
         }
-        uint16_t* e = aux_head ? aux_head + (size_t)i * d + j0 : NULL;
-        flags |= orc_int8_block(tmp + j0, L->block, wb->mode, wb->seed, step, h, b, i * d + j0, e,
-                                codes + (size_t)i * d + j0, &sz[((size_t)i * nb + bl) * 2 + 0],
-                                &sz[((size_t)i * nb + bl) * 2 + 1],
-                                t_head ? t_head + (size_t)i * d + j0 : NULL);
+        for (int j = 0; j < L->block; ++j) code_put(codes, (size_t)i * d + j0 + j, bits, cb[j]);
       }
     }
   }
   free(tmp);
   free(xp);
   free(mm);
+  free(cb);
   return flags;
 }
 
@@ -1103,6 +1144,7 @@ static int run_seq_unit(const orc_layout* L, const orc_writeback* wb, int64_t st
 }
 
 static int layout_ok(const orc_layout* L) {
+  if (L->low_bits != 0 && L->low_bits != 8 && L->low_bits != 4) return 0;
   if (L->B <= 0 || L->H <= 0 || L->Hk <= 0 || L->H % L->Hk) return 0;
   if (L->d != 16 && L->d != 32 && L->d != 64 && L->d != 128) return 0;
   if (L->storage == ORC_STORE_DAMP) {
@@ -1228,7 +1270,7 @@ int orc_state_unpack(const orc_layout* L, const void* packed, const int16_t* per
 
 /* ------------------------------------------------------------------------ */
 /* Protected-row selection ([DAMP] Risk scoring and selection; Calibration): */
-/*   E_u  = mean squared error energy of row u under Hadamard-INT8           */
+/*   E_u  = mean squared error energy of row u under Hadamard-INT8 (INT4)    */
 /*          quantize -> dequantize, over the sampled calibration states;     */
 /*   a_eff,u = exp(mean log a_u);  P_u = 1 / max(1 - a_eff,u^2, tau);        */
 /*   C_u = E_u P_u; the top k_hi rows of each head are protected (ties to    */
@@ -1270,8 +1312,8 @@ int orc_calibrate(const orc_layout* L, int Bc, int T, int every, double tau,
             for (int bl = 0; bl < nb; ++bl) {
               uint16_t sh, zh;
               int j0 = bl * L->block;
-              orc_int8_block(row + j0, L->block, ORC_ROUND_NEAREST, 0, 0, 0, 0, 0, NULL, codes,
-                             &sh, &zh, NULL);
+              orc_lowbit_block(row + j0, L->block, low_levels(L), ORC_ROUND_NEAREST, 0, 0, 0, 0, 0, NULL,
+                               codes, &sh, &zh, NULL);
               float s = orc_f32_from_f16(sh), z = orc_f32_from_f16(zh);
               for (int j = 0; j < L->block; ++j) {
                 double e = (double)row[j0 + j] - (double)fmaf((float)codes[j], s, z);

@@ -46,6 +46,7 @@ typedef struct {
   int budget_scope;     /* VARBIT: 1 layer (all H*d rows of a sequence), 0 head */
   int domain;           /* ORC_DOMAIN_*: where the FP32 update is computed    */
   int persistence;      /* VARBIT cost weight: 0 erasure rate Gamma_hat, 1 w^(1), 2 h^(C) */
+  int low_bits;         /* DAMP low tier: 8 (also 0) or 4 bits per code       */
 } orc_layout;
 
 /* persistence weight of a row from A = EMA(a^2), K = EMA(beta (2-beta) k^2) */
@@ -74,6 +75,12 @@ float    orc_hadamard_scale(int n);
 int orc_int8_block(const float* y, int n, int mode, uint64_t seed, int64_t step, int h, int b,
                    int elem0, uint16_t* e_inout, uint8_t* codes, uint16_t* scale_h,
                    uint16_t* zero_h, float* t_out);
+
+/* The same asymmetric block with `levels` + 1 codes (255: INT8, 15: INT4):
+ * scale = fp16((max - min) / levels), codes clipped to [0, levels]. */
+int orc_lowbit_block(const float* y, int n, int levels, int mode, uint64_t seed, int64_t step, int h,
+                     int b, int elem0, uint16_t* e_inout, uint8_t* codes, uint16_t* scale_h,
+                     uint16_t* zero_h, float* t_out);
 
 /* The INT8 block under direction memory: nearest codes of y on the block's
  * grid, then 2-bit sign counters m_inout (values -1, 0, 1) take a vote from

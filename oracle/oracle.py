@@ -53,6 +53,7 @@ class Layout(ct.Structure):
         ("hadamard", ct.c_int), ("decay_per_key", ct.c_int),
         ("avg_bits", ct.c_double), ("b_min", ct.c_int), ("b_max", ct.c_int),
         ("budget_scope", ct.c_int), ("domain", ct.c_int), ("persistence", ct.c_int),
+        ("low_bits", ct.c_int),
     ]
 
 
@@ -82,6 +83,9 @@ def lib():
             L.orc_int8_block.restype = ct.c_int
             L.orc_int8_block.argtypes = [P, ct.c_int, ct.c_int, ct.c_uint64, ct.c_int64, ct.c_int,
                                          ct.c_int, ct.c_int, P, P, P, P, P]
+            L.orc_lowbit_block.restype = ct.c_int
+            L.orc_lowbit_block.argtypes = [P, ct.c_int, ct.c_int, ct.c_int, ct.c_uint64, ct.c_int64, ct.c_int,
+                                           ct.c_int, ct.c_int, P, P, P, P, P]
             L.orc_int8_block_dm.restype = ct.c_int
             L.orc_int8_block_dm.argtypes = [P, P, ct.c_int, P, P, P, P, P]
             L.orc_int8_block_rm.restype = ct.c_int
@@ -141,11 +145,12 @@ class Config:
     budget_scope: int = 1
     domain: int = DOMAIN_CANONICAL
     persistence: int = 0
+    low_bits: int = 8
 
     def layout(self) -> Layout:
         return Layout(self.B, self.H, self.Hk or self.H, self.d, self.storage, self.k_hi,
                       self.block, self.hadamard, self.decay_per_key, self.avg_bits, self.b_min,
-                      self.b_max, self.budget_scope, self.domain, self.persistence)
+                      self.b_max, self.budget_scope, self.domain, self.persistence, self.low_bits)
 
 
 # ---------------------------------------------------------------- scalars
@@ -189,6 +194,20 @@ def int8_block(y, mode=ROUND_NEAREST, seed=0, step=0, h=0, b=0, elem0=0, e=None)
     e = None if e is None else np.array(e, dtype=np.uint16)
     fl = lib().orc_int8_block(_p(y), n, mode, seed, step, h, b, elem0, _p(e), _p(codes), _p(sh),
                               _p(zh), _p(t))
+    return dict(codes=codes, scale=sh[0], zero=zh[0], t=t, e=e, flags=fl)
+
+
+def lowbit_block(y, levels, mode=ROUND_NEAREST, seed=0, step=0, h=0, b=0, elem0=0, e=None):
+    """One asymmetric block with levels + 1 codes (255: INT8, 15: INT4)."""
+    y = _c(y, np.float32)
+    n = y.size
+    codes = np.zeros(n, np.uint8)
+    sh = np.zeros(1, np.uint16)
+    zh = np.zeros(1, np.uint16)
+    t = np.zeros(n, np.float32)
+    e = None if e is None else np.array(e, dtype=np.uint16)
+    fl = lib().orc_lowbit_block(_p(y), n, int(levels), mode, seed, step, h, b, elem0, _p(e), _p(codes), _p(sh),
+                                _p(zh), _p(t))
     return dict(codes=codes, scale=sh[0], zero=zh[0], t=t, e=e, flags=fl)
 
 

@@ -39,22 +39,28 @@ def hadamard_n(n):
     return hadamard(n).astype(np.float64) / np.sqrt(n)
 
 
-def damp_head_sections(packed_head, d, k_hi, block):
+def damp_head_sections(packed_head, d, k_hi, block, bits=8):
     """Stored head -> (FP16 rows [k_hi][d], codes [d-k_hi][d], (scale, zero)
-    [d-k_hi][d/block][2]); INT8 rows come first in stored order."""
+    [d-k_hi][d/block][2]); low-tier rows come first in stored order, their
+    codes one per byte (bits = 8) or two per byte, code j in the low nibble
+    for even j (bits = 4)."""
     nb = d // block
     nlo = d - k_hi
-    codes = packed_head[: nlo * d].reshape(nlo, d)
-    f16rows = np.frombuffer(packed_head[nlo * d: nlo * d + k_hi * d * 2].tobytes(),
-                            np.uint16).reshape(k_hi, d)
-    sz = np.frombuffer(packed_head[nlo * d + k_hi * d * 2:].tobytes(), np.uint16)
+    cb = nlo * d * bits // 8
+    raw = np.asarray(packed_head[:cb], dtype=np.uint8)
+    if bits == 8:
+        codes = raw.reshape(nlo, d)
+    else:
+        codes = np.stack([raw & 15, raw >> 4], axis=-1).reshape(nlo, d)
+    f16rows = np.frombuffer(packed_head[cb: cb + k_hi * d * 2].tobytes(), np.uint16).reshape(k_hi, d)
+    sz = np.frombuffer(packed_head[cb + k_hi * d * 2:].tobytes(), np.uint16)
     sz = sz.reshape(nlo, nb, 2)
     return f16rows, codes, sz
 
 
-def damp_dequant64(packed_head, d, k_hi, block, had):
+def damp_dequant64(packed_head, d, k_hi, block, had, bits=8):
     """Stored head -> FP64 canonical state (stored row order)."""
-    f16rows, codes, sz = damp_head_sections(packed_head, d, k_hi, block)
+    f16rows, codes, sz = damp_head_sections(packed_head, d, k_hi, block, bits)
     nlo = d - k_hi
     S = np.zeros((d, d))
     S[nlo:] = f16_bits_to_f64(f16rows)
@@ -65,15 +71,16 @@ def damp_dequant64(packed_head, d, k_hi, block, had):
     return S
 
 
-def int8_nearest64(y):
-    """FP64 reference of one INT8 block: the FP16 step and zero from the
-    block's range, then the nearest of the 256 levels (exhaustive)."""
+def int8_nearest64(y, levels=255):
+    """FP64 reference of one asymmetric block (levels = 255: INT8, 15: INT4):
+    the FP16 step and zero from the block's range, then the nearest of the
+    levels + 1 grid points (exhaustive)."""
     mn, mx = y.min(), y.max()
-    s = float(np.float16((mx - mn) / 255.0))
+    s = float(np.float16((mx - mn) / levels))
     z = float(np.float16(mn))
     if s == 0:
         return np.zeros(len(y), int), s, z, np.zeros(len(y))
-    lev = np.arange(256) * s + z
+    lev = np.arange(levels + 1) * s + z
     dist = np.abs(y[:, None] - lev[None, :])
     return np.argmin(dist, axis=1), s, z, (y - z) / s
 

@@ -131,3 +131,12 @@ def test_storage_accounting(orc):
     assert orc.state_bytes(orc.Config(B=1, H=2, d=32, k_hi=4, block=32))[0] == 1264 * 2
     assert orc.state_bytes(orc.Config(B=256, H=32, Hk=16, d=128, k_hi=0, block=128,
                                       decay_per_key=0))[0] == 16896 * 256 * 32
+    # the 4-bit low tier ([DAMP] b = 4): 16 FP16 rows, 112 rows of 4-bit codes
+    # (64 bytes each) and the same FP16 scale/zero per block
+    int4_32 = orc.Config(B=1, H=1, d=128, k_hi=16, block=32, low_bits=4)
+    int4_128 = orc.Config(B=1, H=1, d=128, k_hi=16, block=128, low_bits=4)
+    assert orc.state_bytes(int4_32)[0] == 16 * 128 * 2 + 112 * 64 + 112 * 4 * 4
+    assert orc.state_bytes(int4_128)[0] == 16 * 128 * 2 + 112 * 64 + 112 * 4
+    assert orc.bits_per_value(int4_32) == 6.375 and orc.bits_per_value(int4_128) == 5.71875
+    for cfg in (int4_32, int4_128):
+        assert orc.bits_per_value(cfg) == orc.state_bytes(cfg)[0] * 8 / (128 * 128)

@@ -45,6 +45,37 @@ def test_int8_ties_to_even_and_rails(orc):
     assert r2["codes"].min() == 0 and r2["codes"].max() <= 255
 
 
+def test_int4_codes_are_nearest_level(orc):
+    """The 4-bit low tier ([DAMP] per-block asymmetric affine, b = 4): 16
+    levels, step fp16((max - min) / 15); every code is the nearest of the 16
+    levels (exhaustive), up to the FP32 rounding of the grid coordinate."""
+    rng = np.random.default_rng(11)
+    for trial in range(200):
+        n = [32, 128][trial % 2]
+        y = (rng.standard_normal(n) * 10.0 ** rng.uniform(-3, 2)).astype(np.float32)
+        r = orc.lowbit_block(y, 15)
+        s = np.float64(np.uint16(r["scale"]).view(np.float16))
+        z = np.float64(np.uint16(r["zero"]).view(np.float16))
+        assert abs(s * 15 - (y.max() - y.min())) <= 15 * 2 ** -11 * s + 2 ** -24 * 15
+        assert r["codes"].max() <= 15
+        levels = np.arange(16) * s + z
+        dist = np.abs(y[:, None].astype(np.float64) - levels[None, :])
+        got = dist[np.arange(n), r["codes"]]
+        assert np.all(got - dist.min(axis=1) <= 1e-5 * s + 1e-30), trial
+
+
+def test_int4_ties_to_even_and_rails(orc):
+    # a block spanning [0, 15] has step 1 and zero 0: the grid coordinate is y
+    y = np.zeros(32, np.float32)
+    y[0], y[1] = 0.0, 15.0
+    y[2:8] = [2.5, 3.5, 4.5, 0.5, 13.5, 14.5]
+    r = orc.lowbit_block(y, 15)
+    assert r["scale"] == np.float16(1.0).view(np.uint16)
+    assert list(r["codes"][2:8]) == [2, 4, 4, 0, 14, 14]
+    # the INT8 quantizer is the same block with 255 levels
+    np.testing.assert_array_equal(orc.lowbit_block(y * 17, 255)["codes"], orc.int8_block(y * 17)["codes"])
+
+
 def test_int8_constant_block(orc):
     y = np.full(32, 3.25, np.float32)
     r = orc.int8_block(y)

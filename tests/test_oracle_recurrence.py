@@ -94,7 +94,8 @@ def test_unit_key_beta_one_writes_v(orc):
         np.testing.assert_array_equal(S1[others], S0[0, 0][others])
 
 
-def test_damp_step_matches_fp64_brute_force(orc):
+@pytest.mark.parametrize("bits", [8, 4])
+def test_damp_step_matches_fp64_brute_force(orc, bits):
     """Teacher-forced: each step starts from the oracle's stored state; the
     FP64 reference dequantizes, runs the matrix-form update, re-applies the
     Hadamard and picks every code by exhaustive search.  Codes may differ
@@ -102,8 +103,9 @@ def test_damp_step_matches_fp64_brute_force(orc):
     FP32/FP64 gap of the recurrence); a block whose FP16 step or zero flips
     must sit within 1e-5 (relative) of an FP16 rounding midpoint."""
     d, H, k_hi, block = 16, 2, 4, 16
+    levels = (1 << bits) - 1
     w = synth.Workload("t", B=2, H=H, d=d, T=8, k_hi=k_hi, block=block, seed=5)
-    cfg = _cfg(orc, w)
+    cfg = _cfg(orc, w, low_bits=bits)
     rng = np.random.default_rng(3)
     perm = _rand_perm(rng, H, d)
     inp_all = synth.run_inputs(w, 0, w.T)
@@ -121,11 +123,11 @@ def test_damp_step_matches_fp64_brute_force(orc):
         for b in range(w.B):
             for h in range(H):
                 u = b * H + h
-                S = damp_dequant64(before[u * hb:(u + 1) * hb], d, k_hi, block, True)
+                S = damp_dequant64(before[u * hb:(u + 1) * hb], d, k_hi, block, True, bits)
                 k, q, v, a, beta = token_vectors(inp, 0, b, h, H, H, perm[h], True)
                 S, oo = dense_step(S, k, q, v, a, beta)
                 assert np.max(np.abs(o[0, b, h] - oo)) <= 1e-5 * (np.max(np.abs(oo)) + 1e-30)
-                f16rows, codes, sz = damp_head_sections(packed[u * hb:(u + 1) * hb], d, k_hi, block)
+                f16rows, codes, sz = damp_head_sections(packed[u * hb:(u + 1) * hb], d, k_hi, block, bits)
                 ref16 = S[d - k_hi:].astype(np.float16).view(np.uint16)
                 bad = f16rows != ref16
                 if bad.any():
@@ -137,12 +139,12 @@ def test_damp_step_matches_fp64_brute_force(orc):
                     mism += int(bad.sum())
                 R = S[:d - k_hi] @ Hn
                 for r in range(d - k_hi):
-                    c64, s64, z64, t64 = int8_nearest64(R[r])
+                    c64, s64, z64, t64 = int8_nearest64(R[r], levels)
                     s_o = f16_bits_to_f64(sz[r, 0, 0])
                     z_o = f16_bits_to_f64(sz[r, 0, 1])
                     if s_o != s64 or z_o != z64:
                         mid = lambda x: abs(abs(x) / np.spacing(np.float16(abs(x)), dtype=np.float16).astype(float) % 1 - 0.5)
-                        assert min(mid((R[r].max() - R[r].min()) / 255.0), mid(R[r].min())) < 1e-2
+                        assert min(mid((R[r].max() - R[r].min()) / levels), mid(R[r].min())) < 1e-2
                         continue
                     diff = codes[r].astype(int) != c64
                     if diff.any():
