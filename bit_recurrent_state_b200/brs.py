@@ -43,7 +43,7 @@ class Layout(ct.Structure):
                 ("storage", ct.c_int32), ("k_hi", ct.c_int32), ("block", ct.c_int32),
                 ("hadamard", ct.c_int32), ("decay_per_key", ct.c_int32),
                 ("avg_bits", ct.c_double), ("b_min", ct.c_int32), ("b_max", ct.c_int32),
-                ("budget_scope", ct.c_int32), ("persistence", ct.c_int32)]
+                ("budget_scope", ct.c_int32), ("persistence", ct.c_int32), ("low_bits", ct.c_int32)]
 
 
 class WriteBack(ct.Structure):
@@ -55,7 +55,7 @@ def layout_of(w, **override) -> Layout:
     f = dict(B=w.B, H=w.H, H_k=w.hk, d=w.d, storage=STORES[w.storage], k_hi=w.k_hi,
              block=w.block, hadamard=w.hadamard, decay_per_key=w.decay_per_key,
              avg_bits=w.avg_bits, b_min=w.b_min, b_max=w.b_max, budget_scope=1,
-             persistence=w.persistence)
+             persistence=w.persistence, low_bits=w.low_bits)
     f.update(override)
     return Layout(**f)
 

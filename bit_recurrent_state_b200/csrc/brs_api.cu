@@ -46,6 +46,8 @@ brs_status check_layout(const brs_layout* L) {
     if (L->k_hi < 0 || L->k_hi > L->d || (L->k_hi % 4)) return fail(BRS_EINVAL, "k_hi must be a multiple of 4 in [0, d]");
     if (!pow2(L->block) || L->block < 4 || L->block > L->d)
       return fail(BRS_EINVAL, "block must be a power of two in [4, d] (got %d)", L->block);
+    if (L->low_bits != 0 && L->low_bits != 8 && L->low_bits != 4)
+      return fail(BRS_EINVAL, "low_bits must be 8 (or 0) or 4 (got %d)", L->low_bits);
   } else if (L->storage == BRS_STORE_VARBIT) {
     if (L->hadamard) return fail(BRS_EUNSUPPORTED, "variable-width storage is stored without the Hadamard");
     if (L->b_min < 1 || L->b_max > 16 || L->b_min > L->b_max) return fail(BRS_EINVAL, "need 1 <= b_min <= b_max <= 16");
@@ -59,9 +61,12 @@ brs_status check_layout(const brs_layout* L) {
   return BRS_OK;
 }
 
+// width of the DAMP low tier: 8 unless the layout asks for 4
+int low_bits(const brs_layout* L) { return L->low_bits == 4 ? 4 : 8; }
+
 size_t damp_head_bytes(const brs_layout* L) {
   const size_t d = (size_t)L->d, kh = (size_t)L->k_hi;
-  return (d - kh) * d + kh * d * 2 + (d - kh) * (d / (size_t)L->block) * 4;
+  return (d - kh) * d * (size_t)low_bits(L) / 8 + kh * d * 2 + (d - kh) * (d / (size_t)L->block) * 4;
 }
 
 size_t head_bytes(const brs_layout* L) {
@@ -133,7 +138,7 @@ brs_status brs_state_pack(const brs_layout* L, const float* S, const int16_t* pe
     return fail(BRS_EALIGN, "device pointers must be 16-byte aligned");
   brs::PackArgs a{};
   a.B = L->B; a.H = L->H; a.d = L->d; a.storage = L->storage; a.k_hi = L->k_hi;
-  a.block = L->block; a.hadamard = L->hadamard; a.head_bytes = head_bytes(L);
+  a.block = L->block; a.hadamard = L->hadamard; a.low_bits = low_bits(L); a.head_bytes = head_bytes(L);
   a.hscale = hadamard_scale(L->d); a.S = S; a.perm = perm; a.packed = packed;
   a.flags = (uint32_t*)workspace;
   cudaError_t e = brs::launch_pack(a, (cudaStream_t)stream);
@@ -161,7 +166,7 @@ brs_status brs_state_unpack(const brs_layout* L, const void* packed, const int16
     return fail(BRS_EALIGN, "device pointers must be 16-byte aligned");
   brs::PackArgs a{};
   a.B = L->B; a.H = L->H; a.d = L->d; a.storage = L->storage; a.k_hi = L->k_hi;
-  a.block = L->block; a.hadamard = L->hadamard; a.head_bytes = head_bytes(L);
+  a.block = L->block; a.hadamard = L->hadamard; a.low_bits = low_bits(L); a.head_bytes = head_bytes(L);
   a.hscale = hadamard_scale(L->d); a.perm = perm; a.flags = (uint32_t*)workspace;
   cudaError_t e = brs::launch_unpack(a, S, packed, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "unpack launch");
@@ -229,6 +234,7 @@ brs_status brs_decode_step(const brs_layout* L, const brs_writeback* wb, int64_t
   a.q = q; a.k = k; a.v = v; a.beta = beta; a.decay = decay; a.o = o;
   a.flags = (uint32_t*)workspace;
   a.tx_extra = brs::starve_tx_bytes();
+  a.low_bits = L->storage == BRS_STORE_DAMP ? low_bits(L) : 8;
   const bool had = L->storage == BRS_STORE_DAMP && L->hadamard;
   cudaError_t e = brs::launch_decode(a, L->d, L->storage, had, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
@@ -280,6 +286,7 @@ brs_status brs_decode_step_deferred(const brs_layout* L, const brs_writeback* wb
   a.q = q; a.k = k; a.v = v; a.beta = beta; a.decay = decay; a.o = o;
   a.flags = (uint32_t*)workspace;
   a.s32 = (float*)state32; a.src32 = src32; a.dst32 = dst32;
+  a.low_bits = low_bits(L);
   cudaError_t e = (src32 || dst32) ? brs::launch_decode_deferred(a, L->d, L->hadamard != 0, (cudaStream_t)stream)
                                    : brs::launch_decode(a, L->d, L->storage, L->hadamard != 0, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
@@ -297,6 +304,7 @@ brs_status brs_chunk_prefill(const brs_layout* L, const brs_writeback* wb, int64
   if (L->storage != BRS_STORE_DAMP) return fail(BRS_EUNSUPPORTED, "chunked prefill is built for DAMP storage");
   if (!brs::prefill_supported(L->d, L->block, L->k_hi, wb->C))
     return fail(BRS_EUNSUPPORTED, "chunked prefill is built for d = 128, C = 64, block 128 or 32");
+  if (low_bits(L) != 8) return fail(BRS_EUNSUPPORTED, "chunked prefill is built for the INT8 low tier");
   if (wb->mode < 0 || wb->mode > 6) return fail(BRS_EINVAL, "unknown rounding mode %d", wb->mode);
   if (wb->mode >= BRS_ROUND_DIRECTION)
     return fail(BRS_EUNSUPPORTED, "direction and residual memory are not built for the prefill");
@@ -323,8 +331,8 @@ brs_status brs_chunk_prefill(const brs_layout* L, const brs_writeback* wb, int64
 
 size_t brs_prefill_workspace_bytes(const brs_layout* L) {
   if (check_layout(L) != BRS_OK) return 0;
-  if (L->storage != BRS_STORE_DAMP || L->d != 128) {
-    fail(BRS_EUNSUPPORTED, "chunked prefill is built for DAMP storage at d = 128");
+  if (L->storage != BRS_STORE_DAMP || L->d != 128 || low_bits(L) != 8) {
+    fail(BRS_EUNSUPPORTED, "chunked prefill is built for DAMP storage at d = 128 with the INT8 low tier");
     return 0;
   }
   ok();
@@ -410,6 +418,7 @@ brs_status brs_calibrate(const brs_layout* L, int Bc, int T, int every, double t
   brs::CalibArgs c{};
   c.B = Bc; c.H = L->H; c.d = L->d; c.block = L->block; c.hadamard = L->hadamard; c.k_hi = L->k_hi;
   c.T = T; c.nsamp = T / every; c.decay_per_key = L->decay_per_key; c.hscale = hadamard_scale(L->d);
+  c.levels = (float)((1 << low_bits(L)) - 1);
   c.tau = tau; c.S = states; c.err = (double*)(ws + cl.err); c.decay = decay; c.score = score;
   c.perm = perm_out; c.flags = (uint32_t*)ws;
   const size_t qk = (size_t)Bc * L->H_k * L->d, vv = (size_t)Bc * L->H * L->d, bh = (size_t)Bc * L->H;

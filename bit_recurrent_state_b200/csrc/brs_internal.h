@@ -33,6 +33,7 @@ struct DecodeArgs {
   // test hook (brs_test_starve_copies): bytes a head's copy barrier expects
   // beyond what its copies deliver (0 in normal use)
   uint32_t tx_extra = 0;
+  int low_bits = 8;              // DAMP low tier: 8 (INT8) or 4 (two codes per byte)
 };
 
 // the host thread's test-hook setting (brs_test_starve_copies)
@@ -46,6 +47,7 @@ bool decode_supported(int d, int block, int k_hi);
 
 struct CalibArgs {
   int B, H, d, block, hadamard, k_hi, T, nsamp, sample, decay_per_key;
+  float levels;                  // top code of the low tier: 255 (INT8) or 15 (INT4)
   float hscale;
   double tau;
   const float* S;                // [B][H][d][d] FP32 calibration states
@@ -64,6 +66,7 @@ cudaError_t launch_decode_cta(const DecodeArgs& a, bool had, cudaStream_t st);
 
 struct PackArgs {
   int B, H, d, storage, k_hi, block, hadamard;
+  int low_bits;                  // DAMP low tier: 8 or 4
   size_t head_bytes;
   float hscale;
   const float* S;                // [B][H][d][d] key-channel order

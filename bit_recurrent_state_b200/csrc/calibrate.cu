@@ -43,12 +43,12 @@ __global__ void calib_sample_kernel(const CalibArgs a) {
       if (y[j] > mx || (y[j] == mx && !signbit(y[j]))) mx = y[j];
     }
     if (!isfinite(mn) || !isfinite(mx)) raise_flag(a.flags, BRS_FLAG_NONFINITE);
-    const float s = f16_to_f32(f32_to_f16(__fdiv_rn(__fsub_rn(mx, mn), 255.0f)));
+    const float s = f16_to_f32(f32_to_f16(__fdiv_rn(__fsub_rn(mx, mn), a.levels)));
     const float z = f16_to_f32(f32_to_f16(mn));
     const float rcp = (s == 0.0f) ? 0.0f : __frcp_rn(s);
     for (int j = 0; j < a.block; ++j) {
       float c = 0.0f;
-      if (s != 0.0f) c = fminf(fmaxf(rintf(__fmul_rn(__fsub_rn(y[j], z), rcp)), 0.0f), 255.0f);
+      if (s != 0.0f) c = fminf(fmaxf(rintf(__fmul_rn(__fsub_rn(y[j], z), rcp)), 0.0f), a.levels);
       const double e = (double)y[j] - (double)__fmaf_rn(c, s, z);
       err = __dadd_rn(err, __dmul_rn(e, e));
     }

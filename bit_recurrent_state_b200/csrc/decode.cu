@@ -123,6 +123,42 @@ __device__ __forceinline__ void dequant_int8(float (&x)[C], uint32_t w, float s0
   }
 }
 
+// CPL codes of the low tier starting at byte p (the lane's first column):
+// LB = 8, one byte each; LB = 4, two to a byte (element e in bits 4 (e % 2)),
+// for CPL = 1 the lane's nibble (column parity nsh / 4) alone
+template <int C, int LB>
+__device__ __forceinline__ uint32_t ld_codes(const uint8_t* p, int nsh) {
+  if constexpr (LB == 8) {
+    if constexpr (C == 4) return __ldg((const uint32_t*)p);
+    else if constexpr (C == 2) return __ldg((const uint16_t*)p);
+    else return __ldg(p);
+  } else {
+    if constexpr (C == 4) return __ldg((const uint16_t*)p);
+    else if constexpr (C == 2) return __ldg(p);
+    else return ((uint32_t)__ldg(p) >> nsh) & 15u;
+  }
+}
+
+// dequantize CPL codes of either width: value = fmaf(code, scale, zero)
+template <int C, int LB>
+__device__ __forceinline__ void dequant_codes(float (&x)[C], uint32_t w, float s0, float s1, float z0,
+                                              float z1) {
+  if constexpr (LB == 8) {
+    dequant_int8<C>(x, w, s0, s1, z0, z1);
+  } else if constexpr (C == 1) {
+    const float c0 = __fsub_rn(__uint_as_float(0x4B000000u | (w & 15u)), kTwo23);
+    x[0] = __fmaf_rn(c0, s0, z0);
+  } else {
+#pragma unroll
+    for (int c = 0; c < C; c += 2) {
+      float c0 = __uint_as_float(0x4B000000u | ((w >> (4 * c)) & 15u));
+      float c1 = __uint_as_float(0x4B000000u | ((w >> (4 * c + 4)) & 15u));
+      sub2(c0, c1, c0, c1, kTwo23, kTwo23);
+      fma2(x[c], x[c + 1], c0, c1, s0, s1, z0, z1);
+    }
+  }
+}
+
 // Sylvester Hadamard of a D-vector held CPL values per lane (lane l holds
 // elements CPL*l ..), butterflies h = 1, 2, 4, ... then one scaling; every
 // output is the same single add or subtract as in the sequential
@@ -159,10 +195,12 @@ __device__ __forceinline__ uint32_t f16x2_overflow(uint32_t w) {
 // packed code byte of a float holding (code + 1.5*2^23)
 __device__ __forceinline__ uint32_t magic_byte(float m) { return __float_as_uint(m) & 0xffu; }
 
-template <int D, int STORE, bool HAD, int BLOCK, int MODE>
+template <int D, int STORE, bool HAD, int BLOCK, int MODE, int LB>
 __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const DecodeArgs a) {
   using G = WGeo<D>;
   constexpr int C = G::CPL, NRB = G::NRB;
+  constexpr int RB = D * LB / 8;                 // bytes of one low-tier code row
+  constexpr float LV = (float)((1 << LB) - 1);   // top code: 255 (INT8) or 15 (INT4)
   constexpr int NB = D / BLOCK;                  // blocks per row
   constexpr int GL = BLOCK / C;                  // lanes per block
   constexpr int V = 2 * NRB;                     // (min, max) entries per lane and batch
@@ -178,12 +216,13 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
   const int kh = h * a.Hk / a.H;
   const int nlo = (STORE == BRS_STORE_FP32) ? D : D - a.k_hi;   // INT8 rows 0..nlo-1
   const int col0 = C * lane;
+  const int cb0 = col0 * LB / 8, nsh = 4 * (col0 & 1);   // my first code byte; my nibble (LB = 4, CPL = 1)
   const uint8_t* hin = (const uint8_t*)a.packed_in + (size_t)head * a.head_bytes;
   uint8_t* hout = (uint8_t*)a.packed_out + (size_t)head * a.head_bytes;
-  const uint32_t* szin = (const uint32_t*)(hin + (size_t)nlo * D + (size_t)a.k_hi * D * 2);
-  uint32_t* szout = (uint32_t*)(hout + (size_t)nlo * D + (size_t)a.k_hi * D * 2);
-  const uint8_t* f16in = hin + (size_t)nlo * D;
-  uint16_t* f16out = (uint16_t*)(hout + (size_t)nlo * D);
+  const uint32_t* szin = (const uint32_t*)(hin + (size_t)nlo * RB + (size_t)a.k_hi * D * 2);
+  uint32_t* szout = (uint32_t*)(hout + (size_t)nlo * RB + (size_t)a.k_hi * D * 2);
+  const uint8_t* f16in = hin + (size_t)nlo * RB;
+  uint16_t* f16out = (uint16_t*)(hout + (size_t)nlo * RB);
   uint16_t* auxb = (MODE == BRS_ROUND_ERRFEEDBACK) ? (uint16_t*)a.aux + (size_t)head * nlo * D : nullptr;
   // direction memory: 2-bit counters, four to a byte in column order
   uint8_t* dmb = (MODE == BRS_ROUND_DIRECTION) ? (uint8_t*)a.aux + (size_t)head * nlo * (D / 4) : nullptr;
@@ -238,17 +277,14 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
       }
     } else {
       if (i < nlo) {
-        uint32_t w;
-        if constexpr (C == 4) w = __ldg((const uint32_t*)(hin + (size_t)i * D + col0));
-        else if constexpr (C == 2) w = __ldg((const uint16_t*)(hin + (size_t)i * D + col0));
-        else w = __ldg(hin + (size_t)i * D + col0);
+        const uint32_t w = ld_codes<C, LB>(hin + (size_t)i * RB + cb0, nsh);
         if constexpr (NB == 1) {
           const float4 g = sm.rs[i].sz;
-          dequant_int8<C>(x, w, g.x, g.y, g.z, g.w);
+          dequant_codes<C, LB>(x, w, g.x, g.y, g.z, g.w);
         } else {
           const uint32_t szw = __ldg(szin + i * NB + col0 / BLOCK);
           const float sv = f16_to_f32((uint16_t)(szw & 0xffffu)), zv = f16_to_f32((uint16_t)(szw >> 16));
-          dequant_int8<C>(x, w, sv, sv, zv, zv);
+          dequant_codes<C, LB>(x, w, sv, sv, zv, zv);
         }
       } else {
         const uint16_t* src = (const uint16_t*)f16in + (size_t)(i - nlo) * D + col0;
@@ -339,17 +375,15 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
     // chunks of CH = NRB rows (nlo is a multiple of NRB), two in flight
     constexpr int CH = NRB;
     uint32_t cw[2][CH], sw[2][(NB > 1) ? CH : 1];
-    const uint8_t* crow = hin + col0;
+    const uint8_t* crow = hin + cb0;
     const uint32_t* srow = szin + col0 / BLOCK;
     auto fetch = [&](int buf) {
 #pragma unroll
       for (int r = 0; r < CH; ++r) {
-        if constexpr (C == 4) cw[buf][r] = __ldg((const uint32_t*)(crow + r * D));
-        else if constexpr (C == 2) cw[buf][r] = __ldg((const uint16_t*)(crow + r * D));
-        else cw[buf][r] = __ldg(crow + r * D);
+        cw[buf][r] = ld_codes<C, LB>(crow + r * RB, nsh);
         if constexpr (NB > 1) sw[buf][r] = __ldg(srow + r * NB);
       }
-      crow += CH * D;
+      crow += CH * RB;
       srow += CH * NB;
     };
     auto consume = [&](int buf, int i0) {
@@ -358,11 +392,11 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
         float x[C];
         const RowScal rsc = sm.rs[i0 + r];
         if constexpr (NB == 1) {
-          dequant_int8<C>(x, cw[buf][r], rsc.sz.x, rsc.sz.y, rsc.sz.z, rsc.sz.w);
+          dequant_codes<C, LB>(x, cw[buf][r], rsc.sz.x, rsc.sz.y, rsc.sz.z, rsc.sz.w);
         } else {
           const float sv = f16_to_f32((uint16_t)(sw[buf][r] & 0xffffu));
           const float zv = f16_to_f32((uint16_t)(sw[buf][r] >> 16));
-          dequant_int8<C>(x, cw[buf][r], sv, sv, zv, zv);
+          dequant_codes<C, LB>(x, cw[buf][r], sv, sv, zv, zv);
         }
         v_scale<C>(x, rsc.ka.z, rsc.ka.w);
         feed(i0 + r, rsc.ka.x, rsc.ka.y, x, u1);
@@ -408,17 +442,15 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
   tree.n = 0;
   // the next batch's rows are fetched while this batch is requantized
   uint32_t pw[NRB], ps[(NB > 1) ? NRB : 1];
-  const uint8_t* prow = hin + col0;
+  const uint8_t* prow = hin + cb0;
   const uint32_t* psrow = szin + col0 / BLOCK;
   auto prefetch = [&]() {
 #pragma unroll
     for (int r = 0; r < NRB; ++r) {
-      if constexpr (C == 4) pw[r] = __ldg((const uint32_t*)(prow + r * D));
-      else if constexpr (C == 2) pw[r] = __ldg((const uint16_t*)(prow + r * D));
-      else pw[r] = __ldg(prow + r * D);
+      pw[r] = ld_codes<C, LB>(prow + r * RB, nsh);
       if constexpr (NB > 1) ps[r] = __ldg(psrow + r * NB);
     }
-    prow += NRB * D;
+    prow += NRB * RB;
     psrow += NRB * NB;
   };
   if (STORE != BRS_STORE_FP32 && !src32 && nlo > 0) prefetch();
@@ -434,11 +466,11 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
       for (int r = 0; r < NRB; ++r) {
         if constexpr (NB == 1) {
           const float4 g = sm.rs[i0 + r].sz;
-          dequant_int8<C>(x[r], pw[r], g.x, g.y, g.z, g.w);
+          dequant_codes<C, LB>(x[r], pw[r], g.x, g.y, g.z, g.w);
           if constexpr (MODE == kModeResidual) sp[r] = g.x;
         } else {
           const float sv = f16_to_f32((uint16_t)(ps[r] & 0xffffu)), zv = f16_to_f32((uint16_t)(ps[r] >> 16));
-          dequant_int8<C>(x[r], pw[r], sv, sv, zv, zv);
+          dequant_codes<C, LB>(x[r], pw[r], sv, sv, zv, zv);
           if constexpr (MODE == kModeResidual) sp[r] = sv;
         }
         if constexpr (MODE == BRS_ROUND_DIRECTION) {
@@ -614,18 +646,18 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
       }
       // the grid of each (row, block), one division per lane; ok = the
       // block's extreme grid coordinates (the same monotone FP32 operations
-      // as its elements') round into [0, 255]: no clip needed
+      // as its elements') round into [0, LV]: no clip needed
       bool ok = true;
       if (param_lane) {
         const int i = i0 + prow;
         if (!isfinite(mnv) || !isfinite(mxv)) raise_flag(a.flags, BRS_FLAG_NONFINITE);
-        const uint16_t sh = f32_to_f16(__fdiv_rn(__fsub_rn(mxv, mnv), 255.0f));
+        const uint16_t sh = f32_to_f16(__fdiv_rn(__fsub_rn(mxv, mnv), LV));
         const uint16_t zh = f32_to_f16(mnv);
         if (f16_inf_or_nan(sh) || f16_inf_or_nan(zh)) raise_flag(a.flags, BRS_FLAG_OVERFLOW);
         const float s = f16_to_f32(sh), z = f16_to_f32(zh);
         const float rcp = (s == 0.0f) ? 0.0f : __frcp_rn(s);
         const float tlo = __fmul_rn(__fsub_rn(mnv, z), rcp), thi = __fmul_rn(__fsub_rn(mxv, z), rcp);
-        ok = (tlo >= -0.5f) && (thi < 255.5f);
+        ok = (tlo >= -0.5f) && (thi < LV + 0.5f);
         QPrm p;
         p.z = z; p.rcp = rcp; p.s = s; p.pad = 0;
         sm.prm[prow][blk] = p;
@@ -633,7 +665,7 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
       }
       const bool fast = (MODE != BRS_ROUND_STOCHASTIC) && __all_sync(0xffffffffu, ok);
       __syncwarp();
-      // ---- codes: clamp(round((y - zero) * (1/scale)), 0, 255); a zero
+      // ---- codes: clamp(round((y - zero) * (1/scale)), 0, LV); a zero
       // scale has 1/scale = 0, so every code of the block is 0
 #pragma unroll
       for (int r = 0; r < NRB; ++r) {
@@ -660,7 +692,7 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
             for (int c = 0; c < C; ++c) tq[c] = sr_round(tq[c], words[(e0 + c) & 3] >> 8);
           }
 #pragma unroll
-          for (int c = 0; c < C; ++c) tq[c] = fminf(fmaxf(tq[c], 0.0f), 255.0f);
+          for (int c = 0; c < C; ++c) tq[c] = fminf(fmaxf(tq[c], 0.0f), LV);
         }
         // nearest integer (ties to even): the low byte of t + 1.5*2^23; the
         // paired add is written t * one + magic with one = 1 read at run
@@ -675,7 +707,7 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
         if constexpr (MODE == BRS_ROUND_DIRECTION) {
           // votes of the proposed changes y - xp inside (scale/8, scale/2);
           // a counter at +-2 moves the nearest code one level (clipped to
-          // [0, 255]) and is reset.  The lanes of one counter byte merge
+          // [0, LV]) and is reset.  The lanes of one counter byte merge
           // their fields before one of them stores it.
           uint8_t* dmp = dmb + (size_t)i * (D / 4) + col0 / 4;
           const uint32_t old = *dmp;
@@ -691,7 +723,7 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
             if (ad > lo && ad < hi) m += (dl > 0.0f) ? 1 : -1;
             if (m >= 2 || m <= -2) {
               const uint32_t mb = __float_as_uint(mq[c]);
-              const int code = min(max((int)(mb & 0xffu) + (m > 0 ? 1 : -1), 0), 255);
+              const int code = min(max((int)(mb & 0xffu) + (m > 0 ? 1 : -1), 0), (int)LV);
               mq[c] = __uint_as_float((mb & ~0xffu) | (uint32_t)code);
               m = 0;
             }
@@ -701,8 +733,22 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
           if constexpr (C == 1) nb |= __shfl_xor_sync(0xffffffffu, nb, 2);
           if ((col0 & 3) == 0) *dmp = (uint8_t)nb;
         }
-        uint8_t* dst = hout + (size_t)i * D + col0;
-        if constexpr (C == 4) {
+        uint8_t* dst = hout + (size_t)i * RB + cb0;
+        if constexpr (LB == 4) {
+          // codes 0..15 in the low nibble of each magic float's byte
+          uint32_t nbl = 0;
+#pragma unroll
+          for (int c = 0; c < C; ++c) nbl |= (magic_byte(mq[c]) & 15u) << (4 * c);
+          if constexpr (C == 4) {
+            *(uint16_t*)dst = (uint16_t)nbl;
+          } else if constexpr (C == 2) {
+            *dst = (uint8_t)nbl;
+          } else {
+            nbl <<= nsh;
+            nbl |= __shfl_xor_sync(0xffffffffu, nbl, 1);
+            if ((col0 & 1) == 0) *dst = (uint8_t)nbl;
+          }
+        } else if constexpr (C == 4) {
           *(uint32_t*)dst = __byte_perm(__byte_perm(__float_as_uint(mq[0]), __float_as_uint(mq[1]), 0x0040u),
                                         __byte_perm(__float_as_uint(mq[2]), __float_as_uint(mq[3]), 0x0040u), 0x5410u);
         } else if constexpr (C == 2) {
@@ -770,31 +816,38 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 8) decode_warp_kernel(const
   else *od = ov[0];
 }
 
-template <int D, int BLOCK, int MODE>
+template <int D, int BLOCK, int MODE, int LB = 8>
 static cudaError_t launch_dbm(const DecodeArgs& a, int store, bool had, cudaStream_t st) {
   const int heads = a.B * a.H;
   const dim3 grid((heads + kWarpsPerCta - 1) / kWarpsPerCta), block(32 * kWarpsPerCta);
   if (store == BRS_STORE_FP32)
-    decode_warp_kernel<D, BRS_STORE_FP32, false, D, BRS_ROUND_NEAREST><<<grid, block, 0, st>>>(a);
+    decode_warp_kernel<D, BRS_STORE_FP32, false, D, BRS_ROUND_NEAREST, 8><<<grid, block, 0, st>>>(a);
   else if (had)
-    decode_warp_kernel<D, BRS_STORE_DAMP, true, BLOCK, MODE><<<grid, block, 0, st>>>(a);
+    decode_warp_kernel<D, BRS_STORE_DAMP, true, BLOCK, MODE, LB><<<grid, block, 0, st>>>(a);
   else
-    decode_warp_kernel<D, BRS_STORE_DAMP, false, BLOCK, MODE><<<grid, block, 0, st>>>(a);
+    decode_warp_kernel<D, BRS_STORE_DAMP, false, BLOCK, MODE, LB><<<grid, block, 0, st>>>(a);
   return cudaGetLastError();
 }
 
-template <int D, int BLOCK>
-static cudaError_t launch_db(const DecodeArgs& a, int store, bool had, cudaStream_t st) {
+template <int D, int BLOCK, int LB>
+static cudaError_t launch_dbl(const DecodeArgs& a, int store, bool had, cudaStream_t st) {
   switch (a.mode) {
-    case BRS_ROUND_NEAREST: return launch_dbm<D, BLOCK, BRS_ROUND_NEAREST>(a, store, had, st);
-    case BRS_ROUND_STOCHASTIC: return launch_dbm<D, BLOCK, BRS_ROUND_STOCHASTIC>(a, store, had, st);
-    case BRS_ROUND_ERRFEEDBACK: return launch_dbm<D, BLOCK, BRS_ROUND_ERRFEEDBACK>(a, store, had, st);
-    case BRS_ROUND_DIRECTION: return launch_dbm<D, BLOCK, BRS_ROUND_DIRECTION>(a, store, had, st);
+    case BRS_ROUND_NEAREST: return launch_dbm<D, BLOCK, BRS_ROUND_NEAREST, LB>(a, store, had, st);
+    case BRS_ROUND_STOCHASTIC: return launch_dbm<D, BLOCK, BRS_ROUND_STOCHASTIC, LB>(a, store, had, st);
+    case BRS_ROUND_ERRFEEDBACK: return launch_dbm<D, BLOCK, BRS_ROUND_ERRFEEDBACK, LB>(a, store, had, st);
+    case BRS_ROUND_DIRECTION: return launch_dbm<D, BLOCK, BRS_ROUND_DIRECTION, LB>(a, store, had, st);
     case BRS_ROUND_RESIDUAL2:
     case BRS_ROUND_RESIDUAL3:
-    case BRS_ROUND_RESIDUAL4: return launch_dbm<D, BLOCK, kModeResidual>(a, store, had, st);
+    case BRS_ROUND_RESIDUAL4: return launch_dbm<D, BLOCK, kModeResidual, LB>(a, store, had, st);
   }
   return cudaErrorInvalidValue;
+}
+
+// low tier width: 8 (INT8) or 4 (two codes per byte)
+template <int D, int BLOCK>
+static cudaError_t launch_db(const DecodeArgs& a, int store, bool had, cudaStream_t st) {
+  if (a.low_bits == 4) return launch_dbl<D, BLOCK, 4>(a, store, had, st);
+  return launch_dbl<D, BLOCK, 8>(a, store, had, st);
 }
 
 cudaError_t launch_decode_deferred(const DecodeArgs& a, int d, bool had, cudaStream_t st) {
@@ -824,7 +877,7 @@ cudaError_t launch_decode(const DecodeArgs& a, int d, int store, bool had, cudaS
     }
     return cudaErrorInvalidValue;
   }
-  if (decode_cta_supported(d, store, a.block, a.k_hi, a.mode)) return launch_decode_cta(a, had, st);
+  if (a.low_bits == 8 && decode_cta_supported(d, store, a.block, a.k_hi, a.mode)) return launch_decode_cta(a, had, st);
   if (d == 128 && a.block == 128) return launch_db<128, 128>(a, store, had, st);
   if (d == 128 && a.block == 32) return launch_db<128, 32>(a, store, had, st);
   if (d == 64 && a.block == 64) return launch_db<64, 64>(a, store, had, st);

@@ -50,6 +50,7 @@ class Workload:
     b_max: int = 8
     C: int = 1
     persistence: int = 0              # variable-width cost weight (0 Gamma_hat, 1 w^(1), 2 h^(C))
+    low_bits: int = 8                 # DAMP low tier: 8 (INT8) or 4 (two codes per byte)
     mode: str = "nearest"          # "nearest" | "stochastic" | "errfeedback" | "direction"
     seed: int = 0
 

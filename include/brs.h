@@ -51,6 +51,14 @@
  *                                                zero).
  *                    Stored row i holds key channel perm[h][i] (the
  *                    protected channels are the last k_hi entries).
+ *                    With low_bits = 4 ([DAMP] Key Points, b = 4) the code
+ *                    rows hold two codes per byte ((d-k_hi)*d/2 bytes;
+ *                    element e of a row in bits 4 (e % 2) of byte e/2),
+ *                    codes run 0..15 and the scale divides the block's
+ *                    range by 15; the rest is unchanged.  Pack, unpack,
+ *                    calibration and brs_decode_step accept it; the
+ *                    deferred, no-allocation and prefill paths return
+ *                    BRS_EUNSUPPORTED.
  *                    Error-feedback residuals: f16 [B][H][d-k_hi][d].
  *   BRS_STORE_VARBIT [LB] State bit allocation, Allocation units, Levels and
  *                    storage.  Sections, each starting on a 256-byte
@@ -161,6 +169,8 @@ typedef struct {
                             Choice of persistence factor): 0 = the erasure
                             rate Gamma_hat, 1 = DAMP's uncapped w^(1) =
                             1/(1 - e^-2s), 2 = h^(C) = 1/(1 - e^-2Cs)           */
+  int32_t low_bits;      /* DAMP: width b of the low tier, 8 (0 reads as 8) or
+                            4 ([DAMP] Key Points: an INT4 low tier b = 4)      */
 } brs_layout;
 
 typedef struct {

@@ -17,6 +17,7 @@ def oracle_cfg(w: synth.Workload) -> O.Config:
     return O.Config(B=w.B, H=w.H, Hk=w.hk, d=w.d, storage=STORE[w.storage], k_hi=w.k_hi,
                     block=w.block, hadamard=w.hadamard, decay_per_key=w.decay_per_key,
                     avg_bits=w.avg_bits, b_min=w.b_min, b_max=w.b_max, persistence=w.persistence,
+                    low_bits=w.low_bits,
                     domain=O.DOMAIN_MIXED if w.storage == "damp" else O.DOMAIN_CANONICAL)
 
 

@@ -34,6 +34,11 @@ def test_host_only_calls_without_gpu():
     assert brs.state_bytes(brs.layout_of(w))[0] == 16896 * 256 * 32
     with pytest.raises(brs.BrsError):
         brs.state_bytes(brs.layout_of(w, H_k=5))
+    # the 4-bit low tier: 112 code rows of 64 bytes, the same FP16 rows and grid
+    w4 = synth.WORKLOADS["kda_decode"].with_(low_bits=4)
+    n4, aux4, _, _ = brs.state_bytes(brs.layout_of(w4))
+    assert n4 == (112 * 64 + 16 * 128 * 2 + 112 * 4) * 64 * 32 and aux4 == aux
+    assert brs.state_bytes(brs.layout_of(w4, low_bits=0))[0] == 18880 * 64 * 32   # 0 reads as 8
 
 
 def test_prefill_workspace_size():
@@ -45,6 +50,9 @@ def test_prefill_workspace_size():
     assert brs.prefill_workspace_bytes(brs.layout_of(w)) == 256 + 8 * 32 * 128 * 128 * 4
     with pytest.raises(brs.BrsError) as e:
         brs.prefill_workspace_bytes(brs.layout_of(synth.WORKLOADS["kda_tiny"]))
+    assert e.value.status == brs.EUNSUPPORTED
+    with pytest.raises(brs.BrsError) as e:                 # the prefill keeps the INT8 low tier
+        brs.prefill_workspace_bytes(brs.layout_of(w, low_bits=4))
     assert e.value.status == brs.EUNSUPPORTED
 
 
@@ -221,6 +229,7 @@ def test_layout_and_conversion_argument_errors():
     assert size_status(block=48) == brs.EINVAL             # power of two
     assert size_status(block=256) == brs.EINVAL            # at most d
     assert size_status(B=0) == brs.EINVAL
+    assert size_status(low_bits=5) == brs.EINVAL           # 8 (or 0) or 4
     wv = synth.WORKLOADS["varbit_decode"]
 
     def vsize_status(**kw):

@@ -54,6 +54,8 @@ def _compare(perm_g, score_g, perm_o, score_o, k_hi):
     ("kda64_b16_nohad", dict(B=1, H=3, d=64, k_hi=8, block=16, hadamard=0), 3, 40, 8),
     ("gdn128", dict(B=1, H=4, Hk=2, d=128, k_hi=16, block=128, decay_per_key=0), 4, 48, 8),
     ("kda128_every5", dict(B=1, H=2, d=128, k_hi=24, block=32), 2, 33, 5),
+    ("kda128_int4", dict(B=1, H=2, d=128, k_hi=16, block=32, low_bits=4), 2, 24, 8),
+    ("kda32_int4_nohad", dict(B=1, H=2, d=32, k_hi=4, block=16, hadamard=0, low_bits=4), 3, 24, 6),
 ])
 def test_small_configs(name, kw, Bc, T, every):
     w = synth.Workload(name, T=1, seed=11, **kw)

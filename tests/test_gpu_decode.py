@@ -101,6 +101,23 @@ def test_kda_tiny_full_trajectory():
     ("gdn128_rm2", dict(B=3, H=4, Hk=2, d=128, k_hi=0, block=128, decay_per_key=0, mode="residual2")),
     ("fp32_64", dict(B=2, H=3, d=64, storage="fp32")),
     ("fp32_gdn128", dict(B=2, H=4, Hk=2, d=128, storage="fp32", decay_per_key=0)),
+    # the 4-bit low tier (two codes per byte, 16 levels per block)
+    ("kda128_int4_ragged", dict(B=3, H=5, d=128, k_hi=16, block=128, low_bits=4)),
+    ("kda128_b32_int4_sr", dict(B=2, H=2, d=128, k_hi=16, block=32, mode="stochastic", low_bits=4)),
+    ("kda128_int4_ef", dict(B=2, H=3, d=128, k_hi=16, block=128, mode="errfeedback", low_bits=4)),
+    ("kda128_b32_int4_dm", dict(B=2, H=2, d=128, k_hi=16, block=32, mode="direction", low_bits=4)),
+    ("kda128_int4_rm4", dict(B=2, H=3, d=128, k_hi=16, block=128, mode="residual4", low_bits=4)),
+    ("kda64_int4_khi16", dict(B=2, H=3, d=64, k_hi=16, block=64, low_bits=4)),
+    ("kda64_int4_ef", dict(B=2, H=3, d=64, k_hi=8, block=64, mode="errfeedback", low_bits=4)),
+    ("kda32_int4", dict(B=2, H=2, d=32, k_hi=4, block=32, low_bits=4)),
+    ("kda32_nohad_int4_sr", dict(B=2, H=2, d=32, k_hi=4, block=32, hadamard=0, mode="stochastic",
+                                 low_bits=4)),
+    ("kda32_int4_dm", dict(B=2, H=2, d=32, k_hi=8, block=32, mode="direction", low_bits=4)),
+    ("kda32_nohad_int4_rm3", dict(B=2, H=2, d=32, k_hi=4, block=32, hadamard=0, mode="residual3",
+                                  low_bits=4)),
+    ("gdn128_int4", dict(B=3, H=4, Hk=2, d=128, k_hi=0, block=128, decay_per_key=0, low_bits=4)),
+    ("gdn128_int4_rm2", dict(B=3, H=4, Hk=2, d=128, k_hi=0, block=128, decay_per_key=0, mode="residual2",
+                             low_bits=4)),
 ])
 def test_small_configs_bit_exact(name, kw):
     w = synth.Workload(name, T=12, seed=7, **kw)
@@ -127,12 +144,25 @@ def test_kda_decode_aux_memory_full_size_sampled(mode):
         np.testing.assert_array_equal(ag[units[0] * nel: units[1] * nel], ao[units[0] * nel: units[1] * nel])
 
 
-def test_unpack_matches_oracle():
+def test_kda_decode_int4_full_size_sampled():
+    """The 4-bit low tier at the KDA decode size (B=64, H=32, d=128, k_hi=16,
+    block 128; the general kernel) for 16 tokens from a nonzero state: codes,
+    FP16 rows and grids of 64 of the 2048 heads match the oracle."""
+    import dataclasses
+    w = dataclasses.replace(synth.WORKLOADS["kda_decode"], low_bits=4)
+    perm = random_perm(w, seed=8)
+    units = (1200, 1264)
+    steps = _run_both(w, 16, perm=perm, units=units, init_scale=0.05)
+    _compare(w, steps, units=units)
+
+
+@pytest.mark.parametrize("low_bits", [8, 4])
+def test_unpack_matches_oracle(low_bits):
     import torch
     from bit_recurrent_state_b200 import brs
     from bit_recurrent_state_b200.state import LayerState
     from oracle import oracle as O
-    w = synth.Workload("u", B=2, H=3, d=128, T=1, k_hi=16, block=32)
+    w = synth.Workload("u", B=2, H=3, d=128, T=1, k_hi=16, block=32, low_bits=low_bits)
     perm = random_perm(w, seed=9)
     cfg = oracle_cfg(w)
     S0 = np.random.default_rng(4).standard_normal((w.B, w.H, w.d, w.d)).astype(np.float32)

@@ -69,6 +69,8 @@ def _run(w, C, T, perm=None, units=None, init_scale=0.05):
     ("kda64_c3", 3, dict(B=2, H=3, d=64, k_hi=8, block=64)),
     ("kda32_nohad_c2", 2, dict(B=2, H=2, d=32, k_hi=4, block=32, hadamard=0)),
     ("gdn128_c4", 4, dict(B=3, H=4, Hk=2, d=128, k_hi=0, block=128, decay_per_key=0)),
+    ("kda128_int4_c4", 4, dict(B=2, H=3, d=128, k_hi=16, block=128, low_bits=4)),
+    ("kda32_int4_ef_c3", 3, dict(B=2, H=2, d=32, k_hi=4, block=32, mode="errfeedback", low_bits=4)),
 ])
 def test_deferred_small_bit_exact(name, C, kw):
     w = synth.Workload(name, T=2 * C, seed=11, **kw)
