@@ -5,9 +5,9 @@
 //
 // Source: DAMP summary, Key Points > Implementation (a permutation per head
 // places the protected channels contiguously; the low tier is INT8 after a
-// Hadamard along the value axis; the INT4 low tier b = 4) and Data &
-// Methods > Quantization & calibration details (per-block asymmetric affine
-// INT8).
+// Hadamard along the value axis) and Data & Methods > Quantization &
+// calibration details (per-block asymmetric affine quantization with
+// b = 8 or b = 4).
 #include <cuda_runtime.h>
 #include <cstdint>
 

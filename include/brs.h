@@ -51,7 +51,7 @@
  *                                                zero).
  *                    Stored row i holds key channel perm[h][i] (the
  *                    protected channels are the last k_hi entries).
- *                    With low_bits = 4 ([DAMP] Key Points, b = 4) the code
+ *                    With low_bits = 4 (b = 4 of the same section) the code
  *                    rows hold two codes per byte ((d-k_hi)*d/2 bytes;
  *                    element e of a row in bits 4 (e % 2) of byte e/2),
  *                    codes run 0..15 and the scale divides the block's
@@ -170,7 +170,8 @@ typedef struct {
                             rate Gamma_hat, 1 = DAMP's uncapped w^(1) =
                             1/(1 - e^-2s), 2 = h^(C) = 1/(1 - e^-2Cs)           */
   int32_t low_bits;      /* DAMP: width b of the low tier, 8 (0 reads as 8) or
-                            4 ([DAMP] Key Points: an INT4 low tier b = 4)      */
+                            4 ([DAMP] Data & Methods > Quantization &
+                            calibration details: b = 8 or b = 4)               */
 } brs_layout;
 
 typedef struct {
