@@ -324,6 +324,17 @@ int orc_int8_block_rm(const float* y, int n, int kbits, float sprev, int8_t* m_i
 int orc_varbit_row(const float* x, int n, int bw, int mode, uint64_t seed, int64_t step, int h,
                    int b, int elem0, uint16_t* e_inout, int32_t* q_out, uint16_t* delta_h,
                    int* m_star, float* t_out) {
+  return orc_varbit_group(x, n, bw, mode, seed, step, h, b, elem0, 1, e_inout, q_out, delta_h,
+                          m_star, t_out);
+}
+
+/* The same quantizer on any scale group: a row of a row unit, or one block
+ * of 32 key channels of one column of a head unit ([LB] Allocation units:
+ * scales per block of 32 key channels).  Only the stochastic-rounding
+ * element index depends on where the group sits in the head. */
+int orc_varbit_group(const float* x, int n, int bw, int mode, uint64_t seed, int64_t step, int h,
+                     int b, int elem0, int estride, uint16_t* e_inout, int32_t* q_out,
+                     uint16_t* delta_h, int* m_star, float* t_out) {
   int flags = 0;
   int nl = (1 << (bw - 1)) - 1;
   float fnl = (float)nl;
@@ -356,7 +367,7 @@ int orc_varbit_row(const float* x, int n, int bw, int mode, uint64_t seed, int64
       float t = tgt[j] * inv1;
       int u;
       if (mode == ORC_ROUND_STOCHASTIC) {
-        float c = sr_round((t + 1.0f) * 0.5f, sr_bits24(seed, step, h, b, elem0 + j));
+        float c = sr_round((t + 1.0f) * 0.5f, sr_bits24(seed, step, h, b, elem0 + j * estride));
         if (c < 0.0f) c = 0.0f;
         if (c > 1.0f) c = 1.0f;
         if (!(c == c)) c = 0.0f;
@@ -424,7 +435,7 @@ int orc_varbit_row(const float* x, int n, int bw, int mode, uint64_t seed, int64
     if (ok) {
       t = tgt[j] * inv;
       if (mode == ORC_ROUND_STOCHASTIC)
-        qf = sr_round(t, sr_bits24(seed, step, h, b, elem0 + j));
+        qf = sr_round(t, sr_bits24(seed, step, h, b, elem0 + j * estride));
       else
         qf = nearbyintf(t);
       if (qf < -fnl) qf = -fnl;
@@ -602,14 +613,24 @@ typedef struct {
   size_t payload_per_seq, off_scale, off_width, off_offsets, total;
 } vb_sections;
 
+/* Row units: one FP16 step, width and offset per row.  Head units ([LB]
+ * Allocation units, per-head decay): one width and offset per head, one
+ * FP16 step per (block of 32 key channels, column). */
 static vb_sections varbit_sections(const orc_layout* L) {
   vb_sections s;
-  size_t rows = (size_t)L->H * (size_t)L->d;
+  size_t rows = (size_t)L->H * (size_t)L->d, B = (size_t)L->B;
   s.payload_per_seq = (size_t)((double)(L->d / 8) * L->avg_bits * (double)rows);
-  s.off_scale = round256(s.payload_per_seq * (size_t)L->B);
-  s.off_width = s.off_scale + round256(rows * (size_t)L->B * 2);
-  s.off_offsets = s.off_width + round256(rows * (size_t)L->B);
-  s.total = s.off_offsets + round256((rows + 1) * (size_t)L->B * 4);
+  s.off_scale = round256(s.payload_per_seq * B);
+  if (L->storage == ORC_STORE_VARBIT_HEAD) {
+    size_t H = (size_t)L->H, d = (size_t)L->d;
+    s.off_width = s.off_scale + round256(B * H * (d / 32) * d * 2);
+    s.off_offsets = s.off_width + round256(B * H);
+    s.total = s.off_offsets + round256(B * (H + 1) * 4);
+    return s;
+  }
+  s.off_width = s.off_scale + round256(rows * B * 2);
+  s.off_offsets = s.off_width + round256(rows * B);
+  s.total = s.off_offsets + round256((rows + 1) * B * 4);
   return s;
 }
 
@@ -640,6 +661,8 @@ double orc_bits_per_value(const orc_layout* L) {
   if (L->storage == ORC_STORE_FP32) return 32.0;
   if (L->storage == ORC_STORE_DAMP)
     return (kh * d * 16.0 + (d - kh) * d * (double)low_bits(L) + (d - kh) * (d / L->block) * 32.0) / (d * d);
+  if (L->storage == ORC_STORE_VARBIT_HEAD)   /* 16-bit step per 32 values; one width per head */
+    return L->avg_bits + 16.0 / 32.0 + (L->b_max > 8 ? 4.0 : 3.0) / (d * d);
   return L->avg_bits + (16.0 + 3.0) / d;
 }
 
@@ -1015,6 +1038,71 @@ static void varbit_load_seq(const orc_layout* L, const uint8_t* packed, int b, f
   }
 }
 
+/* Head units: element (i, j) of head h at bit (i d + j) w_h of the head's
+ * payload; value = (u - n) * step of (block i / 32, column j). */
+static void varbit_head_load_seq(const orc_layout* L, const uint8_t* packed, int b, float* S) {
+  vb_sections sec = varbit_sections(L);
+  int d = L->d, H = L->H, nbk = d / 32;
+  const uint8_t* pay = packed + (size_t)b * sec.payload_per_seq;
+  const uint16_t* sc = (const uint16_t*)(packed + sec.off_scale) + (size_t)b * H * nbk * d;
+  const uint8_t* wd = packed + sec.off_width + (size_t)b * H;
+  const uint32_t* of = (const uint32_t*)(packed + sec.off_offsets) + (size_t)b * (H + 1);
+  for (int h = 0; h < H; ++h) {
+    int bw = wd[h];
+    int nl = (1 << (bw - 1)) - 1;
+    for (int i = 0; i < d; ++i)
+      for (int j = 0; j < d; ++j) {
+        uint32_t u = get_bits(pay + of[h], ((size_t)i * d + j) * bw, bw);
+        float D = orc_f32_from_f16(sc[((size_t)h * nbk + i / 32) * d + j]);
+        S[((size_t)h * d + i) * d + j] = (float)((int)u - nl) * D;
+      }
+  }
+}
+
+/* Quantize every head of sequence b with widths bits[H]: each (block of 32
+ * key channels, column) group gets its own fitted step. */
+static int varbit_head_store_seq(const orc_layout* L, const orc_writeback* wb, int64_t step, int b,
+                                 const float* S, const uint8_t* bits, uint8_t* packed, uint16_t* aux,
+                                 float* t_dump) {
+  vb_sections sec = varbit_sections(L);
+  int d = L->d, H = L->H, nbk = d / 32, flags = 0;
+  uint8_t* pay = packed + (size_t)b * sec.payload_per_seq;
+  uint16_t* sc = (uint16_t*)(packed + sec.off_scale) + (size_t)b * H * nbk * d;
+  uint8_t* wd = packed + sec.off_width + (size_t)b * H;
+  uint32_t* of = (uint32_t*)(packed + sec.off_offsets) + (size_t)b * (H + 1);
+  float x[32], tt[32];
+  uint16_t e[32];
+  int32_t q[32];
+  uint32_t off = 0;
+  for (int h = 0; h < H; ++h) {
+    of[h] = off;
+    off += (uint32_t)(d * d / 8) * bits[h];
+  }
+  of[H] = off;
+  for (int h = 0; h < H; ++h) {
+    int bw = bits[h], nl = (1 << (bw - 1)) - 1;
+    wd[h] = (uint8_t)bw;
+    for (int g = 0; g < nbk; ++g)
+      for (int j = 0; j < d; ++j) {
+        for (int r = 0; r < 32; ++r) {
+          size_t el = ((size_t)h * d + 32 * g + r) * d + j;
+          x[r] = S[el];
+          if (aux) e[r] = aux[(size_t)b * H * d * d + el];
+        }
+        flags |= orc_varbit_group(x, 32, bw, wb ? wb->mode : ORC_ROUND_NEAREST, wb ? wb->seed : 0,
+                                  step, h, b, 32 * g * d + j, d, aux ? e : NULL, q,
+                                  &sc[((size_t)h * nbk + g) * d + j], NULL, tt);
+        for (int r = 0; r < 32; ++r) {
+          size_t el = ((size_t)h * d + 32 * g + r) * d + j;
+          if (aux) aux[(size_t)b * H * d * d + el] = e[r];
+          if (t_dump) t_dump[(size_t)b * H * d * d + el] = tt[r];
+          put_bits(pay + of[h], ((size_t)(32 * g + r) * d + j) * bw, bw, (uint32_t)(q[r] + nl));
+        }
+      }
+  }
+  return flags;
+}
+
 /* Quantize every row of sequence b with widths `bits` and write payload,
  * scales, widths and offsets. */
 static int varbit_store_seq(const orc_layout* L, const orc_writeback* wb, int64_t step, int b,
@@ -1065,7 +1153,11 @@ static int run_seq_unit(const orc_layout* L, const orc_writeback* wb, int64_t st
   double lam = 1.0;
   for (int c = 0; c < C; ++c) lam *= (1.0 - 2.0 / 65.0);
 
-  varbit_load_seq(L, pin, b, S);
+  int head_units = L->storage == ORC_STORE_VARBIT_HEAD;
+  if (head_units)
+    varbit_head_load_seq(L, pin, b, S);
+  else
+    varbit_load_seq(L, pin, b, S);
   for (int t = 0; t < T; ++t) {
     int64_t step = step0 + t;
     for (int h = 0; h < H; ++h) {
@@ -1095,6 +1187,24 @@ static int run_seq_unit(const orc_layout* L, const orc_writeback* wb, int64_t st
         }
         ca2[r] = 0.0;
         ck[r] = 0.0;
+      }
+      if (head_units) {
+        /* head units ([LB] Allocation units): R~ = 1, so the cost of a head
+         * is its decay weight alone, the mean of its rows' weights (rows
+         * summed in order in FP64); one budget over the layer's heads */
+        for (int h = 0; h < H; ++h) {
+          double sum = 0.0;
+          for (int i = 0; i < d; ++i) {
+            int r = h * d + i;
+            sum += orc_persistence(L->persistence, st[2 * r + 0], st[2 * r + 1], C);
+          }
+          cost[h] = sum / (double)d;
+        }
+        flags |= orc_allocate_bits(H, cost, L->avg_bits, L->b_min, L->b_max, bits);
+        if (flags & ORC_EINVAL) break;
+        flags |= varbit_head_store_seq(L, wb, step, b, S, bits, pout, aux, t_dump);
+        varbit_head_load_seq(L, pout, b, S);
+        continue;
       }
       /* cost c_i = Gamma_hat_i * R~_i^2 with R~ the row range normalised by
        * the RMS of the ranges of its output group (one head) */
@@ -1157,6 +1267,15 @@ static int layout_ok(const orc_layout* L) {
     double tot = L->avg_bits * (double)(L->H * L->d);
     if (tot != floor(tot)) return 0;
   }
+  if (L->storage == ORC_STORE_VARBIT_HEAD) {
+    /* head units: b_min >= 2 (a one-bit head is ruled out), blocks of 32
+     * key channels, one budget over the layer's heads */
+    if (L->hadamard || L->b_min < 2 || L->b_max > 16 || L->b_min > L->b_max) return 0;
+    if (L->d % 32 || L->budget_scope != 1) return 0;
+    double tot = L->avg_bits * (double)L->H;
+    if (tot != floor(tot) || L->avg_bits < L->b_min || L->avg_bits > L->b_max) return 0;
+  }
+  if (L->storage < ORC_STORE_FP32 || L->storage > ORC_STORE_VARBIT_HEAD) return 0;
   return 1;
 }
 
@@ -1174,7 +1293,7 @@ int orc_run(const orc_layout* L, const orc_writeback* wb, int64_t step0, int T, 
     return ORC_EINVAL;
   orc_inputs in = {q, k, v, beta, decay, o};
   int flags = 0;
-  if (L->storage == ORC_STORE_VARBIT) {
+  if (L->storage == ORC_STORE_VARBIT || L->storage == ORC_STORE_VARBIT_HEAD) {
     for (int b = u0; b < u1; ++b)
       flags |= run_seq_unit(L, wb, step0, T, b, (const uint8_t*)packed_in, (uint8_t*)packed_out,
                             (uint16_t*)aux, stats, &in, t_dump);
@@ -1197,7 +1316,24 @@ int orc_state_pack(const orc_layout* L, const float* S, const int16_t* perm,
   orc_layout Lc = *L;
   Lc.domain = ORC_DOMAIN_CANONICAL;
   float* tmp = (float*)malloc(sizeof(float) * (size_t)d * d);
-  if (L->storage == ORC_STORE_VARBIT) {
+  if (L->storage == ORC_STORE_VARBIT_HEAD) {
+    /* widths [B][H] (or avg_bits for every head) summing to avg_bits * H */
+    int H = L->H;
+    uint8_t* bits = (uint8_t*)malloc((size_t)H);
+    for (int b = 0; b < L->B && !(flags & ORC_EINVAL); ++b) {
+      long sum = 0;
+      for (int h = 0; h < H; ++h) {
+        bits[h] = widths ? widths[(size_t)b * H + h] : (uint8_t)nearbyint(L->avg_bits);
+        sum += bits[h];
+        if (bits[h] < 1 || bits[h] > 16) flags |= ORC_EINVAL;
+      }
+      if ((double)sum != L->avg_bits * (double)H) flags |= ORC_EINVAL;
+      if (!(flags & ORC_EINVAL))
+        flags |= varbit_head_store_seq(L, NULL, 0, b, S + (size_t)b * H * d * d, bits, (uint8_t*)packed,
+                                       NULL, NULL);
+    }
+    free(bits);
+  } else if (L->storage == ORC_STORE_VARBIT) {
     int rows = L->H * d;
     uint8_t* bits = (uint8_t*)malloc((size_t)rows);
     float* seq = (float*)malloc(sizeof(float) * (size_t)rows * d);
@@ -1244,9 +1380,13 @@ int orc_state_unpack(const orc_layout* L, const void* packed, const int16_t* per
   int d = L->d;
   orc_layout Lc = *L;
   Lc.domain = ORC_DOMAIN_CANONICAL;
-  if (L->storage == ORC_STORE_VARBIT) {
-    for (int b = 0; b < L->B; ++b)
-      varbit_load_seq(L, (const uint8_t*)packed, b, S + (size_t)b * L->H * d * d);
+  if (L->storage == ORC_STORE_VARBIT || L->storage == ORC_STORE_VARBIT_HEAD) {
+    for (int b = 0; b < L->B; ++b) {
+      if (L->storage == ORC_STORE_VARBIT_HEAD)
+        varbit_head_load_seq(L, (const uint8_t*)packed, b, S + (size_t)b * L->H * d * d);
+      else
+        varbit_load_seq(L, (const uint8_t*)packed, b, S + (size_t)b * L->H * d * d);
+    }
     return ORC_OK;
   }
   float* tmp = (float*)malloc(sizeof(float) * (size_t)d * d);

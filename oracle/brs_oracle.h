@@ -26,7 +26,7 @@
 extern "C" {
 #endif
 
-enum { ORC_STORE_FP32 = 0, ORC_STORE_DAMP = 1, ORC_STORE_VARBIT = 2 };
+enum { ORC_STORE_FP32 = 0, ORC_STORE_DAMP = 1, ORC_STORE_VARBIT = 2, ORC_STORE_VARBIT_HEAD = 3 };
 enum { ORC_ROUND_NEAREST = 0, ORC_ROUND_STOCHASTIC = 1, ORC_ROUND_ERRFEEDBACK = 2, ORC_ROUND_DIRECTION = 3,
        ORC_ROUND_RESIDUAL2 = 4, ORC_ROUND_RESIDUAL3 = 5, ORC_ROUND_RESIDUAL4 = 6 };
 enum { ORC_DOMAIN_CANONICAL = 0, ORC_DOMAIN_ROTATED = 1, ORC_DOMAIN_MIXED = 2 };
@@ -98,10 +98,18 @@ int orc_int8_block_dm(const float* y, const float* xprev, int n, int8_t* m_inout
 int orc_int8_block_rm(const float* y, int n, int kbits, float sprev, int8_t* m_inout, uint8_t* codes,
                       uint16_t* scale_h, uint16_t* zero_h, float* t_out);
 
-/* One variable-width row (decay-aware allocation tier), width bw in [2, 8]. */
+/* One variable-width row (decay-aware allocation tier), width bw in [1, 16]. */
 int orc_varbit_row(const float* x, int n, int bw, int mode, uint64_t seed, int64_t step, int h,
                    int b, int elem0, uint16_t* e_inout, int32_t* q_out, uint16_t* delta_h,
                    int* m_star, float* t_out);
+
+/* One scale group of the same quantizer whose elements sit estride apart in
+ * the head (element j of the group is element elem0 + j * estride of the
+ * head for the stochastic-rounding counters); x, e_inout, q_out and t_out
+ * hold the group contiguously.  orc_varbit_row is the case estride = 1. */
+int orc_varbit_group(const float* x, int n, int bw, int mode, uint64_t seed, int64_t step, int h,
+                     int b, int elem0, int estride, uint16_t* e_inout, int32_t* q_out,
+                     uint16_t* delta_h, int* m_star, float* t_out);
 
 /* Approximate erasure-rate persistence weight, rho = 1. */
 double orc_gamma_hat(double A, double K, int C);

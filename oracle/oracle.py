@@ -25,7 +25,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "brs_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
-STORE_FP32, STORE_DAMP, STORE_VARBIT = 0, 1, 2
+STORE_FP32, STORE_DAMP, STORE_VARBIT, STORE_VARBIT_HEAD = 0, 1, 2, 3
 ROUND_NEAREST, ROUND_STOCHASTIC, ROUND_ERRFEEDBACK, ROUND_DIRECTION = 0, 1, 2, 3
 ROUND_RESIDUAL2, ROUND_RESIDUAL3, ROUND_RESIDUAL4 = 4, 5, 6
 DOMAIN_CANONICAL, DOMAIN_ROTATED, DOMAIN_MIXED = 0, 1, 2
@@ -92,6 +92,9 @@ def lib():
             L.orc_int8_block_rm.argtypes = [P, ct.c_int, ct.c_int, ct.c_float, P, P, P, P, P]
             L.orc_persistence.restype = ct.c_double
             L.orc_persistence.argtypes = [ct.c_int, ct.c_double, ct.c_double, ct.c_int]
+            L.orc_varbit_group.restype = ct.c_int
+            L.orc_varbit_group.argtypes = [P, ct.c_int, ct.c_int, ct.c_int, ct.c_uint64, ct.c_int64,
+                                           ct.c_int, ct.c_int, ct.c_int, ct.c_int, P, P, P, P, P]
             L.orc_varbit_row.restype = ct.c_int
             L.orc_varbit_row.argtypes = [P, ct.c_int, ct.c_int, ct.c_int, ct.c_uint64, ct.c_int64,
                                          ct.c_int, ct.c_int, ct.c_int, P, P, P, P, P]
@@ -252,6 +255,19 @@ def varbit_row(x, bw, mode=ROUND_NEAREST, seed=0, step=0, h=0, b=0, elem0=0, e=N
     return dict(q=q, delta=dh[0], m=int(ms[0]), t=t, e=e, flags=fl)
 
 
+def varbit_group(x, bw, mode=ROUND_NEAREST, seed=0, step=0, h=0, b=0, elem0=0, estride=1, e=None):
+    x = _c(x, np.float32)
+    n = x.size
+    q = np.zeros(n, np.int32)
+    dh = np.zeros(1, np.uint16)
+    ms = np.zeros(1, np.int32)
+    t = np.zeros(n, np.float32)
+    e = None if e is None else np.array(e, dtype=np.uint16)
+    fl = lib().orc_varbit_group(_p(x), n, bw, mode, seed, step, h, b, elem0, estride, _p(e), _p(q),
+                                _p(dh), _p(ms), _p(t))
+    return dict(q=q, delta=dh[0], m=int(ms[0]), t=t, e=e, flags=fl)
+
+
 def gamma_hat(A: float, K: float, C: int) -> float:
     return lib().orc_gamma_hat(A, K, C)
 
@@ -322,7 +338,7 @@ def run(cfg: Config, wb_mode: int, seed: int, C: int, step0: int, inputs: dict, 
     decay = _c(inputs["decay"], np.float32)
     T = q.shape[0]
     o = np.zeros((T, cfg.B, cfg.H, cfg.d), np.float32)
-    nunits = cfg.B if cfg.storage == STORE_VARBIT else cfg.B * cfg.H
+    nunits = cfg.B if cfg.storage in (STORE_VARBIT, STORE_VARBIT_HEAD) else cfg.B * cfg.H
     u0, u1 = (0, nunits) if units is None else units
     t = np.zeros(cfg.B * cfg.H * cfg.d * cfg.d, np.float32) if dump_t else None
     sd = np.zeros((cfg.B, cfg.H, cfg.d, cfg.d), np.float32) if dump_s else None
@@ -355,7 +371,7 @@ def run_parallel(cfg: Config, wb_mode: int, seed: int, C: int, step0: int, input
 
     Returns (o, flags, threads_used), and the state dump of ``run`` last when
     ``dump_s`` is set."""
-    nunits = cfg.B if cfg.storage == STORE_VARBIT else cfg.B * cfg.H
+    nunits = cfg.B if cfg.storage in (STORE_VARBIT, STORE_VARBIT_HEAD) else cfg.B * cfg.H
     u0, u1 = (0, nunits) if units is None else units
     nthr = max(1, min(threads or os.cpu_count() or 1, u1 - u0))
     L = cfg.layout()

@@ -108,3 +108,26 @@ def varbit_row_codes(pay_seq, off, bw, d):
     nbytes = d * bw // 8
     raw = np.unpackbits(pay_seq[off: off + nbytes], bitorder="little")
     return raw.reshape(d, bw) @ (1 << np.arange(bw))
+
+
+def varbit_head_sections(packed, B, H, d, avg_bits):
+    """Split a per-head variable-width state into its documented sections:
+    payload [B][P], FP16 steps [B][H][d/32][d], widths [B][H], head offsets
+    [B][H+1]."""
+    nbk = d // 32
+    P = int(d * d // 8 * avg_bits * H)
+    off_scale = r256(P * B)
+    off_width = off_scale + r256(B * H * nbk * d * 2)
+    off_offs = off_width + r256(B * H)
+    pay = packed[: P * B].reshape(B, P)
+    sc = np.frombuffer(packed[off_scale: off_scale + B * H * nbk * d * 2].tobytes(), np.uint16)
+    wd = packed[off_width: off_width + B * H].reshape(B, H)
+    of = np.frombuffer(packed[off_offs: off_offs + B * (H + 1) * 4].tobytes(), np.uint32)
+    return pay, sc.reshape(B, H, nbk, d), wd, of.reshape(B, H + 1)
+
+
+def varbit_head_codes(pay_seq, off, bw, d):
+    """Unsigned codes [d][d] of one head: element (i, j) at bit (i d + j) bw."""
+    nbytes = d * d * bw // 8
+    raw = np.unpackbits(pay_seq[off: off + nbytes], bitorder="little")
+    return (raw.reshape(d * d, bw) @ (1 << np.arange(bw))).reshape(d, d)
