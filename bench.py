@@ -3,7 +3,7 @@ GB/s against the measured B200 copy bandwidth).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload kda_decode|gdn_decode|gdn_decode_fp32|varbit_decode|
-                                kda_decode_c8|kda_prefill|kda_tiny]
+                                gdn_varbit_decode|kda_decode_c8|kda_prefill|kda_tiny]
 
 A step is one decode token for every (sequence, head) of the workload: one
 launch of the fused decode kernel (dequantize, decay, delta-rule write, read
@@ -18,6 +18,9 @@ over the whole batch (B x T tokens x H heads, write-back every 64 tokens).
 `--workload kda_decode_c8` decodes with write-back every 8 tokens (the FP32
 state carried in HBM between write-backs; state bytes averaged over the
 interval).
+
+`--workload gdn_varbit_decode` runs GDN heads with one width per head (steps
+per block of 32 key channels), three launches per step as for varbit_decode.
 
 `--impl reference` times the plain CPU oracle on this host's cores on the
 same workload and metric (bounded samples), which is the only other place
@@ -50,12 +53,16 @@ KERNEL_SOURCES = {
     "warp": ["bit_recurrent_state_b200/csrc/decode.cu", "bit_recurrent_state_b200/csrc/brs_device.cuh"],
     "varbit": ["bit_recurrent_state_b200/csrc/varbit.cu", "bit_recurrent_state_b200/csrc/allocate.cu",
                "bit_recurrent_state_b200/csrc/brs_device.cuh"],
+    "varbit_head": ["bit_recurrent_state_b200/csrc/varbit_head.cu", "bit_recurrent_state_b200/csrc/allocate.cu",
+                    "bit_recurrent_state_b200/csrc/brs_device.cuh"],
 }
+
+VARBIT_STORES = ("varbit", "varbit_head")
 
 
 def kernel_family(w) -> str:
-    if w.storage == "varbit":
-        return "varbit"
+    if w.storage in VARBIT_STORES:
+        return w.storage
     cta = (w.storage == "damp" and w.d == 128 and w.C == 1 and w.k_hi % 16 == 0 and
            w.mode in ("nearest", "stochastic", "errfeedback"))
     return "cta" if cta else "warp"
@@ -77,7 +84,7 @@ def algorithmic_bytes(w) -> dict:
     heads = w.B * w.H
     inputs = (2 * w.B * w.hk * w.d * 2 + heads * w.d * 2 + heads * 4 +
               (heads * w.d * 4 if w.decay_per_key else heads * 4) +
-              (w.H * w.d * 2 if w.storage != "varbit" else 0))
+              (w.H * w.d * 2 if w.storage not in VARBIT_STORES else 0))
     out = heads * w.d * 4
     ef = 2 * aux if w.mode == "errfeedback" else 0
     if w.mode == "direction":
@@ -120,6 +127,8 @@ def kernel_name(w) -> str:
     """The kernel a decode step of workload w launches (the dominant one)."""
     if w.storage == "varbit":
         return "brs::varbit_kernel (update pass + fit pass) and brs::allocate_kernel"
+    if w.storage == "varbit_head":
+        return "brs::varbit_head_kernel (update pass + fit pass) and brs::allocate_kernel"
     if kernel_family(w) == "cta":
         return "brs::decode_cta_kernel"
     return "brs::decode_warp_kernel"
@@ -241,7 +250,8 @@ class ClockSampler:
 
 def _oracle_cfg(w):
     from oracle import oracle as O
-    st = {"fp32": O.STORE_FP32, "damp": O.STORE_DAMP, "varbit": O.STORE_VARBIT}[w.storage]
+    st = {"fp32": O.STORE_FP32, "damp": O.STORE_DAMP, "varbit": O.STORE_VARBIT,
+          "varbit_head": O.STORE_VARBIT_HEAD}[w.storage]
     return O.Config(B=w.B, H=w.H, Hk=w.hk, d=w.d, storage=st, k_hi=w.k_hi, block=w.block,
                     hadamard=w.hadamard, decay_per_key=w.decay_per_key, avg_bits=w.avg_bits,
                     b_min=w.b_min, b_max=w.b_max,
@@ -261,7 +271,7 @@ def workload_config(w, world: int) -> dict:
            "block": w.block, "mode": w.mode, "per_rank_batch": w.B, "parallelism": f"dp{world}"}
     if w.C > 1:
         cfg.update(T=w.T, C=w.C)
-    if w.storage == "varbit":
+    if w.storage in VARBIT_STORES:
         cfg.update(avg_bits=w.avg_bits, b_min=w.b_min, b_max=w.b_max)
     cfg["l2"] = l2_policy(w)
     return cfg
@@ -294,7 +304,7 @@ class OracleRunner:
         self.cores = os.cpu_count() or 1
         self.t = 0
         self.cache = {}
-        self.varbit = w.storage == "varbit"
+        self.varbit = w.storage in VARBIT_STORES
         self.units_total = w.B if self.varbit else w.B * w.H
         self.heads_per_unit = w.H if self.varbit else 1
         self.mode = {"nearest": O.ROUND_NEAREST, "stochastic": O.ROUND_STOCHASTIC,
@@ -562,7 +572,7 @@ def run_ours(args, w):
     wb = brs.writeback_of(wr)
     rng = np.random.default_rng(wr.seed)
     perm = np.stack([rng.permutation(w.d) for _ in range(w.H)]).astype(np.int16)
-    varbit = w.storage == "varbit"
+    varbit = w.storage in VARBIT_STORES
     if varbit:
         perm = None                    # variable-width rows stay in key-channel order
     layers, spares, inputs, host_inputs = [], [], [], []

@@ -14,15 +14,15 @@ import os
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libbrs.so")
 
-STORE_FP32, STORE_DAMP, STORE_VARBIT = 0, 1, 2
+STORE_FP32, STORE_DAMP, STORE_VARBIT, STORE_VARBIT_HEAD = 0, 1, 2, 3
 ROUND_NEAREST, ROUND_STOCHASTIC, ROUND_ERRFEEDBACK, ROUND_DIRECTION = 0, 1, 2, 3
 ROUND_RESIDUAL2, ROUND_RESIDUAL3, ROUND_RESIDUAL4 = 4, 5, 6
 OK, EINVAL, EUNSUPPORTED, EALIGN, ECUDA, ENONFINITE, EOVERFLOW, ETIMEOUT = range(8)
-FLAG_NONFINITE, FLAG_OVERFLOW, FLAG_TIMEOUT = 1, 2, 4
+FLAG_NONFINITE, FLAG_OVERFLOW, FLAG_TIMEOUT, FLAG_INVALID = 1, 2, 4, 8
 MODES = {"nearest": ROUND_NEAREST, "stochastic": ROUND_STOCHASTIC,
          "errfeedback": ROUND_ERRFEEDBACK, "direction": ROUND_DIRECTION,
          "residual2": ROUND_RESIDUAL2, "residual3": ROUND_RESIDUAL3, "residual4": ROUND_RESIDUAL4}
-STORES = {"fp32": STORE_FP32, "damp": STORE_DAMP, "varbit": STORE_VARBIT}
+STORES = {"fp32": STORE_FP32, "damp": STORE_DAMP, "varbit": STORE_VARBIT, "varbit_head": STORE_VARBIT_HEAD}
 
 # exported symbols declared in include/brs.h
 SYMBOLS = ["brs_state_bytes", "brs_state_pack", "brs_state_unpack", "brs_decode_step",
@@ -233,7 +233,7 @@ def fetch_errors(workspace, stream=None) -> int:
     """Raw device flag bits (also raises BrsError if any is set)."""
     fl = ct.c_uint32(0)
     st = lib().brs_fetch_errors(_ptr(workspace), ct.byref(fl), _stream(stream))
-    if st != OK and st not in (ENONFINITE, EOVERFLOW, ETIMEOUT):
+    if st != OK and fl.value == 0:                 # a call error, not a device flag
         _check(st)
     return int(fl.value)
 
@@ -243,7 +243,7 @@ def fetch_errors_noalloc(stream=None) -> int:
     current device since the last read (also cleared)."""
     fl = ct.c_uint32(0)
     st = lib().brs_fetch_errors_noalloc(ct.byref(fl), _stream(stream))
-    if st != OK and st not in (ENONFINITE, EOVERFLOW, ETIMEOUT):
+    if st != OK and fl.value == 0:                 # a call error, not a device flag
         _check(st)
     return int(fl.value)
 

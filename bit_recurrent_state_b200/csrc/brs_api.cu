@@ -55,10 +55,29 @@ brs_status check_layout(const brs_layout* L) {
     const double tot = L->avg_bits * (double)L->H * (double)L->d;
     if (tot != std::floor(tot)) return fail(BRS_EINVAL, "avg_bits * H * d must be an integer");
     if (L->avg_bits < L->b_min || L->avg_bits > L->b_max) return fail(BRS_EINVAL, "avg_bits outside [b_min, b_max]");
+  } else if (L->storage == BRS_STORE_VARBIT_HEAD) {
+    if (L->hadamard) return fail(BRS_EUNSUPPORTED, "variable-width storage is stored without the Hadamard");
+    if (L->d != 128) return fail(BRS_EUNSUPPORTED, "per-head widths are built for d = 128 (got %d)", L->d);
+    if (L->b_min < 2 || L->b_max > 16 || L->b_min > L->b_max)
+      return fail(BRS_EINVAL, "per-head widths need 2 <= b_min <= b_max <= 16");
+    if (L->budget_scope != 1) return fail(BRS_EINVAL, "per-head widths share one budget over the layer (budget_scope 1)");
+    if (L->persistence < 0 || L->persistence > 2) return fail(BRS_EINVAL, "persistence must be 0, 1 or 2");
+    const double tot = L->avg_bits * (double)L->H;
+    if (tot != std::floor(tot)) return fail(BRS_EINVAL, "avg_bits * H must be an integer");
+    if (L->avg_bits < L->b_min || L->avg_bits > L->b_max) return fail(BRS_EINVAL, "avg_bits outside [b_min, b_max]");
   } else if (L->storage != BRS_STORE_FP32) {
     return fail(BRS_EINVAL, "unknown storage %d", L->storage);
   }
   return BRS_OK;
+}
+
+bool varbit_like(const brs_layout* L) {
+  return L->storage == BRS_STORE_VARBIT || L->storage == BRS_STORE_VARBIT_HEAD;
+}
+
+brs::VbSections vb_sections_of(const brs_layout* L) {
+  return L->storage == BRS_STORE_VARBIT_HEAD ? brs::varbit_head_sections(L->B, L->H, L->d, L->avg_bits)
+                                             : brs::varbit_sections(L->B, L->H, L->d, L->avg_bits);
 }
 
 // width of the DAMP low tier: 8 unless the layout asks for 4
@@ -102,10 +121,11 @@ size_t brs_state_bytes(const brs_layout* L, size_t* aux_bytes, size_t* stats_byt
     total = heads * damp_head_bytes(L);
     aux = heads * (d - (size_t)L->k_hi) * d * 2;
   } else {
-    total = brs::varbit_sections(L->B, L->H, L->d, L->avg_bits).total;
+    total = vb_sections_of(L).total;
     aux = heads * d * d * 2;
     stats = heads * d * 2 * sizeof(double);
-    ws = 256 + heads * d * sizeof(double);   // flag word, then one FP64 cost per row
+    // flag word, then one FP64 cost per row (per head for head units)
+    ws = 256 + heads * (L->storage == BRS_STORE_VARBIT_HEAD ? 1 : d) * sizeof(double);
   }
   if (aux_bytes) *aux_bytes = aux;
   if (stats_bytes) *stats_bytes = stats;
@@ -119,7 +139,7 @@ brs_status brs_state_pack(const brs_layout* L, const float* S, const int16_t* pe
   brs_status st = check_layout(L);
   if (st != BRS_OK) return st;
   if (!S || !packed || !workspace) return fail(BRS_EINVAL, "S, packed and workspace are required");
-  if (L->storage == BRS_STORE_VARBIT) {
+  if (varbit_like(L)) {
     if (perm) return fail(BRS_EINVAL, "variable-width storage keeps rows in key-channel order (perm must be NULL)");
     if (!widths && L->avg_bits != std::floor(L->avg_bits))
       return fail(BRS_EINVAL, "uniform widths need an integer avg_bits");
@@ -127,9 +147,10 @@ brs_status brs_state_pack(const brs_layout* L, const float* S, const int16_t* pe
       return fail(BRS_EALIGN, "device pointers must be 16-byte aligned");
     brs::VbPackArgs v{};
     v.B = L->B; v.H = L->H; v.d = L->d; v.avg_bits = L->avg_bits;
-    v.sec = brs::varbit_sections(L->B, L->H, L->d, L->avg_bits);
+    v.sec = vb_sections_of(L);
     v.S = S; v.widths = widths; v.packed = packed; v.flags = (uint32_t*)workspace;
-    cudaError_t e = brs::launch_varbit_pack(v, (cudaStream_t)stream);
+    cudaError_t e = L->storage == BRS_STORE_VARBIT_HEAD ? brs::launch_varbit_head_pack(v, (cudaStream_t)stream)
+                                                        : brs::launch_varbit_pack(v, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "variable-width pack launch");
     return ok();
   }
@@ -151,14 +172,16 @@ brs_status brs_state_unpack(const brs_layout* L, const void* packed, const int16
   brs_status st = check_layout(L);
   if (st != BRS_OK) return st;
   if (!S || !packed) return fail(BRS_EINVAL, "S and packed are required");
-  if (L->storage == BRS_STORE_VARBIT) {
+  if (varbit_like(L)) {
     if (perm) return fail(BRS_EINVAL, "variable-width storage keeps rows in key-channel order (perm must be NULL)");
     if (!aligned16(S) || !aligned16(packed)) return fail(BRS_EALIGN, "device pointers must be 16-byte aligned");
     brs::VbPackArgs v{};
     v.B = L->B; v.H = L->H; v.d = L->d; v.avg_bits = L->avg_bits;
-    v.sec = brs::varbit_sections(L->B, L->H, L->d, L->avg_bits);
+    v.sec = vb_sections_of(L);
     v.flags = (uint32_t*)workspace;
-    cudaError_t e = brs::launch_varbit_unpack(v, packed, S, (cudaStream_t)stream);
+    cudaError_t e = L->storage == BRS_STORE_VARBIT_HEAD
+                        ? brs::launch_varbit_head_unpack(v, packed, S, (cudaStream_t)stream)
+                        : brs::launch_varbit_unpack(v, packed, S, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "variable-width unpack launch");
     return ok();
   }
@@ -191,7 +214,7 @@ brs_status brs_decode_step(const brs_layout* L, const brs_writeback* wb, int64_t
   if (step < 0) return fail(BRS_EINVAL, "step must be >= 0");
   if (!packed_in || !packed_out || !workspace || !q || !k || !v || !beta || !decay || !o)
     return fail(BRS_EINVAL, "a required pointer is NULL");
-  if (L->storage == BRS_STORE_VARBIT) {
+  if (varbit_like(L)) {
     if (L->d != 128) return fail(BRS_EUNSUPPORTED, "variable-width decode is built for d = 128");
     if (packed_in == packed_out) return fail(BRS_EINVAL, "variable-width decode needs packed_out != packed_in");
     if (perm) return fail(BRS_EINVAL, "variable-width storage keeps rows in key-channel order (perm must be NULL)");
@@ -207,11 +230,12 @@ brs_status brs_decode_step(const brs_layout* L, const brs_writeback* wb, int64_t
     double lam = 1.0;
     for (int c = 0; c < wb->C; ++c) lam *= (1.0 - 2.0 / 65.0);   // EMA weight of a C-token chunk, span 64
     a.lambda = lam; a.avg_bits = L->avg_bits;
-    a.sec = brs::varbit_sections(L->B, L->H, L->d, L->avg_bits);
+    a.sec = vb_sections_of(L);
     a.packed_in = packed_in; a.packed_out = packed_out; a.aux = aux; a.stats = (double*)stats;
     a.cost = (double*)((uint8_t*)workspace + 256);
     a.q = q; a.k = k; a.v = v; a.beta = beta; a.decay = decay; a.o = o; a.flags = (uint32_t*)workspace;
-    cudaError_t e = brs::launch_varbit_decode(a, (cudaStream_t)stream);
+    cudaError_t e = L->storage == BRS_STORE_VARBIT_HEAD ? brs::launch_varbit_head_decode(a, (cudaStream_t)stream)
+                                                        : brs::launch_varbit_decode(a, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "variable-width decode launch");
     return ok();
   }
@@ -449,6 +473,7 @@ brs_status brs_fetch_errors(void* workspace, uint32_t* flags_out, void* stream) 
   if (fl & BRS_FLAG_NONFINITE) return fail(BRS_ENONFINITE, "a kernel met a non-finite state value");
   if (fl & BRS_FLAG_OVERFLOW) return fail(BRS_EOVERFLOW, "an FP16 row, scale or zero overflowed");
   if (fl & BRS_FLAG_TIMEOUT) return fail(BRS_ETIMEOUT, "a bounded device wait gave up");
+  if (fl & BRS_FLAG_INVALID) return fail(BRS_EINVAL, "a device-side argument check failed (widths off the budget)");
   return ok();
 }
 

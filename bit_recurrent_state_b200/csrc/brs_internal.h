@@ -87,6 +87,7 @@ VbSections varbit_sections(int B, int H, int d, double avg_bits);
 struct VbPackArgs {
   int B, H, d;
   double avg_bits;
+  float one = 1.0f;              // 1 read at run time: a multiplier the compiler cannot fold
   VbSections sec;
   const float* S;                // [B][H][d][d]
   const uint8_t* widths;         // [B][H*d] or null (avg_bits everywhere)
@@ -115,6 +116,12 @@ struct VbArgs {
 };
 cudaError_t launch_varbit_decode(const VbArgs& a, cudaStream_t st);
 cudaError_t launch_varbit_offsets(const VbArgs& a, cudaStream_t st);
+
+// per-head widths (one width per head, steps per block of 32 key channels)
+VbSections varbit_head_sections(int B, int H, int d, double avg_bits);
+cudaError_t launch_varbit_head_decode(const VbArgs& a, cudaStream_t st);
+cudaError_t launch_varbit_head_pack(const VbPackArgs& a, cudaStream_t st);
+cudaError_t launch_varbit_head_unpack(const VbPackArgs& a, const void* packed, float* S, cudaStream_t st);
 
 struct PrefillArgs {
   int B, H, Hk, T, k_hi, block, decay_per_key, mode;

@@ -40,7 +40,7 @@ class Workload:
     d: int
     T: int
     Hk: int = 0
-    storage: str = "damp"          # "fp32" | "damp" | "varbit"
+    storage: str = "damp"          # "fp32" | "damp" | "varbit" | "varbit_head"
     k_hi: int = 0
     block: int = 128
     hadamard: int = 1
@@ -76,6 +76,11 @@ WORKLOADS = {
                             seed=4),
     # decode with deferred write-back every 8 tokens (a NEXT configuration)
     "kda_decode_c8": Workload("kda_decode_c8", B=64, H=32, d=128, T=1024, k_hi=16, block=128, C=8, seed=1),
+    # GDN heads with one width per head (a NEXT configuration): the GDN decode
+    # shape and inputs, 4.0 bits per value on average, widths 2..8
+    "gdn_varbit_decode": Workload("gdn_varbit_decode", B=256, H=32, Hk=16, d=128, T=512,
+                                  storage="varbit_head", hadamard=0, avg_bits=4.0, b_min=2, b_max=8,
+                                  decay_per_key=0, seed=2),
 }
 
 

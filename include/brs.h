@@ -71,6 +71,23 @@
  *                    widths of rows < r); value = (u - n) * step.
  *                    Residuals f16 [B][H][d][d]; statistics f64
  *                    [B][H][d][2] = (EMA of a^2, EMA of beta (2-beta) k^2).
+ *   BRS_STORE_VARBIT_HEAD [LB] Allocation units (per-head decay, as in
+ *                    Gated DeltaNet): one width per head, one FP16 step
+ *                    per block of 32 key channels and column.  Sections,
+ *                    each starting on a 256-byte boundary: payload [B][P]
+ *                    with P = d*d/8 * avg_bits * H; f16 step
+ *                    [B][H][d/32][d]; u8 width [B][H] (b_min >= 2);
+ *                    u32 head offset [B][H+1].  Head h of sequence b holds
+ *                    element (i, j) (key channel i, value column j) as a
+ *                    w-bit code u = q + n at bit (i*d + j)*w of its bytes,
+ *                    starting at offset[h] = d*d/8 * (sum of the widths of
+ *                    heads < h); value = (u - n) * step[i/32][j].  The
+ *                    steps are fitted per (block, column) group as for a
+ *                    row; the allocator runs over each sequence's H heads
+ *                    with a head's cost the mean of its rows' decay
+ *                    weights (no range term).  d = 128; residuals and
+ *                    statistics as for VARBIT; the workspace holds the
+ *                    flag word and one f64 cost per head.
  *
  * Arithmetic (identical on every path that produces stored codes)
  *   The update runs in FP32 ([DAMP] Implementation): per token and head,
@@ -114,7 +131,7 @@ typedef enum {
   BRS_ETIMEOUT = 7       /* a bounded device-side wait gave up                  */
 } brs_status;
 
-typedef enum { BRS_STORE_FP32 = 0, BRS_STORE_DAMP = 1, BRS_STORE_VARBIT = 2 } brs_storage;
+typedef enum { BRS_STORE_FP32 = 0, BRS_STORE_DAMP = 1, BRS_STORE_VARBIT = 2, BRS_STORE_VARBIT_HEAD = 3 } brs_storage;
 
 typedef enum {
   BRS_ROUND_NEAREST = 0,
@@ -150,6 +167,7 @@ typedef enum {
 #define BRS_FLAG_NONFINITE 0x1u
 #define BRS_FLAG_OVERFLOW 0x2u
 #define BRS_FLAG_TIMEOUT 0x4u
+#define BRS_FLAG_INVALID 0x8u   /* a device-side argument check failed (e.g. widths off the budget) */
 
 typedef struct {
   int32_t B;             /* sequences                                          */
@@ -193,8 +211,11 @@ size_t brs_state_bytes(const brs_layout* L, size_t* aux_bytes, size_t* stats_byt
 /* FP32 state S [B][H][d][d] (rows in key-channel order) -> stored format,
  * deterministic rounding.  perm [H][d] int16 (stored row i of head h holds
  * channel perm[h][i]); NULL = identity.  widths (VARBIT only) u8 [B][H*d]
- * device array of row widths, NULL = avg_bits for every row (which must
- * then be an integer).  All pointers device, `packed` sized by
+ * device array of row widths (VARBIT_HEAD: u8 [B][H], head widths), NULL =
+ * avg_bits for every row or head (which must then be an integer).  A
+ * VARBIT_HEAD width map whose sequence total is not avg_bits * H, or with a
+ * width outside 1..16, stores nothing for that sequence and raises
+ * BRS_FLAG_INVALID.  All pointers device, `packed` sized by
  * brs_state_bytes.  [DAMP] Implementation (static permuted layout). */
 brs_status brs_state_pack(const brs_layout* L, const float* S, const int16_t* perm,
                           const uint8_t* widths, void* packed, void* workspace, void* stream);

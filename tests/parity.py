@@ -8,7 +8,8 @@ from oracle import oracle as O
 MODE = {"nearest": O.ROUND_NEAREST, "stochastic": O.ROUND_STOCHASTIC,
         "errfeedback": O.ROUND_ERRFEEDBACK, "direction": O.ROUND_DIRECTION,
         "residual2": O.ROUND_RESIDUAL2, "residual3": O.ROUND_RESIDUAL3, "residual4": O.ROUND_RESIDUAL4}
-STORE = {"fp32": O.STORE_FP32, "damp": O.STORE_DAMP, "varbit": O.STORE_VARBIT}
+STORE = {"fp32": O.STORE_FP32, "damp": O.STORE_DAMP, "varbit": O.STORE_VARBIT,
+         "varbit_head": O.STORE_VARBIT_HEAD}
 
 
 def oracle_cfg(w: synth.Workload) -> O.Config:

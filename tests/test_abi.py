@@ -39,6 +39,20 @@ def test_host_only_calls_without_gpu():
     n4, aux4, _, _ = brs.state_bytes(brs.layout_of(w4))
     assert n4 == (112 * 64 + 16 * 128 * 2 + 112 * 4) * 64 * 32 and aux4 == aux
     assert brs.state_bytes(brs.layout_of(w4, low_bits=0))[0] == 18880 * 64 * 32   # 0 reads as 8
+    # per-head widths: payload, steps per (block of 32 keys, column), widths, head offsets
+    wh = synth.WORKLOADS["gdn_varbit_decode"]
+    nh, auxh, sth, wsh = brs.state_bytes(brs.layout_of(wh))
+    heads = 256 * 32
+    assert nh == 2048 * 4 * heads + heads * 4 * 128 * 2 + heads + 256 * 33 * 4
+    assert auxh == heads * 128 * 128 * 2 and sth == heads * 128 * 16 and wsh == 256 + heads * 8
+    for bad, msg in ((dict(b_min=1), "b_min"), (dict(avg_bits=4.01), "integer"), (dict(d=64), "d = 128"),
+                     (dict(hadamard=1), "Hadamard")):
+        with pytest.raises(brs.BrsError) as e:               # state_bytes reports every layout error as EINVAL
+            brs.state_bytes(brs.layout_of(wh.with_(**bad)))
+        assert msg in str(e.value), bad
+    with pytest.raises(brs.BrsError) as e:
+        brs.state_bytes(brs.layout_of(wh, budget_scope=0))
+    assert "budget" in str(e.value)
 
 
 def test_prefill_workspace_size():
