@@ -51,6 +51,8 @@ class Workload:
     C: int = 1
     persistence: int = 0              # variable-width cost weight (0 Gamma_hat, 1 w^(1), 2 h^(C))
     low_bits: int = 8                 # DAMP low tier: 8 (INT8) or 4 (two codes per byte)
+    s_min: float = 1e-3               # decay rates s log-uniform in [s_min, 1]
+    persistent_keys: int = 0          # 1: one fixed key per (sequence, key head) for every token
     mode: str = "nearest"          # "nearest" | "stochastic" | "errfeedback" | "direction"
     seed: int = 0
 
@@ -85,10 +87,11 @@ WORKLOADS = {
 
 
 def decay_table(w: Workload) -> np.ndarray:
-    """a = exp(-s), s log-uniform in [1e-3, 1]: [H][d] (KDA) or [H] (GDN)."""
+    """a = exp(-s), s log-uniform in [s_min, 1] (s_min = 1e-3 unless the
+    workload says otherwise): [H][d] (KDA) or [H] (GDN)."""
     rng = np.random.default_rng([w.seed, 0])
     shape = (w.H, w.d) if w.decay_per_key else (w.H,)
-    s = np.exp(rng.uniform(np.log(1e-3), np.log(1.0), size=shape))
+    s = np.exp(rng.uniform(np.log(w.s_min), np.log(1.0), size=shape))
     return np.exp(-s).astype(np.float32)
 
 
@@ -103,6 +106,8 @@ def token_inputs(w: Workload, t: int, batch: slice | None = None) -> dict:
     k = rng.standard_normal((B, Hk, d))
     v = rng.standard_normal((B, H, d))
     beta = 1.0 / (1.0 + np.exp(-rng.standard_normal((B, H))))
+    if w.persistent_keys:
+        k = np.random.default_rng([w.seed, 2]).standard_normal((B, Hk, d))
     q /= np.linalg.norm(q, axis=-1, keepdims=True)
     k /= np.linalg.norm(k, axis=-1, keepdims=True)
     a = decay_table(w)
