@@ -46,13 +46,20 @@ def build(force: bool = False, verbose: bool = False) -> str:
     objdir = os.path.join(ROOT, "_build")
     os.makedirs(objdir, exist_ok=True)
     objs, cmds = [], []
+    headers = glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh"))
+    headers += glob.glob(os.path.join(ROOT, "include", "*.h"))
+    newest_header = max((os.path.getmtime(p) for p in headers), default=0.0)
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
+        objs.append(obj)
+        # an object newer than its source and every header is kept
+        if (not force and not verbose and os.path.exists(obj) and
+                os.path.getmtime(obj) > max(os.path.getmtime(src), newest_header)):
+            continue
         cmd = [nvcc, *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-I", CSRC, "-c", src, "-o", obj]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
         cmds.append(cmd)
-        objs.append(obj)
     # one nvcc per translation unit, run side by side
     with ThreadPoolExecutor(max_workers=max(1, min(len(cmds), os.cpu_count() or 1))) as ex:
         for f in [ex.submit(subprocess.check_call, c) for c in cmds]:

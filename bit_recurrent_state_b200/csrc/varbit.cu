@@ -68,9 +68,10 @@ __device__ __forceinline__ void vb_dequant(float (&x)[C], const uint8_t* rowbase
     chunk = lo >> sh;
     if (need > 64) chunk |= (uint64_t)__ldg(rp + w0 + 2) << (64 - sh);
   } else {
-    uint32_t c32 = __ldg(rp + (sb >> 5)) >> sh;
-    if (sh + C * r.bw > 32) c32 |= __ldg(rp + (sb >> 5) + 1) << (32 - sh);
-    chunk = c32;
+    // both words loaded unconditionally (no divergent second load): the word
+    // after a row's last one is the next row's, or past the payload the
+    // first of the step section, inside the stored state either way
+    chunk = __funnelshift_r(__ldg(rp + (sb >> 5)), __ldg(rp + (sb >> 5) + 1), sh);
   }
   const uint32_t mask = (1u << r.bw) - 1u;
 #pragma unroll

@@ -37,12 +37,13 @@ struct __align__(16) VhRow {
   float k, a, q, pad;
 };
 
-// the stored code of element bit position p (width bw, mask (1 << bw) - 1)
+// the stored code of element bit position p (width bw, mask (1 << bw) - 1).
+// Both words are loaded unconditionally (no divergent second load): the
+// word after a head's last one is the next head's, or past the payload the
+// first of the step section, inside the stored state either way.
 __device__ __forceinline__ uint32_t vh_code(const uint32_t* words, uint32_t p, int bw, uint32_t mask) {
-  const uint32_t wi = p >> 5, sh = p & 31u;
-  uint32_t u = __ldg(words + wi) >> sh;
-  if (sh + (uint32_t)bw > 32u) u |= __ldg(words + wi + 1) << (32u - sh);
-  return u & mask;
+  const uint32_t wi = p >> 5;
+  return __funnelshift_r(__ldg(words + wi), __ldg(words + wi + 1), p & 31u) & mask;
 }
 
 // fitted step of one scale group of 32 targets y (levels -n..n): the

@@ -41,3 +41,15 @@ def test_reference_arm_direction_mode():
     w = synth.WORKLOADS["kda_tiny"].with_(mode="direction")
     assert line["config"] == bench.workload_config(w, 1)
     assert "l2" in line["config"]
+
+
+def test_fit_roofline_arithmetic():
+    """The variable-width decodes report the step fit against the FP32 issue
+    peak: 16 candidates x 7 operations per stored value, 148 x 128 lanes at
+    1965 MHz."""
+    import bench
+    from bit_recurrent_state_b200 import synth
+    w = synth.WORKLOADS["varbit_decode"]
+    assert bench.fit_ops(w) == 128 * 32 * 128 * 128 * 112
+    assert bench.fp32_issue_peak() == 148 * 128 * 1965e6 / 1e9
+    assert bench.kernel_family(synth.WORKLOADS["gdn_varbit_decode"]) == "varbit_head"
