@@ -63,7 +63,7 @@ VARBIT_STORES = ("varbit", "varbit_head")
 def kernel_family(w) -> str:
     if w.storage in VARBIT_STORES:
         return w.storage
-    cta = (w.storage == "damp" and w.d == 128 and w.C == 1 and w.k_hi % 16 == 0 and
+    cta = (w.storage == "damp" and w.d == 128 and w.C == 1 and w.k_hi % 16 == 0 and w.low_bits == 8 and
            w.mode in ("nearest", "stochastic", "errfeedback"))
     return "cta" if cta else "warp"
 
@@ -273,7 +273,7 @@ def _oracle_cfg(w):
           "varbit_head": O.STORE_VARBIT_HEAD}[w.storage]
     return O.Config(B=w.B, H=w.H, Hk=w.hk, d=w.d, storage=st, k_hi=w.k_hi, block=w.block,
                     hadamard=w.hadamard, decay_per_key=w.decay_per_key, avg_bits=w.avg_bits,
-                    b_min=w.b_min, b_max=w.b_max,
+                    b_min=w.b_min, b_max=w.b_max, low_bits=w.low_bits,
                     domain=O.DOMAIN_MIXED if w.storage == "damp" else O.DOMAIN_CANONICAL)
 
 
@@ -292,6 +292,8 @@ def workload_config(w, world: int) -> dict:
         cfg.update(T=w.T, C=w.C)
     if w.storage in VARBIT_STORES:
         cfg.update(avg_bits=w.avg_bits, b_min=w.b_min, b_max=w.b_max)
+    if w.storage == "damp" and w.low_bits != 8:
+        cfg.update(low_bits=w.low_bits)
     cfg["l2"] = l2_policy(w)
     return cfg
 
@@ -568,6 +570,30 @@ def run_prefill(args, w):
         dist.destroy_process_group()
 
 
+def staged_inputs(inp: dict, dev):
+    """One token's inputs in one pinned host buffer and one device buffer
+    (each tensor a view at a 256-byte aligned offset), so that a token's
+    host-to-device transfer is a single copy.  Returns (host buffer, device
+    buffer, device views by name)."""
+    import torch
+    offs, total = {}, 0
+    for k, v in inp.items():
+        offs[k] = total
+        total += (v.nbytes + 255) // 256 * 256
+    host = torch.empty(total, dtype=torch.uint8).pin_memory()
+    hv = host.numpy()
+    for k, v in inp.items():
+        a = np.ascontiguousarray(v)
+        hv[offs[k]: offs[k] + a.nbytes] = a.view(np.uint8).ravel()
+    devbuf = host.to(dev)
+    views = {}
+    for k, v in inp.items():
+        dt = torch.int16 if v.dtype == np.uint16 else torch.float32
+        n = int(np.prod(v.shape))
+        views[k] = devbuf[offs[k]: offs[k] + n * (2 if dt == torch.int16 else 4)].view(dt).view(v.shape)
+    return host, devbuf, views
+
+
 def run_ours(args, w):
     import torch
     import torch.distributed as dist
@@ -601,10 +627,9 @@ def run_ours(args, w):
         layers.append(st)
         spares.append(torch.empty_like(st.packed) if varbit else None)
         inp = synth.token_inputs(wr.with_(seed=wr.seed + 17 * l), 0)
-        host = {k: torch.from_numpy(v.view(np.int16) if v.dtype == np.uint16 else v).pin_memory()
-                for k, v in inp.items()}
-        host_inputs.append(host)
-        inputs.append({k: v.to(dev) for k, v in host.items()})
+        host, devbuf, views = staged_inputs(inp, dev)
+        host_inputs.append((host, devbuf))
+        inputs.append(views)
     o = torch.zeros((w.B, w.H, w.d), dtype=torch.float32, device=dev)
     o_host = torch.zeros_like(o, device="cpu").pin_memory()
 
@@ -646,7 +671,7 @@ def run_ours(args, w):
     # output move while token i's kernel runs; events order each buffer's reuse
     # (an input set is rewritten only after the kernel that read it, an o
     # buffer only after its read-back).
-    h2d = sum(v.numel() * v.element_size() for v in host_inputs[0].values())
+    h2d = host_inputs[0][0].numel()                  # the one buffer copied per token
     d2h = o.numel() * o.element_size()
     h2d_s, d2h_s = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     outs = [o, torch.zeros_like(o)]
@@ -663,8 +688,8 @@ def run_ours(args, w):
         if i >= NLAYERS:
             h2d_s.wait_event(k_done[(i - NLAYERS) % R])
         with torch.cuda.stream(h2d_s):
-            for k, v in host_inputs[l].items():
-                inputs[l][k].copy_(v, non_blocking=True)
+            host, devbuf = host_inputs[l]
+            devbuf.copy_(host, non_blocking=True)          # the token's inputs, one copy
         in_ready[i % R].record(h2d_s)
 
     barrier()
@@ -749,6 +774,8 @@ def main():
     ap.add_argument("--eager", action="store_true",
                     help="launch the timed steps one by one instead of replaying them as a CUDA graph")
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (small profiling cases)")
+    ap.add_argument("--low-bits", type=int, default=None, choices=[4, 8],
+                    help="DAMP low-tier width (4: the INT4 tier; the workload is then named *_int4)")
     ap.add_argument("--tokens", type=int, default=None, help="override the prefill length (small profiling cases)")
     ap.add_argument("--ref-budget", type=float, default=120.0,
                     help="seconds of oracle work for the whole --impl reference run")
@@ -761,6 +788,8 @@ def main():
         w = w.with_(mode=args.mode)
     if args.batch:
         w = w.with_(B=args.batch)
+    if args.low_bits == 4:
+        w = w.with_(low_bits=4, name=w.name + "_int4")
     if args.tokens:
         w = w.with_(T=args.tokens)
     if args.steps is None:
