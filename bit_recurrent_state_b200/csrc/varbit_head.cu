@@ -110,8 +110,18 @@ __device__ __forceinline__ uint16_t vh_fit(const float (&y)[32], int n, float on
 }
 
 // the warp's 32 codes of one row segment (lane l's code at bit l * bw)
-// OR-ed into bw words; lane k stores word k
+// OR-ed into bw words.  A width that divides 32 puts 32 / bw whole codes in
+// each word: the lanes of a word combine theirs with a butterfly of
+// shuffles and the word's first lane stores it.  Other widths straddle
+// words: one OR-reduction over the warp per word, lane k storing word k.
 __device__ __forceinline__ void vh_store_segment(uint32_t* dst, uint32_t u, int bw, int lane) {
+  if ((bw & (bw - 1)) == 0) {
+    const int g = 32 >> (__ffs(bw) - 1);              // lanes per word
+    uint32_t v = u << ((lane & (g - 1)) * bw);
+    for (int s = 1; s < g; s <<= 1) v |= __shfl_xor_sync(0xffffffffu, v, s);
+    if ((lane & (g - 1)) == 0) dst[lane / g] = v;
+    return;
+  }
   const int lb = lane * bw, lw = lb >> 5, sh = lb & 31;
   const uint32_t lo = u << sh;
   const uint32_t hi = (sh + bw > 32) ? (u >> (32 - sh)) : 0u;
@@ -123,7 +133,7 @@ __device__ __forceinline__ void vh_store_segment(uint32_t* dst, uint32_t u, int 
 }
 
 template <int PHASE, int MODE>
-__global__ void __launch_bounds__(32 * kVhWarps) varbit_head_kernel(const VbArgs a) {
+__global__ void __launch_bounds__(32 * kVhWarps, PHASE == 0 ? 1 : 7) varbit_head_kernel(const VbArgs a) {
   constexpr int D = kVhD;
   __shared__ VhRow rows[D];
   __shared__ double gam[D];
