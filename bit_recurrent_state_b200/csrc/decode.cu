@@ -877,7 +877,7 @@ cudaError_t launch_decode(const DecodeArgs& a, int d, int store, bool had, cudaS
     }
     return cudaErrorInvalidValue;
   }
-  if (a.low_bits == 8 && decode_cta_supported(d, store, a.block, a.k_hi, a.mode)) return launch_decode_cta(a, had, st);
+  if (decode_cta_supported(d, store, a.block, a.k_hi, a.mode)) return launch_decode_cta(a, had, st);
   if (d == 128 && a.block == 128) return launch_db<128, 128>(a, store, had, st);
   if (d == 128 && a.block == 32) return launch_db<128, 32>(a, store, had, st);
   if (d == 64 && a.block == 64) return launch_db<64, 64>(a, store, had, st);

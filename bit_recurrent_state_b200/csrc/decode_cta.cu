@@ -35,10 +35,14 @@
 // BRS_FLAG_TIMEOUT, waits (again bounded) for its copies in flight and
 // leaves; all its threads take that decision together at a barrier.
 //
+// The low tier is INT8 or INT4 (b = 4: a lane's four codes are 16 bits of
+// the code row, spread to bytes before the dequantization and gathered back
+// after the rounding; the grid divides the block's range by 15).
+//
 // Sources: DAMP summary, Key Points > Implementation (fused executor:
 // reconstruct INT8 channels, update in FP32, re-quantize, write back) and
 // Data & Methods > Quantization & calibration details (per-block asymmetric
-// INT8 after a Hadamard along the value axis); "Low-Bit Recurrent States in
+// quantization with b = 8 or 4 after a Hadamard along the value axis); "Low-Bit Recurrent States in
 // Hybrid Language Models", Accumulated readout error (outputs precede
 // quantization) and Protocol (quantized and dequantized before reuse).
 #include <cuda_runtime.h>
@@ -179,6 +183,17 @@ __device__ __forceinline__ uint32_t f16x2_overflow(uint32_t w) {
 // rounded quotient.
 __device__ __forceinline__ float div255(float x) { return (float)((double)x * (1.0 / 255.0)); }
 
+// the 4-bit low tier: four codes of 4 bits (16 bits, element e in bits 4e)
+// spread to one byte each, and back
+__device__ __forceinline__ uint32_t nib_spread(uint32_t w) {
+  w = (w | (w << 8)) & 0x00FF00FFu;
+  return (w | (w << 4)) & 0x0F0F0F0Fu;
+}
+__device__ __forceinline__ uint32_t nib_gather(uint32_t w) {
+  w = (w | (w >> 4)) & 0x00FF00FFu;
+  return (w | (w >> 8)) & 0xFFFFu;
+}
+
 // fl(1 / s) for s a positive binary16 value (held as a float): one
 // Newton-Raphson correction of the hardware approximation r0,
 // r = r0 + r0 (1 - s r0), with the residual 1 - s r0 exact in one fma
@@ -265,9 +280,11 @@ __device__ __forceinline__ float4 part_tree(const float4 (*part)[32], int lo, in
 
 // the INT8 rows of a batch of 8 (rows i0 .. i0+7 of my warp, values xb(r))
 // -> codes, grids (and residuals) in global memory
-template <int NB, int MODE>
+template <int NB, int MODE, int LB>
 struct Requant {
   static constexpr bool EF = MODE == BRS_ROUND_ERRFEEDBACK;
+  static constexpr int CR = kD * LB / 8;           // bytes of one code row
+  static constexpr float LV = (float)((1 << LB) - 1);   // top code: 255 or 15
   const DecodeArgs& a;
   CtaShared& sm;
   int warp, lane, blk, col0, b, h;
@@ -339,7 +356,8 @@ struct Requant {
     // operations as its elements') round into [0, 255]
     bool ok;
     {
-      const uint32_t g = f16x2_of(div255(__fsub_rn(mxv, mnv)), mnv);   // lo scale, hi zero
+      const float rng = __fsub_rn(mxv, mnv);
+      const uint32_t g = f16x2_of(LB == 8 ? div255(rng) : __fdiv_rn(rng, LV), mnv);   // lo scale, hi zero
       const float sc = f16_to_f32((uint16_t)(g & 0xffffu)), z = f16_to_f32((uint16_t)(g >> 16));
       err |= (!isfinite(mnv) || !isfinite(mxv)) ? BRS_FLAG_NONFINITE : 0u;
       err |= f16x2_overflow(g) ? BRS_FLAG_OVERFLOW : 0u;
@@ -347,7 +365,7 @@ struct Requant {
       float tlo, thi;
       sub2(tlo, thi, mnv, mxv, z, z);
       mul2(tlo, thi, tlo, thi, rcp, rcp);
-      ok = (tlo >= -0.5f) && (thi < 255.5f);
+      ok = (tlo >= -0.5f) && (thi < LV + 0.5f);
       if (NB == 4 || lane < 8) {
         sm.prm[warp][prow][blk] = make_float4(z, z, rcp, rcp);
         if constexpr (EF) sm.prs[warp][prow][blk] = sc;
@@ -385,7 +403,7 @@ struct Requant {
           tq[3] = sr_round(tq[3], rnd.w >> 8);
         }
 #pragma unroll
-        for (int c = 0; c < kC; ++c) tq[c] = fminf(fmaxf(tq[c], 0.0f), 255.0f);
+        for (int c = 0; c < kC; ++c) tq[c] = fminf(fmaxf(tq[c], 0.0f), LV);
       }
       // nearest integer (ties to even): the low byte of t + 1.5*2^23, the
       // add written as t * 1 + magic with the 1 read at run time, so that it
@@ -394,9 +412,10 @@ struct Requant {
       float mq[kC];
       fma2(mq[0], mq[1], tq[0], tq[1], one, one, kRoundMagic, kRoundMagic);
       fma2(mq[2], mq[3], tq[2], tq[3], one, one, kRoundMagic, kRoundMagic);
-      *(uint32_t*)(hout + (size_t)i * kD + col0) =
-          __byte_perm(__byte_perm(__float_as_uint(mq[0]), __float_as_uint(mq[1]), 0x0040u),
-                      __byte_perm(__float_as_uint(mq[2]), __float_as_uint(mq[3]), 0x0040u), 0x5410u);
+      const uint32_t cw = __byte_perm(__byte_perm(__float_as_uint(mq[0]), __float_as_uint(mq[1]), 0x0040u),
+                                      __byte_perm(__float_as_uint(mq[2]), __float_as_uint(mq[3]), 0x0040u), 0x5410u);
+      if constexpr (LB == 8) *(uint32_t*)(hout + (size_t)i * CR + col0) = cw;
+      else *(uint16_t*)(hout + (size_t)i * CR + col0 / 2) = (uint16_t)nib_gather(cw);
       if constexpr (EF) {
         const float sc = sm.prs[warp][r][blk];
         uint16_t ev[kC];
@@ -434,9 +453,10 @@ __device__ __forceinline__ void out_o(const CtaShared& sm, const DecodeArgs& a, 
   *(float4*)(a.o + (size_t)head * kD + col0) = make_float4(ov[0], ov[1], ov[2], ov[3]);
 }
 
-template <bool HAD, int BLOCK, int MODE>
+template <bool HAD, int BLOCK, int MODE, int LB>
 __global__ void __launch_bounds__(kThreads, 3) decode_cta_kernel(const DecodeArgs a) {
   constexpr int NB = kD / BLOCK;                   // blocks per row: 1 (whole row) or 4
+  constexpr int CR = kD * LB / 8;                  // bytes of one code row (INT8 or INT4)
   static_assert(NB == 1 || NB == 4, "blocks of 128 or 32 columns");
   constexpr bool EF = MODE == BRS_ROUND_ERRFEEDBACK;
   extern __shared__ __align__(128) uint8_t dsm[];
@@ -540,7 +560,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_cta_kernel(const DecodeArg
         sm.kq[i] = make_float4(kv, kv, qv, qv);
       }
       if (int8w) {
-        const uint32_t* szin = (const uint32_t*)(hb + (size_t)nlo * kD + (size_t)a.k_hi * kD * 2);
+        const uint32_t* szin = (const uint32_t*)(hb + (size_t)nlo * CR + (size_t)a.k_hi * kD * 2);
 #pragma unroll
         for (int e = lane; e < kRW * NB; e += 32) {
           const int i = r0 + e / NB, bb = e % NB;
@@ -561,11 +581,16 @@ __global__ void __launch_bounds__(kThreads, 3) decode_cta_kernel(const DecodeArg
           const int ra = q + r, rc = q + r + 8;
           const float4 ka = sm.ka[r0 + ra], kc = sm.ka[r0 + rc];
           if (int8w) {
-            const uint8_t* crow = hb + (size_t)r0 * kD + col0;
-            dequant4(xa[r], *(const uint32_t*)(crow + ra * kD), sm.sz[r0 + ra][blk]);
-            dequant4(xc[r], *(const uint32_t*)(crow + rc * kD), sm.sz[r0 + rc][blk]);
+            const uint8_t* crow = hb + (size_t)r0 * CR + col0 * LB / 8;
+            if constexpr (LB == 8) {
+              dequant4(xa[r], *(const uint32_t*)(crow + ra * CR), sm.sz[r0 + ra][blk]);
+              dequant4(xc[r], *(const uint32_t*)(crow + rc * CR), sm.sz[r0 + rc][blk]);
+            } else {
+              dequant4(xa[r], nib_spread(*(const uint16_t*)(crow + ra * CR)), sm.sz[r0 + ra][blk]);
+              dequant4(xc[r], nib_spread(*(const uint16_t*)(crow + rc * CR)), sm.sz[r0 + rc][blk]);
+            }
           } else {
-            const uint8_t* frow = hb + (size_t)nlo * kD + (size_t)(r0 - nlo) * kD * 2 + 2 * col0;
+            const uint8_t* frow = hb + (size_t)nlo * CR + (size_t)(r0 - nlo) * kD * 2 + 2 * col0;
             f16x4_to_f32(xa[r], *(const uint2*)(frow + ra * kD * 2));
             f16x4_to_f32(xc[r], *(const uint2*)(frow + rc * kD * 2));
           }
@@ -634,8 +659,8 @@ __global__ void __launch_bounds__(kThreads, 3) decode_cta_kernel(const DecodeArg
     {
       const float4 wl = int8w ? sm.wtv[lane] : sm.wv[lane];
       float ga[kC] = {0.f, 0.f, 0.f, 0.f}, gb[kC] = {0.f, 0.f, 0.f, 0.f};
-      const Requant<NB, MODE> rq{a, sm, warp, lane, blk, col0, b, h, hout,
-                                 (uint32_t*)(hout + (size_t)nlo * kD + (size_t)a.k_hi * kD * 2),
+      const Requant<NB, MODE, LB> rq{a, sm, warp, lane, blk, col0, b, h, hout,
+                                     (uint32_t*)(hout + (size_t)nlo * CR + (size_t)a.k_hi * kD * 2),
                                  EF ? (const uint16_t*)(bufs + 2 * bstride + j * auxp) : nullptr,
                                  EF ? (uint16_t*)a.aux + (size_t)head * nlo * kD : nullptr, err, one};
       uint32_t ovf = 0;
@@ -664,7 +689,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_cta_kernel(const DecodeArg
           rq(xb, r0 + 8 * bt);
         } else {
           // protected rows: FP16, nearest
-          uint16_t* f16out = (uint16_t*)(hout + (size_t)nlo * kD) + (size_t)(r0 + 8 * bt - nlo) * kD + col0;
+          uint16_t* f16out = (uint16_t*)(hout + (size_t)nlo * CR) + (size_t)(r0 + 8 * bt - nlo) * kD + col0;
 #pragma unroll
           for (int r = 0; r < 8; ++r) {
             const uint32_t lo = f16x2_of(xb[r][0], xb[r][1]), hi = f16x2_of(xb[r][2], xb[r][3]);
@@ -696,13 +721,13 @@ __global__ void __launch_bounds__(kThreads, 3) decode_cta_kernel(const DecodeArg
   }
 }
 
-template <bool HAD, int BLOCK, int MODE>
+template <bool HAD, int BLOCK, int MODE, int LB>
 cudaError_t launch_hbm(const DecodeArgs& a, cudaStream_t st) {
   const int heads = a.B * a.H;
   const size_t hbp = (a.head_bytes + 127) & ~(size_t)127;
   const size_t auxp = ((size_t)(kD - a.k_hi) * kD * 2 + 127) & ~(size_t)127;
   const size_t smem = sizeof(CtaShared) + 2 * (kInBytes + hbp) + (MODE == BRS_ROUND_ERRFEEDBACK ? 2 * auxp : 0);
-  auto kern = decode_cta_kernel<HAD, BLOCK, MODE>;
+  auto kern = decode_cta_kernel<HAD, BLOCK, MODE, LB>;
   // per instantiation: the opt-in shared-memory size (largest seen) and the
   // device's SM count
   static size_t set_smem = 0;
@@ -745,14 +770,20 @@ cudaError_t launch_hbm(const DecodeArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <bool HAD, int BLOCK>
-cudaError_t launch_hb(const DecodeArgs& a, cudaStream_t st) {
+template <bool HAD, int BLOCK, int LB>
+cudaError_t launch_hbl(const DecodeArgs& a, cudaStream_t st) {
   switch (a.mode) {
-    case BRS_ROUND_NEAREST: return launch_hbm<HAD, BLOCK, BRS_ROUND_NEAREST>(a, st);
-    case BRS_ROUND_STOCHASTIC: return launch_hbm<HAD, BLOCK, BRS_ROUND_STOCHASTIC>(a, st);
-    case BRS_ROUND_ERRFEEDBACK: return launch_hbm<HAD, BLOCK, BRS_ROUND_ERRFEEDBACK>(a, st);
+    case BRS_ROUND_NEAREST: return launch_hbm<HAD, BLOCK, BRS_ROUND_NEAREST, LB>(a, st);
+    case BRS_ROUND_STOCHASTIC: return launch_hbm<HAD, BLOCK, BRS_ROUND_STOCHASTIC, LB>(a, st);
+    case BRS_ROUND_ERRFEEDBACK: return launch_hbm<HAD, BLOCK, BRS_ROUND_ERRFEEDBACK, LB>(a, st);
   }
   return cudaErrorInvalidValue;
+}
+
+// the low tier's width: 8 (INT8) or 4 (two codes per byte)
+template <bool HAD, int BLOCK>
+cudaError_t launch_hb(const DecodeArgs& a, cudaStream_t st) {
+  return a.low_bits == 4 ? launch_hbl<HAD, BLOCK, 4>(a, st) : launch_hbl<HAD, BLOCK, 8>(a, st);
 }
 
 }  // namespace
