@@ -29,7 +29,7 @@ SYMBOLS = ["brs_state_bytes", "brs_state_pack", "brs_state_unpack", "brs_decode_
            "brs_decode_step_noalloc", "brs_chunk_prefill", "brs_allocate_bits", "brs_fetch_errors",
            "brs_last_error", "brs_calibrate_workspace_bytes", "brs_calibrate", "brs_decode_state32_bytes",
            "brs_decode_step_deferred", "brs_prefill_workspace_bytes", "brs_fetch_errors_noalloc",
-           "brs_test_starve_copies"]
+           "brs_test_starve_copies", "brs_test_prefill_ctas"]
 
 
 class BrsError(RuntimeError):
@@ -107,6 +107,8 @@ def lib():
         L.brs_fetch_errors_noalloc.argtypes = [P, P]
         L.brs_test_starve_copies.restype = None
         L.brs_test_starve_copies.argtypes = [ct.c_int]
+        L.brs_test_prefill_ctas.restype = None
+        L.brs_test_prefill_ctas.argtypes = [ct.c_int]
         L.brs_last_error.restype = ct.c_char_p
         L.brs_last_error.argtypes = []
         _lib = L
@@ -246,6 +248,12 @@ def fetch_errors_noalloc(stream=None) -> int:
     if st != OK and fl.value == 0:                 # a call error, not a device flag
         _check(st)
     return int(fl.value)
+
+
+def test_prefill_ctas(n: int):
+    """brs_test_prefill_ctas: cap the prefill's CTAs at n (0: the default),
+    so that small batches exercise the hand-over of heads (test hook)."""
+    lib().brs_test_prefill_ctas(int(n))
 
 
 def test_starve_copies(on: bool):

@@ -14,6 +14,7 @@ namespace {
 
 thread_local char g_err[512] = "";
 thread_local uint32_t g_starve_tx = 0;   // test hook: brs_test_starve_copies
+thread_local int g_prefill_ctas = 0;     // test hook: brs_test_prefill_ctas
 
 brs_status fail(brs_status st, const char* fmt, ...) {
   va_list ap;
@@ -102,6 +103,7 @@ namespace brs {
 // lets other translation units of the library report through brs_last_error
 void set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
 uint32_t starve_tx_bytes() { return g_starve_tx; }
+int prefill_cta_cap() { return g_prefill_ctas; }
 }  // namespace brs
 
 extern "C" {
@@ -109,6 +111,8 @@ extern "C" {
 const char* brs_last_error(void) { return g_err; }
 
 void brs_test_starve_copies(int on) { g_starve_tx = on ? 16u : 0u; }
+
+void brs_test_prefill_ctas(int n) { g_prefill_ctas = n > 0 ? n : 0; }
 
 size_t brs_state_bytes(const brs_layout* L, size_t* aux_bytes, size_t* stats_bytes,
                        size_t* workspace_bytes) {
@@ -346,9 +350,13 @@ brs_status brs_chunk_prefill(const brs_layout* L, const brs_writeback* wb, int64
   a.head_bytes = head_bytes(L); a.hscale = hadamard_scale(L->d);
   a.packed = packed; a.aux = aux; a.perm = perm; a.q = q; a.k = k; a.v = v; a.beta = beta;
   a.decay = decay; a.o = o; a.sdump = state_dump; a.flags = (uint32_t*)workspace;
-  // the FP32 state between chunks: the caller's workspace after the flag word
+  // the FP32 state between chunks: the caller's workspace after the flag
+  // word; then the heads' hand-over counters, zeroed for this call
   a.s0 = (float*)((uint8_t*)workspace + 256);
-  cudaError_t e = brs::launch_prefill_tc(a, L->hadamard != 0, (cudaStream_t)stream);
+  a.handover = (uint32_t*)((uint8_t*)workspace + 256 + brs::prefill_tc_scratch_bytes(L->B, L->H));
+  cudaError_t e = cudaMemsetAsync(a.handover, 0, (size_t)L->B * L->H * 4, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill hand-over counters");
+  e = brs::launch_prefill_tc(a, L->hadamard != 0, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
   return ok();
 }
@@ -360,7 +368,7 @@ size_t brs_prefill_workspace_bytes(const brs_layout* L) {
     return 0;
   }
   ok();
-  return 256 + brs::prefill_tc_scratch_bytes(L->B, L->H);
+  return 256 + brs::prefill_tc_scratch_bytes(L->B, L->H) + round256((size_t)L->B * L->H * 4);
 }
 
 brs_status brs_allocate_bits(int n_rows, int rows_per_group, const double* cost, double avg_bits,

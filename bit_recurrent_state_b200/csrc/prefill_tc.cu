@@ -135,6 +135,17 @@ __device__ __forceinline__ unsigned long long global_ns() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
+// hand-over of a head between CTAs: the chunk count a CTA has finished,
+// published with release semantics and read with acquire semantics (GPU scope)
+__device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 // bounded wait for one phase of an MMA-completion barrier
 __device__ __forceinline__ bool mbar_wait_tc(uint32_t bar, uint32_t parity) {
   if (mbar_try(bar, parity)) return true;
@@ -323,12 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int sub = warp & 3;                        // tensor-memory lanes 32 sub .. 32 sub + 31
   const int part = warp >> 2;                      // which part of a readout's columns
-  const int head = blockIdx.x;
-  const int b = head / a.H, h = head - b * a.H, kh = h * a.Hk / a.H;
   const int nlo = kD - a.k_hi;
-  uint8_t* hst = (uint8_t*)a.packed + (size_t)head * a.head_bytes;
-  uint16_t* aux = (MODE == BRS_ROUND_ERRFEEDBACK) ? (uint16_t*)a.aux + (size_t)head * nlo * kD : nullptr;
-  float* S0g = a.s0 + (size_t)head * kD * kD;      // FP32 state between chunks
   float* Kt = (float*)(smem + kOffKt);
   float* Kh = (float*)(smem + kOffKh);
   float* Qt = (float*)(smem + kOffQt);
@@ -351,8 +357,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar0 + 8u));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (tid < kD) permS[tid] = a.perm ? a.perm[h * kD + tid] : (int16_t)tid;
-  tc_load_state<HAD, BLOCK>(hst, S0g, nlo, a.k_hi, a.hscale);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -370,8 +374,77 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
     return !__syncthreads_or(ok ? 0 : 1);
   };
 
-  const int nchunks = a.T / kC;
-  for (int ch = 0; ch < nchunks && alive; ++ch) {
+  // This CTA's share of the (head, chunk) units, in head-major order: units
+  // [u0, u1) with equal shares per CTA (one CTA per SM, all resident).  The
+  // share is cut at head boundaries into segments, taken in this order: the
+  // leading chunks of the last head when it is cut (another CTA continues
+  // it, so they come first), whole heads, and last the continuation of the
+  // first head when it is cut (its leading chunks are the previous CTA's
+  // first segment; a bounded wait on that head's hand-over counter).
+  const int nchunks = a.T / kC, heads = a.B * a.H;
+  const long long U = (long long)heads * nchunks;
+  const long long u0 = U * blockIdx.x / gridDim.x, u1 = U * (blockIdx.x + 1) / gridDim.x;
+  const int hf = (int)(u0 / nchunks), kf = (int)(u0 % nchunks);
+  const int hl = (int)((u1 - 1) / nchunks), ke = (int)((u1 - 1) % nchunks) + 1;
+  const int nmid = hl > hf ? hl - hf - 1 : 0;
+  const bool lead = hl > hf && ke < nchunks;       // the last head's leading chunks
+  const bool cont = kf > 0;                        // the first head's continuation
+  const int nseg = (u1 <= u0) ? 0
+                   : (hl == hf) ? 1
+                                : (lead ? 1 : 0) + (kf == 0 ? 1 : 0) + nmid + (ke == nchunks ? 1 : 0) + (cont ? 1 : 0);
+  for (int sg = 0; sg < nseg && alive; ++sg) {
+    int head, c0, c1;
+    {
+      int idx = sg;
+      if (hl == hf) {
+        head = hf; c0 = kf; c1 = ke;
+      } else if (lead && idx == 0) {
+        head = hl; c0 = 0; c1 = ke;
+      } else {
+        idx -= lead ? 1 : 0;
+        if (kf == 0 && idx == 0) {
+          head = hf; c0 = 0; c1 = nchunks;
+        } else {
+          idx -= (kf == 0) ? 1 : 0;
+          if (idx < nmid) {
+            head = hf + 1 + idx; c0 = 0; c1 = nchunks;
+          } else if (ke == nchunks && idx == nmid) {
+            head = hl; c0 = 0; c1 = nchunks;
+          } else {
+            head = hf; c0 = kf; c1 = nchunks;      // the continuation
+          }
+        }
+      }
+    }
+    const int b = head / a.H, h = head - b * a.H, kh = h * a.Hk / a.H;
+    uint8_t* hst = (uint8_t*)a.packed + (size_t)head * a.head_bytes;
+    uint16_t* aux = (MODE == BRS_ROUND_ERRFEEDBACK) ? (uint16_t*)a.aux + (size_t)head * nlo * kD : nullptr;
+    float* S0g = a.s0 + (size_t)head * kD * kD;    // FP32 state between chunks
+    if (tid < kD) permS[tid] = a.perm ? a.perm[h * kD + tid] : (int16_t)tid;
+    if (c0 == 0) {
+      tc_load_state<HAD, BLOCK>(hst, S0g, nlo, a.k_hi, a.hscale);
+    } else {
+      // the head's state after chunk c0 - 1 is in the scratch, the stored
+      // state and the residuals once the hand-over counter reaches c0
+      bool ok = true;
+      if (tid == 0) {
+        const unsigned long long tw = global_ns();
+        while (ld_acquire_u32(a.handover + head) < (uint32_t)c0)
+          if (global_ns() - tw > kTcWaitNs) {
+            ok = false;
+            break;
+          }
+      }
+      if (!__syncthreads_and(ok)) {
+        alive = false;
+        break;
+      }
+      __threadfence();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  for (int ch = c0; ch < c1 && alive; ++ch) {
     const int t0 = ch * kC;
     const size_t tokb = (size_t)b * a.T + t0;                 // first token of the chunk
     // ---- chunk inputs: thread (row i, quarter qq) takes tokens 16 qq .. 16 qq + 15
@@ -652,6 +725,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
                                      (last && a.sdump) ? a.sdump + (size_t)head * kD * kD : nullptr, err);
     __syncthreads();
   }
+    if (alive && c1 < nchunks) {
+      // hand the head over: every thread's writes of the scratch, the stored
+      // state and the residuals are made visible, then the counter moves
+      __threadfence();
+      __syncthreads();
+      if (tid == 0) st_release_u32(a.handover + head, (uint32_t)c1);
+    }
+  }
   if (!alive) err |= BRS_FLAG_TIMEOUT;
   if (err) raise_flag(a.flags, err);
   tc_fence_before();
@@ -664,8 +745,29 @@ cudaError_t tc_launch(const PrefillArgs& a, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<HAD, BLOCK, MODE>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
-  prefill_tc_kernel<HAD, BLOCK, MODE><<<a.B * a.H, kThreads, kSmem, st>>>(a);
-  return cudaGetLastError();
+  // one CTA per SM (the kernel's shared memory and tensor-memory columns
+  // allow one), at most one per head; a cooperative launch, so that every
+  // CTA is resident while another waits for its hand-over
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return cudaErrorInvalidValue;
+  }
+  int grid = a.B * a.H < sms ? a.B * a.H : sms;
+  const int cap = prefill_cta_cap();
+  if (cap > 0 && cap < grid) grid = cap;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, prefill_tc_kernel<HAD, BLOCK, MODE>, a);
 }
 
 template <bool HAD, int BLOCK>

@@ -285,8 +285,13 @@ brs_status brs_decode_step_deferred(const brs_layout* L, const brs_writeback* wb
  *     feedback; direction memory is not built for the prefill).
  *   workspace: brs_prefill_workspace_bytes(L) bytes, 16-byte aligned: the
  *     flag word in its first 256 bytes (as brs_decode_step), then the FP32
- *     state carried between the chunks of the call, B*H*d*d floats, which
- *     the call overwrites (its contents between calls do not matter).
+ *     state carried between the chunks of the call, B*H*d*d floats, then
+ *     B*H u32 hand-over counters (rounded to 256 bytes), all of which the
+ *     call overwrites (their contents between calls do not matter).  The
+ *     call runs one CTA per SM, each taking an equal share of the
+ *     (head, chunk) units; a head cut between two CTAs passes from one to
+ *     the next through the scratch state and its counter (a bounded wait:
+ *     BRS_ETIMEOUT if the hand-over does not come).
  *   q, k [B][T][H_k][d] bf16; v [B][T][H][d] bf16; beta [B][T][H] f32;
  *     decay [B][T][H][d] (KDA) or [B][T][H] (GDN) f32; o [B][T][H][d] f32.
  *   state_dump (optional): [B][H][d][d] f32, the state just before the last
@@ -390,6 +395,14 @@ brs_status brs_fetch_errors_noalloc(uint32_t* flags_out, void* stream);
  * BRS_ETIMEOUT for the first flag set; *flags_out (optional) receives the
  * raw bits. */
 brs_status brs_fetch_errors(void* workspace, uint32_t* flags_out, void* stream);
+
+/* Test hook for the prefill's work split (the pages have no counterpart).
+ * While `n` is positive, brs_chunk_prefill calls made from this host thread
+ * launch at most n CTAs (by default one per SM, at most one per head), so
+ * that small batches cut heads between CTAs and exercise the hand-over.
+ * Results do not depend on n.  0 restores the default; not for use outside
+ * tests. */
+void brs_test_prefill_ctas(int n);
 
 /* Test hook for the bounded device waits (the pages have no counterpart).
  * While `on` is nonzero, brs_decode_step calls made from this host thread

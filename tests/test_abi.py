@@ -56,12 +56,13 @@ def test_host_only_calls_without_gpu():
 
 
 def test_prefill_workspace_size():
-    """The prefill's workspace: the 256-byte flag word, then the FP32 state
-    carried between chunks (B*H*d*d floats); layouts the prefill does not
-    support have none."""
+    """The prefill's workspace: the 256-byte flag word, the FP32 state
+    carried between chunks (B*H*d*d floats), then one u32 hand-over counter
+    per head (rounded to 256 bytes); layouts the prefill does not support
+    have none."""
     from bit_recurrent_state_b200 import brs, synth
     w = synth.WORKLOADS["kda_prefill"]
-    assert brs.prefill_workspace_bytes(brs.layout_of(w)) == 256 + 8 * 32 * 128 * 128 * 4
+    assert brs.prefill_workspace_bytes(brs.layout_of(w)) == 256 + 8 * 32 * 128 * 128 * 4 + 8 * 32 * 4
     with pytest.raises(brs.BrsError) as e:
         brs.prefill_workspace_bytes(brs.layout_of(synth.WORKLOADS["kda_tiny"]))
     assert e.value.status == brs.EUNSUPPORTED

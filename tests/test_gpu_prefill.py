@@ -93,16 +93,33 @@ def test_prefill_teacher_forced(kw, mode):
     _run_chunks(w, 3, mode=mode)
 
 
-@pytest.mark.parametrize("kw,mode", [
-    (dict(B=2, H=3, d=128, k_hi=16, block=128), "nearest"),
-    (dict(B=1, H=4, Hk=2, d=128, k_hi=0, block=128, decay_per_key=0), "nearest"),
-    (dict(B=1, H=2, d=128, k_hi=16, block=32), "errfeedback"),
+@pytest.mark.parametrize("kw,mode,ctas", [
+    (dict(B=2, H=3, d=128, k_hi=16, block=128), "nearest", 0),
+    (dict(B=1, H=4, Hk=2, d=128, k_hi=0, block=128, decay_per_key=0), "nearest", 0),
+    (dict(B=1, H=2, d=128, k_hi=16, block=32), "errfeedback", 0),
+    (dict(B=2, H=3, d=128, k_hi=16, block=128), "nearest", 5),
+    (dict(B=2, H=3, d=128, k_hi=16, block=128), "stochastic", 4),
+    (dict(B=1, H=4, Hk=2, d=128, k_hi=0, block=128, decay_per_key=0), "nearest", 3),
+    (dict(B=1, H=2, d=128, k_hi=16, block=32), "errfeedback", 1),
 ])
-def test_prefill_multi_chunk_one_launch(kw, mode):
+def test_prefill_multi_chunk_one_launch(kw, mode, ctas):
     """Four chunks in ONE launch (the chunk-to-chunk hand-over inside the
     kernel) equal, bit for bit, four one-chunk launches (each of which the
     teacher-forced tests compare with the oracle): the same outputs, the same
-    stored state and residuals, the same state before the last write-back."""
+    stored state and residuals, the same state before the last write-back.
+    With the CTAs capped below the heads (`ctas`), the one launch cuts heads
+    between CTAs, which hand them over through the scratch state."""
+    import torch
+    from bit_recurrent_state_b200 import brs
+    from bit_recurrent_state_b200.state import LayerState
+    brs.test_prefill_ctas(ctas)
+    try:
+        _multi_chunk_compare(kw, mode)
+    finally:
+        brs.test_prefill_ctas(0)
+
+
+def _multi_chunk_compare(kw, mode):
     import torch
     from bit_recurrent_state_b200 import brs
     from bit_recurrent_state_b200.state import LayerState
