@@ -63,8 +63,7 @@ VARBIT_STORES = ("varbit", "varbit_head")
 def kernel_family(w) -> str:
     if w.storage in VARBIT_STORES:
         return w.storage
-    cta = (w.storage == "damp" and w.d == 128 and w.C == 1 and w.k_hi % 16 == 0 and
-           w.mode in ("nearest", "stochastic", "errfeedback"))
+    cta = w.storage == "damp" and w.d == 128 and w.C == 1 and w.k_hi % 16 == 0
     return "cta" if cta else "warp"
 
 

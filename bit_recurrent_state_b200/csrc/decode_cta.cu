@@ -56,6 +56,8 @@ namespace brs {
 namespace {
 
 constexpr int kD = 128, kW = 8, kRW = 16, kC = 4, kThreads = 32 * kW;
+// kernel instantiation of k-bit residual memory (modes BRS_ROUND_RESIDUAL2..4; k at run time)
+constexpr int kModeResidual = 16;
 constexpr unsigned long long kWaitNs = 200000000ull;   // bound on one copy wait (200 ms)
 // a head's input vectors at the start of its buffer: q, k, v (bf16), the
 // permutation (int16), the per-key decays (f32)
@@ -283,6 +285,8 @@ __device__ __forceinline__ float4 part_tree(const float4 (*part)[32], int lo, in
 template <int NB, int MODE, int LB>
 struct Requant {
   static constexpr bool EF = MODE == BRS_ROUND_ERRFEEDBACK;
+  static constexpr bool DM = MODE == BRS_ROUND_DIRECTION;
+  static constexpr bool RM = MODE == kModeResidual;
   static constexpr int CR = kD * LB / 8;           // bytes of one code row
   static constexpr float LV = (float)((1 << LB) - 1);   // top code: 255 or 15
   const DecodeArgs& a;
@@ -294,9 +298,38 @@ struct Requant {
   uint16_t* auxg;
   uint32_t& err;
   float one;
+  // direction memory: the head's stored bytes in shared memory (the values
+  // the step started from) and its 2-bit counters (global, four to a byte);
+  // residual memory: its k-bit integers (global, two to a byte) and k
+  const uint8_t* hin;
+  uint8_t* mem;
+  int rmk;
 
   __device__ __forceinline__ void operator()(float (&xb)[8][kC], int i0) const {
     const int prow = lane & 7;                     // the batch row whose grid this lane computes
+    // direction memory: the batch's counter bytes, all loads issued before
+    // the first use (they would otherwise wait behind the previous row's stores)
+    uint32_t dmo[DM ? 8 : 1] = {};
+    if constexpr (DM) {
+#pragma unroll
+      for (int r = 0; r < 8; ++r) dmo[r] = mem[(size_t)(i0 + r) * (kD / 4) + lane];
+    }
+    if constexpr (RM) {
+      // the target y + m (sprev / 2^k): sprev the block's stored step the
+      // token started from, m the k-bit integer kept for the element
+      const float rinv = __fdiv_rn(1.0f, (float)(1 << rmk));    // 2^-k, exact
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const uint32_t rw = *(const uint16_t*)(mem + (size_t)(i0 + r) * (kD / 2) + col0 / 2);
+        const float su = __fmul_rn(sm.sz[i0 + r][blk].x, rinv);  // exact
+#pragma unroll
+        for (int c = 0; c < kC; ++c) {
+          const int f = (int)((rw >> (4 * c)) & 15u);
+          const int m = (f & 8) ? f - 16 : f;
+          xb[r][c] = __fadd_rn(xb[r][c], __fmul_rn((float)m, su));
+        }
+      }
+    }
     if constexpr (EF) {
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
@@ -368,7 +401,7 @@ struct Requant {
       ok = (tlo >= -0.5f) && (thi < LV + 0.5f);
       if (NB == 4 || lane < 8) {
         sm.prm[warp][prow][blk] = make_float4(z, z, rcp, rcp);
-        if constexpr (EF) sm.prs[warp][prow][blk] = sc;
+        if constexpr (EF || DM || RM) sm.prs[warp][prow][blk] = sc;
         szout[(i0 + prow) * NB + blk] = g;
       }
     }
@@ -376,13 +409,13 @@ struct Requant {
     __syncwarp();
     // ---- codes: clamp(round((y - zero) * (1/scale)), 0, 255); a zero
     // scale has 1/scale = 0, so every code of the block is 0
-    if (fast) codes<false>(xb, i0);
-    else codes<true>(xb, i0);
+    if (fast) codes<false>(xb, i0, dmo);
+    else codes<true>(xb, i0, dmo);
     __syncwarp();                                  // prm reused by the next batch
   }
 
   template <bool CLIP>
-  __device__ __forceinline__ void codes(float (&xb)[8][kC], int i0) const {
+  __device__ __forceinline__ void codes(float (&xb)[8][kC], int i0, const uint32_t* dmo) const {
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const int i = i0 + r;
@@ -412,6 +445,54 @@ struct Requant {
       float mq[kC];
       fma2(mq[0], mq[1], tq[0], tq[1], one, one, kRoundMagic, kRoundMagic);
       fma2(mq[2], mq[3], tq[2], tq[3], one, one, kRoundMagic, kRoundMagic);
+      if constexpr (DM) {
+        // votes of the proposed changes y - xp inside (scale/8, scale/2), xp
+        // the stored value the step started from (dequantized again from the
+        // head's bytes in shared memory); a counter at +-2 moves the nearest
+        // code one level (clipped to [0, LV]) and is reset.  A lane's four
+        // counters are one byte.
+        float xp[kC];
+        if constexpr (LB == 8) dequant4(xp, *(const uint32_t*)(hin + (size_t)i * CR + col0), sm.sz[i][blk]);
+        else dequant4(xp, nib_spread(*(const uint16_t*)(hin + (size_t)i * CR + col0 / 2)), sm.sz[i][blk]);
+        uint8_t* dmp = mem + (size_t)i * (kD / 4) + lane;
+        const uint32_t old = dmo[r];
+        const float sc = sm.prs[warp][r][blk];
+        const float lo = __fmul_rn(sc, 0.125f), hi = __fmul_rn(sc, 0.5f);
+        uint32_t nb = 0;
+#pragma unroll
+        for (int c = 0; c < kC; ++c) {
+          const int f = (int)((old >> (2 * c)) & 3u);
+          int m = (f & 2) ? f - 4 : f;
+          const float dl = __fsub_rn(xb[r][c], xp[c]);
+          const float ad = fabsf(dl);
+          if (ad > lo && ad < hi) m += (dl > 0.0f) ? 1 : -1;
+          if (m >= 2 || m <= -2) {
+            const uint32_t mb = __float_as_uint(mq[c]);
+            const int code = min(max((int)(mb & 0xffu) + (m > 0 ? 1 : -1), 0), (int)LV);
+            mq[c] = __uint_as_float((mb & ~0xffu) | (uint32_t)code);
+            m = 0;
+          }
+          nb |= ((uint32_t)m & 3u) << (2 * c);
+        }
+        *dmp = (uint8_t)nb;
+      }
+      if constexpr (RM) {
+        // the new integers: rne((y - value) * (1/scale) * 2^k), clipped to
+        // +-(2^(k-1) - 1); a lane's four are 16 bits
+        const float unit = (float)(1 << rmk);
+        const int rmax = (1 << (rmk - 1)) - 1;
+        const float sc = sm.prs[warp][r][blk];
+        uint32_t nb = 0;
+#pragma unroll
+        for (int c = 0; c < kC; ++c) {
+          const float code = __fsub_rn(mq[c], kRoundMagic);          // exact
+          const float res = __fsub_rn(xb[r][c], __fmaf_rn(code, sc, p.x));
+          const float q = rintf(__fmul_rn(__fmul_rn(res, p.z), unit));
+          const int m = (q != q) ? 0 : (int)fminf(fmaxf(q, (float)-rmax), (float)rmax);
+          nb |= ((uint32_t)m & 15u) << (4 * c);
+        }
+        *(uint16_t*)(mem + (size_t)i * (kD / 2) + col0 / 2) = (uint16_t)nb;
+      }
       const uint32_t cw = __byte_perm(__byte_perm(__float_as_uint(mq[0]), __float_as_uint(mq[1]), 0x0040u),
                                       __byte_perm(__float_as_uint(mq[2]), __float_as_uint(mq[3]), 0x0040u), 0x5410u);
       if constexpr (LB == 8) *(uint32_t*)(hout + (size_t)i * CR + col0) = cw;
@@ -659,10 +740,14 @@ __global__ void __launch_bounds__(kThreads, 3) decode_cta_kernel(const DecodeArg
     {
       const float4 wl = int8w ? sm.wtv[lane] : sm.wv[lane];
       float ga[kC] = {0.f, 0.f, 0.f, 0.f}, gb[kC] = {0.f, 0.f, 0.f, 0.f};
+      uint8_t* mem = nullptr;                      // direction counters / residual integers of the head
+      if constexpr (MODE == BRS_ROUND_DIRECTION) mem = (uint8_t*)a.aux + (size_t)head * nlo * (kD / 4);
+      if constexpr (MODE == kModeResidual) mem = (uint8_t*)a.aux + (size_t)head * nlo * (kD / 2);
       const Requant<NB, MODE, LB> rq{a, sm, warp, lane, blk, col0, b, h, hout,
                                      (uint32_t*)(hout + (size_t)nlo * CR + (size_t)a.k_hi * kD * 2),
-                                 EF ? (const uint16_t*)(bufs + 2 * bstride + j * auxp) : nullptr,
-                                 EF ? (uint16_t*)a.aux + (size_t)head * nlo * kD : nullptr, err, one};
+                                     EF ? (const uint16_t*)(bufs + 2 * bstride + j * auxp) : nullptr,
+                                     EF ? (uint16_t*)a.aux + (size_t)head * nlo * kD : nullptr, err, one,
+                                     hb, mem, a.mode - BRS_ROUND_RESIDUAL2 + 2};
       uint32_t ovf = 0;
 #pragma unroll
       for (int bt = 0; bt < 2; ++bt) {
@@ -776,6 +861,10 @@ cudaError_t launch_hbl(const DecodeArgs& a, cudaStream_t st) {
     case BRS_ROUND_NEAREST: return launch_hbm<HAD, BLOCK, BRS_ROUND_NEAREST, LB>(a, st);
     case BRS_ROUND_STOCHASTIC: return launch_hbm<HAD, BLOCK, BRS_ROUND_STOCHASTIC, LB>(a, st);
     case BRS_ROUND_ERRFEEDBACK: return launch_hbm<HAD, BLOCK, BRS_ROUND_ERRFEEDBACK, LB>(a, st);
+    case BRS_ROUND_DIRECTION: return launch_hbm<HAD, BLOCK, BRS_ROUND_DIRECTION, LB>(a, st);
+    case BRS_ROUND_RESIDUAL2:
+    case BRS_ROUND_RESIDUAL3:
+    case BRS_ROUND_RESIDUAL4: return launch_hbm<HAD, BLOCK, kModeResidual, LB>(a, st);
   }
   return cudaErrorInvalidValue;
 }
@@ -790,7 +879,7 @@ cudaError_t launch_hb(const DecodeArgs& a, cudaStream_t st) {
 
 bool decode_cta_supported(int d, int store, int block, int k_hi, int mode) {
   return d == kD && store == BRS_STORE_DAMP && (block == 128 || block == 32) && k_hi % kRW == 0 &&
-         (mode == BRS_ROUND_NEAREST || mode == BRS_ROUND_STOCHASTIC || mode == BRS_ROUND_ERRFEEDBACK);
+         mode >= BRS_ROUND_NEAREST && mode <= BRS_ROUND_RESIDUAL4;
 }
 
 cudaError_t launch_decode_cta(const DecodeArgs& a, bool had, cudaStream_t st) {

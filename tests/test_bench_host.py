@@ -16,7 +16,9 @@ def test_kernel_family_and_bytes():
     from bit_recurrent_state_b200 import synth
     w = synth.WORKLOADS["kda_decode"]
     assert bench.kernel_family(w) == "cta"
-    assert bench.kernel_family(w.with_(mode="direction")) == "warp"      # direction memory: general kernel
+    assert bench.kernel_family(w.with_(mode="direction")) == "cta"       # every write-back mode at C = 1
+    assert bench.kernel_family(w.with_(mode="residual3", low_bits=4)) == "cta"
+    assert bench.kernel_family(w.with_(d=64, k_hi=8, block=64)) == "warp"
     assert bench.kernel_family(synth.WORKLOADS["kda_decode_c8"]) == "warp"
     assert bench.kernel_family(synth.WORKLOADS["varbit_decode"]) == "varbit"
     base = bench.algorithmic_bytes(w)
