@@ -29,7 +29,7 @@ SYMBOLS = ["brs_state_bytes", "brs_state_pack", "brs_state_unpack", "brs_decode_
            "brs_decode_step_noalloc", "brs_chunk_prefill", "brs_allocate_bits", "brs_fetch_errors",
            "brs_last_error", "brs_calibrate_workspace_bytes", "brs_calibrate", "brs_decode_state32_bytes",
            "brs_decode_step_deferred", "brs_prefill_workspace_bytes", "brs_fetch_errors_noalloc",
-           "brs_test_starve_copies", "brs_test_prefill_ctas"]
+           "brs_test_starve_copies", "brs_test_prefill_ctas", "brs_test_prefill_withhold"]
 
 
 class BrsError(RuntimeError):
@@ -109,6 +109,8 @@ def lib():
         L.brs_test_starve_copies.argtypes = [ct.c_int]
         L.brs_test_prefill_ctas.restype = None
         L.brs_test_prefill_ctas.argtypes = [ct.c_int]
+        L.brs_test_prefill_withhold.restype = None
+        L.brs_test_prefill_withhold.argtypes = [ct.c_int]
         L.brs_last_error.restype = ct.c_char_p
         L.brs_last_error.argtypes = []
         _lib = L
@@ -254,6 +256,12 @@ def test_prefill_ctas(n: int):
     """brs_test_prefill_ctas: cap the prefill's CTAs at n (0: the default),
     so that small batches exercise the hand-over of heads (test hook)."""
     lib().brs_test_prefill_ctas(int(n))
+
+
+def test_prefill_withhold(on: bool):
+    """brs_test_prefill_withhold: the prefill hands no head over, so that the
+    bounded hand-over waits run out (test hook)."""
+    lib().brs_test_prefill_withhold(1 if on else 0)
 
 
 def test_starve_copies(on: bool):

@@ -15,6 +15,7 @@ namespace {
 thread_local char g_err[512] = "";
 thread_local uint32_t g_starve_tx = 0;   // test hook: brs_test_starve_copies
 thread_local int g_prefill_ctas = 0;     // test hook: brs_test_prefill_ctas
+thread_local int g_prefill_withhold = 0; // test hook: brs_test_prefill_withhold
 
 brs_status fail(brs_status st, const char* fmt, ...) {
   va_list ap;
@@ -104,6 +105,7 @@ namespace brs {
 void set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
 uint32_t starve_tx_bytes() { return g_starve_tx; }
 int prefill_cta_cap() { return g_prefill_ctas; }
+int prefill_withhold() { return g_prefill_withhold; }
 }  // namespace brs
 
 extern "C" {
@@ -113,6 +115,8 @@ const char* brs_last_error(void) { return g_err; }
 void brs_test_starve_copies(int on) { g_starve_tx = on ? 16u : 0u; }
 
 void brs_test_prefill_ctas(int n) { g_prefill_ctas = n > 0 ? n : 0; }
+
+void brs_test_prefill_withhold(int on) { g_prefill_withhold = on ? 1 : 0; }
 
 size_t brs_state_bytes(const brs_layout* L, size_t* aux_bytes, size_t* stats_bytes,
                        size_t* workspace_bytes) {
@@ -356,6 +360,7 @@ brs_status brs_chunk_prefill(const brs_layout* L, const brs_writeback* wb, int64
   a.handover = (uint32_t*)((uint8_t*)workspace + 256 + brs::prefill_tc_scratch_bytes(L->B, L->H));
   cudaError_t e = cudaMemsetAsync(a.handover, 0, (size_t)L->B * L->H * 4, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "prefill hand-over counters");
+  a.skip_handover = brs::prefill_withhold();
   e = brs::launch_prefill_tc(a, L->hadamard != 0, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
   return ok();

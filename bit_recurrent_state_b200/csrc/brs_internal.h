@@ -139,11 +139,13 @@ struct PrefillArgs {
   uint32_t* flags;
   float* s0;                     // scratch [B][H][d][d]: the FP32 state between chunks
   uint32_t* handover;            // [B*H] chunks finished by the CTA that hands a head over (zeroed per call)
+  int skip_handover = 0;         // test hook (brs_test_prefill_withhold): producers publish nothing
 };
 size_t prefill_tc_scratch_bytes(int B, int H);
 // the host thread's test-hook setting (brs_test_prefill_ctas): a cap on the
 // prefill's CTAs (0: one per SM), so that small batches exercise hand-overs
 int prefill_cta_cap();
+int prefill_withhold();
 cudaError_t launch_prefill_tc(const PrefillArgs& a, bool had, cudaStream_t st);
 bool prefill_supported(int d, int block, int k_hi, int C);
 

@@ -730,7 +730,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
       // state and the residuals are made visible, then the counter moves
       __threadfence();
       __syncthreads();
-      if (tid == 0) st_release_u32(a.handover + head, (uint32_t)c1);
+      if (tid == 0 && !a.skip_handover) st_release_u32(a.handover + head, (uint32_t)c1);
     }
   }
   if (!alive) err |= BRS_FLAG_TIMEOUT;

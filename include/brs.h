@@ -404,6 +404,15 @@ brs_status brs_fetch_errors(void* workspace, uint32_t* flags_out, void* stream);
  * tests. */
 void brs_test_prefill_ctas(int n);
 
+/* Test hook for the bounded wait of the prefill's hand-over (the pages have
+ * no counterpart).  While `on` is nonzero, brs_chunk_prefill calls made from
+ * this host thread hand no head over: a CTA that continues a head cut at
+ * the start of its share waits out its bound (200 ms), raises
+ * BRS_FLAG_TIMEOUT and leaves that head where it is; nothing faults and the
+ * context stays usable (brs_fetch_errors reports BRS_ETIMEOUT).  Off by
+ * default; not for use outside tests. */
+void brs_test_prefill_withhold(int on);
+
 /* Test hook for the bounded device waits (the pages have no counterpart).
  * While `on` is nonzero, brs_decode_step calls made from this host thread
  * make the copy barrier of every head of the CTA-per-head decode kernel

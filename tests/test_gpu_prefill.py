@@ -148,3 +148,39 @@ def _multi_chunk_compare(kw, mode):
         runs.append((o.cpu().numpy(), st.packed.cpu().numpy(), st.aux.cpu().numpy(), dump.cpu().numpy()))
     for a, b in zip(runs[0], runs[1]):
         np.testing.assert_array_equal(a.view(np.uint8), b.view(np.uint8))
+
+
+def test_handover_wait_runs_out():
+    """With the hand-over withheld and the CTAs capped below the heads, every
+    CTA that continues a cut head waits out its bound, the call reports
+    BRS_ETIMEOUT through the flag word, and the next call (hand-over on) is
+    correct again: it equals the same launch on a fresh state bit for bit."""
+    import torch
+    from bit_recurrent_state_b200 import brs
+    from bit_recurrent_state_b200.state import LayerState
+    w = synth.Workload("pfw", B=1, H=3, d=128, T=256, C=64, k_hi=16, block=128, seed=62)
+    perm = random_perm(w, seed=13)
+    L, wb = brs.layout_of(w), brs.writeback_of(w, C=64, mode=brs.ROUND_NEAREST)
+    d = {k: _dev(v) for k, v in _seq_major(w, 0, w.T).items()}
+
+    def run(withhold):
+        st = LayerState(L, perm=perm)
+        st.zero()
+        o = torch.zeros((w.B, w.T, w.H, w.d), device="cuda")
+        brs.test_prefill_ctas(2)                      # 3 heads of 4 chunks on 2 CTAs: head 1 is cut
+        brs.test_prefill_withhold(withhold)
+        try:
+            st.prefill(wb, 0, w.T, d["q"], d["k"], d["v"], d["beta"], d["decay"], o)
+            fl = st.errors()
+        finally:
+            brs.test_prefill_withhold(False)
+            brs.test_prefill_ctas(0)
+        return fl, o.cpu().numpy(), st.packed.cpu().numpy()
+
+    fl, _, _ = run(True)
+    assert fl & brs.FLAG_TIMEOUT
+    fl1, o1, p1 = run(False)
+    fl2, o2, p2 = run(False)
+    assert fl1 == 0 and fl2 == 0
+    np.testing.assert_array_equal(o1.view(np.uint32), o2.view(np.uint32))
+    np.testing.assert_array_equal(p1, p2)
