@@ -84,12 +84,19 @@ __device__ long long block_exclusive_scan(long long v, AllocShared& sh, long lon
   return before + x - v;
 }
 
-// candidate value of (row, step s) as ordered bits: decrements take levels
-// b, b-1, ..., b_min+1 with cost 3c 4^-L; increments take levels b, b+1,
-// ..., b_max-1 with gain 3/4 c 4^-L, ordered descending (complemented bits)
-__device__ __forceinline__ unsigned long long cand_key(double c, int level, bool dec) {
-  if (dec) return (unsigned long long)__double_as_longlong((3.0 * c) * ldexp(1.0, -2 * level));
-  return ~(unsigned long long)__double_as_longlong((0.75 * c) * ldexp(1.0, -2 * level));
+// candidate value of (row, level L) as ordered bits: decrements take levels
+// b, b-1, ..., b_min+1 with cost (3c) 4^-L; increments take levels b, b+1,
+// ..., b_max-1 with gain (3/4 c) 4^-L, ordered descending (complemented
+// bits).  p is the row's product 3c or 0.75c; scaling it by 4^-L only lowers
+// the exponent field by 2L while the result stays normal, so the key is p's
+// bit pattern minus 2L << 52 (exact, the same double as p * 4^-L); a zero,
+// subnormal or underflowing result takes the multiplication itself.
+__device__ __forceinline__ unsigned long long cand_key(double p, int level, bool dec) {
+  const unsigned long long pb = (unsigned long long)__double_as_longlong(p);
+  const int ex = (int)((pb >> 52) & 0x7ffu);
+  const unsigned long long k = (ex > 2 * level && ex < 0x7ff) ? pb - ((unsigned long long)(2 * level) << 52)
+                                                              : (unsigned long long)__double_as_longlong(p * ldexp(1.0, -2 * level));
+  return dec ? k : ~k;
 }
 
 // RPT rows per thread at most (8 for groups up to 4096 rows: fewer registers)
@@ -163,8 +170,9 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const AllocArgs
       for (int q = 0; q < RPT; ++q) {
         if (q < rpt && r0 + q < N) {
           const int lo = dec ? a.b_min + 1 : bv[q], hi = dec ? bv[q] : a.b_max - 1;
+          const double pq = dec ? 3.0 * cv[q] : 0.75 * cv[q];
           for (int L = lo; L <= hi; ++L) {
-            const unsigned long long k = cand_key(cv[q], L, dec);
+            const unsigned long long k = cand_key(pq, L, dec);
             if ((k & hmask) == (pre & hmask)) {
               const unsigned dg = (unsigned)((k >> shift) & 0xffu);
               if (dg != run_digit) {
@@ -218,8 +226,9 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const AllocArgs
       eq[q] = 0;
       if (q < rpt && r0 + q < N) {
         const int lo = dec ? a.b_min + 1 : bv[q], hi = dec ? bv[q] : a.b_max - 1;
+        const double pq = dec ? 3.0 * cv[q] : 0.75 * cv[q];
         for (int L = lo; L <= hi; ++L) {
-          const unsigned long long k = cand_key(cv[q], L, dec);
+          const unsigned long long k = cand_key(pq, L, dec);
           if (k < tau) ++below;
           else if (k == tau) ++eq[q];
         }
@@ -235,8 +244,9 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const AllocArgs
       if (q < rpt && r0 + q < N) {
         const int lo = dec ? a.b_min + 1 : bv[q], hi = dec ? bv[q] : a.b_max - 1;
         long long take = 0;
+        const double pq = dec ? 3.0 * cv[q] : 0.75 * cv[q];
         for (int L = lo; L <= hi; ++L)
-          if (cand_key(cv[q], L, dec) < tau) ++take;
+          if (cand_key(pq, L, dec) < tau) ++take;
         long long tie = rem - eqbefore;
         tie = tie < 0 ? 0 : (tie > (long long)eq[q] ? (long long)eq[q] : tie);
         eqbefore += eq[q];
