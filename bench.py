@@ -279,7 +279,7 @@ def _oracle_cfg(w):
 def is_prefill(w) -> bool:
     """Workloads whose step is one chunked-prefill launch (decode workloads
     may still write back every C > 1 tokens)."""
-    return w.name == "kda_prefill"
+    return w.name == "kda_prefill" or w.name.startswith("kda_prefill_")
 
 
 def workload_config(w, world: int) -> dict:
@@ -786,7 +786,8 @@ def main():
     if args.mode:
         w = w.with_(mode=args.mode)
     if args.batch:
-        w = w.with_(B=args.batch)
+        # another batch is another workload (no committed DRAM record applies)
+        w = w.with_(B=args.batch, name=f"{w.name}_b{args.batch}")
     if args.low_bits == 4:
         w = w.with_(low_bits=4, name=w.name + "_int4")
     if args.tokens:
