@@ -665,14 +665,16 @@ def run_ours(args, w):
 
     # ---- end to end through the public API with host buffers: every token's
     # inputs are copied from pinned host memory and its o read back inside the
-    # timed region.  Copies run on their own streams (host to device on one,
-    # device to host on another) so that token i+1's inputs and token i-1's
-    # output move while token i's kernel runs; events order each buffer's reuse
-    # (an input set is rewritten only after the kernel that read it, an o
-    # buffer only after its read-back).
+    # timed region.  Copies run on their own streams (host to device on two,
+    # alternating by token, so that two transfers overlap their fixed costs;
+    # device to host on a third) so that the next tokens' inputs and token
+    # i-1's output move while token i's kernel runs; events order each
+    # buffer's reuse (an input set is rewritten only after the kernel that read
+    # it, an o buffer only after its read-back).
     h2d = host_inputs[0][0].numel()                  # the one buffer copied per token
     d2h = o.numel() * o.element_size()
-    h2d_s, d2h_s = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    h2d_ss = [torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)]
+    d2h_s = torch.cuda.Stream(device=dev)
     outs = [o, torch.zeros_like(o)]
     outs_h = [o_host, torch.zeros_like(o_host).pin_memory()]
     R = 2 * NLAYERS                                  # event ring (slots reused after R tokens)
@@ -684,6 +686,7 @@ def run_ours(args, w):
 
     def issue_h2d(i):
         l = (base + i) % NLAYERS                     # the input set token base + i reads
+        h2d_s = h2d_ss[i % 2]
         if i >= NLAYERS:
             h2d_s.wait_event(k_done[(i - NLAYERS) % R])
         with torch.cuda.stream(h2d_s):
@@ -693,7 +696,8 @@ def run_ours(args, w):
 
     barrier()
     ev0.record(stream)
-    h2d_s.wait_event(ev0)
+    for hs in h2d_ss:
+        hs.wait_event(ev0)
     d2h_s.wait_event(ev0)
     issue_h2d(0)
     for i in range(n):
