@@ -194,8 +194,8 @@ def erasure_study(w, T: int, starts, lags: int, avg_bits: float, b_min: int, b_m
 
 
 def summary(tokens: int = 2048, device="cuda") -> dict:
-    """Both studies at the sizes the design doc reports: 4 sequences x 4 KDA heads
-    of d = 128, s log-uniform in [1e-4, 1], widths 3..6 and 8 bits; the
+    """Both studies at their reporting sizes: 4 sequences x 4 KDA heads of
+    d = 128, s log-uniform in [1e-4, 1], widths 3..6 and 8 bits; the
     erasure study on 4 heads with lags up to 4096 tokens."""
     out = {"rounding": {}, "erasure": {}}
     w = synth.Workload("sim", B=4, H=4, d=128, T=tokens, s_min=1e-4, seed=11)
