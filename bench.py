@@ -63,7 +63,8 @@ VARBIT_STORES = ("varbit", "varbit_head")
 def kernel_family(w) -> str:
     if w.storage in VARBIT_STORES:
         return w.storage
-    cta = w.storage == "damp" and w.d == 128 and w.C == 1 and w.k_hi % 16 == 0
+    cta = (w.storage == "damp" and w.d == 128 and w.k_hi % 16 == 0 and
+           (w.C == 1 or w.mode in ("nearest", "stochastic", "errfeedback")))
     return "cta" if cta else "warp"
 
 

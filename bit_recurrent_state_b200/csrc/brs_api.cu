@@ -319,8 +319,11 @@ brs_status brs_decode_step_deferred(const brs_layout* L, const brs_writeback* wb
   a.flags = (uint32_t*)workspace;
   a.s32 = (float*)state32; a.src32 = src32; a.dst32 = dst32;
   a.low_bits = low_bits(L);
-  cudaError_t e = (src32 || dst32) ? brs::launch_decode_deferred(a, L->d, L->hadamard != 0, (cudaStream_t)stream)
-                                   : brs::launch_decode(a, L->d, L->storage, L->hadamard != 0, (cudaStream_t)stream);
+  // the CTA-per-head kernel takes every token it supports (its deferred
+  // instantiations inside an interval), the general kernel the rest
+  const bool cta = brs::decode_cta_supported(L->d, L->storage, L->block, L->k_hi, wb->mode);
+  cudaError_t e = (src32 || dst32) && !cta ? brs::launch_decode_deferred(a, L->d, L->hadamard != 0, (cudaStream_t)stream)
+                                           : brs::launch_decode(a, L->d, L->storage, L->hadamard != 0, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return ok();
 }

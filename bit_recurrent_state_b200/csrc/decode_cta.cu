@@ -534,9 +534,13 @@ __device__ __forceinline__ void out_o(const CtaShared& sm, const DecodeArgs& a, 
   *(float4*)(a.o + (size_t)head * kD + col0) = make_float4(ov[0], ov[1], ov[2], ov[3]);
 }
 
-template <bool HAD, int BLOCK, int MODE, int LB>
+template <bool HAD, int BLOCK, int MODE, int LB, bool DEF>
 __global__ void __launch_bounds__(kThreads, 3) decode_cta_kernel(const DecodeArgs a) {
   constexpr int NB = kD / BLOCK;                   // blocks per row: 1 (whole row) or 4
+  // deferred write-back (write-back every C > 1 tokens): rows come from the
+  // FP32 interval state when src32 is set, and go to it instead of the
+  // write-back when dst32 is set (DEF instantiations only)
+  const bool src32 = DEF && a.src32, dst32 = DEF && a.dst32;
   constexpr int CR = kD * LB / 8;                  // bytes of one code row (INT8 or INT4)
   static_assert(NB == 1 || NB == 4, "blocks of 128 or 32 columns");
   constexpr bool EF = MODE == BRS_ROUND_ERRFEEDBACK;
@@ -572,8 +576,11 @@ __global__ void __launch_bounds__(kThreads, 3) decode_cta_kernel(const DecodeArg
     const uint32_t bar = bar0 + 8u * j;
     const size_t qk = ((size_t)hb_ * a.Hk + hh * a.Hk / a.H) * kD;
     const uint32_t in = smem_u32(bufs + j * bstride);
-    const uint32_t tx = (uint32_t)a.head_bytes + 3u * kD * 2 + (a.perm ? kD * 2u : 0u) +
-                        (a.decay_per_key ? kD * 4u : 0u) + (EF ? aux_bytes : 0u) + a.tx_extra;
+    // the stored bytes are read only when the rows come from them; the
+    // residuals only at a write-back
+    const bool codes_in = !src32, ef_in = EF && !dst32;
+    const uint32_t tx = (codes_in ? (uint32_t)a.head_bytes : 0u) + 3u * kD * 2 + (a.perm ? kD * 2u : 0u) +
+                        (a.decay_per_key ? kD * 4u : 0u) + (ef_in ? aux_bytes : 0u) + a.tx_extra;
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(in + kOffBeta), "l"(a.beta + hd) : "memory");
     if (!a.decay_per_key)
       asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(in + kOffDecay), "l"(a.decay + hd) : "memory");
@@ -584,8 +591,9 @@ __global__ void __launch_bounds__(kThreads, 3) decode_cta_kernel(const DecodeArg
     bulk_load(bar, in + kOffV, a.v + (size_t)hd * kD, kD * 2);
     if (a.perm) bulk_load(bar, in + kOffPerm, a.perm + (size_t)hh * kD, kD * 2);
     if (a.decay_per_key) bulk_load(bar, in + kOffDecay, a.decay + (size_t)hd * kD, kD * 4);
-    bulk_load(bar, in + kInBytes, (const uint8_t*)a.packed_in + (size_t)hd * a.head_bytes, (uint32_t)a.head_bytes);
-    if (EF && aux_bytes > 0)
+    if (codes_in)
+      bulk_load(bar, in + kInBytes, (const uint8_t*)a.packed_in + (size_t)hd * a.head_bytes, (uint32_t)a.head_bytes);
+    if (ef_in && aux_bytes > 0)
       bulk_load(bar, smem_u32(bufs + 2 * bstride + j * auxp), (const uint8_t*)a.aux + (size_t)hd * aux_bytes,
                 aux_bytes);
   };
@@ -640,7 +648,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_cta_kernel(const DecodeArg
         sm.ka[i] = make_float4(kv, kv, av, av);
         sm.kq[i] = make_float4(kv, kv, qv, qv);
       }
-      if (int8w) {
+      if (int8w && !src32) {
         const uint32_t* szin = (const uint32_t*)(hb + (size_t)nlo * CR + (size_t)a.k_hi * kD * 2);
 #pragma unroll
         for (int e = lane; e < kRW * NB; e += 32) {
@@ -661,7 +669,12 @@ __global__ void __launch_bounds__(kThreads, 3) decode_cta_kernel(const DecodeArg
         for (int r = 0; r < 4; ++r) {
           const int ra = q + r, rc = q + r + 8;
           const float4 ka = sm.ka[r0 + ra], kc = sm.ka[r0 + rc];
-          if (int8w) {
+          if (src32) {
+            // the interval state's rows (stored order, each tier in its basis)
+            const float* srow = a.s32 + ((size_t)head * kD + r0) * kD + col0;
+            to4(xa[r], __ldg((const float4*)(srow + (size_t)ra * kD)));
+            to4(xc[r], __ldg((const float4*)(srow + (size_t)rc * kD)));
+          } else if (int8w) {
             const uint8_t* crow = hb + (size_t)r0 * CR + col0 * LB / 8;
             if constexpr (LB == 8) {
               dequant4(xa[r], *(const uint32_t*)(crow + ra * CR), sm.sz[r0 + ra][blk]);
@@ -770,7 +783,13 @@ __global__ void __launch_bounds__(kThreads, 3) decode_cta_kernel(const DecodeArg
           axpy4(xb[r], kq.x, kq.y, wl);
           chain4(g, kq.z, kq.w, xb[r]);
         }
-        if (int8w) {
+        if (dst32) {
+          // the updated rows to the interval state instead of a write-back
+          float* drow = a.s32 + ((size_t)head * kD + r0 + 8 * bt) * kD + col0;
+#pragma unroll
+          for (int r = 0; r < 8; ++r)
+            *(float4*)(drow + (size_t)r * kD) = make_float4(xb[r][0], xb[r][1], xb[r][2], xb[r][3]);
+        } else if (int8w) {
           rq(xb, r0 + 8 * bt);
         } else {
           // protected rows: FP16, nearest
@@ -806,13 +825,13 @@ __global__ void __launch_bounds__(kThreads, 3) decode_cta_kernel(const DecodeArg
   }
 }
 
-template <bool HAD, int BLOCK, int MODE, int LB>
+template <bool HAD, int BLOCK, int MODE, int LB, bool DEF>
 cudaError_t launch_hbm(const DecodeArgs& a, cudaStream_t st) {
   const int heads = a.B * a.H;
   const size_t hbp = (a.head_bytes + 127) & ~(size_t)127;
   const size_t auxp = ((size_t)(kD - a.k_hi) * kD * 2 + 127) & ~(size_t)127;
   const size_t smem = sizeof(CtaShared) + 2 * (kInBytes + hbp) + (MODE == BRS_ROUND_ERRFEEDBACK ? 2 * auxp : 0);
-  auto kern = decode_cta_kernel<HAD, BLOCK, MODE, LB>;
+  auto kern = decode_cta_kernel<HAD, BLOCK, MODE, LB, DEF>;
   // per instantiation: the opt-in shared-memory size (largest seen) and the
   // device's SM count
   static size_t set_smem = 0;
@@ -857,14 +876,23 @@ cudaError_t launch_hbm(const DecodeArgs& a, cudaStream_t st) {
 
 template <bool HAD, int BLOCK, int LB>
 cudaError_t launch_hbl(const DecodeArgs& a, cudaStream_t st) {
+  if (a.src32 || a.dst32) {
+    // a token inside a write-back interval (the deferred instantiations)
+    switch (a.mode) {
+      case BRS_ROUND_NEAREST: return launch_hbm<HAD, BLOCK, BRS_ROUND_NEAREST, LB, true>(a, st);
+      case BRS_ROUND_STOCHASTIC: return launch_hbm<HAD, BLOCK, BRS_ROUND_STOCHASTIC, LB, true>(a, st);
+      case BRS_ROUND_ERRFEEDBACK: return launch_hbm<HAD, BLOCK, BRS_ROUND_ERRFEEDBACK, LB, true>(a, st);
+    }
+    return cudaErrorInvalidValue;
+  }
   switch (a.mode) {
-    case BRS_ROUND_NEAREST: return launch_hbm<HAD, BLOCK, BRS_ROUND_NEAREST, LB>(a, st);
-    case BRS_ROUND_STOCHASTIC: return launch_hbm<HAD, BLOCK, BRS_ROUND_STOCHASTIC, LB>(a, st);
-    case BRS_ROUND_ERRFEEDBACK: return launch_hbm<HAD, BLOCK, BRS_ROUND_ERRFEEDBACK, LB>(a, st);
-    case BRS_ROUND_DIRECTION: return launch_hbm<HAD, BLOCK, BRS_ROUND_DIRECTION, LB>(a, st);
+    case BRS_ROUND_NEAREST: return launch_hbm<HAD, BLOCK, BRS_ROUND_NEAREST, LB, false>(a, st);
+    case BRS_ROUND_STOCHASTIC: return launch_hbm<HAD, BLOCK, BRS_ROUND_STOCHASTIC, LB, false>(a, st);
+    case BRS_ROUND_ERRFEEDBACK: return launch_hbm<HAD, BLOCK, BRS_ROUND_ERRFEEDBACK, LB, false>(a, st);
+    case BRS_ROUND_DIRECTION: return launch_hbm<HAD, BLOCK, BRS_ROUND_DIRECTION, LB, false>(a, st);
     case BRS_ROUND_RESIDUAL2:
     case BRS_ROUND_RESIDUAL3:
-    case BRS_ROUND_RESIDUAL4: return launch_hbm<HAD, BLOCK, kModeResidual, LB>(a, st);
+    case BRS_ROUND_RESIDUAL4: return launch_hbm<HAD, BLOCK, kModeResidual, LB, false>(a, st);
   }
   return cudaErrorInvalidValue;
 }

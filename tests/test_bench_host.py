@@ -19,7 +19,8 @@ def test_kernel_family_and_bytes():
     assert bench.kernel_family(w.with_(mode="direction")) == "cta"       # every write-back mode at C = 1
     assert bench.kernel_family(w.with_(mode="residual3", low_bits=4)) == "cta"
     assert bench.kernel_family(w.with_(d=64, k_hi=8, block=64)) == "warp"
-    assert bench.kernel_family(synth.WORKLOADS["kda_decode_c8"]) == "warp"
+    assert bench.kernel_family(synth.WORKLOADS["kda_decode_c8"]) == "cta"    # deferred instantiations
+    assert bench.kernel_family(synth.WORKLOADS["kda_decode_c8"].with_(d=64, k_hi=8, block=64)) == "warp"
     assert bench.kernel_family(synth.WORKLOADS["varbit_decode"]) == "varbit"
     base = bench.algorithmic_bytes(w)
     assert base["state"] == 2 * 64 * 32 * 18880                           # stored state read + written
