@@ -199,6 +199,8 @@ def traffic_record(w):
         rec = json.load(f)
     if rec.get("kernel_hash") != kernel_hash(kernel_family(w)):
         return None
+    if w.mode != rec.get("mode", "nearest"):           # the records are captured in nearest mode
+        return None
     return rec.get("dram_bytes_per_launch")
 
 
