@@ -339,7 +339,6 @@ brs_status brs_chunk_prefill(const brs_layout* L, const brs_writeback* wb, int64
   if (L->storage != BRS_STORE_DAMP) return fail(BRS_EUNSUPPORTED, "chunked prefill is built for DAMP storage");
   if (!brs::prefill_supported(L->d, L->block, L->k_hi, wb->C))
     return fail(BRS_EUNSUPPORTED, "chunked prefill is built for d = 128, C = 64, block 128 or 32");
-  if (low_bits(L) != 8) return fail(BRS_EUNSUPPORTED, "chunked prefill is built for the INT8 low tier");
   if (wb->mode < 0 || wb->mode > 6) return fail(BRS_EINVAL, "unknown rounding mode %d", wb->mode);
   if (wb->mode >= BRS_ROUND_DIRECTION)
     return fail(BRS_EUNSUPPORTED, "direction and residual memory are not built for the prefill");
@@ -364,6 +363,7 @@ brs_status brs_chunk_prefill(const brs_layout* L, const brs_writeback* wb, int64
   cudaError_t e = cudaMemsetAsync(a.handover, 0, (size_t)L->B * L->H * 4, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "prefill hand-over counters");
   a.skip_handover = brs::prefill_withhold();
+  a.low_bits = low_bits(L);
   e = brs::launch_prefill_tc(a, L->hadamard != 0, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
   return ok();
@@ -371,8 +371,8 @@ brs_status brs_chunk_prefill(const brs_layout* L, const brs_writeback* wb, int64
 
 size_t brs_prefill_workspace_bytes(const brs_layout* L) {
   if (check_layout(L) != BRS_OK) return 0;
-  if (L->storage != BRS_STORE_DAMP || L->d != 128 || low_bits(L) != 8) {
-    fail(BRS_EUNSUPPORTED, "chunked prefill is built for DAMP storage at d = 128 with the INT8 low tier");
+  if (L->storage != BRS_STORE_DAMP || L->d != 128) {
+    fail(BRS_EUNSUPPORTED, "chunked prefill is built for DAMP storage at d = 128");
     return 0;
   }
   ok();

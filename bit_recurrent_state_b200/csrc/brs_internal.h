@@ -125,6 +125,7 @@ cudaError_t launch_varbit_head_unpack(const VbPackArgs& a, const void* packed, f
 
 struct PrefillArgs {
   int B, H, Hk, T, k_hi, block, decay_per_key, mode;
+  int low_bits = 8;              // DAMP low tier: 8 or 4
   uint64_t seed;
   int64_t step0;
   size_t head_bytes;

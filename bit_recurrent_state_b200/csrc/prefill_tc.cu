@@ -193,16 +193,29 @@ __device__ __forceinline__ void st_split4(uint8_t* hi, uint8_t* lo, uint32_t off
 }
 
 // stored head -> FP32 rows (stored order, value basis) in the global scratch
-template <bool HAD, int BLOCK>
+// the 4-bit low tier: a lane's four codes (16 bits, element e in bits 4e)
+// spread to one byte each, and four codes held one per byte gathered back
+__device__ __forceinline__ uint32_t pf_nib_spread(uint32_t w) {
+  w = (w | (w << 8)) & 0x00FF00FFu;
+  return (w | (w << 4)) & 0x0F0F0F0Fu;
+}
+__device__ __forceinline__ uint32_t pf_nib_gather(uint32_t w) {
+  w = (w | (w >> 4)) & 0x00FF00FFu;
+  return (w | (w >> 8)) & 0xFFFFu;
+}
+
+// LB: the low tier's width, 8 (INT8) or 4 (two codes per byte)
+template <bool HAD, int BLOCK, int LB>
 __device__ void tc_load_state(const uint8_t* head, float* S, int nlo, int k_hi, float hscale) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, col0 = 4 * lane;
-  constexpr int NB = kD / BLOCK;
-  const uint8_t* f16in = head + (size_t)nlo * kD;
-  const uint32_t* szin = (const uint32_t*)(head + (size_t)nlo * kD + (size_t)k_hi * kD * 2);
+  constexpr int NB = kD / BLOCK, CR = kD * LB / 8;
+  const uint8_t* f16in = head + (size_t)nlo * CR;
+  const uint32_t* szin = (const uint32_t*)(head + (size_t)nlo * CR + (size_t)k_hi * kD * 2);
   for (int r = warp; r < kD; r += kThreads / 32) {
     float x[4];
     if (r < nlo) {
-      const uint32_t c4 = *(const uint32_t*)(head + (size_t)r * kD + col0);
+      const uint32_t c4 = (LB == 8) ? *(const uint32_t*)(head + (size_t)r * CR + col0)
+                                    : pf_nib_spread(*(const uint16_t*)(head + (size_t)r * CR + col0 / 2));
       const uint32_t sz = szin[r * NB + col0 / BLOCK];
       const float s = f16_to_f32((uint16_t)(sz & 0xffffu)), z = f16_to_f32((uint16_t)(sz >> 16));
 #pragma unroll
@@ -222,14 +235,15 @@ __device__ void tc_load_state(const uint8_t* head, float* S, int nlo, int k_hi, 
 // product rows Ds (shared, stride kSStride) and S_0 (the global scratch,
 // whole rows per load), then the stored row; the dequantized row (the state
 // the next chunk starts from) replaces S_0 in the scratch.
-template <bool HAD, int BLOCK, int MODE>
+template <bool HAD, int BLOCK, int MODE, int LB>
 __device__ void tc_store_state(const float* Ds, const float* g63, float* S, uint8_t* head, uint16_t* aux, int nlo,
                                int k_hi, float hscale, const PrefillArgs& a, int64_t step, int h, int b, float* sdump,
                                uint32_t& err) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, col0 = 4 * lane;
-  constexpr int NB = kD / BLOCK, GL = BLOCK / 4, kRowsW = kD / (kThreads / 32);
-  uint16_t* f16out = (uint16_t*)(head + (size_t)nlo * kD);
-  uint32_t* szout = (uint32_t*)(head + (size_t)nlo * kD + (size_t)k_hi * kD * 2);
+  constexpr int NB = kD / BLOCK, GL = BLOCK / 4, kRowsW = kD / (kThreads / 32), CR = kD * LB / 8;
+  constexpr float LV = (float)((1 << LB) - 1);    // top code: 255 or 15
+  uint16_t* f16out = (uint16_t*)(head + (size_t)nlo * CR);
+  uint32_t* szout = (uint32_t*)(head + (size_t)nlo * CR + (size_t)k_hi * kD * 2);
   float4 s0r[kRowsW];                              // this warp's S_0 rows, all loads in flight at once
 #pragma unroll
   for (int k = 0; k < kRowsW; ++k) s0r[k] = *(const float4*)&S[(size_t)(warp + 16 * k) * kD + col0];
@@ -287,7 +301,8 @@ __device__ void tc_store_state(const float* Ds, const float* g63, float* S, uint
       if (mx == 0.0f) mx = apz ? 0.0f : -0.0f;
     }
     if (!isfinite(mn) || !isfinite(mx)) err |= BRS_FLAG_NONFINITE;
-    const uint32_t gz = f16x2_of(div255(__fsub_rn(mx, mn)), mn);    // lo scale, hi zero
+    const float rng = __fsub_rn(mx, mn);
+    const uint32_t gz = f16x2_of(LB == 8 ? div255(rng) : __fdiv_rn(rng, LV), mn);    // lo scale, hi zero
     const uint16_t sh = (uint16_t)(gz & 0xffffu), zh = (uint16_t)(gz >> 16);
     if (f16_inf_or_nan(sh) || f16_inf_or_nan(zh)) err |= BRS_FLAG_OVERFLOW;
     const float s = f16_to_f32(sh), z = f16_to_f32(zh);
@@ -307,7 +322,7 @@ __device__ void tc_store_state(const float* Ds, const float* g63, float* S, uint
       if (MODE == BRS_ROUND_STOCHASTIC) tt = sr_round(tt, rw[c]);
       // clip, then the nearest integer (ties to even) as the low byte of
       // t + 1.5*2^23 (exact for the integers SR produces)
-      const float m = __fadd_rn(fminf(fmaxf(tt, 0.0f), 255.0f), kRoundMagic);
+      const float m = __fadd_rn(fminf(fmaxf(tt, 0.0f), LV), kRoundMagic);
       const float code = __fsub_rn(m, kRoundMagic);
       packed4 |= (__float_as_uint(m) & 0xffu) << (8 * c);
       xh[c] = __fmaf_rn(code, s, z);
@@ -318,7 +333,8 @@ __device__ void tc_store_state(const float* Ds, const float* g63, float* S, uint
         e16[c] = f32_to_f16(e);
       }
     }
-    *(uint32_t*)(head + (size_t)r * kD + col0) = packed4;
+    if (LB == 8) *(uint32_t*)(head + (size_t)r * CR + col0) = packed4;
+    else *(uint16_t*)(head + (size_t)r * CR + col0 / 2) = (uint16_t)pf_nib_gather(packed4);
     if ((col0 % BLOCK) == 0) szout[r * NB + col0 / BLOCK] = (uint32_t)sh | ((uint32_t)zh << 16);
     if (MODE == BRS_ROUND_ERRFEEDBACK)
       *(uint2*)&aux[(size_t)r * kD + col0] =
@@ -328,7 +344,7 @@ __device__ void tc_store_state(const float* Ds, const float* g63, float* S, uint
   }
 }
 
-template <bool HAD, int BLOCK, int MODE>
+template <bool HAD, int BLOCK, int MODE, int LB>
 __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
@@ -422,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
     float* S0g = a.s0 + (size_t)head * kD * kD;    // FP32 state between chunks
     if (tid < kD) permS[tid] = a.perm ? a.perm[h * kD + tid] : (int16_t)tid;
     if (c0 == 0) {
-      tc_load_state<HAD, BLOCK>(hst, S0g, nlo, a.k_hi, a.hscale);
+      tc_load_state<HAD, BLOCK, LB>(hst, S0g, nlo, a.k_hi, a.hscale);
     } else {
       // the head's state after chunk c0 - 1 is in the scratch, the stored
       // state and the residuals once the hand-over counter reaches c0
@@ -720,7 +736,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
     __syncthreads();
     // ---- write-back of the chunk
     const bool last = ch == nchunks - 1;
-    tc_store_state<HAD, BLOCK, MODE>((const float*)smem, g63, S0g, hst, aux, nlo, a.k_hi, a.hscale, a,
+    tc_store_state<HAD, BLOCK, MODE, LB>((const float*)smem, g63, S0g, hst, aux, nlo, a.k_hi, a.hscale, a,
                                      a.step0 + t0 + kC - 1, h, b,
                                      (last && a.sdump) ? a.sdump + (size_t)head * kD * kD : nullptr, err);
     __syncthreads();
@@ -740,9 +756,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillAr
   if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tm), "r"(512));
 }
 
-template <bool HAD, int BLOCK, int MODE>
+template <bool HAD, int BLOCK, int MODE, int LB>
 cudaError_t tc_launch(const PrefillArgs& a, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<HAD, BLOCK, MODE>,
+  cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<HAD, BLOCK, MODE, LB>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
   // one CTA per SM (the kernel's shared memory and tensor-memory columns
@@ -767,17 +783,22 @@ cudaError_t tc_launch(const PrefillArgs& a, cudaStream_t st) {
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, prefill_tc_kernel<HAD, BLOCK, MODE>, a);
+  return cudaLaunchKernelEx(&cfg, prefill_tc_kernel<HAD, BLOCK, MODE, LB>, a);
+}
+
+template <bool HAD, int BLOCK, int LB>
+cudaError_t tc_launch_hbl(const PrefillArgs& a, cudaStream_t st) {
+  switch (a.mode) {
+    case BRS_ROUND_NEAREST: return tc_launch<HAD, BLOCK, BRS_ROUND_NEAREST, LB>(a, st);
+    case BRS_ROUND_STOCHASTIC: return tc_launch<HAD, BLOCK, BRS_ROUND_STOCHASTIC, LB>(a, st);
+    case BRS_ROUND_ERRFEEDBACK: return tc_launch<HAD, BLOCK, BRS_ROUND_ERRFEEDBACK, LB>(a, st);
+  }
+  return cudaErrorInvalidValue;
 }
 
 template <bool HAD, int BLOCK>
 cudaError_t tc_launch_hb(const PrefillArgs& a, cudaStream_t st) {
-  switch (a.mode) {
-    case BRS_ROUND_NEAREST: return tc_launch<HAD, BLOCK, BRS_ROUND_NEAREST>(a, st);
-    case BRS_ROUND_STOCHASTIC: return tc_launch<HAD, BLOCK, BRS_ROUND_STOCHASTIC>(a, st);
-    case BRS_ROUND_ERRFEEDBACK: return tc_launch<HAD, BLOCK, BRS_ROUND_ERRFEEDBACK>(a, st);
-  }
-  return cudaErrorInvalidValue;
+  return a.low_bits == 4 ? tc_launch_hbl<HAD, BLOCK, 4>(a, st) : tc_launch_hbl<HAD, BLOCK, 8>(a, st);
 }
 
 }  // namespace

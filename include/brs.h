@@ -55,9 +55,8 @@
  *                    rows hold two codes per byte ((d-k_hi)*d/2 bytes;
  *                    element e of a row in bits 4 (e % 2) of byte e/2),
  *                    codes run 0..15 and the scale divides the block's
- *                    range by 15; the rest is unchanged.  Pack, unpack,
- *                    calibration and the decode entry points accept it;
- *                    brs_chunk_prefill returns BRS_EUNSUPPORTED.
+ *                    range by 15; the rest is unchanged.  Every entry
+ *                    point that takes DAMP storage accepts it.
  *                    Error-feedback residuals: f16 [B][H][d-k_hi][d].
  *   BRS_STORE_VARBIT [LB] State bit allocation, Allocation units, Levels and
  *                    storage.  Sections, each starting on a 256-byte

@@ -36,7 +36,8 @@ def _run_chunks(w, nchunks, units=None, mode="nearest"):
     from bit_recurrent_state_b200.state import LayerState
     perm = random_perm(w, seed=11)
     cfg = O.Config(B=w.B, H=w.H, Hk=w.hk, d=w.d, storage=O.STORE_DAMP, k_hi=w.k_hi, block=w.block,
-                   hadamard=w.hadamard, decay_per_key=w.decay_per_key, domain=O.DOMAIN_CANONICAL)
+                   hadamard=w.hadamard, decay_per_key=w.decay_per_key, low_bits=w.low_bits,
+                   domain=O.DOMAIN_CANONICAL)
     L, wb = brs.layout_of(w), brs.writeback_of(w, C=64, mode=brs.MODES[mode])
     rng = np.random.default_rng(5)
     S0 = (rng.standard_normal((w.B, w.H, w.d, w.d)) * 0.05).astype(np.float32)
@@ -87,6 +88,10 @@ def _run_chunks(w, nchunks, units=None, mode="nearest"):
     (dict(B=2, H=4, Hk=2, d=128, k_hi=0, block=128, decay_per_key=0), "nearest"),
     (dict(B=1, H=2, d=128, k_hi=16, block=128), "errfeedback"),
     (dict(B=1, H=2, d=128, k_hi=16, block=128), "stochastic"),
+    # the 4-bit low tier
+    (dict(B=2, H=3, d=128, k_hi=16, block=128, low_bits=4), "nearest"),
+    (dict(B=1, H=2, d=128, k_hi=16, block=32, low_bits=4), "errfeedback"),
+    (dict(B=1, H=2, d=128, k_hi=0, block=128, decay_per_key=0, low_bits=4), "stochastic"),
 ])
 def test_prefill_teacher_forced(kw, mode):
     w = synth.Workload("pf", T=192, C=64, seed=60, **kw)
@@ -101,6 +106,7 @@ def test_prefill_teacher_forced(kw, mode):
     (dict(B=2, H=3, d=128, k_hi=16, block=128), "stochastic", 4),
     (dict(B=1, H=4, Hk=2, d=128, k_hi=0, block=128, decay_per_key=0), "nearest", 3),
     (dict(B=1, H=2, d=128, k_hi=16, block=32), "errfeedback", 1),
+    (dict(B=2, H=3, d=128, k_hi=16, block=128, low_bits=4), "nearest", 4),
 ])
 def test_prefill_multi_chunk_one_launch(kw, mode, ctas):
     """Four chunks in ONE launch (the chunk-to-chunk hand-over inside the
@@ -126,7 +132,8 @@ def _multi_chunk_compare(kw, mode):
     w = synth.Workload("pf1", T=256, C=64, seed=61, **kw)
     perm = random_perm(w, seed=12)
     cfg = O.Config(B=w.B, H=w.H, Hk=w.hk, d=w.d, storage=O.STORE_DAMP, k_hi=w.k_hi, block=w.block,
-                   hadamard=w.hadamard, decay_per_key=w.decay_per_key, domain=O.DOMAIN_CANONICAL)
+                   hadamard=w.hadamard, decay_per_key=w.decay_per_key, low_bits=w.low_bits,
+                   domain=O.DOMAIN_CANONICAL)
     L, wb = brs.layout_of(w), brs.writeback_of(w, C=64, mode=brs.MODES[mode])
     S0 = (np.random.default_rng(6).standard_normal((w.B, w.H, w.d, w.d)) * 0.05).astype(np.float32)
     packed0, _ = O.state_pack(cfg, S0, perm)
