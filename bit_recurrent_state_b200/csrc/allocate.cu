@@ -33,6 +33,7 @@ struct AllocShared {
   unsigned hist[256];
   unsigned long long prefix;               // radix-select state
   int rank;                                // candidates still to take below the prefix
+  int uniq;                                // the selected digit holds one candidate
   double gm;
   int all_zero;
   long long total;
@@ -156,7 +157,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const AllocArgs
     const bool dec = E > 0;
     const long long need = dec ? E : -E;
     // ---- radix select: the need-th smallest candidate key, 8 bits at a time
-    if (t == 0) { sh.prefix = 0ull; sh.rank = (int)need; }
+    if (t == 0) { sh.prefix = 0ull; sh.rank = (int)need; sh.uniq = 0; }
     __syncthreads();
     for (int shift = 56; shift >= 0; shift -= 8) {
       for (int i = t; i < 256; i += kAllocThreads) sh.hist[i] = 0u;
@@ -204,17 +205,36 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(const AllocArgs
         const unsigned before = incl - tot;
         if ((int)before < r && r <= (int)incl) {
           int rr = r - (int)before;
-          unsigned digit = 8 * lane;
+          unsigned digit = 8 * lane, dcnt = 0;
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            if (rr <= (int)cnt[e]) { digit = 8 * lane + e; break; }
+            if (rr <= (int)cnt[e]) { digit = 8 * lane + e; dcnt = cnt[e]; break; }
             rr -= (int)cnt[e];
           }
           sh.prefix = pre | ((unsigned long long)digit << shift);
           sh.rank = rr;
+          sh.uniq = dcnt == 1u;
         }
       }
       __syncthreads();
+      if (sh.uniq && shift > 0) {
+        // one candidate carries the selected prefix: its key is the answer,
+        // found in one pass instead of the remaining digit passes
+        const unsigned long long pre2 = sh.prefix, m2 = ~0ull << shift;
+#pragma unroll
+        for (int q = 0; q < RPT; ++q) {
+          if (q < rpt && r0 + q < N) {
+            const int lo = dec ? a.b_min + 1 : bv[q], hi = dec ? bv[q] : a.b_max - 1;
+            const double pq = dec ? 3.0 * cv[q] : 0.75 * cv[q];
+            for (int L = lo; L <= hi; ++L) {
+              const unsigned long long k = cand_key(pq, L, dec);
+              if ((k & m2) == pre2) sh.prefix = k;
+            }
+          }
+        }
+        __syncthreads();
+        break;
+      }
     }
     const unsigned long long tau = sh.prefix;   // key of the need-th candidate
     // every candidate below tau is taken; among those equal to tau, the
