@@ -56,3 +56,23 @@ def test_fit_roofline_arithmetic():
     assert bench.fit_ops(w) == 128 * 32 * 128 * 128 * 112
     assert bench.fp32_issue_peak() == 148 * 128 * 1965e6 / 1e9
     assert bench.kernel_family(synth.WORKLOADS["gdn_varbit_decode"]) == "varbit_head"
+
+
+def test_staged_inputs_layout(monkeypatch):
+    """A token's inputs staged in one buffer for a single host-to-device
+    copy: each tensor a view at a 256-byte aligned offset holding exactly the
+    input's values (checked on the host with a CPU 'device')."""
+    import numpy as np
+    import torch
+    import bench
+    from bit_recurrent_state_b200 import synth
+    monkeypatch.setattr(torch.Tensor, "pin_memory", lambda self: self)     # no CUDA here
+    for name in ("kda_decode", "gdn_decode"):
+        inp = synth.token_inputs(synth.WORKLOADS[name], 3)
+        host, dev, views = bench.staged_inputs(inp, "cpu")
+        assert host.numel() == dev.numel() >= sum(v.nbytes for v in inp.values())
+        for k, v in inp.items():
+            a = views[k].numpy()
+            assert a.shape == v.shape
+            assert (views[k].data_ptr() - dev.data_ptr()) % 256 == 0
+            np.testing.assert_array_equal(a.view(np.uint16) if v.dtype == np.uint16 else a, v)
