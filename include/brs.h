@@ -227,12 +227,16 @@ brs_status brs_state_unpack(const brs_layout* L, const void* packed, const int16
  * state, then (when (step + 1) % C == 0) requantize and write back
  * ([DAMP] Implementation; [LB] Accumulated readout error: outputs precede
  * quantization; [LB] Protocol: each write-back is quantized and dequantized
- * before reuse).  Decode supports C == 1.
+ * before reuse).  Decode supports C == 1 (brs_decode_step_deferred takes
+ * C > 1).
  *   packed_in / packed_out: stored state before / after; they may alias
- *     for FP32 and DAMP storage, must not alias for VARBIT.
- *   aux: residuals (ERRFEEDBACK) or direction counters (DIRECTION, DAMP
- *     only), updated in place; else may be NULL.
- *   stats: VARBIT statistics, updated in place (else may be NULL).
+ *     for FP32 and DAMP storage, must not alias for VARBIT and
+ *     VARBIT_HEAD.
+ *   aux: residuals (ERRFEEDBACK), direction counters (DIRECTION) or
+ *     residual integers (RESIDUAL2..4; the last two DAMP only), updated in
+ *     place; else may be NULL.
+ *   stats: VARBIT / VARBIT_HEAD statistics, updated in place (else may be
+ *     NULL).
  *   workspace: brs_state_bytes(...workspace) bytes; its first word
  *     collects device flags and must be zeroed once before first use
  *     (brs_fetch_errors clears it).
@@ -255,8 +259,8 @@ brs_status brs_decode_step(const brs_layout* L, const brs_writeback* wb, int64_t
  *     step % C != 0 (else the stored state is read), written when
  *     (step + 1) % C != 0.  May be NULL when C == 1.
  *   packed: stored state, updated in place at write-backs.  aux: residuals
- *     (error feedback), used and updated at write-backs only; direction
- *     memory needs C == 1.
+ *     (error feedback), used and updated at write-backs only; direction and
+ *     residual memory need C == 1.
  *   workspace: flag word (as brs_decode_step).
  * Calls must cover consecutive steps, starting at a multiple of C, for the
  * result to equal the recurrence with write-back every C tokens (the state
