@@ -315,14 +315,17 @@ def test_pack_unpack_roundtrip(orc):
     assert err <= (S.max() - S.min()) / 255 * 2     # half a step per coordinate, spread by H
 
 
-@pytest.mark.parametrize("mode,dom", [(0, 0), (1, 0), (2, 0), (3, 2), (2, 2)])
-def test_writeback_replay_equals_the_run(orc, mode, dom):
+@pytest.mark.parametrize("mode,dom,low_bits", [(0, 0, 8), (1, 0, 8), (2, 0, 8), (3, 2, 8), (2, 2, 8),
+                                                (4, 2, 8), (6, 2, 8), (0, 0, 4), (1, 0, 4), (2, 2, 4),
+                                                (3, 2, 4), (5, 2, 4)])
+def test_writeback_replay_equals_the_run(orc, mode, dom, low_bits):
     """The write-back entry (the quantizer alone, used to replay a state
     computed elsewhere) applied to the FP32 state the recurrence held just
     before its write-back reproduces the recurrence's stored bytes and
-    residuals / counters, in every rounding mode."""
+    residuals / counters / residual integers, in every rounding mode and for
+    both low tiers."""
     w = synth.Workload("rp", B=2, H=3, d=32, T=4, k_hi=4, block=32, seed=21)
-    cfg = _cfg(orc, w, domain=dom)
+    cfg = _cfg(orc, w, domain=dom, low_bits=low_bits)
     rng = np.random.default_rng(22)
     perm = _rand_perm(rng, w.H, w.d)
     S0 = (rng.standard_normal((w.B, w.H, w.d, w.d)) * 0.1).astype(np.float32)
